@@ -1,0 +1,96 @@
+"""Pins of the oracle's real spherical harmonics and fitted Wigner-D matrices.
+
+None of these re-types the harmonics' formula: they check properties that any
+correct real, component-normalised degree-l basis must have."""
+import numpy as np
+import pytest
+
+import oracle
+from workloads import real_sh
+
+LMAX = 6
+
+
+def _unit(g, n):
+    v = g.normal(size=(n, 3))
+    return v / np.linalg.norm(v, axis=1, keepdims=True)
+
+
+@pytest.mark.parametrize("l", range(LMAX + 1))
+def test_addition_theorem(l):
+    # sum_m Y_lm(v)^2 = 2l+1 for every unit v (component normalisation)
+    v = _unit(np.random.default_rng(l), 500)
+    y = oracle.sh_l(l, v)
+    np.testing.assert_allclose((y * y).sum(1), 2 * l + 1, rtol=1e-13)
+
+
+@pytest.mark.parametrize("l", range(LMAX + 1))
+def test_addition_theorem_two_points(l):
+    # sum_m Y_lm(a) Y_lm(b) = (2l+1) P_l(a.b): the Legendre polynomial of the angle
+    g = np.random.default_rng(10 + l)
+    a, b = _unit(g, 200), _unit(g, 200)
+    lhs = (oracle.sh_l(l, a) * oracle.sh_l(l, b)).sum(1)
+    from numpy.polynomial import legendre
+    rhs = (2 * l + 1) * legendre.legval((a * b).sum(1), [0] * l + [1])
+    np.testing.assert_allclose(lhs, rhs, atol=1e-12)
+
+
+def test_orthonormal_by_exact_quadrature():
+    # Gauss-Legendre in z (n nodes) x uniform phi (M points) integrates the
+    # products of degree <= 2*LMAX exactly; (1/4pi) int Y Y' = identity.
+    n, M = LMAX + 2, 2 * LMAX + 3
+    z, wz = np.polynomial.legendre.leggauss(n)
+    phi = 2 * np.pi * np.arange(M) / M
+    Z, PHI = np.meshgrid(z, phi, indexing="ij")
+    rho = np.sqrt(1 - Z ** 2)
+    v = np.stack([rho * np.cos(PHI), rho * np.sin(PHI), Z], -1).reshape(-1, 3)
+    w = (wz[:, None] * np.full(M, 2 * np.pi / M)[None, :]).reshape(-1) / (4 * np.pi)
+    Y = oracle.sh(LMAX, v)
+    G = (Y * w[:, None]).T @ Y
+    np.testing.assert_allclose(G, np.eye(len(G)), atol=1e-12)
+
+
+@pytest.mark.parametrize("l", range(LMAX + 1))
+def test_parity(l):
+    v = _unit(np.random.default_rng(20 + l), 100)
+    np.testing.assert_allclose(oracle.sh_l(l, -v), (-1) ** l * oracle.sh_l(l, v), atol=1e-13)
+
+
+@pytest.mark.parametrize("l", range(LMAX + 1))
+def test_span_is_rotation_invariant(l):
+    # The fitted D^l reproduces Y_l(R v) on directions not used by the fit:
+    # only a true degree-l harmonic basis spans a rotation-invariant space.
+    g = np.random.default_rng(30 + l)
+    for _ in range(3):
+        R = oracle.random_rotation(g)
+        D = oracle.wigner_d(l, R)
+        v = _unit(g, 50)
+        np.testing.assert_allclose(oracle.sh_l(l, v @ R.T), oracle.sh_l(l, v) @ D.T, atol=1e-12)
+
+
+@pytest.mark.parametrize("l", range(LMAX + 1))
+def test_wigner_d_is_orthogonal_representation(l):
+    g = np.random.default_rng(40 + l)
+    R1, R2 = oracle.random_rotation(g), oracle.random_rotation(g)
+    D1, D2 = oracle.wigner_d(l, R1), oracle.wigner_d(l, R2)
+    np.testing.assert_allclose(D1 @ D1.T, np.eye(2 * l + 1), atol=1e-12)
+    np.testing.assert_allclose(oracle.wigner_d(l, R1 @ R2), D1 @ D2, atol=1e-12)
+    np.testing.assert_allclose(oracle.wigner_d(l, np.eye(3)), np.eye(2 * l + 1), atol=1e-12)
+    np.testing.assert_allclose(np.linalg.det(D1), 1.0, atol=1e-11)
+
+
+def test_l1_is_scaled_direction_in_yzx_order():
+    # basis convention (our choice, the pages print none): l=1 is sqrt(3)(y, z, x)
+    v = _unit(np.random.default_rng(50), 20)
+    np.testing.assert_allclose(oracle.sh_l(1, v), np.sqrt(3) * v[:, [1, 2, 0]], atol=1e-14)
+    np.testing.assert_allclose(oracle.sh_l(0, v), 1.0)
+
+
+def test_workload_harmonics_match_oracle():
+    # two independent implementations (recurrence vs Rodrigues polynomial)
+    g = np.random.default_rng(60)
+    v = g.normal(size=(300, 3)) * g.uniform(0.1, 5, size=(300, 1))
+    u = v / np.linalg.norm(v, axis=1, keepdims=True)
+    np.testing.assert_allclose(real_sh(v, LMAX), oracle.sh(LMAX, u), atol=1e-11)
+    z = real_sh(np.zeros((2, 3)), 3)
+    assert np.all(z[:, 0] == 1) and np.all(z[:, 1:] == 0)
