@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Benchmark of the equivariant message-passing convolution on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input
+already resident in HBM: receiver-sorted CSR indexing of the edge list
+(e3conv_build_csr) followed by the fused forward (e3conv_forward: gather,
+channelwise CG product, scalar mix, segmented sum, 1/N scale, store).
+
+Default workload: the large mixed-precision graph (100,000 nodes, ~4.0M
+edges, 128x(0e+1o+2e+3o) float16 node features, Y for l <= 3, float16 edge
+scalars, float32 accumulation and output, outputs l <= 3).  Its inputs
+(~37 GB) are larger than L2, so no flush is needed between steps.
+
+Prints one JSON line (rank 0).  `--impl reference` times the float64 CPU
+oracle on a bounded sample of the same workload instead.
+Multi-GPU (torchrun): every rank runs an independent graph of the same size
+(weak scaling, no collective on the data path); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "edges/sec and achieved fraction of roofline (HBM GB/s or FP32 FMA) at 1 B200"
+UNIT = "edges/s"
+SMS = 148
+FP32_LANES_PER_SM = 128
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="large_f16")
+    ap.add_argument("--nodes", type=int, default=None,
+                    help="override the node count at the same density (profiling cases)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--channels-per-lane", type=int, default=0)
+    ap.add_argument("--block-threads", type=int, default=0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# accounting
+
+def peaks():
+    hbm, sm_max, src = FALLBACK_HBM_GBS, 1965.0, "fallback"
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        hbm = float(d.get("hbm_gbs", hbm))
+        sm_max = float(d.get("sm_max_mhz", sm_max))
+        src = "measured"
+    fp32_tflops = SMS * FP32_LANES_PER_SM * 2 * sm_max * 1e6 / 1e12
+    return {"hbm_gbs": hbm, "fp32_tflops": fp32_tflops, "sm_max_mhz": sm_max, "source": src}
+
+
+def algorithmic(conv, N, E, in_bytes):
+    """Algorithmic bytes and FLOPs of one forward.
+
+    bytes = E (ny + P C) b + 4E (senders) + N (nx C b + 4 nout C + 4 (row_ptr)):
+            every edge's Y and s once, every node's features once, every output once.
+    flops = 2 E C (sum of CG nonzeros over paths + sum over paths of (2 l3 + 1)).
+    """
+    import numpy as np
+    nnz = sum(int((np.abs(conv.cg(p)) > 1e-12).sum()) for p in range(conv.num_paths))
+    mix = sum(2 * q.l3 + 1 for q in conv.paths)
+    nbytes = E * (conv.ny + conv.num_paths * conv.C) * in_bytes + 4 * E + \
+        N * (conv.nx * conv.C * in_bytes + 4 * conv.nout * conv.C + 4)
+    flops = 2 * E * conv.C * (nnz + mix)
+    return nbytes, flops, nnz, mix
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.ident = str(device_index)
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.ident, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == len(self.FIELDS):
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(power) if power else None}
+
+
+def kernel_hash(conv) -> str:
+    return hashlib.sha1(conv.kernel_source().encode()).hexdigest()[:16]
+
+
+def traffic_for(workload, conv, E):
+    """DRAM bytes per forward launch from the committed ncu summary, if the kernel is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None, None
+    d = json.load(open(p)).get(workload)
+    if not d or d.get("kernel_sha1") != kernel_hash(conv):
+        return None, None
+    return d["dram_bytes_per_edge"] * E, d.get("source")
+
+
+# ---------------------------------------------------------------------------
+# oracle sample (CPU baseline and reference arm)
+
+def oracle_sample_rate(spec, graph, rows, x_rows_fn, Y_fn, s_fn, threads=0):
+    """Times the oracle on the receivers `rows` (all their edges); returns (edges/s, edges, secs)."""
+    import numpy as np
+
+    import oracle
+    rp = np.zeros(graph.num_nodes + 1, np.int64)
+    np.cumsum(np.bincount(graph.receivers, minlength=graph.num_nodes), out=rp[1:])
+    edges = np.concatenate([np.arange(rp[b], rp[b + 1]) for b in rows])
+    senders = graph.senders[edges]
+    uniq, inv = np.unique(senders, return_inverse=True)
+    x = x_rows_fn(uniq).astype(np.float64)
+    Y = Y_fn(edges).astype(np.float64)
+    s = s_fn(edges).astype(np.float64)
+    n = max(len(rows), len(uniq))
+    xr = np.zeros((n,) + x.shape[1:])
+    xr[:len(uniq)] = x
+    recv = np.repeat(np.arange(len(rows)), np.diff(rp)[rows])
+    t0 = time.perf_counter()
+    oracle.forward(spec.irreps_node, spec.irreps_sh, spec.irreps_out, xr, Y, s, inv, recv, n,
+                   graph.avg_num_neighbors, threads=threads)
+    dt = time.perf_counter() - t0
+    return len(edges) / dt, len(edges), dt
+
+
+def calibrated_rows(spec, graph, x_rows_fn, Y_fn, s_fn, target_s, seed=2024):
+    import numpy as np
+    order = np.random.default_rng(seed).permutation(graph.num_nodes)
+    probe = order[: min(16, graph.num_nodes)]
+    rate, ne, dt = oracle_sample_rate(spec, graph, probe, x_rows_fn, Y_fn, s_fn)
+    per_row = max(ne / len(probe), 1e-9)
+    want = int(max(1, min(graph.num_nodes, rate * target_s / per_row)))
+    return np.sort(order[:want])
+
+
+def device_inputs_fns(x_d, Y_d, s_d):
+    import torch
+
+    def xf(rows):
+        return x_d[torch.from_numpy(rows).to(x_d.device)].cpu().numpy()
+
+    def yf(edges):
+        return Y_d[torch.from_numpy(edges).to(Y_d.device)].cpu().numpy()
+
+    def sf(edges):
+        return s_d[torch.from_numpy(edges).to(s_d.device)].cpu().numpy()
+    return xf, yf, sf
+
+
+# ---------------------------------------------------------------------------
+
+def spec_for_rank(name, rank):
+    from dataclasses import replace
+
+    from workloads import SPECS
+    spec = SPECS[name]
+    if rank:
+        spec = replace(spec, graph_seed=spec.graph_seed + 1000 * rank, seed=spec.seed + 1000 * rank)
+    return spec
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    from workloads import configs
+    spec = spec_for_rank(args.workload, 0)
+    g = configs.make_graph(spec, args.nodes)
+    xf = lambda rows: configs.node_features_np(spec, g.num_nodes, rows)
+    yf = lambda edges: configs.real_sh(g.vec[edges], spec.lmax).astype(configs.np_dtype(spec))
+    sf = lambda edges: configs.scalars_np(spec, g, edges)
+    per_step = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    rows = calibrated_rows(spec, g, xf, yf, sf, per_step)
+    for _ in range(args.warmup):
+        oracle_sample_rate(spec, g, rows, xf, yf, sf)
+    tot_e, tot_t = 0, 0.0
+    for _ in range(args.steps):
+        _, ne, dt = oracle_sample_rate(spec, g, rows, xf, yf, sf)
+        tot_e += ne
+        tot_t += dt
+    value = tot_e / tot_t
+    cores = oracle.max_threads()
+    sample = (f"{len(rows)} seeded receivers of {g.num_nodes} with all their "
+              f"{tot_e // max(1, args.steps)} edges per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": spec.name, "description": spec.description, "nodes": g.num_nodes,
+                   "edges": g.num_edges},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import equivariant_graph_message_b200 as e3
+    from workloads import configs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    spec = spec_for_rank(args.workload, rank)
+    g = configs.make_graph(spec, args.nodes)
+    N, E = g.num_nodes, g.num_edges
+    x = configs.node_features_torch(spec, N, dev)
+    Y = torch.from_numpy(configs.edge_sh(spec, g)).to(dev)
+    s = configs.scalars_torch(spec, g, dev)
+    senders = torch.from_numpy(g.senders.astype(np.int32)).to(dev)
+    receivers = torch.from_numpy(g.receivers.astype(np.int32)).to(dev)
+    conv = e3.Conv(spec.irreps_node, spec.irreps_sh, spec.irreps_out, g.avg_num_neighbors,
+                   dtype=spec.dtype)
+    if args.channels_per_lane or args.block_threads:
+        conv.set_launch_config(args.channels_per_lane, args.block_threads)
+    row_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(E, dtype=torch.int32, device=dev)
+    ws = torch.empty(e3.csr_workspace_size(E, N), dtype=torch.uint8, device=dev)
+    out = torch.empty((N, conv.nout, conv.C), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    sh = e3._stream_handle(stream)
+    px, pY, ps, psend, prp, pout = (e3._ptr(t) for t in (x, Y, s, senders, row_ptr, out))
+    precv, pperm, pws = e3._ptr(receivers), e3._ptr(perm), e3._ptr(ws)
+    ws_bytes = ws.numel()
+
+    def step(fwd_events=None):
+        e3._ok(e3._build_csr(precv, E, N, prp, pperm, pws, ws_bytes, sh), "e3conv_build_csr")
+        if fwd_events:
+            fwd_events[0].record(stream)
+        conv.forward_raw(px, pY, ps, psend, prp, N, E, pout, sh)
+        if fwd_events:
+            fwd_events[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert e3.csr_check(ws) and conv.check(), "bad index met during warm-up"
+    info = conv.kernel_info()
+
+    clocks = Clocks(local)
+    clocks.start()
+    fwd = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for k in range(args.steps):
+        step(fwd[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd)
+    ms_t = torch.tensor([ms, fwd_ms], dtype=torch.float64, device=dev)
+    e_t = torch.tensor([float(E)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(e_t, op=dist.ReduceOp.SUM)
+    ms, fwd_ms = ms_t.tolist()
+    total_edges = e_t.item()
+    ms_per_step = ms / args.steps
+    value = total_edges / (ms_per_step / 1000.0)
+
+    pk = peaks()
+    in_bytes = 2 if spec.dtype == "f16" else 4
+    nbytes, flops, nnz, mix = algorithmic(conv, N, E, in_bytes)
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    t_alu = flops / (pk["fp32_tflops"] * 1e12)
+    traffic, traffic_src = traffic_for(spec.name if args.nodes is None else None, conv, E)
+    if t_alu >= t_hbm:
+        achieved = flops / (fwd_ms / 1000.0) / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": pk["fp32_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / pk["fp32_tflops"],
+                "traffic": traffic,
+                "peak_source": f"derived: {SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 x "
+                               f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})"}
+    else:
+        achieved = nbytes / (fwd_ms / 1000.0) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                "peak_source": f"hbm_gbs ({pk['source']})"}
+    roof.update({"kernel": "e3conv_fwd", "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+                 "forward_ms": fwd_ms, "hbm_frac": nbytes / (fwd_ms / 1000.0) / 1e9 / pk["hbm_gbs"],
+                 "alu_frac": flops / (fwd_ms / 1000.0) / 1e12 / pk["fp32_tflops"],
+                 "traffic_source": traffic_src})
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        xf, yf, sf = device_inputs_fns(x, Y, s)
+        rows = calibrated_rows(spec, g, xf, yf, sf, args.cpu_seconds)
+        rate, ne, dt = oracle_sample_rate(spec, g, rows, xf, yf, sf)
+        cpu = {"value": rate, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+               "sample": f"{len(rows)} seeded receivers of {N} with all their {ne} edges "
+                         f"({dt:.1f} s, float64 loops, OpenMP over receivers)"}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, conv, spec, g, x, Y, s, senders, receivers, row_ptr, perm, ws, out,
+                      world, dev)
+
+    launches = args.steps * (e3.csr_kernel_count(E, N) + 1)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": spec.name, "description": spec.description, "nodes": N,
+                   "edges": E, "edges_total": int(total_edges), "channels": conv.C,
+                   "irreps_node": spec.irreps_node, "irreps_sh": spec.irreps_sh,
+                   "irreps_out": spec.irreps_out, "input_dtype": spec.dtype,
+                   "step": "e3conv_build_csr + e3conv_forward",
+                   "l2": f"inputs larger than L2 ({nbytes / 1e9:.1f} GB read per forward)",
+                   "forward_edges_per_s": total_edges / (fwd_ms / 1000.0),
+                   "kernel": info},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(args, conv, spec, g, x, Y, s, senders, receivers, row_ptr, perm, ws, out, world, dev):
+    """Same step through the public API with pinned host inputs and a host result."""
+    import torch
+    import torch.distributed as dist
+
+    import equivariant_graph_message_b200 as e3
+    tensors = [x, Y, s, senders, receivers]
+    h2d = sum(t.numel() * t.element_size() for t in tensors)
+    d2h = out.numel() * out.element_size()
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = 0
+    ok = torch.tensor([1 if avail > 1.3 * (h2d + d2h) + (8 << 30) else 0], device=dev)
+    if world > 1:
+        dist.all_reduce(ok, op=dist.ReduceOp.MIN)
+    if not ok.item():
+        return {"value": None, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "skipped": f"host memory available {avail / 2**30:.0f} GiB < needed pinned "
+                           f"{(h2d + d2h) / 2**30:.0f} GiB"}
+    host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in tensors]
+    for h, t in zip(host, tensors):
+        h.copy_(t)
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    steps = max(1, min(args.steps, 5))
+    N, E = g.num_nodes, g.num_edges
+
+    def step():
+        for h, t in zip(host, tensors):
+            t.copy_(h, non_blocking=True)
+        e3.build_csr(receivers, N, row_ptr=row_ptr, perm=perm, workspace=ws)
+        conv.forward(x, Y, s, senders, row_ptr, out=out)
+        out_h.copy_(out, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = torch.tensor([a.elapsed_time(b) / steps], dtype=torch.float64, device=dev)
+    e_t = torch.tensor([float(E)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+        dist.all_reduce(e_t, op=dist.ReduceOp.SUM)
+    del host, out_h
+    return {"value": e_t.item() / (ms.item() / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms.item()}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,282 @@
+"""Equivariant message-passing convolution for NVIDIA B200 (sm_100a).
+
+Thin ctypes binding of libe3conv.so (C ABI in include/e3conv.h).  This
+module only marshals arguments: every step of the convolution, the CSR
+indexing and the row gather run in the library's CUDA kernels.  PyTorch is
+used for device memory and streams only.  There is no CPU fallback: if the
+library is missing, importing this package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libe3conv.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -c 'import __graft_entry__ as g; g.build()'` "
+                      "or `python -m equivariant_graph_message_b200._build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+F32, F16 = 0, 1
+NORM = {"SQRT_DIM_OUT": 0, "NONE": 1}
+ERR_BAD_INDEX = 8
+
+_c_int_p = ctypes.POINTER(ctypes.c_int)
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+
+
+def _sig(name, restype, *argtypes):
+    fn = getattr(_lib, name)
+    fn.restype = restype
+    fn.argtypes = list(argtypes)
+    return fn
+
+
+_create = _sig("e3conv_create", ctypes.c_int, ctypes.POINTER(_vp), ctypes.c_char_p,
+               ctypes.c_char_p, ctypes.c_char_p, ctypes.c_double, ctypes.c_int)
+_destroy = _sig("e3conv_destroy", None, _vp)
+_set_dtype = _sig("e3conv_set_input_dtype", ctypes.c_int, _vp, ctypes.c_int)
+_set_launch = _sig("e3conv_set_launch_config", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_int)
+_query = _sig("e3conv_query", ctypes.c_int, _vp, *([_c_int_p] * 5))
+_path = _sig("e3conv_path", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 7))
+_num_outputs = _sig("e3conv_num_outputs", ctypes.c_int, _vp, _c_int_p)
+_output_irrep = _sig("e3conv_output_irrep", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 3))
+_cg = _sig("e3conv_cg", ctypes.c_int, _vp, ctypes.c_int, ctypes.POINTER(ctypes.c_double))
+_kernel_info = _sig("e3conv_kernel_info", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 5))
+_kernel_source = _sig("e3conv_kernel_source", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_char_p,
+                      ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t))
+_forward = _sig("e3conv_forward", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp,
+                _vp)
+_check = _sig("e3conv_check", ctypes.c_int, _vp, _vp)
+_csr_ws = _sig("e3conv_csr_workspace_size", ctypes.c_int, _i64, _i64,
+               ctypes.POINTER(ctypes.c_size_t))
+_build_csr = _sig("e3conv_build_csr", ctypes.c_int, _vp, _i64, _i64, _vp, _vp, _vp,
+                  ctypes.c_size_t, _vp)
+_csr_check = _sig("e3conv_csr_check", ctypes.c_int, _vp, _vp)
+_csr_count = _sig("e3conv_csr_kernel_count", ctypes.c_int, _i64, _i64, _c_int_p)
+_permute = _sig("e3conv_permute_rows", ctypes.c_int, _vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp)
+_strerror = _sig("e3conv_strerror", ctypes.c_char_p, ctypes.c_int)
+_last_error = _sig("e3conv_last_error", ctypes.c_char_p)
+_version = _sig("e3conv_version", ctypes.c_int)
+
+EXPORTED = ["e3conv_create", "e3conv_destroy", "e3conv_set_input_dtype",
+            "e3conv_set_launch_config", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
+            "e3conv_output_irrep", "e3conv_cg", "e3conv_kernel_info", "e3conv_kernel_source",
+            "e3conv_forward", "e3conv_check", "e3conv_csr_workspace_size", "e3conv_build_csr",
+            "e3conv_csr_check", "e3conv_csr_kernel_count", "e3conv_permute_rows", "e3conv_strerror", "e3conv_last_error",
+            "e3conv_version"]
+
+
+class E3ConvError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        msg = _last_error().decode(errors="replace")
+        super().__init__(f"{where}: {_strerror(code).decode()} ({code}): {msg}")
+
+
+def _ok(code: int, where: str):
+    if code != 0:
+        raise E3ConvError(code, where)
+
+
+def version() -> int:
+    return _version()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+@dataclass(frozen=True)
+class PathInfo:
+    l1: int
+    p1: int
+    l2: int
+    l3: int
+    p3: int
+    x_off: int
+    out_off: int
+
+
+class Conv:
+    """One plan of the convolution (e3conv_create / e3conv_forward)."""
+
+    def __init__(self, irreps_node: str, irreps_sh: str, irreps_out: str,
+                 avg_num_neighbors: float, normalization: str = "SQRT_DIM_OUT",
+                 dtype: str = "f32"):
+        h = _vp()
+        _ok(_create(ctypes.byref(h), irreps_node.encode(), irreps_sh.encode(),
+                    irreps_out.encode(), float(avg_num_neighbors), NORM[normalization]),
+            "e3conv_create")
+        self._h = h
+        vals = [ctypes.c_int() for _ in range(5)]
+        _ok(_query(h, *[ctypes.byref(v) for v in vals]), "e3conv_query")
+        self.C, self.nx, self.ny, self.nout, self.num_paths = (v.value for v in vals)
+        self.dtype = "f32"
+        if dtype != "f32":
+            self.set_dtype(dtype)
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h:
+            _destroy(h)
+            self._h = None
+
+    def close(self):
+        self.__del__()
+
+    # ---- plan inspection
+    @property
+    def paths(self) -> list[PathInfo]:
+        out = []
+        for p in range(self.num_paths):
+            v = [ctypes.c_int() for _ in range(7)]
+            _ok(_path(self._h, p, *[ctypes.byref(x) for x in v]), "e3conv_path")
+            out.append(PathInfo(*(x.value for x in v)))
+        return out
+
+    @property
+    def outputs(self) -> list[tuple[int, int, int]]:
+        n = ctypes.c_int()
+        _ok(_num_outputs(self._h, ctypes.byref(n)), "e3conv_num_outputs")
+        res = []
+        for k in range(n.value):
+            v = [ctypes.c_int() for _ in range(3)]
+            _ok(_output_irrep(self._h, k, *[ctypes.byref(x) for x in v]), "e3conv_output_irrep")
+            res.append(tuple(x.value for x in v))
+        return res
+
+    def cg(self, p: int) -> np.ndarray:
+        q = self.paths[p]
+        shape = (2 * q.l1 + 1, 2 * q.l2 + 1, 2 * q.l3 + 1)
+        buf = np.zeros(int(np.prod(shape)), dtype=np.float64)
+        _ok(_cg(self._h, p, buf.ctypes.data_as(ctypes.POINTER(ctypes.c_double))), "e3conv_cg")
+        return buf.reshape(shape)
+
+    def set_dtype(self, dtype: str):
+        _ok(_set_dtype(self._h, {"f32": F32, "f16": F16}[dtype]), "e3conv_set_input_dtype")
+        self.dtype = dtype
+
+    def set_launch_config(self, channels_per_lane: int = 0, block_threads: int = 0):
+        _ok(_set_launch(self._h, channels_per_lane, block_threads), "e3conv_set_launch_config")
+
+    def kernel_info(self, dtype: str | None = None) -> dict:
+        v = [ctypes.c_int() for _ in range(5)]
+        _ok(_kernel_info(self._h, {"f32": F32, "f16": F16}[dtype or self.dtype],
+                         *[ctypes.byref(x) for x in v]), "e3conv_kernel_info")
+        keys = ["channels_per_lane", "lanes_per_tile", "block_threads", "registers", "local_bytes"]
+        return dict(zip(keys, (x.value for x in v)))
+
+    def kernel_source(self, dtype: str | None = None) -> str:
+        d = {"f32": F32, "f16": F16}[dtype or self.dtype]
+        n = ctypes.c_size_t()
+        _ok(_kernel_source(self._h, d, None, 0, ctypes.byref(n)), "e3conv_kernel_source")
+        buf = ctypes.create_string_buffer(n.value)
+        _ok(_kernel_source(self._h, d, buf, n.value, ctypes.byref(n)), "e3conv_kernel_source")
+        return buf.value.decode()
+
+    # ---- device calls
+    def forward(self, x, Y, s, senders, row_ptr, out=None, stream=None):
+        """out[N][nout][C] float32 from receiver-sorted edges (torch CUDA tensors)."""
+        import torch
+        N = x.shape[0]
+        E = senders.shape[0]
+        want = torch.float16 if self.dtype == "f16" else torch.float32
+        for name, t in (("x", x), ("Y", Y), ("s", s)):
+            if t.dtype != want or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous {want} tensor")
+        if tuple(x.shape) != (N, self.nx, self.C):
+            raise ValueError(f"x shape {tuple(x.shape)} != {(N, self.nx, self.C)}")
+        if tuple(Y.shape) != (E, self.ny) or tuple(s.shape) != (E, self.num_paths, self.C):
+            raise ValueError("Y / s shapes do not match the plan")
+        if senders.dtype != torch.int32 or row_ptr.dtype != torch.int32:
+            raise ValueError("senders and row_ptr must be int32")
+        if row_ptr.shape[0] != N + 1:
+            raise ValueError("row_ptr must have num_nodes + 1 entries")
+        if out is None:
+            out = torch.empty((N, self.nout, self.C), dtype=torch.float32, device=x.device)
+        _ok(_forward(self._h, _ptr(x), _ptr(Y) if E else None, _ptr(s) if E else None,
+                     _ptr(senders) if E else None, _ptr(row_ptr), N, E, _ptr(out),
+                     _stream_handle(stream)), "e3conv_forward")
+        return out
+
+    def forward_raw(self, x_ptr, Y_ptr, s_ptr, senders_ptr, row_ptr_ptr, num_nodes, num_edges,
+                    out_ptr, stream_handle):
+        """Pointer-level call of e3conv_forward (for timing loops)."""
+        _ok(_forward(self._h, x_ptr, Y_ptr, s_ptr, senders_ptr, row_ptr_ptr, num_nodes,
+                     num_edges, out_ptr, stream_handle), "e3conv_forward")
+
+    def check(self, stream=None) -> bool:
+        """True if no forward since the last check met a bad index."""
+        rc = _check(self._h, _stream_handle(stream))
+        if rc == ERR_BAD_INDEX:
+            return False
+        _ok(rc, "e3conv_check")
+        return True
+
+
+def csr_workspace_size(num_edges: int, num_nodes: int) -> int:
+    n = ctypes.c_size_t()
+    _ok(_csr_ws(num_edges, num_nodes, ctypes.byref(n)), "e3conv_csr_workspace_size")
+    return n.value
+
+
+def build_csr(receivers, num_nodes: int, row_ptr=None, perm=None, workspace=None, stream=None):
+    """(row_ptr int32 [N+1], perm int32 [E]) of int32 device `receivers`."""
+    import torch
+    E = receivers.shape[0]
+    dev = receivers.device
+    if receivers.dtype != torch.int32:
+        raise ValueError("receivers must be int32")
+    if row_ptr is None:
+        row_ptr = torch.empty(num_nodes + 1, dtype=torch.int32, device=dev)
+    if perm is None:
+        perm = torch.empty(max(E, 1), dtype=torch.int32, device=dev)[:E]
+    nbytes = csr_workspace_size(E, num_nodes)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _ok(_build_csr(_ptr(receivers) if E else None, E, num_nodes, _ptr(row_ptr),
+                   _ptr(perm) if E else None, _ptr(workspace), workspace.numel(),
+                   _stream_handle(stream)), "e3conv_build_csr")
+    return row_ptr, perm, workspace
+
+
+def csr_kernel_count(num_edges: int, num_nodes: int) -> int:
+    n = ctypes.c_int()
+    _ok(_csr_count(num_edges, num_nodes, ctypes.byref(n)), "e3conv_csr_kernel_count")
+    return n.value
+
+
+def csr_check(workspace, stream=None) -> bool:
+    rc = _csr_check(_ptr(workspace), _stream_handle(stream))
+    if rc == ERR_BAD_INDEX:
+        return False
+    _ok(rc, "e3conv_csr_check")
+    return True
+
+
+def permute_rows(src, perm, dst=None, status=None, stream=None):
+    """dst[t] = src[perm[t]] along the first axis (device)."""
+    import torch
+    rows = perm.shape[0]
+    row_bytes = src[0].numel() * src.element_size() if src.shape[0] else 0
+    if dst is None:
+        dst = torch.empty((rows,) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    _ok(_permute(_ptr(src), src.shape[0], _ptr(perm), rows, row_bytes, _ptr(dst), _ptr(status),
+                 _stream_handle(stream)), "e3conv_permute_rows")
+    return dst

@@ -1,0 +1,493 @@
+// C ABI of libe3conv: plans, NVRTC compilation, launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <nvrtc.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <regex>
+#include <stdexcept>
+#include <string>
+
+#include "plan.h"
+
+namespace e3c {
+size_t csr_workspace_bytes(int64_t E, int64_t N);
+int csr_build(const int* recv, int64_t E, int64_t N, int* row_ptr, int* perm, void* ws,
+              size_t ws_bytes, cudaStream_t st, std::string& err, int* count);
+int csr_read_status(const void* ws, cudaStream_t st, unsigned* out);
+int permute_rows(const void* src, int64_t num_src, const int* perm, int64_t rows, int64_t row_bytes,
+                 void* dst, int* status, cudaStream_t st, std::string& err);
+}  // namespace e3c
+
+using namespace e3c;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const std::string& msg) {
+  g_last_error = msg;
+  return code;
+}
+
+// Driver API entry points, resolved through the runtime so the library does
+// not link libcuda (it must load on machines without a GPU driver).
+struct Driver {
+  CUresult (*ModuleLoadData)(CUmodule*, const void*) = nullptr;
+  CUresult (*ModuleUnload)(CUmodule) = nullptr;
+  CUresult (*ModuleGetFunction)(CUfunction*, CUmodule, const char*) = nullptr;
+  CUresult (*LaunchKernel)(CUfunction, unsigned, unsigned, unsigned, unsigned, unsigned, unsigned,
+                           unsigned, CUstream, void**, void**) = nullptr;
+  CUresult (*FuncGetAttribute)(int*, CUfunction_attribute, CUfunction) = nullptr;
+  CUresult (*CtxGetCurrent)(CUcontext*) = nullptr;
+  bool ok = false;
+};
+
+Driver& driver() {
+  static Driver d;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    auto get = [](const char* name, void** fn) {
+      cudaDriverEntryPointQueryResult q;
+      return cudaGetDriverEntryPoint(name, fn, cudaEnableDefault, &q) == cudaSuccess &&
+             q == cudaDriverEntryPointSuccess && *fn != nullptr;
+    };
+    d.ok = get("cuModuleLoadData", reinterpret_cast<void**>(&d.ModuleLoadData)) &&
+           get("cuModuleUnload", reinterpret_cast<void**>(&d.ModuleUnload)) &&
+           get("cuModuleGetFunction", reinterpret_cast<void**>(&d.ModuleGetFunction)) &&
+           get("cuLaunchKernel", reinterpret_cast<void**>(&d.LaunchKernel)) &&
+           get("cuFuncGetAttribute", reinterpret_cast<void**>(&d.FuncGetAttribute)) &&
+           get("cuCtxGetCurrent", reinterpret_cast<void**>(&d.CtxGetCurrent));
+    cudaGetLastError();
+  });
+  return d;
+}
+
+bool has_device() {
+  int n = 0;
+  cudaError_t e = cudaGetDeviceCount(&n);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return n > 0;
+}
+
+int compile_variant(Plan& pl, int dtype) {
+  Variant& v = pl.var[dtype];
+  v = Variant{};
+  v.shape = choose_shape(pl, dtype);
+  v.source = generate_forward_source(pl, dtype, v.shape);
+  nvrtcProgram prog;
+  if (nvrtcCreateProgram(&prog, v.source.c_str(), "e3conv_fwd.cu", 0, nullptr, nullptr) !=
+      NVRTC_SUCCESS)
+    return fail(E3CONV_ERR_COMPILE, "nvrtcCreateProgram failed");
+  const char* opts[] = {"--gpu-architecture=sm_100a", "--std=c++17", "-lineinfo",
+                        "--ptxas-options=-v"};
+  nvrtcResult rc = nvrtcCompileProgram(prog, 4, opts);
+  size_t log_size = 0;
+  nvrtcGetProgramLogSize(prog, &log_size);
+  v.log.assign(log_size, '\0');
+  if (log_size) nvrtcGetProgramLog(prog, &v.log[0]);
+  if (rc != NVRTC_SUCCESS) {
+    nvrtcDestroyProgram(&prog);
+    return fail(E3CONV_ERR_COMPILE, "NVRTC compile failed: " + v.log.substr(0, 2000));
+  }
+  size_t n = 0;
+  nvrtcGetCUBINSize(prog, &n);
+  v.cubin.resize(n);
+  nvrtcGetCUBIN(prog, v.cubin.data());
+  nvrtcDestroyProgram(&prog);
+  std::smatch m;
+  if (std::regex_search(v.log, m, std::regex("Used ([0-9]+) registers"))) v.regs = std::stoi(m[1]);
+  if (std::regex_search(v.log, m, std::regex("([0-9]+) bytes spill stores")))
+    v.local_bytes = std::stoi(m[1]);
+  v.compiled = true;
+  if (pl.device >= 0) {
+    Driver& d = driver();
+    if (d.ModuleLoadData(&v.module, v.cubin.data()) != CUDA_SUCCESS)
+      return fail(E3CONV_ERR_CUDA, "cuModuleLoadData failed");
+    if (d.ModuleGetFunction(&v.fn, v.module, "e3conv_fwd") != CUDA_SUCCESS)
+      return fail(E3CONV_ERR_CUDA, "cuModuleGetFunction failed");
+    int regs = 0, local = 0;
+    d.FuncGetAttribute(&regs, CU_FUNC_ATTRIBUTE_NUM_REGS, v.fn);
+    d.FuncGetAttribute(&local, CU_FUNC_ATTRIBUTE_LOCAL_SIZE_BYTES, v.fn);
+    v.regs = regs;
+    v.local_bytes = local;
+  }
+  return E3CONV_OK;
+}
+
+void release_variant(Variant& v) {
+  if (v.module) driver().ModuleUnload(v.module);
+  v.module = nullptr;
+  v.fn = nullptr;
+  v.compiled = false;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Makes the plan's device current for the duration of a call.
+struct DeviceGuard {
+  int prev = -1;
+  bool changed = false;
+  explicit DeviceGuard(int dev) {
+    if (dev < 0) return;
+    if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) {
+      changed = cudaSetDevice(dev) == cudaSuccess;
+    }
+  }
+  ~DeviceGuard() {
+    if (changed) cudaSetDevice(prev);
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+int e3conv_version(void) { return E3CONV_VERSION; }
+
+const char* e3conv_strerror(int code) {
+  switch (code) {
+    case E3CONV_OK: return "ok";
+    case E3CONV_ERR_INVALID_ARG: return "invalid argument";
+    case E3CONV_ERR_IRREPS: return "invalid irreps";
+    case E3CONV_ERR_UNSUPPORTED: return "unsupported";
+    case E3CONV_ERR_CUDA: return "CUDA error";
+    case E3CONV_ERR_NOMEM: return "out of memory";
+    case E3CONV_ERR_COMPILE: return "kernel compilation failed";
+    case E3CONV_ERR_NO_DEVICE: return "plan has no device module";
+    case E3CONV_ERR_BAD_INDEX: return "out-of-range index met by a kernel";
+    case E3CONV_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown error code";
+  }
+}
+
+const char* e3conv_last_error(void) { return g_last_error.c_str(); }
+
+int e3conv_create(e3conv_plan* out, const char* irreps_node, const char* irreps_sh,
+                  const char* irreps_out, double avg_num_neighbors, int normalization) {
+  if (!out) return fail(E3CONV_ERR_INVALID_ARG, "plan pointer is NULL");
+  *out = nullptr;
+  if (!(avg_num_neighbors > 0) || !std::isfinite(avg_num_neighbors))
+    return fail(E3CONV_ERR_INVALID_ARG, "avg_num_neighbors must be positive and finite");
+  if (normalization != E3CONV_NORM_SQRT_DIM_OUT && normalization != E3CONV_NORM_NONE)
+    return fail(E3CONV_ERR_UNSUPPORTED, "unknown normalization");
+  e3conv_plan h = new (std::nothrow) e3conv_plan_s;
+  if (!h) return fail(E3CONV_ERR_NOMEM, "host allocation failed");
+  Plan& pl = h->p;
+  pl.avg = avg_num_neighbors;
+  pl.norm = normalization;
+  std::string err;
+  std::vector<Irrep> sh;
+  if (!parse_irreps(irreps_node, pl.node, err) || !parse_irreps(irreps_sh, sh, err) ||
+      !parse_irreps(irreps_out, pl.filt, err)) {
+    delete h;
+    return fail(E3CONV_ERR_IRREPS, err);
+  }
+  for (size_t k = 0; k < sh.size(); ++k) {
+    if (sh[k].mul != 1 || sh[k].l != static_cast<int>(k) || sh[k].p != ((k % 2) ? -1 : 1)) {
+      delete h;
+      return fail(E3CONV_ERR_IRREPS,
+                  "irreps_sh must be 1x0e+1x1o+1x2e+... (consecutive l from 0, parity (-1)^l)");
+    }
+  }
+  pl.lmax = static_cast<int>(sh.size()) - 1;
+  if (pl.lmax > 6) {
+    delete h;
+    return fail(E3CONV_ERR_UNSUPPORTED, "spherical-harmonic degree above 6");
+  }
+  int rc;
+  try {
+    rc = build_paths(pl, err);
+  } catch (const std::exception& ex) {
+    rc = E3CONV_ERR_IRREPS;
+    err = ex.what();
+  }
+  if (rc != E3CONV_OK) {
+    delete h;
+    return fail(rc, err);
+  }
+  if (pl.paths.empty()) {
+    delete h;
+    return fail(E3CONV_ERR_IRREPS, "no path produces any requested output irrep");
+  }
+  if (static_cast<long long>(pl.nx) * pl.C >= (1ll << 31) ||
+      static_cast<long long>(pl.nout) * pl.C >= (1ll << 31)) {
+    delete h;
+    return fail(E3CONV_ERR_UNSUPPORTED, "feature row too large");
+  }
+  if (has_device()) {
+    if (!driver().ok) {
+      delete h;
+      return fail(E3CONV_ERR_CUDA, "CUDA driver entry points unavailable");
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaFree(nullptr) != cudaSuccess) {
+      cudaGetLastError();
+      delete h;
+      return fail(E3CONV_ERR_CUDA, "cannot initialise the CUDA context");
+    }
+    pl.device = dev;
+    driver().CtxGetCurrent(&pl.ctx);
+    if (cudaMalloc(&pl.status, sizeof(unsigned int)) != cudaSuccess) {
+      cudaGetLastError();
+      delete h;
+      return fail(E3CONV_ERR_NOMEM, "cudaMalloc of the status word failed");
+    }
+    cudaMemset(pl.status, 0, sizeof(unsigned int));
+  }
+  rc = compile_variant(pl, E3CONV_F32);
+  if (rc != E3CONV_OK) {
+    std::string msg = g_last_error;
+    e3conv_destroy(h);
+    return fail(rc, msg);
+  }
+  *out = h;
+  return E3CONV_OK;
+}
+
+void e3conv_destroy(e3conv_plan h) {
+  if (!h) return;
+  Plan& pl = h->p;
+  {
+    DeviceGuard g(pl.device);
+    for (auto& v : pl.var) release_variant(v);
+    if (pl.status) cudaFree(pl.status);
+  }
+  delete h;
+}
+
+int e3conv_set_input_dtype(e3conv_plan h, int dtype) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  if (dtype != E3CONV_F32 && dtype != E3CONV_F16)
+    return fail(E3CONV_ERR_UNSUPPORTED, "dtype must be E3CONV_F32 or E3CONV_F16");
+  Plan& pl = h->p;
+  if (!pl.var[dtype].compiled) {
+    DeviceGuard g(pl.device);
+    int rc = compile_variant(pl, dtype);
+    if (rc != E3CONV_OK) return rc;
+  }
+  pl.dtype = dtype;
+  return E3CONV_OK;
+}
+
+int e3conv_set_launch_config(e3conv_plan h, int channels_per_lane, int block_threads) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  Plan& pl = h->p;
+  const int V = channels_per_lane;
+  if (V != 0 && V != 1 && V != 2 && V != 4 && V != 8)
+    return fail(E3CONV_ERR_INVALID_ARG, "channels_per_lane must be 0, 1, 2, 4 or 8");
+  if (V > 0 && pl.C % V != 0)
+    return fail(E3CONV_ERR_INVALID_ARG, "channels_per_lane must divide C");
+  if (V * (pl.dtype == E3CONV_F16 ? 2 : 4) > 16)
+    return fail(E3CONV_ERR_INVALID_ARG, "channels_per_lane exceeds one 16-byte load");
+  if (block_threads != 0 && (block_threads < 32 || block_threads > 1024 || block_threads % 32))
+    return fail(E3CONV_ERR_INVALID_ARG, "block_threads must be 0 or a multiple of 32 in [32, 1024]");
+  pl.req_V = V;
+  pl.req_block = block_threads;
+  DeviceGuard g(pl.device);
+  const int other = pl.dtype == E3CONV_F32 ? E3CONV_F16 : E3CONV_F32;
+  release_variant(pl.var[other]);
+  release_variant(pl.var[pl.dtype]);
+  return compile_variant(pl, pl.dtype);
+}
+
+int e3conv_query(e3conv_plan h, int* C, int* nx, int* ny, int* nout, int* num_paths) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  const Plan& pl = h->p;
+  if (C) *C = pl.C;
+  if (nx) *nx = pl.nx;
+  if (ny) *ny = pl.ny;
+  if (nout) *nout = pl.nout;
+  if (num_paths) *num_paths = static_cast<int>(pl.paths.size());
+  return E3CONV_OK;
+}
+
+int e3conv_path(e3conv_plan h, int p, int* l1, int* p1, int* l2, int* l3, int* p3, int* x_off,
+                int* out_off) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  const Plan& pl = h->p;
+  if (p < 0 || p >= static_cast<int>(pl.paths.size()))
+    return fail(E3CONV_ERR_INVALID_ARG, "path index out of range");
+  const Path& q = pl.paths[p];
+  if (l1) *l1 = q.l1;
+  if (p1) *p1 = q.p1;
+  if (l2) *l2 = q.l2;
+  if (l3) *l3 = q.l3;
+  if (p3) *p3 = q.p3;
+  if (x_off) *x_off = q.x_off;
+  if (out_off) *out_off = q.out_off;
+  return E3CONV_OK;
+}
+
+int e3conv_num_outputs(e3conv_plan h, int* count) {
+  if (!h || !count) return fail(E3CONV_ERR_INVALID_ARG, "NULL argument");
+  *count = static_cast<int>(h->p.outputs.size());
+  return E3CONV_OK;
+}
+
+int e3conv_output_irrep(e3conv_plan h, int k, int* l, int* p, int* offset) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  const Plan& pl = h->p;
+  if (k < 0 || k >= static_cast<int>(pl.outputs.size()))
+    return fail(E3CONV_ERR_INVALID_ARG, "output index out of range");
+  if (l) *l = pl.outputs[k].l;
+  if (p) *p = pl.outputs[k].p;
+  if (offset) *offset = pl.outputs[k].off;
+  return E3CONV_OK;
+}
+
+int e3conv_cg(e3conv_plan h, int p, double* dense_out) {
+  if (!h || !dense_out) return fail(E3CONV_ERR_INVALID_ARG, "NULL argument");
+  const Plan& pl = h->p;
+  if (p < 0 || p >= static_cast<int>(pl.paths.size()))
+    return fail(E3CONV_ERR_INVALID_ARG, "path index out of range");
+  std::memcpy(dense_out, pl.paths[p].cg.data(), sizeof(double) * pl.paths[p].cg.size());
+  return E3CONV_OK;
+}
+
+int e3conv_kernel_info(e3conv_plan h, int dtype, int* V, int* TL, int* block, int* regs,
+                       int* local_bytes) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  if (dtype != E3CONV_F32 && dtype != E3CONV_F16)
+    return fail(E3CONV_ERR_UNSUPPORTED, "unknown dtype");
+  const Variant& v = h->p.var[dtype];
+  if (!v.compiled) return fail(E3CONV_ERR_INVALID_ARG, "variant not compiled (set_input_dtype)");
+  if (V) *V = v.shape.V;
+  if (TL) *TL = v.shape.TL;
+  if (block) *block = v.shape.block;
+  if (regs) *regs = v.regs;
+  if (local_bytes) *local_bytes = v.local_bytes;
+  return E3CONV_OK;
+}
+
+int e3conv_kernel_source(e3conv_plan h, int dtype, char* buf, size_t buf_len, size_t* needed) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  if (dtype != E3CONV_F32 && dtype != E3CONV_F16)
+    return fail(E3CONV_ERR_UNSUPPORTED, "unknown dtype");
+  const Variant& v = h->p.var[dtype];
+  if (!v.compiled) return fail(E3CONV_ERR_INVALID_ARG, "variant not compiled (set_input_dtype)");
+  if (needed) *needed = v.source.size() + 1;
+  if (buf && buf_len >= v.source.size() + 1) std::memcpy(buf, v.source.c_str(), v.source.size() + 1);
+  return E3CONV_OK;
+}
+
+int e3conv_forward(e3conv_plan h, const void* x, const void* Y, const void* s,
+                   const int32_t* senders, const int32_t* row_ptr, int64_t num_nodes,
+                   int64_t num_edges, float* out, e3conv_stream stream) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  Plan& pl = h->p;
+  if (num_nodes < 0 || num_edges < 0 || num_nodes >= (1ll << 31) || num_edges >= (1ll << 31))
+    return fail(E3CONV_ERR_INVALID_ARG, "num_nodes / num_edges out of range");
+  if (num_nodes == 0) return E3CONV_OK;
+  if (!x || !row_ptr || !out)
+    return fail(E3CONV_ERR_INVALID_ARG, "node_features, receiver_row_ptr and out are required");
+  if (num_edges > 0 && (!Y || !s || !senders))
+    return fail(E3CONV_ERR_INVALID_ARG, "edge_sh, edge_scalars and senders are required");
+  if (!aligned16(x) || !aligned16(out) || (num_edges > 0 && (!aligned16(Y) || !aligned16(s))))
+    return fail(E3CONV_ERR_INVALID_ARG, "feature buffers must be 16-byte aligned");
+  const Variant& v = pl.var[pl.dtype];
+  if (pl.device < 0 || !v.fn) return fail(E3CONV_ERR_NO_DEVICE, "plan has no device module");
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess || cur != pl.device)
+    return fail(E3CONV_ERR_INVALID_ARG, "current device differs from the plan's device");
+  const Shape& sh = v.shape;
+  const long long items = num_nodes * sh.tiles;
+  const long long warps = (items + sh.ipw - 1) / sh.ipw;
+  const long long blocks = (warps * 32 + sh.block - 1) / sh.block;
+  if (blocks >= (1ll << 31)) return fail(E3CONV_ERR_UNSUPPORTED, "grid too large");
+  int n32 = static_cast<int>(num_nodes), e32 = static_cast<int>(num_edges);
+  float inv_avg = static_cast<float>(1.0 / pl.avg);
+  void* args[] = {const_cast<void**>(&x), const_cast<void**>(&Y), const_cast<void**>(&s),
+                  const_cast<int32_t**>(&senders), const_cast<int32_t**>(&row_ptr),
+                  &n32, &e32, &out, &inv_avg, &pl.status};
+  CUresult r = driver().LaunchKernel(v.fn, static_cast<unsigned>(blocks), 1, 1,
+                                     static_cast<unsigned>(sh.block), 1, 1, 0,
+                                     reinterpret_cast<CUstream>(stream), args, nullptr);
+  if (r != CUDA_SUCCESS) return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed");
+  return E3CONV_OK;
+}
+
+int e3conv_check(e3conv_plan h, e3conv_stream stream) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  Plan& pl = h->p;
+  if (pl.device < 0) return fail(E3CONV_ERR_NO_DEVICE, "plan has no device");
+  unsigned st = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&st, pl.status, sizeof st, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return fail(E3CONV_ERR_CUDA, "reading the status word failed");
+  if (st) {
+    cudaMemsetAsync(pl.status, 0, sizeof st, s);
+    cudaStreamSynchronize(s);
+    return fail(E3CONV_ERR_BAD_INDEX, std::string("forward met ") +
+                                          ((st & 1u) ? "an invalid receiver_row_ptr range " : "") +
+                                          ((st & 2u) ? "an out-of-range sender" : ""));
+  }
+  return E3CONV_OK;
+}
+
+int e3conv_csr_workspace_size(int64_t num_edges, int64_t num_nodes, size_t* bytes) {
+  if (!bytes) return fail(E3CONV_ERR_INVALID_ARG, "bytes is NULL");
+  if (num_edges < 0 || num_nodes < 0 || num_edges >= (1ll << 31) || num_nodes >= (1ll << 31) - 1)
+    return fail(E3CONV_ERR_INVALID_ARG, "sizes out of range");
+  *bytes = csr_workspace_bytes(num_edges, num_nodes);
+  return E3CONV_OK;
+}
+
+int e3conv_build_csr(const int32_t* receivers, int64_t num_edges, int64_t num_nodes,
+                     int32_t* row_ptr, int32_t* perm, void* workspace, size_t workspace_bytes,
+                     e3conv_stream stream) {
+  if (num_edges < 0 || num_nodes < 0 || num_edges >= (1ll << 31) || num_nodes >= (1ll << 31) - 1)
+    return fail(E3CONV_ERR_INVALID_ARG, "sizes out of range");
+  if (!row_ptr || (num_edges > 0 && (!receivers || !perm)))
+    return fail(E3CONV_ERR_INVALID_ARG, "NULL buffer");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(E3CONV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (!has_device()) return fail(E3CONV_ERR_NO_DEVICE, "no CUDA device");
+  std::string err;
+  int rc = csr_build(receivers, num_edges, num_nodes, row_ptr, perm, workspace, workspace_bytes,
+                     reinterpret_cast<cudaStream_t>(stream), err, nullptr);
+  return rc == E3CONV_OK ? rc : fail(rc, err);
+}
+
+int e3conv_csr_kernel_count(int64_t num_edges, int64_t num_nodes, int* count) {
+  if (!count) return fail(E3CONV_ERR_INVALID_ARG, "count is NULL");
+  if (num_edges < 0 || num_nodes < 0 || num_edges >= (1ll << 31) || num_nodes >= (1ll << 31) - 1)
+    return fail(E3CONV_ERR_INVALID_ARG, "sizes out of range");
+  std::string err;
+  return csr_build(nullptr, num_edges, num_nodes, nullptr, nullptr, nullptr, 0, nullptr, err,
+                   count);
+}
+
+int e3conv_csr_check(const void* workspace, e3conv_stream stream) {
+  if (!workspace) return fail(E3CONV_ERR_INVALID_ARG, "workspace is NULL");
+  unsigned st = 0;
+  if (csr_read_status(workspace, reinterpret_cast<cudaStream_t>(stream), &st) != E3CONV_OK)
+    return fail(E3CONV_ERR_CUDA, "reading the CSR status word failed");
+  if (st) return fail(E3CONV_ERR_BAD_INDEX, "receivers outside [0, num_nodes)");
+  return E3CONV_OK;
+}
+
+int e3conv_permute_rows(const void* src, int64_t num_src_rows, const int32_t* perm,
+                        int64_t num_rows, int64_t row_bytes, void* dst, int32_t* status,
+                        e3conv_stream stream) {
+  if (num_rows < 0 || num_src_rows < 0 || row_bytes < 0 || row_bytes % 4)
+    return fail(E3CONV_ERR_INVALID_ARG, "bad sizes (row_bytes must be a multiple of 4)");
+  if (num_rows == 0 || row_bytes == 0) return E3CONV_OK;
+  if (!src || !dst || !perm) return fail(E3CONV_ERR_INVALID_ARG, "NULL buffer");
+  if (!aligned16(src) || !aligned16(dst))
+    return fail(E3CONV_ERR_INVALID_ARG, "src and dst must be 16-byte aligned");
+  if (!has_device()) return fail(E3CONV_ERR_NO_DEVICE, "no CUDA device");
+  std::string err;
+  int rc = permute_rows(src, num_src_rows, perm, num_rows, row_bytes, dst, status,
+                        reinterpret_cast<cudaStream_t>(stream), err);
+  return rc == E3CONV_OK ? rc : fail(rc, err);
+}
+
+}  // extern "C"

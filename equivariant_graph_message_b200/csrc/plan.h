@@ -1,0 +1,87 @@
+// Internal plan structures of libe3conv (host side).
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include <cuda.h>
+
+#include "../../include/e3conv.h"
+
+namespace e3c {
+
+struct Irrep {
+  int mul, l, p;  // p = +1 even, -1 odd
+  int dim() const { return 2 * l + 1; }
+};
+
+// One nonzero CG coefficient of a path: out[k] += c * x[i] * Y[j].
+struct Nnz {
+  int i, j, k;
+  double c;
+};
+
+struct Path {
+  int n1, l1, p1, x_off;  // node irrep index, degree, parity, first component
+  int l2, y_off;          // harmonic degree, first component (l2^2)
+  int o, l3, p3, out_off; // output irrep index, degree, parity, first component
+  std::vector<double> cg; // dense [2l1+1][2l2+1][2l3+1], normalisation included
+  std::vector<Nnz> nnz;   // entries with |c| > 1e-12
+};
+
+struct Output {
+  int l, p, off;
+};
+
+// Launch shape of the generated forward kernel.
+struct Shape {
+  int V = 1;       // channels per lane
+  int TL = 32;     // lanes per (receiver, channel tile) item
+  int tiles = 1;   // channel tiles per receiver
+  int ipw = 1;     // items per warp
+  int block = 128; // threads per block
+};
+
+struct Variant {
+  bool compiled = false;
+  Shape shape;
+  std::string source;
+  std::vector<char> cubin;
+  std::string log;
+  int regs = -1, local_bytes = -1;
+  CUmodule module = nullptr;
+  CUfunction fn = nullptr;
+};
+
+struct Plan {
+  int C = 0, nx = 0, ny = 0, nout = 0, lmax = 0;
+  std::vector<Irrep> node, filt;
+  std::vector<Path> paths;
+  std::vector<Output> outputs;
+  double avg = 1.0;
+  int norm = 0;
+  int dtype = E3CONV_F32;
+  int req_V = 0, req_block = 0;
+  int device = -1;                 // -1: host-only plan
+  CUcontext ctx = nullptr;
+  unsigned int* status = nullptr;  // device status word
+  Variant var[2];
+};
+
+// irreps.cpp
+bool parse_irreps(const char* text, std::vector<Irrep>& out, std::string& err);
+int build_paths(Plan& plan, std::string& err);
+
+// cg.cpp
+std::vector<double> real_wigner_3j(int l1, int l2, int l3);
+
+// codegen.cpp
+Shape choose_shape(const Plan& plan, int dtype);
+std::string generate_forward_source(const Plan& plan, int dtype, const Shape& shape);
+
+}  // namespace e3c
+
+struct e3conv_plan_s {
+  e3c::Plan p;
+};

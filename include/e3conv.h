@@ -1,0 +1,247 @@
+/*
+ * e3conv — equivariant message-passing convolution on one NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libe3conv.so.  Plain pointers and sizes only; every device buffer
+ * is owned and allocated by the caller.
+ *
+ * The operation (page "e3j.core.Convolution", class docstring and the
+ * "__call__" parameter list):
+ *
+ *     m_b = (1/N) sum_{a -> b} (x_a (x)_CG Y_ab) . s_ab
+ *
+ *   x_a   node features of the sender a, irreps `irreps_node`, all with one
+ *         multiplicity C (the channels);
+ *   Y_ab  edge features, the real spherical harmonics of the edge (no channel
+ *         axis; broadcast over channels, "__call__" notes);
+ *   (x)_CG the channelwise ("uvu") Clebsch-Gordan tensor product: channel u
+ *         of x times Y gives channel u of every produced irrep (cuEquivariance
+ *         notes, "Dense polynomial": channelwise products, weights first);
+ *   . s_ab  every path p and channel u is scaled by its own edge scalar
+ *         s_ab[p, u] (e3j "__call__": edge_scalars (num_edges, num_scalars, C));
+ *         paths that produce the same output irrep are summed;
+ *   1/N   avg_num_neighbors (e3j parameters), N > 0.
+ *
+ * Layout (trailing channels, e3j "layout: TRAILING_CHANNELS is faster"):
+ *   node_features [num_nodes][nx][C]     nx = sum over node irreps of 2l+1
+ *   edge_sh       [num_edges][ny]        ny = (lmax+1)^2, l-major, m = -l..l
+ *   edge_scalars  [num_edges][P][C]      P paths in the canonical order below
+ *   out           [num_nodes][nout][C]   float32, nout = sum over produced
+ *                                        output irreps of 2l+1
+ * Edges must be sorted by receiver (e3j "__call__" note: fused kernels need
+ * edges sorted by the endpoint of the graph ordering; RECEIVER ordering is
+ * the one used here): the edges of receiver b are
+ * receiver_row_ptr[b] .. receiver_row_ptr[b+1]-1, in any order.
+ *
+ * Canonical path order: node irrep (in the order given) -> spherical-harmonic
+ * degree l2 (ascending) -> output irrep (in the order of `irreps_out`).  A
+ * path (l1,p1) x (l2,(-1)^l2) -> (l3,p3) exists iff |l1-l2| <= l3 <= l1+l2
+ * and p3 = p1 (-1)^l2.  `irreps_out` is a filter: output irreps no path
+ * produces are dropped from `out` (e3j "target ... enforces a filter").
+ *
+ * Spherical-harmonic basis: real, component-normalised (sum_m Y_lm^2 = 2l+1),
+ * no Condon-Shortley phase, z polar axis, components m = -l..l; l = 1 is
+ * sqrt(3) (y, z, x).  The CG tensors are the real Wigner-3j tensors of this
+ * basis with unit Frobenius norm, sign fixed so that the first nonzero entry
+ * in row-major (i, j, k) order is positive, times sqrt(2 l3 + 1) for
+ * E3CONV_NORM_SQRT_DIM_OUT (the e3j default normalisation) or times 1 for
+ * E3CONV_NORM_NONE.
+ *
+ * Errors: every int-returning call returns E3CONV_OK (0) or an E3CONV_ERR_*
+ * code; nothing is thrown across the ABI.  e3conv_last_error() gives a
+ * message for the last failing call of the calling thread.  Device kernels
+ * never trap: out-of-range indices they read are skipped and recorded in a
+ * status word that e3conv_check() / e3conv_csr_check() report.
+ *
+ * Streams: every device call is stream-ordered on the given stream (NULL is
+ * the legacy default stream), does not synchronise the host and does not
+ * allocate memory.  e3conv_stream has the same type as cudaStream_t.
+ */
+#ifndef E3CONV_H
+#define E3CONV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define E3CONV_VERSION 1
+
+#if defined(__GNUC__)
+#define E3CONV_API __attribute__((visibility("default")))
+#else
+#define E3CONV_API
+#endif
+
+typedef struct e3conv_plan_s* e3conv_plan;
+typedef struct CUstream_st* e3conv_stream;
+
+/* error codes */
+#define E3CONV_OK 0
+#define E3CONV_ERR_INVALID_ARG 1   /* null pointer, negative size, misaligned buffer ... */
+#define E3CONV_ERR_IRREPS 2        /* irreps string malformed or inconsistent */
+#define E3CONV_ERR_UNSUPPORTED 3   /* valid request this library does not implement */
+#define E3CONV_ERR_CUDA 4          /* a CUDA runtime / driver call failed */
+#define E3CONV_ERR_NOMEM 5         /* host or device allocation failed (plan creation only) */
+#define E3CONV_ERR_COMPILE 6       /* NVRTC failed to compile the generated kernel */
+#define E3CONV_ERR_NO_DEVICE 7     /* plan has no device module (created without a GPU) */
+#define E3CONV_ERR_BAD_INDEX 8     /* a kernel met an out-of-range index (see checks) */
+#define E3CONV_ERR_WORKSPACE 9     /* workspace missing or too small */
+
+/* input element types */
+#define E3CONV_F32 0
+#define E3CONV_F16 1
+
+/* CG normalisations */
+#define E3CONV_NORM_SQRT_DIM_OUT 0
+#define E3CONV_NORM_NONE 1
+
+/* ---------------------------------------------------------------------------
+ * Plans
+ */
+
+/* Builds a plan: parses the irreps, enumerates the paths, generates the real
+ * CG tables in float64 on the host and compiles the forward kernel for
+ * sm_100a with NVRTC (all CG coefficients unrolled as constants).  If a CUDA
+ * device is current, the kernel module is loaded on it and a 4-byte status
+ * word is allocated there; without a device the plan is host-only (queries
+ * work, e3conv_forward returns E3CONV_ERR_NO_DEVICE).
+ *   irreps_node: e.g. "128x0e+128x1o"; every multiplicity equal (C >= 1).
+ *   irreps_sh:   "1x0e+1x1o+...+1xLp", consecutive l from 0, parity (-1)^l.
+ *   irreps_out:  filter, e.g. "128x0e+128x1o+128x2e"; multiplicities = C;
+ *                no irrep twice.
+ *   avg_num_neighbors: N > 0 (finite).
+ *   normalization: E3CONV_NORM_SQRT_DIM_OUT or E3CONV_NORM_NONE.
+ * The input dtype starts as E3CONV_F32.  Degrees up to l = 6 are accepted.
+ * On success *plan owns its host tables, module and status word; release it
+ * with e3conv_destroy.  On failure *plan is set to NULL. */
+E3CONV_API int e3conv_create(e3conv_plan* plan, const char* irreps_node, const char* irreps_sh,
+                  const char* irreps_out, double avg_num_neighbors, int normalization);
+
+/* Frees everything the plan owns.  NULL is accepted.  The caller must make
+ * sure no forward launched with this plan is still running. */
+E3CONV_API void e3conv_destroy(e3conv_plan plan);
+
+/* Selects the element type of node_features, edge_sh and edge_scalars
+ * (E3CONV_F32 or E3CONV_F16; accumulation and output stay float32).
+ * Compiles and loads that kernel variant on first use (host-side, blocking). */
+E3CONV_API int e3conv_set_input_dtype(e3conv_plan plan, int dtype);
+
+/* Overrides the launch shape of the forward kernel: channels_per_lane in
+ * {0 (automatic), 1, 2, 4, 8} (must divide C and fit one 16-byte load) and
+ * block_threads in {0 (automatic), 32, 64, ..., 1024}.  Recompiles the
+ * current dtype's kernel (host-side, blocking). */
+E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane, int block_threads);
+
+/* Sizes: C channels, nx node components, ny edge components, nout output
+ * components, num_paths P.  Any pointer may be NULL. */
+E3CONV_API int e3conv_query(e3conv_plan plan, int* C, int* nx, int* ny, int* nout, int* num_paths);
+
+/* Path p (0 <= p < P): (l1, p1) x l2 -> (l3, p3), with x_off the first node
+ * component of the input irrep and out_off the first output component of
+ * the output irrep.  Parities are +1 (even) or -1 (odd).  NULL outputs are
+ * skipped. */
+E3CONV_API int e3conv_path(e3conv_plan plan, int p, int* l1, int* p1, int* l2, int* l3, int* p3,
+                int* x_off, int* out_off);
+
+/* Number of produced output irreps, and irrep k's (l, parity, offset). */
+E3CONV_API int e3conv_num_outputs(e3conv_plan plan, int* count);
+E3CONV_API int e3conv_output_irrep(e3conv_plan plan, int k, int* l, int* p, int* offset);
+
+/* Dense CG tensor of path p, including the normalisation factor, written to
+ * dense_out[(2l1+1)*(2l2+1)*(2l3+1)] in row-major (i, j, k) order (host). */
+E3CONV_API int e3conv_cg(e3conv_plan plan, int p, double* dense_out);
+
+/* Launch shape and resources of the forward kernel for `dtype`:
+ * channels per lane, lanes per receiver tile, block threads, registers per
+ * thread, local-memory (spill) bytes per thread.  Any pointer may be NULL.
+ * Returns E3CONV_ERR_NO_DEVICE for the resource fields' source if the plan
+ * has no module, after filling the shape fields. */
+E3CONV_API int e3conv_kernel_info(e3conv_plan plan, int dtype, int* channels_per_lane, int* lanes_per_tile,
+                       int* block_threads, int* registers, int* local_bytes);
+
+/* Copies the generated CUDA source for `dtype` (NUL-terminated) into buf if
+ * buf_len is large enough; *needed receives the required size in bytes. */
+E3CONV_API int e3conv_kernel_source(e3conv_plan plan, int dtype, char* buf, size_t buf_len, size_t* needed);
+
+/* ---------------------------------------------------------------------------
+ * Forward (the fused gather -> CG product -> scalar mix -> segmented sum ->
+ * 1/N scale -> store of e3j's four plain steps; one kernel launch)
+ *
+ * node_features: device, [num_nodes][nx][C] of the plan's dtype.
+ * edge_sh:       device, [num_edges][ny], receiver-sorted.
+ * edge_scalars:  device, [num_edges][P][C], receiver-sorted.
+ * senders:       device int32 [num_edges], receiver-sorted, in [0, num_nodes).
+ * receiver_row_ptr: device int32 [num_nodes+1], nondecreasing, row_ptr[0] = 0,
+ *                row_ptr[num_nodes] = num_edges (e3conv_build_csr makes it).
+ * out:           device float32 [num_nodes][nout][C]; fully overwritten
+ *                (rows of receivers without edges become 0).
+ * All buffers must be 16-byte aligned.  0 <= num_nodes, num_edges < 2^31.
+ * With num_nodes == 0 nothing is launched; with num_edges == 0 the edge
+ * pointers may be NULL.
+ * Out-of-range senders are skipped and row ranges outside [0, num_edges]
+ * are treated as empty; both set the plan's status word (e3conv_check).
+ * Launches exactly one kernel on `stream`; no host synchronisation, no
+ * allocation.  Concurrent forwards with one plan share its status word. */
+E3CONV_API int e3conv_forward(e3conv_plan plan, const void* node_features, const void* edge_sh,
+                   const void* edge_scalars, const int32_t* senders,
+                   const int32_t* receiver_row_ptr, int64_t num_nodes, int64_t num_edges,
+                   float* out, e3conv_stream stream);
+
+/* Synchronises `stream`, reads and clears the plan's status word.  Returns
+ * E3CONV_OK or E3CONV_ERR_BAD_INDEX if a forward since the last check met an
+ * out-of-range sender or row range. */
+E3CONV_API int e3conv_check(e3conv_plan plan, e3conv_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * Receiver-sorted CSR indexing (e3j "graph_ordering": RECEIVER, edges sorted
+ * by receiver so aggregation is a segmented reduction without atomics).
+ */
+
+/* Workspace bytes e3conv_build_csr needs for these sizes. */
+E3CONV_API int e3conv_csr_workspace_size(int64_t num_edges, int64_t num_nodes, size_t* bytes);
+
+/* From receivers[e] (device int32, any order) computes, on the device:
+ *   row_ptr[b] = #{e : receivers[e] < b}, b = 0..num_nodes  (int32 [num_nodes+1])
+ *   perm[t]    = the t-th edge in (receiver, original index) order, i.e. a
+ *                stable counting sort of the edges by receiver (int32 [num_edges]).
+ * Bit-exact and deterministic.  Receivers outside [0, num_nodes) are placed
+ * after all valid edges in perm, are not counted in row_ptr, and set the
+ * workspace status word (e3conv_csr_check).  `workspace` is device memory
+ * of at least e3conv_csr_workspace_size bytes, 256-byte aligned; its
+ * contents need not be initialised and it must not be used by another call
+ * until this one has finished on `stream`.  No host synchronisation. */
+E3CONV_API int e3conv_build_csr(const int32_t* receivers, int64_t num_edges, int64_t num_nodes,
+                     int32_t* row_ptr, int32_t* perm, void* workspace, size_t workspace_bytes,
+                     e3conv_stream stream);
+
+/* Number of kernels one e3conv_build_csr call with these sizes launches
+ * (it also issues two cudaMemsetAsync calls).  Host only. */
+E3CONV_API int e3conv_csr_kernel_count(int64_t num_edges, int64_t num_nodes, int* count);
+
+/* Synchronises `stream` and reports the status word of the last
+ * e3conv_build_csr that used `workspace`: E3CONV_OK or E3CONV_ERR_BAD_INDEX. */
+E3CONV_API int e3conv_csr_check(const void* workspace, e3conv_stream stream);
+
+/* dst[t] = src[perm[t]] for rows of row_bytes bytes, t < num_rows (device).
+ * Puts edge features / scalars into CSR order.  Rows whose perm entry is
+ * outside [0, num_src_rows) are zero-filled and set *status (device int32,
+ * may be NULL) to a nonzero value.  row_bytes must be a multiple of 4 and
+ * src / dst 16-byte aligned. */
+E3CONV_API int e3conv_permute_rows(const void* src, int64_t num_src_rows, const int32_t* perm,
+                        int64_t num_rows, int64_t row_bytes, void* dst, int32_t* status,
+                        e3conv_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * Errors and version
+ */
+E3CONV_API const char* e3conv_strerror(int code);
+E3CONV_API const char* e3conv_last_error(void);
+E3CONV_API int e3conv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* E3CONV_H */

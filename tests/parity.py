@@ -1,0 +1,101 @@
+"""Shared helpers of the GPU parity tests: input generation, oracle calls and
+the error metric.
+
+Error metric: for every flattened output column c = (component, channel),
+scale_c = max_b |ref[b, c]| (1 if the column is all zero), and
+err = max_{b,c} |gpu - ref| / scale_c.  The bars are 1e-5 for float32 inputs
+and 5e-3 for float16 inputs (both accumulate in float32; the oracle consumes
+the same rounded inputs upcast exactly to float64)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import equivariant_graph_message_b200 as e3
+import oracle
+from workloads import SPECS, edge_sh, make_graph, node_features_np, node_features_torch, \
+    scalars_np, scalars_torch
+
+TOL = {"f32": 1e-5, "f16": 5e-3}
+
+
+def column_scaled_error(gpu: np.ndarray, ref: np.ndarray) -> float:
+    g = gpu.reshape(gpu.shape[0], -1).astype(np.float64)
+    r = ref.reshape(ref.shape[0], -1)
+    scale = np.abs(r).max(axis=0) if len(r) else np.ones(r.shape[1])
+    scale = np.where(scale == 0, 1.0, scale)
+    return float((np.abs(g - r) / scale).max()) if g.size else 0.0
+
+
+def row_ptr_of(receivers: np.ndarray, num_nodes: int) -> np.ndarray:
+    counts = np.bincount(receivers, minlength=num_nodes) if len(receivers) else \
+        np.zeros(num_nodes, np.int64)
+    rp = np.zeros(num_nodes + 1, np.int64)
+    np.cumsum(counts, out=rp[1:])
+    return rp
+
+
+def to_dev(a, dtype=None, device="cuda"):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.to(device)
+
+
+def run_gpu(conv: e3.Conv, x, Y, s, senders, receivers, num_nodes, prefill=float("nan")):
+    """Receiver-sorted host arrays -> GPU output (host, float32)."""
+    tdt = torch.float16 if conv.dtype == "f16" else torch.float32
+    rp = row_ptr_of(np.asarray(receivers), num_nodes)
+    out = torch.full((num_nodes, conv.nout, conv.C), prefill, dtype=torch.float32, device="cuda")
+    conv.forward(to_dev(x, tdt), to_dev(Y, tdt), to_dev(s, tdt),
+                 to_dev(np.asarray(senders, np.int32)), to_dev(rp.astype(np.int32)), out=out)
+    torch.cuda.synchronize()
+    assert conv.check()
+    return out.cpu().numpy()
+
+
+def oracle_out(irreps, x, Y, s, senders, receivers, num_nodes, avg, norm="SQRT_DIM_OUT"):
+    return oracle.forward(*irreps, np.asarray(x, np.float64), np.asarray(Y, np.float64),
+                          np.asarray(s, np.float64), senders, receivers, num_nodes, avg, norm)
+
+
+class DeviceWorkload:
+    """A full-size workload generated on the device, as the benchmark times it."""
+
+    def __init__(self, name: str, device="cuda", nodes: int | None = None):
+        self.spec = spec = SPECS[name]
+        self.graph = g = make_graph(spec, nodes)
+        self.N, self.E = g.num_nodes, g.num_edges
+        tdt = torch.float16 if spec.dtype == "f16" else torch.float32
+        self.x = node_features_torch(spec, g.num_nodes, device)
+        self.Y = torch.from_numpy(edge_sh(spec, g)).to(device)
+        self.s = scalars_torch(spec, g, device)
+        self.senders = torch.from_numpy(g.senders.astype(np.int32)).to(device)
+        self.receivers = torch.from_numpy(g.receivers.astype(np.int32)).to(device)
+        self.row_ptr = torch.from_numpy(row_ptr_of(g.receivers, g.num_nodes).astype(np.int32)).to(device)
+        assert self.x.dtype == tdt and self.Y.dtype == tdt and self.s.dtype == tdt
+        self.conv = e3.Conv(spec.irreps_node, spec.irreps_sh, spec.irreps_out,
+                            g.avg_num_neighbors, dtype=spec.dtype)
+
+    @property
+    def irreps(self):
+        return (self.spec.irreps_node, self.spec.irreps_sh, self.spec.irreps_out)
+
+    def sample_reference(self, receivers: np.ndarray) -> np.ndarray:
+        """Oracle output rows for the given receivers, from the device inputs."""
+        g = self.graph
+        rp = row_ptr_of(g.receivers, g.num_nodes)
+        edges = np.concatenate([np.arange(rp[b], rp[b + 1]) for b in receivers]) \
+            if len(receivers) else np.zeros(0, np.int64)
+        senders = g.senders[edges]
+        uniq, inv = np.unique(senders, return_inverse=True)
+        x = self.x[torch.from_numpy(uniq).to(self.x.device)].cpu().numpy()
+        eidx = torch.from_numpy(edges).to(self.s.device)
+        Y = self.Y[eidx].cpu().numpy()
+        s = self.s[eidx].cpu().numpy()
+        local_recv = np.repeat(np.arange(len(receivers)), np.diff(rp)[receivers])
+        # sample rows: receivers 0..len-1; senders remapped into the gathered x rows
+        xr = np.zeros((max(len(receivers), len(uniq)),) + x.shape[1:], x.dtype)
+        xr[:len(uniq)] = x
+        out = oracle_out(self.irreps, xr, Y, s, inv, local_recv, len(xr), g.avg_num_neighbors)
+        return out[:len(receivers)]

@@ -1,0 +1,147 @@
+"""Host-side checks of libe3conv.so (no GPU needed): exports, plans, CG tables,
+path enumeration, code generation, error codes."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import equivariant_graph_message_b200 as e3
+import oracle
+from workloads import ORDER, SPECS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "e3conv.h")).read()
+    return sorted(set(re.findall(r"^E3CONV_API\s+[\w\s\*]*?\b(e3conv_\w+)\s*\(", text, re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared_symbols()
+    assert len(declared) >= 20
+    lib = ctypes.CDLL(e3.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(e3.EXPORTED) == declared
+    assert e3.version() == 1
+
+
+def test_strerror_covers_codes():
+    for code in range(10):
+        assert e3._strerror(code).decode() not in ("", "unknown error code")
+    assert e3._strerror(99).decode() == "unknown error code"
+
+
+@pytest.mark.parametrize("name", ORDER)
+def test_paths_match_oracle(name):
+    s = SPECS[name]
+    c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 3.0)
+    pl = oracle.plan(s.irreps_node, s.irreps_sh, s.irreps_out)
+    assert (c.C, c.nx, c.ny, c.nout, c.num_paths) == (pl.C, pl.nx, pl.ny, pl.nout, len(pl.paths))
+    assert c.num_paths == s.num_paths and c.nx == s.nx
+    for q, r in zip(c.paths, pl.paths):
+        assert (q.l1, q.p1, q.l2, q.l3, q.p3, q.x_off, q.out_off) == \
+               (r.l1, r.p1, r.l2, r.l3, r.p3, r.x_off, r.out_off)
+    assert c.outputs == [tuple(o) for o in pl.outputs]
+
+
+@pytest.mark.parametrize("norm", ["SQRT_DIM_OUT", "NONE"])
+def test_cg_tables_match_oracle_to_1e13(norm):
+    # Racah closed form + real-basis map (library) vs intertwiner null space (oracle)
+    irreps = ("1x0e+1x1o+1x2e+1x3o+1x4e+1x1e+1x2o", "1x0e+1x1o+1x2e+1x3o+1x4e",
+              "+".join(f"1x{l}{p}" for l in range(7) for p in "eo"))
+    c = e3.Conv(*irreps, 1.0, normalization=norm)
+    assert c.num_paths > 60
+    for p, q in enumerate(c.paths):
+        np.testing.assert_allclose(c.cg(p), oracle.cg(q.l1, q.l2, q.l3, norm), atol=1e-13,
+                                   err_msg=str(q))
+
+
+def test_output_filter_drops_unreachable_irreps():
+    c = e3.Conv("2x0e+2x1o+2x2e", "1x0e+1x1o+1x2e+1x3o", "2x0e+2x0o+2x1e+2x1o+2x2e+2x2o", 1.0)
+    assert (0, -1) not in [(l, p) for l, p, _ in c.outputs]
+    assert c.nout == 17
+
+
+@pytest.mark.parametrize("args,code", [
+    (("4x0e+5x1o", "1x0e", "4x0e"), 2),            # unequal multiplicities
+    (("4x0e", "1x0e+1x2e", "4x0e"), 2),            # edge degrees not consecutive
+    (("4x0e", "1x0e+1x1e", "4x0e"), 2),            # wrong edge parity
+    (("4x0e", "2x0e", "4x0e"), 2),                 # edge multiplicity != 1
+    (("4x0e", "1x0e", "4x0o"), 2),                 # no path reaches the filter
+    (("4x0e", "1x0e", "4x0e+4x0e"), 2),            # duplicate output irrep
+    (("4x0q", "1x0e", "4x0e"), 2),                 # malformed
+    (("4x0e", "1x0e", "3x0e"), 2),                 # output multiplicity != C
+    (("", "1x0e", "4x0e"), 2),
+    (("1x7e", "1x0e", "1x7e"), 3),                 # degree above 6
+])
+def test_create_errors(args, code):
+    with pytest.raises(e3.E3ConvError) as ei:
+        e3.Conv(*args, 1.0)
+    assert ei.value.code == code
+
+
+def test_create_rejects_bad_scalars():
+    for avg in (0.0, -1.0, float("nan"), float("inf")):
+        with pytest.raises(e3.E3ConvError) as ei:
+            e3.Conv("1x0e", "1x0e", "1x0e", avg)
+        assert ei.value.code == 1
+    with pytest.raises(KeyError):
+        e3.Conv("1x0e", "1x0e", "1x0e", 1.0, normalization="COMPONENT")
+    h = ctypes.c_void_p()
+    assert e3._create(ctypes.byref(h), b"1x0e", b"1x0e", b"1x0e", 1.0, 7) == 3
+    assert not h.value
+
+
+def test_generated_kernel_unrolls_every_coefficient():
+    s = SPECS["large_f16"]
+    c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 40.0, dtype="f16")
+    src = c.kernel_source()
+    info = c.kernel_info()
+    V = info["channels_per_lane"]
+    nnz = sum(int((np.abs(c.cg(p)) > 1e-12).sum()) for p in range(c.num_paths))
+    assert nnz == 611
+    n_fma = src.count("fmaf(")
+    n_mul = len(re.findall(r"= c\d+ \* x", src)) + len(re.findall(r"= s_\d \* x", src))
+    assert n_fma + n_mul >= nnz * V
+    assert "e3conv_fwd" in src and "row_ptr" in src and "atomicAdd" not in src
+    assert info["local_bytes"] == 0
+
+
+@pytest.mark.parametrize("V,block", [(1, 64), (2, 256), (4, 128)])
+def test_launch_config_recompiles(V, block):
+    s = SPECS["mace"]
+    c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 30.0)
+    c.set_launch_config(V, block)
+    info = c.kernel_info()
+    assert info["channels_per_lane"] == V and info["block_threads"] == block
+    with pytest.raises(e3.E3ConvError):
+        c.set_launch_config(3, 0)
+    with pytest.raises(e3.E3ConvError):
+        c.set_launch_config(0, 100)
+
+
+def test_host_only_plan_forward_reports_no_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present; covered by the GPU tests")
+    c = e3.Conv("1x0e", "1x0e", "1x0e", 1.0)
+    rc = e3._forward(c._h, ctypes.c_void_p(16), None, None, None, ctypes.c_void_p(16), 1, 0,
+                     ctypes.c_void_p(16), None)
+    assert rc == 7
+    ws = ctypes.c_size_t()
+    assert e3._csr_ws(10, 5, ctypes.byref(ws)) == 0 and ws.value > 0
+
+
+def test_forward_argument_validation_precedes_device():
+    c = e3.Conv("1x0e", "1x0e", "1x0e", 1.0)
+    assert e3._forward(c._h, None, None, None, None, None, -1, 0, None, None) == 1
+    assert e3._forward(c._h, None, None, None, None, None, 0, 0, None, None) == 0   # nothing to do
+    assert e3._forward(c._h, None, None, None, None, None, 3, 0, None, None) == 1
+    # misaligned feature buffer
+    assert e3._forward(c._h, ctypes.c_void_p(18), None, None, None, ctypes.c_void_p(16), 3, 0,
+                       ctypes.c_void_p(16), None) == 1
+    assert e3._build_csr(None, -1, 3, None, None, None, 0, None) == 1
