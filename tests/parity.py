@@ -27,6 +27,33 @@ def column_scaled_error(gpu: np.ndarray, ref: np.ndarray) -> float:
     return float((np.abs(g - r) / scale).max()) if g.size else 0.0
 
 
+def abs_bound(irreps, x, Y, s, senders, receivers, num_nodes, avg, norm="SQRT_DIM_OUT"):
+    """Elementwise float32 error bound of the kernel's arithmetic.
+
+    The kernel sums, for each output element, every product s*c*x*Y of every
+    edge of its row in one float32 chain of length L (recursive summation,
+    Higham's bound gamma_L = L u / (1 - L u), u = 2^-24), after rounding the
+    CG constant, c*Y and s*x (or c*Y*x) once each (3u).  With
+    A = (1/N) sum |s| |c| |x| |Y| (the same sum over absolute values):
+        |gpu - exact| <= (gamma_L + 3u) A  (+ the float64 oracle's own error).
+    L is bounded by (max row degree) x (max terms per edge of one element)."""
+    pl = oracle.plan(*irreps)
+    u = 2.0 ** -24
+    A = np.zeros((num_nodes, pl.nout, pl.C))
+    terms = np.zeros(pl.nout)
+    for p, path in enumerate(pl.paths):
+        W = np.abs(oracle.cg(path.l1, path.l2, path.l3, norm))
+        terms[path.out_off:path.out_off + 2 * path.l3 + 1] += (W > 1e-12).sum(axis=(0, 1))
+        xa = np.abs(np.asarray(x, np.float64)[senders][:, path.x_off:path.x_off + 2 * path.l1 + 1])
+        ye = np.abs(np.asarray(Y, np.float64)[:, path.y_off:path.y_off + 2 * path.l2 + 1])
+        msg = np.einsum("ijk,eiu,ej,eu->eku", W, xa, ye, np.abs(np.asarray(s, np.float64)[:, p]))
+        np.add.at(A[:, path.out_off:path.out_off + 2 * path.l3 + 1, :], receivers, msg)
+    deg = np.bincount(receivers, minlength=num_nodes).max() if len(receivers) else 0
+    L = deg * terms.max() + 2
+    gamma = L * u / (1 - L * u)
+    return (gamma + 3 * u) * A / avg
+
+
 def row_ptr_of(receivers: np.ndarray, num_nodes: int) -> np.ndarray:
     counts = np.bincount(receivers, minlength=num_nodes) if len(receivers) else \
         np.zeros(num_nodes, np.int64)

