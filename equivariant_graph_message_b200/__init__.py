@@ -44,13 +44,14 @@ _create = _sig("e3conv_create", ctypes.c_int, ctypes.POINTER(_vp), ctypes.c_char
                ctypes.c_char_p, ctypes.c_char_p, ctypes.c_double, ctypes.c_int)
 _destroy = _sig("e3conv_destroy", None, _vp)
 _set_dtype = _sig("e3conv_set_input_dtype", ctypes.c_int, _vp, ctypes.c_int)
-_set_launch = _sig("e3conv_set_launch_config", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_int)
+_set_launch = _sig("e3conv_set_launch_config", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_int,
+                   ctypes.c_int)
 _query = _sig("e3conv_query", ctypes.c_int, _vp, *([_c_int_p] * 5))
 _path = _sig("e3conv_path", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 7))
 _num_outputs = _sig("e3conv_num_outputs", ctypes.c_int, _vp, _c_int_p)
 _output_irrep = _sig("e3conv_output_irrep", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 3))
 _cg = _sig("e3conv_cg", ctypes.c_int, _vp, ctypes.c_int, ctypes.POINTER(ctypes.c_double))
-_kernel_info = _sig("e3conv_kernel_info", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 5))
+_kernel_info = _sig("e3conv_kernel_info", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 6))
 _kernel_source = _sig("e3conv_kernel_source", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_char_p,
                       ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t))
 _forward = _sig("e3conv_forward", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp,
@@ -172,14 +173,17 @@ class Conv:
         _ok(_set_dtype(self._h, {"f32": F32, "f16": F16}[dtype]), "e3conv_set_input_dtype")
         self.dtype = dtype
 
-    def set_launch_config(self, channels_per_lane: int = 0, block_threads: int = 0):
-        _ok(_set_launch(self._h, channels_per_lane, block_threads), "e3conv_set_launch_config")
+    def set_launch_config(self, channels_per_lane: int = 0, block_threads: int = 0,
+                          stages: int = -1):
+        _ok(_set_launch(self._h, channels_per_lane, block_threads, stages),
+            "e3conv_set_launch_config")
 
     def kernel_info(self, dtype: str | None = None) -> dict:
-        v = [ctypes.c_int() for _ in range(5)]
+        v = [ctypes.c_int() for _ in range(6)]
         _ok(_kernel_info(self._h, {"f32": F32, "f16": F16}[dtype or self.dtype],
                          *[ctypes.byref(x) for x in v]), "e3conv_kernel_info")
-        keys = ["channels_per_lane", "lanes_per_tile", "block_threads", "registers", "local_bytes"]
+        keys = ["channels_per_lane", "lanes_per_tile", "block_threads", "stages", "registers",
+                "local_bytes"]
         return dict(zip(keys, (x.value for x in v)))
 
     def kernel_source(self, dtype: str | None = None) -> str:

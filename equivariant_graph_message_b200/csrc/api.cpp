@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <nvrtc.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -43,6 +44,8 @@ struct Driver {
                            unsigned, CUstream, void**, void**) = nullptr;
   CUresult (*FuncGetAttribute)(int*, CUfunction_attribute, CUfunction) = nullptr;
   CUresult (*CtxGetCurrent)(CUcontext*) = nullptr;
+  CUresult (*FuncSetAttribute)(CUfunction, CUfunction_attribute, int) = nullptr;
+  CUresult (*OccupancyMaxActiveBlocksPerMultiprocessor)(int*, CUfunction, int, size_t) = nullptr;
   bool ok = false;
 };
 
@@ -60,7 +63,10 @@ Driver& driver() {
            get("cuModuleGetFunction", reinterpret_cast<void**>(&d.ModuleGetFunction)) &&
            get("cuLaunchKernel", reinterpret_cast<void**>(&d.LaunchKernel)) &&
            get("cuFuncGetAttribute", reinterpret_cast<void**>(&d.FuncGetAttribute)) &&
-           get("cuCtxGetCurrent", reinterpret_cast<void**>(&d.CtxGetCurrent));
+           get("cuCtxGetCurrent", reinterpret_cast<void**>(&d.CtxGetCurrent)) &&
+           get("cuFuncSetAttribute", reinterpret_cast<void**>(&d.FuncSetAttribute)) &&
+           get("cuOccupancyMaxActiveBlocksPerMultiprocessor",
+               reinterpret_cast<void**>(&d.OccupancyMaxActiveBlocksPerMultiprocessor));
     cudaGetLastError();
   });
   return d;
@@ -117,6 +123,20 @@ int compile_variant(Plan& pl, int dtype) {
     d.FuncGetAttribute(&local, CU_FUNC_ATTRIBUTE_LOCAL_SIZE_BYTES, v.fn);
     v.regs = regs;
     v.local_bytes = local;
+    if (v.shape.stages > 0) {
+      const int smem = v.shape.warp_smem * (v.shape.block / 32);
+      if (d.FuncSetAttribute(v.fn, CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES, smem) !=
+          CUDA_SUCCESS)
+        return fail(E3CONV_ERR_CUDA, "cannot reserve the shared-memory ring");
+      int per_sm = 0, sms = 0;
+      if (d.OccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, v.shape.block, smem) !=
+              CUDA_SUCCESS ||
+          per_sm < 1)
+        return fail(E3CONV_ERR_CUDA, "staged kernel does not fit on an SM");
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, pl.device) != cudaSuccess)
+        return fail(E3CONV_ERR_CUDA, "cannot query the SM count");
+      v.grid_blocks = per_sm * sms;
+    }
   }
   return E3CONV_OK;
 }
@@ -276,7 +296,8 @@ int e3conv_set_input_dtype(e3conv_plan h, int dtype) {
   return E3CONV_OK;
 }
 
-int e3conv_set_launch_config(e3conv_plan h, int channels_per_lane, int block_threads) {
+int e3conv_set_launch_config(e3conv_plan h, int channels_per_lane, int block_threads,
+                             int stages) {
   if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
   Plan& pl = h->p;
   const int V = channels_per_lane;
@@ -288,8 +309,11 @@ int e3conv_set_launch_config(e3conv_plan h, int channels_per_lane, int block_thr
     return fail(E3CONV_ERR_INVALID_ARG, "channels_per_lane exceeds one 16-byte load");
   if (block_threads != 0 && (block_threads < 32 || block_threads > 1024 || block_threads % 32))
     return fail(E3CONV_ERR_INVALID_ARG, "block_threads must be 0 or a multiple of 32 in [32, 1024]");
+  if (stages < -1 || stages == 1 || stages > 8)
+    return fail(E3CONV_ERR_INVALID_ARG, "stages must be -1 (automatic), 0 (direct) or 2..8");
   pl.req_V = V;
   pl.req_block = block_threads;
+  pl.req_stages = stages;
   DeviceGuard g(pl.device);
   const int other = pl.dtype == E3CONV_F32 ? E3CONV_F16 : E3CONV_F32;
   release_variant(pl.var[other]);
@@ -351,8 +375,8 @@ int e3conv_cg(e3conv_plan h, int p, double* dense_out) {
   return E3CONV_OK;
 }
 
-int e3conv_kernel_info(e3conv_plan h, int dtype, int* V, int* TL, int* block, int* regs,
-                       int* local_bytes) {
+int e3conv_kernel_info(e3conv_plan h, int dtype, int* V, int* TL, int* block, int* stages,
+                       int* regs, int* local_bytes) {
   if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
   if (dtype != E3CONV_F32 && dtype != E3CONV_F16)
     return fail(E3CONV_ERR_UNSUPPORTED, "unknown dtype");
@@ -361,6 +385,7 @@ int e3conv_kernel_info(e3conv_plan h, int dtype, int* V, int* TL, int* block, in
   if (V) *V = v.shape.V;
   if (TL) *TL = v.shape.TL;
   if (block) *block = v.shape.block;
+  if (stages) *stages = v.shape.stages;
   if (regs) *regs = v.regs;
   if (local_bytes) *local_bytes = v.local_bytes;
   return E3CONV_OK;
@@ -397,9 +422,17 @@ int e3conv_forward(e3conv_plan h, const void* x, const void* Y, const void* s,
   if (cudaGetDevice(&cur) != cudaSuccess || cur != pl.device)
     return fail(E3CONV_ERR_INVALID_ARG, "current device differs from the plan's device");
   const Shape& sh = v.shape;
-  const long long items = num_nodes * sh.tiles;
-  const long long warps = (items + sh.ipw - 1) / sh.ipw;
-  const long long blocks = (warps * 32 + sh.block - 1) / sh.block;
+  long long blocks;
+  unsigned smem = 0;
+  if (sh.stages > 0) {
+    const long long wpb = sh.block / 32;
+    blocks = std::min<long long>(v.grid_blocks, (num_nodes + wpb - 1) / wpb);
+    smem = static_cast<unsigned>(sh.warp_smem * wpb);
+  } else {
+    const long long items = num_nodes * sh.tiles;
+    const long long warps = (items + sh.ipw - 1) / sh.ipw;
+    blocks = (warps * 32 + sh.block - 1) / sh.block;
+  }
   if (blocks >= (1ll << 31)) return fail(E3CONV_ERR_UNSUPPORTED, "grid too large");
   int n32 = static_cast<int>(num_nodes), e32 = static_cast<int>(num_edges);
   float inv_avg = static_cast<float>(1.0 / pl.avg);
@@ -407,7 +440,7 @@ int e3conv_forward(e3conv_plan h, const void* x, const void* Y, const void* s,
                   const_cast<int32_t**>(&senders), const_cast<int32_t**>(&row_ptr),
                   &n32, &e32, &out, &inv_avg, &pl.status};
   CUresult r = driver().LaunchKernel(v.fn, static_cast<unsigned>(blocks), 1, 1,
-                                     static_cast<unsigned>(sh.block), 1, 1, 0,
+                                     static_cast<unsigned>(sh.block), 1, 1, smem,
                                      reinterpret_cast<CUstream>(stream), args, nullptr);
   if (r != CUDA_SUCCESS) return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed");
   return E3CONV_OK;
@@ -425,6 +458,7 @@ int e3conv_check(e3conv_plan h, e3conv_stream stream) {
   if (st) {
     cudaMemsetAsync(pl.status, 0, sizeof st, s);
     cudaStreamSynchronize(s);
+    if (st & 4u) return fail(E3CONV_ERR_CUDA, "a forward's shared-memory pipeline wait timed out");
     return fail(E3CONV_ERR_BAD_INDEX, std::string("forward met ") +
                                           ((st & 1u) ? "an invalid receiver_row_ptr range " : "") +
                                           ((st & 2u) ? "an out-of-range sender" : ""));

@@ -3,17 +3,25 @@
 // The kernel evaluates, for receiver b and channel u,
 //   out[b, o+k, u] = inv_avg * sum_{e in row b} sum_{p -> o}
 //                    s[e,p,u] * sum_{(i,j,k,c) in nnz(p)} c * Y[e, y_p + j] * x[a_e, x_p + i, u]
-// with every path's nonzero CG coefficients unrolled as float32 immediates.
+// with every path's nonzero CG coefficients unrolled as float32 immediates
+// (the per-edge gather, tensor product, scalar mix, segmented sum over the
+// receiver's CSR row and 1/N scale of e3j.core.Convolution, fused).
 //
-// Work decomposition: an "item" is (receiver b, channel tile t).  A team of
-// TL lanes handles one item, each lane V consecutive channels, so a warp
-// holds ipw = 32 / TL items (small C) or one 32*V-channel tile of one
-// receiver (large C).  Each lane walks the receiver's CSR row sequentially
-// and keeps its nout*V partial sums in registers: the segmented reduction
-// needs no atomics and no cross-lane traffic.  Per edge it loads the sender
-// row slice x[a, :, u0:u0+V) and the scalar slice s[e, :, u0:u0+V) with
-// vector loads (16 bytes at most), and the edge's Y row (the same address
-// for all lanes of the team).
+// Lane mapping: each lane owns V consecutive channels u0..u0+V-1 and keeps
+// its nout*V partial sums in registers while it walks the receiver's row
+// sequentially, so the segmented reduction needs no atomics and no
+// cross-lane traffic.  Channels are independent in the channelwise product.
+//
+// Two variants:
+//  * direct:  an "item" (receiver, channel tile) per team of TL lanes; each
+//             lane loads its x / s slices with vector loads (<= 16 bytes).
+//  * staged:  persistent warps, one 32*V-channel receiver row per warp at a
+//             time (receivers w, w+W, w+2W, ...).  Lane 0 copies the next
+//             edges' s row, sender x row and Y row into a per-warp ring of
+//             shared-memory stages with 1-D bulk async copies (no multicast)
+//             completed on mbarriers; the warp computes the current edge from
+//             shared memory.  Waits are bounded: on timeout the kernel sets
+//             bit 4 of the status word, drains its copies (bounded) and exits.
 //
 // Per path the cheaper of two equivalent evaluation orders is emitted:
 //   scale-input  (2l1+1 <= 2l3+1): z_i = s_p x_i, then acc_k += (c Y_j) z_i
@@ -30,6 +38,12 @@
 
 namespace e3c {
 
+namespace {
+
+int align_up(int v, int a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
 Shape choose_shape(const Plan& pl, int dtype) {
   Shape s;
   const int elem = dtype == E3CONV_F16 ? 2 : 4;
@@ -44,6 +58,9 @@ Shape choose_shape(const Plan& pl, int dtype) {
         break;
       }
     }
+    // the staged variant wants one warp to cover a receiver's channels
+    if (pl.req_stages != 0 && pl.C % 32 == 0 && pl.C / 32 <= vmax && pl.nout * (pl.C / 32) <= 128)
+      V = pl.C / 32;
   }
   s.V = V;
   const int lanes = pl.C / V;
@@ -57,6 +74,28 @@ Shape choose_shape(const Plan& pl, int dtype) {
     s.ipw = 32 / lanes;
   }
   s.block = pl.req_block > 0 ? pl.req_block : 128;
+
+  // staged variant: one warp covers all C channels; all rows 16-byte multiples
+  s.s_bytes = static_cast<int>(pl.paths.size()) * pl.C * elem;
+  s.x_bytes = pl.nx * pl.C * elem;
+  s.y_bytes = pl.ny * elem;
+  const bool shape_ok = s.TL == 32 && s.tiles == 1 && 32 * V == pl.C;
+  const bool bytes_ok = s.s_bytes % 16 == 0 && s.x_bytes % 16 == 0 && s.y_bytes % 16 == 0;
+  if (shape_ok && bytes_ok && pl.req_stages != 0) {
+    s.s_off = 0;
+    s.x_off = align_up(s.s_bytes, 128);
+    s.y_off = s.x_off + align_up(s.x_bytes, 128);
+    s.stage_bytes = s.y_off + align_up(s.y_bytes, 128);
+    int S = pl.req_stages > 0 ? pl.req_stages : (s.stage_bytes > 10240 ? 2 : 3);
+    const int warps = s.block / 32;
+    // keep one block within 227 KB of shared memory
+    while (S > 2 && warps * (S * s.stage_bytes + 256) > 227 * 1024) --S;
+    s.stages = S;
+    s.bar_off = S * s.stage_bytes;
+    s.hdr_off = s.bar_off + 8 * S;
+    s.warp_smem = align_up(s.hdr_off + 16 * S, 128);
+    if (warps * s.warp_smem > 227 * 1024) s.stages = 0;
+  }
   return s;
 }
 
@@ -77,134 +116,99 @@ struct Emitter {
   }
 };
 
-// Emits loads of V consecutive elements at `ptr` into float variables name_0 .. name_{V-1}.
-void emit_vec_load(Emitter& em, int dtype, int V, const std::string& ptr, const std::string& name) {
+std::string S(long long v) { return std::to_string(v); }
+
+// Loads V consecutive elements at `ptr` into float variables name_0 .. name_{V-1};
+// `pre` is "ldg" (read-only global) or "lds" (shared).
+void emit_vec_load(Emitter& em, int dtype, int V, const std::string& pre, const std::string& ptr,
+                   const std::string& name) {
   if (dtype == E3CONV_F32) {
     if (V == 4) {
-      em.line("{ const float4 t_ = ldg_f4(" + ptr + "); " + name + "_0 = t_.x; " + name +
+      em.line("{ const float4 t_ = " + pre + "_f4(" + ptr + "); " + name + "_0 = t_.x; " + name +
               "_1 = t_.y; " + name + "_2 = t_.z; " + name + "_3 = t_.w; }");
     } else if (V == 2) {
-      em.line("{ const float2 t_ = ldg_f2(" + ptr + "); " + name + "_0 = t_.x; " + name +
+      em.line("{ const float2 t_ = " + pre + "_f2(" + ptr + "); " + name + "_0 = t_.x; " + name +
               "_1 = t_.y; }");
     } else {
-      em.line(name + "_0 = ldg_f1(" + ptr + ");");
+      em.line(name + "_0 = " + pre + "_f1(" + ptr + ");");
     }
   } else {
     if (V == 8) {
-      em.line("{ const uint4 t_ = ldg_u4(" + ptr + ");");
+      em.line("{ const uint4 t_ = " + pre + "_u4(" + ptr + ");");
       const char* w[4] = {"t_.x", "t_.y", "t_.z", "t_.w"};
       for (int q = 0; q < 4; ++q)
-        em.line("  " + name + "_" + std::to_string(2 * q) + " = lo_h2f(" + w[q] + "); " + name +
-                "_" + std::to_string(2 * q + 1) + " = hi_h2f(" + w[q] + ");");
+        em.line("  " + name + "_" + S(2 * q) + " = lo_h2f(" + w[q] + "); " + name + "_" +
+                S(2 * q + 1) + " = hi_h2f(" + w[q] + ");");
       em.line("}");
     } else if (V == 4) {
-      em.line("{ const uint2 t_ = ldg_u2(" + ptr + "); " + name + "_0 = lo_h2f(t_.x); " + name +
-              "_1 = hi_h2f(t_.x); " + name + "_2 = lo_h2f(t_.y); " + name + "_3 = hi_h2f(t_.y); }");
+      em.line("{ const uint2 t_ = " + pre + "_u2(" + ptr + "); " + name + "_0 = lo_h2f(t_.x); " +
+              name + "_1 = hi_h2f(t_.x); " + name + "_2 = lo_h2f(t_.y); " + name +
+              "_3 = hi_h2f(t_.y); }");
     } else if (V == 2) {
-      em.line("{ const unsigned int t_ = ldg_u1(" + ptr + "); " + name + "_0 = lo_h2f(t_); " +
-              name + "_1 = hi_h2f(t_); }");
+      em.line("{ const unsigned int t_ = " + pre + "_u1(" + ptr + "); " + name +
+              "_0 = lo_h2f(t_); " + name + "_1 = hi_h2f(t_); }");
     } else {
-      em.line(name + "_0 = ldg_h1(" + ptr + ");");
+      em.line(name + "_0 = " + pre + "_h1(" + ptr + ");");
     }
   }
 }
 
-}  // namespace
-
-std::string generate_forward_source(const Plan& pl, int dtype, const Shape& sh) {
-  Emitter em;
-  const int V = sh.V;
-  const bool f16 = dtype == E3CONV_F16;
-  const std::string T = f16 ? "unsigned short" : "float";
-  em.line("// generated by libe3conv: fused equivariant convolution forward");
-  em.line("// irreps C=" + std::to_string(pl.C) + " nx=" + std::to_string(pl.nx) +
-          " ny=" + std::to_string(pl.ny) + " nout=" + std::to_string(pl.nout) +
-          " paths=" + std::to_string(pl.paths.size()) + " dtype=" + (f16 ? "f16" : "f32") +
-          " V=" + std::to_string(V) + " TL=" + std::to_string(sh.TL) +
-          " tiles=" + std::to_string(sh.tiles) + " ipw=" + std::to_string(sh.ipw));
-  // helpers (read-only global loads; half -> float via cvt)
-  em.line("__device__ __forceinline__ float ldg_f1(const float* p) { return __ldg(p); }");
-  em.line("__device__ __forceinline__ float2 ldg_f2(const float* p) { return __ldg(reinterpret_cast<const float2*>(p)); }");
-  em.line("__device__ __forceinline__ float4 ldg_f4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }");
-  em.line("__device__ __forceinline__ unsigned int ldg_u1(const unsigned short* p) { return __ldg(reinterpret_cast<const unsigned int*>(p)); }");
-  em.line("__device__ __forceinline__ uint2 ldg_u2(const unsigned short* p) { return __ldg(reinterpret_cast<const uint2*>(p)); }");
-  em.line("__device__ __forceinline__ uint4 ldg_u4(const unsigned short* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }");
+void emit_prelude(Emitter& em) {
   em.line("__device__ __forceinline__ float h2f(unsigned short h) { float f; asm(\"cvt.f32.f16 %0, %1;\" : \"=f\"(f) : \"h\"(h)); return f; }");
-  em.line("__device__ __forceinline__ float ldg_h1(const unsigned short* p) { return h2f(__ldg(p)); }");
   em.line("__device__ __forceinline__ float lo_h2f(unsigned int w) { return h2f(static_cast<unsigned short>(w & 0xffffu)); }");
   em.line("__device__ __forceinline__ float hi_h2f(unsigned int w) { return h2f(static_cast<unsigned short>(w >> 16)); }");
-  em.line("");
-  em.line("extern \"C\" __global__ void __launch_bounds__(" + std::to_string(sh.block) +
-          ") e3conv_fwd(");
-  em.line("    const " + T + "* __restrict__ x, const " + T + "* __restrict__ Y, const " + T +
-          "* __restrict__ s,");
-  em.line("    const int* __restrict__ senders, const int* __restrict__ row_ptr,");
-  em.line("    int num_nodes, int num_edges, float* __restrict__ out, float inv_avg,");
-  em.line("    unsigned int* __restrict__ status)");
-  em.line("{");
-  em.ind++;
-  em.line("const int lane = threadIdx.x & 31;");
-  em.line("const long long gwarp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;");
-  em.line("const int sub = lane / " + std::to_string(sh.TL) + ";");
-  em.line("const int within = lane - sub * " + std::to_string(sh.TL) + ";");
-  em.line("if (sub >= " + std::to_string(sh.ipw) + ") return;");
-  em.line("const long long item = gwarp * " + std::to_string(sh.ipw) + " + sub;");
-  em.line("const long long b = item / " + std::to_string(sh.tiles) + ";");
-  em.line("const int tile = (int)(item - b * " + std::to_string(sh.tiles) + ");");
-  em.line("if (b >= num_nodes) return;");
-  em.line("const int u0 = tile * " + std::to_string(sh.TL * V) + " + within * " +
-          std::to_string(V) + ";");
-  em.line("if (u0 >= " + std::to_string(pl.C) + ") return;");
-  // accumulators
-  for (int c = 0; c < pl.nout; ++c) {
-    std::string l = "float";
-    for (int v = 0; v < V; ++v)
-      l += std::string(v ? "," : "") + " a" + std::to_string(c) + "_" + std::to_string(v) + " = 0.f";
-    em.line(l + ";");
+  for (const char* pre : {"ldg", "lds"}) {
+    const bool g = pre[2] == 'g';
+    auto rd = [&](const std::string& type, const std::string& p) {
+      return g ? "__ldg(reinterpret_cast<const " + type + "*>(" + p + "))"
+               : "*reinterpret_cast<const " + type + "*>(" + p + ")";
+    };
+    const std::string P(pre);
+    em.line("__device__ __forceinline__ float " + P + "_f1(const float* p) { return " + rd("float", "p") + "; }");
+    em.line("__device__ __forceinline__ float2 " + P + "_f2(const float* p) { return " + rd("float2", "p") + "; }");
+    em.line("__device__ __forceinline__ float4 " + P + "_f4(const float* p) { return " + rd("float4", "p") + "; }");
+    em.line("__device__ __forceinline__ float " + P + "_h1(const unsigned short* p) { return h2f(" + rd("unsigned short", "p") + "); }");
+    em.line("__device__ __forceinline__ unsigned int " + P + "_u1(const unsigned short* p) { return " + rd("unsigned int", "p") + "; }");
+    em.line("__device__ __forceinline__ uint2 " + P + "_u2(const unsigned short* p) { return " + rd("uint2", "p") + "; }");
+    em.line("__device__ __forceinline__ uint4 " + P + "_u4(const unsigned short* p) { return " + rd("uint4", "p") + "; }");
   }
-  em.line("int e0 = row_ptr[b];");
-  em.line("int e1 = row_ptr[b + 1];");
-  em.line("if (e0 < 0 || e1 < e0 || e1 > num_edges) { atomicOr(status, 1u); e1 = e0; }");
-  em.line("#pragma unroll 1");
-  em.line("for (int e = e0; e < e1; ++e) {");
-  em.ind++;
-  em.line("const int a = senders[e];");
-  em.line("if ((unsigned int)a >= (unsigned int)num_nodes) { atomicOr(status, 2u); continue; }");
-  // Y row
-  {
-    std::string decl = "float";
-    for (int j = 0; j < pl.ny; ++j) decl += std::string(j ? "," : "") + " y" + std::to_string(j);
-    em.line(decl + ";");
-    em.line("const " + T + "* yr = Y + (long long)e * " + std::to_string(pl.ny) + ";");
-    if (!f16 && pl.ny % 4 == 0) {
-      for (int j = 0; j < pl.ny; j += 4)
-        em.line("{ const float4 t_ = ldg_f4(yr + " + std::to_string(j) + "); y" +
-                std::to_string(j) + " = t_.x; y" + std::to_string(j + 1) + " = t_.y; y" +
-                std::to_string(j + 2) + " = t_.z; y" + std::to_string(j + 3) + " = t_.w; }");
-    } else if (f16 && pl.ny % 8 == 0) {
-      for (int j = 0; j < pl.ny; j += 8) {
-        em.line("{ const uint4 t_ = ldg_u4(yr + " + std::to_string(j) + ");");
-        const char* w[4] = {"t_.x", "t_.y", "t_.z", "t_.w"};
-        for (int q = 0; q < 4; ++q)
-          em.line("  y" + std::to_string(j + 2 * q) + " = lo_h2f(" + w[q] + "); y" +
-                  std::to_string(j + 2 * q + 1) + " = hi_h2f(" + w[q] + ");");
-        em.line("}");
-      }
-    } else if (f16 && pl.ny % 2 == 0) {
-      for (int j = 0; j < pl.ny; j += 2)
-        em.line("{ const unsigned int t_ = ldg_u1(yr + " + std::to_string(j) + "); y" +
-                std::to_string(j) + " = lo_h2f(t_); y" + std::to_string(j + 1) +
-                " = hi_h2f(t_); }");
-    } else {
-      for (int j = 0; j < pl.ny; ++j)
-        em.line("y" + std::to_string(j) + " = " + (f16 ? "ldg_h1" : "ldg_f1") + "(yr + " +
-                std::to_string(j) + ");");
+}
+
+// Declares and loads y0..y{ny-1} from `yr` (global or shared).
+void emit_y_load(Emitter& em, const Plan& pl, int dtype, const std::string& pre,
+                 const std::string& yr) {
+  const bool f16 = dtype == E3CONV_F16;
+  std::string decl = "float";
+  for (int j = 0; j < pl.ny; ++j) decl += std::string(j ? "," : "") + " y" + S(j);
+  em.line(decl + ";");
+  if (!f16 && pl.ny % 4 == 0) {
+    for (int j = 0; j < pl.ny; j += 4)
+      em.line("{ const float4 t_ = " + pre + "_f4(" + yr + " + " + S(j) + "); y" + S(j) +
+              " = t_.x; y" + S(j + 1) + " = t_.y; y" + S(j + 2) + " = t_.z; y" + S(j + 3) +
+              " = t_.w; }");
+  } else if (f16 && pl.ny % 8 == 0) {
+    for (int j = 0; j < pl.ny; j += 8) {
+      em.line("{ const uint4 t_ = " + pre + "_u4(" + yr + " + " + S(j) + ");");
+      const char* w[4] = {"t_.x", "t_.y", "t_.z", "t_.w"};
+      for (int q = 0; q < 4; ++q)
+        em.line("  y" + S(j + 2 * q) + " = lo_h2f(" + w[q] + "); y" + S(j + 2 * q + 1) +
+                " = hi_h2f(" + w[q] + ");");
+      em.line("}");
     }
+  } else if (f16 && pl.ny % 2 == 0) {
+    for (int j = 0; j < pl.ny; j += 2)
+      em.line("{ const unsigned int t_ = " + pre + "_u1(" + yr + " + " + S(j) + "); y" + S(j) +
+              " = lo_h2f(t_); y" + S(j + 1) + " = hi_h2f(t_); }");
+  } else {
+    for (int j = 0; j < pl.ny; ++j)
+      em.line("y" + S(j) + " = " + pre + (f16 ? "_h1" : "_f1") + "(" + yr + " + " + S(j) + ");");
   }
-  em.line("const " + T + "* xr = x + (long long)a * " + std::to_string(pl.nx * pl.C) + " + u0;");
-  em.line("const " + T + "* sr = s + (long long)e * " +
-          std::to_string(static_cast<long long>(pl.paths.size()) * pl.C) + " + u0;");
-  // paths grouped by node irrep (canonical order keeps them contiguous)
+}
+
+// The per-edge contribution: x slices at xr + comp*C, s slices at sr + p*C
+// (both already offset by the lane's first channel), Y in y0..; adds into a*.
+void emit_edge_body(Emitter& em, const Plan& pl, int dtype, int V, const std::string& pre,
+                    const std::string& xr, const std::string& sr) {
   size_t p = 0;
   while (p < pl.paths.size()) {
     const int n1 = pl.paths[p].n1;
@@ -212,77 +216,69 @@ std::string generate_forward_source(const Plan& pl, int dtype, const Shape& sh) 
     while (q < pl.paths.size() && pl.paths[q].n1 == n1) ++q;
     const Path& first = pl.paths[p];
     const int d1 = 2 * first.l1 + 1;
-    em.line("{  // node irrep " + std::to_string(n1) + " (l=" + std::to_string(first.l1) + ")");
+    em.line("{  // node irrep " + S(n1) + " (l=" + S(first.l1) + ")");
     em.ind++;
     for (int i = 0; i < d1; ++i) {
       std::string decl = "float";
-      for (int v = 0; v < V; ++v)
-        decl += std::string(v ? "," : "") + " x" + std::to_string(i) + "_" + std::to_string(v);
+      for (int v = 0; v < V; ++v) decl += std::string(v ? "," : "") + " x" + S(i) + "_" + S(v);
       em.line(decl + ";");
-      emit_vec_load(em, dtype, V, "xr + " + std::to_string((first.x_off + i) * pl.C),
-                    "x" + std::to_string(i));
+      emit_vec_load(em, dtype, V, pre, xr + " + " + S((first.x_off + i) * pl.C), "x" + S(i));
     }
     for (size_t r = p; r < q; ++r) {
       const Path& P = pl.paths[r];
       const int d3 = 2 * P.l3 + 1;
-      em.line("{  // path " + std::to_string(r) + ": " + std::to_string(P.l1) + " x " +
-              std::to_string(P.l2) + " -> " + std::to_string(P.l3) + ", " +
-              std::to_string(P.nnz.size()) + " coefficients");
+      em.line("{  // path " + S(r) + ": " + S(P.l1) + " x " + S(P.l2) + " -> " + S(P.l3) + ", " +
+              S(P.nnz.size()) + " coefficients");
       em.ind++;
       {
         std::string decl = "float";
-        for (int v = 0; v < V; ++v) decl += std::string(v ? "," : "") + " s_" + std::to_string(v);
+        for (int v = 0; v < V; ++v) decl += std::string(v ? "," : "") + " s_" + S(v);
         em.line(decl + ";");
-        emit_vec_load(em, dtype, V, "sr + " + std::to_string(r * pl.C), "s");
+        emit_vec_load(em, dtype, V, pre, sr + " + " + S(static_cast<long long>(r) * pl.C), "s");
       }
-      // c * Y_j products, one per distinct (c, j)
       std::map<std::pair<float, int>, std::string> cy;
       auto cyname = [&](const Nnz& n) -> std::string {
         auto key = std::make_pair(static_cast<float>(n.c), n.j);
         auto it = cy.find(key);
         if (it != cy.end()) return it->second;
-        std::string nm = "c" + std::to_string(cy.size());
-        em.line("const float " + nm + " = " + flt(n.c) + " * y" + std::to_string(P.y_off + n.j) + ";");
+        std::string nm = "c" + S(cy.size());
+        em.line("const float " + nm + " = " + flt(n.c) + " * y" + S(P.y_off + n.j) + ";");
         cy[key] = nm;
         return nm;
       };
       std::vector<Nnz> nz = P.nnz;
-      std::stable_sort(nz.begin(), nz.end(),
-                       [](const Nnz& a, const Nnz& b) { return a.k < b.k; });
+      std::stable_sort(nz.begin(), nz.end(), [](const Nnz& a, const Nnz& b) { return a.k < b.k; });
       for (const auto& n : nz) cyname(n);
-      const bool scale_input = d1 <= d3;
-      if (scale_input) {
+      if (d1 <= d3) {  // scale-input
         std::vector<bool> used(d1, false);
         for (const auto& n : nz) used[n.i] = true;
         for (int i = 0; i < d1; ++i) {
           if (!used[i]) continue;
           for (int v = 0; v < V; ++v)
-            em.line("const float z" + std::to_string(i) + "_" + std::to_string(v) + " = s_" +
-                    std::to_string(v) + " * x" + std::to_string(i) + "_" + std::to_string(v) + ";");
+            em.line("const float z" + S(i) + "_" + S(v) + " = s_" + S(v) + " * x" + S(i) + "_" +
+                    S(v) + ";");
         }
         for (const auto& n : nz) {
           const std::string c = cyname(n);
           for (int v = 0; v < V; ++v) {
-            std::string acc = "a" + std::to_string(P.out_off + n.k) + "_" + std::to_string(v);
-            em.line(acc + " = fmaf(" + c + ", z" + std::to_string(n.i) + "_" + std::to_string(v) +
-                    ", " + acc + ");");
+            std::string acc = "a" + S(P.out_off + n.k) + "_" + S(v);
+            em.line(acc + " = fmaf(" + c + ", z" + S(n.i) + "_" + S(v) + ", " + acc + ");");
           }
         }
-      } else {
+      } else {  // scale-output
         for (int k = 0; k < d3; ++k) {
           std::vector<Nnz> row;
           for (const auto& n : nz)
             if (n.k == k) row.push_back(n);
           if (row.empty()) continue;
           for (int v = 0; v < V; ++v) {
-            std::string t = "t" + std::to_string(k) + "_" + std::to_string(v);
-            std::string xv0 = "x" + std::to_string(row[0].i) + "_" + std::to_string(v);
-            em.line("float " + t + " = " + cyname(row[0]) + " * " + xv0 + ";");
+            std::string t = "t" + S(k) + "_" + S(v);
+            em.line("float " + t + " = " + cyname(row[0]) + " * x" + S(row[0].i) + "_" + S(v) + ";");
             for (size_t m = 1; m < row.size(); ++m)
-              em.line(t + " = fmaf(" + cyname(row[m]) + ", x" + std::to_string(row[m].i) + "_" +
-                      std::to_string(v) + ", " + t + ");");
-            std::string acc = "a" + std::to_string(P.out_off + k) + "_" + std::to_string(v);
-            em.line(acc + " = fmaf(s_" + std::to_string(v) + ", " + t + ", " + acc + ");");
+              em.line(t + " = fmaf(" + cyname(row[m]) + ", x" + S(row[m].i) + "_" + S(v) + ", " +
+                      t + ");");
+            std::string acc = "a" + S(P.out_off + k) + "_" + S(v);
+            em.line(acc + " = fmaf(s_" + S(v) + ", " + t + ", " + acc + ");");
           }
         }
       }
@@ -293,27 +289,238 @@ std::string generate_forward_source(const Plan& pl, int dtype, const Shape& sh) 
     em.line("}");
     p = q;
   }
-  em.ind--;
-  em.line("}");
-  // store
-  em.line("float* orow = out + (long long)b * " + std::to_string(pl.nout * pl.C) + " + u0;");
+}
+
+void emit_acc_decl(Emitter& em, const Plan& pl, int V) {
   for (int c = 0; c < pl.nout; ++c) {
-    auto a = [&](int v) { return "a" + std::to_string(c) + "_" + std::to_string(v) + " * inv_avg"; };
-    const std::string dst = "orow + " + std::to_string(c * pl.C);
+    std::string l = "float";
+    for (int v = 0; v < V; ++v)
+      l += std::string(v ? "," : "") + " a" + S(c) + "_" + S(v) + " = 0.f";
+    em.line(l + ";");
+  }
+}
+
+// Stores acc * scale (or zeros) at orow + comp*C (+ lane offset already applied).
+void emit_store(Emitter& em, const Plan& pl, int V, const std::string& orow, bool zero,
+                bool reset) {
+  for (int c = 0; c < pl.nout; ++c) {
+    auto a = [&](int v) {
+      return zero ? std::string("0.f") : "a" + S(c) + "_" + S(v) + " * inv_avg";
+    };
+    const std::string dst = orow + " + " + S(c * pl.C);
     if (V % 4 == 0) {
       for (int v = 0; v < V; v += 4)
-        em.line("*reinterpret_cast<float4*>(" + dst + " + " + std::to_string(v) +
-                ") = make_float4(" + a(v) + ", " + a(v + 1) + ", " + a(v + 2) + ", " + a(v + 3) +
-                ");");
+        em.line("*reinterpret_cast<float4*>(" + dst + " + " + S(v) + ") = make_float4(" + a(v) +
+                ", " + a(v + 1) + ", " + a(v + 2) + ", " + a(v + 3) + ");");
     } else if (V == 2) {
       em.line("*reinterpret_cast<float2*>(" + dst + ") = make_float2(" + a(0) + ", " + a(1) + ");");
     } else {
       em.line("*(" + dst + ") = " + a(0) + ";");
     }
+    if (reset)
+      for (int v = 0; v < V; ++v) em.line("a" + S(c) + "_" + S(v) + " = 0.f;");
   }
+}
+
+void emit_signature(Emitter& em, const std::string& T, int block, int minb) {
+  em.line("extern \"C\" __global__ void __launch_bounds__(" + S(block) +
+          (minb > 0 ? ", " + S(minb) : std::string()) + ") e3conv_fwd(");
+  em.line("    const " + T + "* __restrict__ x, const " + T + "* __restrict__ Y, const " + T +
+          "* __restrict__ s,");
+  em.line("    const int* __restrict__ senders, const int* __restrict__ row_ptr,");
+  em.line("    int num_nodes, int num_edges, float* __restrict__ out, float inv_avg,");
+  em.line("    unsigned int* __restrict__ status)");
+}
+
+std::string direct_source(const Plan& pl, int dtype, const Shape& sh) {
+  Emitter em;
+  const int V = sh.V;
+  const bool f16 = dtype == E3CONV_F16;
+  const std::string T = f16 ? "unsigned short" : "float";
+  em.line("// generated by libe3conv: fused equivariant convolution forward (direct loads)");
+  em.line("// C=" + S(pl.C) + " nx=" + S(pl.nx) + " ny=" + S(pl.ny) + " nout=" + S(pl.nout) +
+          " paths=" + S(pl.paths.size()) + " dtype=" + (f16 ? "f16" : "f32") + " V=" + S(V) +
+          " TL=" + S(sh.TL) + " tiles=" + S(sh.tiles) + " ipw=" + S(sh.ipw));
+  emit_prelude(em);
+  emit_signature(em, T, sh.block, 0);
+  em.line("{");
+  em.ind++;
+  em.line("const int lane = threadIdx.x & 31;");
+  em.line("const long long gwarp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;");
+  em.line("const int sub = lane / " + S(sh.TL) + ";");
+  em.line("const int within = lane - sub * " + S(sh.TL) + ";");
+  em.line("if (sub >= " + S(sh.ipw) + ") return;");
+  em.line("const long long item = gwarp * " + S(sh.ipw) + " + sub;");
+  em.line("const long long b = item / " + S(sh.tiles) + ";");
+  em.line("const int tile = (int)(item - b * " + S(sh.tiles) + ");");
+  em.line("if (b >= num_nodes) return;");
+  em.line("const int u0 = tile * " + S(sh.TL * V) + " + within * " + S(V) + ";");
+  em.line("if (u0 >= " + S(pl.C) + ") return;");
+  emit_acc_decl(em, pl, V);
+  em.line("int e0 = row_ptr[b];");
+  em.line("int e1 = row_ptr[b + 1];");
+  em.line("if (e0 < 0 || e1 < e0 || e1 > num_edges) { atomicOr(status, 1u); e1 = e0; }");
+  em.line("#pragma unroll 1");
+  em.line("for (int e = e0; e < e1; ++e) {");
+  em.ind++;
+  em.line("const int a = senders[e];");
+  em.line("if ((unsigned int)a >= (unsigned int)num_nodes) { atomicOr(status, 2u); continue; }");
+  em.line("const " + T + "* yr = Y + (long long)e * " + S(pl.ny) + ";");
+  emit_y_load(em, pl, dtype, "ldg", "yr");
+  em.line("const " + T + "* xr = x + (long long)a * " + S(pl.nx * pl.C) + " + u0;");
+  em.line("const " + T + "* sr = s + (long long)e * " +
+          S(static_cast<long long>(pl.paths.size()) * pl.C) + " + u0;");
+  emit_edge_body(em, pl, dtype, V, "ldg", "xr", "sr");
+  em.ind--;
+  em.line("}");
+  em.line("float* orow = out + (long long)b * " + S(pl.nout * pl.C) + " + u0;");
+  emit_store(em, pl, V, "orow", false, false);
   em.ind--;
   em.line("}");
   return em.o.str();
+}
+
+std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
+  Emitter em;
+  const int V = sh.V;
+  const int NS = sh.stages;
+  const bool f16 = dtype == E3CONV_F16;
+  const std::string T = f16 ? "unsigned short" : "float";
+  const int warps = sh.block / 32;
+  const long long s_row = static_cast<long long>(pl.paths.size()) * pl.C;
+  em.line("// generated by libe3conv: fused equivariant convolution forward (staged ring)");
+  em.line("// C=" + S(pl.C) + " nx=" + S(pl.nx) + " ny=" + S(pl.ny) + " nout=" + S(pl.nout) +
+          " paths=" + S(pl.paths.size()) + " dtype=" + (f16 ? "f16" : "f32") + " V=" + S(V) +
+          " stages=" + S(NS) + " stage_bytes=" + S(sh.stage_bytes) + " warps/block=" + S(warps));
+  emit_prelude(em);
+  em.line("#define E3_SPIN_LIMIT (1u << 22)");
+  em.line("__device__ __forceinline__ unsigned int smem_u32(const void* p) { return static_cast<unsigned int>(__cvta_generic_to_shared(p)); }");
+  em.line("__device__ __forceinline__ void bar_init(unsigned long long* b) { asm volatile(\"mbarrier.init.shared::cta.b64 [%0], 1;\" :: \"r\"(smem_u32(b)) : \"memory\"); }");
+  em.line("__device__ __forceinline__ void bar_expect(unsigned long long* b, unsigned int bytes) { asm volatile(\"mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\" :: \"r\"(smem_u32(b)), \"r\"(bytes) : \"memory\"); }");
+  em.line("__device__ __forceinline__ bool bar_try(unsigned long long* b, unsigned int parity) {");
+  em.line("  unsigned int ok; asm volatile(\"{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }\" : \"=r\"(ok) : \"r\"(smem_u32(b)), \"r\"(parity) : \"memory\"); return ok != 0; }");
+  em.line("__device__ __forceinline__ bool bar_wait(unsigned long long* b, unsigned int parity) {");
+  em.line("  for (unsigned int it = 0; it < E3_SPIN_LIMIT; ++it) if (bar_try(b, parity)) return true; return false; }");
+  em.line("__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned int bytes, unsigned long long* b, unsigned long long policy) {");
+  em.line("  asm volatile(\"cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;\" :: \"r\"(smem_u32(dst)), \"l\"(src), \"r\"(bytes), \"r\"(smem_u32(b)), \"l\"(policy) : \"memory\"); }");
+  em.line("__device__ __forceinline__ unsigned long long policy_evict_first() { unsigned long long p; asm volatile(\"createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\" : \"=l\"(p)); return p; }");
+  em.line("__device__ __forceinline__ unsigned long long policy_evict_last() { unsigned long long p; asm volatile(\"createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\" : \"=l\"(p)); return p; }");
+  em.line("__device__ __forceinline__ void fence_async_smem() { asm volatile(\"fence.proxy.async.shared::cta;\" ::: \"memory\"); }");
+  emit_signature(em, T, sh.block, 1);
+  em.line("{");
+  em.ind++;
+  em.line("extern __shared__ __align__(128) unsigned char smem[];");
+  em.line("const int lane = threadIdx.x & 31;");
+  em.line("unsigned char* wbase = smem + (threadIdx.x >> 5) * " + S(sh.warp_smem) + ";");
+  em.line("unsigned long long* bars = reinterpret_cast<unsigned long long*>(wbase + " +
+          S(sh.bar_off) + ");");
+  em.line("int* hdr = reinterpret_cast<int*>(wbase + " + S(sh.hdr_off) + ");  // per stage: sender, receiver, last");
+  em.line("if (lane == 0) {");
+  em.line("  for (int k = 0; k < " + S(NS) + "; ++k) bar_init(bars + k);");
+  em.line("  asm volatile(\"fence.mbarrier_init.release.cluster;\" ::: \"memory\");");
+  em.line("}");
+  em.line("__syncwarp();");
+  em.line("const unsigned long long pol_stream = policy_evict_first();");
+  em.line("const unsigned long long pol_keep = policy_evict_last();");
+  em.line("const long long W = (long long)gridDim.x * " + S(warps) + ";");
+  em.line("const int u0 = lane * " + S(V) + ";");
+  // producer state (warp-uniform)
+  em.line("long long pb = (long long)blockIdx.x * " + S(warps) + " + (threadIdx.x >> 5) - W;  // producer receiver");
+  em.line("int pe = 0, pe1 = 0;      // producer edge cursor within row pb");
+  em.line("int pwin = -1, psw = 0;   // sender window base (edge index) and this lane's sender");
+  em.line("bool pdone = false;");
+  em.line("unsigned int ppos = 0, cpos = 0;");
+  emit_acc_decl(em, pl, V);
+  // produce lambda as a macro-like block: emitted inline via a device lambda
+  em.line("auto produce = [&]() {");
+  em.ind++;
+  em.line("while (!pdone && pe >= pe1) {");
+  em.line("  pb += W;");
+  em.line("  if (pb >= num_nodes) { pdone = true; break; }");
+  em.line("  int r0 = row_ptr[pb], r1 = row_ptr[pb + 1];");
+  em.line("  if (r0 < 0 || r1 < r0 || r1 > num_edges) { if (lane == 0) atomicOr(status, 1u); r1 = r0; }");
+  em.line("  pe = r0; pe1 = r1; pwin = -1;");
+  em.line("  if (r0 == r1) {  // empty row: zeros");
+  em.line("    float* zrow = out + pb * " + S(static_cast<long long>(pl.nout) * pl.C) + " + u0;");
+  em.ind += 2;
+  emit_store(em, pl, V, "zrow", true, false);
+  em.ind -= 2;
+  em.line("  }");
+  em.line("}");
+  em.line("if (pdone) return;");
+  em.line("if (pwin < 0 || pe >= pwin + 32) {");
+  em.line("  pwin = pe;");
+  em.line("  psw = (pe + lane < pe1) ? senders[pe + lane] : 0;");
+  em.line("}");
+  em.line("const int a = __shfl_sync(0xffffffffu, psw, pe - pwin);");
+  em.line("const bool valid = (unsigned int)a < (unsigned int)num_nodes;");
+  em.line("const unsigned int st = ppos % " + S(NS) + ";");
+  em.line("if (lane == 0) {");
+  em.line("  unsigned char* stg = wbase + st * " + S(sh.stage_bytes) + ";");
+  em.line("  hdr[4 * st] = valid ? a : -1;");
+  em.line("  hdr[4 * st + 1] = (int)pb;");
+  em.line("  hdr[4 * st + 2] = (pe + 1 == pe1) ? 1 : 0;");
+  em.line("  fence_async_smem();");
+  em.line("  bar_expect(bars + st, " + S(sh.s_bytes + sh.y_bytes) + "u + (valid ? " +
+          S(sh.x_bytes) + "u : 0u));");
+  em.line("  bulk_g2s(stg + " + S(sh.s_off) + ", s + (long long)pe * " + S(s_row) + ", " +
+          S(sh.s_bytes) + "u, bars + st, pol_stream);");
+  em.line("  bulk_g2s(stg + " + S(sh.y_off) + ", Y + (long long)pe * " + S(pl.ny) + ", " +
+          S(sh.y_bytes) + "u, bars + st, pol_stream);");
+  em.line("  if (valid) bulk_g2s(stg + " + S(sh.x_off) + ", x + (long long)a * " +
+          S(static_cast<long long>(pl.nx) * pl.C) + ", " + S(sh.x_bytes) +
+          "u, bars + st, pol_keep);");
+  em.line("}");
+  em.line("++pe;");
+  em.line("++ppos;");
+  em.ind--;
+  em.line("};");
+  em.line("for (int k = 0; k < " + S(NS) + "; ++k) produce();");
+  em.line("__syncwarp();");
+  em.line("#pragma unroll 1");
+  em.line("while (cpos != ppos) {");
+  em.ind++;
+  em.line("const unsigned int st = cpos % " + S(NS) + ";");
+  em.line("if (!bar_wait(bars + st, (cpos / " + S(NS) + ") & 1u)) {");
+  em.line("  if (lane == 0) atomicOr(status, 4u);");
+  em.line("  for (unsigned int q = cpos; q != ppos; ++q) bar_wait(bars + q % " + S(NS) + ", (q / " + S(NS) + ") & 1u);");
+  em.line("  return;");
+  em.line("}");
+  em.line("const unsigned char* stg = wbase + st * " + S(sh.stage_bytes) + ";");
+  em.line("const int a = hdr[4 * st];");
+  em.line("const long long b = hdr[4 * st + 1];");
+  em.line("const int last = hdr[4 * st + 2];");
+  em.line("if (a >= 0) {");
+  em.ind++;
+  em.line("const " + T + "* ys = reinterpret_cast<const " + T + "*>(stg + " + S(sh.y_off) + ");");
+  emit_y_load(em, pl, dtype, "lds", "ys");
+  em.line("const " + T + "* xs = reinterpret_cast<const " + T + "*>(stg + " + S(sh.x_off) + ") + u0;");
+  em.line("const " + T + "* ss = reinterpret_cast<const " + T + "*>(stg + " + S(sh.s_off) + ") + u0;");
+  emit_edge_body(em, pl, dtype, V, "lds", "xs", "ss");
+  em.ind--;
+  em.line("} else if (lane == 0) {");
+  em.line("  atomicOr(status, 2u);");
+  em.line("}");
+  em.line("if (last) {");
+  em.ind++;
+  em.line("float* orow = out + b * " + S(static_cast<long long>(pl.nout) * pl.C) + " + u0;");
+  emit_store(em, pl, V, "orow", false, true);
+  em.ind--;
+  em.line("}");
+  em.line("__syncwarp();");
+  em.line("++cpos;");
+  em.line("produce();");
+  em.ind--;
+  em.line("}");
+  em.ind--;
+  em.line("}");
+  return em.o.str();
+}
+
+}  // namespace
+
+std::string generate_forward_source(const Plan& pl, int dtype, const Shape& sh) {
+  return sh.stages > 0 ? staged_source(pl, dtype, sh) : direct_source(pl, dtype, sh);
 }
 
 }  // namespace e3c

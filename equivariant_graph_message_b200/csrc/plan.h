@@ -41,6 +41,13 @@ struct Shape {
   int tiles = 1;   // channel tiles per receiver
   int ipw = 1;     // items per warp
   int block = 128; // threads per block
+  // Staged (persistent, shared-memory ring) variant; stages == 0: direct loads.
+  int stages = 0;
+  int s_bytes = 0, x_bytes = 0, y_bytes = 0;  // row sizes staged per edge
+  int s_off = 0, x_off = 0, y_off = 0;        // offsets inside one stage
+  int stage_bytes = 0;                        // one stage, 128-byte aligned
+  int warp_smem = 0;                          // stages + barriers + headers of one warp
+  int bar_off = 0, hdr_off = 0;               // offsets inside a warp's region
 };
 
 struct Variant {
@@ -52,6 +59,7 @@ struct Variant {
   int regs = -1, local_bytes = -1;
   CUmodule module = nullptr;
   CUfunction fn = nullptr;
+  int grid_blocks = 0;  // persistent grid of the staged variant (blocks per SM x SMs)
 };
 
 struct Plan {
@@ -62,7 +70,7 @@ struct Plan {
   double avg = 1.0;
   int norm = 0;
   int dtype = E3CONV_F32;
-  int req_V = 0, req_block = 0;
+  int req_V = 0, req_block = 0, req_stages = -1;  // -1: automatic
   int device = -1;                 // -1: host-only plan
   CUcontext ctx = nullptr;
   unsigned int* status = nullptr;  // device status word

@@ -129,10 +129,15 @@ E3CONV_API void e3conv_destroy(e3conv_plan plan);
 E3CONV_API int e3conv_set_input_dtype(e3conv_plan plan, int dtype);
 
 /* Overrides the launch shape of the forward kernel: channels_per_lane in
- * {0 (automatic), 1, 2, 4, 8} (must divide C and fit one 16-byte load) and
- * block_threads in {0 (automatic), 32, 64, ..., 1024}.  Recompiles the
- * current dtype's kernel (host-side, blocking). */
-E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane, int block_threads);
+ * {0 (automatic), 1, 2, 4, 8} (must divide C and fit one 16-byte load),
+ * block_threads in {0 (automatic), 32, 64, ..., 1024}, and stages: -1
+ * (automatic), 0 (direct global loads) or 2..8 (persistent warps with a
+ * shared-memory ring of that many edges, used when one warp covers all C
+ * channels and every staged row is a multiple of 16 bytes; otherwise the
+ * direct variant is used).  Recompiles the current dtype's kernel
+ * (host-side, blocking). */
+E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane, int block_threads,
+                                        int stages);
 
 /* Sizes: C channels, nx node components, ny edge components, nout output
  * components, num_paths P.  Any pointer may be NULL. */
@@ -154,12 +159,11 @@ E3CONV_API int e3conv_output_irrep(e3conv_plan plan, int k, int* l, int* p, int*
 E3CONV_API int e3conv_cg(e3conv_plan plan, int p, double* dense_out);
 
 /* Launch shape and resources of the forward kernel for `dtype`:
- * channels per lane, lanes per receiver tile, block threads, registers per
- * thread, local-memory (spill) bytes per thread.  Any pointer may be NULL.
- * Returns E3CONV_ERR_NO_DEVICE for the resource fields' source if the plan
- * has no module, after filling the shape fields. */
+ * channels per lane, lanes per receiver tile, block threads, ring stages
+ * (0: direct variant), registers per thread and local-memory (spill) bytes
+ * per thread.  Any pointer may be NULL. */
 E3CONV_API int e3conv_kernel_info(e3conv_plan plan, int dtype, int* channels_per_lane, int* lanes_per_tile,
-                       int* block_threads, int* registers, int* local_bytes);
+                       int* block_threads, int* stages, int* registers, int* local_bytes);
 
 /* Copies the generated CUDA source for `dtype` (NUL-terminated) into buf if
  * buf_len is large enough; *needed receives the required size in bytes. */
@@ -182,6 +186,8 @@ E3CONV_API int e3conv_kernel_source(e3conv_plan plan, int dtype, char* buf, size
  * pointers may be NULL.
  * Out-of-range senders are skipped and row ranges outside [0, num_edges]
  * are treated as empty; both set the plan's status word (e3conv_check).
+ * The staged variant's bounded waits on its shared-memory ring, if they
+ * ever time out, also set the status word and end the kernel early.
  * Launches exactly one kernel on `stream`; no host synchronisation, no
  * allocation.  Concurrent forwards with one plan share its status word. */
 E3CONV_API int e3conv_forward(e3conv_plan plan, const void* node_features, const void* edge_sh,
@@ -190,8 +196,9 @@ E3CONV_API int e3conv_forward(e3conv_plan plan, const void* node_features, const
                    float* out, e3conv_stream stream);
 
 /* Synchronises `stream`, reads and clears the plan's status word.  Returns
- * E3CONV_OK or E3CONV_ERR_BAD_INDEX if a forward since the last check met an
- * out-of-range sender or row range. */
+ * E3CONV_OK, E3CONV_ERR_BAD_INDEX if a forward since the last check met an
+ * out-of-range sender or row range, or E3CONV_ERR_CUDA if a pipeline wait
+ * timed out. */
 E3CONV_API int e3conv_check(e3conv_plan plan, e3conv_stream stream);
 
 /* ---------------------------------------------------------------------------

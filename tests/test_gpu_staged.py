@@ -1,0 +1,141 @@
+"""GPU parity of the staged (persistent warps + shared-memory ring) forward variant."""
+import numpy as np
+import pytest
+import torch
+
+import equivariant_graph_message_b200 as e3
+import oracle
+from parity import TOL, column_scaled_error, oracle_out, row_ptr_of, run_gpu, to_dev
+
+pytestmark = pytest.mark.gpu
+
+SH3 = "1x0e+1x1o+1x2e+1x3o"
+IRREPS = {
+    32: ("32x0e+32x1o+32x2e", SH3, "32x0e+32x1o+32x2e+32x3o"),
+    64: ("64x0e+64x1o", SH3, "64x0e+64x1o+64x2e+64x1e"),
+    128: ("128x0e+128x1o+128x2e+128x3o", SH3, "128x0e+128x1o+128x2e+128x3o+128x1e"),
+}
+
+
+def _graph(rng, n, e, empty_frac=0.0):
+    recv = rng.integers(0, n, e)
+    if empty_frac:
+        keep = rng.random(n) >= empty_frac
+        pool = np.nonzero(keep)[0]
+        recv = pool[rng.integers(0, len(pool), e)]
+    send = rng.integers(0, n, e)
+    o = np.lexsort((send, recv))
+    return send[o], recv[o]
+
+
+def _inputs(rng, irreps, n, e, dt):
+    pl = oracle.plan(*irreps)
+    npdt = np.float16 if dt == "f16" else np.float32
+    return (pl, rng.normal(size=(n, pl.nx, pl.C)).astype(npdt),
+            rng.normal(size=(e, pl.ny)).astype(npdt),
+            rng.normal(size=(e, len(pl.paths), pl.C)).astype(npdt))
+
+
+@pytest.mark.parametrize("C", [32, 64, 128])
+@pytest.mark.parametrize("dt", ["f32", "f16"])
+def test_staged_parity_with_empty_rows(cuda_device, C, dt):
+    irreps = IRREPS[C]
+    rng = np.random.default_rng(C + (dt == "f16"))
+    n, e = 700, 9000
+    send, recv = _graph(rng, n, e, empty_frac=0.2)
+    pl, x, Y, s = _inputs(rng, irreps, n, e, dt)
+    conv = e3.Conv(*irreps, 12.0, dtype=dt)
+    assert conv.kernel_info()["stages"] >= 2
+    gpu = run_gpu(conv, x, Y, s, send, recv, n)
+    ref = oracle_out(irreps, x, Y, s, send, recv, n, 12.0)
+    assert column_scaled_error(gpu, ref) <= TOL[dt]
+    empty = np.setdiff1d(np.arange(n), recv)
+    assert len(empty) > 50 and np.all(gpu[empty] == 0)
+
+
+@pytest.mark.parametrize("stages,block", [(2, 32), (2, 128), (3, 64), (4, 96), (5, 32), (8, 32)])
+def test_staged_ring_depths(cuda_device, stages, block):
+    irreps = IRREPS[64]
+    rng = np.random.default_rng(stages * 100 + block)
+    n, e = 333, 5000
+    send, recv = _graph(rng, n, e)
+    pl, x, Y, s = _inputs(rng, irreps, n, e, "f32")
+    conv = e3.Conv(*irreps, 9.0)
+    conv.set_launch_config(0, block, stages)
+    info = conv.kernel_info()
+    assert info["stages"] == stages and info["block_threads"] == block
+    gpu = run_gpu(conv, x, Y, s, send, recv, n)
+    ref = oracle_out(irreps, x, Y, s, send, recv, n, 9.0)
+    assert column_scaled_error(gpu, ref) <= 1e-5
+
+
+def test_staged_few_nodes_many_warps_and_no_edges(cuda_device):
+    irreps = IRREPS[32]
+    rng = np.random.default_rng(9)
+    conv = e3.Conv(*irreps, 3.0)
+    assert conv.kernel_info()["stages"] >= 2
+    for n, e in ((1, 0), (3, 0), (1, 50), (5, 200)):
+        send, recv = _graph(rng, n, e) if e else (np.zeros(0, np.int64), np.zeros(0, np.int64))
+        pl, x, Y, s = _inputs(rng, irreps, n, e, "f32")
+        gpu = run_gpu(conv, x, Y, s, send, recv, n)
+        if e == 0:
+            assert np.all(gpu == 0)
+        else:
+            ref = oracle_out(irreps, x, Y, s, send, recv, n, 3.0)
+            assert np.all(np.abs(gpu - ref) <= 1e-5 * np.abs(ref).max())
+
+
+def test_staged_long_rows(cuda_device):
+    irreps = IRREPS[64]
+    rng = np.random.default_rng(10)
+    n, e = 40, 8000          # ~200 edges per row: several sender windows per row
+    send, recv = _graph(rng, n, e)
+    pl, x, Y, s = _inputs(rng, irreps, n, e, "f32")
+    conv = e3.Conv(*irreps, 200.0)
+    gpu = run_gpu(conv, x, Y, s, send, recv, n)
+    ref = oracle_out(irreps, x, Y, s, send, recv, n, 200.0)
+    assert column_scaled_error(gpu, ref) <= 1e-5
+
+
+def test_staged_bad_indices_flagged(cuda_device):
+    irreps = IRREPS[64]
+    rng = np.random.default_rng(11)
+    n, e = 50, 600
+    send, recv = _graph(rng, n, e)
+    pl, x, Y, s = _inputs(rng, irreps, n, e, "f32")
+    conv = e3.Conv(*irreps, 1.0)
+    assert conv.kernel_info()["stages"] >= 2
+    xd, Yd, sd = to_dev(x), to_dev(Y), to_dev(s)
+    rp = row_ptr_of(recv, n).astype(np.int32)
+    bad = send.copy()
+    bad[[5, 77, 300]] = [n, -1, 1 << 30]
+    out = conv.forward(xd, Yd, sd, to_dev(bad.astype(np.int32)), to_dev(rp))
+    assert not conv.check()
+    keep = np.ones(e, bool)
+    keep[[5, 77, 300]] = False
+    ref = oracle_out(irreps, x, Y[keep], s[keep], send[keep], recv[keep], n, 1.0)
+    assert column_scaled_error(out.cpu().numpy(), ref) <= 1e-5
+    bad_rp = rp.copy()
+    bad_rp[10] = e + 7
+    out = conv.forward(xd, Yd, sd, to_dev(send.astype(np.int32)), to_dev(bad_rp))
+    assert not conv.check()
+    assert conv.check()
+    assert torch.isfinite(out).all()
+
+
+def test_staged_matches_direct_bitwise_order_free(cuda_device):
+    # both variants sum a row's edges in row order with the same per-edge code
+    irreps = IRREPS[128]
+    rng = np.random.default_rng(12)
+    n, e = 500, 15000
+    send, recv = _graph(rng, n, e)
+    pl, x, Y, s = _inputs(rng, irreps, n, e, "f16")
+    a = e3.Conv(*irreps, 30.0, dtype="f16")
+    b = e3.Conv(*irreps, 30.0, dtype="f16")
+    b.set_launch_config(0, 0, 0)
+    assert a.kernel_info()["stages"] >= 2 and b.kernel_info()["stages"] == 0
+    ga = run_gpu(a, x, Y, s, send, recv, n)
+    gb = run_gpu(b, x, Y, s, send, recv, n)
+    ref = oracle_out(irreps, x, Y, s, send, recv, n, 30.0)
+    assert column_scaled_error(ga, ref) <= 5e-3 and column_scaled_error(gb, ref) <= 5e-3
+    np.testing.assert_allclose(ga, gb, rtol=1e-5, atol=1e-5 * np.abs(ref).max())
