@@ -51,7 +51,9 @@ _path = _sig("e3conv_path", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 7))
 _num_outputs = _sig("e3conv_num_outputs", ctypes.c_int, _vp, _c_int_p)
 _output_irrep = _sig("e3conv_output_irrep", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 3))
 _cg = _sig("e3conv_cg", ctypes.c_int, _vp, ctypes.c_int, ctypes.POINTER(ctypes.c_double))
-_kernel_info = _sig("e3conv_kernel_info", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 6))
+_kernel_info = _sig("e3conv_kernel_info", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 7))
+_set_option = _sig("e3conv_set_option", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_int)
+OPT_CONTRACT_FIRST = 1
 _kernel_source = _sig("e3conv_kernel_source", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_char_p,
                       ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t))
 _forward = _sig("e3conv_forward", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp,
@@ -69,7 +71,7 @@ _last_error = _sig("e3conv_last_error", ctypes.c_char_p)
 _version = _sig("e3conv_version", ctypes.c_int)
 
 EXPORTED = ["e3conv_create", "e3conv_destroy", "e3conv_set_input_dtype",
-            "e3conv_set_launch_config", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
+            "e3conv_set_launch_config", "e3conv_set_option", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
             "e3conv_output_irrep", "e3conv_cg", "e3conv_kernel_info", "e3conv_kernel_source",
             "e3conv_forward", "e3conv_check", "e3conv_csr_workspace_size", "e3conv_build_csr",
             "e3conv_csr_check", "e3conv_csr_kernel_count", "e3conv_permute_rows", "e3conv_strerror", "e3conv_last_error",
@@ -178,12 +180,15 @@ class Conv:
         _ok(_set_launch(self._h, channels_per_lane, block_threads, stages),
             "e3conv_set_launch_config")
 
+    def set_contract_first(self, value: int = -1):
+        _ok(_set_option(self._h, OPT_CONTRACT_FIRST, value), "e3conv_set_option")
+
     def kernel_info(self, dtype: str | None = None) -> dict:
-        v = [ctypes.c_int() for _ in range(6)]
+        v = [ctypes.c_int() for _ in range(7)]
         _ok(_kernel_info(self._h, {"f32": F32, "f16": F16}[dtype or self.dtype],
                          *[ctypes.byref(x) for x in v]), "e3conv_kernel_info")
-        keys = ["channels_per_lane", "lanes_per_tile", "block_threads", "stages", "registers",
-                "local_bytes"]
+        keys = ["channels_per_lane", "lanes_per_tile", "block_threads", "stages", "contract_first",
+                "registers", "local_bytes"]
         return dict(zip(keys, (x.value for x in v)))
 
     def kernel_source(self, dtype: str | None = None) -> str:

@@ -321,6 +321,20 @@ int e3conv_set_launch_config(e3conv_plan h, int channels_per_lane, int block_thr
   return compile_variant(pl, pl.dtype);
 }
 
+int e3conv_set_option(e3conv_plan h, int option, int value) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  Plan& pl = h->p;
+  if (option != E3CONV_OPT_CONTRACT_FIRST)
+    return fail(E3CONV_ERR_UNSUPPORTED, "unknown option");
+  if (value < -1 || value > 1) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1, 0 or 1");
+  pl.req_coop = value;
+  DeviceGuard g(pl.device);
+  const int other = pl.dtype == E3CONV_F32 ? E3CONV_F16 : E3CONV_F32;
+  release_variant(pl.var[other]);
+  release_variant(pl.var[pl.dtype]);
+  return compile_variant(pl, pl.dtype);
+}
+
 int e3conv_query(e3conv_plan h, int* C, int* nx, int* ny, int* nout, int* num_paths) {
   if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
   const Plan& pl = h->p;
@@ -376,7 +390,7 @@ int e3conv_cg(e3conv_plan h, int p, double* dense_out) {
 }
 
 int e3conv_kernel_info(e3conv_plan h, int dtype, int* V, int* TL, int* block, int* stages,
-                       int* regs, int* local_bytes) {
+                       int* contract_first, int* regs, int* local_bytes) {
   if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
   if (dtype != E3CONV_F32 && dtype != E3CONV_F16)
     return fail(E3CONV_ERR_UNSUPPORTED, "unknown dtype");
@@ -386,6 +400,7 @@ int e3conv_kernel_info(e3conv_plan h, int dtype, int* V, int* TL, int* block, in
   if (TL) *TL = v.shape.TL;
   if (block) *block = v.shape.block;
   if (stages) *stages = v.shape.stages;
+  if (contract_first) *contract_first = v.shape.coop ? 1 : 0;
   if (regs) *regs = v.regs;
   if (local_bytes) *local_bytes = v.local_bytes;
   return E3CONV_OK;

@@ -31,6 +31,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstring>
 #include <map>
 #include <sstream>
 
@@ -43,6 +44,30 @@ namespace {
 int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
 }  // namespace
+
+std::vector<AEntry> build_a_entries(const Plan& pl) {
+  std::vector<AEntry> out;
+  for (size_t p = 0; p < pl.paths.size(); ++p) {
+    const Path& P = pl.paths[p];
+    std::map<std::pair<int, int>, size_t> where;  // (k, i) -> entry
+    std::vector<AEntry> mine;
+    for (const auto& n : P.nnz) {
+      auto key = std::make_pair(n.k, n.i);
+      auto it = where.find(key);
+      if (it == where.end()) {
+        where[key] = mine.size();
+        mine.push_back(AEntry{static_cast<int>(p), n.i, n.k, {}});
+        it = where.find(key);
+      }
+      mine[it->second].terms.push_back({P.y_off + n.j, n.c});  // index into the full Y row
+    }
+    std::sort(mine.begin(), mine.end(), [](const AEntry& a, const AEntry& b) {
+      return a.k != b.k ? a.k < b.k : a.i < b.i;
+    });
+    out.insert(out.end(), mine.begin(), mine.end());
+  }
+  return out;
+}
 
 Shape choose_shape(const Plan& pl, int dtype) {
   Shape s;
@@ -86,12 +111,17 @@ Shape choose_shape(const Plan& pl, int dtype) {
     s.x_off = align_up(s.s_bytes, 128);
     s.y_off = s.x_off + align_up(s.x_bytes, 128);
     s.stage_bytes = s.y_off + align_up(s.y_bytes, 128);
+    s.coop = pl.req_coop != 0 && (V == 1 || V % 2 == 0);
+    s.na = s.coop ? static_cast<int>(build_a_entries(pl).size()) : 0;
+    const int extra = s.coop ? align_up(4 * s.na, 16) + align_up(4 * pl.ny, 16) : 0;
     int S = pl.req_stages > 0 ? pl.req_stages : (s.stage_bytes > 10240 ? 2 : 3);
     const int warps = s.block / 32;
     // keep one block within 227 KB of shared memory
-    while (S > 2 && warps * (S * s.stage_bytes + 256) > 227 * 1024) --S;
+    while (S > 2 && warps * (S * s.stage_bytes + extra + 256) > 227 * 1024) --S;
     s.stages = S;
-    s.bar_off = S * s.stage_bytes;
+    s.a_off = S * s.stage_bytes;
+    s.yf_off = s.a_off + (s.coop ? align_up(4 * s.na, 16) : 0);
+    s.bar_off = align_up(s.yf_off + (s.coop ? 4 * pl.ny : 0), 8);
     s.hdr_off = s.bar_off + 8 * S;
     s.warp_smem = align_up(s.hdr_off + 16 * S, 128);
     if (warps * s.warp_smem > 227 * 1024) s.stages = 0;
@@ -380,6 +410,246 @@ std::string direct_source(const Plan& pl, int dtype, const Shape& sh) {
   return em.o.str();
 }
 
+
+// ---------------------------------------------------------------------------
+// Cooperative contraction body (staged variant).
+//
+// Phase 1: lanes 0..ny-1 convert the edge's Y row to float32 in shared
+// memory; then every lane forms its share of the A entries (entries sorted by
+// term count and dealt to lanes in rounds of 32, so a round runs the same
+// number of terms in every lane) from a coefficient table in global memory,
+// and writes them to the warp's A area.
+// Phase 2: every lane applies A to its V channels: packed float32x2 FMAs on
+// channel pairs (V even) or scalar FMAs (V == 1).
+
+struct Lanes {
+  int V;
+  bool pairs() const { return V % 2 == 0; }
+  int groups() const { return pairs() ? V / 2 : 1; }
+  std::string type() const { return pairs() ? "unsigned long long" : "float"; }
+  std::string fma(const std::string& a, const std::string& b, const std::string& c) const {
+    return pairs() ? "fma2(" + a + ", " + b + ", " + c + ")" : "fmaf(" + a + ", " + b + ", " + c + ")";
+  }
+  std::string mul(const std::string& a, const std::string& b) const {
+    return pairs() ? "mul2(" + a + ", " + b + ")" : "(" + a + " * " + b + ")";
+  }
+  std::string bc(const std::string& a) const { return pairs() ? "bc(" + a + ")" : a; }
+};
+
+// Loads the lane's V channels at `ptr` (shared) into groups name_0..name_{G-1}.
+void emit_group_load(Emitter& em, int dtype, const Lanes& L, const std::string& ptr,
+                     const std::string& name) {
+  const bool f16 = dtype == E3CONV_F16;
+  std::string decl = L.type();
+  for (int g = 0; g < L.groups(); ++g) decl += std::string(g ? "," : "") + " " + name + "_" + S(g);
+  em.line(decl + ";");
+  if (!L.pairs()) {
+    em.line(name + "_0 = " + (f16 ? "lds_h1(" : "lds_f1(") + ptr + ");");
+    return;
+  }
+  if (!f16) {
+    for (int g = 0; g < L.groups(); g += 2) {
+      if (g + 1 < L.groups())
+        em.line("{ const ulonglong2 t_ = *reinterpret_cast<const ulonglong2*>(" + ptr + " + " +
+                S(2 * g) + "); " + name + "_" + S(g) + " = t_.x; " + name + "_" + S(g + 1) +
+                " = t_.y; }");
+      else
+        em.line(name + "_" + S(g) + " = *reinterpret_cast<const unsigned long long*>(" + ptr +
+                " + " + S(2 * g) + ");");
+    }
+  } else {
+    for (int g = 0; g < L.groups(); g += 2) {
+      if (g + 1 < L.groups())
+        em.line("{ const uint2 t_ = lds_u2(" + ptr + " + " + S(2 * g) + "); " + name + "_" + S(g) +
+                " = pk(lo_h2f(t_.x), hi_h2f(t_.x)); " + name + "_" + S(g + 1) +
+                " = pk(lo_h2f(t_.y), hi_h2f(t_.y)); }");
+      else
+        em.line("{ const unsigned int t_ = lds_u1(" + ptr + " + " + S(2 * g) + "); " + name + "_" +
+                S(g) + " = pk(lo_h2f(t_), hi_h2f(t_)); }");
+    }
+  }
+}
+
+struct CoopTables {
+  std::string source;  // __device__ tables
+  int rounds = 0;
+  std::vector<int> terms;  // per round
+};
+
+CoopTables coop_tables(const std::vector<AEntry>& ent) {
+  CoopTables T;
+  std::vector<int> order(ent.size());
+  for (size_t n = 0; n < ent.size(); ++n) order[n] = static_cast<int>(n);
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+    return ent[a].terms.size() > ent[b].terms.size();
+  });
+  T.rounds = static_cast<int>((ent.size() + 31) / 32);
+  std::ostringstream c, d;
+  c << "__device__ const int2 e3_atab[] = {\n";
+  d << "__device__ const short e3_adst[] = {\n";
+  for (int r = 0; r < T.rounds; ++r) {
+    int tr = 0;
+    for (int l = 0; l < 32; ++l) {
+      size_t q = static_cast<size_t>(r) * 32 + l;
+      if (q < order.size()) tr = std::max<int>(tr, static_cast<int>(ent[order[q]].terms.size()));
+    }
+    T.terms.push_back(tr);
+    for (int t = 0; t < tr; ++t) {
+      for (int l = 0; l < 32; ++l) {
+        size_t q = static_cast<size_t>(r) * 32 + l;
+        double cv = 0.0;
+        int j = 0;
+        if (q < order.size() && t < static_cast<int>(ent[order[q]].terms.size())) {
+          j = ent[order[q]].terms[t].first;
+          cv = ent[order[q]].terms[t].second;
+        }
+        const float cf = static_cast<float>(cv);
+        unsigned int bits;
+        std::memcpy(&bits, &cf, sizeof bits);
+        c << "{" << static_cast<int>(bits) << ", " << j << "},";
+      }
+      c << "\n";
+    }
+    for (int l = 0; l < 32; ++l) {
+      size_t q = static_cast<size_t>(r) * 32 + l;
+      d << (q < order.size() ? order[q] : -1) << ",";
+    }
+    d << "\n";
+  }
+  c << "};\n";
+  d << "};\n";
+  T.source = c.str() + d.str();
+  return T;
+}
+
+// Phase 1 + phase 2 for the edge staged at `stg`; y entries offset per path.
+void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
+                    const std::vector<AEntry>& ent, const CoopTables& T) {
+  const bool f16 = dtype == E3CONV_F16;
+  const std::string Ty = f16 ? "unsigned short" : "float";
+  const Lanes L{sh.V};
+  em.line("float* Aw = reinterpret_cast<float*>(wbase + " + S(sh.a_off) + ");");
+  em.line("float* yf = reinterpret_cast<float*>(wbase + " + S(sh.yf_off) + ");");
+  em.line("if (lane < " + S(pl.ny) + ") yf[lane] = " + (f16 ? "h2f" : "") + "(reinterpret_cast<const " +
+          Ty + "*>(stg + " + S(sh.y_off) + ")[lane]);");
+  em.line("__syncwarp();");
+  int base = 0;
+  for (int r = 0; r < T.rounds; ++r) {
+    em.line("{");
+    em.ind++;
+    for (int t = 0; t < T.terms[r]; ++t) {
+      em.line("const int2 k" + S(t) + " = __ldg(&e3_atab[" + S(base + t * 32) + " + lane]);");
+    }
+    std::string v = "__int_as_float(k0.x) * yf[k0.y]";
+    for (int t = 1; t < T.terms[r]; ++t)
+      v = "fmaf(__int_as_float(k" + S(t) + ".x), yf[k" + S(t) + ".y], " + v + ")";
+    em.line("const int dst = __ldg(&e3_adst[" + S(r * 32) + " + lane]);");
+    em.line("if (dst >= 0) Aw[dst] = " + v + ";");
+    em.ind--;
+    em.line("}");
+    base += T.terms[r] * 32;
+  }
+  em.line("__syncwarp();");
+  em.line("const " + Ty + "* xs = reinterpret_cast<const " + Ty + "*>(stg + " + S(sh.x_off) + ") + u0;");
+  em.line("const " + Ty + "* ss = reinterpret_cast<const " + Ty + "*>(stg + " + S(sh.s_off) + ") + u0;");
+  // entry index of (path, i, k)
+  std::map<std::tuple<int, int, int>, int> idx;
+  for (size_t n = 0; n < ent.size(); ++n) idx[{ent[n].path, ent[n].i, ent[n].k}] = static_cast<int>(n);
+  const int G = L.groups();
+  size_t p = 0;
+  while (p < pl.paths.size()) {
+    const int n1 = pl.paths[p].n1;
+    size_t q = p;
+    while (q < pl.paths.size() && pl.paths[q].n1 == n1) ++q;
+    const Path& first = pl.paths[p];
+    const int d1 = 2 * first.l1 + 1;
+    em.line("{  // node irrep " + S(n1) + " (l=" + S(first.l1) + ")");
+    em.ind++;
+    for (int i = 0; i < d1; ++i)
+      emit_group_load(em, dtype, L, "xs + " + S((first.x_off + i) * pl.C), "x" + S(i));
+    for (size_t r = p; r < q; ++r) {
+      const Path& P = pl.paths[r];
+      const int d3 = 2 * P.l3 + 1;
+      std::vector<const AEntry*> pe;
+      for (const auto& e : ent)
+        if (e.path == static_cast<int>(r)) pe.push_back(&e);
+      em.line("{  // path " + S(r) + ": " + S(P.l1) + " x " + S(P.l2) + " -> " + S(P.l3) + ", " +
+              S(pe.size()) + " entries");
+      em.ind++;
+      emit_group_load(em, dtype, L, "ss + " + S(static_cast<long long>(r) * pl.C), "s");
+      auto aval = [&](const AEntry* e) {
+        return "A" + S(idx[{e->path, e->i, e->k}]);
+      };
+      for (const AEntry* e : pe)
+        em.line("const " + L.type() + " " + aval(e) + " = " + L.bc("Aw[" + S(idx[{e->path, e->i, e->k}]) + "]") + ";");
+      if (d1 <= d3) {  // scale-input
+        std::vector<bool> used(d1, false);
+        for (const AEntry* e : pe) used[e->i] = true;
+        for (int i = 0; i < d1; ++i) {
+          if (!used[i]) continue;
+          for (int g = 0; g < G; ++g)
+            em.line("const " + L.type() + " z" + S(i) + "_" + S(g) + " = " +
+                    L.mul("s_" + S(g), "x" + S(i) + "_" + S(g)) + ";");
+        }
+        for (const AEntry* e : pe)
+          for (int g = 0; g < G; ++g) {
+            std::string acc = "q" + S(P.out_off + e->k) + "_" + S(g);
+            em.line(acc + " = " + L.fma(aval(e), "z" + S(e->i) + "_" + S(g), acc) + ";");
+          }
+      } else {  // scale-output
+        for (int k = 0; k < d3; ++k) {
+          std::vector<const AEntry*> row;
+          for (const AEntry* e : pe)
+            if (e->k == k) row.push_back(e);
+          if (row.empty()) continue;
+          for (int g = 0; g < G; ++g) {
+            std::string t = "t" + S(k) + "_" + S(g);
+            em.line(L.type() + " " + t + " = " + L.mul(aval(row[0]), "x" + S(row[0]->i) + "_" + S(g)) + ";");
+            for (size_t m = 1; m < row.size(); ++m)
+              em.line(t + " = " + L.fma(aval(row[m]), "x" + S(row[m]->i) + "_" + S(g), t) + ";");
+            std::string acc = "q" + S(P.out_off + k) + "_" + S(g);
+            em.line(acc + " = " + L.fma("s_" + S(g), t, acc) + ";");
+          }
+        }
+      }
+      em.ind--;
+      em.line("}");
+    }
+    em.ind--;
+    em.line("}");
+    p = q;
+  }
+}
+
+void emit_group_acc_decl(Emitter& em, const Plan& pl, const Lanes& L) {
+  for (int c = 0; c < pl.nout; ++c) {
+    std::string l = L.type();
+    for (int g = 0; g < L.groups(); ++g)
+      l += std::string(g ? "," : "") + " q" + S(c) + "_" + S(g) + (L.pairs() ? " = 0ull" : " = 0.f");
+    em.line(l + ";");
+  }
+}
+
+void emit_group_store(Emitter& em, const Plan& pl, const Lanes& L, const std::string& orow) {
+  for (int c = 0; c < pl.nout; ++c) {
+    const std::string dst = orow + " + " + S(c * pl.C);
+    if (!L.pairs()) {
+      em.line("*(" + dst + ") = q" + S(c) + "_0 * inv_avg;");
+      em.line("q" + S(c) + "_0 = 0.f;");
+      continue;
+    }
+    for (int g = 0; g < L.groups(); g += 2) {
+      if (g + 1 < L.groups())
+        em.line("*reinterpret_cast<ulonglong2*>(" + dst + " + " + S(2 * g) + ") = make_ulonglong2(mul2(q" +
+                S(c) + "_" + S(g) + ", inv2), mul2(q" + S(c) + "_" + S(g + 1) + ", inv2));");
+      else
+        em.line("*reinterpret_cast<unsigned long long*>(" + dst + " + " + S(2 * g) + ") = mul2(q" + S(c) +
+                "_" + S(g) + ", inv2);");
+    }
+    for (int g = 0; g < L.groups(); ++g) em.line("q" + S(c) + "_" + S(g) + " = 0ull;");
+  }
+}
+
 std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   Emitter em;
   const int V = sh.V;
@@ -393,6 +663,18 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
           " paths=" + S(pl.paths.size()) + " dtype=" + (f16 ? "f16" : "f32") + " V=" + S(V) +
           " stages=" + S(NS) + " stage_bytes=" + S(sh.stage_bytes) + " warps/block=" + S(warps));
   emit_prelude(em);
+  std::vector<AEntry> ent;
+  CoopTables tabs;
+  const Lanes L{V};
+  if (sh.coop) {
+    ent = build_a_entries(pl);
+    tabs = coop_tables(ent);
+    em.o << tabs.source;
+    em.line("__device__ __forceinline__ unsigned long long pk(float lo, float hi) { unsigned long long r; asm(\"mov.b64 %0, {%1, %2};\" : \"=l\"(r) : \"f\"(lo), \"f\"(hi)); return r; }");
+    em.line("__device__ __forceinline__ unsigned long long bc(float a) { return pk(a, a); }");
+    em.line("__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) { unsigned long long d; asm(\"fma.rn.f32x2 %0, %1, %2, %3;\" : \"=l\"(d) : \"l\"(a), \"l\"(b), \"l\"(c)); return d; }");
+    em.line("__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) { unsigned long long d; asm(\"mul.rn.f32x2 %0, %1, %2;\" : \"=l\"(d) : \"l\"(a), \"l\"(b)); return d; }");
+  }
   em.line("#define E3_SPIN_LIMIT (1u << 22)");
   em.line("__device__ __forceinline__ unsigned int smem_u32(const void* p) { return static_cast<unsigned int>(__cvta_generic_to_shared(p)); }");
   em.line("__device__ __forceinline__ void bar_init(unsigned long long* b) { asm volatile(\"mbarrier.init.shared::cta.b64 [%0], 1;\" :: \"r\"(smem_u32(b)) : \"memory\"); }");
@@ -430,7 +712,12 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("int pwin = -1, psw = 0;   // sender window base (edge index) and this lane's sender");
   em.line("bool pdone = false;");
   em.line("unsigned int ppos = 0, cpos = 0;");
-  emit_acc_decl(em, pl, V);
+  if (sh.coop) {
+    emit_group_acc_decl(em, pl, L);
+    if (L.pairs()) em.line("const unsigned long long inv2 = bc(inv_avg);");
+  } else {
+    emit_acc_decl(em, pl, V);
+  }
   // produce lambda as a macro-like block: emitted inline via a device lambda
   em.line("auto produce = [&]() {");
   em.ind++;
@@ -492,11 +779,15 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("const int last = hdr[4 * st + 2];");
   em.line("if (a >= 0) {");
   em.ind++;
-  em.line("const " + T + "* ys = reinterpret_cast<const " + T + "*>(stg + " + S(sh.y_off) + ");");
-  emit_y_load(em, pl, dtype, "lds", "ys");
-  em.line("const " + T + "* xs = reinterpret_cast<const " + T + "*>(stg + " + S(sh.x_off) + ") + u0;");
-  em.line("const " + T + "* ss = reinterpret_cast<const " + T + "*>(stg + " + S(sh.s_off) + ") + u0;");
-  emit_edge_body(em, pl, dtype, V, "lds", "xs", "ss");
+  if (sh.coop) {
+    emit_coop_edge(em, pl, dtype, sh, ent, tabs);
+  } else {
+    em.line("const " + T + "* ys = reinterpret_cast<const " + T + "*>(stg + " + S(sh.y_off) + ");");
+    emit_y_load(em, pl, dtype, "lds", "ys");
+    em.line("const " + T + "* xs = reinterpret_cast<const " + T + "*>(stg + " + S(sh.x_off) + ") + u0;");
+    em.line("const " + T + "* ss = reinterpret_cast<const " + T + "*>(stg + " + S(sh.s_off) + ") + u0;");
+    emit_edge_body(em, pl, dtype, V, "lds", "xs", "ss");
+  }
   em.ind--;
   em.line("} else if (lane == 0) {");
   em.line("  atomicOr(status, 2u);");
@@ -504,7 +795,10 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("if (last) {");
   em.ind++;
   em.line("float* orow = out + b * " + S(static_cast<long long>(pl.nout) * pl.C) + " + u0;");
-  emit_store(em, pl, V, "orow", false, true);
+  if (sh.coop)
+    emit_group_store(em, pl, L, "orow");
+  else
+    emit_store(em, pl, V, "orow", false, true);
   em.ind--;
   em.line("}");
   em.line("__syncwarp();");

@@ -48,6 +48,18 @@ struct Shape {
   int stage_bytes = 0;                        // one stage, 128-byte aligned
   int warp_smem = 0;                          // stages + barriers + headers of one warp
   int bar_off = 0, hdr_off = 0;               // offsets inside a warp's region
+  // Cooperative contraction (staged variant): per edge the warp first forms
+  // A_p[i,k] = sum_j CG_p[i,j,k] Y_j in shared memory, then every lane applies
+  // it to its channels with packed float32x2 FMAs.
+  bool coop = false;
+  int na = 0;                                 // number of A entries (all paths)
+  int a_off = 0, yf_off = 0;                  // A entries and float32 Y inside a warp's region
+};
+
+// One entry A_p[i,k] of the per-edge contraction of CG with Y.
+struct AEntry {
+  int path, i, k;
+  std::vector<std::pair<int, double>> terms;  // (index into the edge's Y row, CG coefficient)
 };
 
 struct Variant {
@@ -71,6 +83,7 @@ struct Plan {
   int norm = 0;
   int dtype = E3CONV_F32;
   int req_V = 0, req_block = 0, req_stages = -1;  // -1: automatic
+  int req_coop = -1;                               // -1: automatic, 0: off, 1: on
   int device = -1;                 // -1: host-only plan
   CUcontext ctx = nullptr;
   unsigned int* status = nullptr;  // device status word
@@ -85,6 +98,7 @@ int build_paths(Plan& plan, std::string& err);
 std::vector<double> real_wigner_3j(int l1, int l2, int l3);
 
 // codegen.cpp
+std::vector<AEntry> build_a_entries(const Plan& plan);
 Shape choose_shape(const Plan& plan, int dtype);
 std::string generate_forward_source(const Plan& plan, int dtype, const Shape& shape);
 

@@ -139,6 +139,17 @@ E3CONV_API int e3conv_set_input_dtype(e3conv_plan plan, int dtype);
 E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane, int block_threads,
                                         int stages);
 
+/* Options of the forward kernel (host-side; each recompiles the current
+ * dtype's kernel):
+ *   E3CONV_OPT_CONTRACT_FIRST: -1 automatic (default), 0 or 1.  With 1 the
+ *   staged variant first contracts every path's CG tensor with the edge's Y
+ *   into A_p[i,k] = sum_j CG_p[i,j,k] Y_j (channel-independent, shared by the
+ *   warp in shared memory) and then applies A_p to each channel with packed
+ *   float32x2 FMAs; with 0 every lane forms the products CG*Y_j itself.
+ *   Same arithmetic up to rounding order. */
+#define E3CONV_OPT_CONTRACT_FIRST 1
+E3CONV_API int e3conv_set_option(e3conv_plan plan, int option, int value);
+
 /* Sizes: C channels, nx node components, ny edge components, nout output
  * components, num_paths P.  Any pointer may be NULL. */
 E3CONV_API int e3conv_query(e3conv_plan plan, int* C, int* nx, int* ny, int* nout, int* num_paths);
@@ -160,10 +171,12 @@ E3CONV_API int e3conv_cg(e3conv_plan plan, int p, double* dense_out);
 
 /* Launch shape and resources of the forward kernel for `dtype`:
  * channels per lane, lanes per receiver tile, block threads, ring stages
- * (0: direct variant), registers per thread and local-memory (spill) bytes
- * per thread.  Any pointer may be NULL. */
-E3CONV_API int e3conv_kernel_info(e3conv_plan plan, int dtype, int* channels_per_lane, int* lanes_per_tile,
-                       int* block_threads, int* stages, int* registers, int* local_bytes);
+ * (0: direct variant), whether the CG x Y contraction is formed first
+ * (E3CONV_OPT_CONTRACT_FIRST), registers per thread and local-memory (spill)
+ * bytes per thread.  Any pointer may be NULL. */
+E3CONV_API int e3conv_kernel_info(e3conv_plan plan, int dtype, int* channels_per_lane,
+                                  int* lanes_per_tile, int* block_threads, int* stages,
+                                  int* contract_first, int* registers, int* local_bytes);
 
 /* Copies the generated CUDA source for `dtype` (NUL-terminated) into buf if
  * buf_len is large enough; *needed receives the required size in bytes. */

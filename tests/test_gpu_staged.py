@@ -38,14 +38,17 @@ def _inputs(rng, irreps, n, e, dt):
 
 @pytest.mark.parametrize("C", [32, 64, 128])
 @pytest.mark.parametrize("dt", ["f32", "f16"])
-def test_staged_parity_with_empty_rows(cuda_device, C, dt):
+@pytest.mark.parametrize("contract_first", [0, 1])
+def test_staged_parity_with_empty_rows(cuda_device, C, dt, contract_first):
     irreps = IRREPS[C]
     rng = np.random.default_rng(C + (dt == "f16"))
     n, e = 700, 9000
     send, recv = _graph(rng, n, e, empty_frac=0.2)
     pl, x, Y, s = _inputs(rng, irreps, n, e, dt)
     conv = e3.Conv(*irreps, 12.0, dtype=dt)
-    assert conv.kernel_info()["stages"] >= 2
+    conv.set_contract_first(contract_first)
+    info = conv.kernel_info()
+    assert info["stages"] >= 2 and info["contract_first"] == contract_first
     gpu = run_gpu(conv, x, Y, s, send, recv, n)
     ref = oracle_out(irreps, x, Y, s, send, recv, n, 12.0)
     assert column_scaled_error(gpu, ref) <= TOL[dt]
@@ -54,13 +57,15 @@ def test_staged_parity_with_empty_rows(cuda_device, C, dt):
 
 
 @pytest.mark.parametrize("stages,block", [(2, 32), (2, 128), (3, 64), (4, 96), (5, 32), (8, 32)])
-def test_staged_ring_depths(cuda_device, stages, block):
+@pytest.mark.parametrize("contract_first", [0, 1])
+def test_staged_ring_depths(cuda_device, stages, block, contract_first):
     irreps = IRREPS[64]
     rng = np.random.default_rng(stages * 100 + block)
     n, e = 333, 5000
     send, recv = _graph(rng, n, e)
     pl, x, Y, s = _inputs(rng, irreps, n, e, "f32")
     conv = e3.Conv(*irreps, 9.0)
+    conv.set_contract_first(contract_first)
     conv.set_launch_config(0, block, stages)
     info = conv.kernel_info()
     assert info["stages"] == stages and info["block_threads"] == block

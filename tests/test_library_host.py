@@ -99,11 +99,26 @@ def test_create_rejects_bad_scalars():
 def test_generated_kernel_unrolls_every_coefficient():
     s = SPECS["large_f16"]
     c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 40.0, dtype="f16")
-    src = c.kernel_source()
-    info = c.kernel_info()
-    V = info["channels_per_lane"]
     nnz = sum(int((np.abs(c.cg(p)) > 1e-12).sum()) for p in range(c.num_paths))
     assert nnz == 611
+    # contraction-first (default for this shape): one table entry per nonzero
+    # A_p[i,k] = sum_j CG_p[i,j,k] Y_j, each applied to every channel pair
+    info = c.kernel_info()
+    assert info["contract_first"] == 1 and info["stages"] >= 2 and info["local_bytes"] == 0
+    src = c.kernel_source()
+    na = sum(int((np.abs(c.cg(p)) > 1e-12).any(axis=1).sum()) for p in range(c.num_paths))
+    assert na == 541
+    dst = re.search(r"e3_adst\[\] = \{([^}]*)\}", src).group(1)
+    entries = sorted(int(v) for v in dst.replace("\n", "").split(",") if v.strip() not in ("", "-1"))
+    assert entries == list(range(na))
+    groups = info["channels_per_lane"] // 2
+    assert src.count("fma2(") + src.count("mul2(") >= na * groups
+    # per-lane products (contract_first = 0): every CG nonzero for every channel
+    c.set_contract_first(0)
+    info = c.kernel_info()
+    assert info["contract_first"] == 0
+    src = c.kernel_source()
+    V = info["channels_per_lane"]
     n_fma = src.count("fmaf(")
     n_mul = len(re.findall(r"= c\d+ \* x", src)) + len(re.findall(r"= s_\d \* x", src))
     assert n_fma + n_mul >= nnz * V
