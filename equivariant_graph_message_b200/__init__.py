@@ -65,6 +65,7 @@ _build_csr = _sig("e3conv_build_csr", ctypes.c_int, _vp, _i64, _i64, _vp, _vp, _
                   ctypes.c_size_t, _vp)
 _csr_check = _sig("e3conv_csr_check", ctypes.c_int, _vp, _vp)
 _csr_count = _sig("e3conv_csr_kernel_count", ctypes.c_int, _i64, _i64, _c_int_p)
+_build_csr_noalloc = _sig("e3conv_build_csr_noalloc", ctypes.c_int, _vp, _i64, _i64, _vp, _vp, _vp)
 _permute = _sig("e3conv_permute_rows", ctypes.c_int, _vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp)
 _strerror = _sig("e3conv_strerror", ctypes.c_char_p, ctypes.c_int)
 _last_error = _sig("e3conv_last_error", ctypes.c_char_p)
@@ -74,7 +75,7 @@ EXPORTED = ["e3conv_create", "e3conv_destroy", "e3conv_set_input_dtype",
             "e3conv_set_launch_config", "e3conv_set_option", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
             "e3conv_output_irrep", "e3conv_cg", "e3conv_kernel_info", "e3conv_kernel_source",
             "e3conv_forward", "e3conv_check", "e3conv_csr_workspace_size", "e3conv_build_csr",
-            "e3conv_csr_check", "e3conv_csr_kernel_count", "e3conv_permute_rows", "e3conv_strerror", "e3conv_last_error",
+            "e3conv_csr_check", "e3conv_build_csr_noalloc", "e3conv_csr_kernel_count", "e3conv_permute_rows", "e3conv_strerror", "e3conv_last_error",
             "e3conv_version"]
 
 
@@ -263,6 +264,23 @@ def build_csr(receivers, num_nodes: int, row_ptr=None, perm=None, workspace=None
                    _ptr(perm) if E else None, _ptr(workspace), workspace.numel(),
                    _stream_handle(stream)), "e3conv_build_csr")
     return row_ptr, perm, workspace
+
+
+def build_csr_noalloc(receivers, num_nodes: int, row_ptr=None, perm=None, stream=None):
+    """e3conv_build_csr_noalloc: the CSR build with the library's fixed scratch
+    (for callers that cannot allocate device memory; outputs may be passed in)."""
+    import torch
+    E = receivers.shape[0]
+    if receivers.dtype != torch.int32:
+        raise ValueError("receivers must be int32")
+    if row_ptr is None:
+        row_ptr = torch.empty(num_nodes + 1, dtype=torch.int32, device=receivers.device)
+    if perm is None:
+        perm = torch.empty(max(E, 1), dtype=torch.int32, device=receivers.device)[:E]
+    _ok(_build_csr_noalloc(_ptr(receivers) if E else None, E, num_nodes, _ptr(row_ptr),
+                           _ptr(perm) if E else None, _stream_handle(stream)),
+        "e3conv_build_csr_noalloc")
+    return row_ptr, perm
 
 
 def csr_kernel_count(num_edges: int, num_nodes: int) -> int:

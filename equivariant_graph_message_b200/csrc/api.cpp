@@ -19,6 +19,8 @@ size_t csr_workspace_bytes(int64_t E, int64_t N);
 int csr_build(const int* recv, int64_t E, int64_t N, int* row_ptr, int* perm, void* ws,
               size_t ws_bytes, cudaStream_t st, std::string& err, int* count);
 int csr_read_status(const void* ws, cudaStream_t st, unsigned* out);
+int csr_build_static(const int* recv, int64_t E, int64_t N, int* row_ptr, int* perm,
+                     cudaStream_t st, std::string& err);
 int permute_rows(const void* src, int64_t num_src, const int* perm, int64_t rows, int64_t row_bytes,
                  void* dst, int* status, cudaStream_t st, std::string& err);
 }  // namespace e3c
@@ -502,6 +504,19 @@ int e3conv_build_csr(const int32_t* receivers, int64_t num_edges, int64_t num_no
   std::string err;
   int rc = csr_build(receivers, num_edges, num_nodes, row_ptr, perm, workspace, workspace_bytes,
                      reinterpret_cast<cudaStream_t>(stream), err, nullptr);
+  return rc == E3CONV_OK ? rc : fail(rc, err);
+}
+
+int e3conv_build_csr_noalloc(const int32_t* receivers, int64_t num_edges, int64_t num_nodes,
+                             int32_t* row_ptr, int32_t* perm, e3conv_stream stream) {
+  if (num_edges < 0 || num_nodes < 0 || num_edges >= (1ll << 31) || num_nodes >= (1ll << 31) - 1)
+    return fail(E3CONV_ERR_INVALID_ARG, "sizes out of range");
+  if (!row_ptr || (num_edges > 0 && (!receivers || !perm)))
+    return fail(E3CONV_ERR_INVALID_ARG, "NULL buffer");
+  if (!has_device()) return fail(E3CONV_ERR_NO_DEVICE, "no CUDA device");
+  std::string err;
+  int rc = csr_build_static(receivers, num_edges, num_nodes, row_ptr, perm,
+                            reinterpret_cast<cudaStream_t>(stream), err);
   return rc == E3CONV_OK ? rc : fail(rc, err);
 }
 

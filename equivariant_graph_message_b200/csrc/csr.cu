@@ -15,6 +15,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 #include <string>
 
 #include "../../include/e3conv.h"
@@ -343,6 +344,60 @@ int csr_build(const int* recv, int64_t E, int64_t N, int* row_ptr, int* perm, vo
     return E3CONV_ERR_CUDA;
   }
   return E3CONV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free CSR build: the same kernels with a fixed scratch area.
+//
+// For callers that must not allocate device memory themselves (see
+// e3conv_build_csr_noalloc in e3conv.h).  The scratch is a file-scope device
+// array, so every GPU that loads this library holds kStaticScratchBytes of it
+// until the process exits.  Host code cannot use the array's name as a device
+// address (it names a host-side shadow); its device address is looked up once
+// per device with cudaGetSymbolAddress, with that device current.
+
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_csr_scratch[kStaticScratchBytes];
+
+size_t csr_static_scratch_bytes() { return kStaticScratchBytes; }
+
+int csr_build_static(const int* recv, int64_t E, int64_t N, int* row_ptr, int* perm,
+                     cudaStream_t st, std::string& err) {
+  const size_t need = csr_workspace_bytes(E, N);
+  if (need > kStaticScratchBytes) {
+    err = "e3conv_build_csr_noalloc: these sizes need " + std::to_string(need) +
+          " bytes of scratch, more than its fixed " + std::to_string(kStaticScratchBytes) +
+          " bytes; use e3conv_build_csr with a caller-provided workspace";
+    return E3CONV_ERR_WORKSPACE;
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    err = "no current CUDA device";
+    return E3CONV_ERR_CUDA;
+  }
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  if (dev >= kMaxDevices) {
+    err = "device ordinal above 63";
+    return E3CONV_ERR_UNSUPPORTED;
+  }
+  void* ptr = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+      void* p = nullptr;
+      // set-up, once per device, with that device current
+      if (cudaGetSymbolAddress(&p, g_csr_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        err = "cudaGetSymbolAddress of the static CSR scratch failed";
+        return E3CONV_ERR_CUDA;
+      }
+      addr[dev] = p;
+    }
+    ptr = addr[dev];
+  }
+  return csr_build(recv, E, N, row_ptr, perm, ptr, kStaticScratchBytes, st, err, nullptr);
 }
 
 int csr_read_status(const void* ws, cudaStream_t st, unsigned* out) {

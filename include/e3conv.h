@@ -236,6 +236,33 @@ E3CONV_API int e3conv_build_csr(const int32_t* receivers, int64_t num_edges, int
                      int32_t* row_ptr, int32_t* perm, void* workspace, size_t workspace_bytes,
                      e3conv_stream stream);
 
+/* Allocation-free variant of e3conv_build_csr (no counterpart on the pages
+ * this library follows; it exists for callers that cannot allocate device
+ * memory: code that runs where a framework's allocator owns all device
+ * memory, plugins handed a fixed memory budget, or latency-critical paths
+ * that must not call cudaMalloc because it can synchronise the device).
+ * Same arguments, results and kernels as e3conv_build_csr, but the scratch
+ * is a fixed 32 MiB array of device memory inside this library (every GPU
+ * that loads the library holds it until the process exits), so the caller
+ * passes only inputs and outputs.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *   - Sizes whose workspace (e3conv_csr_workspace_size) exceeds 32 MiB are
+ *     rejected with E3CONV_ERR_WORKSPACE before anything is launched (about
+ *     two million edges fit).
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents:
+ *     every call clears what must start at zero itself, but two calls whose
+ *     work overlaps on the GPU (different streams, or different host threads,
+ *     on one device) race on the array and give wrong results.  Order them.
+ *   - Receivers outside [0, num_nodes) are sorted after all valid edges and
+ *     not counted, so row_ptr[num_nodes] < num_edges reveals them (there is
+ *     no workspace status word to read). */
+E3CONV_API int e3conv_build_csr_noalloc(const int32_t* receivers, int64_t num_edges,
+                                        int64_t num_nodes, int32_t* row_ptr, int32_t* perm,
+                                        e3conv_stream stream);
+
 /* Number of kernels one e3conv_build_csr call with these sizes launches
  * (it also issues two cudaMemsetAsync calls).  Host only. */
 E3CONV_API int e3conv_csr_kernel_count(int64_t num_edges, int64_t num_nodes, int* count);
