@@ -471,11 +471,16 @@ void emit_group_load(Emitter& em, int dtype, const Lanes& L, const std::string& 
 }
 
 struct CoopTables {
-  std::string source;  // __device__ tables
+  std::string source;      // __device__ table of phase 1
   int rounds = 0;
-  std::vector<int> terms;  // per round
+  std::vector<int> terms;  // terms per round
+  std::vector<int> slot;   // entry -> position in the warp's A area
 };
 
+// Phase 1 deals the entries to lanes in rounds of 32, longest first, and
+// stores entry number q of that order at A[q]: every round writes 32
+// consecutive words (no bank conflicts) and phase 2 reads A at the
+// compile-time position slot[n] of entry n.
 CoopTables coop_tables(const std::vector<AEntry>& ent) {
   CoopTables T;
   std::vector<int> order(ent.size());
@@ -483,10 +488,15 @@ CoopTables coop_tables(const std::vector<AEntry>& ent) {
   std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
     return ent[a].terms.size() > ent[b].terms.size();
   });
+  T.slot.assign(ent.size(), -1);
+  for (size_t q = 0; q < order.size(); ++q) T.slot[order[q]] = static_cast<int>(q);
   T.rounds = static_cast<int>((ent.size() + 31) / 32);
-  std::ostringstream c, d;
+  std::ostringstream c, lay;
   c << "__device__ const int2 e3_atab[] = {\n";
-  d << "__device__ const short e3_adst[] = {\n";
+  lay << "// A layout (slot: path i k):";
+  for (size_t q = 0; q < order.size(); ++q)
+    lay << " " << ent[order[q]].path << ":" << ent[order[q]].i << ":" << ent[order[q]].k;
+  lay << "\n";
   for (int r = 0; r < T.rounds; ++r) {
     int tr = 0;
     for (int l = 0; l < 32; ++l) {
@@ -510,15 +520,9 @@ CoopTables coop_tables(const std::vector<AEntry>& ent) {
       }
       c << "\n";
     }
-    for (int l = 0; l < 32; ++l) {
-      size_t q = static_cast<size_t>(r) * 32 + l;
-      d << (q < order.size() ? order[q] : -1) << ",";
-    }
-    d << "\n";
   }
   c << "};\n";
-  d << "};\n";
-  T.source = c.str() + d.str();
+  T.source = lay.str() + c.str();
   return T;
 }
 
@@ -535,7 +539,7 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
   em.line("__syncwarp();");
   int base = 0;
   for (int r = 0; r < T.rounds; ++r) {
-    em.line("{");
+    em.line("{  // round terms: " + S(T.terms[r]));
     em.ind++;
     for (int t = 0; t < T.terms[r]; ++t) {
       em.line("const int2 k" + S(t) + " = __ldg(&e3_atab[" + S(base + t * 32) + " + lane]);");
@@ -543,8 +547,11 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
     std::string v = "__int_as_float(k0.x) * yf[k0.y]";
     for (int t = 1; t < T.terms[r]; ++t)
       v = "fmaf(__int_as_float(k" + S(t) + ".x), yf[k" + S(t) + ".y], " + v + ")";
-    em.line("const int dst = __ldg(&e3_adst[" + S(r * 32) + " + lane]);");
-    em.line("if (dst >= 0) Aw[dst] = " + v + ";");
+    const int na = static_cast<int>(ent.size());
+    if ((r + 1) * 32 <= na)
+      em.line("Aw[" + S(r * 32) + " + lane] = " + v + ";");
+    else
+      em.line("if (lane < " + S(na - r * 32) + ") Aw[" + S(r * 32) + " + lane] = " + v + ";");
     em.ind--;
     em.line("}");
     base += T.terms[r] * 32;
@@ -581,7 +588,8 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
         return "A" + S(idx[{e->path, e->i, e->k}]);
       };
       for (const AEntry* e : pe)
-        em.line("const " + L.type() + " " + aval(e) + " = " + L.bc("Aw[" + S(idx[{e->path, e->i, e->k}]) + "]") + ";");
+        em.line("const " + L.type() + " " + aval(e) + " = " +
+                L.bc("Aw[" + S(T.slot[idx[{e->path, e->i, e->k}]]) + "]") + ";");
       if (d1 <= d3) {  // scale-input
         std::vector<bool> used(d1, false);
         for (const AEntry* e : pe) used[e->i] = true;
@@ -591,24 +599,37 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
             em.line("const " + L.type() + " z" + S(i) + "_" + S(g) + " = " +
                     L.mul("s_" + S(g), "x" + S(i) + "_" + S(g)) + ";");
         }
-        for (const AEntry* e : pe)
+        // i outer, k inner: consecutive FMAs update different accumulators
+        std::vector<const AEntry*> byi(pe);
+        std::stable_sort(byi.begin(), byi.end(), [](const AEntry* a, const AEntry* b) {
+          return a->i != b->i ? a->i < b->i : a->k < b->k;
+        });
+        for (const AEntry* e : byi)
           for (int g = 0; g < G; ++g) {
             std::string acc = "q" + S(P.out_off + e->k) + "_" + S(g);
             em.line(acc + " = " + L.fma(aval(e), "z" + S(e->i) + "_" + S(g), acc) + ";");
           }
-      } else {  // scale-output
-        for (int k = 0; k < d3; ++k) {
-          std::vector<const AEntry*> row;
-          for (const AEntry* e : pe)
-            if (e->k == k) row.push_back(e);
-          if (row.empty()) continue;
+      } else {  // scale-output: t_k = sum_i A[i,k] x_i (i outer, k inner), then acc_k += s t_k
+        std::vector<const AEntry*> byi(pe);
+        std::stable_sort(byi.begin(), byi.end(), [](const AEntry* a, const AEntry* b) {
+          return a->i != b->i ? a->i < b->i : a->k < b->k;
+        });
+        std::vector<bool> started(d3, false);
+        for (const AEntry* e : byi)
           for (int g = 0; g < G; ++g) {
-            std::string t = "t" + S(k) + "_" + S(g);
-            em.line(L.type() + " " + t + " = " + L.mul(aval(row[0]), "x" + S(row[0]->i) + "_" + S(g)) + ";");
-            for (size_t m = 1; m < row.size(); ++m)
-              em.line(t + " = " + L.fma(aval(row[m]), "x" + S(row[m]->i) + "_" + S(g), t) + ";");
+            std::string tv = "t" + S(e->k) + "_" + S(g);
+            std::string xv = "x" + S(e->i) + "_" + S(g);
+            if (!started[e->k])
+              em.line(L.type() + " " + tv + " = " + L.mul(aval(e), xv) + ";");
+            else
+              em.line(tv + " = " + L.fma(aval(e), xv, tv) + ";");
+            if (g == G - 1) started[e->k] = true;
+          }
+        for (int k = 0; k < d3; ++k) {
+          if (!started[k]) continue;
+          for (int g = 0; g < G; ++g) {
             std::string acc = "q" + S(P.out_off + k) + "_" + S(g);
-            em.line(acc + " = " + L.fma("s_" + S(g), t, acc) + ";");
+            em.line(acc + " = " + L.fma("s_" + S(g), "t" + S(k) + "_" + S(g), acc) + ";");
           }
         }
       }

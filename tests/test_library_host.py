@@ -108,9 +108,28 @@ def test_generated_kernel_unrolls_every_coefficient():
     src = c.kernel_source()
     na = sum(int((np.abs(c.cg(p)) > 1e-12).any(axis=1).sum()) for p in range(c.num_paths))
     assert na == 541
-    dst = re.search(r"e3_adst\[\] = \{([^}]*)\}", src).group(1)
-    entries = sorted(int(v) for v in dst.replace("\n", "").split(",") if v.strip() not in ("", "-1"))
-    assert entries == list(range(na))
+    # emulate the generated phase-1 table on the host: slot q of the warp's A
+    # area must hold sum_j CG[i,j,k] Y_j of the (path, i, k) the layout names
+    layout = re.search(r"// A layout \(slot: path i k\):(.*)", src).group(1).split()
+    assert len(layout) == na
+    tab = re.search(r"e3_atab\[\] = \{(.*?)\};", src, re.S).group(1)
+    pairs = [(int(a), int(b)) for a, b in re.findall(r"\{(-?\d+), (\d+)\}", tab)]
+    Y = np.random.default_rng(1).normal(size=c.ny)
+    A = np.zeros(32 * ((na + 31) // 32))
+    base = 0
+    for r, nterms in enumerate(int(m) for m in re.findall(r"// round terms: (\d+)", src)):
+        for lane in range(32):
+            for term in range(nterms):
+                cb, j = pairs[base + term * 32 + lane]
+                A[32 * r + lane] += np.frombuffer(np.int32(cb).tobytes(), np.float32)[0] * Y[j]
+        base += nterms * 32
+    assert base == len(pairs)
+    for q, item in enumerate(layout):
+        p, i, k = (int(v) for v in item.split(":"))
+        W = c.cg(p)
+        l2 = c.paths[p].l2
+        expect = sum(W[i, j, k] * Y[l2 * l2 + j] for j in range(W.shape[1]))
+        assert abs(A[q] - expect) < 1e-6 * (1 + abs(expect)), (q, item)
     groups = info["channels_per_lane"] // 2
     assert src.count("fma2(") + src.count("mul2(") >= na * groups
     # per-lane products (contract_first = 0): every CG nonzero for every channel
