@@ -54,6 +54,8 @@ def parse_args():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--channels-per-lane", type=int, default=0)
     ap.add_argument("--block-threads", type=int, default=0)
+    ap.add_argument("--stages", type=int, default=-1)
+    ap.add_argument("--contract-first", type=int, default=-1)
     return ap.parse_args()
 
 
@@ -289,8 +291,10 @@ def run_ours(args):
     receivers = torch.from_numpy(g.receivers.astype(np.int32)).to(dev)
     conv = e3.Conv(spec.irreps_node, spec.irreps_sh, spec.irreps_out, g.avg_num_neighbors,
                    dtype=spec.dtype)
-    if args.channels_per_lane or args.block_threads:
-        conv.set_launch_config(args.channels_per_lane, args.block_threads)
+    if args.channels_per_lane or args.block_threads or args.stages != -1:
+        conv.set_launch_config(args.channels_per_lane, args.block_threads, args.stages)
+    if args.contract_first != -1:
+        conv.set_contract_first(args.contract_first)
     row_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
     perm = torch.empty(E, dtype=torch.int32, device=dev)
     ws = torch.empty(e3.csr_workspace_size(E, N), dtype=torch.uint8, device=dev)

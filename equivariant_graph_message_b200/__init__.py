@@ -137,7 +137,7 @@ class Conv:
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h:
+        if h and _destroy is not None:   # (module globals may be gone at interpreter exit)
             _destroy(h)
             self._h = None
 

@@ -4,6 +4,8 @@
 #include <nvrtc.h>
 
 #include <algorithm>
+#include <utility>
+#include <vector>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -84,7 +86,7 @@ bool has_device() {
   return n > 0;
 }
 
-int compile_variant(Plan& pl, int dtype) {
+int compile_once(Plan& pl, int dtype) {
   Variant& v = pl.var[dtype];
   v = Variant{};
   v.shape = choose_shape(pl, dtype);
@@ -114,6 +116,57 @@ int compile_variant(Plan& pl, int dtype) {
   if (std::regex_search(v.log, m, std::regex("([0-9]+) bytes spill stores")))
     v.local_bytes = std::stoi(m[1]);
   v.compiled = true;
+  return E3CONV_OK;
+}
+
+// Staged variant without a requested block size: a first compile gives the
+// register count R; the block size is then the one that keeps the most warps
+// resident per SM (228 KB of shared memory per SM with 1 KB reserved per
+// block, 64K registers, 2048 threads, 32 blocks), larger blocks on ties; the
+// launch bounds of the final compile keep R within budget.
+int blocks_per_sm(const Shape& s, int regs, int block) {
+  const int teams = block / (32 * s.team);
+  const int smem = teams * s.warp_smem + 1024;
+  const int r = (std::max(regs, 8) + 7) / 8 * 8;
+  const int by_smem = (228 * 1024) / smem;
+  const int by_regs = 65536 / (r * block);
+  const int by_threads = 2048 / block;
+  return std::min({by_smem, by_regs, by_threads, 32});
+}
+
+int compile_variant(Plan& pl, int dtype) {
+  pl.auto_block = 0;
+  int rc = compile_once(pl, dtype);
+  if (rc != E3CONV_OK) return rc;
+  Variant& v = pl.var[dtype];
+  if (v.shape.stages > 0 && pl.req_block == 0 && v.regs > 0) {
+    const int tt = 32 * v.shape.team;
+    const int first_block = v.shape.block;
+    const bool first_spills = v.local_bytes > 0;
+    std::vector<std::pair<int, int>> cand;  // (resident warps, block)
+    for (int k = 1; k <= 15 && k * tt <= 1024; ++k) {
+      if (k * v.shape.warp_smem > 227 * 1024) break;
+      cand.push_back({blocks_per_sm(v.shape, v.regs, k * tt) * k * v.shape.team, k * tt});
+    }
+    std::sort(cand.begin(), cand.end(), [](const std::pair<int, int>& a, const std::pair<int, int>& b) {
+      return a.first != b.first ? a.first > b.first : a.second > b.second;
+    });
+    bool done = false;
+    for (size_t c = 0; c < cand.size() && c < 4 && !done; ++c) {
+      if (cand[c].second == first_block && !first_spills) {
+        rc = compile_once(pl, dtype);  // restore the first compile
+        done = true;
+        break;
+      }
+      pl.auto_block = cand[c].second;
+      rc = compile_once(pl, dtype);
+      if (rc != E3CONV_OK) break;
+      done = v.local_bytes <= 0;  // keep only a spill-free choice
+    }
+    pl.auto_block = 0;
+    if (rc == E3CONV_OK && !done) rc = compile_once(pl, dtype);
+    if (rc != E3CONV_OK) return rc;
+  }
   if (pl.device >= 0) {
     Driver& d = driver();
     if (d.ModuleLoadData(&v.module, v.cubin.data()) != CUDA_SUCCESS)
@@ -126,7 +179,7 @@ int compile_variant(Plan& pl, int dtype) {
     v.regs = regs;
     v.local_bytes = local;
     if (v.shape.stages > 0) {
-      const int smem = v.shape.warp_smem * (v.shape.block / 32);
+      const int smem = v.shape.warp_smem * (v.shape.block / (32 * v.shape.team));
       if (d.FuncSetAttribute(v.fn, CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES, smem) !=
           CUDA_SUCCESS)
         return fail(E3CONV_ERR_CUDA, "cannot reserve the shared-memory ring");
@@ -442,9 +495,9 @@ int e3conv_forward(e3conv_plan h, const void* x, const void* Y, const void* s,
   long long blocks;
   unsigned smem = 0;
   if (sh.stages > 0) {
-    const long long wpb = sh.block / 32;
-    blocks = std::min<long long>(v.grid_blocks, (num_nodes + wpb - 1) / wpb);
-    smem = static_cast<unsigned>(sh.warp_smem * wpb);
+    const long long tpb = sh.block / (32 * sh.team);  // teams per block
+    blocks = std::min<long long>(v.grid_blocks, (num_nodes + tpb - 1) / tpb);
+    smem = static_cast<unsigned>(sh.warp_smem * tpb);
   } else {
     const long long items = num_nodes * sh.tiles;
     const long long warps = (items + sh.ipw - 1) / sh.ipw;

@@ -73,7 +73,78 @@ Shape choose_shape(const Plan& pl, int dtype) {
   Shape s;
   const int elem = dtype == E3CONV_F16 ? 2 : 4;
   const int vmax = 16 / elem;
-  int V = 1;
+  s.s_bytes = static_cast<int>(pl.paths.size()) * pl.C * elem;
+  s.x_bytes = pl.nx * pl.C * elem;
+  s.y_bytes = pl.ny * elem;
+  const bool bytes_ok = s.s_bytes % 16 == 0 && s.x_bytes % 16 == 0 && s.y_bytes % 16 == 0;
+
+  // Staged variant: a team of `team` warps covers the C channels of one
+  // receiver row, V channels per lane.  Preferred: one channel pair per lane
+  // (V = 2, team = C / 64), which keeps registers low and warps many.
+  int V = 0, team = 0;
+  if (pl.req_stages != 0 && bytes_ok && pl.C % 32 == 0) {
+    if (pl.req_V > 0) {
+      if (pl.C % (32 * pl.req_V) == 0 && pl.req_V <= vmax) {
+        V = pl.req_V;
+        team = pl.C / (32 * V);
+      }
+    } else if (pl.C / 32 <= vmax && pl.nout * (pl.C / 32) <= 128 && pl.C / 32 != 3) {
+      V = pl.C / 32;  // one warp per receiver row (measured fastest)
+      team = 1;
+    } else if (pl.C % 64 == 0) {
+      V = 2;          // channel pairs, teams of C/64 warps share the row
+      team = pl.C / 64;
+    } else {
+      V = 1;
+      team = pl.C / 32;
+    }
+    if (team > 8) V = team = 0;
+  }
+  if (V > 0) {
+    s.V = V;
+    s.team = team;
+    s.TL = 32;
+    s.tiles = 1;
+    s.ipw = 1;
+    s.s_off = 0;
+    s.x_off = align_up(s.s_bytes, 128);
+    s.y_off = s.x_off + align_up(s.x_bytes, 128);
+    s.stage_bytes = s.y_off + align_up(s.y_bytes, 128);
+    s.coop = pl.req_coop != 0 && (V == 1 || V % 2 == 0);
+    s.dup_a = s.coop && V == 2;
+    s.na = s.coop ? static_cast<int>(build_a_entries(pl).size()) : 0;
+    const int a_bytes = s.coop ? align_up((s.dup_a ? 8 : 4) * s.na, 16) : 0;
+    const int y_bytes = s.coop ? align_up(4 * pl.ny, 16) : 0;
+    const int S = pl.req_stages > 0 ? pl.req_stages : 2;
+    s.stages = S;
+    s.a_off = S * s.stage_bytes;
+    s.yf_off = s.a_off + a_bytes;
+    s.bar_off = align_up(s.yf_off + y_bytes, 8);
+    s.hdr_off = s.bar_off + 8 * S;
+    s.warp_smem = align_up(s.hdr_off + 16 * S, 128);
+    const int team_threads = 32 * team;
+    int block = pl.req_block > 0 ? pl.req_block : (pl.auto_block > 0 ? pl.auto_block : 4 * team_threads);
+    if (block % team_threads != 0 || block / team_threads > 15 ||
+        (block / team_threads) * s.warp_smem > 227 * 1024) {
+      if (pl.req_block > 0) {
+        s.stages = 0;  // the requested block does not fit the staged variant
+      } else {
+        int teams = std::max(1, std::min(15, 227 * 1024 / s.warp_smem));
+        block = teams * team_threads;
+        if (block > 1024) block = (1024 / team_threads) * team_threads;
+      }
+    }
+    if (s.stages > 0 && s.warp_smem > 227 * 1024) s.stages = 0;
+    s.block = block;
+    if (s.stages > 0) return s;
+    s = Shape{};
+    s.s_bytes = static_cast<int>(pl.paths.size()) * pl.C * elem;
+    s.x_bytes = pl.nx * pl.C * elem;
+    s.y_bytes = pl.ny * elem;
+  }
+
+  // Direct variant.
+  V = 1;
   if (pl.req_V > 0) {
     V = pl.req_V;
   } else {
@@ -83,9 +154,6 @@ Shape choose_shape(const Plan& pl, int dtype) {
         break;
       }
     }
-    // the staged variant wants one warp to cover a receiver's channels
-    if (pl.req_stages != 0 && pl.C % 32 == 0 && pl.C / 32 <= vmax && pl.nout * (pl.C / 32) <= 128)
-      V = pl.C / 32;
   }
   s.V = V;
   const int lanes = pl.C / V;
@@ -99,33 +167,6 @@ Shape choose_shape(const Plan& pl, int dtype) {
     s.ipw = 32 / lanes;
   }
   s.block = pl.req_block > 0 ? pl.req_block : 128;
-
-  // staged variant: one warp covers all C channels; all rows 16-byte multiples
-  s.s_bytes = static_cast<int>(pl.paths.size()) * pl.C * elem;
-  s.x_bytes = pl.nx * pl.C * elem;
-  s.y_bytes = pl.ny * elem;
-  const bool shape_ok = s.TL == 32 && s.tiles == 1 && 32 * V == pl.C;
-  const bool bytes_ok = s.s_bytes % 16 == 0 && s.x_bytes % 16 == 0 && s.y_bytes % 16 == 0;
-  if (shape_ok && bytes_ok && pl.req_stages != 0) {
-    s.s_off = 0;
-    s.x_off = align_up(s.s_bytes, 128);
-    s.y_off = s.x_off + align_up(s.x_bytes, 128);
-    s.stage_bytes = s.y_off + align_up(s.y_bytes, 128);
-    s.coop = pl.req_coop != 0 && (V == 1 || V % 2 == 0);
-    s.na = s.coop ? static_cast<int>(build_a_entries(pl).size()) : 0;
-    const int extra = s.coop ? align_up(4 * s.na, 16) + align_up(4 * pl.ny, 16) : 0;
-    int S = pl.req_stages > 0 ? pl.req_stages : (s.stage_bytes > 10240 ? 2 : 3);
-    const int warps = s.block / 32;
-    // keep one block within 227 KB of shared memory
-    while (S > 2 && warps * (S * s.stage_bytes + extra + 256) > 227 * 1024) --S;
-    s.stages = S;
-    s.a_off = S * s.stage_bytes;
-    s.yf_off = s.a_off + (s.coop ? align_up(4 * s.na, 16) : 0);
-    s.bar_off = align_up(s.yf_off + (s.coop ? 4 * pl.ny : 0), 8);
-    s.hdr_off = s.bar_off + 8 * S;
-    s.warp_smem = align_up(s.hdr_off + 16 * S, 128);
-    if (warps * s.warp_smem > 227 * 1024) s.stages = 0;
-  }
   return s;
 }
 
@@ -477,11 +518,11 @@ struct CoopTables {
   std::vector<int> slot;   // entry -> position in the warp's A area
 };
 
-// Phase 1 deals the entries to lanes in rounds of 32, longest first, and
-// stores entry number q of that order at A[q]: every round writes 32
-// consecutive words (no bank conflicts) and phase 2 reads A at the
-// compile-time position slot[n] of entry n.
-CoopTables coop_tables(const std::vector<AEntry>& ent) {
+// Phase 1 deals the entries to the team's RW = 32 * team lanes in rounds,
+// longest first, and stores entry number q of that order at A[q]: every
+// round writes RW consecutive slots (no bank conflicts) and phase 2 reads A
+// at the compile-time position slot[n] of entry n.
+CoopTables coop_tables(const std::vector<AEntry>& ent, int RW) {
   CoopTables T;
   std::vector<int> order(ent.size());
   for (size_t n = 0; n < ent.size(); ++n) order[n] = static_cast<int>(n);
@@ -490,7 +531,7 @@ CoopTables coop_tables(const std::vector<AEntry>& ent) {
   });
   T.slot.assign(ent.size(), -1);
   for (size_t q = 0; q < order.size(); ++q) T.slot[order[q]] = static_cast<int>(q);
-  T.rounds = static_cast<int>((ent.size() + 31) / 32);
+  T.rounds = static_cast<int>((ent.size() + RW - 1) / RW);
   std::ostringstream c, lay;
   c << "__device__ const int2 e3_atab[] = {\n";
   lay << "// A layout (slot: path i k):";
@@ -499,14 +540,14 @@ CoopTables coop_tables(const std::vector<AEntry>& ent) {
   lay << "\n";
   for (int r = 0; r < T.rounds; ++r) {
     int tr = 0;
-    for (int l = 0; l < 32; ++l) {
-      size_t q = static_cast<size_t>(r) * 32 + l;
+    for (int l = 0; l < RW; ++l) {
+      size_t q = static_cast<size_t>(r) * RW + l;
       if (q < order.size()) tr = std::max<int>(tr, static_cast<int>(ent[order[q]].terms.size()));
     }
     T.terms.push_back(tr);
     for (int t = 0; t < tr; ++t) {
-      for (int l = 0; l < 32; ++l) {
-        size_t q = static_cast<size_t>(r) * 32 + l;
+      for (int l = 0; l < RW; ++l) {
+        size_t q = static_cast<size_t>(r) * RW + l;
         double cv = 0.0;
         int j = 0;
         if (q < order.size() && t < static_cast<int>(ent[order[q]].terms.size())) {
@@ -526,37 +567,42 @@ CoopTables coop_tables(const std::vector<AEntry>& ent) {
   return T;
 }
 
-// Phase 1 + phase 2 for the edge staged at `stg`; y entries offset per path.
+// Phase 1 + phase 2 for the edge staged at `stg`.  `tl` is the lane's index
+// in its team, `team_sync()` a barrier of the team's warps.
 void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
                     const std::vector<AEntry>& ent, const CoopTables& T) {
   const bool f16 = dtype == E3CONV_F16;
   const std::string Ty = f16 ? "unsigned short" : "float";
   const Lanes L{sh.V};
-  em.line("float* Aw = reinterpret_cast<float*>(wbase + " + S(sh.a_off) + ");");
-  em.line("float* yf = reinterpret_cast<float*>(wbase + " + S(sh.yf_off) + ");");
-  em.line("if (lane < " + S(pl.ny) + ") yf[lane] = " + (f16 ? "h2f" : "") + "(reinterpret_cast<const " +
-          Ty + "*>(stg + " + S(sh.y_off) + ")[lane]);");
-  em.line("__syncwarp();");
+  const int RW = 32 * sh.team;
+  if (sh.dup_a)
+    em.line("unsigned long long* Aw = reinterpret_cast<unsigned long long*>(tbase + " + S(sh.a_off) + ");");
+  else
+    em.line("float* Aw = reinterpret_cast<float*>(tbase + " + S(sh.a_off) + ");");
+  em.line("float* yf = reinterpret_cast<float*>(tbase + " + S(sh.yf_off) + ");");
+  em.line("if (tl < " + S(pl.ny) + ") yf[tl] = " + (f16 ? "h2f" : "") + "(reinterpret_cast<const " +
+          Ty + "*>(stg + " + S(sh.y_off) + ")[tl]);");
+  em.line("team_sync();");
   int base = 0;
+  const int na = static_cast<int>(ent.size());
   for (int r = 0; r < T.rounds; ++r) {
     em.line("{  // round terms: " + S(T.terms[r]));
     em.ind++;
-    for (int t = 0; t < T.terms[r]; ++t) {
-      em.line("const int2 k" + S(t) + " = __ldg(&e3_atab[" + S(base + t * 32) + " + lane]);");
-    }
+    for (int t = 0; t < T.terms[r]; ++t)
+      em.line("const int2 k" + S(t) + " = __ldg(&e3_atab[" + S(base + t * RW) + " + tl]);");
     std::string v = "__int_as_float(k0.x) * yf[k0.y]";
     for (int t = 1; t < T.terms[r]; ++t)
       v = "fmaf(__int_as_float(k" + S(t) + ".x), yf[k" + S(t) + ".y], " + v + ")";
-    const int na = static_cast<int>(ent.size());
-    if ((r + 1) * 32 <= na)
-      em.line("Aw[" + S(r * 32) + " + lane] = " + v + ";");
+    if (sh.dup_a) v = "bc(" + v + ")";
+    if ((r + 1) * RW <= na)
+      em.line("Aw[" + S(r * RW) + " + tl] = " + v + ";");
     else
-      em.line("if (lane < " + S(na - r * 32) + ") Aw[" + S(r * 32) + " + lane] = " + v + ";");
+      em.line("if (tl < " + S(na - r * RW) + ") Aw[" + S(r * RW) + " + tl] = " + v + ";");
     em.ind--;
     em.line("}");
-    base += T.terms[r] * 32;
+    base += T.terms[r] * RW;
   }
-  em.line("__syncwarp();");
+  em.line("team_sync();");
   em.line("const " + Ty + "* xs = reinterpret_cast<const " + Ty + "*>(stg + " + S(sh.x_off) + ") + u0;");
   em.line("const " + Ty + "* ss = reinterpret_cast<const " + Ty + "*>(stg + " + S(sh.s_off) + ") + u0;");
   // entry index of (path, i, k)
@@ -587,9 +633,10 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
       auto aval = [&](const AEntry* e) {
         return "A" + S(idx[{e->path, e->i, e->k}]);
       };
-      for (const AEntry* e : pe)
-        em.line("const " + L.type() + " " + aval(e) + " = " +
-                L.bc("Aw[" + S(T.slot[idx[{e->path, e->i, e->k}]]) + "]") + ";");
+      for (const AEntry* e : pe) {
+        const std::string ld = "Aw[" + S(T.slot[idx[{e->path, e->i, e->k}]]) + "]";
+        em.line("const " + L.type() + " " + aval(e) + " = " + (sh.dup_a ? ld : L.bc(ld)) + ";");
+      }
       if (d1 <= d3) {  // scale-input
         std::vector<bool> used(d1, false);
         for (const AEntry* e : pe) used[e->i] = true;
@@ -677,24 +724,27 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   const int NS = sh.stages;
   const bool f16 = dtype == E3CONV_F16;
   const std::string T = f16 ? "unsigned short" : "float";
-  const int warps = sh.block / 32;
+  const int TW = sh.team;                  // warps per team
+  const int teams = sh.block / (32 * TW);  // teams per block
   const long long s_row = static_cast<long long>(pl.paths.size()) * pl.C;
+  const long long o_row = static_cast<long long>(pl.nout) * pl.C;
   em.line("// generated by libe3conv: fused equivariant convolution forward (staged ring)");
   em.line("// C=" + S(pl.C) + " nx=" + S(pl.nx) + " ny=" + S(pl.ny) + " nout=" + S(pl.nout) +
           " paths=" + S(pl.paths.size()) + " dtype=" + (f16 ? "f16" : "f32") + " V=" + S(V) +
-          " stages=" + S(NS) + " stage_bytes=" + S(sh.stage_bytes) + " warps/block=" + S(warps));
+          " team=" + S(TW) + " teams/block=" + S(teams) + " stages=" + S(NS) +
+          " stage_bytes=" + S(sh.stage_bytes) + " contract_first=" + S(sh.coop ? 1 : 0));
   emit_prelude(em);
   std::vector<AEntry> ent;
   CoopTables tabs;
   const Lanes L{V};
+  em.line("__device__ __forceinline__ unsigned long long pk(float lo, float hi) { unsigned long long r; asm(\"mov.b64 %0, {%1, %2};\" : \"=l\"(r) : \"f\"(lo), \"f\"(hi)); return r; }");
+  em.line("__device__ __forceinline__ unsigned long long bc(float a) { return pk(a, a); }");
+  em.line("__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) { unsigned long long d; asm(\"fma.rn.f32x2 %0, %1, %2, %3;\" : \"=l\"(d) : \"l\"(a), \"l\"(b), \"l\"(c)); return d; }");
+  em.line("__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) { unsigned long long d; asm(\"mul.rn.f32x2 %0, %1, %2;\" : \"=l\"(d) : \"l\"(a), \"l\"(b)); return d; }");
   if (sh.coop) {
     ent = build_a_entries(pl);
-    tabs = coop_tables(ent);
+    tabs = coop_tables(ent, 32 * TW);
     em.o << tabs.source;
-    em.line("__device__ __forceinline__ unsigned long long pk(float lo, float hi) { unsigned long long r; asm(\"mov.b64 %0, {%1, %2};\" : \"=l\"(r) : \"f\"(lo), \"f\"(hi)); return r; }");
-    em.line("__device__ __forceinline__ unsigned long long bc(float a) { return pk(a, a); }");
-    em.line("__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) { unsigned long long d; asm(\"fma.rn.f32x2 %0, %1, %2, %3;\" : \"=l\"(d) : \"l\"(a), \"l\"(b), \"l\"(c)); return d; }");
-    em.line("__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) { unsigned long long d; asm(\"mul.rn.f32x2 %0, %1, %2;\" : \"=l\"(d) : \"l\"(a), \"l\"(b)); return d; }");
   }
   em.line("#define E3_SPIN_LIMIT (1u << 22)");
   em.line("__device__ __forceinline__ unsigned int smem_u32(const void* p) { return static_cast<unsigned int>(__cvta_generic_to_shared(p)); }");
@@ -714,21 +764,32 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.ind++;
   em.line("extern __shared__ __align__(128) unsigned char smem[];");
   em.line("const int lane = threadIdx.x & 31;");
-  em.line("unsigned char* wbase = smem + (threadIdx.x >> 5) * " + S(sh.warp_smem) + ";");
-  em.line("unsigned long long* bars = reinterpret_cast<unsigned long long*>(wbase + " +
-          S(sh.bar_off) + ");");
-  em.line("int* hdr = reinterpret_cast<int*>(wbase + " + S(sh.hdr_off) + ");  // per stage: sender, receiver, last");
-  em.line("if (lane == 0) {");
+  em.line("const int warp = threadIdx.x >> 5;");
+  em.line("const int team = warp / " + S(TW) + ";       // team in this block");
+  em.line("const int tw = warp - team * " + S(TW) + ";  // warp in team");
+  em.line("const int tl = tw * 32 + lane;               // lane in team");
+  if (TW > 1) {
+    em.line("const unsigned int bar_id = 1u + (unsigned int)team;");
+    em.line("auto team_sync = [&]() { asm volatile(\"bar.sync %0, " + S(32 * TW) + ";\" :: \"r\"(bar_id) : \"memory\"); };");
+    em.line("auto team_all = [&](bool ok) { unsigned int r; asm volatile(\"{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.and.pred q, %2, " + S(32 * TW) + ", p; selp.u32 %0, 1, 0, q; }\" : \"=r\"(r) : \"r\"((unsigned int)ok), \"r\"(bar_id) : \"memory\"); return r != 0u; };");
+  } else {
+    em.line("auto team_sync = [&]() { __syncwarp(); };");
+    em.line("auto team_all = [&](bool ok) { return __all_sync(0xffffffffu, ok) != 0; };");
+  }
+  em.line("unsigned char* tbase = smem + team * " + S(sh.warp_smem) + ";");
+  em.line("unsigned long long* bars = reinterpret_cast<unsigned long long*>(tbase + " + S(sh.bar_off) + ");");
+  em.line("int* hdr = reinterpret_cast<int*>(tbase + " + S(sh.hdr_off) + ");  // per stage: sender, receiver, last");
+  em.line("const bool issuer = tw == 0 && lane == 0;  // the lane that issues the team's copies");
+  em.line("if (issuer) {");
   em.line("  for (int k = 0; k < " + S(NS) + "; ++k) bar_init(bars + k);");
   em.line("  asm volatile(\"fence.mbarrier_init.release.cluster;\" ::: \"memory\");");
   em.line("}");
-  em.line("__syncwarp();");
+  em.line("team_sync();");
   em.line("const unsigned long long pol_stream = policy_evict_first();");
   em.line("const unsigned long long pol_keep = policy_evict_last();");
-  em.line("const long long W = (long long)gridDim.x * " + S(warps) + ";");
-  em.line("const int u0 = lane * " + S(V) + ";");
-  // producer state (warp-uniform)
-  em.line("long long pb = (long long)blockIdx.x * " + S(warps) + " + (threadIdx.x >> 5) - W;  // producer receiver");
+  em.line("const long long W = (long long)gridDim.x * " + S(teams) + ";  // teams in the grid");
+  em.line("const int u0 = tl * " + S(V) + ";  // first channel of this lane");
+  em.line("long long pb = (long long)blockIdx.x * " + S(teams) + " + team - W;  // producer receiver");
   em.line("int pe = 0, pe1 = 0;      // producer edge cursor within row pb");
   em.line("int pwin = -1, psw = 0;   // sender window base (edge index) and this lane's sender");
   em.line("bool pdone = false;");
@@ -739,17 +800,18 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   } else {
     emit_acc_decl(em, pl, V);
   }
-  // produce lambda as a macro-like block: emitted inline via a device lambda
+  // Every warp of the team walks the same rows (same decisions); only the
+  // issuer lane writes the stage header and issues the bulk copies.
   em.line("auto produce = [&]() {");
   em.ind++;
   em.line("while (!pdone && pe >= pe1) {");
   em.line("  pb += W;");
   em.line("  if (pb >= num_nodes) { pdone = true; break; }");
   em.line("  int r0 = row_ptr[pb], r1 = row_ptr[pb + 1];");
-  em.line("  if (r0 < 0 || r1 < r0 || r1 > num_edges) { if (lane == 0) atomicOr(status, 1u); r1 = r0; }");
+  em.line("  if (r0 < 0 || r1 < r0 || r1 > num_edges) { if (issuer) atomicOr(status, 1u); r1 = r0; }");
   em.line("  pe = r0; pe1 = r1; pwin = -1;");
   em.line("  if (r0 == r1) {  // empty row: zeros");
-  em.line("    float* zrow = out + pb * " + S(static_cast<long long>(pl.nout) * pl.C) + " + u0;");
+  em.line("    float* zrow = out + pb * " + S(o_row) + " + u0;");
   em.ind += 2;
   emit_store(em, pl, V, "zrow", true, false);
   em.ind -= 2;
@@ -763,8 +825,8 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("const int a = __shfl_sync(0xffffffffu, psw, pe - pwin);");
   em.line("const bool valid = (unsigned int)a < (unsigned int)num_nodes;");
   em.line("const unsigned int st = ppos % " + S(NS) + ";");
-  em.line("if (lane == 0) {");
-  em.line("  unsigned char* stg = wbase + st * " + S(sh.stage_bytes) + ";");
+  em.line("if (issuer) {");
+  em.line("  unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
   em.line("  hdr[4 * st] = valid ? a : -1;");
   em.line("  hdr[4 * st + 1] = (int)pb;");
   em.line("  hdr[4 * st + 2] = (pe + 1 == pe1) ? 1 : 0;");
@@ -784,17 +846,20 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.ind--;
   em.line("};");
   em.line("for (int k = 0; k < " + S(NS) + "; ++k) produce();");
-  em.line("__syncwarp();");
+  em.line("team_sync();");
   em.line("#pragma unroll 1");
   em.line("while (cpos != ppos) {");
   em.ind++;
   em.line("const unsigned int st = cpos % " + S(NS) + ";");
-  em.line("if (!bar_wait(bars + st, (cpos / " + S(NS) + ") & 1u)) {");
-  em.line("  if (lane == 0) atomicOr(status, 4u);");
-  em.line("  for (unsigned int q = cpos; q != ppos; ++q) bar_wait(bars + q % " + S(NS) + ", (q / " + S(NS) + ") & 1u);");
+  em.line("if (!team_all(bar_wait(bars + st, (cpos / " + S(NS) + ") & 1u))) {");
+  em.line("  // bounded wait ran out: flag it, let the issuer drain its copies (bounded), stop");
+  em.line("  if (issuer) {");
+  em.line("    atomicOr(status, 4u);");
+  em.line("    for (unsigned int q = cpos; q != ppos; ++q) bar_wait(bars + q % " + S(NS) + ", (q / " + S(NS) + ") & 1u);");
+  em.line("  }");
   em.line("  return;");
   em.line("}");
-  em.line("const unsigned char* stg = wbase + st * " + S(sh.stage_bytes) + ";");
+  em.line("const unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
   em.line("const int a = hdr[4 * st];");
   em.line("const long long b = hdr[4 * st + 1];");
   em.line("const int last = hdr[4 * st + 2];");
@@ -810,19 +875,19 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
     emit_edge_body(em, pl, dtype, V, "lds", "xs", "ss");
   }
   em.ind--;
-  em.line("} else if (lane == 0) {");
+  em.line("} else if (issuer) {");
   em.line("  atomicOr(status, 2u);");
   em.line("}");
   em.line("if (last) {");
   em.ind++;
-  em.line("float* orow = out + b * " + S(static_cast<long long>(pl.nout) * pl.C) + " + u0;");
+  em.line("float* orow = out + b * " + S(o_row) + " + u0;");
   if (sh.coop)
     emit_group_store(em, pl, L, "orow");
   else
     emit_store(em, pl, V, "orow", false, true);
   em.ind--;
   em.line("}");
-  em.line("__syncwarp();");
+  em.line("team_sync();  // stage and A area free for reuse");
   em.line("++cpos;");
   em.line("produce();");
   em.ind--;

@@ -46,14 +46,16 @@ struct Shape {
   int s_bytes = 0, x_bytes = 0, y_bytes = 0;  // row sizes staged per edge
   int s_off = 0, x_off = 0, y_off = 0;        // offsets inside one stage
   int stage_bytes = 0;                        // one stage, 128-byte aligned
-  int warp_smem = 0;                          // stages + barriers + headers of one warp
-  int bar_off = 0, hdr_off = 0;               // offsets inside a warp's region
+  int team = 1;                               // warps that share one receiver row (32*V*team = C)
+  int warp_smem = 0;                          // shared memory of one team (ring, A, barriers)
+  int bar_off = 0, hdr_off = 0;               // offsets inside a team's region
   // Cooperative contraction (staged variant): per edge the warp first forms
   // A_p[i,k] = sum_j CG_p[i,j,k] Y_j in shared memory, then every lane applies
   // it to its channels with packed float32x2 FMAs.
   bool coop = false;
+  bool dup_a = false;                         // A stored as (a, a) pairs (one channel pair per lane)
   int na = 0;                                 // number of A entries (all paths)
-  int a_off = 0, yf_off = 0;                  // A entries and float32 Y inside a warp's region
+  int a_off = 0, yf_off = 0;                  // A entries and float32 Y inside a team's region
 };
 
 // One entry A_p[i,k] of the per-edge contraction of CG with Y.
@@ -83,6 +85,7 @@ struct Plan {
   int norm = 0;
   int dtype = E3CONV_F32;
   int req_V = 0, req_block = 0, req_stages = -1;  // -1: automatic
+  int auto_block = 0;                              // block chosen after a first compile (0: none)
   int req_coop = -1;                               // -1: automatic, 0: off, 1: on
   int device = -1;                 // -1: host-only plan
   CUcontext ctx = nullptr;

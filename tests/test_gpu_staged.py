@@ -144,3 +144,25 @@ def test_staged_matches_direct_bitwise_order_free(cuda_device):
     ref = oracle_out(irreps, x, Y, s, send, recv, n, 30.0)
     assert column_scaled_error(ga, ref) <= 5e-3 and column_scaled_error(gb, ref) <= 5e-3
     np.testing.assert_allclose(ga, gb, rtol=1e-5, atol=1e-5 * np.abs(ref).max())
+
+
+@pytest.mark.parametrize("V,block,stages", [(2, 64, 2), (2, 128, 3), (2, 192, 2), (2, 448, 2),
+                                            (4, 32, 2), (4, 256, 2), (1, 128, 2)])
+@pytest.mark.parametrize("contract_first", [0, 1])
+def test_staged_team_shapes(cuda_device, V, block, stages, contract_first):
+    # C = 128: V=2 -> teams of 2 warps sharing one ring; V=4 -> one warp; V=1 -> 4 warps
+    irreps = IRREPS[128]
+    rng = np.random.default_rng(V * 1000 + block + stages)
+    n, e = 400, 7000
+    send, recv = _graph(rng, n, e, empty_frac=0.1)
+    pl, x, Y, s = _inputs(rng, irreps, n, e, "f16")
+    conv = e3.Conv(*irreps, 17.0, dtype="f16")
+    conv.set_contract_first(contract_first)
+    conv.set_launch_config(V, block, stages)
+    info = conv.kernel_info()
+    assert info["stages"] == stages and info["block_threads"] == block
+    assert info["channels_per_lane"] == V
+    gpu = run_gpu(conv, x, Y, s, send, recv, n)
+    ref = oracle_out(irreps, x, Y, s, send, recv, n, 17.0)
+    assert column_scaled_error(gpu, ref) <= 5e-3
+    assert np.all(gpu[np.setdiff1d(np.arange(n), recv)] == 0)

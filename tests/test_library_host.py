@@ -115,14 +115,15 @@ def test_generated_kernel_unrolls_every_coefficient():
     tab = re.search(r"e3_atab\[\] = \{(.*?)\};", src, re.S).group(1)
     pairs = [(int(a), int(b)) for a, b in re.findall(r"\{(-?\d+), (\d+)\}", tab)]
     Y = np.random.default_rng(1).normal(size=c.ny)
-    A = np.zeros(32 * ((na + 31) // 32))
+    rw = 32 * int(re.search(r" team=(\d+)", src).group(1))   # lanes of one team
+    A = np.zeros(rw * ((na + rw - 1) // rw))
     base = 0
     for r, nterms in enumerate(int(m) for m in re.findall(r"// round terms: (\d+)", src)):
-        for lane in range(32):
+        for lane in range(rw):
             for term in range(nterms):
-                cb, j = pairs[base + term * 32 + lane]
-                A[32 * r + lane] += np.frombuffer(np.int32(cb).tobytes(), np.float32)[0] * Y[j]
-        base += nterms * 32
+                cb, j = pairs[base + term * rw + lane]
+                A[rw * r + lane] += np.frombuffer(np.int32(cb).tobytes(), np.float32)[0] * Y[j]
+        base += nterms * rw
     assert base == len(pairs)
     for q, item in enumerate(layout):
         p, i, k = (int(v) for v in item.split(":"))
