@@ -188,12 +188,20 @@ def oracle_sample_rate(spec, graph, rows, x_rows_fn, Y_fn, s_fn, threads=0):
 
 
 def calibrated_rows(spec, graph, x_rows_fn, Y_fn, s_fn, target_s, seed=2024):
+    """Seeded receivers whose oracle run takes about target_s seconds (two probes: a
+    tiny one, then one of ~1/8 of the target, so thread start-up does not skew the rate)."""
     import numpy as np
     order = np.random.default_rng(seed).permutation(graph.num_nodes)
-    probe = order[: min(16, graph.num_nodes)]
-    rate, ne, dt = oracle_sample_rate(spec, graph, probe, x_rows_fn, Y_fn, s_fn)
-    per_row = max(ne / len(probe), 1e-9)
-    want = int(max(1, min(graph.num_nodes, rate * target_s / per_row)))
+    n = min(16, graph.num_nodes)
+    for frac in (None, 0.125):
+        probe = order[:n]
+        rate, ne, dt = oracle_sample_rate(spec, graph, probe, x_rows_fn, Y_fn, s_fn)
+        per_row = max(ne / len(probe), 1e-9)
+        want = int(max(1, min(graph.num_nodes, rate * target_s / per_row)))
+        if frac is None:
+            n = int(max(n, min(graph.num_nodes, want * 0.125)))
+            if n >= graph.num_nodes:
+                break
     return np.sort(order[:want])
 
 
