@@ -221,6 +221,18 @@ def device_inputs_fns(x_d, Y_d, s_d):
 
 # ---------------------------------------------------------------------------
 
+def reduce_over_ranks(times_ms, edges, world, device=None):
+    """Max of each time and sum of edges over the ranks (identity for one rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(times_ms), dtype=torch.float64, device=device)
+    e = torch.tensor([float(edges)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(e, op=dist.ReduceOp.SUM)
+    return t.tolist(), e.item()
+
+
 def spec_for_rank(name, rank):
     from dataclasses import replace
 
@@ -345,13 +357,7 @@ def run_ours(args):
     clk = clocks.stop()
     ms = t0.elapsed_time(t1)
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd)
-    ms_t = torch.tensor([ms, fwd_ms], dtype=torch.float64, device=dev)
-    e_t = torch.tensor([float(E)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-        dist.all_reduce(e_t, op=dist.ReduceOp.SUM)
-    ms, fwd_ms = ms_t.tolist()
-    total_edges = e_t.item()
+    (ms, fwd_ms), total_edges = reduce_over_ranks([ms, fwd_ms], E, world, dev)
     ms_per_step = ms / args.steps
     value = total_edges / (ms_per_step / 1000.0)
 
@@ -465,14 +471,10 @@ def run_e2e(args, conv, spec, g, x, Y, s, senders, receivers, row_ptr, perm, ws,
         step()
     b.record()
     torch.cuda.synchronize()
-    ms = torch.tensor([a.elapsed_time(b) / steps], dtype=torch.float64, device=dev)
-    e_t = torch.tensor([float(E)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-        dist.all_reduce(e_t, op=dist.ReduceOp.SUM)
+    (ms,), total = reduce_over_ranks([a.elapsed_time(b) / steps], E, world, dev)
     del host, out_h
-    return {"value": e_t.item() / (ms.item() / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms.item()}
+    return {"value": total / (ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms}
 
 
 def main():

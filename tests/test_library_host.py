@@ -180,3 +180,17 @@ def test_forward_argument_validation_precedes_device():
     assert e3._forward(c._h, ctypes.c_void_p(18), None, None, None, ctypes.c_void_p(16), 3, 0,
                        ctypes.c_void_p(16), None) == 1
     assert e3._build_csr(None, -1, 3, None, None, None, 0, None) == 1
+
+
+def test_size_limits_rejected_on_host():
+    # indices are int32: sizes of 2^31 and above are refused before any launch
+    c = e3.Conv("1x0e", "1x0e", "1x0e", 1.0)
+    p16 = ctypes.c_void_p(16)
+    assert e3._forward(c._h, p16, p16, p16, p16, p16, 1, 1 << 31, p16, None) == 1
+    assert e3._forward(c._h, p16, p16, p16, p16, p16, 1 << 31, 1, p16, None) == 1
+    n = ctypes.c_size_t()
+    assert e3._csr_ws(1 << 31, 10, ctypes.byref(n)) == 1
+    assert e3._csr_ws(10, (1 << 31) - 1, ctypes.byref(n)) == 1
+    assert e3._csr_ws((1 << 31) - 1, (1 << 31) - 2, ctypes.byref(n)) == 0
+    cnt = ctypes.c_int()
+    assert e3._csr_count((1 << 31) - 1, 100000, ctypes.byref(cnt)) == 0 and cnt.value > 0
