@@ -71,7 +71,11 @@ def peaks():
         sm_max = float(d.get("sm_max_mhz", sm_max))
         src = "measured"
     fp32_tflops = SMS * FP32_LANES_PER_SM * 2 * sm_max * 1e6 / 1e12
-    return {"hbm_gbs": hbm, "fp32_tflops": fp32_tflops, "sm_max_mhz": sm_max, "source": src}
+    f16 = 1590.0
+    if src == "measured":
+        f16 = float(json.load(open(p)).get("bf16_tflops", f16))
+    return {"hbm_gbs": hbm, "fp32_tflops": fp32_tflops, "f16_tflops": f16, "sm_max_mhz": sm_max,
+            "source": src}
 
 
 def algorithmic(conv, N, E, in_bytes):
@@ -364,24 +368,42 @@ def run_ours(args):
     pk = peaks()
     in_bytes = 2 if spec.dtype == "f16" else 4
     nbytes, flops, nnz, mix = algorithmic(conv, N, E, in_bytes)
-    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
-    t_alu = flops / (pk["fp32_tflops"] * 1e12)
     traffic, traffic_src = traffic_for(spec.name if args.nodes is None else None, conv, E)
-    if t_alu >= t_hbm:
-        achieved = flops / (fwd_ms / 1000.0) / 1e12
-        roof = {"bound": "alu", "achieved": achieved, "peak": pk["fp32_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / pk["fp32_tflops"],
-                "traffic": traffic,
-                "peak_source": f"derived: {SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 x "
-                               f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})"}
+    sec = fwd_ms / 1000.0
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    if info.get("tensor_cores"):
+        # tensor-core variant: the CG x Y contraction runs as two tcgen05 MMAs per edge
+        # (M = C, N = path outputs padded to 16, K = 16); only the s-scaling stays on FP32.
+        ncols = -(-mix // 16) * 16
+        tc_flops = 2 * 2 * E * conv.C * ncols * 16
+        fp32_flops = 2 * E * conv.C * mix
+        times = {"hbm": t_hbm, "tensor": tc_flops / (pk["f16_tflops"] * 1e12),
+                 "alu": fp32_flops / (pk["fp32_tflops"] * 1e12)}
     else:
-        achieved = nbytes / (fwd_ms / 1000.0) / 1e9
+        tc_flops, fp32_flops = 0, flops
+        times = {"hbm": t_hbm, "alu": flops / (pk["fp32_tflops"] * 1e12)}
+    bound = max(times, key=times.get)
+    if bound == "hbm":
+        achieved = nbytes / sec / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
                 "peak_source": f"hbm_gbs ({pk['source']})"}
+    elif bound == "tensor":
+        achieved = tc_flops / sec / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["f16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / pk["f16_tflops"], "traffic": traffic,
+                "peak_source": f"bf16_tflops ({pk['source']}); f16 dense = bf16 dense"}
+    else:
+        achieved = fp32_flops / sec / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": pk["fp32_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / pk["fp32_tflops"], "traffic": traffic,
+                "peak_source": f"derived: {SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 x "
+                               f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})"}
     roof.update({"kernel": "e3conv_fwd", "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
-                 "forward_ms": fwd_ms, "hbm_frac": nbytes / (fwd_ms / 1000.0) / 1e9 / pk["hbm_gbs"],
-                 "alu_frac": flops / (fwd_ms / 1000.0) / 1e12 / pk["fp32_tflops"],
+                 "fp32_flops": fp32_flops, "tensor_flops": tc_flops, "forward_ms": fwd_ms,
+                 "hbm_frac": nbytes / sec / 1e9 / pk["hbm_gbs"],
+                 "fp32_equivalent_tflops": flops / sec / 1e12,
+                 "roofline_times_ms": {k: 1000 * v for k, v in times.items()},
                  "traffic_source": traffic_src})
 
     cpu = None

@@ -51,9 +51,10 @@ _path = _sig("e3conv_path", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 7))
 _num_outputs = _sig("e3conv_num_outputs", ctypes.c_int, _vp, _c_int_p)
 _output_irrep = _sig("e3conv_output_irrep", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 3))
 _cg = _sig("e3conv_cg", ctypes.c_int, _vp, ctypes.c_int, ctypes.POINTER(ctypes.c_double))
-_kernel_info = _sig("e3conv_kernel_info", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 7))
+_kernel_info = _sig("e3conv_kernel_info", ctypes.c_int, _vp, ctypes.c_int, *([_c_int_p] * 8))
 _set_option = _sig("e3conv_set_option", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_int)
 OPT_CONTRACT_FIRST = 1
+OPT_TENSOR_CORES = 2
 _kernel_source = _sig("e3conv_kernel_source", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_char_p,
                       ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t))
 _forward = _sig("e3conv_forward", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp,
@@ -184,12 +185,15 @@ class Conv:
     def set_contract_first(self, value: int = -1):
         _ok(_set_option(self._h, OPT_CONTRACT_FIRST, value), "e3conv_set_option")
 
+    def set_tensor_cores(self, value: int = -1):
+        _ok(_set_option(self._h, OPT_TENSOR_CORES, value), "e3conv_set_option")
+
     def kernel_info(self, dtype: str | None = None) -> dict:
-        v = [ctypes.c_int() for _ in range(7)]
+        v = [ctypes.c_int() for _ in range(8)]
         _ok(_kernel_info(self._h, {"f32": F32, "f16": F16}[dtype or self.dtype],
                          *[ctypes.byref(x) for x in v]), "e3conv_kernel_info")
         keys = ["channels_per_lane", "lanes_per_tile", "block_threads", "stages", "contract_first",
-                "registers", "local_bytes"]
+                "tensor_cores", "registers", "local_bytes"]
         return dict(zip(keys, (x.value for x in v)))
 
     def kernel_source(self, dtype: str | None = None) -> str:

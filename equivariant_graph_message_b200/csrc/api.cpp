@@ -50,6 +50,10 @@ struct Driver {
   CUresult (*CtxGetCurrent)(CUcontext*) = nullptr;
   CUresult (*FuncSetAttribute)(CUfunction, CUfunction_attribute, int) = nullptr;
   CUresult (*OccupancyMaxActiveBlocksPerMultiprocessor)(int*, CUfunction, int, size_t) = nullptr;
+  CUresult (*TensorMapEncodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill) = nullptr;
   bool ok = false;
 };
 
@@ -70,7 +74,8 @@ Driver& driver() {
            get("cuCtxGetCurrent", reinterpret_cast<void**>(&d.CtxGetCurrent)) &&
            get("cuFuncSetAttribute", reinterpret_cast<void**>(&d.FuncSetAttribute)) &&
            get("cuOccupancyMaxActiveBlocksPerMultiprocessor",
-               reinterpret_cast<void**>(&d.OccupancyMaxActiveBlocksPerMultiprocessor));
+               reinterpret_cast<void**>(&d.OccupancyMaxActiveBlocksPerMultiprocessor)) &&
+           get("cuTensorMapEncodeTiled", reinterpret_cast<void**>(&d.TensorMapEncodeTiled));
     cudaGetLastError();
   });
   return d;
@@ -139,7 +144,7 @@ int compile_variant(Plan& pl, int dtype) {
   int rc = compile_once(pl, dtype);
   if (rc != E3CONV_OK) return rc;
   Variant& v = pl.var[dtype];
-  if (v.shape.stages > 0 && pl.req_block == 0 && v.regs > 0) {
+  if (v.shape.stages > 0 && !v.shape.tc && pl.req_block == 0 && v.regs > 0) {
     const int tt = 32 * v.shape.team;
     const int first_block = v.shape.block;
     const bool first_spills = v.local_bytes > 0;
@@ -179,7 +184,8 @@ int compile_variant(Plan& pl, int dtype) {
     v.regs = regs;
     v.local_bytes = local;
     if (v.shape.stages > 0) {
-      const int smem = v.shape.warp_smem * (v.shape.block / (32 * v.shape.team));
+      const int smem = v.shape.tc ? v.shape.smem_request
+                                  : v.shape.warp_smem * (v.shape.block / (32 * v.shape.team));
       if (d.FuncSetAttribute(v.fn, CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES, smem) !=
           CUDA_SUCCESS)
         return fail(E3CONV_ERR_CUDA, "cannot reserve the shared-memory ring");
@@ -379,10 +385,13 @@ int e3conv_set_launch_config(e3conv_plan h, int channels_per_lane, int block_thr
 int e3conv_set_option(e3conv_plan h, int option, int value) {
   if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
   Plan& pl = h->p;
-  if (option != E3CONV_OPT_CONTRACT_FIRST)
+  if (option != E3CONV_OPT_CONTRACT_FIRST && option != E3CONV_OPT_TENSOR_CORES)
     return fail(E3CONV_ERR_UNSUPPORTED, "unknown option");
   if (value < -1 || value > 1) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1, 0 or 1");
-  pl.req_coop = value;
+  if (option == E3CONV_OPT_CONTRACT_FIRST)
+    pl.req_coop = value;
+  else
+    pl.req_tc = value;
   DeviceGuard g(pl.device);
   const int other = pl.dtype == E3CONV_F32 ? E3CONV_F16 : E3CONV_F32;
   release_variant(pl.var[other]);
@@ -445,7 +454,7 @@ int e3conv_cg(e3conv_plan h, int p, double* dense_out) {
 }
 
 int e3conv_kernel_info(e3conv_plan h, int dtype, int* V, int* TL, int* block, int* stages,
-                       int* contract_first, int* regs, int* local_bytes) {
+                       int* contract_first, int* tensor_cores, int* regs, int* local_bytes) {
   if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
   if (dtype != E3CONV_F32 && dtype != E3CONV_F16)
     return fail(E3CONV_ERR_UNSUPPORTED, "unknown dtype");
@@ -455,7 +464,8 @@ int e3conv_kernel_info(e3conv_plan h, int dtype, int* V, int* TL, int* block, in
   if (TL) *TL = v.shape.TL;
   if (block) *block = v.shape.block;
   if (stages) *stages = v.shape.stages;
-  if (contract_first) *contract_first = v.shape.coop ? 1 : 0;
+  if (contract_first) *contract_first = (v.shape.coop || v.shape.tc) ? 1 : 0;
+  if (tensor_cores) *tensor_cores = v.shape.tc ? 1 : 0;
   if (regs) *regs = v.regs;
   if (local_bytes) *local_bytes = v.local_bytes;
   return E3CONV_OK;
@@ -494,7 +504,23 @@ int e3conv_forward(e3conv_plan h, const void* x, const void* Y, const void* s,
   const Shape& sh = v.shape;
   long long blocks;
   unsigned smem = 0;
-  if (sh.stages > 0) {
+  CUtensorMap xmap;
+  std::memset(&xmap, 0, sizeof xmap);
+  if (sh.tc) {
+    // x viewed as [num_nodes * nx rows][C columns] of float16; box = nx rows x 64 channels
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(pl.C),
+                                static_cast<cuuint64_t>(num_nodes) * pl.nx};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(pl.C) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(pl.nx)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (driver().TensorMapEncodeTiled(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(x),
+                                      gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return fail(E3CONV_ERR_CUDA, "cuTensorMapEncodeTiled failed for node_features");
+    blocks = std::min<long long>(v.grid_blocks, num_nodes);
+    smem = static_cast<unsigned>(sh.smem_request);
+  } else if (sh.stages > 0) {
     const long long tpb = sh.block / (32 * sh.team);  // teams per block
     blocks = std::min<long long>(v.grid_blocks, (num_nodes + tpb - 1) / tpb);
     smem = static_cast<unsigned>(sh.warp_smem * tpb);
@@ -508,7 +534,7 @@ int e3conv_forward(e3conv_plan h, const void* x, const void* Y, const void* s,
   float inv_avg = static_cast<float>(1.0 / pl.avg);
   void* args[] = {const_cast<void**>(&x), const_cast<void**>(&Y), const_cast<void**>(&s),
                   const_cast<int32_t**>(&senders), const_cast<int32_t**>(&row_ptr),
-                  &n32, &e32, &out, &inv_avg, &pl.status};
+                  &n32, &e32, &out, &inv_avg, &pl.status, &xmap};
   CUresult r = driver().LaunchKernel(v.fn, static_cast<unsigned>(blocks), 1, 1,
                                      static_cast<unsigned>(sh.block), 1, 1, smem,
                                      reinterpret_cast<CUstream>(stream), args, nullptr);

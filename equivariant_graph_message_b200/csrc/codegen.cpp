@@ -78,6 +78,50 @@ Shape choose_shape(const Plan& pl, int dtype) {
   s.y_bytes = pl.ny * elem;
   const bool bytes_ok = s.s_bytes % 16 == 0 && s.x_bytes % 16 == 0 && s.y_bytes % 16 == 0;
 
+  // Tensor-core variant: float16 inputs, 128 channels (the MMA's M), at most
+  // 16 node components (one K step) and at most 256 path outputs (N).
+  const bool want_tc = pl.req_tc == 1;  // opt-in (E3CONV_OPT_TENSOR_CORES)
+  if (want_tc && pl.req_stages != 0 && dtype == E3CONV_F16 && pl.C == 128 && pl.nx <= 16 &&
+      bytes_ok) {
+    int ncols = 0;
+    for (const auto& P : pl.paths) ncols += 2 * P.l3 + 1;
+    ncols = align_up(ncols, 16);
+    if (ncols <= 256) {
+      s.tc = true;
+      s.V = 1;
+      s.team = 4;
+      s.TL = 32;
+      s.tiles = 1;
+      s.ipw = 1;
+      s.block = 192;                                // 4 consumer warps + 2 producer warps
+      s.ncols = ncols;
+      s.tmem_cols = 512;                            // two T buffers at columns 0 and 256
+      // ring depth: copies run up to S-2 edges ahead of the MMA cursor, leaving two
+      // stages for the edges the consumers are still reading
+      const int S = pl.req_stages > 0 ? std::max(pl.req_stages, 3) : 6;
+      s.stages = S;
+      s.x_off = 0;                                  // 16 rows x 128 channels x 2 B, 128B-swizzled
+      s.s_off = 4096;
+      s.y_off = s.s_off + align_up(s.s_bytes, 128);
+      s.stage_bytes = align_up(s.y_off + 128, 1024);
+      s.b_off = S * s.stage_bytes;
+      s.b_bytes = 32 * ncols;                       // 16 x ncols f16, K-major core matrices
+      s.yf_off = s.b_off + 4 * s.b_bytes;           // two buffers of (A_hi, A_lo)
+      s.bar_off = align_up(s.yf_off + 4 * pl.ny, 8);
+      s.mbar_off = s.bar_off;                       // sfull[S] sempty[S] bfree[2] tfull[2] tempty[2]
+      s.hdr_off = s.bar_off + 8 * (2 * S + 6);
+      s.tslot_off = s.hdr_off + 16 * S;
+      s.warp_smem = align_up(s.tslot_off + 16, 1024);
+      // one block per SM (it allocates all 512 tensor-memory columns)
+      s.smem_request = std::max(s.warp_smem, 116 * 1024);
+      if (s.smem_request <= 227 * 1024) return s;
+      s = Shape{};
+      s.s_bytes = static_cast<int>(pl.paths.size()) * pl.C * elem;
+      s.x_bytes = pl.nx * pl.C * elem;
+      s.y_bytes = pl.ny * elem;
+    }
+  }
+
   // Staged variant: a team of `team` warps covers the C channels of one
   // receiver row, V channels per lane.  Preferred: one channel pair per lane
   // (V = 2, team = C / 64), which keeps registers low and warps many.
@@ -897,9 +941,372 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   return em.o.str();
 }
 
+
+// ---------------------------------------------------------------------------
+// Tensor-core variant (float16 inputs, C = 128).
+//
+// Per edge e of receiver b (one block = 4 warps = 128 threads, thread u owns
+// channel u):
+//   T[u, n] = sum_i x[a, i, u] * B[i, n],   n = (p, k),  B[i,(p,k)] = A_p[i,k]
+// with A_p[i,k] = sum_j CG_p[i,j,k] Y_j formed per edge by the block (each
+// entry split into float16 hi + lo parts, so hi + lo carries ~22 bits), and
+//   m[b, o(p)+k, u] += s[e, p, u] * T[u, (p,k)]   (float32 FMA per channel).
+// T is produced by two tcgen05.mma (kind::f16, M = 128, N = ncols, K = 16:
+// A operand = the sender's x rows staged by a 2-D TMA copy with 128-byte
+// swizzle, MN-major; B operand = A_hi / A_lo in shared memory, K-major, no
+// swizzle) into tensor memory and read back with tcgen05.ld.
+// Copies (2-D TMA for x, 1-D bulk for s and Y) go through the same ring of
+// stages as the staged variant; all waits are bounded.
+
+struct BTable {
+  std::string source;
+  int rounds = 0;
+  std::vector<int> terms;
+};
+
+// Entries dealt to the 128 threads in rounds, longest first; per entry the
+// byte offset of its element in the K-major B tile.
+BTable tc_tables(const Plan& pl, const std::vector<AEntry>& ent, const std::vector<int>& colbase,
+                 int RW) {
+  BTable T;
+  std::vector<int> order(ent.size());
+  for (size_t n = 0; n < ent.size(); ++n) order[n] = static_cast<int>(n);
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+    return ent[a].terms.size() > ent[b].terms.size();
+  });
+  T.rounds = static_cast<int>((ent.size() + RW - 1) / RW);
+  std::ostringstream c, d;
+  c << "__device__ const int2 e3_btab[] = {\n";
+  d << "__device__ const int e3_boff[] = {\n";
+  for (int r = 0; r < T.rounds; ++r) {
+    int tr = 0;
+    for (int l = 0; l < RW; ++l) {
+      size_t q = static_cast<size_t>(r) * RW + l;
+      if (q < order.size()) tr = std::max<int>(tr, static_cast<int>(ent[order[q]].terms.size()));
+    }
+    T.terms.push_back(tr);
+    for (int t = 0; t < tr; ++t) {
+      for (int l = 0; l < RW; ++l) {
+        size_t q = static_cast<size_t>(r) * RW + l;
+        double cv = 0.0;
+        int j = 0;
+        if (q < order.size() && t < static_cast<int>(ent[order[q]].terms.size())) {
+          j = ent[order[q]].terms[t].first;
+          cv = ent[order[q]].terms[t].second;
+        }
+        const float cf = static_cast<float>(cv);
+        unsigned int bits;
+        std::memcpy(&bits, &cf, sizeof bits);
+        c << "{" << static_cast<int>(bits) << ", " << j << "},";
+      }
+      c << "\n";
+    }
+    for (int l = 0; l < RW; ++l) {
+      size_t q = static_cast<size_t>(r) * RW + l;
+      int off = -1;
+      if (q < order.size()) {
+        const AEntry& e = ent[order[q]];
+        const int i = pl.paths[e.path].x_off + e.i;       // K index: node component
+        const int n = colbase[e.path] + e.k;               // N index: path output column
+        off = (n / 8) * 256 + (i / 8) * 128 + (n % 8) * 16 + (i % 8) * 2;
+      }
+      d << off << ",";
+    }
+    d << "\n";
+  }
+  c << "};\n";
+  d << "};\n";
+  T.source = c.str() + d.str();
+  return T;
+}
+
+std::string tc_source(const Plan& pl, const Shape& sh) {
+  Emitter em;
+  const int NS = sh.stages;
+  const int PR = 64;  // producer threads (warps 4 and 5)
+  const long long s_row = static_cast<long long>(pl.paths.size()) * pl.C;
+  const long long o_row = static_cast<long long>(pl.nout) * pl.C;
+  std::vector<int> colbase(pl.paths.size());
+  int col = 0;
+  for (size_t p = 0; p < pl.paths.size(); ++p) {
+    colbase[p] = col;
+    col += 2 * pl.paths[p].l3 + 1;
+  }
+  std::vector<AEntry> ent = build_a_entries(pl);
+  BTable tab = tc_tables(pl, ent, colbase, PR);
+  em.line("// generated by libe3conv: fused equivariant convolution forward (tensor cores)");
+  em.line("// C=" + S(pl.C) + " nx=" + S(pl.nx) + " ny=" + S(pl.ny) + " nout=" + S(pl.nout) +
+          " paths=" + S(pl.paths.size()) + " dtype=f16 ncols=" + S(sh.ncols) + " tmem_cols=" +
+          S(sh.tmem_cols) + " stages=" + S(NS) + " stage_bytes=" + S(sh.stage_bytes) +
+          " entries=" + S(ent.size()) + " producer_threads=" + S(PR) + " warps=4 consumers + 2 producers");
+  em.o << tab.source;
+  em.line("__device__ __forceinline__ float h2f(unsigned short h) { float f; asm(\"cvt.f32.f16 %0, %1;\" : \"=f\"(f) : \"h\"(h)); return f; }");
+  em.line("__device__ __forceinline__ unsigned short f2h(float f) { unsigned short h; asm(\"cvt.rn.f16.f32 %0, %1;\" : \"=h\"(h) : \"f\"(f)); return h; }");
+  em.line("#define E3_SPIN_LIMIT (1u << 22)");
+  em.line("struct __align__(64) E3TensorMap { unsigned long long v[16]; };");
+  em.line("__device__ __forceinline__ unsigned int smem_u32(const void* p) { return static_cast<unsigned int>(__cvta_generic_to_shared(p)); }");
+  em.line("__device__ __forceinline__ void bar_init(unsigned long long* b, unsigned int count) { asm volatile(\"mbarrier.init.shared::cta.b64 [%0], %1;\" :: \"r\"(smem_u32(b)), \"r\"(count) : \"memory\"); }");
+  em.line("__device__ __forceinline__ void bar_arrive(unsigned long long* b) { asm volatile(\"mbarrier.arrive.shared::cta.b64 _, [%0];\" :: \"r\"(smem_u32(b)) : \"memory\"); }");
+  em.line("__device__ __forceinline__ void bar_expect(unsigned long long* b, unsigned int bytes) { asm volatile(\"mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\" :: \"r\"(smem_u32(b)), \"r\"(bytes) : \"memory\"); }");
+  em.line("__device__ __forceinline__ bool bar_try(unsigned long long* b, unsigned int parity) {");
+  em.line("  unsigned int ok; asm volatile(\"{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }\" : \"=r\"(ok) : \"r\"(smem_u32(b)), \"r\"(parity) : \"memory\"); return ok != 0; }");
+  em.line("__device__ __forceinline__ bool bar_wait(unsigned long long* b, unsigned int parity) {");
+  em.line("  for (unsigned int it = 0; it < E3_SPIN_LIMIT; ++it) if (bar_try(b, parity)) return true; return false; }");
+  em.line("__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned int bytes, unsigned long long* b, unsigned long long policy) {");
+  em.line("  asm volatile(\"cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;\" :: \"r\"(smem_u32(dst)), \"l\"(src), \"r\"(bytes), \"r\"(smem_u32(b)), \"l\"(policy) : \"memory\"); }");
+  em.line("__device__ __forceinline__ void tma2d_g2s(void* dst, const E3TensorMap* map, int c0, int c1, unsigned long long* b, unsigned long long policy) {");
+  em.line("  asm volatile(\"cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;\" :: \"r\"(smem_u32(dst)), \"l\"(map), \"r\"(c0), \"r\"(c1), \"r\"(smem_u32(b)), \"l\"(policy) : \"memory\"); }");
+  em.line("__device__ __forceinline__ unsigned long long policy_evict_first() { unsigned long long p; asm volatile(\"createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\" : \"=l\"(p)); return p; }");
+  em.line("__device__ __forceinline__ unsigned long long policy_evict_last() { unsigned long long p; asm volatile(\"createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\" : \"=l\"(p)); return p; }");
+  em.line("__device__ __forceinline__ void fence_async_smem() { asm volatile(\"fence.proxy.async.shared::cta;\" ::: \"memory\"); }");
+  em.line("__device__ __forceinline__ void prod_sync() { asm volatile(\"bar.sync 2, 64;\" ::: \"memory\"); }");
+  em.line("__device__ __forceinline__ bool prod_all(bool ok) { unsigned int r; asm volatile(\"{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.and.pred q, 2, 64, p; selp.u32 %0, 1, 0, q; }\" : \"=r\"(r) : \"r\"((unsigned int)ok) : \"memory\"); return r != 0u; }");
+  em.line("__device__ __forceinline__ bool cons_all(bool ok) { unsigned int r; asm volatile(\"{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.and.pred q, 3, 128, p; selp.u32 %0, 1, 0, q; }\" : \"=r\"(r) : \"r\"((unsigned int)ok) : \"memory\"); return r != 0u; }");
+  em.line("__device__ __forceinline__ void tc_before() { asm volatile(\"tcgen05.fence::before_thread_sync;\" ::: \"memory\"); }");
+  em.line("__device__ __forceinline__ void tc_after() { asm volatile(\"tcgen05.fence::after_thread_sync;\" ::: \"memory\"); }");
+  em.line("#define TMEM_LD32(addr, r) asm volatile(\"tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\" : \"=r\"(r[0]), \"=r\"(r[1]), \"=r\"(r[2]), \"=r\"(r[3]), \"=r\"(r[4]), \"=r\"(r[5]), \"=r\"(r[6]), \"=r\"(r[7]), \"=r\"(r[8]), \"=r\"(r[9]), \"=r\"(r[10]), \"=r\"(r[11]), \"=r\"(r[12]), \"=r\"(r[13]), \"=r\"(r[14]), \"=r\"(r[15]), \"=r\"(r[16]), \"=r\"(r[17]), \"=r\"(r[18]), \"=r\"(r[19]), \"=r\"(r[20]), \"=r\"(r[21]), \"=r\"(r[22]), \"=r\"(r[23]), \"=r\"(r[24]), \"=r\"(r[25]), \"=r\"(r[26]), \"=r\"(r[27]), \"=r\"(r[28]), \"=r\"(r[29]), \"=r\"(r[30]), \"=r\"(r[31]) : \"r\"(addr))");
+  em.line("extern \"C\" __global__ void __launch_bounds__(192, 1) e3conv_fwd(");
+  em.line("    const unsigned short* __restrict__ x, const unsigned short* __restrict__ Y,");
+  em.line("    const unsigned short* __restrict__ s, const int* __restrict__ senders,");
+  em.line("    const int* __restrict__ row_ptr, int num_nodes, int num_edges, float* __restrict__ out,");
+  em.line("    float inv_avg, unsigned int* __restrict__ status, const __grid_constant__ E3TensorMap xmap)");
+  em.line("{");
+  em.ind++;
+  em.line("extern __shared__ __align__(1024) unsigned char smem[];");
+  em.line("const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;");
+  em.line("unsigned char* tbase = smem;");
+  em.line("unsigned long long* sfull = reinterpret_cast<unsigned long long*>(tbase + " + S(sh.bar_off) + ");");
+  em.line("unsigned long long* sempty = sfull + " + S(NS) + ";");
+  em.line("unsigned long long* bfree = sempty + " + S(NS) + ";");
+  em.line("unsigned long long* tfull = bfree + 2;");
+  em.line("unsigned long long* tempty = tfull + 2;");
+  em.line("int* hdr = reinterpret_cast<int*>(tbase + " + S(sh.hdr_off) + ");  // per stage: sender (-1 invalid, -2 end), receiver, last");
+  em.line("unsigned int* tslot = reinterpret_cast<unsigned int*>(tbase + " + S(sh.tslot_off) + ");");
+  em.line("float* yf = reinterpret_cast<float*>(tbase + " + S(sh.yf_off) + ");");
+  em.line("unsigned char* Bt = tbase + " + S(sh.b_off) + ";  // buffer bb: A_hi at bb*" + S(2 * sh.b_bytes) + ", A_lo at +" + S(sh.b_bytes));
+  em.line("for (int q = tid; q < " + S(4 * sh.b_bytes / 16) + "; q += 192) reinterpret_cast<uint4*>(Bt)[q] = make_uint4(0u, 0u, 0u, 0u);");
+  em.line("for (int k = 0; k < " + S(NS) + "; ++k)");
+  em.line("  for (int q = tid; q < 256; q += 192) reinterpret_cast<uint4*>(tbase + k * " + S(sh.stage_bytes) + ")[q] = make_uint4(0u, 0u, 0u, 0u);");
+  em.line("if (tid == 0) {");
+  em.line("  for (int k = 0; k < " + S(NS) + "; ++k) { bar_init(sfull + k, 1u); bar_init(sempty + k, 128u); }");
+  em.line("  for (int k = 0; k < 2; ++k) { bar_init(bfree + k, 1u); bar_init(tfull + k, 1u); bar_init(tempty + k, 128u); }");
+  em.line("  asm volatile(\"fence.mbarrier_init.release.cluster;\" ::: \"memory\");");
+  em.line("}");
+  em.line("if (warp == 0) {");
+  em.line("  asm volatile(\"tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], " + S(sh.tmem_cols) + ";\" :: \"r\"(smem_u32(tslot)) : \"memory\");");
+  em.line("  asm volatile(\"tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\" ::: \"memory\");");
+  em.line("}");
+  em.line("fence_async_smem();");
+  em.line("tc_before();");
+  em.line("__syncthreads();");
+  em.line("tc_after();");
+  em.line("const unsigned int tmem = *tslot;");
+  em.line("const long long W = (long long)gridDim.x;");
+  em.line("if (warp >= 4) {");
+  em.ind++;
+  // ---------------- producers ----------------
+  em.line("// producers: row walk, copies, A tiles, MMA issue");
+  em.line("const int pt = tid - 128;  // 0..63");
+  em.line("const bool issuer = pt == 0;");
+  em.line("const unsigned long long pol_stream = policy_evict_first();");
+  em.line("const unsigned long long pol_keep = policy_evict_last();");
+  em.line("const unsigned int idesc = (1u << 4) | (1u << 15) | ((unsigned int)(" + S(sh.ncols) + " >> 3) << 17) | ((unsigned int)(128 >> 4) << 24);");
+  em.line("long long pb = (long long)blockIdx.x - W;");
+  em.line("int pe = 0, pe1 = 0, pwin = -1, psw = 0;");
+  em.line("bool walk_done = false, ok = true;");
+  em.line("unsigned int qi = 0, qm = 0, v = 0;  // next position to copy, next position to multiply, valid edges multiplied");
+  em.line("#pragma unroll 1");
+  em.line("while (ok) {");
+  em.ind++;
+  em.line("// copies for positions ahead of the MMA cursor (ring of " + S(NS) + " stages, two kept");
+  em.line("// for the consumers so this wait targets an edge they have already finished)");
+  em.line("#pragma unroll 1");
+  em.line("while (ok && !walk_done && qi < qm + " + S(NS - 2) + ") {");
+  em.ind++;
+  em.line("const unsigned int st = qi % " + S(NS) + ";");
+  em.line("if (qi >= " + S(NS) + "u) { ok = prod_all(bar_wait(sempty + st, ((qi / " + S(NS) + ") - 1u) & 1u)); if (!ok) break; }");
+  em.line("while (pe >= pe1) {");
+  em.line("  pb += W;");
+  em.line("  if (pb >= num_nodes) { walk_done = true; break; }");
+  em.line("  int r0 = row_ptr[pb], r1 = row_ptr[pb + 1];");
+  em.line("  if (r0 < 0 || r1 < r0 || r1 > num_edges) { if (issuer) atomicOr(status, 1u); r1 = r0; }");
+  em.line("  pe = r0; pe1 = r1; pwin = -1;");
+  em.line("  if (r0 == r1) {");
+  em.line("    float* zrow = out + pb * " + S(o_row) + ";");
+  em.line("    for (int q = pt; q < " + S(o_row) + "; q += 64) zrow[q] = 0.f;");
+  em.line("  }");
+  em.line("}");
+  em.line("if (walk_done) {");
+  em.line("  if (issuer) { hdr[4 * st] = -2; bar_arrive(sfull + st); }  // end marker");
+  em.line("  ++qi;");
+  em.line("  break;");
+  em.line("}");
+  em.line("if (pwin < 0 || pe >= pwin + 32) { pwin = pe; psw = (pe + lane < pe1) ? senders[pe + lane] : 0; }");
+  em.line("const int a = __shfl_sync(0xffffffffu, psw, pe - pwin);");
+  em.line("const bool valid = (unsigned int)a < (unsigned int)num_nodes;");
+  em.line("if (issuer) {");
+  em.line("  unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
+  em.line("  hdr[4 * st] = valid ? a : -1;");
+  em.line("  hdr[4 * st + 1] = (int)pb;");
+  em.line("  hdr[4 * st + 2] = (pe + 1 == pe1) ? 1 : 0;");
+  em.line("  fence_async_smem();");
+  em.line("  bar_expect(sfull + st, " + S(sh.s_bytes + sh.y_bytes) + "u + (valid ? " + S(sh.x_bytes) + "u : 0u));");
+  em.line("  bulk_g2s(stg + " + S(sh.s_off) + ", s + (long long)pe * " + S(s_row) + ", " + S(sh.s_bytes) + "u, sfull + st, pol_stream);");
+  em.line("  bulk_g2s(stg + " + S(sh.y_off) + ", Y + (long long)pe * " + S(pl.ny) + ", " + S(sh.y_bytes) + "u, sfull + st, pol_stream);");
+  em.line("  if (valid) {");
+  em.line("    tma2d_g2s(stg, &xmap, 0, a * " + S(pl.nx) + ", sfull + st, pol_keep);");
+  em.line("    tma2d_g2s(stg + 2048, &xmap, 64, a * " + S(pl.nx) + ", sfull + st, pol_keep);");
+  em.line("  }");
+  em.line("}");
+  em.line("++pe;");
+  em.line("++qi;");
+  em.ind--;
+  em.line("}");
+  em.line("if (!ok || qm == qi) break;");
+  em.line("// position qm: wait for its copies, build A, multiply");
+  em.line("const unsigned int st = qm % " + S(NS) + ";");
+  em.line("ok = prod_all(bar_wait(sfull + st, (qm / " + S(NS) + ") & 1u));");
+  em.line("if (!ok) break;");
+  em.line("const int a = hdr[4 * st];");
+  em.line("if (a == -2) break;");
+  em.line("if (a >= 0) {");
+  em.ind++;
+  em.line("const unsigned int bb = v & 1u;");
+  em.line("if (v >= 2u) { ok = prod_all(bar_wait(bfree + bb, ((v >> 1) - 1u) & 1u)); if (!ok) break; }");
+  em.line("unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
+  em.line("unsigned char* Bhi = Bt + bb * " + S(2 * sh.b_bytes) + ";");
+  em.line("unsigned char* Blo = Bhi + " + S(sh.b_bytes) + ";");
+  em.line("if (pt < " + S(pl.ny) + ") yf[pt] = h2f(reinterpret_cast<const unsigned short*>(stg + " + S(sh.y_off) + ")[pt]);");
+  em.line("prod_sync();");
+  int base = 0;
+  for (int r = 0; r < tab.rounds; ++r) {
+    em.line("{");
+    em.ind++;
+    for (int t2 = 0; t2 < tab.terms[r]; ++t2)
+      em.line("const int2 k" + S(t2) + " = __ldg(&e3_btab[" + S(base + t2 * PR) + " + pt]);");
+    std::string val = "__int_as_float(k0.x) * yf[k0.y]";
+    for (int t2 = 1; t2 < tab.terms[r]; ++t2)
+      val = "fmaf(__int_as_float(k" + S(t2) + ".x), yf[k" + S(t2) + ".y], " + val + ")";
+    em.line("const int off = __ldg(&e3_boff[" + S(r * PR) + " + pt]);");
+    em.line("if (off >= 0) {");
+    em.line("  const float val = " + val + ";");
+    em.line("  const unsigned short hi = f2h(val);");
+    em.line("  *reinterpret_cast<unsigned short*>(Bhi + off) = hi;");
+    em.line("  *reinterpret_cast<unsigned short*>(Blo + off) = f2h(val - h2f(hi));");
+    em.line("}");
+    em.ind--;
+    em.line("}");
+    base += tab.terms[r] * PR;
+  }
+  em.line("fence_async_smem();");
+  em.line("prod_sync();");
+  em.line("const unsigned int tb = v & 1u;");
+  em.line("if (v >= 2u) { ok = prod_all(bar_wait(tempty + tb, ((v >> 1) - 1u) & 1u)); if (!ok) break; }");
+  em.line("tc_after();");
+  em.line("if (issuer) {");
+  em.line("  const unsigned long long adesc = (unsigned long long)((smem_u32(stg) & 0x3FFFF) >> 4) | (128ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);");
+  em.line("  const unsigned long long hdesc = (unsigned long long)((smem_u32(Bhi) & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
+  em.line("  const unsigned long long ldesc = (unsigned long long)((smem_u32(Blo) & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
+  em.line("  const unsigned int dt = tmem + tb * 256u;");
+  em.line("  asm volatile(\"{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }\" :: \"r\"(dt), \"l\"(adesc), \"l\"(hdesc), \"r\"(idesc), \"r\"(0u) : \"memory\");");
+  em.line("  asm volatile(\"{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }\" :: \"r\"(dt), \"l\"(adesc), \"l\"(ldesc), \"r\"(idesc), \"r\"(1u) : \"memory\");");
+  em.line("  asm volatile(\"tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\" :: \"r\"(smem_u32(tfull + tb)) : \"memory\");");
+  em.line("  asm volatile(\"tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\" :: \"r\"(smem_u32(bfree + bb)) : \"memory\");");
+  em.line("}");
+  em.line("++v;");
+  em.ind--;
+  em.line("}");
+  em.line("++qm;");
+  em.ind--;
+  em.line("}");
+  em.line("if (!ok && issuer) atomicOr(status, 4u);");
+  em.line("// drain: every issued copy and MMA completes before the block leaves (bounded)");
+  em.line("if (issuer) {");
+  em.line("  for (unsigned int q = qm; q < qi; ++q) bar_wait(sfull + q % " + S(NS) + ", (q / " + S(NS) + ") & 1u);");
+  em.line("  if (v > 0u) bar_wait(bfree + ((v - 1u) & 1u), ((v - 1u) >> 1) & 1u);");
+  em.line("}");
+  em.ind--;
+  em.line("} else {");
+  em.ind++;
+  // ---------------- consumers ----------------
+  em.line("// consumers: thread tid owns channel tid; tensor-memory lanes 32*warp .. 32*warp+31");
+  {
+    std::string decl = "float";
+    for (int c = 0; c < pl.nout; ++c) decl += std::string(c ? "," : "") + " a" + S(c) + " = 0.f";
+    em.line(decl + ";");
+  }
+  em.line("const unsigned int tmem_lane = tmem + ((unsigned int)(warp * 32) << 16);");
+  em.line("unsigned int q = 0, v = 0;");
+  em.line("bool ok = true;");
+  em.line("#pragma unroll 1");
+  em.line("while (true) {");
+  em.ind++;
+  em.line("const unsigned int st = q % " + S(NS) + ";");
+  em.line("ok = cons_all(bar_wait(sfull + st, (q / " + S(NS) + ") & 1u));");
+  em.line("if (!ok) break;");
+  em.line("unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
+  em.line("const int a = hdr[4 * st];");
+  em.line("if (a == -2) break;");
+  em.line("const long long b = hdr[4 * st + 1];");
+  em.line("const int last = hdr[4 * st + 2];");
+  em.line("if (a >= 0) {");
+  em.ind++;
+  em.line("const unsigned int tb = v & 1u;");
+  em.line("ok = cons_all(bar_wait(tfull + tb, (v >> 1) & 1u));");
+  em.line("if (!ok) break;");
+  em.line("tc_after();");
+  em.line("const unsigned short* sv = reinterpret_cast<const unsigned short*>(stg + " + S(sh.s_off) + ") + tid;");
+  em.line("const unsigned int tcol = tmem_lane + tb * 256u;");
+  {
+    std::vector<std::pair<int, int>> colmap;
+    for (size_t p = 0; p < pl.paths.size(); ++p)
+      for (int k = 0; k < 2 * pl.paths[p].l3 + 1; ++k) colmap.push_back({static_cast<int>(p), k});
+    const int nchunk = (static_cast<int>(colmap.size()) + 31) / 32;
+    // edge scalars first (shared-memory loads overlap the tensor-memory loads)
+    for (size_t p = 0; p < pl.paths.size(); ++p)
+      em.line("const float s" + S(p) + " = h2f(sv[" + S(static_cast<long long>(p) * pl.C) + "]);");
+    for (int c = 0; c < nchunk; ++c) {
+      em.line("unsigned int r" + S(c) + "[32];");
+      em.line("TMEM_LD32(tcol + " + S(32 * c) + "u, r" + S(c) + ");");
+    }
+    em.line("asm volatile(\"tcgen05.wait::ld.sync.aligned;\" ::: \"memory\");");
+    em.line("tc_before();");
+    em.line("bar_arrive(tempty + tb);  // T is in registers: the buffer is free for the next MMA");
+    for (int cc = 0; cc < static_cast<int>(colmap.size()); ++cc) {
+      const int p = colmap[cc].first, k = colmap[cc].second;
+      const std::string acc = "a" + S(pl.paths[p].out_off + k);
+      em.line(acc + " = fmaf(s" + S(p) + ", __uint_as_float(r" + S(cc / 32) + "[" + S(cc % 32) + "]), " + acc + ");");
+    }
+  }
+  em.line("++v;");
+  em.ind--;
+  em.line("} else if (tid == 0) {");
+  em.line("  atomicOr(status, 2u);");
+  em.line("}");
+  em.line("bar_arrive(sempty + st);");
+  em.line("if (last) {");
+  em.line("  float* orow = out + b * " + S(o_row) + " + tid;");
+  for (int c = 0; c < pl.nout; ++c) em.line("  orow[" + S(c * pl.C) + "] = a" + S(c) + " * inv_avg; a" + S(c) + " = 0.f;");
+  em.line("}");
+  em.line("++q;");
+  em.ind--;
+  em.line("}");
+  em.line("if (!ok && tid == 0) atomicOr(status, 4u);");
+  em.ind--;
+  em.line("}");
+  em.line("tc_before();");
+  em.line("__syncthreads();");
+  em.line("tc_after();");
+  em.line("if (warp == 0) asm volatile(\"tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, " + S(sh.tmem_cols) + ";\" :: \"r\"(tmem) : \"memory\");");
+  em.ind--;
+  em.line("}");
+  return em.o.str();
+}
+
 }  // namespace
 
 std::string generate_forward_source(const Plan& pl, int dtype, const Shape& sh) {
+  if (sh.tc) return tc_source(pl, sh);
   return sh.stages > 0 ? staged_source(pl, dtype, sh) : direct_source(pl, dtype, sh);
 }
 

@@ -56,6 +56,15 @@ struct Shape {
   bool dup_a = false;                         // A stored as (a, a) pairs (one channel pair per lane)
   int na = 0;                                 // number of A entries (all paths)
   int a_off = 0, yf_off = 0;                  // A entries and float32 Y inside a team's region
+  // Tensor-core variant (float16 inputs, C = 128): per edge, T = x^T (A_hi + A_lo)
+  // with tcgen05.mma (M = 128 channels, K = 16 node components, N = ncols path
+  // outputs) into tensor memory, then T is scaled by s per channel.
+  bool tc = false;
+  int ncols = 0;                              // sum over paths of 2l3+1, padded to 16
+  int tmem_cols = 0;                          // tensor-memory columns allocated (power of 2)
+  int b_off = 0, b_bytes = 0;                 // A_hi at b_off, A_lo at b_off + b_bytes
+  int mbar_off = 0, tslot_off = 0;            // MMA barrier, tensor-memory address slot
+  int smem_request = 0;                       // dynamic shared memory requested per block
 };
 
 // One entry A_p[i,k] of the per-edge contraction of CG with Y.
@@ -87,6 +96,7 @@ struct Plan {
   int req_V = 0, req_block = 0, req_stages = -1;  // -1: automatic
   int auto_block = 0;                              // block chosen after a first compile (0: none)
   int req_coop = -1;                               // -1: automatic, 0: off, 1: on
+  int req_tc = -1;                                 // -1: automatic, 0: off, 1: on
   int device = -1;                 // -1: host-only plan
   CUcontext ctx = nullptr;
   unsigned int* status = nullptr;  // device status word

@@ -148,6 +148,14 @@ E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane,
  *   float32x2 FMAs; with 0 every lane forms the products CG*Y_j itself.
  *   Same arithmetic up to rounding order. */
 #define E3CONV_OPT_CONTRACT_FIRST 1
+/*   E3CONV_OPT_TENSOR_CORES: 0 (default; -1 means the same) or 1.  With float16
+ *   inputs, C = 128, at most 16 node components and at most 256 path outputs,
+ *   the forward forms per edge T = x^T A on the tensor cores (tcgen05.mma,
+ *   M = 128 channels, K = node components, N = path outputs; A = sum_j CG Y_j
+ *   split into float16 hi + lo parts, float32 accumulation in tensor memory)
+ *   and then scales T by the edge scalars with float32 FMAs.  Requesting it
+ *   for a shape outside those limits keeps the float32 staged variant. */
+#define E3CONV_OPT_TENSOR_CORES 2
 E3CONV_API int e3conv_set_option(e3conv_plan plan, int option, int value);
 
 /* Sizes: C channels, nx node components, ny edge components, nout output
@@ -172,11 +180,13 @@ E3CONV_API int e3conv_cg(e3conv_plan plan, int p, double* dense_out);
 /* Launch shape and resources of the forward kernel for `dtype`:
  * channels per lane, lanes per receiver tile, block threads, ring stages
  * (0: direct variant), whether the CG x Y contraction is formed first
- * (E3CONV_OPT_CONTRACT_FIRST), registers per thread and local-memory (spill)
+ * (E3CONV_OPT_CONTRACT_FIRST), whether the tensor-core variant is used
+ * (E3CONV_OPT_TENSOR_CORES), registers per thread and local-memory (spill)
  * bytes per thread.  Any pointer may be NULL. */
 E3CONV_API int e3conv_kernel_info(e3conv_plan plan, int dtype, int* channels_per_lane,
                                   int* lanes_per_tile, int* block_threads, int* stages,
-                                  int* contract_first, int* registers, int* local_bytes);
+                                  int* contract_first, int* tensor_cores, int* registers,
+                                  int* local_bytes);
 
 /* Copies the generated CUDA source for `dtype` (NUL-terminated) into buf if
  * buf_len is large enough; *needed receives the required size in bytes. */

@@ -46,6 +46,7 @@ def test_staged_parity_with_empty_rows(cuda_device, C, dt, contract_first):
     send, recv = _graph(rng, n, e, empty_frac=0.2)
     pl, x, Y, s = _inputs(rng, irreps, n, e, dt)
     conv = e3.Conv(*irreps, 12.0, dtype=dt)
+    conv.set_tensor_cores(0)          # the float32 staged path (tensor cores: test_gpu_tensor_cores)
     conv.set_contract_first(contract_first)
     info = conv.kernel_info()
     assert info["stages"] >= 2 and info["contract_first"] == contract_first

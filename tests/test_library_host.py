@@ -101,8 +101,9 @@ def test_generated_kernel_unrolls_every_coefficient():
     c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 40.0, dtype="f16")
     nnz = sum(int((np.abs(c.cg(p)) > 1e-12).sum()) for p in range(c.num_paths))
     assert nnz == 611
-    # contraction-first (default for this shape): one table entry per nonzero
+    # contraction-first (the float32 path): one table entry per nonzero
     # A_p[i,k] = sum_j CG_p[i,j,k] Y_j, each applied to every channel pair
+    c.set_tensor_cores(0)
     info = c.kernel_info()
     assert info["contract_first"] == 1 and info["stages"] >= 2 and info["local_bytes"] == 0
     src = c.kernel_source()
@@ -194,3 +195,50 @@ def test_size_limits_rejected_on_host():
     assert e3._csr_ws((1 << 31) - 1, (1 << 31) - 2, ctypes.byref(n)) == 0
     cnt = ctypes.c_int()
     assert e3._csr_count((1 << 31) - 1, 100000, ctypes.byref(cnt)) == 0 and cnt.value > 0
+
+
+def test_tensor_core_tables_emulated_on_host():
+    # The tensor-core kernel writes A_p[i,k] = sum_j CG_p[i,j,k] Y_j into a
+    # K-major B tile (K = node component, N = path output column); decode the
+    # generated table and offsets and compare with the direct contraction.
+    s = SPECS["large_f16"]
+    c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 40.0, dtype="f16")
+    c.set_tensor_cores(1)
+    info = c.kernel_info()
+    assert info["tensor_cores"] == 1 and info["local_bytes"] == 0
+    src = c.kernel_source()
+    ncols = int(re.search(r"ncols=(\d+)", src).group(1))
+    tab = re.search(r"e3_btab\[\] = \{(.*?)\};", src, re.S).group(1)
+    pairs = [(int(a), int(b)) for a, b in re.findall(r"\{(-?\d+), (\d+)\}", tab)]
+    offs = [int(v) for v in re.search(r"e3_boff\[\] = \{(.*?)\};", src, re.S).group(1)
+            .replace("\n", "").split(",") if v.strip()]
+    terms = [int(m) for m in re.findall(r"// round terms: (\d+)", src)] or None
+    Y = np.random.default_rng(3).normal(size=c.ny)
+    B = np.zeros((16, ncols))
+    base = 0
+    lanes = int(re.search(r"producer_threads=(\d+)", src).group(1))
+    rounds = re.findall(r"\{\n((?:\s+const int2 k\d+ = __ldg\(&e3_btab\[(\d+) \+ pt\]\);\n)+)", src)
+    assert len(rounds) == -(-541 // lanes)
+    for r, (body, _) in enumerate(rounds):
+        bases = [int(b) for b in re.findall(r"e3_btab\[(\d+) \+ pt\]", body)]
+        for lane in range(lanes):
+            off = offs[r * lanes + lane]
+            if off < 0:
+                continue
+            v = sum(np.frombuffer(np.int32(pairs[b + lane][0]).tobytes(), np.float32)[0] *
+                    Y[pairs[b + lane][1]] for b in bases)
+            n = (off // 256) * 8 + (off % 128) // 16           # K-major core-matrix layout
+            i = ((off % 256) // 128) * 8 + (off % 16) // 2
+            assert B[i, n] == 0
+            B[i, n] = v
+    expect = np.zeros((16, ncols))
+    col = 0
+    for p, q in enumerate(c.paths):
+        W = c.cg(p)
+        d1, d2, d3 = W.shape
+        for i in range(d1):
+            for k in range(d3):
+                expect[q.x_off + i, col + k] = W[i, :, k] @ Y[q.l2 ** 2:q.l2 ** 2 + d2]
+        col += d3
+    np.testing.assert_allclose(B, expect, atol=1e-5)
+    assert (np.abs(expect) > 1e-9).sum() == 541
