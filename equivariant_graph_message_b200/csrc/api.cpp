@@ -507,13 +507,17 @@ int e3conv_forward(e3conv_plan h, const void* x, const void* Y, const void* s,
   CUtensorMap xmap;
   std::memset(&xmap, 0, sizeof xmap);
   if (sh.tc) {
-    // x viewed as [num_nodes * nx rows][C columns] of float16; box = nx rows x 64 channels
-    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(pl.C),
-                                static_cast<cuuint64_t>(num_nodes) * pl.nx};
-    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(pl.C) * 2};
-    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(pl.nx)};
-    const cuuint32_t estr[2] = {1, 1};
-    if (driver().TensorMapEncodeTiled(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(x),
+    // x viewed as a 4-D tensor {64 channels, nx components, C / 64 channel halves, nodes}
+    // (strides C * 2, 128 and nx * C * 2 bytes).  One box {64, 16, 2, 1} is a sender's
+    // whole tile: two 128B-swizzled 64-channel halves of 16 rows each, 2048 bytes apart;
+    // rows nx..15 lie outside the tensor and are filled with zeros.
+    const cuuint64_t gdim[4] = {64, static_cast<cuuint64_t>(pl.nx), static_cast<cuuint64_t>(pl.C / 64),
+                                static_cast<cuuint64_t>(num_nodes)};
+    const cuuint64_t gstride[3] = {static_cast<cuuint64_t>(pl.C) * 2, 128,
+                                   static_cast<cuuint64_t>(pl.nx) * pl.C * 2};
+    const cuuint32_t box[4] = {64, 16, static_cast<cuuint32_t>(pl.C / 64), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (driver().TensorMapEncodeTiled(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(x),
                                       gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)

@@ -93,23 +93,25 @@ Shape choose_shape(const Plan& pl, int dtype) {
       s.TL = 32;
       s.tiles = 1;
       s.ipw = 1;
-      s.block = 192;                                // 4 consumer warps + 2 producer warps
+      s.block = 480;                                // 8 consumer, 2 copy, 1 MMA, 4 builder warps
       s.ncols = ncols;
-      s.tmem_cols = 512;                            // two T buffers at columns 0 and 256
-      // ring depth: copies run up to S-2 edges ahead of the MMA cursor, leaving two
-      // stages for the edges the consumers are still reading
-      const int S = pl.req_stages > 0 ? std::max(pl.req_stages, 3) : 6;
+      s.tmem_cols = 512;
+      s.tstride = align_up(ncols, 32);              // T buffers start on 32-column boundaries
+      s.tbufs = std::min(3, 512 / s.tstride);
+      s.bbufs = s.tbufs;                            // one A tile per T buffer
+      const int S = pl.req_stages > 0 ? std::max(pl.req_stages, 2) : 8;
       s.stages = S;
-      s.x_off = 0;                                  // 16 rows x 128 channels x 2 B, 128B-swizzled
+      s.x_off = 0;                                  // nx rows x 128 channels x 2 B, two 128B-swizzled halves
       s.s_off = 4096;
       s.y_off = s.s_off + align_up(s.s_bytes, 128);
-      s.stage_bytes = align_up(s.y_off + 128, 1024);
+      s.stage_bytes = align_up(s.y_off + s.y_bytes, 1024);
       s.b_off = S * s.stage_bytes;
       s.b_bytes = 32 * ncols;                       // 16 x ncols f16, K-major core matrices
-      s.yf_off = s.b_off + 4 * s.b_bytes;           // two buffers of (A_hi, A_lo)
-      s.bar_off = align_up(s.yf_off + 4 * pl.ny, 8);
-      s.mbar_off = s.bar_off;                       // sfull[S] sempty[S] bfree[2] tfull[2] tempty[2]
-      s.hdr_off = s.bar_off + 8 * (2 * S + 6);
+      s.b_stride = s.b_bytes + 128;                 // + scratch for the builders' padding lanes
+      s.yf_off = s.b_off + 2 * s.bbufs * s.b_stride; // bbufs buffers of (A_hi, A_lo)
+      s.bar_off = align_up(s.yf_off + 4 * 4 * align_up(pl.ny, 4), 8);  // Y as float32, per builder warp
+      s.mbar_off = s.bar_off;                       // sfull[S] sempty[S] bfull[T] tfull[T] tempty[T]
+      s.hdr_off = s.bar_off + 8 * (2 * S + s.bbufs + 2 * s.tbufs);
       s.tslot_off = s.hdr_off + 16 * S;
       s.warp_smem = align_up(s.tslot_off + 16, 1024);
       // one block per SM (it allocates all 512 tensor-memory columns)
@@ -1020,25 +1022,69 @@ BTable tc_tables(const Plan& pl, const std::vector<AEntry>& ent, const std::vect
   return T;
 }
 
+// Tensor-core forward.  Warp roles of one block (one block per SM):
+//   warps 0..7   consumers: warp w reads tensor-memory lanes 32*(w%4).. (its
+//                channels) and the path columns of output group w/4, scales
+//                them by s and accumulates the receiver row in registers;
+//   warps 8, 9   copies: both walk the block's rows; warp 8 fills the even
+//                ring positions, warp 9 the odd ones (TMA of the sender's
+//                nx x 128 tile, bulk copies of the edge's s and Y rows);
+//   warp 10      MMA: T = x^T (A_hi + A_lo) into one of NT tensor-memory buffers;
+//   warps 11..14 build A = sum_j CG Y_j (K-major float16 hi/lo tiles, one per T buffer).
+// Every hand-off is an mbarrier with one arrival per warp (or a TMA / MMA
+// completion); every wait is bounded and agreed within the warp only.  One MMA
+// commit per edge (tfull) serves both the consumers (T ready) and the builders
+// (the A tile of that buffer is free again).  A ring stage is released once its
+// readers are done: builders once Y is in their buffer, the MMA warp once it
+// has issued, consumers once s is in registers and the MMA has completed (so x
+// has been read).
 std::string tc_source(const Plan& pl, const Shape& sh) {
   Emitter em;
   const int NS = sh.stages;
-  const int PR = 64;  // producer threads (warps 4 and 5)
+  const int NT = sh.tbufs;
+  const int NB = 4, BT = 32 * NB;             // builder warps / threads
+  const int NBUF = NT;                        // A tile buffers, paired with the T buffers
+  const int BS = sh.b_stride;                 // bytes between A_hi and A_lo (tile + scratch)
+  const int TID_B = 352, W_COPY = 8, W_MMA = 10, W_B = 11;
   const long long s_row = static_cast<long long>(pl.paths.size()) * pl.C;
   const long long o_row = static_cast<long long>(pl.nout) * pl.C;
+  // outputs split into two groups of similar column count; group 0's paths
+  // take the first columns of T
+  std::vector<int> ocols(pl.outputs.size(), 0), og(pl.outputs.size(), 0);
+  for (const auto& P : pl.paths) ocols[P.o] += 2 * P.l3 + 1;
+  {
+    std::vector<int> ord(pl.outputs.size());
+    for (size_t o = 0; o < ord.size(); ++o) ord[o] = static_cast<int>(o);
+    std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return ocols[a] > ocols[b]; });
+    int load[2] = {0, 0};
+    for (int o : ord) {
+      const int g = load[1] < load[0] ? 1 : 0;
+      og[o] = g;
+      load[g] += ocols[o];
+    }
+  }
   std::vector<int> colbase(pl.paths.size());
-  int col = 0;
-  for (size_t p = 0; p < pl.paths.size(); ++p) {
-    colbase[p] = col;
-    col += 2 * pl.paths[p].l3 + 1;
+  int gcol[3];
+  {
+    int col = 0;
+    for (int g = 0; g < 2; ++g) {
+      gcol[g] = col;
+      for (size_t p = 0; p < pl.paths.size(); ++p)
+        if (og[pl.paths[p].o] == g) {
+          colbase[p] = col;
+          col += 2 * pl.paths[p].l3 + 1;
+        }
+    }
+    gcol[2] = col;
   }
   std::vector<AEntry> ent = build_a_entries(pl);
-  BTable tab = tc_tables(pl, ent, colbase, PR);
+  BTable tab = tc_tables(pl, ent, colbase, BT);
   em.line("// generated by libe3conv: fused equivariant convolution forward (tensor cores)");
   em.line("// C=" + S(pl.C) + " nx=" + S(pl.nx) + " ny=" + S(pl.ny) + " nout=" + S(pl.nout) +
-          " paths=" + S(pl.paths.size()) + " dtype=f16 ncols=" + S(sh.ncols) + " tmem_cols=" +
-          S(sh.tmem_cols) + " stages=" + S(NS) + " stage_bytes=" + S(sh.stage_bytes) +
-          " entries=" + S(ent.size()) + " producer_threads=" + S(PR) + " warps=4 consumers + 2 producers");
+          " paths=" + S(pl.paths.size()) + " dtype=f16 ncols=" + S(sh.ncols) + " tbufs=" + S(NT) +
+          " tstride=" + S(sh.tstride) + " bbufs=" + S(NBUF) + " stages=" + S(NS) + " stage_bytes=" + S(sh.stage_bytes) +
+          " entries=" + S(ent.size()) + " producer_threads=" + S(BT) +
+          " group_cols=" + S(gcol[1] - gcol[0]) + "," + S(gcol[2] - gcol[1]));
   em.o << tab.source;
   em.line("__device__ __forceinline__ float h2f(unsigned short h) { float f; asm(\"cvt.f32.f16 %0, %1;\" : \"=f\"(f) : \"h\"(h)); return f; }");
   em.line("__device__ __forceinline__ unsigned short f2h(float f) { unsigned short h; asm(\"cvt.rn.f16.f32 %0, %1;\" : \"=h\"(h) : \"f\"(f)); return h; }");
@@ -1052,20 +1098,30 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("  unsigned int ok; asm volatile(\"{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }\" : \"=r\"(ok) : \"r\"(smem_u32(b)), \"r\"(parity) : \"memory\"); return ok != 0; }");
   em.line("__device__ __forceinline__ bool bar_wait(unsigned long long* b, unsigned int parity) {");
   em.line("  for (unsigned int it = 0; it < E3_SPIN_LIMIT; ++it) if (bar_try(b, parity)) return true; return false; }");
+  em.line("// bounded wait agreed by the warp (a lane that gave up makes the whole warp give up)");
+  em.line("__device__ __forceinline__ bool warp_wait(unsigned long long* b, unsigned int parity) { return __all_sync(0xffffffffu, bar_wait(b, parity)); }");
+  em.line("__device__ __forceinline__ void warp_arrive(unsigned long long* b, int lane) { __syncwarp(); if (lane == 0) bar_arrive(b); }");
   em.line("__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned int bytes, unsigned long long* b, unsigned long long policy) {");
   em.line("  asm volatile(\"cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;\" :: \"r\"(smem_u32(dst)), \"l\"(src), \"r\"(bytes), \"r\"(smem_u32(b)), \"l\"(policy) : \"memory\"); }");
-  em.line("__device__ __forceinline__ void tma2d_g2s(void* dst, const E3TensorMap* map, int c0, int c1, unsigned long long* b, unsigned long long policy) {");
-  em.line("  asm volatile(\"cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;\" :: \"r\"(smem_u32(dst)), \"l\"(map), \"r\"(c0), \"r\"(c1), \"r\"(smem_u32(b)), \"l\"(policy) : \"memory\"); }");
+  em.line("// the sender's tile: box {64 channels, 16 rows, 2 halves} of node `node` (rows >= nx zero-filled)");
+  em.line("__device__ __forceinline__ void tma_x_g2s(void* dst, const E3TensorMap* map, int node, unsigned long long* b, unsigned long long policy) {");
+  em.line("  asm volatile(\"cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %2, %2, %3}], [%4], %5;\" :: \"r\"(smem_u32(dst)), \"l\"(map), \"r\"(0), \"r\"(node), \"r\"(smem_u32(b)), \"l\"(policy) : \"memory\"); }");
   em.line("__device__ __forceinline__ unsigned long long policy_evict_first() { unsigned long long p; asm volatile(\"createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\" : \"=l\"(p)); return p; }");
   em.line("__device__ __forceinline__ unsigned long long policy_evict_last() { unsigned long long p; asm volatile(\"createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\" : \"=l\"(p)); return p; }");
   em.line("__device__ __forceinline__ void fence_async_smem() { asm volatile(\"fence.proxy.async.shared::cta;\" ::: \"memory\"); }");
-  em.line("__device__ __forceinline__ void prod_sync() { asm volatile(\"bar.sync 2, 64;\" ::: \"memory\"); }");
-  em.line("__device__ __forceinline__ bool prod_all(bool ok) { unsigned int r; asm volatile(\"{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.and.pred q, 2, 64, p; selp.u32 %0, 1, 0, q; }\" : \"=r\"(r) : \"r\"((unsigned int)ok) : \"memory\"); return r != 0u; }");
-  em.line("__device__ __forceinline__ bool cons_all(bool ok) { unsigned int r; asm volatile(\"{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.and.pred q, 3, 128, p; selp.u32 %0, 1, 0, q; }\" : \"=r\"(r) : \"r\"((unsigned int)ok) : \"memory\"); return r != 0u; }");
   em.line("__device__ __forceinline__ void tc_before() { asm volatile(\"tcgen05.fence::before_thread_sync;\" ::: \"memory\"); }");
   em.line("__device__ __forceinline__ void tc_after() { asm volatile(\"tcgen05.fence::after_thread_sync;\" ::: \"memory\"); }");
-  em.line("#define TMEM_LD32(addr, r) asm volatile(\"tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\" : \"=r\"(r[0]), \"=r\"(r[1]), \"=r\"(r[2]), \"=r\"(r[3]), \"=r\"(r[4]), \"=r\"(r[5]), \"=r\"(r[6]), \"=r\"(r[7]), \"=r\"(r[8]), \"=r\"(r[9]), \"=r\"(r[10]), \"=r\"(r[11]), \"=r\"(r[12]), \"=r\"(r[13]), \"=r\"(r[14]), \"=r\"(r[15]), \"=r\"(r[16]), \"=r\"(r[17]), \"=r\"(r[18]), \"=r\"(r[19]), \"=r\"(r[20]), \"=r\"(r[21]), \"=r\"(r[22]), \"=r\"(r[23]), \"=r\"(r[24]), \"=r\"(r[25]), \"=r\"(r[26]), \"=r\"(r[27]), \"=r\"(r[28]), \"=r\"(r[29]), \"=r\"(r[30]), \"=r\"(r[31]) : \"r\"(addr))");
-  em.line("extern \"C\" __global__ void __launch_bounds__(192, 1) e3conv_fwd(");
+  // tensor-memory loads of 1..32 columns (32 lanes x 32 bit)
+  for (int n = 1; n <= 32; n *= 2) {
+    std::string regs, outs;
+    for (int r = 0; r < n; ++r) {
+      regs += std::string(r ? "," : "") + "%" + S(r);
+      outs += std::string(r ? ", " : "") + "\"=r\"(r[" + S(r) + "])";
+    }
+    em.line("#define TMEM_LD" + S(n) + "(addr, r) asm volatile(\"tcgen05.ld.sync.aligned.32x32b.x" + S(n) +
+            ".b32 {" + regs + "}, [%" + S(n) + "];\" : " + outs + " : \"r\"(addr))");
+  }
+  em.line("extern \"C\" __global__ void __launch_bounds__(" + S(sh.block) + ", 1) e3conv_fwd(");
   em.line("    const unsigned short* __restrict__ x, const unsigned short* __restrict__ Y,");
   em.line("    const unsigned short* __restrict__ s, const int* __restrict__ senders,");
   em.line("    const int* __restrict__ row_ptr, int num_nodes, int num_edges, float* __restrict__ out,");
@@ -1074,22 +1130,21 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.ind++;
   em.line("extern __shared__ __align__(1024) unsigned char smem[];");
   em.line("const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;");
-  em.line("unsigned char* tbase = smem;");
-  em.line("unsigned long long* sfull = reinterpret_cast<unsigned long long*>(tbase + " + S(sh.bar_off) + ");");
-  em.line("unsigned long long* sempty = sfull + " + S(NS) + ";");
-  em.line("unsigned long long* bfree = sempty + " + S(NS) + ";");
-  em.line("unsigned long long* tfull = bfree + 2;");
-  em.line("unsigned long long* tempty = tfull + 2;");
-  em.line("int* hdr = reinterpret_cast<int*>(tbase + " + S(sh.hdr_off) + ");  // per stage: sender (-1 invalid, -2 end), receiver, last");
-  em.line("unsigned int* tslot = reinterpret_cast<unsigned int*>(tbase + " + S(sh.tslot_off) + ");");
-  em.line("float* yf = reinterpret_cast<float*>(tbase + " + S(sh.yf_off) + ");");
-  em.line("unsigned char* Bt = tbase + " + S(sh.b_off) + ";  // buffer bb: A_hi at bb*" + S(2 * sh.b_bytes) + ", A_lo at +" + S(sh.b_bytes));
-  em.line("for (int q = tid; q < " + S(4 * sh.b_bytes / 16) + "; q += 192) reinterpret_cast<uint4*>(Bt)[q] = make_uint4(0u, 0u, 0u, 0u);");
+  em.line("unsigned long long* sfull = reinterpret_cast<unsigned long long*>(smem + " + S(sh.bar_off) + ");");
+  em.line("unsigned long long* sempty = sfull + " + S(NS) + ";   // 8 consumer + 4 builder warps + the MMA warp");
+  em.line("unsigned long long* bfull = sempty + " + S(NS) + ";   // 4 builder warps");
+  em.line("unsigned long long* tfull = bfull + " + S(NBUF) + ";      // MMA completion (T ready, A tile free)");
+  em.line("unsigned long long* tempty = tfull + " + S(NT) + ";  // 8 consumer warps");
+  em.line("int* hdr = reinterpret_cast<int*>(smem + " + S(sh.hdr_off) + ");  // per stage: sender (-1 invalid, -2 end), receiver, last");
+  em.line("unsigned int* tslot = reinterpret_cast<unsigned int*>(smem + " + S(sh.tslot_off) + ");");
+  em.line("unsigned char* Bt = smem + " + S(sh.b_off) + ";  // buffer bb: A_hi at bb*" + S(2 * BS) + ", A_lo at +" + S(BS) + "; bytes " + S(sh.b_bytes) + ".. of each are scratch");
+  em.line("for (int q = tid; q < " + S(2 * NBUF * BS / 16) + "; q += " + S(sh.block) + ") reinterpret_cast<uint4*>(Bt)[q] = make_uint4(0u, 0u, 0u, 0u);");
   em.line("for (int k = 0; k < " + S(NS) + "; ++k)");
-  em.line("  for (int q = tid; q < 256; q += 192) reinterpret_cast<uint4*>(tbase + k * " + S(sh.stage_bytes) + ")[q] = make_uint4(0u, 0u, 0u, 0u);");
+  em.line("  for (int q = tid; q < 256; q += " + S(sh.block) + ") reinterpret_cast<uint4*>(smem + k * " + S(sh.stage_bytes) + ")[q] = make_uint4(0u, 0u, 0u, 0u);");
   em.line("if (tid == 0) {");
-  em.line("  for (int k = 0; k < " + S(NS) + "; ++k) { bar_init(sfull + k, 1u); bar_init(sempty + k, 128u); }");
-  em.line("  for (int k = 0; k < 2; ++k) { bar_init(bfree + k, 1u); bar_init(tfull + k, 1u); bar_init(tempty + k, 128u); }");
+  em.line("  for (int k = 0; k < " + S(NS) + "; ++k) { bar_init(sfull + k, 1u); bar_init(sempty + k, 13u); }");
+  em.line("  for (int k = 0; k < " + S(NBUF) + "; ++k) bar_init(bfull + k, " + S(NB) + "u);");
+  em.line("  for (int k = 0; k < " + S(NT) + "; ++k) { bar_init(tfull + k, 1u); bar_init(tempty + k, 8u); }");
   em.line("  asm volatile(\"fence.mbarrier_init.release.cluster;\" ::: \"memory\");");
   em.line("}");
   em.line("if (warp == 0) {");
@@ -1102,196 +1157,266 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("tc_after();");
   em.line("const unsigned int tmem = *tslot;");
   em.line("const long long W = (long long)gridDim.x;");
-  em.line("if (warp >= 4) {");
+
+  // ---------------- copy warps ----------------
+  em.line("if (warp == " + S(W_COPY) + " || warp == " + S(W_COPY + 1) + ") {");
   em.ind++;
-  // ---------------- producers ----------------
-  em.line("// producers: row walk, copies, A tiles, MMA issue");
-  em.line("const int pt = tid - 128;  // 0..63");
-  em.line("const bool issuer = pt == 0;");
+  em.line("const unsigned int cw = (unsigned int)(warp - " + S(W_COPY) + ");  // ring positions q with q % 2 == cw");
   em.line("const unsigned long long pol_stream = policy_evict_first();");
   em.line("const unsigned long long pol_keep = policy_evict_last();");
-  em.line("const unsigned int idesc = (1u << 4) | (1u << 15) | ((unsigned int)(" + S(sh.ncols) + " >> 3) << 17) | ((unsigned int)(128 >> 4) << 24);");
-  em.line("long long pb = (long long)blockIdx.x - W;");
-  em.line("int pe = 0, pe1 = 0, pwin = -1, psw = 0;");
-  em.line("bool walk_done = false, ok = true;");
-  em.line("unsigned int qi = 0, qm = 0, v = 0;  // next position to copy, next position to multiply, valid edges multiplied");
-  em.line("#pragma unroll 1");
-  em.line("while (ok) {");
-  em.ind++;
-  em.line("// copies for positions ahead of the MMA cursor (ring of " + S(NS) + " stages, two kept");
-  em.line("// for the consumers so this wait targets an edge they have already finished)");
-  em.line("#pragma unroll 1");
-  em.line("while (ok && !walk_done && qi < qm + " + S(NS - 2) + ") {");
-  em.ind++;
-  em.line("const unsigned int st = qi % " + S(NS) + ";");
-  em.line("if (qi >= " + S(NS) + "u) { ok = prod_all(bar_wait(sempty + st, ((qi / " + S(NS) + ") - 1u) & 1u)); if (!ok) break; }");
-  em.line("while (pe >= pe1) {");
-  em.line("  pb += W;");
-  em.line("  if (pb >= num_nodes) { walk_done = true; break; }");
-  em.line("  int r0 = row_ptr[pb], r1 = row_ptr[pb + 1];");
-  em.line("  if (r0 < 0 || r1 < r0 || r1 > num_edges) { if (issuer) atomicOr(status, 1u); r1 = r0; }");
-  em.line("  pe = r0; pe1 = r1; pwin = -1;");
-  em.line("  if (r0 == r1) {");
-  em.line("    float* zrow = out + pb * " + S(o_row) + ";");
-  em.line("    for (int q = pt; q < " + S(o_row) + "; q += 64) zrow[q] = 0.f;");
-  em.line("  }");
+  em.line("// row walk with loads one row ahead: the open row [pe, pe1) of receiver pb with its");
+  em.line("// sender windows psw (edges pwin..pwin+31) and psw2 (the next 32); the next row nb");
+  em.line("// [n0, n1) with its first window nsw in flight; row_ptr of the row after (mb) in flight");
+  em.line("long long pb = -1, nb = blockIdx.x, mb = (long long)blockIdx.x + W;");
+  em.line("int pe = 0, pe1 = 0, pwin = 0, psw = 0, psw2 = 0;");
+  em.line("int n0 = 0, n1 = 0, nsw = 0, nsw2 = 0, m0 = 0, m1 = 0;");
+  em.line("if (nb < num_nodes) {");
+  em.line("  n0 = row_ptr[nb]; n1 = row_ptr[nb + 1];");
+  em.line("  if (n0 < 0 || n1 < n0 || n1 > num_edges) { if (lane == 0) atomicOr(status, 1u); n1 = n0; }");
+  em.line("  nsw = (n0 + lane < n1) ? senders[n0 + lane] : 0;");
+  em.line("  nsw2 = (n0 + 32 + lane < n1) ? senders[n0 + 32 + lane] : 0;");
   em.line("}");
-  em.line("if (walk_done) {");
-  em.line("  if (issuer) { hdr[4 * st] = -2; bar_arrive(sfull + st); }  // end marker");
-  em.line("  ++qi;");
+  em.line("if (mb < num_nodes) { m0 = row_ptr[mb]; m1 = row_ptr[mb + 1]; }");
+  em.line("unsigned int q = 0;");
+  em.line("bool ok = true;");
+  em.line("#pragma unroll 1");
+  em.line("while (true) {");
+  em.ind++;
+  em.line("const unsigned int st = q % " + S(NS) + ";");
+  em.line("const bool mine = (q & 1u) == cw;");
+  em.line("if (mine && q >= " + S(NS) + "u) { ok = warp_wait(sempty + st, ((q / " + S(NS) + ") - 1u) & 1u); if (!ok) break; }");
+  em.line("bool done = false;");
+  em.line("while (pe >= pe1) {  // open the next row");
+  em.line("  pb = nb;");
+  em.line("  if (pb >= num_nodes) { done = true; break; }");
+  em.line("  pe = n0; pe1 = n1; pwin = n0; psw = nsw; psw2 = nsw2;");
+  em.line("  if (pe == pe1) {");
+  em.line("    float* zrow = out + pb * " + S(o_row) + ";");
+  em.line("    if (cw == 0u) for (int k = lane; k < " + S(o_row) + "; k += 32) zrow[k] = 0.f;");
+  em.line("  }");
+  em.line("  nb = mb; n0 = m0; n1 = m1;");
+  em.line("  if (nb < num_nodes) {");
+  em.line("    if (n0 < 0 || n1 < n0 || n1 > num_edges) { if (lane == 0) atomicOr(status, 1u); n1 = n0; }");
+  em.line("    nsw = (n0 + lane < n1) ? senders[n0 + lane] : 0;");
+  em.line("    nsw2 = (n0 + 32 + lane < n1) ? senders[n0 + 32 + lane] : 0;");
+  em.line("  }");
+  em.line("  mb = nb + W;");
+  em.line("  if (mb < num_nodes) { m0 = row_ptr[mb]; m1 = row_ptr[mb + 1]; }");
+  em.line("}");
+  em.line("if (done) {");
+  em.line("  if (mine && lane == 0) { hdr[4 * st] = -2; bar_arrive(sfull + st); }  // end marker");
+  em.line("  ++q;");
   em.line("  break;");
   em.line("}");
-  em.line("if (pwin < 0 || pe >= pwin + 32) { pwin = pe; psw = (pe + lane < pe1) ? senders[pe + lane] : 0; }");
+  em.line("if (pe >= pwin + 32) {  // next window of the row");
+  em.line("  pwin += 32; psw = psw2;");
+  em.line("  psw2 = (pwin + 32 + lane < pe1) ? senders[pwin + 32 + lane] : 0;");
+  em.line("}");
   em.line("const int a = __shfl_sync(0xffffffffu, psw, pe - pwin);");
   em.line("const bool valid = (unsigned int)a < (unsigned int)num_nodes;");
-  em.line("if (issuer) {");
-  em.line("  unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
+  em.line("if (mine && lane == 0) {");
+  em.line("  unsigned char* stg = smem + st * " + S(sh.stage_bytes) + ";");
   em.line("  hdr[4 * st] = valid ? a : -1;");
   em.line("  hdr[4 * st + 1] = (int)pb;");
   em.line("  hdr[4 * st + 2] = (pe + 1 == pe1) ? 1 : 0;");
-  em.line("  fence_async_smem();");
-  em.line("  bar_expect(sfull + st, " + S(sh.s_bytes + sh.y_bytes) + "u + (valid ? " + S(sh.x_bytes) + "u : 0u));");
+  em.line("  bar_expect(sfull + st, " + S(sh.s_bytes + sh.y_bytes) + "u + (valid ? 4096u : 0u));");
   em.line("  bulk_g2s(stg + " + S(sh.s_off) + ", s + (long long)pe * " + S(s_row) + ", " + S(sh.s_bytes) + "u, sfull + st, pol_stream);");
   em.line("  bulk_g2s(stg + " + S(sh.y_off) + ", Y + (long long)pe * " + S(pl.ny) + ", " + S(sh.y_bytes) + "u, sfull + st, pol_stream);");
-  em.line("  if (valid) {");
-  em.line("    tma2d_g2s(stg, &xmap, 0, a * " + S(pl.nx) + ", sfull + st, pol_keep);");
-  em.line("    tma2d_g2s(stg + 2048, &xmap, 64, a * " + S(pl.nx) + ", sfull + st, pol_keep);");
-  em.line("  }");
+  em.line("  if (valid) tma_x_g2s(stg, &xmap, a, sfull + st, pol_keep);");
   em.line("}");
+  em.line("__syncwarp();");
   em.line("++pe;");
-  em.line("++qi;");
+  em.line("++q;");
   em.ind--;
   em.line("}");
-  em.line("if (!ok || qm == qi) break;");
-  em.line("// position qm: wait for its copies, build A, multiply");
-  em.line("const unsigned int st = qm % " + S(NS) + ";");
-  em.line("ok = prod_all(bar_wait(sfull + st, (qm / " + S(NS) + ") & 1u));");
-  em.line("if (!ok) break;");
-  em.line("const int a = hdr[4 * st];");
-  em.line("if (a == -2) break;");
-  em.line("if (a >= 0) {");
+  em.line("if (!ok && lane == 0) atomicOr(status, 4u);");
+  em.line("// drain: this warp's copies of the last positions land before the block leaves (bounded)");
+  em.line("if (lane == 0)");
+  em.line("  for (unsigned int k = q > " + S(NS) + "u ? q - " + S(NS) + "u : 0u; k < q; ++k)");
+  em.line("    if ((k & 1u) == cw) bar_wait(sfull + k % " + S(NS) + ", (k / " + S(NS) + ") & 1u);");
+  em.ind--;
+  // ---------------- MMA warp ----------------
+  em.line("} else if (warp == " + S(W_MMA) + ") {");
   em.ind++;
-  em.line("const unsigned int bb = v & 1u;");
-  em.line("if (v >= 2u) { ok = prod_all(bar_wait(bfree + bb, ((v >> 1) - 1u) & 1u)); if (!ok) break; }");
-  em.line("unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
-  em.line("unsigned char* Bhi = Bt + bb * " + S(2 * sh.b_bytes) + ";");
-  em.line("unsigned char* Blo = Bhi + " + S(sh.b_bytes) + ";");
-  em.line("if (pt < " + S(pl.ny) + ") yf[pt] = h2f(reinterpret_cast<const unsigned short*>(stg + " + S(sh.y_off) + ")[pt]);");
-  em.line("prod_sync();");
-  int base = 0;
-  for (int r = 0; r < tab.rounds; ++r) {
-    em.line("{");
-    em.ind++;
-    for (int t2 = 0; t2 < tab.terms[r]; ++t2)
-      em.line("const int2 k" + S(t2) + " = __ldg(&e3_btab[" + S(base + t2 * PR) + " + pt]);");
-    std::string val = "__int_as_float(k0.x) * yf[k0.y]";
-    for (int t2 = 1; t2 < tab.terms[r]; ++t2)
-      val = "fmaf(__int_as_float(k" + S(t2) + ".x), yf[k" + S(t2) + ".y], " + val + ")";
-    em.line("const int off = __ldg(&e3_boff[" + S(r * PR) + " + pt]);");
-    em.line("if (off >= 0) {");
-    em.line("  const float val = " + val + ";");
-    em.line("  const unsigned short hi = f2h(val);");
-    em.line("  *reinterpret_cast<unsigned short*>(Bhi + off) = hi;");
-    em.line("  *reinterpret_cast<unsigned short*>(Blo + off) = f2h(val - h2f(hi));");
-    em.line("}");
-    em.ind--;
-    em.line("}");
-    base += tab.terms[r] * PR;
-  }
-  em.line("fence_async_smem();");
-  em.line("prod_sync();");
-  em.line("const unsigned int tb = v & 1u;");
-  em.line("if (v >= 2u) { ok = prod_all(bar_wait(tempty + tb, ((v >> 1) - 1u) & 1u)); if (!ok) break; }");
-  em.line("tc_after();");
-  em.line("if (issuer) {");
-  em.line("  const unsigned long long adesc = (unsigned long long)((smem_u32(stg) & 0x3FFFF) >> 4) | (128ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);");
-  em.line("  const unsigned long long hdesc = (unsigned long long)((smem_u32(Bhi) & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
-  em.line("  const unsigned long long ldesc = (unsigned long long)((smem_u32(Blo) & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
-  em.line("  const unsigned int dt = tmem + tb * 256u;");
-  em.line("  asm volatile(\"{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }\" :: \"r\"(dt), \"l\"(adesc), \"l\"(hdesc), \"r\"(idesc), \"r\"(0u) : \"memory\");");
-  em.line("  asm volatile(\"{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }\" :: \"r\"(dt), \"l\"(adesc), \"l\"(ldesc), \"r\"(idesc), \"r\"(1u) : \"memory\");");
-  em.line("  asm volatile(\"tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\" :: \"r\"(smem_u32(tfull + tb)) : \"memory\");");
-  em.line("  asm volatile(\"tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\" :: \"r\"(smem_u32(bfree + bb)) : \"memory\");");
-  em.line("}");
-  em.line("++v;");
-  em.ind--;
-  em.line("}");
-  em.line("++qm;");
-  em.ind--;
-  em.line("}");
-  em.line("if (!ok && issuer) atomicOr(status, 4u);");
-  em.line("// drain: every issued copy and MMA completes before the block leaves (bounded)");
-  em.line("if (issuer) {");
-  em.line("  for (unsigned int q = qm; q < qi; ++q) bar_wait(sfull + q % " + S(NS) + ", (q / " + S(NS) + ") & 1u);");
-  em.line("  if (v > 0u) bar_wait(bfree + ((v - 1u) & 1u), ((v - 1u) >> 1) & 1u);");
-  em.line("}");
-  em.ind--;
-  em.line("} else {");
-  em.ind++;
-  // ---------------- consumers ----------------
-  em.line("// consumers: thread tid owns channel tid; tensor-memory lanes 32*warp .. 32*warp+31");
-  {
-    std::string decl = "float";
-    for (int c = 0; c < pl.nout; ++c) decl += std::string(c ? "," : "") + " a" + S(c) + " = 0.f";
-    em.line(decl + ";");
-  }
-  em.line("const unsigned int tmem_lane = tmem + ((unsigned int)(warp * 32) << 16);");
+  em.line("const unsigned int idesc = (1u << 4) | (1u << 15) | ((unsigned int)(" + S(sh.ncols) + " >> 3) << 17) | ((unsigned int)(128 >> 4) << 24);");
   em.line("unsigned int q = 0, v = 0;");
   em.line("bool ok = true;");
   em.line("#pragma unroll 1");
   em.line("while (true) {");
   em.ind++;
   em.line("const unsigned int st = q % " + S(NS) + ";");
-  em.line("ok = cons_all(bar_wait(sfull + st, (q / " + S(NS) + ") & 1u));");
+  em.line("ok = warp_wait(sfull + st, (q / " + S(NS) + ") & 1u);");
   em.line("if (!ok) break;");
-  em.line("unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
   em.line("const int a = hdr[4 * st];");
   em.line("if (a == -2) break;");
-  em.line("const long long b = hdr[4 * st + 1];");
-  em.line("const int last = hdr[4 * st + 2];");
   em.line("if (a >= 0) {");
   em.ind++;
-  em.line("const unsigned int tb = v & 1u;");
-  em.line("ok = cons_all(bar_wait(tfull + tb, (v >> 1) & 1u));");
+  em.line("const unsigned int tb = v % " + S(NT) + "u;");
+  em.line("ok = warp_wait(bfull + tb, (v / " + S(NT) + "u) & 1u);");
   em.line("if (!ok) break;");
+  em.line("if (v >= " + S(NT) + "u) { ok = warp_wait(tempty + tb, ((v / " + S(NT) + "u) - 1u) & 1u); if (!ok) break; }");
   em.line("tc_after();");
-  em.line("const unsigned short* sv = reinterpret_cast<const unsigned short*>(stg + " + S(sh.s_off) + ") + tid;");
-  em.line("const unsigned int tcol = tmem_lane + tb * 256u;");
-  {
-    std::vector<std::pair<int, int>> colmap;
-    for (size_t p = 0; p < pl.paths.size(); ++p)
-      for (int k = 0; k < 2 * pl.paths[p].l3 + 1; ++k) colmap.push_back({static_cast<int>(p), k});
-    const int nchunk = (static_cast<int>(colmap.size()) + 31) / 32;
-    // edge scalars first (shared-memory loads overlap the tensor-memory loads)
-    for (size_t p = 0; p < pl.paths.size(); ++p)
-      em.line("const float s" + S(p) + " = h2f(sv[" + S(static_cast<long long>(p) * pl.C) + "]);");
-    for (int c = 0; c < nchunk; ++c) {
-      em.line("unsigned int r" + S(c) + "[32];");
-      em.line("TMEM_LD32(tcol + " + S(32 * c) + "u, r" + S(c) + ");");
-    }
-    em.line("asm volatile(\"tcgen05.wait::ld.sync.aligned;\" ::: \"memory\");");
-    em.line("tc_before();");
-    em.line("bar_arrive(tempty + tb);  // T is in registers: the buffer is free for the next MMA");
-    for (int cc = 0; cc < static_cast<int>(colmap.size()); ++cc) {
-      const int p = colmap[cc].first, k = colmap[cc].second;
-      const std::string acc = "a" + S(pl.paths[p].out_off + k);
-      em.line(acc + " = fmaf(s" + S(p) + ", __uint_as_float(r" + S(cc / 32) + "[" + S(cc % 32) + "]), " + acc + ");");
-    }
-  }
+  em.line("if (lane == 0) {");
+  em.line("  const unsigned char* stg = smem + st * " + S(sh.stage_bytes) + ";");
+  em.line("  const unsigned char* Bhi = Bt + tb * " + S(2 * BS) + ";");
+  em.line("  const unsigned long long adesc = (unsigned long long)((smem_u32(stg) & 0x3FFFF) >> 4) | (128ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);");
+  em.line("  const unsigned long long hdesc = (unsigned long long)((smem_u32(Bhi) & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
+  em.line("  const unsigned long long ldesc = (unsigned long long)((smem_u32(Bhi + " + S(BS) + ") & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
+  em.line("  const unsigned int dt = tmem + tb * " + S(sh.tstride) + "u;");
+  em.line("  asm volatile(\"{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }\" :: \"r\"(dt), \"l\"(adesc), \"l\"(hdesc), \"r\"(idesc), \"r\"(0u) : \"memory\");");
+  em.line("  asm volatile(\"{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }\" :: \"r\"(dt), \"l\"(adesc), \"l\"(ldesc), \"r\"(idesc), \"r\"(1u) : \"memory\");");
+  em.line("  asm volatile(\"tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\" :: \"r\"(smem_u32(tfull + tb)) : \"memory\");");
+  em.line("}");
   em.line("++v;");
   em.ind--;
-  em.line("} else if (tid == 0) {");
-  em.line("  atomicOr(status, 2u);");
   em.line("}");
-  em.line("bar_arrive(sempty + st);");
-  em.line("if (last) {");
-  em.line("  float* orow = out + b * " + S(o_row) + " + tid;");
-  for (int c = 0; c < pl.nout; ++c) em.line("  orow[" + S(c * pl.C) + "] = a" + S(c) + " * inv_avg; a" + S(c) + " = 0.f;");
+  em.line("warp_arrive(sempty + st, lane);");
+  em.line("++q;");
+  em.ind--;
+  em.line("}");
+  em.line("if (!ok && lane == 0) atomicOr(status, 4u);");
+  em.line("// drain: the last MMAs complete before tensor memory is released (bounded)");
+  em.line("if (lane == 0 && v > 0u) bar_wait(tfull + (v - 1u) % " + S(NT) + "u, ((v - 1u) / " + S(NT) + "u) & 1u);");
+  em.ind--;
+  // ---------------- builder warps ----------------
+  em.line("} else if (warp >= " + S(W_B) + ") {");
+  em.ind++;
+  em.line("const int bt = tid - " + S(TID_B) + ";  // 0.." + S(BT - 1));
+  em.line("float* yfw = reinterpret_cast<float*>(smem + " + S(sh.yf_off) + ") + (warp - " + S(W_B) + ") * " + S(align_up(pl.ny, 4)) + ";");
+  {
+    int base = 0;
+    for (int r = 0; r < tab.rounds; ++r) {
+      for (int t2 = 0; t2 < tab.terms[r]; ++t2)
+        em.line("const int2 k" + S(r) + "_" + S(t2) + " = __ldg(&e3_btab[" + S(base + t2 * BT) + " + bt]);");
+      em.line("const int off" + S(r) + " = __ldg(&e3_boff[" + S(r * BT) + " + bt]) >= 0 ? __ldg(&e3_boff[" + S(r * BT) + " + bt]) : " + S(sh.b_bytes) + ";  // padding lanes write the scratch bytes");
+      base += tab.terms[r] * BT;
+    }
+  }
+  em.line("unsigned int q = 0, v = 0;");
+  em.line("bool ok = true;");
+  em.line("#pragma unroll 1");
+  em.line("while (true) {");
+  em.ind++;
+  em.line("const unsigned int st = q % " + S(NS) + ";");
+  em.line("ok = warp_wait(sfull + st, (q / " + S(NS) + ") & 1u);");
+  em.line("if (!ok) break;");
+  em.line("const int a = hdr[4 * st];");
+  em.line("if (a == -2) break;");
+  em.line("if (a >= 0) {");
+  em.ind++;
+  em.line("const unsigned short* ys = reinterpret_cast<const unsigned short*>(smem + st * " + S(sh.stage_bytes) + " + " + S(sh.y_off) + ");");
+  em.line("for (int j = lane; j < " + S(pl.ny) + "; j += 32) yfw[j] = h2f(ys[j]);");
+  em.line("warp_arrive(sempty + st, lane);  // Y is in this warp's buffer");
+  em.line("const unsigned int bb = v % " + S(NBUF) + "u;");
+  em.line("if (v >= " + S(NBUF) + "u) { ok = warp_wait(tfull + bb, ((v / " + S(NBUF) + "u) - 1u) & 1u); if (!ok) break; }  // MMA v-" + S(NBUF) + " done");
+  em.line("unsigned char* Bhi = Bt + bb * " + S(2 * BS) + ";");
+  em.line("unsigned char* Blo = Bhi + " + S(BS) + ";");
+  for (int r = 0; r < tab.rounds; ++r) {
+    std::string val = "__int_as_float(k" + S(r) + "_0.x) * yfw[k" + S(r) + "_0.y]";
+    for (int t2 = 1; t2 < tab.terms[r]; ++t2)
+      val = "fmaf(__int_as_float(k" + S(r) + "_" + S(t2) + ".x), yfw[k" + S(r) + "_" + S(t2) + ".y], " + val + ")";
+    em.line("{");
+    em.line("  const float val = " + val + ";");
+    em.line("  const unsigned short hi = f2h(val);");
+    em.line("  *reinterpret_cast<unsigned short*>(Bhi + off" + S(r) + ") = hi;");
+    em.line("  *reinterpret_cast<unsigned short*>(Blo + off" + S(r) + ") = f2h(val - h2f(hi));");
+    em.line("}");
+  }
+  em.line("fence_async_smem();");
+  em.line("warp_arrive(bfull + bb, lane);");
+  em.line("++v;");
+  em.ind--;
+  em.line("} else {");
+  em.line("  warp_arrive(sempty + st, lane);");
   em.line("}");
   em.line("++q;");
   em.ind--;
   em.line("}");
-  em.line("if (!ok && tid == 0) atomicOr(status, 4u);");
+  em.line("if (!ok && lane == 0) atomicOr(status, 4u);");
+  em.ind--;
+  // ---------------- consumer warps ----------------
+  em.line("} else {");
+  em.ind++;
+  em.line("const int c = 32 * (warp & 3) + lane;  // channel = tensor-memory lane");
+  em.line("const unsigned int tmem_lane = tmem + ((unsigned int)(32 * (warp & 3)) << 16);");
+  em.line("unsigned int q = 0, v = 0;");
+  em.line("bool ok = true;");
+  for (int g = 0; g < 2; ++g) {
+    std::vector<int> outs;
+    for (size_t o = 0; o < pl.outputs.size(); ++o)
+      if (og[o] == g)
+        for (int k = 0; k < 2 * pl.outputs[o].l + 1; ++k) outs.push_back(pl.outputs[o].off + k);
+    std::vector<std::pair<int, int>> chunks;  // (start column, width), start a multiple of width
+    for (int pos = gcol[g]; pos < gcol[g + 1];) {
+      int w = 32;
+      while (w > 1 && (pos % w != 0 || pos + w > gcol[g + 1])) w /= 2;
+      chunks.push_back({pos, w});
+      pos += w;
+    }
+    em.line(std::string(g ? "} else {" : "if (warp < 4) {") + "  // output group " + S(g) + ": columns " +
+            S(gcol[g]) + ".." + S(gcol[g + 1] - 1));
+    em.ind++;
+    {
+      std::string decl = "float";
+      for (size_t k = 0; k < outs.size(); ++k) decl += std::string(k ? "," : "") + " a" + S(outs[k]) + " = 0.f";
+      if (!outs.empty()) em.line(decl + ";");
+    }
+    em.line("#pragma unroll 1");
+    em.line("while (true) {");
+    em.ind++;
+    em.line("const unsigned int st = q % " + S(NS) + ";");
+    em.line("ok = warp_wait(sfull + st, (q / " + S(NS) + ") & 1u);");
+    em.line("if (!ok) break;");
+    em.line("const int a = hdr[4 * st];");
+    em.line("if (a == -2) break;");
+    em.line("const long long b = hdr[4 * st + 1];");
+    em.line("const int last = hdr[4 * st + 2];");
+    em.line("if (a >= 0) {");
+    em.ind++;
+    em.line("const unsigned short* sv = reinterpret_cast<const unsigned short*>(smem + st * " + S(sh.stage_bytes) + " + " + S(sh.s_off) + ") + c;");
+    for (size_t p = 0; p < pl.paths.size(); ++p)
+      if (og[pl.paths[p].o] == g)
+        em.line("const float s" + S(p) + " = h2f(sv[" + S(static_cast<long long>(p) * pl.C) + "]);");
+    em.line("const unsigned int tb = v % " + S(NT) + "u;");
+    em.line("ok = warp_wait(tfull + tb, (v / " + S(NT) + "u) & 1u);");
+    em.line("if (!ok) break;");
+    em.line("warp_arrive(sempty + st, lane);  // s is in registers and the MMA has read x");
+    em.line("tc_after();");
+    em.line("const unsigned int tcol = tmem_lane + tb * " + S(sh.tstride) + "u;");
+    for (size_t k = 0; k < chunks.size(); ++k) {
+      em.line("unsigned int r" + S(k) + "[" + S(chunks[k].second) + "];");
+      em.line("TMEM_LD" + S(chunks[k].second) + "(tcol + " + S(chunks[k].first) + "u, r" + S(k) + ");");
+    }
+    em.line("asm volatile(\"tcgen05.wait::ld.sync.aligned;\" ::: \"memory\");");
+    em.line("tc_before();");
+    em.line("warp_arrive(tempty + tb, lane);  // T is in registers: the buffer is free for the next MMA");
+    for (size_t p = 0; p < pl.paths.size(); ++p) {
+      if (og[pl.paths[p].o] != g) continue;
+      for (int k = 0; k < 2 * pl.paths[p].l3 + 1; ++k) {
+        const int colm = colbase[p] + k;
+        size_t ch = 0;
+        while (!(colm >= chunks[ch].first && colm < chunks[ch].first + chunks[ch].second)) ++ch;
+        const std::string acc = "a" + S(pl.paths[p].out_off + k);
+        em.line(acc + " = fmaf(s" + S(p) + ", __uint_as_float(r" + S(ch) + "[" + S(colm - chunks[ch].first) + "]), " + acc + ");");
+      }
+    }
+    em.line("++v;");
+    em.ind--;
+    em.line("} else {");
+    em.line("  if (tid == 0) atomicOr(status, 2u);");
+    em.line("  warp_arrive(sempty + st, lane);");
+    em.line("}");
+    em.line("if (last) {");
+    em.line("  float* orow = out + b * " + S(o_row) + " + c;");
+    for (int o : outs) em.line("  orow[" + S(static_cast<long long>(o) * pl.C) + "] = a" + S(o) + " * inv_avg; a" + S(o) + " = 0.f;");
+    em.line("}");
+    em.line("++q;");
+    em.ind--;
+    em.line("}");
+    em.ind--;
+  }
+  em.line("}");
+  em.line("if (!ok && lane == 0) atomicOr(status, 4u);");
   em.ind--;
   em.line("}");
   em.line("tc_before();");
