@@ -212,15 +212,14 @@ def test_tensor_core_tables_emulated_on_host():
     pairs = [(int(a), int(b)) for a, b in re.findall(r"\{(-?\d+), (\d+)\}", tab)]
     offs = [int(v) for v in re.search(r"e3_boff\[\] = \{(.*?)\};", src, re.S).group(1)
             .replace("\n", "").split(",") if v.strip()]
-    terms = [int(m) for m in re.findall(r"// round terms: (\d+)", src)] or None
     Y = np.random.default_rng(3).normal(size=c.ny)
     B = np.zeros((16, ncols))
-    base = 0
     lanes = int(re.search(r"producer_threads=(\d+)", src).group(1))
-    rounds = re.findall(r"\{\n((?:\s+const int2 k\d+ = __ldg\(&e3_btab\[(\d+) \+ pt\]\);\n)+)", src)
-    assert len(rounds) == -(-541 // lanes)
-    for r, (body, _) in enumerate(rounds):
-        bases = [int(b) for b in re.findall(r"e3_btab\[(\d+) \+ pt\]", body)]
+    loads = re.findall(r"const int2 k(\d+)_(\d+) = __ldg\(&e3_btab\[(\d+) \+ bt\]\);", src)
+    nrounds = max(int(r) for r, _, _ in loads) + 1
+    assert nrounds == -(-541 // lanes)
+    for r in range(nrounds):
+        bases = [int(b) for rr, _, b in loads if int(rr) == r]
         for lane in range(lanes):
             off = offs[r * lanes + lane]
             if off < 0:
@@ -231,9 +230,16 @@ def test_tensor_core_tables_emulated_on_host():
             i = ((off % 256) // 128) * 8 + (off % 16) // 2
             assert B[i, n] == 0
             B[i, n] = v
+    # T columns: the paths of output group 0 (the outputs whose accumulators the
+    # group-0 consumers declare), then those of group 1, each group in path order
+    g0 = re.search(r"output group 0[^\n]*\n\s*float ([^;]*);", src).group(1)
+    group0 = {int(m) for m in re.findall(r"a(\d+) = 0\.f", g0)}
+    order = ([p for p, q in enumerate(c.paths) if q.out_off in group0] +
+             [p for p, q in enumerate(c.paths) if q.out_off not in group0])
     expect = np.zeros((16, ncols))
     col = 0
-    for p, q in enumerate(c.paths):
+    for p in order:
+        q = c.paths[p]
         W = c.cg(p)
         d1, d2, d3 = W.shape
         for i in range(d1):
