@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--block-threads", type=int, default=0)
     ap.add_argument("--stages", type=int, default=-1)
     ap.add_argument("--contract-first", type=int, default=-1)
+    ap.add_argument("--tensor-cores", type=int, default=0,
+                    help="1: the tensor-core forward variant (float16 inputs, 128 channels)")
     return ap.parse_args()
 
 
@@ -192,21 +194,21 @@ def oracle_sample_rate(spec, graph, rows, x_rows_fn, Y_fn, s_fn, threads=0):
 
 
 def calibrated_rows(spec, graph, x_rows_fn, Y_fn, s_fn, target_s, seed=2024):
-    """Seeded receivers whose oracle run takes about target_s seconds (two probes: a
-    tiny one, then one of ~1/8 of the target, so thread start-up does not skew the rate)."""
+    """Seeded receivers whose oracle run takes about target_s seconds.  The oracle's rate
+    grows with the sample (fixed per-call cost, OpenMP balance over few receivers), so the
+    probe grows geometrically until one run takes at least a quarter of the target, and the
+    sample is scaled from that last probe."""
     import numpy as np
     order = np.random.default_rng(seed).permutation(graph.num_nodes)
     n = min(16, graph.num_nodes)
-    for frac in (None, 0.125):
-        probe = order[:n]
-        rate, ne, dt = oracle_sample_rate(spec, graph, probe, x_rows_fn, Y_fn, s_fn)
-        per_row = max(ne / len(probe), 1e-9)
-        want = int(max(1, min(graph.num_nodes, rate * target_s / per_row)))
-        if frac is None:
-            n = int(max(n, min(graph.num_nodes, want * 0.125)))
-            if n >= graph.num_nodes:
-                break
-    return np.sort(order[:want])
+    while True:
+        rate, ne, dt = oracle_sample_rate(spec, graph, order[:n], x_rows_fn, Y_fn, s_fn)
+        if n >= graph.num_nodes:
+            return np.sort(order[:n])
+        if dt >= 0.25 * target_s:
+            want = int(min(graph.num_nodes, n * target_s / max(dt, 1e-9)))
+            return np.sort(order[:max(want, n)])
+        n = int(min(graph.num_nodes, n * min(8.0, max(2.0, 0.3 * target_s / max(dt, 1e-9)))))
 
 
 def device_inputs_fns(x_d, Y_d, s_d):
@@ -319,6 +321,8 @@ def run_ours(args):
         conv.set_launch_config(args.channels_per_lane, args.block_threads, args.stages)
     if args.contract_first != -1:
         conv.set_contract_first(args.contract_first)
+    if args.tensor_cores:
+        conv.set_tensor_cores(1)
     row_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
     perm = torch.empty(E, dtype=torch.int32, device=dev)
     ws = torch.empty(e3.csr_workspace_size(E, N), dtype=torch.uint8, device=dev)
