@@ -93,29 +93,35 @@ Shape choose_shape(const Plan& pl, int dtype) {
       s.TL = 32;
       s.tiles = 1;
       s.ipw = 1;
-      s.block = 480;                                // 8 consumer, 2 copy, 1 MMA, 4 builder warps
       s.ncols = ncols;
       s.tmem_cols = 512;
-      s.tstride = align_up(ncols, 32);              // T buffers start on 32-column boundaries
-      s.tbufs = std::min(3, 512 / s.tstride);
-      s.bbufs = s.tbufs;                            // one A tile per T buffer
-      const int S = pl.req_stages > 0 ? std::max(pl.req_stages, 2) : 8;
-      s.stages = S;
-      s.x_off = 0;                                  // nx rows x 128 channels x 2 B, two 128B-swizzled halves
+      s.tstride = align_up(ncols, 32);              // a team's T columns start on a 32-column boundary
+      s.tbufs = std::min(3, 512 / s.tstride);       // teams per block: T columns fit in 512, registers in 64K
+      s.block = 128 * s.tbufs;                      // four warps per team
+      int S = pl.req_stages > 0 ? std::max(pl.req_stages, 2) : 4;
+      s.x_off = 0;                                  // 16 rows x 128 channels x 2 B, two 128B-swizzled halves
       s.s_off = 4096;
       s.y_off = s.s_off + align_up(s.s_bytes, 128);
       s.stage_bytes = align_up(s.y_off + s.y_bytes, 1024);
-      s.b_off = S * s.stage_bytes;
       s.b_bytes = 32 * ncols;                       // 16 x ncols f16, K-major core matrices
       s.b_stride = s.b_bytes + 128;                 // + scratch for the builders' padding lanes
-      s.yf_off = s.b_off + 2 * s.bbufs * s.b_stride; // bbufs buffers of (A_hi, A_lo)
-      s.bar_off = align_up(s.yf_off + 4 * 4 * align_up(pl.ny, 4), 8);  // Y as float32, per builder warp
-      s.mbar_off = s.bar_off;                       // sfull[S] sempty[S] bfull[T] tfull[T] tempty[T]
-      s.hdr_off = s.bar_off + 8 * (2 * S + s.bbufs + 2 * s.tbufs);
-      s.tslot_off = s.hdr_off + 16 * S;
-      s.warp_smem = align_up(s.tslot_off + 16, 1024);
-      // one block per SM (it allocates all 512 tensor-memory columns)
-      s.smem_request = std::max(s.warp_smem, 116 * 1024);
+      auto layout = [&](int stages) {
+        s.stages = stages;
+        s.b_off = stages * s.stage_bytes;
+        s.yf_off = s.b_off + 2 * s.b_stride;
+        s.hdr_off = s.yf_off + 4 * 4 * align_up(pl.ny, 4);
+        s.bar_off = align_up(s.hdr_off + 16 * stages, 8);
+        s.warp_smem = align_up(s.bar_off + 8 * (stages + 1), 1024);  // one team
+        s.tslot_off = s.tbufs * s.warp_smem;
+        s.smem_request = std::max(s.tslot_off + 16, 116 * 1024);    // one block per SM
+      };
+      layout(S);
+      while (s.smem_request > 227 * 1024 && s.stages > 2) layout(s.stages - 1);
+      while (s.smem_request > 227 * 1024 && s.tbufs > 1) {
+        s.tbufs -= 1;
+        s.block = 128 * s.tbufs;
+        layout(s.stages);
+      }
       if (s.smem_request <= 227 * 1024) return s;
       s = Shape{};
       s.s_bytes = static_cast<int>(pl.paths.size()) * pl.C * elem;
@@ -1022,69 +1028,48 @@ BTable tc_tables(const Plan& pl, const std::vector<AEntry>& ent, const std::vect
   return T;
 }
 
-// Tensor-core forward.  Warp roles of one block (one block per SM):
-//   warps 0..7   consumers: warp w reads tensor-memory lanes 32*(w%4).. (its
-//                channels) and the path columns of output group w/4, scales
-//                them by s and accumulates the receiver row in registers;
-//   warps 8, 9   copies: both walk the block's rows; warp 8 fills the even
-//                ring positions, warp 9 the odd ones (TMA of the sender's
-//                nx x 128 tile, bulk copies of the edge's s and Y rows);
-//   warp 10      MMA: T = x^T (A_hi + A_lo) into one of NT tensor-memory buffers;
-//   warps 11..14 build A = sum_j CG Y_j (K-major float16 hi/lo tiles, one per T buffer).
-// Every hand-off is an mbarrier with one arrival per warp (or a TMA / MMA
-// completion); every wait is bounded and agreed within the warp only.  One MMA
-// commit per edge (tfull) serves both the consumers (T ready) and the builders
-// (the A tile of that buffer is free again).  A ring stage is released once its
-// readers are done: builders once Y is in their buffer, the MMA warp once it
-// has issued, consumers once s is in registers and the MMA has completed (so x
-// has been read).
+// Tensor-core forward, teams of four warps.  A team (128 threads, one warp per
+// tensor-memory lane quarter, thread tl <-> channel tl) owns receiver rows
+// g, g+W, g+2W, ... (g = its index in the grid, W = teams in the grid) and a
+// private ring of S stages, A tile and T columns.  Per edge:
+//   1. wait for the edge's stage (x tile by 4-D TMA, s and Y rows by bulk copy);
+//   2. build A = sum_j CG Y_j as float16 hi/lo K-major tiles (128 threads,
+//      branch-free, coefficient table in registers);
+//   3. one team barrier (bar.red.and.pred: also agrees on bounded-wait timeouts);
+//   4. the team leader issues T = x^T A_hi + x^T A_lo (tcgen05.mma, M = 128
+//      channels) and commits to the team's mbarrier; warp 0 refills the ring
+//      slot the barrier has just freed;
+//   5. every thread loads its channel's s, waits for the commit, reads T from
+//      tensor memory in 32-column chunks and accumulates s * T in registers.
+// Several teams per SM overlap one another's latency.
 std::string tc_source(const Plan& pl, const Shape& sh) {
   Emitter em;
   const int NS = sh.stages;
-  const int NT = sh.tbufs;
-  const int NB = 4, BT = 32 * NB;             // builder warps / threads
-  const int NBUF = NT;                        // A tile buffers, paired with the T buffers
-  const int BS = sh.b_stride;                 // bytes between A_hi and A_lo (tile + scratch)
-  const int TID_B = 352, W_COPY = 8, W_MMA = 10, W_B = 11;
+  const int TEAMS = sh.tbufs;
+  const int TBYTES = sh.warp_smem;            // shared memory of one team
+  const int BS = sh.b_stride;
   const long long s_row = static_cast<long long>(pl.paths.size()) * pl.C;
   const long long o_row = static_cast<long long>(pl.nout) * pl.C;
-  // outputs split into two groups of similar column count; group 0's paths
-  // take the first columns of T
-  std::vector<int> ocols(pl.outputs.size(), 0), og(pl.outputs.size(), 0);
-  for (const auto& P : pl.paths) ocols[P.o] += 2 * P.l3 + 1;
-  {
-    std::vector<int> ord(pl.outputs.size());
-    for (size_t o = 0; o < ord.size(); ++o) ord[o] = static_cast<int>(o);
-    std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return ocols[a] > ocols[b]; });
-    int load[2] = {0, 0};
-    for (int o : ord) {
-      const int g = load[1] < load[0] ? 1 : 0;
-      og[o] = g;
-      load[g] += ocols[o];
-    }
-  }
   std::vector<int> colbase(pl.paths.size());
-  int gcol[3];
-  {
-    int col = 0;
-    for (int g = 0; g < 2; ++g) {
-      gcol[g] = col;
-      for (size_t p = 0; p < pl.paths.size(); ++p)
-        if (og[pl.paths[p].o] == g) {
-          colbase[p] = col;
-          col += 2 * pl.paths[p].l3 + 1;
-        }
-    }
-    gcol[2] = col;
+  int ncols_raw = 0;
+  for (size_t p = 0; p < pl.paths.size(); ++p) {
+    colbase[p] = ncols_raw;
+    ncols_raw += 2 * pl.paths[p].l3 + 1;
   }
   std::vector<AEntry> ent = build_a_entries(pl);
-  BTable tab = tc_tables(pl, ent, colbase, BT);
-  em.line("// generated by libe3conv: fused equivariant convolution forward (tensor cores)");
+  BTable tab = tc_tables(pl, ent, colbase, 128);
+  std::vector<std::pair<int, int>> chunks;  // (start column, width), start a multiple of width
+  for (int pos = 0; pos < ncols_raw;) {
+    int w = 32;
+    while (w > 1 && (pos % w != 0 || pos + w > ncols_raw)) w /= 2;
+    chunks.push_back({pos, w});
+    pos += w;
+  }
+  em.line("// generated by libe3conv: fused equivariant convolution forward (tensor cores, teams)");
   em.line("// C=" + S(pl.C) + " nx=" + S(pl.nx) + " ny=" + S(pl.ny) + " nout=" + S(pl.nout) +
-          " paths=" + S(pl.paths.size()) + " dtype=f16 ncols=" + S(sh.ncols) + " tbufs=" + S(NT) +
-          " tstride=" + S(sh.tstride) + " bbufs=" + S(NBUF) + " stages=" + S(NS) + " stage_bytes=" + S(sh.stage_bytes) +
-          " entries=" + S(ent.size()) + " producer_threads=" + S(BT) +
-          " group_cols=" + S(gcol[1] - gcol[0]) + "," + S(gcol[2] - gcol[1]));
+          " paths=" + S(pl.paths.size()) + " dtype=f16 ncols=" + S(sh.ncols) + " teams=" + S(TEAMS) +
+          " tstride=" + S(sh.tstride) + " stages=" + S(NS) + " stage_bytes=" + S(sh.stage_bytes) +
+          " team_bytes=" + S(TBYTES) + " entries=" + S(ent.size()) + " producer_threads=128");
   em.o << tab.source;
   em.line("__device__ __forceinline__ float h2f(unsigned short h) { float f; asm(\"cvt.f32.f16 %0, %1;\" : \"=f\"(f) : \"h\"(h)); return f; }");
   em.line("__device__ __forceinline__ unsigned short f2h(float f) { unsigned short h; asm(\"cvt.rn.f16.f32 %0, %1;\" : \"=h\"(h) : \"f\"(f)); return h; }");
@@ -1098,9 +1083,6 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("  unsigned int ok; asm volatile(\"{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }\" : \"=r\"(ok) : \"r\"(smem_u32(b)), \"r\"(parity) : \"memory\"); return ok != 0; }");
   em.line("__device__ __forceinline__ bool bar_wait(unsigned long long* b, unsigned int parity) {");
   em.line("  for (unsigned int it = 0; it < E3_SPIN_LIMIT; ++it) if (bar_try(b, parity)) return true; return false; }");
-  em.line("// bounded wait agreed by the warp (a lane that gave up makes the whole warp give up)");
-  em.line("__device__ __forceinline__ bool warp_wait(unsigned long long* b, unsigned int parity) { return __all_sync(0xffffffffu, bar_wait(b, parity)); }");
-  em.line("__device__ __forceinline__ void warp_arrive(unsigned long long* b, int lane) { __syncwarp(); if (lane == 0) bar_arrive(b); }");
   em.line("__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned int bytes, unsigned long long* b, unsigned long long policy) {");
   em.line("  asm volatile(\"cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;\" :: \"r\"(smem_u32(dst)), \"l\"(src), \"r\"(bytes), \"r\"(smem_u32(b)), \"l\"(policy) : \"memory\"); }");
   em.line("// the sender's tile: box {64 channels, 16 rows, 2 halves} of node `node` (rows >= nx zero-filled)");
@@ -1111,7 +1093,8 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("__device__ __forceinline__ void fence_async_smem() { asm volatile(\"fence.proxy.async.shared::cta;\" ::: \"memory\"); }");
   em.line("__device__ __forceinline__ void tc_before() { asm volatile(\"tcgen05.fence::before_thread_sync;\" ::: \"memory\"); }");
   em.line("__device__ __forceinline__ void tc_after() { asm volatile(\"tcgen05.fence::after_thread_sync;\" ::: \"memory\"); }");
-  // tensor-memory loads of 1..32 columns (32 lanes x 32 bit)
+  em.line("// barrier of the team's 128 threads that also ANDs a predicate over them");
+  em.line("__device__ __forceinline__ bool team_all(bool ok, unsigned int id) { unsigned int r; asm volatile(\"{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.and.pred q, %2, 128, p; selp.u32 %0, 1, 0, q; }\" : \"=r\"(r) : \"r\"((unsigned int)ok), \"r\"(id) : \"memory\"); return r != 0u; }");
   for (int n = 1; n <= 32; n *= 2) {
     std::string regs, outs;
     for (int r = 0; r < n; ++r) {
@@ -1130,21 +1113,20 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.ind++;
   em.line("extern __shared__ __align__(1024) unsigned char smem[];");
   em.line("const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;");
-  em.line("unsigned long long* sfull = reinterpret_cast<unsigned long long*>(smem + " + S(sh.bar_off) + ");");
-  em.line("unsigned long long* sempty = sfull + " + S(NS) + ";   // 8 consumer + 4 builder warps + the MMA warp");
-  em.line("unsigned long long* bfull = sempty + " + S(NS) + ";   // 4 builder warps");
-  em.line("unsigned long long* tfull = bfull + " + S(NBUF) + ";      // MMA completion (T ready, A tile free)");
-  em.line("unsigned long long* tempty = tfull + " + S(NT) + ";  // 8 consumer warps");
-  em.line("int* hdr = reinterpret_cast<int*>(smem + " + S(sh.hdr_off) + ");  // per stage: sender (-1 invalid, -2 end), receiver, last");
+  em.line("const int team = warp >> 2, tw = warp & 3, tl = tid & 127;  // tl = channel = tensor-memory lane");
+  em.line("const unsigned int bar_id = 1u + (unsigned int)team;");
+  em.line("unsigned char* tbase = smem + team * " + S(TBYTES) + ";");
+  em.line("unsigned char* Bhi = tbase + " + S(sh.b_off) + ";  // A_hi; A_lo at +" + S(BS) + "; bytes " + S(sh.b_bytes) + ".. of each are scratch");
+  em.line("unsigned char* Blo = Bhi + " + S(BS) + ";");
+  em.line("float* yfw = reinterpret_cast<float*>(tbase + " + S(sh.yf_off) + ") + tw * " + S(align_up(pl.ny, 4)) + ";");
+  em.line("int* hdr = reinterpret_cast<int*>(tbase + " + S(sh.hdr_off) + ");  // per stage: sender (-1 invalid, -2 end), receiver, last");
+  em.line("unsigned long long* sfull = reinterpret_cast<unsigned long long*>(tbase + " + S(sh.bar_off) + ");");
+  em.line("unsigned long long* tdone = sfull + " + S(NS) + ";");
   em.line("unsigned int* tslot = reinterpret_cast<unsigned int*>(smem + " + S(sh.tslot_off) + ");");
-  em.line("unsigned char* Bt = smem + " + S(sh.b_off) + ";  // buffer bb: A_hi at bb*" + S(2 * BS) + ", A_lo at +" + S(BS) + "; bytes " + S(sh.b_bytes) + ".. of each are scratch");
-  em.line("for (int q = tid; q < " + S(2 * NBUF * BS / 16) + "; q += " + S(sh.block) + ") reinterpret_cast<uint4*>(Bt)[q] = make_uint4(0u, 0u, 0u, 0u);");
-  em.line("for (int k = 0; k < " + S(NS) + "; ++k)");
-  em.line("  for (int q = tid; q < 256; q += " + S(sh.block) + ") reinterpret_cast<uint4*>(smem + k * " + S(sh.stage_bytes) + ")[q] = make_uint4(0u, 0u, 0u, 0u);");
-  em.line("if (tid == 0) {");
-  em.line("  for (int k = 0; k < " + S(NS) + "; ++k) { bar_init(sfull + k, 1u); bar_init(sempty + k, 13u); }");
-  em.line("  for (int k = 0; k < " + S(NBUF) + "; ++k) bar_init(bfull + k, " + S(NB) + "u);");
-  em.line("  for (int k = 0; k < " + S(NT) + "; ++k) { bar_init(tfull + k, 1u); bar_init(tempty + k, 8u); }");
+  em.line("for (int q = tl; q < " + S(2 * BS / 16) + "; q += 128) reinterpret_cast<uint4*>(Bhi)[q] = make_uint4(0u, 0u, 0u, 0u);");
+  em.line("if (tl == 0) {");
+  em.line("  for (int k = 0; k < " + S(NS) + "; ++k) bar_init(sfull + k, 1u);");
+  em.line("  bar_init(tdone, 1u);");
   em.line("  asm volatile(\"fence.mbarrier_init.release.cluster;\" ::: \"memory\");");
   em.line("}");
   em.line("if (warp == 0) {");
@@ -1156,43 +1138,51 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("__syncthreads();");
   em.line("tc_after();");
   em.line("const unsigned int tmem = *tslot;");
-  em.line("const long long W = (long long)gridDim.x;");
-
-  // ---------------- copy warps ----------------
-  em.line("if (warp == " + S(W_COPY) + " || warp == " + S(W_COPY + 1) + ") {");
-  em.ind++;
-  em.line("const unsigned int cw = (unsigned int)(warp - " + S(W_COPY) + ");  // ring positions q with q % 2 == cw");
-  em.line("const unsigned long long pol_stream = policy_evict_first();");
-  em.line("const unsigned long long pol_keep = policy_evict_last();");
-  em.line("// row walk with loads one row ahead: the open row [pe, pe1) of receiver pb with its");
-  em.line("// sender windows psw (edges pwin..pwin+31) and psw2 (the next 32); the next row nb");
-  em.line("// [n0, n1) with its first window nsw in flight; row_ptr of the row after (mb) in flight");
-  em.line("long long pb = -1, nb = blockIdx.x, mb = (long long)blockIdx.x + W;");
-  em.line("int pe = 0, pe1 = 0, pwin = 0, psw = 0, psw2 = 0;");
-  em.line("int n0 = 0, n1 = 0, nsw = 0, nsw2 = 0, m0 = 0, m1 = 0;");
-  em.line("if (nb < num_nodes) {");
-  em.line("  n0 = row_ptr[nb]; n1 = row_ptr[nb + 1];");
-  em.line("  if (n0 < 0 || n1 < n0 || n1 > num_edges) { if (lane == 0) atomicOr(status, 1u); n1 = n0; }");
-  em.line("  nsw = (n0 + lane < n1) ? senders[n0 + lane] : 0;");
-  em.line("  nsw2 = (n0 + 32 + lane < n1) ? senders[n0 + 32 + lane] : 0;");
+  em.line("const unsigned int tcol = tmem + ((unsigned int)(32 * tw) << 16) + (unsigned int)(team * " + S(sh.tstride) + ");");
+  em.line("const unsigned int tmma = tmem + (unsigned int)(team * " + S(sh.tstride) + ");");
+  em.line("const unsigned int idesc = (1u << 4) | (1u << 15) | ((unsigned int)(" + S(sh.ncols) + " >> 3) << 17) | ((unsigned int)(128 >> 4) << 24);");
+  em.line("const long long W = (long long)gridDim.x * " + S(TEAMS) + ";");
+  // A-tile table in registers
+  {
+    int base = 0;
+    for (int r = 0; r < tab.rounds; ++r) {
+      for (int t2 = 0; t2 < tab.terms[r]; ++t2)
+        em.line("const int2 k" + S(r) + "_" + S(t2) + " = __ldg(&e3_btab[" + S(base + t2 * 128) + " + tl]);");
+      em.line("const int off" + S(r) + " = __ldg(&e3_boff[" + S(r * 128) + " + tl]) >= 0 ? __ldg(&e3_boff[" + S(r * 128) + " + tl]) : " + S(sh.b_bytes) + ";  // padding lanes write the scratch bytes");
+      base += tab.terms[r] * 128;
+    }
+  }
+  // row walk (warp tw == 0 of the team; lane 0 issues the copies)
+  em.line("// row walk of warp 0 of the team, loads one row ahead: the open row [pe, pe1) of receiver");
+  em.line("// pb with sender windows psw (edges pwin..) and psw2 (the next 32); the next row nb [n0, n1)");
+  em.line("// with its first windows in flight; row_ptr of the row after (mb) in flight");
+  em.line("long long pb = -1, nb = (long long)blockIdx.x * " + S(TEAMS) + " + team, mb = nb + W;");
+  em.line("int pe = 0, pe1 = 0, pwin = 0, psw = 0, psw2 = 0, n0 = 0, n1 = 0, nsw = 0, nsw2 = 0, m0 = 0, m1 = 0;");
+  em.line("unsigned int qi = 0;  // positions issued");
+  em.line("bool walk_done = false;");
+  em.line("unsigned long long pol_stream = 0, pol_keep = 0;");
+  em.line("if (tw == 0) {");
+  em.line("  pol_stream = policy_evict_first();");
+  em.line("  pol_keep = policy_evict_last();");
+  em.line("  if (nb < num_nodes) {");
+  em.line("    n0 = row_ptr[nb]; n1 = row_ptr[nb + 1];");
+  em.line("    if (n0 < 0 || n1 < n0 || n1 > num_edges) { if (lane == 0) atomicOr(status, 1u); n1 = n0; }");
+  em.line("    nsw = (n0 + lane < n1) ? senders[n0 + lane] : 0;");
+  em.line("    nsw2 = (n0 + 32 + lane < n1) ? senders[n0 + 32 + lane] : 0;");
+  em.line("  }");
+  em.line("  if (mb < num_nodes) { m0 = row_ptr[mb]; m1 = row_ptr[mb + 1]; }");
   em.line("}");
-  em.line("if (mb < num_nodes) { m0 = row_ptr[mb]; m1 = row_ptr[mb + 1]; }");
-  em.line("unsigned int q = 0;");
-  em.line("bool ok = true;");
-  em.line("#pragma unroll 1");
-  em.line("while (true) {");
+  em.line("// issue position qi into stage qi % S (warp 0 of the team only)");
+  em.line("auto issue = [&]() {");
   em.ind++;
-  em.line("const unsigned int st = q % " + S(NS) + ";");
-  em.line("const bool mine = (q & 1u) == cw;");
-  em.line("if (mine && q >= " + S(NS) + "u) { ok = warp_wait(sempty + st, ((q / " + S(NS) + ") - 1u) & 1u); if (!ok) break; }");
-  em.line("bool done = false;");
+  em.line("const unsigned int st = qi % " + S(NS) + ";");
   em.line("while (pe >= pe1) {  // open the next row");
   em.line("  pb = nb;");
-  em.line("  if (pb >= num_nodes) { done = true; break; }");
+  em.line("  if (pb >= num_nodes) { walk_done = true; break; }");
   em.line("  pe = n0; pe1 = n1; pwin = n0; psw = nsw; psw2 = nsw2;");
   em.line("  if (pe == pe1) {");
   em.line("    float* zrow = out + pb * " + S(o_row) + ";");
-  em.line("    if (cw == 0u) for (int k = lane; k < " + S(o_row) + "; k += 32) zrow[k] = 0.f;");
+  em.line("    for (int k = lane; k < " + S(o_row) + "; k += 32) zrow[k] = 0.f;");
   em.line("  }");
   em.line("  nb = mb; n0 = m0; n1 = m1;");
   em.line("  if (nb < num_nodes) {");
@@ -1203,10 +1193,10 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("  mb = nb + W;");
   em.line("  if (mb < num_nodes) { m0 = row_ptr[mb]; m1 = row_ptr[mb + 1]; }");
   em.line("}");
-  em.line("if (done) {");
-  em.line("  if (mine && lane == 0) { hdr[4 * st] = -2; bar_arrive(sfull + st); }  // end marker");
-  em.line("  ++q;");
-  em.line("  break;");
+  em.line("if (walk_done) {");
+  em.line("  if (lane == 0) { hdr[4 * st] = -2; bar_arrive(sfull + st); }  // end marker");
+  em.line("  ++qi;");
+  em.line("  return;");
   em.line("}");
   em.line("if (pe >= pwin + 32) {  // next window of the row");
   em.line("  pwin += 32; psw = psw2;");
@@ -1214,8 +1204,8 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("}");
   em.line("const int a = __shfl_sync(0xffffffffu, psw, pe - pwin);");
   em.line("const bool valid = (unsigned int)a < (unsigned int)num_nodes;");
-  em.line("if (mine && lane == 0) {");
-  em.line("  unsigned char* stg = smem + st * " + S(sh.stage_bytes) + ";");
+  em.line("if (lane == 0) {");
+  em.line("  unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
   em.line("  hdr[4 * st] = valid ? a : -1;");
   em.line("  hdr[4 * st + 1] = (int)pb;");
   em.line("  hdr[4 * st + 2] = (pe + 1 == pe1) ? 1 : 0;");
@@ -1226,71 +1216,15 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("}");
   em.line("__syncwarp();");
   em.line("++pe;");
-  em.line("++q;");
+  em.line("++qi;");
   em.ind--;
-  em.line("}");
-  em.line("if (!ok && lane == 0) atomicOr(status, 4u);");
-  em.line("// drain: this warp's copies of the last positions land before the block leaves (bounded)");
-  em.line("if (lane == 0)");
-  em.line("  for (unsigned int k = q > " + S(NS) + "u ? q - " + S(NS) + "u : 0u; k < q; ++k)");
-  em.line("    if ((k & 1u) == cw) bar_wait(sfull + k % " + S(NS) + ", (k / " + S(NS) + ") & 1u);");
-  em.ind--;
-  // ---------------- MMA warp ----------------
-  em.line("} else if (warp == " + S(W_MMA) + ") {");
-  em.ind++;
-  em.line("const unsigned int idesc = (1u << 4) | (1u << 15) | ((unsigned int)(" + S(sh.ncols) + " >> 3) << 17) | ((unsigned int)(128 >> 4) << 24);");
-  em.line("unsigned int q = 0, v = 0;");
-  em.line("bool ok = true;");
-  em.line("#pragma unroll 1");
-  em.line("while (true) {");
-  em.ind++;
-  em.line("const unsigned int st = q % " + S(NS) + ";");
-  em.line("ok = warp_wait(sfull + st, (q / " + S(NS) + ") & 1u);");
-  em.line("if (!ok) break;");
-  em.line("const int a = hdr[4 * st];");
-  em.line("if (a == -2) break;");
-  em.line("if (a >= 0) {");
-  em.ind++;
-  em.line("const unsigned int tb = v % " + S(NT) + "u;");
-  em.line("ok = warp_wait(bfull + tb, (v / " + S(NT) + "u) & 1u);");
-  em.line("if (!ok) break;");
-  em.line("if (v >= " + S(NT) + "u) { ok = warp_wait(tempty + tb, ((v / " + S(NT) + "u) - 1u) & 1u); if (!ok) break; }");
-  em.line("tc_after();");
-  em.line("if (lane == 0) {");
-  em.line("  const unsigned char* stg = smem + st * " + S(sh.stage_bytes) + ";");
-  em.line("  const unsigned char* Bhi = Bt + tb * " + S(2 * BS) + ";");
-  em.line("  const unsigned long long adesc = (unsigned long long)((smem_u32(stg) & 0x3FFFF) >> 4) | (128ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);");
-  em.line("  const unsigned long long hdesc = (unsigned long long)((smem_u32(Bhi) & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
-  em.line("  const unsigned long long ldesc = (unsigned long long)((smem_u32(Bhi + " + S(BS) + ") & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
-  em.line("  const unsigned int dt = tmem + tb * " + S(sh.tstride) + "u;");
-  em.line("  asm volatile(\"{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }\" :: \"r\"(dt), \"l\"(adesc), \"l\"(hdesc), \"r\"(idesc), \"r\"(0u) : \"memory\");");
-  em.line("  asm volatile(\"{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }\" :: \"r\"(dt), \"l\"(adesc), \"l\"(ldesc), \"r\"(idesc), \"r\"(1u) : \"memory\");");
-  em.line("  asm volatile(\"tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\" :: \"r\"(smem_u32(tfull + tb)) : \"memory\");");
-  em.line("}");
-  em.line("++v;");
-  em.ind--;
-  em.line("}");
-  em.line("warp_arrive(sempty + st, lane);");
-  em.line("++q;");
-  em.ind--;
-  em.line("}");
-  em.line("if (!ok && lane == 0) atomicOr(status, 4u);");
-  em.line("// drain: the last MMAs complete before tensor memory is released (bounded)");
-  em.line("if (lane == 0 && v > 0u) bar_wait(tfull + (v - 1u) % " + S(NT) + "u, ((v - 1u) / " + S(NT) + "u) & 1u);");
-  em.ind--;
-  // ---------------- builder warps ----------------
-  em.line("} else if (warp >= " + S(W_B) + ") {");
-  em.ind++;
-  em.line("const int bt = tid - " + S(TID_B) + ";  // 0.." + S(BT - 1));
-  em.line("float* yfw = reinterpret_cast<float*>(smem + " + S(sh.yf_off) + ") + (warp - " + S(W_B) + ") * " + S(align_up(pl.ny, 4)) + ";");
+  em.line("};");
+  em.line("if (tw == 0)");
+  em.line("  for (int k = 0; k < " + S(NS - 1) + " && !walk_done; ++k) issue();");
   {
-    int base = 0;
-    for (int r = 0; r < tab.rounds; ++r) {
-      for (int t2 = 0; t2 < tab.terms[r]; ++t2)
-        em.line("const int2 k" + S(r) + "_" + S(t2) + " = __ldg(&e3_btab[" + S(base + t2 * BT) + " + bt]);");
-      em.line("const int off" + S(r) + " = __ldg(&e3_boff[" + S(r * BT) + " + bt]) >= 0 ? __ldg(&e3_boff[" + S(r * BT) + " + bt]) : " + S(sh.b_bytes) + ";  // padding lanes write the scratch bytes");
-      base += tab.terms[r] * BT;
-    }
+    std::string decl = "float";
+    for (int c = 0; c < pl.nout; ++c) decl += std::string(c ? "," : "") + " a" + S(c) + " = 0.f";
+    em.line(decl + ";");
   }
   em.line("unsigned int q = 0, v = 0;");
   em.line("bool ok = true;");
@@ -1298,19 +1232,13 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("while (true) {");
   em.ind++;
   em.line("const unsigned int st = q % " + S(NS) + ";");
-  em.line("ok = warp_wait(sfull + st, (q / " + S(NS) + ") & 1u);");
-  em.line("if (!ok) break;");
-  em.line("const int a = hdr[4 * st];");
-  em.line("if (a == -2) break;");
-  em.line("if (a >= 0) {");
+  em.line("const unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
+  em.line("const bool landed = bar_wait(sfull + st, (q / " + S(NS) + ") & 1u);");
+  em.line("if (landed && hdr[4 * st] >= 0) {  // A tile of this edge (the MMA of the previous edge has completed)");
   em.ind++;
-  em.line("const unsigned short* ys = reinterpret_cast<const unsigned short*>(smem + st * " + S(sh.stage_bytes) + " + " + S(sh.y_off) + ");");
+  em.line("const unsigned short* ys = reinterpret_cast<const unsigned short*>(stg + " + S(sh.y_off) + ");");
   em.line("for (int j = lane; j < " + S(pl.ny) + "; j += 32) yfw[j] = h2f(ys[j]);");
-  em.line("warp_arrive(sempty + st, lane);  // Y is in this warp's buffer");
-  em.line("const unsigned int bb = v % " + S(NBUF) + "u;");
-  em.line("if (v >= " + S(NBUF) + "u) { ok = warp_wait(tfull + bb, ((v / " + S(NBUF) + "u) - 1u) & 1u); if (!ok) break; }  // MMA v-" + S(NBUF) + " done");
-  em.line("unsigned char* Bhi = Bt + bb * " + S(2 * BS) + ";");
-  em.line("unsigned char* Blo = Bhi + " + S(BS) + ";");
+  em.line("__syncwarp();");
   for (int r = 0; r < tab.rounds; ++r) {
     std::string val = "__int_as_float(k" + S(r) + "_0.x) * yfw[k" + S(r) + "_0.y]";
     for (int t2 = 1; t2 < tab.terms[r]; ++t2)
@@ -1323,101 +1251,63 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
     em.line("}");
   }
   em.line("fence_async_smem();");
-  em.line("warp_arrive(bfull + bb, lane);");
+  em.ind--;
+  em.line("}");
+  em.line("tc_before();");
+  em.line("ok = team_all(ok && landed, bar_id);  // A tile written, T of the previous edge read, all waits in time");
+  em.line("if (!ok) break;");
+  em.line("tc_after();");
+  em.line("const int a = hdr[4 * st];");
+  em.line("if (a == -2) break;");
+  em.line("const long long b = hdr[4 * st + 1];");
+  em.line("const int last = hdr[4 * st + 2];");
+  em.line("if (a >= 0 && tl == 0) {");
+  em.line("  const unsigned long long adesc = (unsigned long long)((smem_u32(stg) & 0x3FFFF) >> 4) | (128ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);");
+  em.line("  const unsigned long long hdesc = (unsigned long long)((smem_u32(Bhi) & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
+  em.line("  const unsigned long long ldesc = (unsigned long long)((smem_u32(Blo) & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
+  em.line("  asm volatile(\"{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }\" :: \"r\"(tmma), \"l\"(adesc), \"l\"(hdesc), \"r\"(idesc), \"r\"(0u) : \"memory\");");
+  em.line("  asm volatile(\"{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }\" :: \"r\"(tmma), \"l\"(adesc), \"l\"(ldesc), \"r\"(idesc), \"r\"(1u) : \"memory\");");
+  em.line("  asm volatile(\"tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\" :: \"r\"(smem_u32(tdone)) : \"memory\");");
+  em.line("}");
+  em.line("// the slot of the previous edge is free: every thread of the team has passed the barrier");
+  em.line("if (tw == 0 && !walk_done) issue();");
+  em.line("if (a >= 0) {");
+  em.ind++;
+  em.line("const unsigned short* sv = reinterpret_cast<const unsigned short*>(stg + " + S(sh.s_off) + ") + tl;");
+  for (size_t p = 0; p < pl.paths.size(); ++p)
+    em.line("const float s" + S(p) + " = h2f(sv[" + S(static_cast<long long>(p) * pl.C) + "]);");
+  em.line("ok = bar_wait(tdone, v & 1u);");
+  em.line("tc_after();");
+  for (size_t k = 0; k < chunks.size(); ++k) {
+    em.line("{");
+    em.line("  unsigned int r[" + S(chunks[k].second) + "];");
+    em.line("  TMEM_LD" + S(chunks[k].second) + "(tcol + " + S(chunks[k].first) + "u, r);");
+    em.line("  asm volatile(\"tcgen05.wait::ld.sync.aligned;\" ::: \"memory\");");
+    for (int col = chunks[k].first; col < chunks[k].first + chunks[k].second; ++col) {
+      size_t p = 0;
+      while (!(col >= colbase[p] && col < colbase[p] + 2 * pl.paths[p].l3 + 1)) ++p;
+      const std::string acc = "a" + S(pl.paths[p].out_off + col - colbase[p]);
+      em.line("  " + acc + " = fmaf(s" + S(p) + ", __uint_as_float(r[" + S(col - chunks[k].first) + "]), " + acc + ");");
+    }
+    em.line("}");
+  }
   em.line("++v;");
   em.ind--;
-  em.line("} else {");
-  em.line("  warp_arrive(sempty + st, lane);");
+  em.line("} else if (tl == 0) {");
+  em.line("  atomicOr(status, 2u);");
+  em.line("}");
+  em.line("if (last) {");
+  em.line("  float* orow = out + b * " + S(o_row) + " + tl;");
+  for (int c = 0; c < pl.nout; ++c) em.line("  orow[" + S(static_cast<long long>(c) * pl.C) + "] = a" + S(c) + " * inv_avg; a" + S(c) + " = 0.f;");
   em.line("}");
   em.line("++q;");
   em.ind--;
   em.line("}");
-  em.line("if (!ok && lane == 0) atomicOr(status, 4u);");
-  em.ind--;
-  // ---------------- consumer warps ----------------
-  em.line("} else {");
-  em.ind++;
-  em.line("const int c = 32 * (warp & 3) + lane;  // channel = tensor-memory lane");
-  em.line("const unsigned int tmem_lane = tmem + ((unsigned int)(32 * (warp & 3)) << 16);");
-  em.line("unsigned int q = 0, v = 0;");
-  em.line("bool ok = true;");
-  for (int g = 0; g < 2; ++g) {
-    std::vector<int> outs;
-    for (size_t o = 0; o < pl.outputs.size(); ++o)
-      if (og[o] == g)
-        for (int k = 0; k < 2 * pl.outputs[o].l + 1; ++k) outs.push_back(pl.outputs[o].off + k);
-    std::vector<std::pair<int, int>> chunks;  // (start column, width), start a multiple of width
-    for (int pos = gcol[g]; pos < gcol[g + 1];) {
-      int w = 32;
-      while (w > 1 && (pos % w != 0 || pos + w > gcol[g + 1])) w /= 2;
-      chunks.push_back({pos, w});
-      pos += w;
-    }
-    em.line(std::string(g ? "} else {" : "if (warp < 4) {") + "  // output group " + S(g) + ": columns " +
-            S(gcol[g]) + ".." + S(gcol[g + 1] - 1));
-    em.ind++;
-    {
-      std::string decl = "float";
-      for (size_t k = 0; k < outs.size(); ++k) decl += std::string(k ? "," : "") + " a" + S(outs[k]) + " = 0.f";
-      if (!outs.empty()) em.line(decl + ";");
-    }
-    em.line("#pragma unroll 1");
-    em.line("while (true) {");
-    em.ind++;
-    em.line("const unsigned int st = q % " + S(NS) + ";");
-    em.line("ok = warp_wait(sfull + st, (q / " + S(NS) + ") & 1u);");
-    em.line("if (!ok) break;");
-    em.line("const int a = hdr[4 * st];");
-    em.line("if (a == -2) break;");
-    em.line("const long long b = hdr[4 * st + 1];");
-    em.line("const int last = hdr[4 * st + 2];");
-    em.line("if (a >= 0) {");
-    em.ind++;
-    em.line("const unsigned short* sv = reinterpret_cast<const unsigned short*>(smem + st * " + S(sh.stage_bytes) + " + " + S(sh.s_off) + ") + c;");
-    for (size_t p = 0; p < pl.paths.size(); ++p)
-      if (og[pl.paths[p].o] == g)
-        em.line("const float s" + S(p) + " = h2f(sv[" + S(static_cast<long long>(p) * pl.C) + "]);");
-    em.line("const unsigned int tb = v % " + S(NT) + "u;");
-    em.line("ok = warp_wait(tfull + tb, (v / " + S(NT) + "u) & 1u);");
-    em.line("if (!ok) break;");
-    em.line("warp_arrive(sempty + st, lane);  // s is in registers and the MMA has read x");
-    em.line("tc_after();");
-    em.line("const unsigned int tcol = tmem_lane + tb * " + S(sh.tstride) + "u;");
-    for (size_t k = 0; k < chunks.size(); ++k) {
-      em.line("unsigned int r" + S(k) + "[" + S(chunks[k].second) + "];");
-      em.line("TMEM_LD" + S(chunks[k].second) + "(tcol + " + S(chunks[k].first) + "u, r" + S(k) + ");");
-    }
-    em.line("asm volatile(\"tcgen05.wait::ld.sync.aligned;\" ::: \"memory\");");
-    em.line("tc_before();");
-    em.line("warp_arrive(tempty + tb, lane);  // T is in registers: the buffer is free for the next MMA");
-    for (size_t p = 0; p < pl.paths.size(); ++p) {
-      if (og[pl.paths[p].o] != g) continue;
-      for (int k = 0; k < 2 * pl.paths[p].l3 + 1; ++k) {
-        const int colm = colbase[p] + k;
-        size_t ch = 0;
-        while (!(colm >= chunks[ch].first && colm < chunks[ch].first + chunks[ch].second)) ++ch;
-        const std::string acc = "a" + S(pl.paths[p].out_off + k);
-        em.line(acc + " = fmaf(s" + S(p) + ", __uint_as_float(r" + S(ch) + "[" + S(colm - chunks[ch].first) + "]), " + acc + ");");
-      }
-    }
-    em.line("++v;");
-    em.ind--;
-    em.line("} else {");
-    em.line("  if (tid == 0) atomicOr(status, 2u);");
-    em.line("  warp_arrive(sempty + st, lane);");
-    em.line("}");
-    em.line("if (last) {");
-    em.line("  float* orow = out + b * " + S(o_row) + " + c;");
-    for (int o : outs) em.line("  orow[" + S(static_cast<long long>(o) * pl.C) + "] = a" + S(o) + " * inv_avg; a" + S(o) + " = 0.f;");
-    em.line("}");
-    em.line("++q;");
-    em.ind--;
-    em.line("}");
-    em.ind--;
-  }
-  em.line("}");
-  em.line("if (!ok && lane == 0) atomicOr(status, 4u);");
-  em.ind--;
+  em.line("if (!ok && tl == 0) atomicOr(status, 4u);");
+  em.line("// drain (bounded): the team's copies still in flight and its last MMA complete");
+  em.line("if (tl == 0) {");
+  em.line("  for (unsigned int k = q; k < qi; ++k) bar_wait(sfull + k % " + S(NS) + ", (k / " + S(NS) + ") & 1u);");
+  em.line("  if (v > 0u) bar_wait(tdone, (v - 1u) & 1u);");
   em.line("}");
   em.line("tc_before();");
   em.line("__syncthreads();");
