@@ -215,7 +215,7 @@ def test_tensor_core_tables_emulated_on_host():
     Y = np.random.default_rng(3).normal(size=c.ny)
     B = np.zeros((16, ncols))
     lanes = int(re.search(r"producer_threads=(\d+)", src).group(1))
-    loads = re.findall(r"const int2 k(\d+)_(\d+) = __ldg\(&e3_btab\[(\d+) \+ bt\]\);", src)
+    loads = re.findall(r"const int2 k(\d+)_(\d+) = __ldg\(&e3_btab\[(\d+) \+ tl\]\);", src)
     nrounds = max(int(r) for r, _, _ in loads) + 1
     assert nrounds == -(-541 // lanes)
     for r in range(nrounds):
@@ -230,12 +230,7 @@ def test_tensor_core_tables_emulated_on_host():
             i = ((off % 256) // 128) * 8 + (off % 16) // 2
             assert B[i, n] == 0
             B[i, n] = v
-    # T columns: the paths of output group 0 (the outputs whose accumulators the
-    # group-0 consumers declare), then those of group 1, each group in path order
-    g0 = re.search(r"output group 0[^\n]*\n\s*float ([^;]*);", src).group(1)
-    group0 = {int(m) for m in re.findall(r"a(\d+) = 0\.f", g0)}
-    order = ([p for p, q in enumerate(c.paths) if q.out_off in group0] +
-             [p for p, q in enumerate(c.paths) if q.out_off not in group0])
+    order = list(range(len(c.paths)))                # T columns in path order
     expect = np.zeros((16, ncols))
     col = 0
     for p in order:
