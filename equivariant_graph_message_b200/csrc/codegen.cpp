@@ -1036,9 +1036,9 @@ BTable tc_tables(const Plan& pl, const std::vector<AEntry>& ent, const std::vect
 //   2. build A = sum_j CG Y_j as float16 hi/lo K-major tiles (128 threads,
 //      branch-free, coefficient table in registers);
 //   3. one team barrier (bar.red.and.pred: also agrees on bounded-wait timeouts);
-//   4. the team leader issues T = x^T A_hi + x^T A_lo (tcgen05.mma, M = 128
-//      channels) and commits to the team's mbarrier; warp 0 refills the ring
-//      slot the barrier has just freed;
+//   4. a thread of warp 1 issues T = x^T A_hi + x^T A_lo (tcgen05.mma, M = 128
+//      channels) and commits to the team's mbarrier while warp 0 refills the
+//      ring slot the barrier has just freed;
 //   5. every thread loads its channel's s, waits for the commit, reads T from
 //      tensor memory in 32-column chunks and accumulates s * T in registers.
 // Several teams per SM overlap one another's latency.
@@ -1239,16 +1239,18 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("const unsigned short* ys = reinterpret_cast<const unsigned short*>(stg + " + S(sh.y_off) + ");");
   em.line("for (int j = lane; j < " + S(pl.ny) + "; j += 32) yfw[j] = h2f(ys[j]);");
   em.line("__syncwarp();");
+  em.line("// all loads and products first, then the float16 splits and the stores");
   for (int r = 0; r < tab.rounds; ++r) {
     std::string val = "__int_as_float(k" + S(r) + "_0.x) * yfw[k" + S(r) + "_0.y]";
     for (int t2 = 1; t2 < tab.terms[r]; ++t2)
       val = "fmaf(__int_as_float(k" + S(r) + "_" + S(t2) + ".x), yfw[k" + S(r) + "_" + S(t2) + ".y], " + val + ")";
-    em.line("{");
-    em.line("  const float val = " + val + ";");
-    em.line("  const unsigned short hi = f2h(val);");
-    em.line("  *reinterpret_cast<unsigned short*>(Bhi + off" + S(r) + ") = hi;");
-    em.line("  *reinterpret_cast<unsigned short*>(Blo + off" + S(r) + ") = f2h(val - h2f(hi));");
-    em.line("}");
+    em.line("const float v" + S(r) + " = " + val + ";");
+  }
+  for (int r = 0; r < tab.rounds; ++r)
+    em.line("const unsigned short h" + S(r) + " = f2h(v" + S(r) + "), l" + S(r) + " = f2h(v" + S(r) + " - h2f(h" + S(r) + "));");
+  for (int r = 0; r < tab.rounds; ++r) {
+    em.line("*reinterpret_cast<unsigned short*>(Bhi + off" + S(r) + ") = h" + S(r) + ";");
+    em.line("*reinterpret_cast<unsigned short*>(Blo + off" + S(r) + ") = l" + S(r) + ";");
   }
   em.line("fence_async_smem();");
   em.ind--;
@@ -1261,7 +1263,7 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("if (a == -2) break;");
   em.line("const long long b = hdr[4 * st + 1];");
   em.line("const int last = hdr[4 * st + 2];");
-  em.line("if (a >= 0 && tl == 0) {");
+  em.line("if (a >= 0 && tl == 32) {  // warp 1 issues the MMAs while warp 0 refills the ring");
   em.line("  const unsigned long long adesc = (unsigned long long)((smem_u32(stg) & 0x3FFFF) >> 4) | (128ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);");
   em.line("  const unsigned long long hdesc = (unsigned long long)((smem_u32(Bhi) & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
   em.line("  const unsigned long long ldesc = (unsigned long long)((smem_u32(Blo) & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
