@@ -62,11 +62,10 @@ struct Shape {
   bool tc = false;
   int ncols = 0;                              // sum over paths of 2l3+1, padded to 16
   int tmem_cols = 0;                          // tensor-memory columns allocated (power of 2)
-  int tbufs = 0, tstride = 0;                 // T buffers in tensor memory, columns between them
-  int bbufs = 0;                              // A tile buffers (each A_hi + A_lo)
+  int tbufs = 0, tstride = 0;                 // teams per block (one T each), columns between their T
   int b_stride = 0;                           // bytes from A_hi to A_lo (tile + scratch)
-  int b_off = 0, b_bytes = 0;                 // A_hi at b_off, A_lo at b_off + b_bytes
-  int mbar_off = 0, tslot_off = 0;            // MMA barrier, tensor-memory address slot
+  int b_off = 0, b_bytes = 0;                 // A_hi at b_off (b_bytes used by the MMA), A_lo at b_off + b_stride
+  int tslot_off = 0;                          // tensor-memory address slot
   int smem_request = 0;                       // dynamic shared memory requested per block
 };
 
