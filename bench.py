@@ -58,6 +58,8 @@ def parse_args():
     ap.add_argument("--contract-first", type=int, default=-1)
     ap.add_argument("--tensor-cores", type=int, default=0,
                     help="1: the tensor-core forward variant (float16 inputs, 128 channels)")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the supplementary timing of the tensor-core variant")
     return ap.parse_args()
 
 
@@ -410,6 +412,11 @@ def run_ours(args):
                  "roofline_times_ms": {k: 1000 * v for k, v in times.items()},
                  "traffic_source": traffic_src})
 
+    variants = None
+    if world == 1 and not info.get("tensor_cores") and not args.no_variants:
+        variants = {"tensor_cores": time_tensor_core_variant(args, spec, g, conv, x, Y, s, senders,
+                                                            row_ptr, out, stream)}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -444,11 +451,45 @@ def run_ours(args):
         "gpu_launches": launches,
         "clocks": clk,
     }
+    if variants is not None:
+        line["variants"] = variants
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def time_tensor_core_variant(args, spec, g, conv, x, Y, s, senders, row_ptr, out, stream):
+    """Supplementary: the opt-in tensor-core forward on the same resident inputs, after the
+    timed region (CUDA events, inputs larger than L2); None where the variant does not apply."""
+    import torch
+
+    import equivariant_graph_message_b200 as e3
+    tc = e3.Conv(spec.irreps_node, spec.irreps_sh, spec.irreps_out, g.avg_num_neighbors,
+                 dtype=spec.dtype)
+    tc.set_tensor_cores(1)
+    if not tc.kernel_info()["tensor_cores"]:
+        return None
+    N, E = g.num_nodes, g.num_edges
+    out_tc = torch.empty_like(out)
+    sh = e3._stream_handle(stream)
+    ptrs = [e3._ptr(t) for t in (x, Y, s, senders, row_ptr)]
+    for _ in range(max(3, args.warmup)):
+        tc.forward_raw(*ptrs, N, E, e3._ptr(out_tc), sh)
+    reps = max(5, min(args.steps, 20))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in ev:
+        a.record(stream)
+        tc.forward_raw(*ptrs, N, E, e3._ptr(out_tc), sh)
+        b.record(stream)
+    torch.cuda.synchronize()
+    assert tc.check(), "tensor-core variant reported a bad index or a wait timeout"
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    diff = ((out_tc - out).abs().max() / out.abs().max().clamp_min(1e-30)).item()
+    return {"forward_ms": ms, "edges_per_s": E / (ms / 1000.0), "launches": reps,
+            "max_abs_diff_vs_default_over_max_abs": diff, "kernel": tc.kernel_info(),
+            "note": "opt-in tcgen05/TMA/tensor-memory forward; not the headline (see roofline)"}
 
 
 def run_e2e(args, conv, spec, g, x, Y, s, senders, receivers, row_ptr, perm, ws, out, world, dev):
