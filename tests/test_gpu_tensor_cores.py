@@ -128,3 +128,30 @@ def test_tensor_core_few_nodes_no_edges_bad_indices(cuda_device):
     assert not conv.check()
     assert conv.check()
     assert torch.isfinite(out).all()
+
+
+def test_tensor_cores_full_size_sampled(cuda_device):
+    # the full large_f16 workload on the device through the tensor-core kernel, checked on 256
+    # seeded receivers (plus the first and last) against the oracle, and everywhere against
+    # the float32 staged path
+    from parity import DeviceWorkload, TOL
+    w = DeviceWorkload("large_f16")
+    w.conv.set_tensor_cores(1)
+    assert w.conv.kernel_info()["tensor_cores"] == 1
+    out = w.conv.forward(w.x, w.Y, w.s, w.senders, w.row_ptr)
+    torch.cuda.synchronize()
+    assert w.conv.check()
+    rng = np.random.default_rng(54321)
+    rows = np.unique(np.concatenate([[0, w.N - 1], rng.choice(w.N, 256, replace=False)]))
+    ref = w.sample_reference(rows)
+    gpu = out[torch.from_numpy(rows).cuda()].cpu().numpy()
+    err = column_scaled_error(gpu, ref)
+    assert err <= TOL["f16"], err
+    assert err <= 1e-5, err        # the hi/lo split keeps the product at float32 accuracy
+    w.conv.set_tensor_cores(0)
+    base = w.conv.forward(w.x, w.Y, w.s, w.senders, w.row_ptr)
+    torch.cuda.synchronize()
+    assert w.conv.check()
+    assert ((out - base).abs().max() / base.abs().max()).item() <= 1e-5
+    del w, out, base
+    torch.cuda.empty_cache()
