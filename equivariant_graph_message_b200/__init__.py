@@ -100,6 +100,21 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _require(name, t, device=None, dtype=None, numel=None):
+    """Checks a tensor handed to the library: a contiguous CUDA tensor (on `device`), of
+    `dtype` and with at least `numel` elements.  Host tensors never reach a kernel."""
+    if not getattr(t, "is_cuda", False):
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name} has {t.numel()} elements, needs {numel}")
+
+
 def _stream_handle(stream):
     import torch
     if stream is None:
@@ -211,9 +226,12 @@ class Conv:
         N = x.shape[0]
         E = senders.shape[0]
         want = torch.float16 if self.dtype == "f16" else torch.float32
-        for name, t in (("x", x), ("Y", Y), ("s", s)):
-            if t.dtype != want or not t.is_contiguous():
-                raise ValueError(f"{name} must be a contiguous {want} tensor")
+        _require("x", x, dtype=want)
+        dev = x.device
+        for name, t in (("Y", Y), ("s", s)):
+            _require(name, t, dev, want)
+        _require("senders", senders, dev, torch.int32)
+        _require("row_ptr", row_ptr, dev, torch.int32)
         if tuple(x.shape) != (N, self.nx, self.C):
             raise ValueError(f"x shape {tuple(x.shape)} != {(N, self.nx, self.C)}")
         if tuple(Y.shape) != (E, self.ny) or tuple(s.shape) != (E, self.num_paths, self.C):
@@ -224,6 +242,8 @@ class Conv:
             raise ValueError("row_ptr must have num_nodes + 1 entries")
         if out is None:
             out = torch.empty((N, self.nout, self.C), dtype=torch.float32, device=x.device)
+        else:
+            _require("out", out, dev, torch.float32, N * self.nout * self.C)
         _ok(_forward(self._h, _ptr(x), _ptr(Y) if E else None, _ptr(s) if E else None,
                      _ptr(senders) if E else None, _ptr(row_ptr), N, E, _ptr(out),
                      _stream_handle(stream)), "e3conv_forward")
@@ -254,16 +274,18 @@ def build_csr(receivers, num_nodes: int, row_ptr=None, perm=None, workspace=None
     """(row_ptr int32 [N+1], perm int32 [E]) of int32 device `receivers`."""
     import torch
     E = receivers.shape[0]
+    _require("receivers", receivers, dtype=torch.int32)
     dev = receivers.device
-    if receivers.dtype != torch.int32:
-        raise ValueError("receivers must be int32")
     if row_ptr is None:
         row_ptr = torch.empty(num_nodes + 1, dtype=torch.int32, device=dev)
+    _require("row_ptr", row_ptr, dev, torch.int32, num_nodes + 1)
     if perm is None:
         perm = torch.empty(max(E, 1), dtype=torch.int32, device=dev)[:E]
+    _require("perm", perm, dev, torch.int32, E)
     nbytes = csr_workspace_size(E, num_nodes)
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _require("workspace", workspace, dev, torch.uint8)
     _ok(_build_csr(_ptr(receivers) if E else None, E, num_nodes, _ptr(row_ptr),
                    _ptr(perm) if E else None, _ptr(workspace), workspace.numel(),
                    _stream_handle(stream)), "e3conv_build_csr")
@@ -275,12 +297,13 @@ def build_csr_noalloc(receivers, num_nodes: int, row_ptr=None, perm=None, stream
     (for callers that cannot allocate device memory; outputs may be passed in)."""
     import torch
     E = receivers.shape[0]
-    if receivers.dtype != torch.int32:
-        raise ValueError("receivers must be int32")
+    _require("receivers", receivers, dtype=torch.int32)
     if row_ptr is None:
         row_ptr = torch.empty(num_nodes + 1, dtype=torch.int32, device=receivers.device)
+    _require("row_ptr", row_ptr, receivers.device, torch.int32, num_nodes + 1)
     if perm is None:
         perm = torch.empty(max(E, 1), dtype=torch.int32, device=receivers.device)[:E]
+    _require("perm", perm, receivers.device, torch.int32, E)
     _ok(_build_csr_noalloc(_ptr(receivers) if E else None, E, num_nodes, _ptr(row_ptr),
                            _ptr(perm) if E else None, _stream_handle(stream)),
         "e3conv_build_csr_noalloc")
@@ -294,6 +317,7 @@ def csr_kernel_count(num_edges: int, num_nodes: int) -> int:
 
 
 def csr_check(workspace, stream=None) -> bool:
+    _require("workspace", workspace)
     rc = _csr_check(_ptr(workspace), _stream_handle(stream))
     if rc == ERR_BAD_INDEX:
         return False
@@ -305,9 +329,14 @@ def permute_rows(src, perm, dst=None, status=None, stream=None):
     """dst[t] = src[perm[t]] along the first axis (device)."""
     import torch
     rows = perm.shape[0]
+    _require("src", src)
+    _require("perm", perm, src.device, torch.int32)
     row_bytes = src[0].numel() * src.element_size() if src.shape[0] else 0
     if dst is None:
         dst = torch.empty((rows,) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    _require("dst", dst, src.device, src.dtype, rows * (src[0].numel() if src.shape[0] else 0))
+    if status is not None:
+        _require("status", status, src.device, torch.int32, 1)
     _ok(_permute(_ptr(src), src.shape[0], _ptr(perm), rows, row_bytes, _ptr(dst), _ptr(status),
                  _stream_handle(stream)), "e3conv_permute_rows")
     return dst

@@ -243,3 +243,26 @@ def test_tensor_core_tables_emulated_on_host():
         col += d3
     np.testing.assert_allclose(B, expect, atol=1e-5)
     assert (np.abs(expect) > 1e-9).sum() == 541
+
+
+def test_binding_rejects_host_tensors_before_any_library_call():
+    # host pointers never reach a kernel: every tensor is checked (CUDA, device, dtype,
+    # contiguity, size) in the binding
+    import torch
+    c = e3.Conv("4x0e+4x1o", "1x0e+1x1o+1x2e", "4x0e+4x1o", 5.0)
+    N, E = 3, 4
+    x = torch.zeros(N, c.nx, c.C)
+    Y = torch.zeros(E, c.ny)
+    s = torch.zeros(E, c.num_paths, c.C)
+    snd = torch.zeros(E, dtype=torch.int32)
+    rp = torch.zeros(N + 1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        c.forward(x, Y, s, snd, rp)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        e3.build_csr(torch.zeros(E, dtype=torch.int32), N)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        e3.build_csr_noalloc(torch.zeros(E, dtype=torch.int32), N)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        e3.permute_rows(torch.zeros(E, 2), torch.zeros(E, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        e3.csr_check(torch.zeros(16, dtype=torch.uint8))
