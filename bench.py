@@ -171,28 +171,37 @@ def traffic_for(workload, conv, E):
 # ---------------------------------------------------------------------------
 # oracle sample (CPU baseline and reference arm)
 
-def oracle_sample_rate(spec, graph, rows, x_rows_fn, Y_fn, s_fn, threads=0):
-    """Times the oracle on the receivers `rows` (all their edges); returns (edges/s, edges, secs)."""
+def prepare_sample(graph, rows, x_rows_fn, Y_fn, s_fn):
+    """The oracle's float64 inputs for the receivers `rows` and all their edges (generated once)."""
     import numpy as np
-
-    import oracle
     rp = np.zeros(graph.num_nodes + 1, np.int64)
     np.cumsum(np.bincount(graph.receivers, minlength=graph.num_nodes), out=rp[1:])
     edges = np.concatenate([np.arange(rp[b], rp[b + 1]) for b in rows])
     senders = graph.senders[edges]
     uniq, inv = np.unique(senders, return_inverse=True)
     x = x_rows_fn(uniq).astype(np.float64)
-    Y = Y_fn(edges).astype(np.float64)
-    s = s_fn(edges).astype(np.float64)
     n = max(len(rows), len(uniq))
     xr = np.zeros((n,) + x.shape[1:])
     xr[:len(uniq)] = x
-    recv = np.repeat(np.arange(len(rows)), np.diff(rp)[rows])
+    return {"x": xr, "Y": Y_fn(edges).astype(np.float64), "s": s_fn(edges).astype(np.float64),
+            "senders": inv, "receivers": np.repeat(np.arange(len(rows)), np.diff(rp)[rows]),
+            "n": n, "edges": len(edges)}
+
+
+def run_oracle(spec, graph, prep, threads=0):
+    """Times one oracle forward on a prepared sample; returns (edges/s, edges, secs)."""
+    import oracle
     t0 = time.perf_counter()
-    oracle.forward(spec.irreps_node, spec.irreps_sh, spec.irreps_out, xr, Y, s, inv, recv, n,
+    oracle.forward(spec.irreps_node, spec.irreps_sh, spec.irreps_out, prep["x"], prep["Y"],
+                   prep["s"], prep["senders"], prep["receivers"], prep["n"],
                    graph.avg_num_neighbors, threads=threads)
     dt = time.perf_counter() - t0
-    return len(edges) / dt, len(edges), dt
+    return prep["edges"] / dt, prep["edges"], dt
+
+
+def oracle_sample_rate(spec, graph, rows, x_rows_fn, Y_fn, s_fn, threads=0):
+    """Times the oracle on the receivers `rows` (all their edges); returns (edges/s, edges, secs)."""
+    return run_oracle(spec, graph, prepare_sample(graph, rows, x_rows_fn, Y_fn, s_fn), threads)
 
 
 def calibrated_rows(spec, graph, x_rows_fn, Y_fn, s_fn, target_s, seed=2024):
@@ -261,16 +270,30 @@ def run_reference(args):
     from workloads import configs
     spec = spec_for_rank(args.workload, 0)
     g = configs.make_graph(spec, args.nodes)
-    xf = lambda rows: configs.node_features_np(spec, g.num_nodes, rows)
-    yf = lambda edges: configs.real_sh(g.vec[edges], spec.lmax).astype(configs.np_dtype(spec))
-    sf = lambda edges: configs.scalars_np(spec, g, edges)
+    try:
+        import torch
+        on_gpu = torch.cuda.is_available()
+    except ImportError:
+        on_gpu = False
+    if on_gpu:
+        # the inputs are drawn with the counter generator's device form and the sample's rows
+        # copied to the host (the numpy form runs at ~6M values/s); the oracle runs on the host
+        dev = torch.device("cuda", 0)
+        xf, yf, sf = device_inputs_fns(configs.node_features_torch(spec, g.num_nodes, dev),
+                                       torch.from_numpy(configs.edge_sh(spec, g)).to(dev),
+                                       configs.scalars_torch(spec, g, dev))
+    else:
+        xf = lambda rows: configs.node_features_np(spec, g.num_nodes, rows)
+        yf = lambda edges: configs.real_sh(g.vec[edges], spec.lmax).astype(configs.np_dtype(spec))
+        sf = lambda edges: configs.scalars_np(spec, g, edges)
     per_step = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
     rows = calibrated_rows(spec, g, xf, yf, sf, per_step)
+    prep = prepare_sample(g, rows, xf, yf, sf)    # inputs generated once; steps time the oracle
     for _ in range(args.warmup):
-        oracle_sample_rate(spec, g, rows, xf, yf, sf)
+        run_oracle(spec, g, prep)
     tot_e, tot_t = 0, 0.0
     for _ in range(args.steps):
-        _, ne, dt = oracle_sample_rate(spec, g, rows, xf, yf, sf)
+        _, ne, dt = run_oracle(spec, g, prep)
         tot_e += ne
         tot_t += dt
     value = tot_e / tot_t
