@@ -141,9 +141,24 @@ int blocks_per_sm(const Shape& s, int regs, int block) {
 
 int compile_variant(Plan& pl, int dtype) {
   pl.auto_block = 0;
+  pl.tc_team_cap = 0;
   int rc = compile_once(pl, dtype);
   if (rc != E3CONV_OK) return rc;
   Variant& v = pl.var[dtype];
+  // Tensor-core variant that spills at three teams per block (168 registers): two teams
+  // (255 registers); if that still spills, the float32 staged variant.
+  if (v.shape.tc && v.local_bytes > 0 && v.shape.tbufs > 2) {
+    pl.tc_team_cap = 2;
+    rc = compile_once(pl, dtype);
+    if (rc != E3CONV_OK) return rc;
+  }
+  if (v.shape.tc && v.local_bytes > 0) {
+    const int keep = pl.req_tc;
+    pl.req_tc = 0;
+    rc = compile_once(pl, dtype);
+    pl.req_tc = keep;
+    if (rc != E3CONV_OK) return rc;
+  }
   if (v.shape.stages > 0 && !v.shape.tc && pl.req_block == 0 && v.regs > 0) {
     const int tt = 32 * v.shape.team;
     const int first_block = v.shape.block;

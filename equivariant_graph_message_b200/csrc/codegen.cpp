@@ -97,6 +97,7 @@ Shape choose_shape(const Plan& pl, int dtype) {
       s.tmem_cols = 512;
       s.tstride = align_up(ncols, 32);              // a team's T columns start on a 32-column boundary
       s.tbufs = std::min(3, 512 / s.tstride);       // teams per block: T columns fit in 512, registers in 64K
+      if (pl.tc_team_cap > 0) s.tbufs = std::min(s.tbufs, pl.tc_team_cap);
       s.block = 128 * s.tbufs;                      // four warps per team
       int S = pl.req_stages > 0 ? std::max(pl.req_stages, 2) : 4;
       s.x_off = 0;                                  // 16 rows x 128 channels x 2 B, two 128B-swizzled halves

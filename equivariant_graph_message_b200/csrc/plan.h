@@ -99,6 +99,7 @@ struct Plan {
   int auto_block = 0;                              // block chosen after a first compile (0: none)
   int req_coop = -1;                               // -1: automatic, 0: off, 1: on
   int req_tc = -1;                                 // -1: automatic, 0: off, 1: on
+  int tc_team_cap = 0;                             // > 0: at most this many tensor-core teams per block
   int device = -1;                 // -1: host-only plan
   CUcontext ctx = nullptr;
   unsigned int* status = nullptr;  // device status word

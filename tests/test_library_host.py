@@ -266,3 +266,36 @@ def test_binding_rejects_host_tensors_before_any_library_call():
         e3.permute_rows(torch.zeros(E, 2), torch.zeros(E, dtype=torch.int32))
     with pytest.raises(ValueError, match="CUDA tensor"):
         e3.csr_check(torch.zeros(16, dtype=torch.uint8))
+
+
+def test_tensor_core_kernels_fit_for_eligible_irreps_sets():
+    # float16, C = 128 sets of up to four node irreps (nx <= 16) with Y l <= 3: the
+    # tensor-core kernel compiles without spills, its teams' T columns fit the 512 of tensor
+    # memory, its ring stages start on 1024-byte boundaries (128-byte swizzle) and the block
+    # fits the 227 KB of shared memory
+    import itertools
+    irs = ["0e", "1o", "2e", "3o", "0o", "1e", "2o", "3e"]
+    out_all = "+".join("128x" + r for r in irs)
+    sh3 = "1x0e+1x1o+1x2e+1x3o"
+    eligible = [combo for k in (1, 2, 3, 4) for combo in itertools.combinations(irs, k)
+                if sum(2 * int(r[0]) + 1 for r in combo) <= 16]
+    assert len(eligible) == 130
+    # a deterministic subset (each compile takes seconds): every 12th set, the two sets that
+    # need the two-team fallback and the benchmark's irreps
+    picked = eligible[::12] + [("2e", "1e", "2o"), ("2e", "1e", "3e"), ("0e", "1o", "2e", "3o")]
+    seen = 0
+    for combo in picked:
+        c = e3.Conv("+".join("128x" + r for r in combo), sh3, out_all, 10.0, dtype="f16")
+        c.set_tensor_cores(1)
+        info = c.kernel_info()
+        assert info["tensor_cores"] == 1, combo
+        assert info["local_bytes"] == 0, (combo, info)
+        m = re.search(r"ncols=(\d+) teams=(\d+) tstride=(\d+) stages=(\d+) stage_bytes=(\d+) "
+                      r"team_bytes=(\d+)", c.kernel_source())
+        ncols, teams, tstride, stages, stage_bytes, team_bytes = map(int, m.groups())
+        assert ncols % 16 == 0 and ncols <= 256 and tstride >= ncols and tstride % 32 == 0
+        assert teams * tstride <= 512 and info["block_threads"] == 128 * teams
+        assert stages >= 3 and stage_bytes % 1024 == 0 and team_bytes % 1024 == 0
+        assert teams * team_bytes + 16 <= 227 * 1024
+        seen += 1
+    assert seen == len(picked)
