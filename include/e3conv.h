@@ -154,11 +154,12 @@ E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane,
  *   M = 128 channels, K = node components, N = path outputs; A = sum_j CG Y_j
  *   split into float16 hi + lo parts, float32 accumulation in tensor memory)
  *   and then scales T by the edge scalars with float32 FMAs.  It launches one
- *   block per SM (three teams of four warps; all 512 tensor-memory columns);
+ *   block per SM (three teams of four warps, or two where three would spill
+ *   registers; all 512 tensor-memory columns);
  *   a requested ring depth below 3 is raised to 3 and one that does not fit
  *   shared memory is lowered (e3conv_kernel_info reports the depth used).
- *   Requesting it for a shape outside those limits keeps the float32 staged
- *   variant. */
+ *   Requesting it for a shape outside those limits, or one whose kernel would
+ *   still spill, keeps the float32 staged variant. */
 #define E3CONV_OPT_TENSOR_CORES 2
 E3CONV_API int e3conv_set_option(e3conv_plan plan, int option, int value);
 
