@@ -362,7 +362,7 @@ def run_ours(args):
         e3._ok(e3._build_csr(precv, E, N, prp, pperm, pws, ws_bytes, sh), "e3conv_build_csr")
         if fwd_events:
             fwd_events[0].record(stream)
-        conv.forward_raw(px, pY, ps, psend, prp, N, E, pout, sh)
+        conv.forward_raw(px, pY, ps, psend, prp, N, pout, sh)
         if fwd_events:
             fwd_events[1].record(stream)
 
@@ -459,7 +459,9 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16 inputs, f32 accumulation" if spec.dtype == "f16" else "f32",
+        "data": "synthetic",
         "config": {"workload": spec.name, "description": spec.description, "nodes": N,
                    "edges": E, "edges_total": int(total_edges), "channels": conv.C,
                    "irreps_node": spec.irreps_node, "irreps_sh": spec.irreps_sh,
@@ -499,12 +501,12 @@ def time_tensor_core_variant(args, spec, g, conv, x, Y, s, senders, row_ptr, out
     sh = e3._stream_handle(stream)
     ptrs = [e3._ptr(t) for t in (x, Y, s, senders, row_ptr)]
     for _ in range(max(3, args.warmup)):
-        tc.forward_raw(*ptrs, N, E, e3._ptr(out_tc), sh)
+        tc.forward_raw(*ptrs, N, e3._ptr(out_tc), sh)
     reps = max(5, min(args.steps, 20))
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
     for a, b in ev:
         a.record(stream)
-        tc.forward_raw(*ptrs, N, E, e3._ptr(out_tc), sh)
+        tc.forward_raw(*ptrs, N, e3._ptr(out_tc), sh)
         b.record(stream)
     torch.cuda.synchronize()
     assert tc.check(), "tensor-core variant reported a bad index or a wait timeout"

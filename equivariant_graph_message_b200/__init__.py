@@ -57,8 +57,9 @@ OPT_CONTRACT_FIRST = 1
 OPT_TENSOR_CORES = 2
 _kernel_source = _sig("e3conv_kernel_source", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_char_p,
                       ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t))
-_forward = _sig("e3conv_forward", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp,
-                _vp)
+_forward = _sig("e3conv_forward", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp)
+_forward_rows = _sig("e3conv_forward_rows", ctypes.c_int, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
+                     _i64, _i64, _vp, _vp)
 _check = _sig("e3conv_check", ctypes.c_int, _vp, _vp)
 _csr_ws = _sig("e3conv_csr_workspace_size", ctypes.c_int, _i64, _i64,
                ctypes.POINTER(ctypes.c_size_t))
@@ -75,7 +76,7 @@ _version = _sig("e3conv_version", ctypes.c_int)
 EXPORTED = ["e3conv_create", "e3conv_destroy", "e3conv_set_input_dtype",
             "e3conv_set_launch_config", "e3conv_set_option", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
             "e3conv_output_irrep", "e3conv_cg", "e3conv_kernel_info", "e3conv_kernel_source",
-            "e3conv_forward", "e3conv_check", "e3conv_csr_workspace_size", "e3conv_build_csr",
+            "e3conv_forward", "e3conv_forward_rows", "e3conv_check", "e3conv_csr_workspace_size", "e3conv_build_csr",
             "e3conv_csr_check", "e3conv_build_csr_noalloc", "e3conv_csr_kernel_count", "e3conv_permute_rows", "e3conv_strerror", "e3conv_last_error",
             "e3conv_version"]
 
@@ -245,15 +246,52 @@ class Conv:
         else:
             _require("out", out, dev, torch.float32, N * self.nout * self.C)
         _ok(_forward(self._h, _ptr(x), _ptr(Y) if E else None, _ptr(s) if E else None,
-                     _ptr(senders) if E else None, _ptr(row_ptr), N, E, _ptr(out),
+                     _ptr(senders) if E else None, _ptr(row_ptr), N, _ptr(out),
                      _stream_handle(stream)), "e3conv_forward")
         return out
 
-    def forward_raw(self, x_ptr, Y_ptr, s_ptr, senders_ptr, row_ptr_ptr, num_nodes, num_edges,
-                    out_ptr, stream_handle):
+    def forward_rows(self, x, Y, s, senders, row_ptr, row_begin: int, row_end: int, out=None,
+                     stream=None):
+        """out[row_end-row_begin][nout][C] for the receiver rows [row_begin, row_end) of
+        row_ptr; Y, s and senders hold those rows' edges only, and x is the table the
+        senders index (any number of rows)."""
+        import torch
+        N = x.shape[0]
+        E = senders.shape[0]
+        want = torch.float16 if self.dtype == "f16" else torch.float32
+        _require("x", x, dtype=want)
+        dev = x.device
+        for name, t in (("Y", Y), ("s", s)):
+            _require(name, t, dev, want)
+        _require("senders", senders, dev, torch.int32)
+        _require("row_ptr", row_ptr, dev, torch.int32)
+        if tuple(x.shape) != (N, self.nx, self.C):
+            raise ValueError(f"x shape {tuple(x.shape)} != {(N, self.nx, self.C)}")
+        if tuple(Y.shape) != (E, self.ny) or tuple(s.shape) != (E, self.num_paths, self.C):
+            raise ValueError("Y / s shapes do not match the plan")
+        if not 0 <= row_begin <= row_end < row_ptr.shape[0]:
+            raise ValueError("rows must satisfy 0 <= row_begin <= row_end < len(row_ptr)")
+        rows = row_end - row_begin
+        if out is None:
+            out = torch.empty((rows, self.nout, self.C), dtype=torch.float32, device=dev)
+        else:
+            _require("out", out, dev, torch.float32, rows * self.nout * self.C)
+        _ok(_forward_rows(self._h, _ptr(x), N, _ptr(Y) if E else None, _ptr(s) if E else None,
+                          _ptr(senders) if E else None, _ptr(row_ptr), row_begin, row_end,
+                          _ptr(out), _stream_handle(stream)), "e3conv_forward_rows")
+        return out
+
+    def forward_raw(self, x_ptr, Y_ptr, s_ptr, senders_ptr, row_ptr_ptr, num_nodes, out_ptr,
+                    stream_handle):
         """Pointer-level call of e3conv_forward (for timing loops)."""
-        _ok(_forward(self._h, x_ptr, Y_ptr, s_ptr, senders_ptr, row_ptr_ptr, num_nodes,
-                     num_edges, out_ptr, stream_handle), "e3conv_forward")
+        _ok(_forward(self._h, x_ptr, Y_ptr, s_ptr, senders_ptr, row_ptr_ptr, num_nodes, out_ptr,
+                     stream_handle), "e3conv_forward")
+
+    def forward_rows_raw(self, x_ptr, num_nodes, Y_ptr, s_ptr, senders_ptr, row_ptr_ptr,
+                         row_begin, row_end, out_ptr, stream_handle):
+        """Pointer-level call of e3conv_forward_rows (for timing loops)."""
+        _ok(_forward_rows(self._h, x_ptr, num_nodes, Y_ptr, s_ptr, senders_ptr, row_ptr_ptr,
+                          row_begin, row_end, out_ptr, stream_handle), "e3conv_forward_rows")
 
     def check(self, stream=None) -> bool:
         """True if no forward since the last check met a bad index."""

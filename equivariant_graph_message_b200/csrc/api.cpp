@@ -118,8 +118,12 @@ int compile_once(Plan& pl, int dtype) {
   nvrtcDestroyProgram(&prog);
   std::smatch m;
   if (std::regex_search(v.log, m, std::regex("Used ([0-9]+) registers"))) v.regs = std::stoi(m[1]);
-  if (std::regex_search(v.log, m, std::regex("([0-9]+) bytes spill stores")))
-    v.local_bytes = std::stoi(m[1]);
+  // Local memory per thread: the stack frame (what the loaded function reports as
+  // CU_FUNC_ATTRIBUTE_LOCAL_SIZE_BYTES), or the spill stores if ptxas reports more.
+  int stack = 0, spill = 0;
+  if (std::regex_search(v.log, m, std::regex("([0-9]+) bytes stack frame"))) stack = std::stoi(m[1]);
+  if (std::regex_search(v.log, m, std::regex("([0-9]+) bytes spill stores"))) spill = std::stoi(m[1]);
+  v.local_bytes = std::max(stack, spill);
   v.compiled = true;
   return E3CONV_OK;
 }
@@ -142,21 +146,21 @@ int blocks_per_sm(const Shape& s, int regs, int block) {
 int compile_variant(Plan& pl, int dtype) {
   pl.auto_block = 0;
   pl.tc_team_cap = 0;
+  pl.tc_fallback = false;
   int rc = compile_once(pl, dtype);
   if (rc != E3CONV_OK) return rc;
   Variant& v = pl.var[dtype];
-  // Tensor-core variant that spills at three teams per block (168 registers): two teams
-  // (255 registers); if that still spills, the float32 staged variant.
+  // Tensor-core variant with local memory at three teams per block (168 registers): two
+  // teams (255 registers); if that still uses local memory, the float32 staged variant,
+  // kept for the rest of this compile (the block-size search below included).
   if (v.shape.tc && v.local_bytes > 0 && v.shape.tbufs > 2) {
     pl.tc_team_cap = 2;
     rc = compile_once(pl, dtype);
     if (rc != E3CONV_OK) return rc;
   }
   if (v.shape.tc && v.local_bytes > 0) {
-    const int keep = pl.req_tc;
-    pl.req_tc = 0;
+    pl.tc_fallback = true;
     rc = compile_once(pl, dtype);
-    pl.req_tc = keep;
     if (rc != E3CONV_OK) return rc;
   }
   if (v.shape.stages > 0 && !v.shape.tc && pl.req_block == 0 && v.regs > 0) {
@@ -497,19 +501,27 @@ int e3conv_kernel_source(e3conv_plan h, int dtype, char* buf, size_t buf_len, si
   return E3CONV_OK;
 }
 
-int e3conv_forward(e3conv_plan h, const void* x, const void* Y, const void* s,
-                   const int32_t* senders, const int32_t* row_ptr, int64_t num_nodes,
-                   int64_t num_edges, float* out, e3conv_stream stream) {
+}  // extern "C"
+
+namespace {
+
+// One launch of the plan's forward kernel over the receiver rows
+// [row_begin, row_end) of row_ptr; x holds num_nodes node rows (the senders' table).
+int launch_forward(e3conv_plan h, const void* x, int64_t num_nodes, const void* Y, const void* s,
+                   const int32_t* senders, const int32_t* row_ptr, int64_t row_begin,
+                   int64_t row_end, float* out, e3conv_stream stream) {
   if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
   Plan& pl = h->p;
-  if (num_nodes < 0 || num_edges < 0 || num_nodes >= (1ll << 31) || num_edges >= (1ll << 31))
-    return fail(E3CONV_ERR_INVALID_ARG, "num_nodes / num_edges out of range");
-  if (num_nodes == 0) return E3CONV_OK;
+  if (num_nodes < 0 || num_nodes >= (1ll << 31))
+    return fail(E3CONV_ERR_INVALID_ARG, "num_nodes out of range");
+  if (row_begin < 0 || row_end < row_begin || row_end >= (1ll << 31))
+    return fail(E3CONV_ERR_INVALID_ARG, "rows must satisfy 0 <= row_begin <= row_end < 2^31");
+  if (row_end == row_begin) return E3CONV_OK;
   if (!x || !row_ptr || !out)
     return fail(E3CONV_ERR_INVALID_ARG, "node_features, receiver_row_ptr and out are required");
-  if (num_edges > 0 && (!Y || !s || !senders))
-    return fail(E3CONV_ERR_INVALID_ARG, "edge_sh, edge_scalars and senders are required");
-  if (!aligned16(x) || !aligned16(out) || (num_edges > 0 && (!aligned16(Y) || !aligned16(s))))
+  // (edge buffers may be NULL only for a graph without edges in these rows: the edge
+  // count lives on the device, so this is the caller's promise, not a host check)
+  if (!aligned16(x) || !aligned16(out) || !aligned16(Y) || !aligned16(s))
     return fail(E3CONV_ERR_INVALID_ARG, "feature buffers must be 16-byte aligned");
   const Variant& v = pl.var[pl.dtype];
   if (pl.device < 0 || !v.fn) return fail(E3CONV_ERR_NO_DEVICE, "plan has no device module");
@@ -517,6 +529,7 @@ int e3conv_forward(e3conv_plan h, const void* x, const void* Y, const void* s,
   if (cudaGetDevice(&cur) != cudaSuccess || cur != pl.device)
     return fail(E3CONV_ERR_INVALID_ARG, "current device differs from the plan's device");
   const Shape& sh = v.shape;
+  const long long rows = row_end - row_begin;
   long long blocks;
   unsigned smem = 0;
   CUtensorMap xmap;
@@ -537,28 +550,45 @@ int e3conv_forward(e3conv_plan h, const void* x, const void* Y, const void* s,
                                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return fail(E3CONV_ERR_CUDA, "cuTensorMapEncodeTiled failed for node_features");
-    blocks = std::min<long long>(v.grid_blocks, num_nodes);
+    blocks = std::min<long long>(v.grid_blocks, rows);
     smem = static_cast<unsigned>(sh.smem_request);
   } else if (sh.stages > 0) {
     const long long tpb = sh.block / (32 * sh.team);  // teams per block
-    blocks = std::min<long long>(v.grid_blocks, (num_nodes + tpb - 1) / tpb);
+    blocks = std::min<long long>(v.grid_blocks, (rows + tpb - 1) / tpb);
     smem = static_cast<unsigned>(sh.warp_smem * tpb);
   } else {
-    const long long items = num_nodes * sh.tiles;
+    const long long items = rows * sh.tiles;
     const long long warps = (items + sh.ipw - 1) / sh.ipw;
     blocks = (warps * 32 + sh.block - 1) / sh.block;
   }
   if (blocks >= (1ll << 31)) return fail(E3CONV_ERR_UNSUPPORTED, "grid too large");
-  int n32 = static_cast<int>(num_nodes), e32 = static_cast<int>(num_edges);
+  int n32 = static_cast<int>(num_nodes), b32 = static_cast<int>(row_begin),
+      r32 = static_cast<int>(row_end);
   float inv_avg = static_cast<float>(1.0 / pl.avg);
   void* args[] = {const_cast<void**>(&x), const_cast<void**>(&Y), const_cast<void**>(&s),
                   const_cast<int32_t**>(&senders), const_cast<int32_t**>(&row_ptr),
-                  &n32, &e32, &out, &inv_avg, &pl.status, &xmap};
+                  &n32, &b32, &r32, &out, &inv_avg, &pl.status, &xmap};
   CUresult r = driver().LaunchKernel(v.fn, static_cast<unsigned>(blocks), 1, 1,
                                      static_cast<unsigned>(sh.block), 1, 1, smem,
                                      reinterpret_cast<CUstream>(stream), args, nullptr);
   if (r != CUDA_SUCCESS) return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed");
   return E3CONV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int e3conv_forward(e3conv_plan h, const void* x, const void* Y, const void* s,
+                   const int32_t* senders, const int32_t* row_ptr, int64_t num_nodes, float* out,
+                   e3conv_stream stream) {
+  return launch_forward(h, x, num_nodes, Y, s, senders, row_ptr, 0, num_nodes, out, stream);
+}
+
+int e3conv_forward_rows(e3conv_plan h, const void* x, int64_t num_nodes, const void* Y,
+                        const void* s, const int32_t* senders, const int32_t* row_ptr,
+                        int64_t row_begin, int64_t row_end, float* out, e3conv_stream stream) {
+  return launch_forward(h, x, num_nodes, Y, s, senders, row_ptr, row_begin, row_end, out, stream);
 }
 
 int e3conv_check(e3conv_plan h, e3conv_stream stream) {

@@ -80,7 +80,7 @@ Shape choose_shape(const Plan& pl, int dtype) {
 
   // Tensor-core variant: float16 inputs, 128 channels (the MMA's M), at most
   // 16 node components (one K step) and at most 256 path outputs (N).
-  const bool want_tc = pl.req_tc == 1;  // opt-in (E3CONV_OPT_TENSOR_CORES)
+  const bool want_tc = pl.req_tc == 1 && !pl.tc_fallback;  // opt-in (E3CONV_OPT_TENSOR_CORES)
   if (want_tc && pl.req_stages != 0 && dtype == E3CONV_F16 && pl.C == 128 && pl.nx <= 16 &&
       bytes_ok) {
     int ncols = 0;
@@ -424,26 +424,53 @@ void emit_acc_decl(Emitter& em, const Plan& pl, int V) {
   }
 }
 
-// Stores acc * scale (or zeros) at orow + comp*C (+ lane offset already applied).
+// Stores acc * scale (or zeros) at orow + comp*C (+ lane offset already applied);
+// with `add` the scaled sums are added to what the row already holds (a
+// previous chunk of the same row, written by the same lane).
 void emit_store(Emitter& em, const Plan& pl, int V, const std::string& orow, bool zero,
-                bool reset) {
+                bool reset, bool add = false) {
   for (int c = 0; c < pl.nout; ++c) {
     auto a = [&](int v) {
       return zero ? std::string("0.f") : "a" + S(c) + "_" + S(v) + " * inv_avg";
     };
     const std::string dst = orow + " + " + S(c * pl.C);
     if (V % 4 == 0) {
-      for (int v = 0; v < V; v += 4)
-        em.line("*reinterpret_cast<float4*>(" + dst + " + " + S(v) + ") = make_float4(" + a(v) +
-                ", " + a(v + 1) + ", " + a(v + 2) + ", " + a(v + 3) + ");");
+      for (int v = 0; v < V; v += 4) {
+        const std::string d = "reinterpret_cast<float4*>(" + dst + " + " + S(v) + ")";
+        if (add)
+          em.line("{ const float4 o_ = *" + d + "; *" + d + " = make_float4(o_.x + " + a(v) +
+                  ", o_.y + " + a(v + 1) + ", o_.z + " + a(v + 2) + ", o_.w + " + a(v + 3) + "); }");
+        else
+          em.line("*" + d + " = make_float4(" + a(v) + ", " + a(v + 1) + ", " + a(v + 2) + ", " +
+                  a(v + 3) + ");");
+      }
     } else if (V == 2) {
-      em.line("*reinterpret_cast<float2*>(" + dst + ") = make_float2(" + a(0) + ", " + a(1) + ");");
+      const std::string d = "reinterpret_cast<float2*>(" + dst + ")";
+      if (add)
+        em.line("{ const float2 o_ = *" + d + "; *" + d + " = make_float2(o_.x + " + a(0) +
+                ", o_.y + " + a(1) + "); }");
+      else
+        em.line("*" + d + " = make_float2(" + a(0) + ", " + a(1) + ");");
     } else {
-      em.line("*(" + dst + ") = " + a(0) + ";");
+      em.line("*(" + dst + ") " + (add ? "+= " : "= ") + a(0) + ";");
     }
     if (reset)
       for (int v = 0; v < V; ++v) em.line("a" + S(c) + "_" + S(v) + " = 0.f;");
   }
+}
+
+// Row flush of the scalar accumulators: store (first chunk of the row) or add.
+void emit_flush(Emitter& em, const Plan& pl, int V, const std::string& orow,
+                const std::string& add_cond, bool reset) {
+  em.line("if (" + add_cond + ") {");
+  em.ind++;
+  emit_store(em, pl, V, orow, false, reset, true);
+  em.ind--;
+  em.line("} else {");
+  em.ind++;
+  emit_store(em, pl, V, orow, false, reset, false);
+  em.ind--;
+  em.line("}");
 }
 
 void emit_signature(Emitter& em, const std::string& T, int block, int minb) {
@@ -452,9 +479,20 @@ void emit_signature(Emitter& em, const std::string& T, int block, int minb) {
   em.line("    const " + T + "* __restrict__ x, const " + T + "* __restrict__ Y, const " + T +
           "* __restrict__ s,");
   em.line("    const int* __restrict__ senders, const int* __restrict__ row_ptr,");
-  em.line("    int num_nodes, int num_edges, float* __restrict__ out, float inv_avg,");
+  em.line("    int num_nodes, int row_begin, int row_end, float* __restrict__ out, float inv_avg,");
   em.line("    unsigned int* __restrict__ status)");
 }
+
+// Edge range of the rows [row_begin, row_end): the edge buffers hold edges
+// e_base .. e_end-1 of row_ptr's numbering at local index e - e_base.
+void emit_edge_range(Emitter& em) {
+  em.line("const int e_base = __ldg(row_ptr + row_begin), e_end = __ldg(row_ptr + row_end);");
+}
+
+// A receiver row is summed in chunks of E3_ROW_CHUNK edges: each chunk in its
+// own float32 accumulators, the scaled chunk sums added into the output row.
+// Only rows longer than one chunk take the extra read-add-write.
+void emit_chunk_define(Emitter& em) { em.line("#define E3_ROW_CHUNK 128"); }
 
 std::string direct_source(const Plan& pl, int dtype, const Shape& sh) {
   Emitter em;
@@ -466,6 +504,7 @@ std::string direct_source(const Plan& pl, int dtype, const Shape& sh) {
           " paths=" + S(pl.paths.size()) + " dtype=" + (f16 ? "f16" : "f32") + " V=" + S(V) +
           " TL=" + S(sh.TL) + " tiles=" + S(sh.tiles) + " ipw=" + S(sh.ipw));
   emit_prelude(em);
+  emit_chunk_define(em);
   emit_signature(em, T, sh.block, 0);
   em.line("{");
   em.ind++;
@@ -475,30 +514,37 @@ std::string direct_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("const int within = lane - sub * " + S(sh.TL) + ";");
   em.line("if (sub >= " + S(sh.ipw) + ") return;");
   em.line("const long long item = gwarp * " + S(sh.ipw) + " + sub;");
-  em.line("const long long b = item / " + S(sh.tiles) + ";");
-  em.line("const int tile = (int)(item - b * " + S(sh.tiles) + ");");
-  em.line("if (b >= num_nodes) return;");
+  em.line("const long long b = row_begin + item / " + S(sh.tiles) + ";");
+  em.line("const int tile = (int)(item - (b - row_begin) * " + S(sh.tiles) + ");");
+  em.line("if (b >= row_end) return;");
   em.line("const int u0 = tile * " + S(sh.TL * V) + " + within * " + S(V) + ";");
   em.line("if (u0 >= " + S(pl.C) + ") return;");
+  emit_edge_range(em);
   emit_acc_decl(em, pl, V);
   em.line("int e0 = row_ptr[b];");
   em.line("int e1 = row_ptr[b + 1];");
-  em.line("if (e0 < 0 || e1 < e0 || e1 > num_edges) { atomicOr(status, 1u); e1 = e0; }");
+  em.line("if (e0 < e_base || e1 < e0 || e1 > e_end) { atomicOr(status, 1u); e1 = e0; }");
+  em.line("float* orow = out + (b - row_begin) * " + S(pl.nout * pl.C) + " + u0;");
   em.line("#pragma unroll 1");
   em.line("for (int e = e0; e < e1; ++e) {");
   em.ind++;
-  em.line("const int a = senders[e];");
+  em.line("if (e > e0 && (e - e0) % E3_ROW_CHUNK == 0) {  // chunk of a long row done");
+  em.ind++;
+  emit_flush(em, pl, V, "orow", "e - e0 > E3_ROW_CHUNK", true);
+  em.ind--;
+  em.line("}");
+  em.line("const long long le = e - e_base;  // local edge index");
+  em.line("const int a = senders[le];");
   em.line("if ((unsigned int)a >= (unsigned int)num_nodes) { atomicOr(status, 2u); continue; }");
-  em.line("const " + T + "* yr = Y + (long long)e * " + S(pl.ny) + ";");
+  em.line("const " + T + "* yr = Y + le * " + S(pl.ny) + ";");
   emit_y_load(em, pl, dtype, "ldg", "yr");
   em.line("const " + T + "* xr = x + (long long)a * " + S(pl.nx * pl.C) + " + u0;");
-  em.line("const " + T + "* sr = s + (long long)e * " +
+  em.line("const " + T + "* sr = s + le * " +
           S(static_cast<long long>(pl.paths.size()) * pl.C) + " + u0;");
   emit_edge_body(em, pl, dtype, V, "ldg", "xr", "sr");
   em.ind--;
   em.line("}");
-  em.line("float* orow = out + (long long)b * " + S(pl.nout * pl.C) + " + u0;");
-  emit_store(em, pl, V, "orow", false, false);
+  emit_flush(em, pl, V, "orow", "e1 - e0 > E3_ROW_CHUNK", false);
   em.ind--;
   em.line("}");
   return em.o.str();
@@ -751,21 +797,33 @@ void emit_group_acc_decl(Emitter& em, const Plan& pl, const Lanes& L) {
   }
 }
 
-void emit_group_store(Emitter& em, const Plan& pl, const Lanes& L, const std::string& orow) {
+// Stores the packed accumulators (times 1/N) at orow + comp*C and resets them;
+// with `add` the values are added to what the row already holds.
+void emit_group_store(Emitter& em, const Plan& pl, const Lanes& L, const std::string& orow,
+                      bool add = false) {
   for (int c = 0; c < pl.nout; ++c) {
     const std::string dst = orow + " + " + S(c * pl.C);
     if (!L.pairs()) {
-      em.line("*(" + dst + ") = q" + S(c) + "_0 * inv_avg;");
+      em.line("*(" + dst + ") " + (add ? "+= " : "= ") + "q" + S(c) + "_0 * inv_avg;");
       em.line("q" + S(c) + "_0 = 0.f;");
       continue;
     }
+    auto val = [&](int g, const std::string& old) {
+      const std::string m = "mul2(q" + S(c) + "_" + S(g) + ", inv2)";
+      return add ? "add2(" + old + ", " + m + ")" : m;
+    };
     for (int g = 0; g < L.groups(); g += 2) {
-      if (g + 1 < L.groups())
-        em.line("*reinterpret_cast<ulonglong2*>(" + dst + " + " + S(2 * g) + ") = make_ulonglong2(mul2(q" +
-                S(c) + "_" + S(g) + ", inv2), mul2(q" + S(c) + "_" + S(g + 1) + ", inv2));");
-      else
-        em.line("*reinterpret_cast<unsigned long long*>(" + dst + " + " + S(2 * g) + ") = mul2(q" + S(c) +
-                "_" + S(g) + ", inv2);");
+      if (g + 1 < L.groups()) {
+        const std::string d = "reinterpret_cast<ulonglong2*>(" + dst + " + " + S(2 * g) + ")";
+        if (add)
+          em.line("{ const ulonglong2 o_ = *" + d + "; *" + d + " = make_ulonglong2(" +
+                  val(g, "o_.x") + ", " + val(g + 1, "o_.y") + "); }");
+        else
+          em.line("*" + d + " = make_ulonglong2(" + val(g, "") + ", " + val(g + 1, "") + ");");
+      } else {
+        const std::string d = "reinterpret_cast<unsigned long long*>(" + dst + " + " + S(2 * g) + ")";
+        em.line("*" + d + " = " + val(g, "*" + d) + ";");
+      }
     }
     for (int g = 0; g < L.groups(); ++g) em.line("q" + S(c) + "_" + S(g) + " = 0ull;");
   }
@@ -794,6 +852,8 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("__device__ __forceinline__ unsigned long long bc(float a) { return pk(a, a); }");
   em.line("__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) { unsigned long long d; asm(\"fma.rn.f32x2 %0, %1, %2, %3;\" : \"=l\"(d) : \"l\"(a), \"l\"(b), \"l\"(c)); return d; }");
   em.line("__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) { unsigned long long d; asm(\"mul.rn.f32x2 %0, %1, %2;\" : \"=l\"(d) : \"l\"(a), \"l\"(b)); return d; }");
+  em.line("__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) { unsigned long long d; asm(\"add.rn.f32x2 %0, %1, %2;\" : \"=l\"(d) : \"l\"(a), \"l\"(b)); return d; }");
+  emit_chunk_define(em);
   if (sh.coop) {
     ent = build_a_entries(pl);
     tabs = coop_tables(ent, 32 * TW);
@@ -842,8 +902,9 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("const unsigned long long pol_keep = policy_evict_last();");
   em.line("const long long W = (long long)gridDim.x * " + S(teams) + ";  // teams in the grid");
   em.line("const int u0 = tl * " + S(V) + ";  // first channel of this lane");
-  em.line("long long pb = (long long)blockIdx.x * " + S(teams) + " + team - W;  // producer receiver");
-  em.line("int pe = 0, pe1 = 0;      // producer edge cursor within row pb");
+  emit_edge_range(em);
+  em.line("long long pb = row_begin + (long long)blockIdx.x * " + S(teams) + " + team - W;  // producer receiver");
+  em.line("int pe = 0, pe1 = 0, pr0 = 0;  // producer edge cursor within row pb, which starts at pr0");
   em.line("int pwin = -1, psw = 0;   // sender window base (edge index) and this lane's sender");
   em.line("bool pdone = false;");
   em.line("unsigned int ppos = 0, cpos = 0;");
@@ -859,12 +920,12 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.ind++;
   em.line("while (!pdone && pe >= pe1) {");
   em.line("  pb += W;");
-  em.line("  if (pb >= num_nodes) { pdone = true; break; }");
+  em.line("  if (pb >= row_end) { pdone = true; break; }");
   em.line("  int r0 = row_ptr[pb], r1 = row_ptr[pb + 1];");
-  em.line("  if (r0 < 0 || r1 < r0 || r1 > num_edges) { if (issuer) atomicOr(status, 1u); r1 = r0; }");
-  em.line("  pe = r0; pe1 = r1; pwin = -1;");
+  em.line("  if (r0 < e_base || r1 < r0 || r1 > e_end) { if (issuer) atomicOr(status, 1u); r1 = r0; }");
+  em.line("  pe = r0; pe1 = r1; pr0 = r0; pwin = -1;");
   em.line("  if (r0 == r1) {  // empty row: zeros");
-  em.line("    float* zrow = out + pb * " + S(o_row) + " + u0;");
+  em.line("    float* zrow = out + (pb - row_begin) * " + S(o_row) + " + u0;");
   em.ind += 2;
   emit_store(em, pl, V, "zrow", true, false);
   em.ind -= 2;
@@ -873,7 +934,7 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("if (pdone) return;");
   em.line("if (pwin < 0 || pe >= pwin + 32) {");
   em.line("  pwin = pe;");
-  em.line("  psw = (pe + lane < pe1) ? senders[pe + lane] : 0;");
+  em.line("  psw = (pe + lane < pe1) ? senders[pe + lane - e_base] : 0;");
   em.line("}");
   em.line("const int a = __shfl_sync(0xffffffffu, psw, pe - pwin);");
   em.line("const bool valid = (unsigned int)a < (unsigned int)num_nodes;");
@@ -881,14 +942,16 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("if (issuer) {");
   em.line("  unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
   em.line("  hdr[4 * st] = valid ? a : -1;");
-  em.line("  hdr[4 * st + 1] = (int)pb;");
-  em.line("  hdr[4 * st + 2] = (pe + 1 == pe1) ? 1 : 0;");
+  em.line("  hdr[4 * st + 1] = (int)(pb - row_begin);");
+  em.line("  // 1: last edge of the row, 2: last edge of a chunk, 4: an earlier chunk was flushed");
+  em.line("  hdr[4 * st + 2] = (pe + 1 == pe1 ? 1 : ((pe + 1 - pr0) % E3_ROW_CHUNK == 0 ? 2 : 0)) |");
+  em.line("                    (pe - pr0 >= E3_ROW_CHUNK ? 4 : 0);");
   em.line("  fence_async_smem();");
   em.line("  bar_expect(bars + st, " + S(sh.s_bytes + sh.y_bytes) + "u + (valid ? " +
           S(sh.x_bytes) + "u : 0u));");
-  em.line("  bulk_g2s(stg + " + S(sh.s_off) + ", s + (long long)pe * " + S(s_row) + ", " +
+  em.line("  bulk_g2s(stg + " + S(sh.s_off) + ", s + (long long)(pe - e_base) * " + S(s_row) + ", " +
           S(sh.s_bytes) + "u, bars + st, pol_stream);");
-  em.line("  bulk_g2s(stg + " + S(sh.y_off) + ", Y + (long long)pe * " + S(pl.ny) + ", " +
+  em.line("  bulk_g2s(stg + " + S(sh.y_off) + ", Y + (long long)(pe - e_base) * " + S(pl.ny) + ", " +
           S(sh.y_bytes) + "u, bars + st, pol_stream);");
   em.line("  if (valid) bulk_g2s(stg + " + S(sh.x_off) + ", x + (long long)a * " +
           S(static_cast<long long>(pl.nx) * pl.C) + ", " + S(sh.x_bytes) +
@@ -915,7 +978,7 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("const unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
   em.line("const int a = hdr[4 * st];");
   em.line("const long long b = hdr[4 * st + 1];");
-  em.line("const int last = hdr[4 * st + 2];");
+  em.line("const int flags = hdr[4 * st + 2];");
   em.line("if (a >= 0) {");
   em.ind++;
   if (sh.coop) {
@@ -931,13 +994,24 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("} else if (issuer) {");
   em.line("  atomicOr(status, 2u);");
   em.line("}");
-  em.line("if (last) {");
+  em.line("if (flags & 3) {  // row (or a chunk of a long row) complete");
   em.ind++;
   em.line("float* orow = out + b * " + S(o_row) + " + u0;");
+  em.line("if (flags & 4) {");
+  em.ind++;
+  if (sh.coop)
+    emit_group_store(em, pl, L, "orow", true);
+  else
+    emit_store(em, pl, V, "orow", false, true, true);
+  em.ind--;
+  em.line("} else {");
+  em.ind++;
   if (sh.coop)
     emit_group_store(em, pl, L, "orow");
   else
     emit_store(em, pl, V, "orow", false, true);
+  em.ind--;
+  em.line("}");
   em.ind--;
   em.line("}");
   em.line("team_sync();  // stage and A area free for reuse");
@@ -1075,6 +1149,7 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("__device__ __forceinline__ float h2f(unsigned short h) { float f; asm(\"cvt.f32.f16 %0, %1;\" : \"=f\"(f) : \"h\"(h)); return f; }");
   em.line("__device__ __forceinline__ unsigned short f2h(float f) { unsigned short h; asm(\"cvt.rn.f16.f32 %0, %1;\" : \"=h\"(h) : \"f\"(f)); return h; }");
   em.line("#define E3_SPIN_LIMIT (1u << 22)");
+  emit_chunk_define(em);
   em.line("struct __align__(64) E3TensorMap { unsigned long long v[16]; };");
   em.line("__device__ __forceinline__ unsigned int smem_u32(const void* p) { return static_cast<unsigned int>(__cvta_generic_to_shared(p)); }");
   em.line("__device__ __forceinline__ void bar_init(unsigned long long* b, unsigned int count) { asm volatile(\"mbarrier.init.shared::cta.b64 [%0], %1;\" :: \"r\"(smem_u32(b)), \"r\"(count) : \"memory\"); }");
@@ -1108,7 +1183,7 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("extern \"C\" __global__ void __launch_bounds__(" + S(sh.block) + ", 1) e3conv_fwd(");
   em.line("    const unsigned short* __restrict__ x, const unsigned short* __restrict__ Y,");
   em.line("    const unsigned short* __restrict__ s, const int* __restrict__ senders,");
-  em.line("    const int* __restrict__ row_ptr, int num_nodes, int num_edges, float* __restrict__ out,");
+  em.line("    const int* __restrict__ row_ptr, int num_nodes, int row_begin, int row_end, float* __restrict__ out,");
   em.line("    float inv_avg, unsigned int* __restrict__ status, const __grid_constant__ E3TensorMap xmap)");
   em.line("{");
   em.ind++;
@@ -1157,7 +1232,9 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("// row walk of warp 0 of the team, loads one row ahead: the open row [pe, pe1) of receiver");
   em.line("// pb with sender windows psw (edges pwin..) and psw2 (the next 32); the next row nb [n0, n1)");
   em.line("// with its first windows in flight; row_ptr of the row after (mb) in flight");
-  em.line("long long pb = -1, nb = (long long)blockIdx.x * " + S(TEAMS) + " + team, mb = nb + W;");
+  emit_edge_range(em);
+  em.line("long long pb = -1, nb = row_begin + (long long)blockIdx.x * " + S(TEAMS) + " + team, mb = nb + W;");
+  em.line("int pr0 = 0;  // first edge of the open row");
   em.line("int pe = 0, pe1 = 0, pwin = 0, psw = 0, psw2 = 0, n0 = 0, n1 = 0, nsw = 0, nsw2 = 0, m0 = 0, m1 = 0;");
   em.line("unsigned int qi = 0;  // positions issued");
   em.line("bool walk_done = false;");
@@ -1165,13 +1242,13 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("if (tw == 0) {");
   em.line("  pol_stream = policy_evict_first();");
   em.line("  pol_keep = policy_evict_last();");
-  em.line("  if (nb < num_nodes) {");
+  em.line("  if (nb < row_end) {");
   em.line("    n0 = row_ptr[nb]; n1 = row_ptr[nb + 1];");
-  em.line("    if (n0 < 0 || n1 < n0 || n1 > num_edges) { if (lane == 0) atomicOr(status, 1u); n1 = n0; }");
-  em.line("    nsw = (n0 + lane < n1) ? senders[n0 + lane] : 0;");
-  em.line("    nsw2 = (n0 + 32 + lane < n1) ? senders[n0 + 32 + lane] : 0;");
+  em.line("    if (n0 < e_base || n1 < n0 || n1 > e_end) { if (lane == 0) atomicOr(status, 1u); n1 = n0; }");
+  em.line("    nsw = (n0 + lane < n1) ? senders[n0 + lane - e_base] : 0;");
+  em.line("    nsw2 = (n0 + 32 + lane < n1) ? senders[n0 + 32 + lane - e_base] : 0;");
   em.line("  }");
-  em.line("  if (mb < num_nodes) { m0 = row_ptr[mb]; m1 = row_ptr[mb + 1]; }");
+  em.line("  if (mb < row_end) { m0 = row_ptr[mb]; m1 = row_ptr[mb + 1]; }");
   em.line("}");
   em.line("// issue position qi into stage qi % S (warp 0 of the team only)");
   em.line("auto issue = [&]() {");
@@ -1179,20 +1256,20 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("const unsigned int st = qi % " + S(NS) + ";");
   em.line("while (pe >= pe1) {  // open the next row");
   em.line("  pb = nb;");
-  em.line("  if (pb >= num_nodes) { walk_done = true; break; }");
-  em.line("  pe = n0; pe1 = n1; pwin = n0; psw = nsw; psw2 = nsw2;");
+  em.line("  if (pb >= row_end) { walk_done = true; break; }");
+  em.line("  pe = n0; pe1 = n1; pr0 = n0; pwin = n0; psw = nsw; psw2 = nsw2;");
   em.line("  if (pe == pe1) {");
-  em.line("    float* zrow = out + pb * " + S(o_row) + ";");
+  em.line("    float* zrow = out + (pb - row_begin) * " + S(o_row) + ";");
   em.line("    for (int k = lane; k < " + S(o_row) + "; k += 32) zrow[k] = 0.f;");
   em.line("  }");
   em.line("  nb = mb; n0 = m0; n1 = m1;");
-  em.line("  if (nb < num_nodes) {");
-  em.line("    if (n0 < 0 || n1 < n0 || n1 > num_edges) { if (lane == 0) atomicOr(status, 1u); n1 = n0; }");
-  em.line("    nsw = (n0 + lane < n1) ? senders[n0 + lane] : 0;");
-  em.line("    nsw2 = (n0 + 32 + lane < n1) ? senders[n0 + 32 + lane] : 0;");
+  em.line("  if (nb < row_end) {");
+  em.line("    if (n0 < e_base || n1 < n0 || n1 > e_end) { if (lane == 0) atomicOr(status, 1u); n1 = n0; }");
+  em.line("    nsw = (n0 + lane < n1) ? senders[n0 + lane - e_base] : 0;");
+  em.line("    nsw2 = (n0 + 32 + lane < n1) ? senders[n0 + 32 + lane - e_base] : 0;");
   em.line("  }");
   em.line("  mb = nb + W;");
-  em.line("  if (mb < num_nodes) { m0 = row_ptr[mb]; m1 = row_ptr[mb + 1]; }");
+  em.line("  if (mb < row_end) { m0 = row_ptr[mb]; m1 = row_ptr[mb + 1]; }");
   em.line("}");
   em.line("if (walk_done) {");
   em.line("  if (lane == 0) { hdr[4 * st] = -2; bar_arrive(sfull + st); }  // end marker");
@@ -1201,18 +1278,20 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("}");
   em.line("if (pe >= pwin + 32) {  // next window of the row");
   em.line("  pwin += 32; psw = psw2;");
-  em.line("  psw2 = (pwin + 32 + lane < pe1) ? senders[pwin + 32 + lane] : 0;");
+  em.line("  psw2 = (pwin + 32 + lane < pe1) ? senders[pwin + 32 + lane - e_base] : 0;");
   em.line("}");
   em.line("const int a = __shfl_sync(0xffffffffu, psw, pe - pwin);");
   em.line("const bool valid = (unsigned int)a < (unsigned int)num_nodes;");
   em.line("if (lane == 0) {");
   em.line("  unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
   em.line("  hdr[4 * st] = valid ? a : -1;");
-  em.line("  hdr[4 * st + 1] = (int)pb;");
-  em.line("  hdr[4 * st + 2] = (pe + 1 == pe1) ? 1 : 0;");
+  em.line("  hdr[4 * st + 1] = (int)(pb - row_begin);");
+  em.line("  // 1: last edge of the row, 2: last edge of a chunk, 4: an earlier chunk was flushed");
+  em.line("  hdr[4 * st + 2] = (pe + 1 == pe1 ? 1 : ((pe + 1 - pr0) % E3_ROW_CHUNK == 0 ? 2 : 0)) |");
+  em.line("                    (pe - pr0 >= E3_ROW_CHUNK ? 4 : 0);");
   em.line("  bar_expect(sfull + st, " + S(sh.s_bytes + sh.y_bytes) + "u + (valid ? 4096u : 0u));");
-  em.line("  bulk_g2s(stg + " + S(sh.s_off) + ", s + (long long)pe * " + S(s_row) + ", " + S(sh.s_bytes) + "u, sfull + st, pol_stream);");
-  em.line("  bulk_g2s(stg + " + S(sh.y_off) + ", Y + (long long)pe * " + S(pl.ny) + ", " + S(sh.y_bytes) + "u, sfull + st, pol_stream);");
+  em.line("  bulk_g2s(stg + " + S(sh.s_off) + ", s + (long long)(pe - e_base) * " + S(s_row) + ", " + S(sh.s_bytes) + "u, sfull + st, pol_stream);");
+  em.line("  bulk_g2s(stg + " + S(sh.y_off) + ", Y + (long long)(pe - e_base) * " + S(pl.ny) + ", " + S(sh.y_bytes) + "u, sfull + st, pol_stream);");
   em.line("  if (valid) tma_x_g2s(stg, &xmap, a, sfull + st, pol_keep);");
   em.line("}");
   em.line("__syncwarp();");
@@ -1263,7 +1342,7 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("const int a = hdr[4 * st];");
   em.line("if (a == -2) break;");
   em.line("const long long b = hdr[4 * st + 1];");
-  em.line("const int last = hdr[4 * st + 2];");
+  em.line("const int flags = hdr[4 * st + 2];");
   em.line("if (a >= 0 && tl == 32) {  // warp 1 issues the MMAs while warp 0 refills the ring");
   em.line("  const unsigned long long adesc = (unsigned long long)((smem_u32(stg) & 0x3FFFF) >> 4) | (128ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);");
   em.line("  const unsigned long long hdesc = (unsigned long long)((smem_u32(Bhi) & 0x3FFFF) >> 4) | (8ull << 16) | (16ull << 32) | (1ull << 46);");
@@ -1299,9 +1378,13 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("} else if (tl == 0) {");
   em.line("  atomicOr(status, 2u);");
   em.line("}");
-  em.line("if (last) {");
+  em.line("if (flags & 3) {  // row (or a chunk of a long row) complete");
   em.line("  float* orow = out + b * " + S(o_row) + " + tl;");
-  for (int c = 0; c < pl.nout; ++c) em.line("  orow[" + S(static_cast<long long>(c) * pl.C) + "] = a" + S(c) + " * inv_avg; a" + S(c) + " = 0.f;");
+  em.line("  if (flags & 4) {");
+  for (int c = 0; c < pl.nout; ++c) em.line("    orow[" + S(static_cast<long long>(c) * pl.C) + "] += a" + S(c) + " * inv_avg; a" + S(c) + " = 0.f;");
+  em.line("  } else {");
+  for (int c = 0; c < pl.nout; ++c) em.line("    orow[" + S(static_cast<long long>(c) * pl.C) + "] = a" + S(c) + " * inv_avg; a" + S(c) + " = 0.f;");
+  em.line("  }");
   em.line("}");
   em.line("++q;");
   em.ind--;

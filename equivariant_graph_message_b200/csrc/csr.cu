@@ -353,8 +353,8 @@ int csr_build(const int* recv, int64_t E, int64_t N, int* row_ptr, int* perm, vo
 // e3conv_build_csr_noalloc in e3conv.h).  The scratch is a file-scope device
 // array, so every GPU that loads this library holds kStaticScratchBytes of it
 // until the process exits.  Host code cannot use the array's name as a device
-// address (it names a host-side shadow); its device address is looked up once
-// per device with cudaGetSymbolAddress, with that device current.
+// address (it names a host-side shadow); its device address on the current
+// device is looked up with cudaGetSymbolAddress on every call.
 
 constexpr size_t kStaticScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) unsigned char g_csr_scratch[kStaticScratchBytes];
@@ -375,27 +375,14 @@ int csr_build_static(const int* recv, int64_t E, int64_t N, int* row_ptr, int* p
     err = "no current CUDA device";
     return E3CONV_ERR_CUDA;
   }
-  constexpr int kMaxDevices = 64;
-  static std::mutex mu;
-  static void* addr[kMaxDevices] = {};
-  if (dev >= kMaxDevices) {
-    err = "device ordinal above 63";
-    return E3CONV_ERR_UNSUPPORTED;
-  }
+  // The array's device address on the current device, looked up on every call (the
+  // lookup is cheap once the module is loaded, and a cached address would go stale if
+  // the caller reset the device).
   void* ptr = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-      void* p = nullptr;
-      // set-up, once per device, with that device current
-      if (cudaGetSymbolAddress(&p, g_csr_scratch) != cudaSuccess || !p) {
-        cudaGetLastError();
-        err = "cudaGetSymbolAddress of the static CSR scratch failed";
-        return E3CONV_ERR_CUDA;
-      }
-      addr[dev] = p;
-    }
-    ptr = addr[dev];
+  if (cudaGetSymbolAddress(&ptr, g_csr_scratch) != cudaSuccess || !ptr) {
+    cudaGetLastError();
+    err = "cudaGetSymbolAddress of the static CSR scratch failed";
+    return E3CONV_ERR_CUDA;
   }
   return csr_build(recv, E, N, row_ptr, perm, ptr, kStaticScratchBytes, st, err, nullptr);
 }

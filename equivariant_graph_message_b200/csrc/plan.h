@@ -81,7 +81,7 @@ struct Variant {
   std::string source;
   std::vector<char> cubin;
   std::string log;
-  int regs = -1, local_bytes = -1;
+  int regs = -1, local_bytes = -1;  // registers per thread; local memory per thread (stack frame)
   CUmodule module = nullptr;
   CUfunction fn = nullptr;
   int grid_blocks = 0;  // persistent grid of the staged variant (blocks per SM x SMs)
@@ -100,6 +100,7 @@ struct Plan {
   int req_coop = -1;                               // -1: automatic, 0: off, 1: on
   int req_tc = -1;                                 // -1: automatic, 0: off, 1: on
   int tc_team_cap = 0;                             // > 0: at most this many tensor-core teams per block
+  bool tc_fallback = false;                        // tensor cores requested but the kernel spills: float32 variant
   int device = -1;                 // -1: host-only plan
   CUcontext ctx = nullptr;
   unsigned int* status = nullptr;  // device status word

@@ -156,10 +156,10 @@ E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane,
  *   and then scales T by the edge scalars with float32 FMAs.  It launches one
  *   block per SM (three teams of four warps, or two where three would spill
  *   registers; all 512 tensor-memory columns);
- *   a requested ring depth below 3 is raised to 3 and one that does not fit
- *   shared memory is lowered (e3conv_kernel_info reports the depth used).
+ *   a requested ring depth is used from 2 up, one that does not fit shared
+ *   memory is lowered (e3conv_kernel_info reports the depth used).
  *   Requesting it for a shape outside those limits, or one whose kernel would
- *   still spill, keeps the float32 staged variant. */
+ *   still use local memory with two teams, keeps the float32 staged variant. */
 #define E3CONV_OPT_TENSOR_CORES 2
 E3CONV_API int e3conv_set_option(e3conv_plan plan, int option, int value);
 
@@ -202,26 +202,54 @@ E3CONV_API int e3conv_kernel_source(e3conv_plan plan, int dtype, char* buf, size
  * 1/N scale -> store of e3j's four plain steps; one kernel launch)
  *
  * node_features: device, [num_nodes][nx][C] of the plan's dtype.
- * edge_sh:       device, [num_edges][ny], receiver-sorted.
- * edge_scalars:  device, [num_edges][P][C], receiver-sorted.
- * senders:       device int32 [num_edges], receiver-sorted, in [0, num_nodes).
- * receiver_row_ptr: device int32 [num_nodes+1], nondecreasing, row_ptr[0] = 0,
- *                row_ptr[num_nodes] = num_edges (e3conv_build_csr makes it).
+ * edge_sh:       device, [E][ny], receiver-sorted.
+ * edge_scalars:  device, [E][P][C], receiver-sorted.
+ * senders:       device int32 [E], receiver-sorted, in [0, num_nodes).
+ * receiver_row_ptr: device int32 [num_nodes+1], nondecreasing, row_ptr[0] = 0
+ *                (e3conv_build_csr makes it).
  * out:           device float32 [num_nodes][nout][C]; fully overwritten
  *                (rows of receivers without edges become 0).
- * All buffers must be 16-byte aligned.  0 <= num_nodes, num_edges < 2^31.
- * With num_nodes == 0 nothing is launched; with num_edges == 0 the edge
- * pointers may be NULL.
- * Out-of-range senders are skipped and row ranges outside [0, num_edges]
- * are treated as empty; both set the plan's status word (e3conv_check).
- * The staged variant's bounded waits on its shared-memory ring, if they
- * ever time out, also set the status word and end the kernel early.
+ * The edge count is E = receiver_row_ptr[num_nodes]; it stays on the device
+ * (the kernel reads it; the host never does), so the edge buffers must hold
+ * at least that many rows.  Edge buffers may be NULL only when E = 0.
+ * Feature buffers must be 16-byte aligned.  0 <= num_nodes < 2^31, E < 2^31.
+ * With num_nodes == 0 nothing is launched.
+ * Out-of-range senders are skipped, and row ranges that decrease or leave
+ * [row_ptr[0], row_ptr[num_nodes]] are treated as empty; both set the plan's
+ * status word (e3conv_check).  The staged and tensor-core variants' bounded
+ * waits on their shared-memory rings, if they ever time out, also set the
+ * status word and end the kernel early.
+ * Each receiver row is summed in float32, in chunks of 128 edges whose scaled
+ * sums are added in the output row (rows of up to 128 edges: one chunk).
  * Launches exactly one kernel on `stream`; no host synchronisation, no
  * allocation.  Concurrent forwards with one plan share its status word. */
 E3CONV_API int e3conv_forward(e3conv_plan plan, const void* node_features, const void* edge_sh,
-                   const void* edge_scalars, const int32_t* senders,
-                   const int32_t* receiver_row_ptr, int64_t num_nodes, int64_t num_edges,
-                   float* out, e3conv_stream stream);
+                              const void* edge_scalars, const int32_t* senders,
+                              const int32_t* receiver_row_ptr, int64_t num_nodes, float* out,
+                              e3conv_stream stream);
+
+/* The forward over the receiver rows row_begin .. row_end-1 only: the rows a
+ * rank owns when receivers are partitioned into contiguous CSR row ranges
+ * (one output row per receiver, so no reduction across ranks follows).
+ *   node_features: [num_nodes][nx][C], the table the senders index: every
+ *                  node a sender may name (on a rank: its own rows plus the
+ *                  rows received from the others).
+ *   receiver_row_ptr: device int32; entries row_begin .. row_end are read,
+ *                  nondecreasing; the edges of row b are row_ptr[b] ..
+ *                  row_ptr[b+1]-1 in row_ptr's numbering.
+ *   edge_sh, edge_scalars, senders: the edges of these rows only, edge e of
+ *                  row_ptr's numbering at index e - receiver_row_ptr[row_begin].
+ *   out:           [row_end - row_begin][nout][C], row b at b - row_begin.
+ * 0 <= row_begin <= row_end < 2^31 (the row count need not equal num_nodes);
+ * nothing is launched for an empty range.  e3conv_forward is this call with
+ * row_begin = 0 and row_end = num_nodes.  A row's result does not depend on
+ * the range it is computed in: the same rows give bitwise the same output.
+ * Everything else as e3conv_forward. */
+E3CONV_API int e3conv_forward_rows(e3conv_plan plan, const void* node_features, int64_t num_nodes,
+                                   const void* edge_sh, const void* edge_scalars,
+                                   const int32_t* senders, const int32_t* receiver_row_ptr,
+                                   int64_t row_begin, int64_t row_end, float* out,
+                                   e3conv_stream stream);
 
 /* Synchronises `stream`, reads and clears the plan's status word.  Returns
  * E3CONV_OK, E3CONV_ERR_BAD_INDEX if a forward since the last check met an
@@ -264,9 +292,10 @@ E3CONV_API int e3conv_build_csr(const int32_t* receivers, int64_t num_edges, int
  *   - Sizes whose workspace (e3conv_csr_workspace_size) exceeds 32 MiB are
  *     rejected with E3CONV_ERR_WORKSPACE before anything is launched (about
  *     two million edges fit).
- *   - The first call on a device looks up the array's device address with
- *     cudaGetSymbolAddress (with that device current); make that first call
- *     before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     with cudaGetSymbolAddress (the first call on a device also loads the
+ *     library's device code there); make the first call on a device before
+ *     any stream capture.
  *   - All calls share the one array, which keeps the last call's contents:
  *     every call clears what must start at zero itself, but two calls whose
  *     work overlaps on the GPU (different streams, or different host threads,

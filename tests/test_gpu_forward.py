@@ -123,9 +123,10 @@ def test_no_edges_and_isolated_nodes(cuda_device):
 
 
 def test_single_node_and_hub(cuda_device):
-    # Rows of ordinary degree meet the 1e-5 bar.  A hub row of 6000 edges sums
-    # ~10^5 float32 products in one chain; it is checked elementwise against the
-    # recursive-summation bound of that arithmetic instead (parity.abs_bound).
+    # Every row, the 6000-edge hub row included, meets the 1e-5 column-scaled bar: a row
+    # is summed in chunks of 128 edges whose scaled sums are added in the output row.  The
+    # elementwise recursive-summation bound of float32 arithmetic (parity.abs_bound) holds
+    # as well.
     irreps = ("32x0e+32x1o+32x2e", "1x0e+1x1o+1x2e+1x3o", "32x0e+32x1o+32x2e+32x3o")
     pl = oracle.plan(*irreps)
     rng = np.random.default_rng(4)
@@ -140,7 +141,8 @@ def test_single_node_and_hub(cuda_device):
         bound = abs_bound(irreps, x, Y, s, send, recv, n, 40.0)
         assert np.all(np.abs(gpu - ref) <= bound + 1e-12)
         if hub is not None:
-            # (with a single row the column scale is the value itself, so only the bound applies)
+            assert column_scaled_error(gpu, ref) <= 1e-5
+            # the other rows scaled by their own columns' maxima, without the hub
             rows = np.setdiff1d(np.arange(n), [hub])
             assert column_scaled_error(gpu[rows], ref[rows]) <= 1e-5
 
@@ -167,7 +169,7 @@ def test_bad_indices_are_flagged_not_faulted(cuda_device):
     ref = oracle_out(irreps, x.cpu().numpy(), Y.cpu().numpy()[keep], s.cpu().numpy()[keep],
                      send[keep], recv[keep], n, 1.0)
     assert column_scaled_error(out.cpu().numpy(), ref) <= 1e-5
-    # a row range beyond num_edges and a decreasing one are treated as empty
+    # a row range beyond row_ptr[num_nodes] and a decreasing one are treated as empty
     bad_rp = row_ptr_of(recv, n).astype(np.int32)
     bad_rp[2] = e + 100
     conv.forward(x, Y, s, to_dev(send.astype(np.int32)), to_dev(bad_rp))

@@ -17,8 +17,8 @@ CASES = {
     "nx9": ("128x0e+128x1o+128x2e", SH3, "128x0e+128x1o+128x2e+128x1e+128x2o"),   # K rows 9..15 zero
     "nx4": ("128x0e+128x1o", SH3, "128x0e+128x1o+128x2e+128x1e+128x3o"),
     "odd_in": ("128x1o+128x0e+128x2o", SH3, "128x0e+128x0o+128x1e+128x1o+128x2e+128x3e+128x3o"),
-    # spills at three teams per block: compiled with two (256 threads)
-    "two_teams": ("128x2e+128x1e+128x2o", SH3,
+    # no scalar input irrep; every path starts from l1 = 1 or 2
+    "l12_inputs": ("128x2e+128x1e+128x2o", SH3,
                   "128x0e+128x0o+128x1e+128x1o+128x2e+128x2o+128x3e+128x3o"),
 }
 

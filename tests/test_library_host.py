@@ -165,30 +165,56 @@ def test_host_only_plan_forward_reports_no_device():
     if torch.cuda.is_available():
         pytest.skip("a device is present; covered by the GPU tests")
     c = e3.Conv("1x0e", "1x0e", "1x0e", 1.0)
-    rc = e3._forward(c._h, ctypes.c_void_p(16), None, None, None, ctypes.c_void_p(16), 1, 0,
+    rc = e3._forward(c._h, ctypes.c_void_p(16), None, None, None, ctypes.c_void_p(16), 1,
                      ctypes.c_void_p(16), None)
     assert rc == 7
     ws = ctypes.c_size_t()
     assert e3._csr_ws(10, 5, ctypes.byref(ws)) == 0 and ws.value > 0
 
 
+def test_forward_signature_has_no_host_edge_count():
+    # e3conv_forward(plan, x, Y, s, senders, row_ptr, num_nodes, out, stream): the edge count
+    # is row_ptr[num_nodes], read on the device only
+    import inspect
+    header = open(os.path.join(ROOT, "include", "e3conv.h")).read()
+    decl = header[header.index("E3CONV_API int e3conv_forward("):]
+    decl = decl[:decl.index(";")]
+    args = [a.split()[-1].strip("*") for a in decl[decl.index("(") + 1:decl.rindex(")")].split(",")]
+    assert args == ["plan", "node_features", "edge_sh", "edge_scalars", "senders",
+                    "receiver_row_ptr", "num_nodes", "out", "stream"]
+    assert len(e3._forward.argtypes) == 9
+    assert "num_edges" not in inspect.signature(e3.Conv.forward_raw).parameters
+
+
 def test_forward_argument_validation_precedes_device():
     c = e3.Conv("1x0e", "1x0e", "1x0e", 1.0)
-    assert e3._forward(c._h, None, None, None, None, None, -1, 0, None, None) == 1
-    assert e3._forward(c._h, None, None, None, None, None, 0, 0, None, None) == 0   # nothing to do
-    assert e3._forward(c._h, None, None, None, None, None, 3, 0, None, None) == 1
-    # misaligned feature buffer
-    assert e3._forward(c._h, ctypes.c_void_p(18), None, None, None, ctypes.c_void_p(16), 3, 0,
+    assert e3._forward(c._h, None, None, None, None, None, -1, None, None) == 1
+    assert e3._forward(c._h, None, None, None, None, None, 0, None, None) == 0   # nothing to do
+    assert e3._forward(c._h, None, None, None, None, None, 3, None, None) == 1
+    # misaligned feature buffers
+    assert e3._forward(c._h, ctypes.c_void_p(18), None, None, None, ctypes.c_void_p(16), 3,
                        ctypes.c_void_p(16), None) == 1
+    assert e3._forward(c._h, ctypes.c_void_p(16), ctypes.c_void_p(20), None, None,
+                       ctypes.c_void_p(16), 3, ctypes.c_void_p(16), None) == 1
     assert e3._build_csr(None, -1, 3, None, None, None, 0, None) == 1
+
+
+def test_forward_rows_range_validation():
+    c = e3.Conv("1x0e", "1x0e", "1x0e", 1.0)
+    p16 = ctypes.c_void_p(16)
+    fr = e3._forward_rows
+    assert fr(c._h, p16, 10, p16, p16, p16, p16, -1, 5, p16, None) == 1      # begin < 0
+    assert fr(c._h, p16, 10, p16, p16, p16, p16, 6, 5, p16, None) == 1       # end < begin
+    assert fr(c._h, p16, 10, p16, p16, p16, p16, 0, 1 << 31, p16, None) == 1  # end >= 2^31
+    assert fr(c._h, None, 10, None, None, None, None, 4, 4, None, None) == 0  # empty range
+    assert fr(c._h, p16, 1 << 31, p16, p16, p16, p16, 0, 1, p16, None) == 1
 
 
 def test_size_limits_rejected_on_host():
     # indices are int32: sizes of 2^31 and above are refused before any launch
     c = e3.Conv("1x0e", "1x0e", "1x0e", 1.0)
     p16 = ctypes.c_void_p(16)
-    assert e3._forward(c._h, p16, p16, p16, p16, p16, 1, 1 << 31, p16, None) == 1
-    assert e3._forward(c._h, p16, p16, p16, p16, p16, 1 << 31, 1, p16, None) == 1
+    assert e3._forward(c._h, p16, p16, p16, p16, p16, 1 << 31, p16, None) == 1
     n = ctypes.c_size_t()
     assert e3._csr_ws(1 << 31, 10, ctypes.byref(n)) == 1
     assert e3._csr_ws(10, (1 << 31) - 1, ctypes.byref(n)) == 1
@@ -299,3 +325,25 @@ def test_tensor_core_kernels_fit_for_eligible_irreps_sets():
         assert teams * team_bytes + 16 <= 227 * 1024
         seen += 1
     assert seen == len(picked)
+
+
+@pytest.mark.parametrize("stages", [2, 4])
+@pytest.mark.parametrize("combo", [("2e", "1e", "2o"), ("2e", "1e", "3e")])
+def test_tensor_core_fallback_ladder_with_ring_depth(combo, stages):
+    # With a requested ring depth (and the automatic block size that follows it) the kernel
+    # is either the tensor-core kernel with no local memory, or the float32 staged kernel
+    # with no local memory: never a tensor-core kernel that spills.  kernel_info describes the
+    # source that was compiled, and its local bytes are the compiled stack frame.
+    irs = ["0e", "1o", "2e", "3o", "0o", "1e", "2o", "3e"]
+    c = e3.Conv("+".join("128x" + r for r in combo), "1x0e+1x1o+1x2e+1x3o",
+                "+".join("128x" + r for r in irs), 10.0, dtype="f16")
+    c.set_tensor_cores(1)
+    c.set_launch_config(0, 0, stages)
+    info = c.kernel_info()
+    src = c.kernel_source()
+    assert info["local_bytes"] == 0, info
+    assert ("(tensor cores, teams)" in src) == bool(info["tensor_cores"])
+    if info["tensor_cores"]:
+        assert "tcgen05.mma" in src
+    else:
+        assert "(staged ring)" in src and "tcgen05" not in src
