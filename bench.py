@@ -13,8 +13,12 @@ scalars, float32 accumulation and output, outputs l <= 3).  Its inputs
 
 Prints one JSON line (rank 0).  `--impl reference` times the float64 CPU
 oracle on a bounded sample of the same workload instead.
-Multi-GPU (torchrun): every rank runs an independent graph of the same size
-(weak scaling, no collective on the data path); times are the max over ranks.
+Multi-GPU (torchrun): one graph, its receiver rows partitioned into contiguous
+CSR row ranges (one per rank, balanced on edges + rows); each step every rank
+builds its rows' CSR, receives the node features its senders need from the
+other ranks (NCCL all-gather, or a halo all-to-all with --exchange halo) and
+runs e3conv_forward_rows on its rows (strong scaling: the total work is fixed).
+Times are the max over ranks; edges/s counts every rank's edges.
 """
 from __future__ import annotations
 
@@ -58,6 +62,8 @@ def parse_args():
     ap.add_argument("--contract-first", type=int, default=-1)
     ap.add_argument("--tensor-cores", type=int, default=0,
                     help="1: the tensor-core forward variant (float16 inputs, 128 channels)")
+    ap.add_argument("--exchange", choices=["allgather", "halo"], default="allgather",
+                    help="multi-GPU: how a rank receives its senders' node features")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the supplementary timing of the tensor-core variant")
     return ap.parse_args()
@@ -250,16 +256,6 @@ def reduce_over_ranks(times_ms, edges, world, device=None):
     return t.tolist(), e.item()
 
 
-def spec_for_rank(name, rank):
-    from dataclasses import replace
-
-    from workloads import SPECS
-    spec = SPECS[name]
-    if rank:
-        spec = replace(spec, graph_seed=spec.graph_seed + 1000 * rank, seed=spec.seed + 1000 * rank)
-    return spec
-
-
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -268,7 +264,7 @@ def run_reference(args):
 
     import oracle
     from workloads import configs
-    spec = spec_for_rank(args.workload, 0)
+    spec = configs.SPECS[args.workload]
     g = configs.make_graph(spec, args.nodes)
     try:
         import torch
@@ -332,14 +328,9 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
 
-    spec = spec_for_rank(args.workload, rank)
-    g = configs.make_graph(spec, args.nodes)
+    spec = configs.SPECS[args.workload]
+    g = configs.make_graph(spec, args.nodes)     # every rank: the same graph
     N, E = g.num_nodes, g.num_edges
-    x = configs.node_features_torch(spec, N, dev)
-    Y = torch.from_numpy(configs.edge_sh(spec, g)).to(dev)
-    s = configs.scalars_torch(spec, g, dev)
-    senders = torch.from_numpy(g.senders.astype(np.int32)).to(dev)
-    receivers = torch.from_numpy(g.receivers.astype(np.int32)).to(dev)
     conv = e3.Conv(spec.irreps_node, spec.irreps_sh, spec.irreps_out, g.avg_num_neighbors,
                    dtype=spec.dtype)
     if args.channels_per_lane or args.block_threads or args.stages != -1:
@@ -348,21 +339,69 @@ def run_ours(args):
         conv.set_contract_first(args.contract_first)
     if args.tensor_cores:
         conv.set_tensor_cores(1)
-    row_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
-    perm = torch.empty(E, dtype=torch.int32, device=dev)
-    ws = torch.empty(e3.csr_workspace_size(E, N), dtype=torch.uint8, device=dev)
-    out = torch.empty((N, conv.nout, conv.C), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     sh = e3._stream_handle(stream)
-    px, pY, ps, psend, prp, pout = (e3._ptr(t) for t in (x, Y, s, senders, row_ptr, out))
+    shard = None
+    if world == 1:
+        rows, E_loc = N, E
+        x = configs.node_features_torch(spec, N, dev)
+        Y = torch.from_numpy(configs.edge_sh(spec, g)).to(dev)
+        s = configs.scalars_torch(spec, g, dev)
+        senders = torch.from_numpy(g.senders.astype(np.int32)).to(dev)
+        receivers = torch.from_numpy(g.receivers.astype(np.int32)).to(dev)
+        table = x
+    else:
+        # receiver sharding: this rank's CSR row range, its edges, its own node rows; the
+        # sender table is filled by the exchange step every forward
+        from equivariant_graph_message_b200 import sharding
+        rp_host = np.zeros(N + 1, np.int64)
+        np.cumsum(np.bincount(g.receivers, minlength=N), out=rp_host[1:])
+        shard = sharding.shard_graph(rp_host, g.senders, rank, world, args.exchange,
+                                     requests=sharding.torch_requests(device=dev))
+        b0, e0, e1 = shard.row_begin, shard.edge_begin, shard.edge_end
+        rows, E_loc = shard.rows, e1 - e0
+        own = configs.node_features_torch(spec, shard.own_rows, dev, first=b0)
+        if args.exchange == "allgather":
+            x = torch.zeros((shard.block_rows, conv.nx, conv.C), dtype=own.dtype, device=dev)
+            x[:shard.own_rows] = own
+        else:
+            x = own
+            send_idx = torch.from_numpy(shard.send_idx).to(dev)
+            send_buf = torch.empty((len(shard.send_idx), conv.nx, conv.C), dtype=own.dtype,
+                                   device=dev)
+        del own
+        table = torch.empty((shard.table_rows, conv.nx, conv.C), dtype=x.dtype, device=dev)
+        Y = torch.from_numpy(configs.real_sh(g.vec[e0:e1], spec.lmax).astype(
+            configs.np_dtype(spec))).to(dev)
+        s = configs.scalars_torch(spec, g, dev, edges=(e0, e1))
+        senders = torch.from_numpy(shard.senders).to(dev)
+        receivers = torch.from_numpy((g.receivers[e0:e1] - b0).astype(np.int32)).to(dev)
+    row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(max(E_loc, 1), dtype=torch.int32, device=dev)
+    ws = torch.empty(e3.csr_workspace_size(E_loc, rows), dtype=torch.uint8, device=dev)
+    out = torch.empty((rows, conv.nout, conv.C), dtype=torch.float32, device=dev)
+    pY, ps, psend, prp, pout = (e3._ptr(t) for t in (Y, s, senders, row_ptr, out))
+    ptab = e3._ptr(table)
     precv, pperm, pws = e3._ptr(receivers), e3._ptr(perm), e3._ptr(ws)
     ws_bytes = ws.numel()
 
+    def exchange():
+        if args.exchange == "halo":
+            sharding.pack_halo(x, send_idx, out=send_buf)
+            sharding.exchange_rows(shard, send_buf, table)
+        else:
+            sharding.exchange_rows(shard, x, table)
+
     def step(fwd_events=None):
-        e3._ok(e3._build_csr(precv, E, N, prp, pperm, pws, ws_bytes, sh), "e3conv_build_csr")
+        e3._ok(e3._build_csr(precv, E_loc, rows, prp, pperm, pws, ws_bytes, sh), "e3conv_build_csr")
+        if shard is not None:
+            exchange()
         if fwd_events:
             fwd_events[0].record(stream)
-        conv.forward_raw(px, pY, ps, psend, prp, N, pout, sh)
+        if shard is None:
+            conv.forward_raw(ptab, pY, ps, psend, prp, N, pout, sh)
+        else:
+            conv.forward_rows_raw(ptab, shard.table_rows, pY, ps, psend, prp, 0, rows, pout, sh)
         if fwd_events:
             fwd_events[1].record(stream)
 
@@ -390,22 +429,26 @@ def run_ours(args):
     clk = clocks.stop()
     ms = t0.elapsed_time(t1)
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd)
-    (ms, fwd_ms), total_edges = reduce_over_ranks([ms, fwd_ms], E, world, dev)
+    (ms, fwd_ms), total_edges = reduce_over_ranks([ms, fwd_ms], E_loc, world, dev)
     ms_per_step = ms / args.steps
     value = total_edges / (ms_per_step / 1000.0)
 
     pk = peaks()
     in_bytes = 2 if spec.dtype == "f16" else 4
+    # per GPU: the whole graph's algorithmic bytes and FLOPs over the ranks (the partition
+    # balances edges + rows), against the slowest rank's forward time
     nbytes, flops, nnz, mix = algorithmic(conv, N, E, in_bytes)
-    traffic, traffic_src = traffic_for(spec.name if args.nodes is None else None, conv, E)
+    nbytes, flops = nbytes / world, flops / world
+    traffic, traffic_src = traffic_for(spec.name if args.nodes is None and world == 1 else None,
+                                       conv, E)
     sec = fwd_ms / 1000.0
     t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
     if info.get("tensor_cores"):
         # tensor-core variant: the CG x Y contraction runs as two tcgen05 MMAs per edge
         # (M = C, N = path outputs padded to 16, K = 16); only the s-scaling stays on FP32.
         ncols = -(-mix // 16) * 16
-        tc_flops = 2 * 2 * E * conv.C * ncols * 16
-        fp32_flops = 2 * E * conv.C * mix
+        tc_flops = 2 * 2 * E * conv.C * ncols * 16 / world
+        fp32_flops = 2 * E * conv.C * mix / world
         times = {"hbm": t_hbm, "tensor": tc_flops / (pk["f16_tflops"] * 1e12),
                  "alu": fp32_flops / (pk["fp32_tflops"] * 1e12)}
     else:
@@ -444,30 +487,44 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         xf, yf, sf = device_inputs_fns(x, Y, s)
-        rows = calibrated_rows(spec, g, xf, yf, sf, args.cpu_seconds)
-        rate, ne, dt = oracle_sample_rate(spec, g, rows, xf, yf, sf)
+        sample_rows = calibrated_rows(spec, g, xf, yf, sf, args.cpu_seconds)
+        rate, ne, dt = oracle_sample_rate(spec, g, sample_rows, xf, yf, sf)
         cpu = {"value": rate, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
-               "sample": f"{len(rows)} seeded receivers of {N} with all their {ne} edges "
+               "sample": f"{len(sample_rows)} seeded receivers of {N} with all their {ne} edges "
                          f"({dt:.1f} s, float64 loops, OpenMP over receivers)"}
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, conv, spec, g, x, Y, s, senders, receivers, row_ptr, perm, ws, out,
-                      world, dev)
+        def device_step():
+            # the public calls a user makes: CSR build, (exchange,) forward
+            e3.build_csr(receivers, rows, row_ptr=row_ptr, perm=perm[:E_loc], workspace=ws)
+            if shard is None:
+                conv.forward(table, Y, s, senders, row_ptr, out=out)
+            else:
+                exchange()
+                conv.forward_rows(table, Y, s, senders, row_ptr, 0, rows, out=out)
+        e2e = run_e2e(args, [x, Y, s, senders, receivers], out, device_step, E_loc, world, dev)
 
-    launches = args.steps * (e3.csr_kernel_count(E, N) + 1)
+    per_step = e3.csr_kernel_count(E_loc, rows) + 1 + (1 if args.exchange == "halo" and
+                                                       world > 1 else 0)
+    launches = args.steps * per_step
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
+        "scaling": "strong", "vs_baseline": None,
         "dtype": "f16 inputs, f32 accumulation" if spec.dtype == "f16" else "f32",
         "data": "synthetic",
         "config": {"workload": spec.name, "description": spec.description, "nodes": N,
                    "edges": E, "edges_total": int(total_edges), "channels": conv.C,
                    "irreps_node": spec.irreps_node, "irreps_sh": spec.irreps_sh,
                    "irreps_out": spec.irreps_out, "input_dtype": spec.dtype,
-                   "step": "e3conv_build_csr + e3conv_forward",
-                   "l2": f"inputs larger than L2 ({nbytes / 1e9:.1f} GB read per forward)",
+                   "step": ("e3conv_build_csr + e3conv_forward" if world == 1 else
+                            f"e3conv_build_csr (own rows) + node-feature {args.exchange} (NCCL) "
+                            "+ e3conv_forward_rows"),
+                   "parallelism": ("one GPU" if world == 1 else
+                                   f"receiver rows sharded over {world} ranks "
+                                   f"(e3conv_partition_rows), {args.exchange} exchange"),
+                   "l2": f"inputs larger than L2 ({nbytes / 1e9:.1f} GB read per forward per GPU)",
                    "forward_edges_per_s": total_edges / (fwd_ms / 1000.0),
                    "kernel": info},
         "roofline": roof,
@@ -517,13 +574,11 @@ def time_tensor_core_variant(args, spec, g, conv, x, Y, s, senders, row_ptr, out
             "note": "opt-in tcgen05/TMA/tensor-memory forward; not the headline (see roofline)"}
 
 
-def run_e2e(args, conv, spec, g, x, Y, s, senders, receivers, row_ptr, perm, ws, out, world, dev):
-    """Same step through the public API with pinned host inputs and a host result."""
+def run_e2e(args, tensors, out, device_step, edges, world, dev):
+    """The same step through the public API, with this step's inputs copied from pinned host
+    memory and its result copied back, every step, inside the timed region."""
     import torch
     import torch.distributed as dist
-
-    import equivariant_graph_message_b200 as e3
-    tensors = [x, Y, s, senders, receivers]
     h2d = sum(t.numel() * t.element_size() for t in tensors)
     d2h = out.numel() * out.element_size()
     try:
@@ -543,13 +598,11 @@ def run_e2e(args, conv, spec, g, x, Y, s, senders, receivers, row_ptr, perm, ws,
         h.copy_(t)
     out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     steps = max(1, min(args.steps, 5))
-    N, E = g.num_nodes, g.num_edges
 
     def step():
         for h, t in zip(host, tensors):
             t.copy_(h, non_blocking=True)
-        e3.build_csr(receivers, N, row_ptr=row_ptr, perm=perm, workspace=ws)
-        conv.forward(x, Y, s, senders, row_ptr, out=out)
+        device_step()
         out_h.copy_(out, non_blocking=True)
 
     step()
@@ -563,7 +616,7 @@ def run_e2e(args, conv, spec, g, x, Y, s, senders, receivers, row_ptr, perm, ws,
         step()
     b.record()
     torch.cuda.synchronize()
-    (ms,), total = reduce_over_ranks([a.elapsed_time(b) / steps], E, world, dev)
+    (ms,), total = reduce_over_ranks([a.elapsed_time(b) / steps], edges, world, dev)
     del host, out_h
     return {"value": total / (ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms}

@@ -61,6 +61,7 @@ _forward = _sig("e3conv_forward", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i
 _forward_rows = _sig("e3conv_forward_rows", ctypes.c_int, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
                      _i64, _i64, _vp, _vp)
 _check = _sig("e3conv_check", ctypes.c_int, _vp, _vp)
+_partition = _sig("e3conv_partition_rows", ctypes.c_int, _vp, _i64, ctypes.c_int, _vp)
 _csr_ws = _sig("e3conv_csr_workspace_size", ctypes.c_int, _i64, _i64,
                ctypes.POINTER(ctypes.c_size_t))
 _build_csr = _sig("e3conv_build_csr", ctypes.c_int, _vp, _i64, _i64, _vp, _vp, _vp,
@@ -76,7 +77,7 @@ _version = _sig("e3conv_version", ctypes.c_int)
 EXPORTED = ["e3conv_create", "e3conv_destroy", "e3conv_set_input_dtype",
             "e3conv_set_launch_config", "e3conv_set_option", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
             "e3conv_output_irrep", "e3conv_cg", "e3conv_kernel_info", "e3conv_kernel_source",
-            "e3conv_forward", "e3conv_forward_rows", "e3conv_check", "e3conv_csr_workspace_size", "e3conv_build_csr",
+            "e3conv_forward", "e3conv_forward_rows", "e3conv_check", "e3conv_partition_rows", "e3conv_csr_workspace_size", "e3conv_build_csr",
             "e3conv_csr_check", "e3conv_build_csr_noalloc", "e3conv_csr_kernel_count", "e3conv_permute_rows", "e3conv_strerror", "e3conv_last_error",
             "e3conv_version"]
 
@@ -300,6 +301,16 @@ class Conv:
             return False
         _ok(rc, "e3conv_check")
         return True
+
+
+def partition_rows(row_ptr, parts: int) -> np.ndarray:
+    """int64 [parts+1] boundaries of `parts` contiguous receiver-row ranges balanced on
+    edges + rows (e3conv_partition_rows; row_ptr is a host array of num_nodes + 1)."""
+    rp = np.ascontiguousarray(np.asarray(row_ptr), dtype=np.int32)
+    bounds = np.zeros(parts + 1, dtype=np.int64)
+    _ok(_partition(rp.ctypes.data_as(_vp), len(rp) - 1, parts, bounds.ctypes.data_as(_vp)),
+        "e3conv_partition_rows")
+    return bounds
 
 
 def csr_workspace_size(num_edges: int, num_nodes: int) -> int:

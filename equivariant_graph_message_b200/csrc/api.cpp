@@ -591,6 +591,34 @@ int e3conv_forward_rows(e3conv_plan h, const void* x, int64_t num_nodes, const v
   return launch_forward(h, x, num_nodes, Y, s, senders, row_ptr, row_begin, row_end, out, stream);
 }
 
+int e3conv_partition_rows(const int32_t* row_ptr, int64_t num_nodes, int parts, int64_t* bounds) {
+  if (!row_ptr || !bounds) return fail(E3CONV_ERR_INVALID_ARG, "row_ptr and bounds are required");
+  if (parts < 1) return fail(E3CONV_ERR_INVALID_ARG, "parts must be at least 1");
+  if (num_nodes < 0 || num_nodes >= (1ll << 31))
+    return fail(E3CONV_ERR_INVALID_ARG, "num_nodes out of range");
+  if (row_ptr[0] < 0) return fail(E3CONV_ERR_INVALID_ARG, "row_ptr[0] is negative");
+  for (int64_t b = 0; b < num_nodes; ++b)
+    if (row_ptr[b + 1] < row_ptr[b]) return fail(E3CONV_ERR_INVALID_ARG, "row_ptr decreases");
+  // cost of the rows before b: their edges plus one per row (every row stores an output
+  // row); strictly increasing in b.  Boundary r is the row whose prefix cost is nearest to
+  // r/parts of the total (of the first row that reaches it and the one before).
+  auto cost = [&](int64_t b) { return static_cast<int64_t>(row_ptr[b]) - row_ptr[0] + b; };
+  const int64_t total = cost(num_nodes);
+  bounds[0] = 0;
+  for (int r = 1; r < parts; ++r) {
+    const int64_t target = static_cast<int64_t>((static_cast<__int128>(total) * r) / parts);
+    int64_t lo = bounds[r - 1], hi = num_nodes;
+    while (lo < hi) {
+      const int64_t mid = lo + (hi - lo) / 2;
+      if (cost(mid) >= target) hi = mid; else lo = mid + 1;
+    }
+    if (lo > bounds[r - 1] && target - cost(lo - 1) < cost(lo) - target) --lo;
+    bounds[r] = lo;
+  }
+  bounds[parts] = num_nodes;
+  return E3CONV_OK;
+}
+
 int e3conv_check(e3conv_plan h, e3conv_stream stream) {
   if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
   Plan& pl = h->p;

@@ -251,6 +251,20 @@ E3CONV_API int e3conv_forward_rows(e3conv_plan plan, const void* node_features, 
                                    int64_t row_begin, int64_t row_end, float* out,
                                    e3conv_stream stream);
 
+/* Partition of the receiver rows into `parts` contiguous CSR row ranges for
+ * as many ranks (host only; row_ptr is HOST memory here, int32
+ * [num_nodes+1], nondecreasing).  Rank r owns rows bounds[r] .. bounds[r+1]-1
+ * (bounds: int64 [parts+1], bounds[0] = 0, bounds[parts] = num_nodes,
+ * nondecreasing, so every row belongs to exactly one range).  The ranges are
+ * balanced on edges plus one per row: boundary r is the row b whose prefix
+ * cost (row_ptr[b] - row_ptr[0]) + b is nearest to r/parts of the total (of
+ * the first row reaching it and the row before), so every boundary's prefix
+ * cost is within one row's cost (its edges + 1) of its share.
+ * Returns E3CONV_ERR_INVALID_ARG for NULL pointers, parts < 1 or a row_ptr
+ * that decreases. */
+E3CONV_API int e3conv_partition_rows(const int32_t* row_ptr, int64_t num_nodes, int parts,
+                                     int64_t* bounds);
+
 /* Synchronises `stream`, reads and clears the plan's status word.  Returns
  * E3CONV_OK, E3CONV_ERR_BAD_INDEX if a forward since the last check met an
  * out-of-range sender or row range, or E3CONV_ERR_CUDA if a pipeline wait

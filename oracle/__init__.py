@@ -2,8 +2,10 @@
 
 TEST INFRASTRUCTURE ONLY: imported by the tests, the smoke check and the
 benchmark's CPU-baseline / reference arm, never by the product path."""
-from .core import (NORMALIZATIONS, Irrep, Path, Plan, cg, forward, max_threads, parse_irreps,
-                   plan, random_rotation, sh, sh_l, wigner_3j, wigner_d)
+from .core import (NORMALIZATIONS, Irrep, Path, Plan, bessel_cutoff, cg, forward, max_threads,
+                   parse_irreps, plan, radial_mlp, random_rotation, sh, sh_l, silu, wigner_3j,
+                   wigner_d)
 
-__all__ = ["NORMALIZATIONS", "Irrep", "Path", "Plan", "cg", "forward", "max_threads",
-           "parse_irreps", "plan", "random_rotation", "sh", "sh_l", "wigner_3j", "wigner_d"]
+__all__ = ["NORMALIZATIONS", "Irrep", "Path", "Plan", "bessel_cutoff", "cg", "forward",
+           "max_threads", "parse_irreps", "plan", "radial_mlp", "random_rotation", "sh", "sh_l",
+           "silu", "wigner_3j", "wigner_d"]

@@ -247,6 +247,51 @@ def cg(l1: int, l2: int, l3: int, normalization: str = "SQRT_DIM_OUT") -> np.nda
 
 
 # ---------------------------------------------------------------------------
+# Radial scalars s_ab: an MLP of radial-basis encodings of the edge length
+# (e3j.core.Convolution, class docstring: the edge scalars are an MLP of RBF
+# encodings; gate_points_2102 page, "Scope": bessel radial bases and a cosine
+# cutoff; its Network parameters number_of_basis, radial_layers and
+# radial_neurons).  The pages print neither formula; the readings are
+#   B_n(d) = sqrt(2 / r) sin(n pi d / r) / d,   n = 1 .. num_basis
+#   u(d)   = (1 + cos(pi d / r)) / 2 for d < r, 0 otherwise (cosine cutoff)
+#   h_0 = B(d) u(d);  h_{l+1} = SiLU(h_l W_l) for the hidden layers;
+#   s = h_L W_L (no activation on the output layer, no biases),
+# with SiLU(v) = v / (1 + exp(-v)).
+
+
+def bessel_cutoff(d, r_max: float, num_basis: int) -> np.ndarray:
+    """[K, num_basis]: B_n(d) u(d) for edge lengths d [K] (d = 0 takes the limit n pi / r)."""
+    d = np.asarray(d, dtype=np.float64)
+    n = np.arange(1, num_basis + 1, dtype=np.float64)
+    out = np.empty((len(d), num_basis))
+    for q in range(len(d)):
+        if d[q] >= r_max:
+            out[q] = 0.0
+            continue
+        u = 0.5 * (1.0 + np.cos(np.pi * d[q] / r_max))
+        if d[q] == 0.0:
+            out[q] = sqrt(2.0 / r_max) * n * np.pi / r_max * u
+        else:
+            out[q] = sqrt(2.0 / r_max) * np.sin(n * np.pi * d[q] / r_max) / d[q] * u
+    return out
+
+
+def silu(v):
+    v = np.asarray(v, dtype=np.float64)
+    return v / (1.0 + np.exp(-v))
+
+
+def radial_mlp(d, r_max: float, weights) -> np.ndarray:
+    """[K, out] edge scalars from edge lengths d [K]; weights = [W_0 (num_basis x h), ...,
+    W_L (h x out)] in float64 (inputs are upcast exactly)."""
+    ws = [np.asarray(w, dtype=np.float64) for w in weights]
+    h = bessel_cutoff(d, r_max, ws[0].shape[0])
+    for w in ws[:-1]:
+        h = silu(h @ w)
+    return h @ ws[-1]
+
+
+# ---------------------------------------------------------------------------
 # Forward (explicit loops in forward.c)
 
 _lib = None

@@ -153,10 +153,11 @@ def node_features_np(spec: Spec, num_nodes: int, rows: np.ndarray | None = None)
     return rng.normal_np(spec.seed, TID_X, k.astype(np.uint64)).astype(np_dtype(spec))
 
 
-def node_features_torch(spec: Spec, num_nodes: int, device):
-    n = num_nodes * spec.nx * spec.C
-    return rng.normal_torch(spec.seed, TID_X, n, torch_dtype(spec), device).view(
-        num_nodes, spec.nx, spec.C)
+def node_features_torch(spec: Spec, num_nodes: int, device, first: int = 0):
+    """x[first : first + num_nodes] on the device (the whole table by default)."""
+    per = spec.nx * spec.C
+    return rng.normal_torch(spec.seed, TID_X, num_nodes * per, torch_dtype(spec), device,
+                            start=first * per).view(num_nodes, spec.nx, spec.C)
 
 
 # --- radial scalars for the MACE-like layer ---------------------------------
@@ -166,6 +167,16 @@ def _bessel_cutoff(d: np.ndarray, r: float, nb: int = 8) -> np.ndarray:
     n = np.arange(1, nb + 1)
     b = sqrt(2.0 / r) * np.sin(n[None, :] * pi * d[:, None] / r) / d[:, None]
     return b * (0.5 * (np.cos(pi * d / r) + 1.0))[:, None]
+
+
+RADIAL_BASIS = 8      # bessel bases of the MACE-like layer
+RADIAL_HIDDEN = 64    # neurons of each of its two hidden layers
+
+
+def radial_weights(spec: Spec):
+    """The seeded MLP weights [W_0 (8 x 64), W_1 (64 x 64), W_2 (64 x P*C)], float64."""
+    return _mlp_weights(spec, [RADIAL_BASIS, RADIAL_HIDDEN, RADIAL_HIDDEN,
+                               spec.num_paths * spec.C])
 
 
 def _mlp_weights(spec: Spec, sizes):
@@ -189,7 +200,7 @@ def scalars_np(spec: Spec, graph: Graph, edges: np.ndarray | None = None) -> np.
             + np.arange(C)[None, None, :]
         return rng.normal_np(spec.seed, TID_S, k.astype(np.uint64)).astype(np_dtype(spec))
     r = spec.graph["r"]
-    w1, w2, w3 = _mlp_weights(spec, [8, 64, 64, P * C])
+    w1, w2, w3 = radial_weights(spec)
     out = np.empty((len(edges), P, C), dtype=np_dtype(spec))
     for c0 in range(0, len(edges), 1 << 15):
         e = edges[c0:c0 + (1 << 15)]
@@ -200,9 +211,12 @@ def scalars_np(spec: Spec, graph: Graph, edges: np.ndarray | None = None) -> np.
     return out
 
 
-def scalars_torch(spec: Spec, graph: Graph, device):
+def scalars_torch(spec: Spec, graph: Graph, device, edges: tuple | None = None):
+    """s[e0:e1] on the device for edges = (e0, e1) (all edges by default)."""
     import torch
-    E, P, C = graph.num_edges, spec.num_paths, spec.C
+    e0, e1 = edges if edges is not None else (0, graph.num_edges)
+    P, C = spec.num_paths, spec.C
     if spec.scalars == "normal":
-        return rng.normal_torch(spec.seed, TID_S, E * P * C, torch_dtype(spec), device).view(E, P, C)
-    return torch.from_numpy(scalars_np(spec, graph)).to(device)
+        return rng.normal_torch(spec.seed, TID_S, (e1 - e0) * P * C, torch_dtype(spec), device,
+                                start=e0 * P * C).view(e1 - e0, P, C)
+    return torch.from_numpy(scalars_np(spec, graph, np.arange(e0, e1))).to(device)
