@@ -60,6 +60,10 @@ def parse_args():
     ap.add_argument("--block-threads", type=int, default=0)
     ap.add_argument("--stages", type=int, default=-1)
     ap.add_argument("--contract-first", type=int, default=-1)
+    ap.add_argument("--path-split", type=int, default=-1,
+                    help="warps that split a receiver row's paths (E3CONV_OPT_PATH_SPLIT)")
+    ap.add_argument("--edge-vectors", type=int, default=0,
+                    help="1: edge vectors as input, harmonics evaluated in the kernel")
     ap.add_argument("--tensor-cores", type=int, default=0,
                     help="1: the tensor-core forward variant (float16 inputs, 128 channels)")
     ap.add_argument("--exchange", choices=["allgather", "halo"], default="allgather",
@@ -91,14 +95,16 @@ def peaks():
 def algorithmic(conv, N, E, in_bytes):
     """Algorithmic bytes and FLOPs of one forward.
 
-    bytes = E (ny + P C) b + 4E (senders) + N (nx C b + 4 nout C + 4 (row_ptr)):
-            every edge's Y and s once, every node's features once, every output once.
+    bytes = E (ny b + P C b) + 4E (senders) + N (nx C b + 4 nout C + 4 (row_ptr)):
+            every edge's Y and s once, every node's features once, every output once
+            (with edge vectors as input, 16 bytes per edge replace the ny b of Y).
     flops = 2 E C (sum of CG nonzeros over paths + sum over paths of (2 l3 + 1)).
     """
     import numpy as np
     nnz = sum(int((np.abs(conv.cg(p)) > 1e-12).sum()) for p in range(conv.num_paths))
     mix = sum(2 * q.l3 + 1 for q in conv.paths)
-    nbytes = E * (conv.ny + conv.num_paths * conv.C) * in_bytes + 4 * E + \
+    y_bytes = 16 if conv.edge_vectors else conv.ny * in_bytes   # vectors: float32 [E][4]
+    nbytes = E * (y_bytes + conv.num_paths * conv.C * in_bytes) + 4 * E + \
         N * (conv.nx * conv.C * in_bytes + 4 * conv.nout * conv.C + 4)
     flops = 2 * E * conv.C * (nnz + mix)
     return nbytes, flops, nnz, mix
@@ -310,6 +316,17 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def edge_input(configs, spec, g, e0, e1, vectors):
+    """The forward's per-edge geometry for edges e0..e1-1: the harmonics [E][ny] in the
+    workload dtype, or the edge vectors as float32 [E][4] (x, y, z, 0)."""
+    import numpy as np
+    if vectors:
+        v = np.zeros((e1 - e0, 4), np.float32)
+        v[:, :3] = g.vec[e0:e1]
+        return v
+    return configs.real_sh(g.vec[e0:e1], spec.lmax).astype(configs.np_dtype(spec))
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -339,13 +356,17 @@ def run_ours(args):
         conv.set_contract_first(args.contract_first)
     if args.tensor_cores:
         conv.set_tensor_cores(1)
+    if args.path_split != -1:
+        conv.set_path_split(args.path_split)
+    if args.edge_vectors:
+        conv.set_edge_vectors(1)
     stream = torch.cuda.current_stream()
     sh = e3._stream_handle(stream)
     shard = None
     if world == 1:
         rows, E_loc = N, E
         x = configs.node_features_torch(spec, N, dev)
-        Y = torch.from_numpy(configs.edge_sh(spec, g)).to(dev)
+        Y = torch.from_numpy(edge_input(configs, spec, g, 0, E, args.edge_vectors)).to(dev)
         s = configs.scalars_torch(spec, g, dev)
         senders = torch.from_numpy(g.senders.astype(np.int32)).to(dev)
         receivers = torch.from_numpy(g.receivers.astype(np.int32)).to(dev)
@@ -371,8 +392,7 @@ def run_ours(args):
                                    device=dev)
         del own
         table = torch.empty((shard.table_rows, conv.nx, conv.C), dtype=x.dtype, device=dev)
-        Y = torch.from_numpy(configs.real_sh(g.vec[e0:e1], spec.lmax).astype(
-            configs.np_dtype(spec))).to(dev)
+        Y = torch.from_numpy(edge_input(configs, spec, g, e0, e1, args.edge_vectors)).to(dev)
         s = configs.scalars_torch(spec, g, dev, edges=(e0, e1))
         senders = torch.from_numpy(shard.senders).to(dev)
         receivers = torch.from_numpy((g.receivers[e0:e1] - b0).astype(np.int32)).to(dev)

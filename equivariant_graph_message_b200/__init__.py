@@ -55,6 +55,11 @@ _kernel_info = _sig("e3conv_kernel_info", ctypes.c_int, _vp, ctypes.c_int, *([_c
 _set_option = _sig("e3conv_set_option", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_int)
 OPT_CONTRACT_FIRST = 1
 OPT_TENSOR_CORES = 2
+OPT_PATH_SPLIT = 3
+OPT_EDGE_VECTORS = 4
+_get_option = _sig("e3conv_get_option", ctypes.c_int, _vp, ctypes.c_int, _c_int_p)
+_sh_host = _sig("e3conv_spherical_harmonics", ctypes.c_int, _vp, ctypes.POINTER(ctypes.c_double),
+                ctypes.POINTER(ctypes.c_double))
 _kernel_source = _sig("e3conv_kernel_source", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_char_p,
                       ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t))
 _forward = _sig("e3conv_forward", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp)
@@ -75,7 +80,8 @@ _last_error = _sig("e3conv_last_error", ctypes.c_char_p)
 _version = _sig("e3conv_version", ctypes.c_int)
 
 EXPORTED = ["e3conv_create", "e3conv_destroy", "e3conv_set_input_dtype",
-            "e3conv_set_launch_config", "e3conv_set_option", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
+            "e3conv_set_launch_config", "e3conv_set_option", "e3conv_get_option",
+            "e3conv_spherical_harmonics", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
             "e3conv_output_irrep", "e3conv_cg", "e3conv_kernel_info", "e3conv_kernel_source",
             "e3conv_forward", "e3conv_forward_rows", "e3conv_check", "e3conv_partition_rows", "e3conv_csr_workspace_size", "e3conv_build_csr",
             "e3conv_csr_check", "e3conv_build_csr_noalloc", "e3conv_csr_kernel_count", "e3conv_permute_rows", "e3conv_strerror", "e3conv_last_error",
@@ -205,6 +211,28 @@ class Conv:
     def set_tensor_cores(self, value: int = -1):
         _ok(_set_option(self._h, OPT_TENSOR_CORES, value), "e3conv_set_option")
 
+    def set_path_split(self, value: int = -1):
+        _ok(_set_option(self._h, OPT_PATH_SPLIT, value), "e3conv_set_option")
+
+    def set_edge_vectors(self, value: int = 1):
+        """1: the forward's Y argument holds edge vectors float32 [E][4]; harmonics in-kernel."""
+        _ok(_set_option(self._h, OPT_EDGE_VECTORS, value), "e3conv_set_option")
+
+    @property
+    def edge_vectors(self) -> bool:
+        v = ctypes.c_int()
+        _ok(_get_option(self._h, OPT_EDGE_VECTORS, ctypes.byref(v)), "e3conv_get_option")
+        return v.value == 1
+
+    def spherical_harmonics(self, vec) -> np.ndarray:
+        """The plan's harmonics of vec / |vec| (host evaluation of the kernel's polynomials)."""
+        v = np.ascontiguousarray(np.asarray(vec, dtype=np.float64).reshape(3))
+        out = np.zeros(self.ny)
+        _ok(_sh_host(self._h, v.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
+                     out.ctypes.data_as(ctypes.POINTER(ctypes.c_double))),
+            "e3conv_spherical_harmonics")
+        return out
+
     def kernel_info(self, dtype: str | None = None) -> dict:
         v = [ctypes.c_int() for _ in range(8)]
         _ok(_kernel_info(self._h, {"f32": F32, "f16": F16}[dtype or self.dtype],
@@ -222,28 +250,36 @@ class Conv:
         return buf.value.decode()
 
     # ---- device calls
-    def forward(self, x, Y, s, senders, row_ptr, out=None, stream=None):
-        """out[N][nout][C] float32 from receiver-sorted edges (torch CUDA tensors)."""
+    def _check_inputs(self, x, Y, s, senders, row_ptr):
         import torch
         N = x.shape[0]
         E = senders.shape[0]
         want = torch.float16 if self.dtype == "f16" else torch.float32
         _require("x", x, dtype=want)
         dev = x.device
-        for name, t in (("Y", Y), ("s", s)):
-            _require(name, t, dev, want)
+        vec = self.edge_vectors
+        _require("Y", Y, dev, torch.float32 if vec else want)
+        _require("s", s, dev, want)
         _require("senders", senders, dev, torch.int32)
         _require("row_ptr", row_ptr, dev, torch.int32)
         if tuple(x.shape) != (N, self.nx, self.C):
             raise ValueError(f"x shape {tuple(x.shape)} != {(N, self.nx, self.C)}")
-        if tuple(Y.shape) != (E, self.ny) or tuple(s.shape) != (E, self.num_paths, self.C):
-            raise ValueError("Y / s shapes do not match the plan")
-        if senders.dtype != torch.int32 or row_ptr.dtype != torch.int32:
-            raise ValueError("senders and row_ptr must be int32")
+        if tuple(Y.shape) != ((E, 4) if vec else (E, self.ny)):
+            raise ValueError("Y shape does not match the plan (edge vectors: [E][4])")
+        if tuple(s.shape) != (E, self.num_paths, self.C):
+            raise ValueError("s shape does not match the plan")
+
+    def forward(self, x, Y, s, senders, row_ptr, out=None, stream=None):
+        """out[N][nout][C] float32 from receiver-sorted edges (torch CUDA tensors)."""
+        import torch
+        N = x.shape[0]
+        E = senders.shape[0]
+        dev = x.device
+        self._check_inputs(x, Y, s, senders, row_ptr)
         if row_ptr.shape[0] != N + 1:
             raise ValueError("row_ptr must have num_nodes + 1 entries")
         if out is None:
-            out = torch.empty((N, self.nout, self.C), dtype=torch.float32, device=x.device)
+            out = torch.empty((N, self.nout, self.C), dtype=torch.float32, device=dev)
         else:
             _require("out", out, dev, torch.float32, N * self.nout * self.C)
         _ok(_forward(self._h, _ptr(x), _ptr(Y) if E else None, _ptr(s) if E else None,
@@ -259,17 +295,8 @@ class Conv:
         import torch
         N = x.shape[0]
         E = senders.shape[0]
-        want = torch.float16 if self.dtype == "f16" else torch.float32
-        _require("x", x, dtype=want)
         dev = x.device
-        for name, t in (("Y", Y), ("s", s)):
-            _require(name, t, dev, want)
-        _require("senders", senders, dev, torch.int32)
-        _require("row_ptr", row_ptr, dev, torch.int32)
-        if tuple(x.shape) != (N, self.nx, self.C):
-            raise ValueError(f"x shape {tuple(x.shape)} != {(N, self.nx, self.C)}")
-        if tuple(Y.shape) != (E, self.ny) or tuple(s.shape) != (E, self.num_paths, self.C):
-            raise ValueError("Y / s shapes do not match the plan")
+        self._check_inputs(x, Y, s, senders, row_ptr)
         if not 0 <= row_begin <= row_end < row_ptr.shape[0]:
             raise ValueError("rows must satisfy 0 <= row_begin <= row_end < len(row_ptr)")
         rows = row_end - row_begin

@@ -404,18 +404,59 @@ int e3conv_set_launch_config(e3conv_plan h, int channels_per_lane, int block_thr
 int e3conv_set_option(e3conv_plan h, int option, int value) {
   if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
   Plan& pl = h->p;
-  if (option != E3CONV_OPT_CONTRACT_FIRST && option != E3CONV_OPT_TENSOR_CORES)
+  if (option != E3CONV_OPT_CONTRACT_FIRST && option != E3CONV_OPT_TENSOR_CORES &&
+      option != E3CONV_OPT_PATH_SPLIT && option != E3CONV_OPT_EDGE_VECTORS)
     return fail(E3CONV_ERR_UNSUPPORTED, "unknown option");
-  if (value < -1 || value > 1) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1, 0 or 1");
-  if (option == E3CONV_OPT_CONTRACT_FIRST)
-    pl.req_coop = value;
-  else
-    pl.req_tc = value;
+  if (option == E3CONV_OPT_EDGE_VECTORS) {
+    if (value != 0 && value != 1) return fail(E3CONV_ERR_INVALID_ARG, "value must be 0 or 1");
+    pl.req_vec = value;
+  } else if (option == E3CONV_OPT_PATH_SPLIT) {
+    if (value < -1 || value > 8) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1 .. 8");
+    pl.req_psplit = value;
+  } else {
+    if (value < -1 || value > 1) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1, 0 or 1");
+    if (option == E3CONV_OPT_CONTRACT_FIRST)
+      pl.req_coop = value;
+    else
+      pl.req_tc = value;
+  }
   DeviceGuard g(pl.device);
   const int other = pl.dtype == E3CONV_F32 ? E3CONV_F16 : E3CONV_F32;
   release_variant(pl.var[other]);
   release_variant(pl.var[pl.dtype]);
   return compile_variant(pl, pl.dtype);
+}
+
+int e3conv_get_option(e3conv_plan h, int option, int* value) {
+  if (!h || !value) return fail(E3CONV_ERR_INVALID_ARG, "NULL argument");
+  const Plan& pl = h->p;
+  switch (option) {
+    case E3CONV_OPT_CONTRACT_FIRST: *value = pl.req_coop; return E3CONV_OK;
+    case E3CONV_OPT_TENSOR_CORES: *value = pl.req_tc; return E3CONV_OK;
+    case E3CONV_OPT_PATH_SPLIT: *value = pl.req_psplit; return E3CONV_OK;
+    case E3CONV_OPT_EDGE_VECTORS: *value = pl.req_vec; return E3CONV_OK;
+    default: return fail(E3CONV_ERR_UNSUPPORTED, "unknown option");
+  }
+}
+
+int e3conv_spherical_harmonics(e3conv_plan h, const double* vec, double* out) {
+  if (!h || !vec || !out) return fail(E3CONV_ERR_INVALID_ARG, "NULL argument");
+  const Plan& pl = h->p;
+  const double r2 = vec[0] * vec[0] + vec[1] * vec[1] + vec[2] * vec[2];
+  if (!(r2 > 0.0)) {
+    for (int j = 0; j < pl.ny; ++j) out[j] = j == 0 ? 1.0 : 0.0;
+    return E3CONV_OK;
+  }
+  const double inv = 1.0 / std::sqrt(r2);
+  const double u[3] = {vec[0] * inv, vec[1] * inv, vec[2] * inv};
+  const auto polys = sh_polynomials(pl.lmax);
+  for (int j = 0; j < pl.ny; ++j) {
+    double v = 0.0;
+    for (const auto& m : polys[j])
+      v += m.coef * std::pow(u[0], m.px) * std::pow(u[1], m.py) * std::pow(u[2], m.pz);
+    out[j] = v;
+  }
+  return E3CONV_OK;
 }
 
 int e3conv_query(e3conv_plan h, int* C, int* nx, int* ny, int* nout, int* num_paths) {

@@ -45,6 +45,21 @@ int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
 }  // namespace
 
+// A group of lanes forming and applying the per-edge A entries of some paths
+// (the staged variant's contract-first form): a whole team, or one warp of a
+// team whose row's paths are split over its warps.
+struct CoopGroupInfo {
+  std::vector<int> paths;       // paths computed, canonical order
+  std::vector<AEntry> ent;      // their A entries, build order within each path
+  std::vector<int> acc;         // output component -> accumulator index (-1: not computed)
+  int nacc = 0;                 // accumulators (output components) of the group
+  bool pairs = false;           // A stored as (a, a) pairs in phase-2 order
+  int a_bytes = 0;              // shared memory of the group's A entries
+};
+
+std::vector<std::vector<int>> path_split_outputs(const Plan& pl, int warps);
+std::vector<CoopGroupInfo> coop_groups(const Plan& pl, const Shape& sh);
+
 std::vector<AEntry> build_a_entries(const Plan& pl) {
   std::vector<AEntry> out;
   for (size_t p = 0; p < pl.paths.size(); ++p) {
@@ -75,7 +90,8 @@ Shape choose_shape(const Plan& pl, int dtype) {
   const int vmax = 16 / elem;
   s.s_bytes = static_cast<int>(pl.paths.size()) * pl.C * elem;
   s.x_bytes = pl.nx * pl.C * elem;
-  s.y_bytes = pl.ny * elem;
+  s.y_bytes = pl.req_vec ? 16 : pl.ny * elem;
+  s.vec = pl.req_vec != 0;
   const bool bytes_ok = s.s_bytes % 16 == 0 && s.x_bytes % 16 == 0 && s.y_bytes % 16 == 0;
 
   // Tensor-core variant: float16 inputs, 128 channels (the MMA's M), at most
@@ -127,16 +143,23 @@ Shape choose_shape(const Plan& pl, int dtype) {
       s = Shape{};
       s.s_bytes = static_cast<int>(pl.paths.size()) * pl.C * elem;
       s.x_bytes = pl.nx * pl.C * elem;
-      s.y_bytes = pl.ny * elem;
+      s.y_bytes = pl.req_vec ? 16 : pl.ny * elem;
+      s.vec = pl.req_vec != 0;
     }
   }
 
   // Staged variant: a team of `team` warps covers the C channels of one
   // receiver row, V channels per lane.  Preferred: one channel pair per lane
   // (V = 2, team = C / 64), which keeps registers low and warps many.
-  int V = 0, team = 0;
+  int V = 0, team = 0, psplit = 1;
+  const int one_warp_V = pl.C / 32;  // channels per lane when one warp covers C
   if (pl.req_stages != 0 && bytes_ok && pl.C % 32 == 0) {
-    if (pl.req_V > 0) {
+    if (pl.req_psplit >= 2 && pl.req_coop != 0 && pl.req_V <= 0 && one_warp_V <= vmax &&
+        (one_warp_V == 1 || one_warp_V % 2 == 0) &&
+        pl.req_psplit <= static_cast<int>(pl.outputs.size())) {
+      V = one_warp_V;  // every warp of the team covers C; the row's paths are split over them
+      team = psplit = pl.req_psplit;
+    } else if (pl.req_V > 0) {
       if (pl.C % (32 * pl.req_V) == 0 && pl.req_V <= vmax) {
         V = pl.req_V;
         team = pl.C / (32 * V);
@@ -164,10 +187,13 @@ Shape choose_shape(const Plan& pl, int dtype) {
     s.y_off = s.x_off + align_up(s.x_bytes, 128);
     s.stage_bytes = s.y_off + align_up(s.y_bytes, 128);
     s.coop = pl.req_coop != 0 && (V == 1 || V % 2 == 0);
-    s.dup_a = s.coop && V == 2;
+    s.psplit = s.coop ? psplit : 1;
+    s.dup_a = s.coop && V % 2 == 0;
     s.na = s.coop ? static_cast<int>(build_a_entries(pl).size()) : 0;
-    const int a_bytes = s.coop ? align_up((s.dup_a ? 8 : 4) * s.na, 16) : 0;
-    const int y_bytes = s.coop ? align_up(4 * pl.ny, 16) : 0;
+    int a_bytes = 0;
+    if (s.coop)
+      for (const auto& g : coop_groups(pl, s)) a_bytes += g.a_bytes;
+    const int y_bytes = s.coop ? s.psplit * align_up(4 * pl.ny, 16) : 0;
     const int S = pl.req_stages > 0 ? pl.req_stages : 2;
     s.stages = S;
     s.a_off = S * s.stage_bytes;
@@ -193,7 +219,8 @@ Shape choose_shape(const Plan& pl, int dtype) {
     s = Shape{};
     s.s_bytes = static_cast<int>(pl.paths.size()) * pl.C * elem;
     s.x_bytes = pl.nx * pl.C * elem;
-    s.y_bytes = pl.ny * elem;
+    s.y_bytes = pl.req_vec ? 16 : pl.ny * elem;
+    s.vec = pl.req_vec != 0;
   }
 
   // Direct variant.
@@ -327,6 +354,95 @@ void emit_y_load(Emitter& em, const Plan& pl, int dtype, const std::string& pre,
     for (int j = 0; j < pl.ny; ++j)
       em.line("y" + S(j) + " = " + pre + (f16 ? "_h1" : "_f1") + "(" + yr + " + " + S(j) + ");");
   }
+}
+
+// Declares y0..y{ny-1} = the real harmonics of the unit vector of (vx, vy, vz)
+// (a zero vector gives Y_0 = 1 and 0 for l > 0), from the plan's polynomials.
+void emit_sh_eval(Emitter& em, const Plan& pl, const std::string& vx, const std::string& vy,
+                  const std::string& vz) {
+  const auto polys = sh_polynomials(pl.lmax);
+  std::string decl = "float";
+  for (int j = 0; j < pl.ny; ++j) decl += std::string(j ? "," : "") + " y" + S(j);
+  em.line(decl + ";");
+  em.line("{");
+  em.ind++;
+  em.line("const float r2_ = fmaf(" + vx + ", " + vx + ", fmaf(" + vy + ", " + vy + ", " + vz +
+          " * " + vz + "));");
+  em.line("const float inv_ = r2_ > 0.f ? 1.f / sqrtf(r2_) : 0.f;");
+  em.line("const float ux_ = " + vx + " * inv_, uy_ = " + vy + " * inv_, uz_ = " + vz + " * inv_;");
+  const char* base[3] = {"ux_", "uy_", "uz_"};
+  const char* nm[3] = {"px", "py", "pz"};
+  for (int d = 0; d < 3; ++d)
+    for (int a = 1; a <= pl.lmax; ++a)
+      em.line(std::string("const float ") + nm[d] + S(a) + "_ = " +
+              (a == 1 ? std::string(base[d]) : std::string(nm[d]) + S(a - 1) + "_ * " + base[d]) + ";");
+  std::map<std::tuple<int, int, int>, std::string> mono;
+  auto monomial = [&](int a, int b, int c) -> std::string {
+    auto key = std::make_tuple(a, b, c);
+    auto it = mono.find(key);
+    if (it != mono.end()) return it->second;
+    std::vector<std::string> f;
+    if (a) f.push_back("px" + S(a) + "_");
+    if (b) f.push_back("py" + S(b) + "_");
+    if (c) f.push_back("pz" + S(c) + "_");
+    std::string name;
+    if (f.size() == 1) {
+      name = f[0];
+    } else {
+      name = "m" + S(a) + S(b) + S(c) + "_";
+      std::string e = f[0];
+      for (size_t k = 1; k < f.size(); ++k) e += " * " + f[k];
+      em.line("const float " + name + " = " + e + ";");
+    }
+    mono[key] = name;
+    return name;
+  };
+  for (int j = 0; j < pl.ny; ++j) {
+    std::string expr;
+    double constant = 0.0;
+    for (const auto& m : polys[j]) {
+      if (m.px + m.py + m.pz == 0) {
+        constant += m.coef;
+        continue;
+      }
+      const std::string mm = monomial(m.px, m.py, m.pz);
+      expr = expr.empty() ? flt(m.coef) + " * " + mm : "fmaf(" + flt(m.coef) + ", " + mm + ", " + expr + ")";
+    }
+    if (constant != 0.0) expr = expr.empty() ? flt(constant) : expr + " + " + flt(constant);
+    if (expr.empty()) expr = "0.f";
+    em.line("y" + S(j) + " = " + expr + ";");
+  }
+  std::string zero = "y0 = 1.f;";
+  for (int j = 1; j < pl.ny; ++j) zero += " y" + S(j) + " = 0.f;";
+  em.line("if (!(r2_ > 0.f)) { " + zero + " }");
+  em.ind--;
+  em.line("}");
+}
+
+// Fills the float32 Y row `yf` (shared memory) of the edge staged at `ysrc`
+// with `nl` lanes (index `ln`): each converts components ln, ln + nl, ... of the
+// staged harmonics, or, from edge vectors, every lane evaluates the harmonics
+// and stores those components.
+void emit_yf_fill(Emitter& em, const Plan& pl, int dtype, const Shape& sh, const std::string& ysrc,
+                  const std::string& ln, int nl, const std::string& yf) {
+  if (!sh.vec) {
+    const bool f16 = dtype == E3CONV_F16;
+    const std::string Ty = f16 ? "unsigned short" : "float";
+    em.line("for (int j_ = " + ln + "; j_ < " + S(pl.ny) + "; j_ += " + S(nl) + ") " + yf +
+            "[j_] = " + (f16 ? "h2f" : "") + "(reinterpret_cast<const " + Ty + "*>(" + ysrc +
+            ")[j_]);");
+    return;
+  }
+  em.line("{");
+  em.ind++;
+  em.line("const float4 v_ = *reinterpret_cast<const float4*>(" + ysrc + ");");
+  emit_sh_eval(em, pl, "v_.x", "v_.y", "v_.z");
+  std::string sel = "y" + S(pl.ny - 1);
+  for (int j = pl.ny - 2; j >= 0; --j) sel = "(j_ == " + S(j) + " ? y" + S(j) + " : " + sel + ")";
+  em.line("for (int j_ = " + ln + "; j_ < " + S(pl.ny) + "; j_ += " + S(nl) + ") " + yf + "[j_] = " +
+          sel + ";");
+  em.ind--;
+  em.line("}");
 }
 
 // The per-edge contribution: x slices at xr + comp*C, s slices at sr + p*C
@@ -473,11 +589,11 @@ void emit_flush(Emitter& em, const Plan& pl, int V, const std::string& orow,
   em.line("}");
 }
 
-void emit_signature(Emitter& em, const std::string& T, int block, int minb) {
+void emit_signature(Emitter& em, const std::string& T, int block, int minb, bool vec) {
   em.line("extern \"C\" __global__ void __launch_bounds__(" + S(block) +
           (minb > 0 ? ", " + S(minb) : std::string()) + ") e3conv_fwd(");
-  em.line("    const " + T + "* __restrict__ x, const " + T + "* __restrict__ Y, const " + T +
-          "* __restrict__ s,");
+  em.line("    const " + T + "* __restrict__ x, const " + (vec ? std::string("float") : T) +
+          "* __restrict__ Y, const " + T + "* __restrict__ s,");
   em.line("    const int* __restrict__ senders, const int* __restrict__ row_ptr,");
   em.line("    int num_nodes, int row_begin, int row_end, float* __restrict__ out, float inv_avg,");
   em.line("    unsigned int* __restrict__ status)");
@@ -505,7 +621,7 @@ std::string direct_source(const Plan& pl, int dtype, const Shape& sh) {
           " TL=" + S(sh.TL) + " tiles=" + S(sh.tiles) + " ipw=" + S(sh.ipw));
   emit_prelude(em);
   emit_chunk_define(em);
-  emit_signature(em, T, sh.block, 0);
+  emit_signature(em, T, sh.block, 0, sh.vec);
   em.line("{");
   em.ind++;
   em.line("const int lane = threadIdx.x & 31;");
@@ -536,8 +652,13 @@ std::string direct_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("const long long le = e - e_base;  // local edge index");
   em.line("const int a = senders[le];");
   em.line("if ((unsigned int)a >= (unsigned int)num_nodes) { atomicOr(status, 2u); continue; }");
-  em.line("const " + T + "* yr = Y + le * " + S(pl.ny) + ";");
-  emit_y_load(em, pl, dtype, "ldg", "yr");
+  if (sh.vec) {
+    em.line("const float4 v_ = __ldg(reinterpret_cast<const float4*>(Y) + le);");
+    emit_sh_eval(em, pl, "v_.x", "v_.y", "v_.z");
+  } else {
+    em.line("const " + T + "* yr = Y + le * " + S(pl.ny) + ";");
+    emit_y_load(em, pl, dtype, "ldg", "yr");
+  }
   em.line("const " + T + "* xr = x + (long long)a * " + S(pl.nx * pl.C) + " + u0;");
   em.line("const " + T + "* sr = s + le * " +
           S(static_cast<long long>(pl.paths.size()) * pl.C) + " + u0;");
@@ -610,18 +731,37 @@ void emit_group_load(Emitter& em, int dtype, const Lanes& L, const std::string& 
   }
 }
 
+// One group of lanes that forms the A entries of some paths and applies them:
+// the whole team (channel split: the team's lanes share one A area) or one warp
+// of the team (path split: each warp owns a set of output irreps, the paths
+// into them and their A entries).
+struct CoopGroup {
+  std::vector<int> paths;       // paths computed, canonical order
+  std::vector<AEntry> ent;      // their A entries, build order within each path
+  int RW = 32;                  // lanes forming the entries
+  std::string lane;             // lane index among them ("tl" or "lane")
+  std::string sfx;              // suffix of the generated table
+  std::vector<int> acc;         // output component -> accumulator index (-1: not computed)
+  int a_off = 0, yf_off = 0;    // the group's A entries and float32 Y (bytes from tbase)
+  bool pairs = false;           // A stored as (a, a) pairs in phase-2 order, read two per load
+};
+
 struct CoopTables {
   std::string source;      // __device__ table of phase 1
   int rounds = 0;
   std::vector<int> terms;  // terms per round
-  std::vector<int> slot;   // entry -> position in the warp's A area
+  std::vector<int> slot;   // entry -> position in the group's A area
 };
 
-// Phase 1 deals the entries to the team's RW = 32 * team lanes in rounds,
-// longest first, and stores entry number q of that order at A[q]: every
-// round writes RW consecutive slots (no bank conflicts) and phase 2 reads A
-// at the compile-time position slot[n] of entry n.
-CoopTables coop_tables(const std::vector<AEntry>& ent, int RW) {
+// Phase 1 deals the entries to the group's RW lanes in rounds, longest first.
+// Without pairs, entry number q of that order goes to A[q] (every round writes
+// RW consecutive slots: no bank conflicts) and phase 2 reads A at slot[n].
+// With pairs, the slots follow phase 2's order (path by path, each path padded
+// to an even count) so that phase 2 loads two entries per 16-byte load; the
+// slot of each dealt entry travels in the high bits of its first term's index.
+CoopTables coop_tables(const CoopGroup& G) {
+  const std::vector<AEntry>& ent = G.ent;
+  const int RW = G.RW;
   CoopTables T;
   std::vector<int> order(ent.size());
   for (size_t n = 0; n < ent.size(); ++n) order[n] = static_cast<int>(n);
@@ -629,13 +769,23 @@ CoopTables coop_tables(const std::vector<AEntry>& ent, int RW) {
     return ent[a].terms.size() > ent[b].terms.size();
   });
   T.slot.assign(ent.size(), -1);
-  for (size_t q = 0; q < order.size(); ++q) T.slot[order[q]] = static_cast<int>(q);
+  if (G.pairs) {
+    int pos = 0;
+    for (int p : G.paths) {
+      for (size_t n = 0; n < ent.size(); ++n)
+        if (ent[n].path == p) T.slot[n] = pos++;
+      pos += pos & 1;
+    }
+  } else {
+    for (size_t q = 0; q < order.size(); ++q) T.slot[order[q]] = static_cast<int>(q);
+  }
   T.rounds = static_cast<int>((ent.size() + RW - 1) / RW);
   std::ostringstream c, lay;
-  c << "__device__ const int2 e3_atab[] = {\n";
-  lay << "// A layout (slot: path i k):";
+  c << "__device__ const int2 e3_atab" << G.sfx << "[] = {\n";
+  lay << "// A layout" << G.sfx << " (entry: path i k slot):";
   for (size_t q = 0; q < order.size(); ++q)
-    lay << " " << ent[order[q]].path << ":" << ent[order[q]].i << ":" << ent[order[q]].k;
+    lay << " " << ent[order[q]].path << ":" << ent[order[q]].i << ":" << ent[order[q]].k << ":"
+        << T.slot[order[q]];
   lay << "\n";
   for (int r = 0; r < T.rounds; ++r) {
     int tr = 0;
@@ -653,6 +803,7 @@ CoopTables coop_tables(const std::vector<AEntry>& ent, int RW) {
           j = ent[order[q]].terms[t].first;
           cv = ent[order[q]].terms[t].second;
         }
+        if (G.pairs && t == 0 && q < order.size()) j |= T.slot[order[q]] << 8;
         const float cf = static_cast<float>(cv);
         unsigned int bits;
         std::memcpy(&bits, &cf, sizeof bits);
@@ -662,69 +813,78 @@ CoopTables coop_tables(const std::vector<AEntry>& ent, int RW) {
     }
   }
   c << "};\n";
+  lay << "// A rounds" << G.sfx << " (lanes " << RW << ", pairs " << (G.pairs ? 1 : 0) << "):";
+  for (int tr : T.terms) lay << " " << tr;
+  lay << "\n";
   T.source = lay.str() + c.str();
   return T;
 }
 
-// Phase 1 + phase 2 for the edge staged at `stg`.  `tl` is the lane's index
-// in its team, `team_sync()` a barrier of the team's warps.
-void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
-                    const std::vector<AEntry>& ent, const CoopTables& T) {
+// Phase 1 + phase 2 of one group for the edge staged at `stg` (Y already in
+// float32 at the group's yf, made visible to the group by the caller).
+void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh, const CoopGroup& G,
+                    const CoopTables& T, const std::string& group_sync) {
   const bool f16 = dtype == E3CONV_F16;
   const std::string Ty = f16 ? "unsigned short" : "float";
   const Lanes L{sh.V};
-  const int RW = 32 * sh.team;
-  if (sh.dup_a)
-    em.line("unsigned long long* Aw = reinterpret_cast<unsigned long long*>(tbase + " + S(sh.a_off) + ");");
+  const int RW = G.RW;
+  const std::string& ln = G.lane;
+  if (G.pairs)
+    em.line("unsigned long long* Aw = reinterpret_cast<unsigned long long*>(tbase + " + S(G.a_off) + ");");
   else
-    em.line("float* Aw = reinterpret_cast<float*>(tbase + " + S(sh.a_off) + ");");
-  em.line("float* yf = reinterpret_cast<float*>(tbase + " + S(sh.yf_off) + ");");
-  em.line("if (tl < " + S(pl.ny) + ") yf[tl] = " + (f16 ? "h2f" : "") + "(reinterpret_cast<const " +
-          Ty + "*>(stg + " + S(sh.y_off) + ")[tl]);");
-  em.line("team_sync();");
+    em.line("float* Aw = reinterpret_cast<float*>(tbase + " + S(G.a_off) + ");");
+  em.line("const float* yf = reinterpret_cast<const float*>(tbase + " + S(G.yf_off) + ");");
   int base = 0;
-  const int na = static_cast<int>(ent.size());
+  const int na = static_cast<int>(G.ent.size());
   for (int r = 0; r < T.rounds; ++r) {
     em.line("{  // round terms: " + S(T.terms[r]));
     em.ind++;
     for (int t = 0; t < T.terms[r]; ++t)
-      em.line("const int2 k" + S(t) + " = __ldg(&e3_atab[" + S(base + t * RW) + " + tl]);");
-    std::string v = "__int_as_float(k0.x) * yf[k0.y]";
+      em.line("const int2 k" + S(t) + " = __ldg(&e3_atab" + G.sfx + "[" + S(base + t * RW) + " + " +
+              ln + "]);");
+    const std::string j0 = G.pairs ? "(k0.y & 255)" : "k0.y";
+    std::string v = "__int_as_float(k0.x) * yf[" + j0 + "]";
     for (int t = 1; t < T.terms[r]; ++t)
       v = "fmaf(__int_as_float(k" + S(t) + ".x), yf[k" + S(t) + ".y], " + v + ")";
-    if (sh.dup_a) v = "bc(" + v + ")";
+    const std::string dst = G.pairs ? "Aw[k0.y >> 8]" : "Aw[" + S(r * RW) + " + " + ln + "]";
+    if (G.pairs) v = "bc(" + v + ")";
     if ((r + 1) * RW <= na)
-      em.line("Aw[" + S(r * RW) + " + tl] = " + v + ";");
+      em.line(dst + " = " + v + ";");
     else
-      em.line("if (tl < " + S(na - r * RW) + ") Aw[" + S(r * RW) + " + tl] = " + v + ";");
+      em.line("if (" + ln + " < " + S(na - r * RW) + ") " + dst + " = " + v + ";");
     em.ind--;
     em.line("}");
     base += T.terms[r] * RW;
   }
-  em.line("team_sync();");
+  em.line(group_sync + ";");
   em.line("const " + Ty + "* xs = reinterpret_cast<const " + Ty + "*>(stg + " + S(sh.x_off) + ") + u0;");
   em.line("const " + Ty + "* ss = reinterpret_cast<const " + Ty + "*>(stg + " + S(sh.s_off) + ") + u0;");
   // entry index of (path, i, k)
   std::map<std::tuple<int, int, int>, int> idx;
-  for (size_t n = 0; n < ent.size(); ++n) idx[{ent[n].path, ent[n].i, ent[n].k}] = static_cast<int>(n);
-  const int G = L.groups();
+  for (size_t n = 0; n < G.ent.size(); ++n)
+    idx[{G.ent[n].path, G.ent[n].i, G.ent[n].k}] = static_cast<int>(n);
+  const int NG = L.groups();
+  auto accv = [&](int comp, int g) {
+    return "q" + S(G.acc[comp]) + "_" + S(g);
+  };
   size_t p = 0;
-  while (p < pl.paths.size()) {
-    const int n1 = pl.paths[p].n1;
+  while (p < G.paths.size()) {
+    const int n1 = pl.paths[G.paths[p]].n1;
     size_t q = p;
-    while (q < pl.paths.size() && pl.paths[q].n1 == n1) ++q;
-    const Path& first = pl.paths[p];
+    while (q < G.paths.size() && pl.paths[G.paths[q]].n1 == n1) ++q;
+    const Path& first = pl.paths[G.paths[p]];
     const int d1 = 2 * first.l1 + 1;
     em.line("{  // node irrep " + S(n1) + " (l=" + S(first.l1) + ")");
     em.ind++;
     for (int i = 0; i < d1; ++i)
       emit_group_load(em, dtype, L, "xs + " + S((first.x_off + i) * pl.C), "x" + S(i));
-    for (size_t r = p; r < q; ++r) {
+    for (size_t rr = p; rr < q; ++rr) {
+      const int r = G.paths[rr];
       const Path& P = pl.paths[r];
       const int d3 = 2 * P.l3 + 1;
       std::vector<const AEntry*> pe;
-      for (const auto& e : ent)
-        if (e.path == static_cast<int>(r)) pe.push_back(&e);
+      for (const auto& e : G.ent)
+        if (e.path == r) pe.push_back(&e);
       em.line("{  // path " + S(r) + ": " + S(P.l1) + " x " + S(P.l2) + " -> " + S(P.l3) + ", " +
               S(pe.size()) + " entries");
       em.ind++;
@@ -732,16 +892,33 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
       auto aval = [&](const AEntry* e) {
         return "A" + S(idx[{e->path, e->i, e->k}]);
       };
-      for (const AEntry* e : pe) {
-        const std::string ld = "Aw[" + S(T.slot[idx[{e->path, e->i, e->k}]]) + "]";
-        em.line("const " + L.type() + " " + aval(e) + " = " + (sh.dup_a ? ld : L.bc(ld)) + ";");
+      if (G.pairs) {
+        // entries in slot order, two per 16-byte load
+        std::vector<const AEntry*> bys(pe);
+        std::sort(bys.begin(), bys.end(), [&](const AEntry* a, const AEntry* b) {
+          return T.slot[idx[{a->path, a->i, a->k}]] < T.slot[idx[{b->path, b->i, b->k}]];
+        });
+        for (size_t m = 0; m < bys.size(); m += 2) {
+          const int s0 = T.slot[idx[{bys[m]->path, bys[m]->i, bys[m]->k}]];
+          if (m + 1 < bys.size())
+            em.line("unsigned long long " + aval(bys[m]) + ", " + aval(bys[m + 1]) +
+                    "; { const ulonglong2 t_ = *reinterpret_cast<const ulonglong2*>(Aw + " + S(s0) +
+                    "); " + aval(bys[m]) + " = t_.x; " + aval(bys[m + 1]) + " = t_.y; }");
+          else
+            em.line("const unsigned long long " + aval(bys[m]) + " = Aw[" + S(s0) + "];");
+        }
+      } else {
+        for (const AEntry* e : pe) {
+          const std::string ld = "Aw[" + S(T.slot[idx[{e->path, e->i, e->k}]]) + "]";
+          em.line("const " + L.type() + " " + aval(e) + " = " + L.bc(ld) + ";");
+        }
       }
       if (d1 <= d3) {  // scale-input
         std::vector<bool> used(d1, false);
         for (const AEntry* e : pe) used[e->i] = true;
         for (int i = 0; i < d1; ++i) {
           if (!used[i]) continue;
-          for (int g = 0; g < G; ++g)
+          for (int g = 0; g < NG; ++g)
             em.line("const " + L.type() + " z" + S(i) + "_" + S(g) + " = " +
                     L.mul("s_" + S(g), "x" + S(i) + "_" + S(g)) + ";");
         }
@@ -751,8 +928,8 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
           return a->i != b->i ? a->i < b->i : a->k < b->k;
         });
         for (const AEntry* e : byi)
-          for (int g = 0; g < G; ++g) {
-            std::string acc = "q" + S(P.out_off + e->k) + "_" + S(g);
+          for (int g = 0; g < NG; ++g) {
+            const std::string acc = accv(P.out_off + e->k, g);
             em.line(acc + " = " + L.fma(aval(e), "z" + S(e->i) + "_" + S(g), acc) + ";");
           }
       } else {  // scale-output: t_k = sum_i A[i,k] x_i (i outer, k inner), then acc_k += s t_k
@@ -762,19 +939,19 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
         });
         std::vector<bool> started(d3, false);
         for (const AEntry* e : byi)
-          for (int g = 0; g < G; ++g) {
+          for (int g = 0; g < NG; ++g) {
             std::string tv = "t" + S(e->k) + "_" + S(g);
             std::string xv = "x" + S(e->i) + "_" + S(g);
             if (!started[e->k])
               em.line(L.type() + " " + tv + " = " + L.mul(aval(e), xv) + ";");
             else
               em.line(tv + " = " + L.fma(aval(e), xv, tv) + ";");
-            if (g == G - 1) started[e->k] = true;
+            if (g == NG - 1) started[e->k] = true;
           }
         for (int k = 0; k < d3; ++k) {
           if (!started[k]) continue;
-          for (int g = 0; g < G; ++g) {
-            std::string acc = "q" + S(P.out_off + k) + "_" + S(g);
+          for (int g = 0; g < NG; ++g) {
+            const std::string acc = accv(P.out_off + k, g);
             em.line(acc + " = " + L.fma("s_" + S(g), "t" + S(k) + "_" + S(g), acc) + ";");
           }
         }
@@ -788,8 +965,8 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
   }
 }
 
-void emit_group_acc_decl(Emitter& em, const Plan& pl, const Lanes& L) {
-  for (int c = 0; c < pl.nout; ++c) {
+void emit_group_acc_decl(Emitter& em, int nacc, const Lanes& L) {
+  for (int c = 0; c < nacc; ++c) {
     std::string l = L.type();
     for (int g = 0; g < L.groups(); ++g)
       l += std::string(g ? "," : "") + " q" + S(c) + "_" + S(g) + (L.pairs() ? " = 0ull" : " = 0.f");
@@ -797,19 +974,22 @@ void emit_group_acc_decl(Emitter& em, const Plan& pl, const Lanes& L) {
   }
 }
 
-// Stores the packed accumulators (times 1/N) at orow + comp*C and resets them;
-// with `add` the values are added to what the row already holds.
+// Stores the packed accumulators (times 1/N) of the group's output components at
+// orow + comp*C and resets them; with `add` the values are added to what the row
+// already holds.
 void emit_group_store(Emitter& em, const Plan& pl, const Lanes& L, const std::string& orow,
-                      bool add = false) {
+                      const std::vector<int>& acc, bool add = false) {
   for (int c = 0; c < pl.nout; ++c) {
+    if (acc[c] < 0) continue;
+    const std::string q = "q" + S(acc[c]);
     const std::string dst = orow + " + " + S(c * pl.C);
     if (!L.pairs()) {
-      em.line("*(" + dst + ") " + (add ? "+= " : "= ") + "q" + S(c) + "_0 * inv_avg;");
-      em.line("q" + S(c) + "_0 = 0.f;");
+      em.line("*(" + dst + ") " + (add ? "+= " : "= ") + q + "_0 * inv_avg;");
+      em.line(q + "_0 = 0.f;");
       continue;
     }
     auto val = [&](int g, const std::string& old) {
-      const std::string m = "mul2(q" + S(c) + "_" + S(g) + ", inv2)";
+      const std::string m = "mul2(" + q + "_" + S(g) + ", inv2)";
       return add ? "add2(" + old + ", " + m + ")" : m;
     };
     for (int g = 0; g < L.groups(); g += 2) {
@@ -825,8 +1005,98 @@ void emit_group_store(Emitter& em, const Plan& pl, const Lanes& L, const std::st
         em.line("*" + d + " = " + val(g, "*" + d) + ";");
       }
     }
-    for (int g = 0; g < L.groups(); ++g) em.line("q" + S(c) + "_" + S(g) + " = 0ull;");
+    for (int g = 0; g < L.groups(); ++g) em.line(q + "_" + S(g) + " = 0ull;");
   }
+}
+
+}  // namespace
+
+// Output irreps of each warp of a path-split team: longest-processing-time
+// assignment of the output irreps, weighted by their per-channel FMA count
+// (A entries + min(2l1+1, 2l3+1) of every path into them).
+std::vector<std::vector<int>> path_split_outputs(const Plan& pl, int warps) {
+  std::vector<double> cost(pl.outputs.size(), 0.0);
+  const std::vector<AEntry> ent = build_a_entries(pl);
+  for (const auto& e : ent) cost[pl.paths[e.path].o] += 1.0;
+  for (const auto& P : pl.paths) cost[P.o] += std::min(2 * P.l1 + 1, 2 * P.l3 + 1);
+  std::vector<int> order(pl.outputs.size());
+  for (size_t k = 0; k < order.size(); ++k) order[k] = static_cast<int>(k);
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+  std::vector<std::vector<int>> out(warps);
+  std::vector<double> load(warps, 0.0);
+  for (int o : order) {
+    int w = static_cast<int>(std::min_element(load.begin(), load.end()) - load.begin());
+    out[w].push_back(o);
+    load[w] += cost[o];
+  }
+  for (auto& v : out) std::sort(v.begin(), v.end());
+  return out;
+}
+
+// The coop groups of a staged shape: one for the whole team, or one per warp
+// of a path-split team (in that case A and yf areas follow one another).
+std::vector<CoopGroupInfo> coop_groups(const Plan& pl, const Shape& sh) {
+  std::vector<CoopGroupInfo> gs;
+  const std::vector<AEntry> all = build_a_entries(pl);
+  const bool pairs = sh.V % 2 == 0;
+  if (sh.psplit <= 1) {
+    CoopGroupInfo g;
+    for (size_t p = 0; p < pl.paths.size(); ++p) g.paths.push_back(static_cast<int>(p));
+    g.ent = all;
+    g.acc.resize(pl.nout);
+    for (int c = 0; c < pl.nout; ++c) g.acc[c] = c;
+    g.pairs = pairs;
+    gs.push_back(g);
+  } else {
+    for (const auto& outs : path_split_outputs(pl, sh.psplit)) {
+      CoopGroupInfo g;
+      g.acc.assign(pl.nout, -1);
+      int n = 0;
+      for (int o : outs)
+        for (int k = 0; k < 2 * pl.outputs[o].l + 1; ++k) g.acc[pl.outputs[o].off + k] = n++;
+      for (size_t p = 0; p < pl.paths.size(); ++p)
+        if (std::find(outs.begin(), outs.end(), pl.paths[p].o) != outs.end())
+          g.paths.push_back(static_cast<int>(p));
+      for (const auto& e : all)
+        if (std::find(g.paths.begin(), g.paths.end(), e.path) != g.paths.end()) g.ent.push_back(e);
+      g.pairs = pairs;
+      gs.push_back(g);
+    }
+  }
+  for (auto& g : gs) {
+    int slots = 0;
+    if (g.pairs) {
+      for (int p : g.paths) {
+        int n = 0;
+        for (const auto& e : g.ent) n += e.path == p;
+        slots += n + (n & 1);
+      }
+    } else {
+      slots = static_cast<int>(g.ent.size());
+    }
+    g.a_bytes = align_up((g.pairs ? 8 : 4) * slots, 16);
+    g.nacc = 0;
+    for (int a : g.acc) g.nacc = std::max(g.nacc, a + 1);
+  }
+  return gs;
+}
+
+namespace {
+
+// The flush of every group's accumulators into the row at `orow`.
+void emit_groups_store(Emitter& em, const Plan& pl, const Lanes& L,
+                       const std::vector<CoopGroup>& groups, bool split, bool add) {
+  if (!split) {
+    emit_group_store(em, pl, L, "orow", groups[0].acc, add);
+    return;
+  }
+  for (size_t w = 0; w < groups.size(); ++w) {
+    em.line(std::string(w ? "} else " : "") + (w + 1 < groups.size() ? "if (tw == " + S(w) + ") " : "") + "{");
+    em.ind++;
+    emit_group_store(em, pl, L, "orow", groups[w].acc, add);
+    em.ind--;
+  }
+  em.line("}");
 }
 
 std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
@@ -843,21 +1113,42 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("// C=" + S(pl.C) + " nx=" + S(pl.nx) + " ny=" + S(pl.ny) + " nout=" + S(pl.nout) +
           " paths=" + S(pl.paths.size()) + " dtype=" + (f16 ? "f16" : "f32") + " V=" + S(V) +
           " team=" + S(TW) + " teams/block=" + S(teams) + " stages=" + S(NS) +
-          " stage_bytes=" + S(sh.stage_bytes) + " contract_first=" + S(sh.coop ? 1 : 0));
+          " stage_bytes=" + S(sh.stage_bytes) + " contract_first=" + S(sh.coop ? 1 : 0) +
+          " path_split=" + S(sh.coop ? sh.psplit : 1) + " a_pairs=" + S(sh.dup_a ? 1 : 0));
   emit_prelude(em);
-  std::vector<AEntry> ent;
-  CoopTables tabs;
+  std::vector<CoopGroup> groups;
+  std::vector<CoopTables> tabs;
   const Lanes L{V};
+  const bool split = sh.coop && sh.psplit > 1;  // a row's paths split over the team's warps
+  const int yf_bytes = align_up(4 * pl.ny, 16);
   em.line("__device__ __forceinline__ unsigned long long pk(float lo, float hi) { unsigned long long r; asm(\"mov.b64 %0, {%1, %2};\" : \"=l\"(r) : \"f\"(lo), \"f\"(hi)); return r; }");
   em.line("__device__ __forceinline__ unsigned long long bc(float a) { return pk(a, a); }");
   em.line("__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) { unsigned long long d; asm(\"fma.rn.f32x2 %0, %1, %2, %3;\" : \"=l\"(d) : \"l\"(a), \"l\"(b), \"l\"(c)); return d; }");
   em.line("__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) { unsigned long long d; asm(\"mul.rn.f32x2 %0, %1, %2;\" : \"=l\"(d) : \"l\"(a), \"l\"(b)); return d; }");
   em.line("__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) { unsigned long long d; asm(\"add.rn.f32x2 %0, %1, %2;\" : \"=l\"(d) : \"l\"(a), \"l\"(b)); return d; }");
   emit_chunk_define(em);
+  int nacc = pl.nout;
   if (sh.coop) {
-    ent = build_a_entries(pl);
-    tabs = coop_tables(ent, 32 * TW);
-    em.o << tabs.source;
+    const std::vector<CoopGroupInfo> infos = coop_groups(pl, sh);
+    int a_off = sh.a_off;
+    nacc = 0;
+    for (size_t w = 0; w < infos.size(); ++w) {
+      CoopGroup G;
+      G.paths = infos[w].paths;
+      G.ent = infos[w].ent;
+      G.acc = infos[w].acc;
+      G.pairs = infos[w].pairs;
+      G.RW = split ? 32 : 32 * TW;
+      G.lane = split ? "lane" : "tl";
+      G.sfx = split ? "_w" + S(w) : "";
+      G.yf_off = sh.yf_off + (split ? static_cast<int>(w) * yf_bytes : 0);
+      G.a_off = a_off;
+      a_off += infos[w].a_bytes;
+      nacc = std::max(nacc, infos[w].nacc);
+      groups.push_back(G);
+      tabs.push_back(coop_tables(G));
+      em.o << tabs.back().source;
+    }
   }
   em.line("#define E3_SPIN_LIMIT (1u << 22)");
   em.line("__device__ __forceinline__ unsigned int smem_u32(const void* p) { return static_cast<unsigned int>(__cvta_generic_to_shared(p)); }");
@@ -872,7 +1163,7 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("__device__ __forceinline__ unsigned long long policy_evict_first() { unsigned long long p; asm volatile(\"createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\" : \"=l\"(p)); return p; }");
   em.line("__device__ __forceinline__ unsigned long long policy_evict_last() { unsigned long long p; asm volatile(\"createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\" : \"=l\"(p)); return p; }");
   em.line("__device__ __forceinline__ void fence_async_smem() { asm volatile(\"fence.proxy.async.shared::cta;\" ::: \"memory\"); }");
-  emit_signature(em, T, sh.block, 1);
+  emit_signature(em, T, sh.block, 1, sh.vec);
   em.line("{");
   em.ind++;
   em.line("extern __shared__ __align__(128) unsigned char smem[];");
@@ -901,7 +1192,8 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("const unsigned long long pol_stream = policy_evict_first();");
   em.line("const unsigned long long pol_keep = policy_evict_last();");
   em.line("const long long W = (long long)gridDim.x * " + S(teams) + ";  // teams in the grid");
-  em.line("const int u0 = tl * " + S(V) + ";  // first channel of this lane");
+  em.line(std::string("const int u0 = ") + (split ? "lane" : "tl") + " * " + S(V) +
+          ";  // first channel of this lane");
   emit_edge_range(em);
   em.line("long long pb = row_begin + (long long)blockIdx.x * " + S(teams) + " + team - W;  // producer receiver");
   em.line("int pe = 0, pe1 = 0, pr0 = 0;  // producer edge cursor within row pb, which starts at pr0");
@@ -909,7 +1201,7 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("bool pdone = false;");
   em.line("unsigned int ppos = 0, cpos = 0;");
   if (sh.coop) {
-    emit_group_acc_decl(em, pl, L);
+    emit_group_acc_decl(em, nacc, L);
     if (L.pairs()) em.line("const unsigned long long inv2 = bc(inv_avg);");
   } else {
     emit_acc_decl(em, pl, V);
@@ -924,7 +1216,7 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("  int r0 = row_ptr[pb], r1 = row_ptr[pb + 1];");
   em.line("  if (r0 < e_base || r1 < r0 || r1 > e_end) { if (issuer) atomicOr(status, 1u); r1 = r0; }");
   em.line("  pe = r0; pe1 = r1; pr0 = r0; pwin = -1;");
-  em.line("  if (r0 == r1) {  // empty row: zeros");
+  em.line(std::string("  if (r0 == r1") + (split ? " && tw == 0" : "") + ") {  // empty row: zeros");
   em.line("    float* zrow = out + (pb - row_begin) * " + S(o_row) + " + u0;");
   em.ind += 2;
   emit_store(em, pl, V, "zrow", true, false);
@@ -951,8 +1243,8 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
           S(sh.x_bytes) + "u : 0u));");
   em.line("  bulk_g2s(stg + " + S(sh.s_off) + ", s + (long long)(pe - e_base) * " + S(s_row) + ", " +
           S(sh.s_bytes) + "u, bars + st, pol_stream);");
-  em.line("  bulk_g2s(stg + " + S(sh.y_off) + ", Y + (long long)(pe - e_base) * " + S(pl.ny) + ", " +
-          S(sh.y_bytes) + "u, bars + st, pol_stream);");
+  em.line("  bulk_g2s(stg + " + S(sh.y_off) + ", Y + (long long)(pe - e_base) * " +
+          S(sh.vec ? 4 : pl.ny) + ", " + S(sh.y_bytes) + "u, bars + st, pol_stream);");
   em.line("  if (valid) bulk_g2s(stg + " + S(sh.x_off) + ", x + (long long)a * " +
           S(static_cast<long long>(pl.nx) * pl.C) + ", " + S(sh.x_bytes) +
           "u, bars + st, pol_keep);");
@@ -982,10 +1274,42 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("if (a >= 0) {");
   em.ind++;
   if (sh.coop) {
-    emit_coop_edge(em, pl, dtype, sh, ent, tabs);
+    if (split) {
+      // every warp converts the edge's Y row into its own float32 copy
+      em.line("{");
+      em.ind++;
+      em.line("float* yfw = reinterpret_cast<float*>(tbase + " + S(sh.yf_off) + " + tw * " +
+              S(yf_bytes) + ");");
+      emit_yf_fill(em, pl, dtype, sh, "stg + " + S(sh.y_off), "lane", 32, "yfw");
+      em.ind--;
+      em.line("}");
+      em.line("__syncwarp();");
+      for (size_t w = 0; w < groups.size(); ++w) {
+        em.line(std::string(w ? "} else " : "") + (w + 1 < groups.size() ? "if (tw == " + S(w) + ") " : "") +
+                "{  // warp " + S(w) + " of the team: " + S(groups[w].paths.size()) + " paths");
+        em.ind++;
+        emit_coop_edge(em, pl, dtype, sh, groups[w], tabs[w], "__syncwarp()");
+        em.ind--;
+      }
+      em.line("}");
+    } else {
+      em.line("{");
+      em.ind++;
+      em.line("float* yfw = reinterpret_cast<float*>(tbase + " + S(sh.yf_off) + ");");
+      emit_yf_fill(em, pl, dtype, sh, "stg + " + S(sh.y_off), "tl", 32 * TW, "yfw");
+      em.ind--;
+      em.line("}");
+      em.line("team_sync();");
+      emit_coop_edge(em, pl, dtype, sh, groups[0], tabs[0], "team_sync()");
+    }
   } else {
-    em.line("const " + T + "* ys = reinterpret_cast<const " + T + "*>(stg + " + S(sh.y_off) + ");");
-    emit_y_load(em, pl, dtype, "lds", "ys");
+    if (sh.vec) {
+      em.line("const float4 v_ = *reinterpret_cast<const float4*>(stg + " + S(sh.y_off) + ");");
+      emit_sh_eval(em, pl, "v_.x", "v_.y", "v_.z");
+    } else {
+      em.line("const " + T + "* ys = reinterpret_cast<const " + T + "*>(stg + " + S(sh.y_off) + ");");
+      emit_y_load(em, pl, dtype, "lds", "ys");
+    }
     em.line("const " + T + "* xs = reinterpret_cast<const " + T + "*>(stg + " + S(sh.x_off) + ") + u0;");
     em.line("const " + T + "* ss = reinterpret_cast<const " + T + "*>(stg + " + S(sh.s_off) + ") + u0;");
     emit_edge_body(em, pl, dtype, V, "lds", "xs", "ss");
@@ -1000,14 +1324,14 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("if (flags & 4) {");
   em.ind++;
   if (sh.coop)
-    emit_group_store(em, pl, L, "orow", true);
+    emit_groups_store(em, pl, L, groups, split, true);
   else
     emit_store(em, pl, V, "orow", false, true, true);
   em.ind--;
   em.line("} else {");
   em.ind++;
   if (sh.coop)
-    emit_group_store(em, pl, L, "orow");
+    emit_groups_store(em, pl, L, groups, split, false);
   else
     emit_store(em, pl, V, "orow", false, true);
   em.ind--;
@@ -1181,7 +1505,8 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
             ".b32 {" + regs + "}, [%" + S(n) + "];\" : " + outs + " : \"r\"(addr))");
   }
   em.line("extern \"C\" __global__ void __launch_bounds__(" + S(sh.block) + ", 1) e3conv_fwd(");
-  em.line("    const unsigned short* __restrict__ x, const unsigned short* __restrict__ Y,");
+  em.line(std::string("    const unsigned short* __restrict__ x, const ") +
+          (sh.vec ? "float" : "unsigned short") + "* __restrict__ Y,");
   em.line("    const unsigned short* __restrict__ s, const int* __restrict__ senders,");
   em.line("    const int* __restrict__ row_ptr, int num_nodes, int row_begin, int row_end, float* __restrict__ out,");
   em.line("    float inv_avg, unsigned int* __restrict__ status, const __grid_constant__ E3TensorMap xmap)");
@@ -1291,7 +1616,7 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("                    (pe - pr0 >= E3_ROW_CHUNK ? 4 : 0);");
   em.line("  bar_expect(sfull + st, " + S(sh.s_bytes + sh.y_bytes) + "u + (valid ? 4096u : 0u));");
   em.line("  bulk_g2s(stg + " + S(sh.s_off) + ", s + (long long)(pe - e_base) * " + S(s_row) + ", " + S(sh.s_bytes) + "u, sfull + st, pol_stream);");
-  em.line("  bulk_g2s(stg + " + S(sh.y_off) + ", Y + (long long)(pe - e_base) * " + S(pl.ny) + ", " + S(sh.y_bytes) + "u, sfull + st, pol_stream);");
+  em.line("  bulk_g2s(stg + " + S(sh.y_off) + ", Y + (long long)(pe - e_base) * " + S(sh.vec ? 4 : pl.ny) + ", " + S(sh.y_bytes) + "u, sfull + st, pol_stream);");
   em.line("  if (valid) tma_x_g2s(stg, &xmap, a, sfull + st, pol_keep);");
   em.line("}");
   em.line("__syncwarp();");
@@ -1316,8 +1641,12 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   em.line("const bool landed = bar_wait(sfull + st, (q / " + S(NS) + ") & 1u);");
   em.line("if (landed && hdr[4 * st] >= 0) {  // A tile of this edge (the MMA of the previous edge has completed)");
   em.ind++;
-  em.line("const unsigned short* ys = reinterpret_cast<const unsigned short*>(stg + " + S(sh.y_off) + ");");
-  em.line("for (int j = lane; j < " + S(pl.ny) + "; j += 32) yfw[j] = h2f(ys[j]);");
+  if (sh.vec) {
+    emit_yf_fill(em, pl, E3CONV_F16, sh, "stg + " + S(sh.y_off), "lane", 32, "yfw");
+  } else {
+    em.line("const unsigned short* ys = reinterpret_cast<const unsigned short*>(stg + " + S(sh.y_off) + ");");
+    em.line("for (int j = lane; j < " + S(pl.ny) + "; j += 32) yfw[j] = h2f(ys[j]);");
+  }
   em.line("__syncwarp();");
   em.line("// all loads and products first, then the float16 splits and the stores");
   for (int r = 0; r < tab.rounds; ++r) {

@@ -53,7 +53,8 @@ struct Shape {
   // A_p[i,k] = sum_j CG_p[i,j,k] Y_j in shared memory, then every lane applies
   // it to its channels with packed float32x2 FMAs.
   bool coop = false;
-  bool dup_a = false;                         // A stored as (a, a) pairs (one channel pair per lane)
+  bool dup_a = false;                         // A stored as (a, a) pairs in phase-2 order (channel pairs)
+  int psplit = 1;                             // > 1: the team's warps split a row's paths (each covers C)
   int na = 0;                                 // number of A entries (all paths)
   int a_off = 0, yf_off = 0;                  // A entries and float32 Y inside a team's region
   // Tensor-core variant (float16 inputs, C = 128): per edge, T = x^T (A_hi + A_lo)
@@ -66,7 +67,16 @@ struct Shape {
   int b_stride = 0;                           // bytes from A_hi to A_lo (tile + scratch)
   int b_off = 0, b_bytes = 0;                 // A_hi at b_off (b_bytes used by the MMA), A_lo at b_off + b_stride
   int tslot_off = 0;                          // tensor-memory address slot
+  // Edge input: false = the harmonics Y [E][ny] in the input dtype; true = the
+  // edge vectors r_ab as float32 [E][4] (x, y, z, unused), Y computed in the kernel.
+  bool vec = false;
   int smem_request = 0;                       // dynamic shared memory requested per block
+};
+
+// One term coef * x^px y^py z^pz of a real spherical harmonic on the unit sphere.
+struct ShMono {
+  double coef;
+  int px, py, pz;
 };
 
 // One entry A_p[i,k] of the per-edge contraction of CG with Y.
@@ -99,6 +109,8 @@ struct Plan {
   int auto_block = 0;                              // block chosen after a first compile (0: none)
   int req_coop = -1;                               // -1: automatic, 0: off, 1: on
   int req_tc = -1;                                 // -1: automatic, 0: off, 1: on
+  int req_vec = 0;                                 // 1: edges given as vectors, Y computed in the kernel
+  int req_psplit = -1;                             // -1: automatic, 0/1: off, k: split a row's paths over k warps
   int tc_team_cap = 0;                             // > 0: at most this many tensor-core teams per block
   bool tc_fallback = false;                        // tensor cores requested but the kernel spills: float32 variant
   int device = -1;                 // -1: host-only plan
@@ -113,6 +125,9 @@ int build_paths(Plan& plan, std::string& err);
 
 // cg.cpp
 std::vector<double> real_wigner_3j(int l1, int l2, int l3);
+
+// sh.cpp: component j = l^2 + l + m of the real harmonics, as polynomial terms
+std::vector<std::vector<ShMono>> sh_polynomials(int lmax);
 
 // codegen.cpp
 std::vector<AEntry> build_a_entries(const Plan& plan);

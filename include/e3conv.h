@@ -141,6 +141,7 @@ E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane,
 
 /* Options of the forward kernel (host-side; each recompiles the current
  * dtype's kernel):
+ *   Each option takes -1 (automatic) and the values listed with it.
  *   E3CONV_OPT_CONTRACT_FIRST: -1 automatic (default), 0 or 1.  With 1 the
  *   staged variant first contracts every path's CG tensor with the edge's Y
  *   into A_p[i,k] = sum_j CG_p[i,j,k] Y_j (channel-independent, shared by the
@@ -161,7 +162,31 @@ E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane,
  *   Requesting it for a shape outside those limits, or one whose kernel would
  *   still use local memory with two teams, keeps the float32 staged variant. */
 #define E3CONV_OPT_TENSOR_CORES 2
+/*   E3CONV_OPT_PATH_SPLIT: -1 automatic (default), 0 or 1 off, k = 2..8.  With
+ *   k the staged contract-first variant gives each receiver row to a team of
+ *   k warps that each cover all C channels (one warp must cover C: C/32
+ *   channels per lane, 1 or even) and split the row's output irreps among
+ *   themselves (balanced on FMA count): each warp forms only its paths' CG x Y
+ *   contractions and keeps only its outputs' sums in registers, so more warps
+ *   fit on an SM.  Same arithmetic per output element as without it.  Ignored
+ *   (the usual shape) where it does not apply. */
+#define E3CONV_OPT_PATH_SPLIT 3
+/*   E3CONV_OPT_EDGE_VECTORS: 0 (default) or 1.  With 1 the forward's edge_sh
+ *   argument holds the edge vectors r_ab = p_b - p_a as float32 [E][4]
+ *   (x, y, z, ignored: 16-byte rows) in every input dtype, and the kernel
+ *   evaluates the real spherical harmonics of r_ab / |r_ab| itself (the basis
+ *   above, l <= the plan's lmax; a zero vector gives Y_0 = 1, the rest 0),
+ *   in float32, instead of reading ny harmonics per edge. */
+#define E3CONV_OPT_EDGE_VECTORS 4
 E3CONV_API int e3conv_set_option(e3conv_plan plan, int option, int value);
+
+/* The current value of an option (as set; -1 where automatic). */
+E3CONV_API int e3conv_get_option(e3conv_plan plan, int option, int* value);
+
+/* The plan's real spherical harmonics of vec[3] / |vec| (host, double; the
+ * polynomials the kernels evaluate with E3CONV_OPT_EDGE_VECTORS), written to
+ * out[ny]; a zero vector gives 1, 0, 0, ... */
+E3CONV_API int e3conv_spherical_harmonics(e3conv_plan plan, const double* vec, double* out);
 
 /* Sizes: C channels, nx node components, ny edge components, nout output
  * components, num_paths P.  Any pointer may be NULL. */
@@ -202,7 +227,8 @@ E3CONV_API int e3conv_kernel_source(e3conv_plan plan, int dtype, char* buf, size
  * 1/N scale -> store of e3j's four plain steps; one kernel launch)
  *
  * node_features: device, [num_nodes][nx][C] of the plan's dtype.
- * edge_sh:       device, [E][ny], receiver-sorted.
+ * edge_sh:       device, [E][ny], receiver-sorted (with E3CONV_OPT_EDGE_VECTORS:
+ *                the edge vectors, float32 [E][4]).
  * edge_scalars:  device, [E][P][C], receiver-sorted.
  * senders:       device int32 [E], receiver-sorted, in [0, num_nodes).
  * receiver_row_ptr: device int32 [num_nodes+1], nondecreasing, row_ptr[0] = 0

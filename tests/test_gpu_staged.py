@@ -167,3 +167,31 @@ def test_staged_team_shapes(cuda_device, V, block, stages, contract_first):
     ref = oracle_out(irreps, x, Y, s, send, recv, n, 17.0)
     assert column_scaled_error(gpu, ref) <= 5e-3
     assert np.all(gpu[np.setdiff1d(np.arange(n), recv)] == 0)
+
+
+@pytest.mark.parametrize("split", [2, 3, 4])
+@pytest.mark.parametrize("C,dt", [(128, "f16"), (128, "f32"), (64, "f32"), (32, "f32")])
+def test_path_split_is_bitwise_the_unsplit_kernel(cuda_device, split, C, dt):
+    # each warp of a path-split team forms and applies only its outputs' paths; every output
+    # element is accumulated by the same FMA sequence as in the one-warp kernel, so the outputs
+    # are bitwise equal (and match the oracle), with empty rows and a row of several chunks
+    irreps = IRREPS[C]
+    rng = np.random.default_rng(100 * split + C)
+    n, e = 900, 16000
+    send, recv = _graph(rng, n, e, empty_frac=0.1)
+    recv[: 400] = 17                      # a row of more than three 128-edge chunks
+    o = np.lexsort((send, recv))
+    send, recv = send[o], recv[o]
+    pl, x, Y, s = _inputs(rng, irreps, n, e, dt)
+    base = e3.Conv(*irreps, 12.0, dtype=dt)
+    base.set_path_split(0)
+    sp = e3.Conv(*irreps, 12.0, dtype=dt)
+    sp.set_path_split(split)
+    src = sp.kernel_source()
+    assert f"path_split={split}" in src, src[:400]
+    assert sp.kernel_info()["local_bytes"] == 0
+    a = run_gpu(base, x, Y, s, send, recv, n)
+    b = run_gpu(sp, x, Y, s, send, recv, n)
+    assert np.array_equal(a, b)
+    ref = oracle_out(irreps, x, Y, s, send, recv, n, 12.0)
+    assert column_scaled_error(b, ref) <= 1e-5

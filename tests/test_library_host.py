@@ -96,6 +96,43 @@ def test_create_rejects_bad_scalars():
     assert not h.value
 
 
+def _emulate_phase1(c, src, Y, expect_entries):
+    """Runs every generated phase-1 table (one per coop group) on the host and checks the A
+    slots against the dense CG tables; returns the number of entries seen."""
+    seen = 0
+    for sfx, items in re.findall(r"// A layout(\S*) \(entry: path i k slot\):(.*)", src):
+        m = re.search(r"// A rounds" + re.escape(sfx) + r" \(lanes (\d+), pairs (\d)\):(.*)", src)
+        rw, pairs, terms = int(m.group(1)), int(m.group(2)), [int(v) for v in m.group(3).split()]
+        entries = [tuple(int(v) for v in it.split(":")) for it in items.split()]
+        tab = re.search(r"e3_atab" + re.escape(sfx) + r"\[\] = \{(.*?)\};", src, re.S).group(1)
+        cells = [(int(a), int(b)) for a, b in re.findall(r"\{(-?\d+), (\d+)\}", tab)]
+        slots = {}
+        base = 0
+        for r, nterms in enumerate(terms):
+            for lane in range(rw):
+                q = r * rw + lane
+                if q >= len(entries):
+                    continue
+                v, slot = 0.0, q
+                for term in range(nterms):
+                    cb, j = cells[base + term * rw + lane]
+                    if pairs and term == 0:
+                        slot, j = j >> 8, j & 255
+                    v += np.frombuffer(np.int32(cb).tobytes(), np.float32)[0] * Y[j]
+                slots[slot] = v
+            base += nterms * rw
+        assert base == len(cells)
+        assert len(slots) == len(entries)                 # distinct slots, one per entry
+        for p, i, k, slot in entries:
+            W = c.cg(p)
+            l2 = c.paths[p].l2
+            expect = sum(W[i, j, k] * Y[l2 * l2 + j] for j in range(W.shape[1]))
+            assert abs(slots[slot] - expect) < 1e-6 * (1 + abs(expect)), (sfx, p, i, k)
+        seen += len(entries)
+    assert seen == expect_entries
+    return seen
+
+
 def test_generated_kernel_unrolls_every_coefficient():
     s = SPECS["large_f16"]
     c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 40.0, dtype="f16")
@@ -109,29 +146,10 @@ def test_generated_kernel_unrolls_every_coefficient():
     src = c.kernel_source()
     na = sum(int((np.abs(c.cg(p)) > 1e-12).any(axis=1).sum()) for p in range(c.num_paths))
     assert na == 541
-    # emulate the generated phase-1 table on the host: slot q of the warp's A
-    # area must hold sum_j CG[i,j,k] Y_j of the (path, i, k) the layout names
-    layout = re.search(r"// A layout \(slot: path i k\):(.*)", src).group(1).split()
-    assert len(layout) == na
-    tab = re.search(r"e3_atab\[\] = \{(.*?)\};", src, re.S).group(1)
-    pairs = [(int(a), int(b)) for a, b in re.findall(r"\{(-?\d+), (\d+)\}", tab)]
+    # emulate the generated phase-1 table on the host: the slot each lane writes must
+    # hold sum_j CG[i,j,k] Y_j of the (path, i, k) the layout names
     Y = np.random.default_rng(1).normal(size=c.ny)
-    rw = 32 * int(re.search(r" team=(\d+)", src).group(1))   # lanes of one team
-    A = np.zeros(rw * ((na + rw - 1) // rw))
-    base = 0
-    for r, nterms in enumerate(int(m) for m in re.findall(r"// round terms: (\d+)", src)):
-        for lane in range(rw):
-            for term in range(nterms):
-                cb, j = pairs[base + term * rw + lane]
-                A[rw * r + lane] += np.frombuffer(np.int32(cb).tobytes(), np.float32)[0] * Y[j]
-        base += nterms * rw
-    assert base == len(pairs)
-    for q, item in enumerate(layout):
-        p, i, k = (int(v) for v in item.split(":"))
-        W = c.cg(p)
-        l2 = c.paths[p].l2
-        expect = sum(W[i, j, k] * Y[l2 * l2 + j] for j in range(W.shape[1]))
-        assert abs(A[q] - expect) < 1e-6 * (1 + abs(expect)), (q, item)
+    _emulate_phase1(c, src, Y, expect_entries=na)
     groups = info["channels_per_lane"] // 2
     assert src.count("fma2(") + src.count("mul2(") >= na * groups
     # per-lane products (contract_first = 0): every CG nonzero for every channel
@@ -347,3 +365,48 @@ def test_tensor_core_fallback_ladder_with_ring_depth(combo, stages):
         assert "tcgen05.mma" in src
     else:
         assert "(staged ring)" in src and "tcgen05" not in src
+
+
+@pytest.mark.parametrize("lmax", [0, 1, 2, 3, 6])
+def test_kernel_harmonics_match_the_oracle(lmax):
+    # the polynomials the kernels evaluate from edge vectors (Bonnet recursion, exact
+    # expansion in C++) against the oracle's Rodrigues-formula harmonics
+    sh = "+".join(f"1x{l}{'eo'[l % 2]}" for l in range(lmax + 1))
+    c = e3.Conv("4x0e", sh, "4x0e", 1.0)
+    rng = np.random.default_rng(lmax)
+    v = rng.normal(size=(40, 3)) * rng.uniform(0.01, 100, size=(40, 1))
+    got = np.array([c.spherical_harmonics(q) for q in v])
+    ref = oracle.sh(lmax, v / np.linalg.norm(v, axis=1, keepdims=True))
+    np.testing.assert_allclose(got, ref, atol=1e-12)
+    z = c.spherical_harmonics([0.0, 0.0, 0.0])
+    assert z[0] == 1.0 and np.all(z[1:] == 0)
+
+
+@pytest.mark.parametrize("name", ORDER)
+def test_edge_vector_kernels_compile_for_every_workload(name):
+    s = SPECS[name]
+    c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 10.0, dtype=s.dtype)
+    c.set_edge_vectors(1)
+    assert c.edge_vectors
+    info = c.kernel_info()
+    assert info["local_bytes"] == 0
+    src = c.kernel_source()
+    assert "sqrtf(r2_)" in src and "const float* __restrict__ Y" in src
+
+
+@pytest.mark.parametrize("split", [2, 3, 4])
+def test_path_split_tables_cover_every_entry_once(split):
+    # the warps of a path-split team own disjoint output irreps; their tables together form
+    # every A entry exactly once, each with the right value
+    s = SPECS["large_f16"]
+    c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 40.0, dtype="f16")
+    c.set_path_split(split)
+    src = c.kernel_source()
+    assert f"path_split={split}" in src and c.kernel_info()["local_bytes"] == 0
+    Y = np.random.default_rng(split).normal(size=c.ny)
+    _emulate_phase1(c, src, Y, expect_entries=541)
+    owned = [set(int(p) for p in re.findall(r"(\d+):\d+:\d+:\d+", items))
+             for _, items in re.findall(r"// A layout(\S*) \(entry: path i k slot\):(.*)", src)]
+    assert len(owned) == split
+    assert set().union(*owned) == set(range(c.num_paths))
+    assert sum(len(o) for o in owned) == c.num_paths          # each path in one warp
