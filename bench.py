@@ -68,6 +68,11 @@ def parse_args():
                     help="1: the tensor-core forward variant (float16 inputs, 128 channels)")
     ap.add_argument("--exchange", choices=["allgather", "halo"], default="allgather",
                     help="multi-GPU: how a rank receives its senders' node features")
+    ap.add_argument("--a-layout", type=int, default=-1,
+                    help="shared-memory layout of the contract-first A entries (0, 1, 2)")
+    ap.add_argument("--radial", action="store_true",
+                    help="edge scalars from the radial MLP on the tensor cores every step "
+                         "(workloads with MLP scalars)")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the supplementary timing of the tensor-core variant")
     return ap.parse_args()
@@ -358,6 +363,15 @@ def run_ours(args):
         conv.set_tensor_cores(1)
     if args.path_split != -1:
         conv.set_path_split(args.path_split)
+    if args.a_layout != -1:
+        conv.set_a_layout(args.a_layout)
+    if args.radial:
+        # the edge scalars come from the radial MLP on the tensor cores every step
+        if spec.scalars != "mlp":
+            raise SystemExit("--radial needs a workload whose scalars are the radial MLP (mace)")
+        conv.set_radial_mlp(spec.graph["r"], [w.astype(np.float32)
+                                               for w in configs.radial_weights(spec)])
+        args.edge_vectors = 1
     if args.edge_vectors:
         conv.set_edge_vectors(1)
     stream = torch.cuda.current_stream()
@@ -412,10 +426,16 @@ def run_ours(args):
         else:
             sharding.exchange_rows(shard, x, table)
 
-    def step(fwd_events=None):
+    def step(fwd_events=None, radial_events=None):
         e3._ok(e3._build_csr(precv, E_loc, rows, prp, pperm, pws, ws_bytes, sh), "e3conv_build_csr")
         if shard is not None:
             exchange()
+        if args.radial:
+            if radial_events:
+                radial_events[0].record(stream)
+            e3._ok(e3._radial_scalars(conv._h, pY, E_loc, ps, sh), "e3conv_radial_scalars")
+            if radial_events:
+                radial_events[1].record(stream)
         if fwd_events:
             fwd_events[0].record(stream)
         if shard is None:
@@ -435,13 +455,15 @@ def run_ours(args):
     clocks.start()
     fwd = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
+    rad = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)] if args.radial else [None] * args.steps
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t0.record(stream)
     for k in range(args.steps):
-        step(fwd[k])
+        step(fwd[k], rad[k])
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -449,7 +471,8 @@ def run_ours(args):
     clk = clocks.stop()
     ms = t0.elapsed_time(t1)
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd)
-    (ms, fwd_ms), total_edges = reduce_over_ranks([ms, fwd_ms], E_loc, world, dev)
+    rad_ms = statistics.mean(a.elapsed_time(b) for a, b in rad) if args.radial else 0.0
+    (ms, fwd_ms, rad_ms), total_edges = reduce_over_ranks([ms, fwd_ms, rad_ms], E_loc, world, dev)
     ms_per_step = ms / args.steps
     value = total_edges / (ms_per_step / 1000.0)
 
@@ -498,8 +521,24 @@ def run_ours(args):
                  "roofline_times_ms": {k: 1000 * v for k, v in times.items()},
                  "traffic_source": traffic_src})
 
+    radial = None
+    if args.radial:
+        # the radial kernel: tensor FLOPs of the hidden and output layers (3 MMAs per product
+        # for the hi/lo splits) and the scalars it writes
+        H = 64
+        tflop = 3 * 2 * E * H * (H + conv.num_paths * conv.C) / world
+        s_bytes = E * conv.num_paths * conv.C * in_bytes / world
+        radial = {"kernel": "k_radial", "radial_ms": rad_ms,
+                  "tensor_flops": tflop, "achieved_tflops": tflop / (rad_ms / 1000) / 1e12,
+                  "tensor_peak_tflops": pk["f16_tflops"],
+                  "tensor_frac": tflop / (rad_ms / 1000) / 1e12 / pk["f16_tflops"],
+                  "scalars_bytes_written": s_bytes,
+                  "write_gbs": s_bytes / (rad_ms / 1000) / 1e9,
+                  "note": "edge scalars s = MLP(bessel x cutoff of |r|) computed every step; "
+                          "the forward reads them back (value counts radial + forward)"}
+
     variants = None
-    if world == 1 and not info.get("tensor_cores") and not args.no_variants:
+    if world == 1 and not info.get("tensor_cores") and not args.no_variants and not args.radial:
         variants = {"tensor_cores": time_tensor_core_variant(args, spec, g, conv, x, Y, s, senders,
                                                             row_ptr, out, stream)}
 
@@ -518,15 +557,18 @@ def run_ours(args):
         def device_step():
             # the public calls a user makes: CSR build, (exchange,) forward
             e3.build_csr(receivers, rows, row_ptr=row_ptr, perm=perm[:E_loc], workspace=ws)
+            if args.radial:
+                conv.radial_scalars(Y, out=s)
             if shard is None:
                 conv.forward(table, Y, s, senders, row_ptr, out=out)
             else:
                 exchange()
                 conv.forward_rows(table, Y, s, senders, row_ptr, 0, rows, out=out)
-        e2e = run_e2e(args, [x, Y, s, senders, receivers], out, device_step, E_loc, world, dev)
+        inputs = [x, Y, senders, receivers] if args.radial else [x, Y, s, senders, receivers]
+        e2e = run_e2e(args, inputs, out, device_step, E_loc, world, dev)
 
     per_step = e3.csr_kernel_count(E_loc, rows) + 1 + (1 if args.exchange == "halo" and
-                                                       world > 1 else 0)
+                                                       world > 1 else 0) + (1 if args.radial else 0)
     launches = args.steps * per_step
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -555,6 +597,10 @@ def run_ours(args):
     }
     if variants is not None:
         line["variants"] = variants
+    if radial is not None:
+        line["radial"] = radial
+        line["config"]["step"] = ("e3conv_build_csr + e3conv_radial_scalars + e3conv_forward "
+                                  "(edge vectors)")
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -57,6 +57,7 @@ OPT_CONTRACT_FIRST = 1
 OPT_TENSOR_CORES = 2
 OPT_PATH_SPLIT = 3
 OPT_EDGE_VECTORS = 4
+OPT_A_LAYOUT = 5
 _get_option = _sig("e3conv_get_option", ctypes.c_int, _vp, ctypes.c_int, _c_int_p)
 _sh_host = _sig("e3conv_spherical_harmonics", ctypes.c_int, _vp, ctypes.POINTER(ctypes.c_double),
                 ctypes.POINTER(ctypes.c_double))
@@ -67,6 +68,9 @@ _forward_rows = _sig("e3conv_forward_rows", ctypes.c_int, _vp, _vp, _i64, _vp, _
                      _i64, _i64, _vp, _vp)
 _check = _sig("e3conv_check", ctypes.c_int, _vp, _vp)
 _partition = _sig("e3conv_partition_rows", ctypes.c_int, _vp, _i64, ctypes.c_int, _vp)
+_set_radial = _sig("e3conv_set_radial_mlp", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_double,
+                   ctypes.c_int, ctypes.c_int, _vp, _vp, _vp)
+_radial_scalars = _sig("e3conv_radial_scalars", ctypes.c_int, _vp, _vp, _i64, _vp, _vp)
 _csr_ws = _sig("e3conv_csr_workspace_size", ctypes.c_int, _i64, _i64,
                ctypes.POINTER(ctypes.c_size_t))
 _build_csr = _sig("e3conv_build_csr", ctypes.c_int, _vp, _i64, _i64, _vp, _vp, _vp,
@@ -83,7 +87,8 @@ EXPORTED = ["e3conv_create", "e3conv_destroy", "e3conv_set_input_dtype",
             "e3conv_set_launch_config", "e3conv_set_option", "e3conv_get_option",
             "e3conv_spherical_harmonics", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
             "e3conv_output_irrep", "e3conv_cg", "e3conv_kernel_info", "e3conv_kernel_source",
-            "e3conv_forward", "e3conv_forward_rows", "e3conv_check", "e3conv_partition_rows", "e3conv_csr_workspace_size", "e3conv_build_csr",
+            "e3conv_forward", "e3conv_forward_rows", "e3conv_check", "e3conv_partition_rows",
+            "e3conv_set_radial_mlp", "e3conv_radial_scalars", "e3conv_csr_workspace_size", "e3conv_build_csr",
             "e3conv_csr_check", "e3conv_build_csr_noalloc", "e3conv_csr_kernel_count", "e3conv_permute_rows", "e3conv_strerror", "e3conv_last_error",
             "e3conv_version"]
 
@@ -214,6 +219,9 @@ class Conv:
     def set_path_split(self, value: int = -1):
         _ok(_set_option(self._h, OPT_PATH_SPLIT, value), "e3conv_set_option")
 
+    def set_a_layout(self, value: int = -1):
+        _ok(_set_option(self._h, OPT_A_LAYOUT, value), "e3conv_set_option")
+
     def set_edge_vectors(self, value: int = 1):
         """1: the forward's Y argument holds edge vectors float32 [E][4]; harmonics in-kernel."""
         _ok(_set_option(self._h, OPT_EDGE_VECTORS, value), "e3conv_set_option")
@@ -307,6 +315,35 @@ class Conv:
         _ok(_forward_rows(self._h, _ptr(x), N, _ptr(Y) if E else None, _ptr(s) if E else None,
                           _ptr(senders) if E else None, _ptr(row_ptr), row_begin, row_end,
                           _ptr(out), _stream_handle(stream)), "e3conv_forward_rows")
+        return out
+
+    def set_radial_mlp(self, r_max: float, weights):
+        """Radial MLP from float32 weights [W_0 (num_basis x hidden), W_1 .. W_{L-1}
+        (hidden x hidden), W_L (hidden x P*C)] (host arrays, input index first)."""
+        ws = [np.ascontiguousarray(np.asarray(w, dtype=np.float32)) for w in weights]
+        nb, hidden = ws[0].shape
+        layers = len(ws) - 1
+        hid = np.ascontiguousarray(np.stack(ws[1:-1])) if layers > 1 else None
+        _ok(_set_radial(self._h, nb, float(r_max), hidden, layers, ws[0].ctypes.data_as(_vp),
+                        hid.ctypes.data_as(_vp) if hid is not None else None,
+                        ws[-1].ctypes.data_as(_vp)), "e3conv_set_radial_mlp")
+        self._radial = (r_max, ws)
+
+    def radial_scalars(self, edge_vectors, out=None, stream=None):
+        """s [E][P][C] (plan dtype) from edge vectors float32 [E][4] on the device."""
+        import torch
+        _require("edge_vectors", edge_vectors, dtype=torch.float32)
+        E = edge_vectors.shape[0]
+        if tuple(edge_vectors.shape) != (E, 4):
+            raise ValueError("edge_vectors must be [E][4]")
+        want = torch.float16 if self.dtype == "f16" else torch.float32
+        if out is None:
+            out = torch.empty((E, self.num_paths, self.C), dtype=want, device=edge_vectors.device)
+        else:
+            _require("out", out, edge_vectors.device, want, E * self.num_paths * self.C)
+        _ok(_radial_scalars(self._h, _ptr(edge_vectors) if E else None, E,
+                            _ptr(out) if E else None, _stream_handle(stream)),
+            "e3conv_radial_scalars")
         return out
 
     def forward_raw(self, x_ptr, Y_ptr, s_ptr, senders_ptr, row_ptr_ptr, num_nodes, out_ptr,

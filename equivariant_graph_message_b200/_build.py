@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libe3conv.so")
 CUDA_HOME = os.environ.get("CUDA_HOME", "/usr/local/cuda")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-SOURCES = ["api.cpp", "irreps.cpp", "cg.cpp", "sh.cpp", "codegen.cpp", "csr.cu"]
+SOURCES = ["api.cpp", "irreps.cpp", "cg.cpp", "sh.cpp", "codegen.cpp", "csr.cu", "radial.cu"]
 
 
 def _nvcc() -> str:

@@ -358,6 +358,8 @@ void e3conv_destroy(e3conv_plan h) {
     DeviceGuard g(pl.device);
     for (auto& v : pl.var) release_variant(v);
     if (pl.status) cudaFree(pl.status);
+    for (void* q : {pl.radial.d_w0, pl.radial.d_wh, pl.radial.d_wo})
+      if (q) cudaFree(q);
   }
   delete h;
 }
@@ -405,9 +407,13 @@ int e3conv_set_option(e3conv_plan h, int option, int value) {
   if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
   Plan& pl = h->p;
   if (option != E3CONV_OPT_CONTRACT_FIRST && option != E3CONV_OPT_TENSOR_CORES &&
-      option != E3CONV_OPT_PATH_SPLIT && option != E3CONV_OPT_EDGE_VECTORS)
+      option != E3CONV_OPT_PATH_SPLIT && option != E3CONV_OPT_EDGE_VECTORS &&
+      option != E3CONV_OPT_A_LAYOUT)
     return fail(E3CONV_ERR_UNSUPPORTED, "unknown option");
-  if (option == E3CONV_OPT_EDGE_VECTORS) {
+  if (option == E3CONV_OPT_A_LAYOUT) {
+    if (value < -1 || value > 2) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1 .. 2");
+    pl.req_alayout = value;
+  } else if (option == E3CONV_OPT_EDGE_VECTORS) {
     if (value != 0 && value != 1) return fail(E3CONV_ERR_INVALID_ARG, "value must be 0 or 1");
     pl.req_vec = value;
   } else if (option == E3CONV_OPT_PATH_SPLIT) {
@@ -435,6 +441,7 @@ int e3conv_get_option(e3conv_plan h, int option, int* value) {
     case E3CONV_OPT_TENSOR_CORES: *value = pl.req_tc; return E3CONV_OK;
     case E3CONV_OPT_PATH_SPLIT: *value = pl.req_psplit; return E3CONV_OK;
     case E3CONV_OPT_EDGE_VECTORS: *value = pl.req_vec; return E3CONV_OK;
+    case E3CONV_OPT_A_LAYOUT: *value = pl.req_alayout; return E3CONV_OK;
     default: return fail(E3CONV_ERR_UNSUPPORTED, "unknown option");
   }
 }
@@ -630,6 +637,70 @@ int e3conv_forward_rows(e3conv_plan h, const void* x, int64_t num_nodes, const v
                         const void* s, const int32_t* senders, const int32_t* row_ptr,
                         int64_t row_begin, int64_t row_end, float* out, e3conv_stream stream) {
   return launch_forward(h, x, num_nodes, Y, s, senders, row_ptr, row_begin, row_end, out, stream);
+}
+
+int e3conv_set_radial_mlp(e3conv_plan h, int num_basis, double r_max, int hidden, int layers,
+                          const float* w0, const float* w_hidden, const float* w_out) {
+  if (!h || !w0 || !w_out || (layers > 1 && !w_hidden))
+    return fail(E3CONV_ERR_INVALID_ARG, "NULL weights");
+  Plan& pl = h->p;
+  const int nout = static_cast<int>(pl.paths.size()) * pl.C;
+  std::vector<const float*> wh;
+  for (int l = 1; l < layers; ++l)
+    wh.push_back(w_hidden + static_cast<size_t>(l - 1) * hidden * hidden);
+  RadialPlan rp;
+  std::string err;
+  int rc = radial_prepare(rp, num_basis, r_max, hidden, layers, w0, wh.data(), w_out, nout, err);
+  if (rc != E3CONV_OK) return fail(rc, err);
+  if (pl.device >= 0) {
+    DeviceGuard g(pl.device);
+    struct Up { void** dst; const void* src; size_t n; };
+    const Up ups[3] = {{&rp.d_w0, rp.w0.data(), rp.w0.size() * sizeof(float)},
+                       {&rp.d_wh, rp.wh.data(), rp.wh.size()},
+                       {&rp.d_wo, rp.wo.data(), rp.wo.size()}};
+    for (const Up& u : ups) {
+      bool good = cudaMalloc(u.dst, std::max<size_t>(u.n, 16)) == cudaSuccess;
+      if (good && u.n) good = cudaMemcpy(*u.dst, u.src, u.n, cudaMemcpyHostToDevice) == cudaSuccess;
+      if (!good) {
+        cudaGetLastError();
+        for (void* q : {rp.d_w0, rp.d_wh, rp.d_wo}) if (q) cudaFree(q);
+        return fail(E3CONV_ERR_NOMEM, "allocating or copying the radial weights failed");
+      }
+    }
+  }
+  for (void* q : {pl.radial.d_w0, pl.radial.d_wh, pl.radial.d_wo})
+    if (q) {
+      DeviceGuard g(pl.device);
+      cudaFree(q);
+    }
+  rp.set = true;
+  pl.radial = std::move(rp);
+  return E3CONV_OK;
+}
+
+int e3conv_radial_scalars(e3conv_plan h, const float* edge_vectors, int64_t num_edges,
+                          void* edge_scalars, e3conv_stream stream) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  Plan& pl = h->p;
+  if (!pl.radial.set) return fail(E3CONV_ERR_INVALID_ARG, "no radial MLP set (e3conv_set_radial_mlp)");
+  if (num_edges < 0 || num_edges >= (1ll << 31))
+    return fail(E3CONV_ERR_INVALID_ARG, "num_edges out of range");
+  if (num_edges == 0) return E3CONV_OK;
+  if (!edge_vectors || !edge_scalars) return fail(E3CONV_ERR_INVALID_ARG, "NULL buffer");
+  if (!aligned16(edge_vectors) || !aligned16(edge_scalars))
+    return fail(E3CONV_ERR_INVALID_ARG, "edge_vectors and edge_scalars must be 16-byte aligned");
+  if (pl.device < 0) return fail(E3CONV_ERR_NO_DEVICE, "plan has no device");
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess || cur != pl.device)
+    return fail(E3CONV_ERR_INVALID_ARG, "current device differs from the plan's device");
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, pl.device) != cudaSuccess)
+    return fail(E3CONV_ERR_CUDA, "cannot query the SM count");
+  std::string err;
+  const int rc = radial_launch(pl.radial, pl.radial.d_w0, pl.radial.d_wh, pl.radial.d_wo,
+                               edge_vectors, num_edges, edge_scalars, pl.dtype == E3CONV_F16 ? 1 : 0,
+                               pl.status, sms, reinterpret_cast<cudaStream_t>(stream), err);
+  return rc == E3CONV_OK ? rc : fail(rc, err);
 }
 
 int e3conv_partition_rows(const int32_t* row_ptr, int64_t num_nodes, int parts, int64_t* bounds) {

@@ -53,7 +53,7 @@ struct CoopGroupInfo {
   std::vector<AEntry> ent;      // their A entries, build order within each path
   std::vector<int> acc;         // output component -> accumulator index (-1: not computed)
   int nacc = 0;                 // accumulators (output components) of the group
-  bool pairs = false;           // A stored as (a, a) pairs in phase-2 order
+  int amode = 0;                // A layout (Shape::amode)
   int a_bytes = 0;              // shared memory of the group's A entries
 };
 
@@ -188,7 +188,13 @@ Shape choose_shape(const Plan& pl, int dtype) {
     s.stage_bytes = s.y_off + align_up(s.y_bytes, 128);
     s.coop = pl.req_coop != 0 && (V == 1 || V % 2 == 0);
     s.psplit = s.coop ? psplit : 1;
-    s.dup_a = s.coop && V % 2 == 0;
+    // A layout: float slots in round order (a lane broadcasts each entry to a pair), or
+    // broadcast pairs in round order (the default where a lane holds one channel pair), or
+    // broadcast pairs in apply order read two per 16-byte load
+    s.amode = 0;
+    if (s.coop && V % 2 == 0)
+      s.amode = pl.req_alayout >= 0 ? pl.req_alayout : (V == 2 ? 1 : 0);
+    s.dup_a = s.amode >= 1;
     s.na = s.coop ? static_cast<int>(build_a_entries(pl).size()) : 0;
     int a_bytes = 0;
     if (s.coop)
@@ -743,7 +749,7 @@ struct CoopGroup {
   std::string sfx;              // suffix of the generated table
   std::vector<int> acc;         // output component -> accumulator index (-1: not computed)
   int a_off = 0, yf_off = 0;    // the group's A entries and float32 Y (bytes from tbase)
-  bool pairs = false;           // A stored as (a, a) pairs in phase-2 order, read two per load
+  int amode = 0;                // A layout (Shape::amode)
 };
 
 struct CoopTables {
@@ -769,7 +775,7 @@ CoopTables coop_tables(const CoopGroup& G) {
     return ent[a].terms.size() > ent[b].terms.size();
   });
   T.slot.assign(ent.size(), -1);
-  if (G.pairs) {
+  if (G.amode == 2) {
     int pos = 0;
     for (int p : G.paths) {
       for (size_t n = 0; n < ent.size(); ++n)
@@ -803,7 +809,7 @@ CoopTables coop_tables(const CoopGroup& G) {
           j = ent[order[q]].terms[t].first;
           cv = ent[order[q]].terms[t].second;
         }
-        if (G.pairs && t == 0 && q < order.size()) j |= T.slot[order[q]] << 8;
+        if (G.amode == 2 && t == 0 && q < order.size()) j |= T.slot[order[q]] << 8;
         const float cf = static_cast<float>(cv);
         unsigned int bits;
         std::memcpy(&bits, &cf, sizeof bits);
@@ -813,7 +819,7 @@ CoopTables coop_tables(const CoopGroup& G) {
     }
   }
   c << "};\n";
-  lay << "// A rounds" << G.sfx << " (lanes " << RW << ", pairs " << (G.pairs ? 1 : 0) << "):";
+  lay << "// A rounds" << G.sfx << " (lanes " << RW << ", mode " << G.amode << "):";
   for (int tr : T.terms) lay << " " << tr;
   lay << "\n";
   T.source = lay.str() + c.str();
@@ -829,7 +835,7 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh, con
   const Lanes L{sh.V};
   const int RW = G.RW;
   const std::string& ln = G.lane;
-  if (G.pairs)
+  if (G.amode >= 1)
     em.line("unsigned long long* Aw = reinterpret_cast<unsigned long long*>(tbase + " + S(G.a_off) + ");");
   else
     em.line("float* Aw = reinterpret_cast<float*>(tbase + " + S(G.a_off) + ");");
@@ -842,12 +848,12 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh, con
     for (int t = 0; t < T.terms[r]; ++t)
       em.line("const int2 k" + S(t) + " = __ldg(&e3_atab" + G.sfx + "[" + S(base + t * RW) + " + " +
               ln + "]);");
-    const std::string j0 = G.pairs ? "(k0.y & 255)" : "k0.y";
+    const std::string j0 = G.amode == 2 ? "(k0.y & 255)" : "k0.y";
     std::string v = "__int_as_float(k0.x) * yf[" + j0 + "]";
     for (int t = 1; t < T.terms[r]; ++t)
       v = "fmaf(__int_as_float(k" + S(t) + ".x), yf[k" + S(t) + ".y], " + v + ")";
-    const std::string dst = G.pairs ? "Aw[k0.y >> 8]" : "Aw[" + S(r * RW) + " + " + ln + "]";
-    if (G.pairs) v = "bc(" + v + ")";
+    const std::string dst = G.amode == 2 ? "Aw[k0.y >> 8]" : "Aw[" + S(r * RW) + " + " + ln + "]";
+    if (G.amode >= 1) v = "bc(" + v + ")";
     if ((r + 1) * RW <= na)
       em.line(dst + " = " + v + ";");
     else
@@ -892,7 +898,7 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh, con
       auto aval = [&](const AEntry* e) {
         return "A" + S(idx[{e->path, e->i, e->k}]);
       };
-      if (G.pairs) {
+      if (G.amode == 2) {
         // entries in slot order, two per 16-byte load
         std::vector<const AEntry*> bys(pe);
         std::sort(bys.begin(), bys.end(), [&](const AEntry* a, const AEntry* b) {
@@ -910,7 +916,7 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh, con
       } else {
         for (const AEntry* e : pe) {
           const std::string ld = "Aw[" + S(T.slot[idx[{e->path, e->i, e->k}]]) + "]";
-          em.line("const " + L.type() + " " + aval(e) + " = " + L.bc(ld) + ";");
+          em.line("const " + L.type() + " " + aval(e) + " = " + (G.amode >= 1 ? ld : L.bc(ld)) + ";");
         }
       }
       if (d1 <= d3) {  // scale-input
@@ -1038,14 +1044,14 @@ std::vector<std::vector<int>> path_split_outputs(const Plan& pl, int warps) {
 std::vector<CoopGroupInfo> coop_groups(const Plan& pl, const Shape& sh) {
   std::vector<CoopGroupInfo> gs;
   const std::vector<AEntry> all = build_a_entries(pl);
-  const bool pairs = sh.V % 2 == 0;
+  const int amode = sh.amode;
   if (sh.psplit <= 1) {
     CoopGroupInfo g;
     for (size_t p = 0; p < pl.paths.size(); ++p) g.paths.push_back(static_cast<int>(p));
     g.ent = all;
     g.acc.resize(pl.nout);
     for (int c = 0; c < pl.nout; ++c) g.acc[c] = c;
-    g.pairs = pairs;
+    g.amode = amode;
     gs.push_back(g);
   } else {
     for (const auto& outs : path_split_outputs(pl, sh.psplit)) {
@@ -1059,13 +1065,13 @@ std::vector<CoopGroupInfo> coop_groups(const Plan& pl, const Shape& sh) {
           g.paths.push_back(static_cast<int>(p));
       for (const auto& e : all)
         if (std::find(g.paths.begin(), g.paths.end(), e.path) != g.paths.end()) g.ent.push_back(e);
-      g.pairs = pairs;
+      g.amode = amode;
       gs.push_back(g);
     }
   }
   for (auto& g : gs) {
     int slots = 0;
-    if (g.pairs) {
+    if (g.amode == 2) {
       for (int p : g.paths) {
         int n = 0;
         for (const auto& e : g.ent) n += e.path == p;
@@ -1074,7 +1080,7 @@ std::vector<CoopGroupInfo> coop_groups(const Plan& pl, const Shape& sh) {
     } else {
       slots = static_cast<int>(g.ent.size());
     }
-    g.a_bytes = align_up((g.pairs ? 8 : 4) * slots, 16);
+    g.a_bytes = align_up((g.amode >= 1 ? 8 : 4) * slots, 16);
     g.nacc = 0;
     for (int a : g.acc) g.nacc = std::max(g.nacc, a + 1);
   }
@@ -1114,7 +1120,7 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
           " paths=" + S(pl.paths.size()) + " dtype=" + (f16 ? "f16" : "f32") + " V=" + S(V) +
           " team=" + S(TW) + " teams/block=" + S(teams) + " stages=" + S(NS) +
           " stage_bytes=" + S(sh.stage_bytes) + " contract_first=" + S(sh.coop ? 1 : 0) +
-          " path_split=" + S(sh.coop ? sh.psplit : 1) + " a_pairs=" + S(sh.dup_a ? 1 : 0));
+          " path_split=" + S(sh.coop ? sh.psplit : 1) + " a_layout=" + S(sh.amode));
   emit_prelude(em);
   std::vector<CoopGroup> groups;
   std::vector<CoopTables> tabs;
@@ -1137,7 +1143,7 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
       G.paths = infos[w].paths;
       G.ent = infos[w].ent;
       G.acc = infos[w].acc;
-      G.pairs = infos[w].pairs;
+      G.amode = infos[w].amode;
       G.RW = split ? 32 : 32 * TW;
       G.lane = split ? "lane" : "tl";
       G.sfx = split ? "_w" + S(w) : "";

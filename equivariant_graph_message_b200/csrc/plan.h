@@ -6,6 +6,7 @@
 #include <vector>
 
 #include <cuda.h>
+#include <cuda_runtime.h>
 
 #include "../../include/e3conv.h"
 
@@ -53,7 +54,9 @@ struct Shape {
   // A_p[i,k] = sum_j CG_p[i,j,k] Y_j in shared memory, then every lane applies
   // it to its channels with packed float32x2 FMAs.
   bool coop = false;
-  bool dup_a = false;                         // A stored as (a, a) pairs in phase-2 order (channel pairs)
+  bool dup_a = false;                         // A stored as (a, a) pairs (amode >= 1)
+  int amode = 0;                              // A layout: 0 float slots, round order; 1 pairs, round
+                                              // order; 2 pairs, apply order (two per 16-byte load)
   int psplit = 1;                             // > 1: the team's warps split a row's paths (each covers C)
   int na = 0;                                 // number of A entries (all paths)
   int a_off = 0, yf_off = 0;                  // A entries and float32 Y inside a team's region
@@ -97,6 +100,20 @@ struct Variant {
   int grid_blocks = 0;  // persistent grid of the staged variant (blocks per SM x SMs)
 };
 
+// Radial MLP of a plan (e3conv_set_radial_mlp): host copies of the packed
+// weights and their device copies (owned by the plan).
+struct RadialPlan {
+  bool set = false;
+  int nb = 0, hidden = 0, layers = 0, nout = 0, chunks = 0;
+  double r_max = 0.0;
+  int scale_exp_h = 0, scale_exp_o = 0;   // weights scaled by 2^s before the float16 split
+  std::vector<float> w0;                  // [nb][hidden] float32
+  std::vector<unsigned char> wh, wo;      // packed hi / lo float16 operands
+  void* d_w0 = nullptr;
+  void* d_wh = nullptr;
+  void* d_wo = nullptr;
+};
+
 struct Plan {
   int C = 0, nx = 0, ny = 0, nout = 0, lmax = 0;
   std::vector<Irrep> node, filt;
@@ -109,6 +126,7 @@ struct Plan {
   int auto_block = 0;                              // block chosen after a first compile (0: none)
   int req_coop = -1;                               // -1: automatic, 0: off, 1: on
   int req_tc = -1;                                 // -1: automatic, 0: off, 1: on
+  int req_alayout = -1;                            // -1: automatic, else Shape::amode (channel pairs only)
   int req_vec = 0;                                 // 1: edges given as vectors, Y computed in the kernel
   int req_psplit = -1;                             // -1: automatic, 0/1: off, k: split a row's paths over k warps
   int tc_team_cap = 0;                             // > 0: at most this many tensor-core teams per block
@@ -117,6 +135,7 @@ struct Plan {
   CUcontext ctx = nullptr;
   unsigned int* status = nullptr;  // device status word
   Variant var[2];
+  RadialPlan radial;
 };
 
 // irreps.cpp
@@ -128,6 +147,14 @@ std::vector<double> real_wigner_3j(int l1, int l2, int l3);
 
 // sh.cpp: component j = l^2 + l + m of the real harmonics, as polynomial terms
 std::vector<std::vector<ShMono>> sh_polynomials(int lmax);
+
+// radial.cu
+int radial_prepare(RadialPlan& rp, int nb, double r_max, int hidden, int layers, const float* w0,
+                   const float* const* wh, const float* wo, int nout, std::string& err);
+size_t radial_smem_bytes(const RadialPlan& rp);
+int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, const void* dev_wo,
+                  const float* vec, long long num_edges, void* s, int out_f16, unsigned* status,
+                  int grid, cudaStream_t st, std::string& err);
 
 // codegen.cpp
 std::vector<AEntry> build_a_entries(const Plan& plan);

@@ -1,0 +1,551 @@
+// Radial scalars s_ab on the tensor cores: bessel basis x cosine cutoff of the
+// edge length, SiLU MLP, output layer of P*C scalars per edge.
+//
+// What it computes (e3j.core.Convolution, class docstring: the edge scalars
+// are an MLP of radial-basis encodings; gate_points_2102 page, "Scope":
+// bessel radial bases and a cosine cutoff, and its Network parameters
+// number_of_basis, radial_layers, radial_neurons), for edge e of length d:
+//   h_0[n] = sqrt(2/r) sin((n+1) pi d / r) / d * (1 + cos(pi d / r)) / 2   (d < r; 0 beyond;
+//            evaluated as sinpi / cospi of (n+1) d / r and d / r
+//            d = 0 takes the limit (n+1) pi / r)
+//   h_1    = SiLU(h_0 W_0)                      (num_basis -> hidden, CUDA cores)
+//   h_l+1  = SiLU(h_l W_l),  l = 1 .. L-1       (hidden -> hidden, tensor cores)
+//   s      = h_L W_L                            (hidden -> P*C, tensor cores)
+// with SiLU(v) = v / (1 + exp(-v)), no biases.
+//
+// Tensor-core layers: one CTA of 128 threads per tile of 128 edges (thread t
+// <-> edge row t <-> tensor-memory lane t).  A = the tile's activations
+// [128 edges x hidden], B = the weights [N outputs x hidden] (both K-major,
+// float16, core matrices of 8 rows x 16 bytes, no swizzle), D = A B^T in
+// tensor memory (float32).  Both operands are split into float16 hi + lo
+// parts, D = A_hi B_hi + A_hi B_lo + A_lo B_hi (the lo x lo term is below
+// float32 rounding), which keeps the products at float32 accuracy; the
+// weights are scaled by a power of two before the split (undone exactly on
+// the way out) so that their lo parts stay normal float16 numbers.
+// The output layer runs in chunks of 128 columns, double-buffered in shared
+// memory (bulk copies of prepacked chunks) and in tensor memory (the MMAs of
+// chunk c overlap the stores of chunk c-1).  All waits are bounded: on
+// timeout a CTA sets bit 4 of the status word, drains what it issued
+// (bounded) and stops.
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "plan.h"
+
+namespace e3c {
+
+namespace {
+
+constexpr int kTile = 128;           // edges per tile (MMA M)
+constexpr int kMaxBasis = 16;        // radial bases (layer 0 is unrolled over them)
+constexpr int kChunk = 128;          // output columns per output-layer chunk (MMA N)
+constexpr unsigned kSpinLimit = 1u << 22;
+
+__device__ __forceinline__ unsigned smem_u32(const void* p) {
+  return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(unsigned long long* b, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect(unsigned long long* b, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(unsigned long long* b, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait(unsigned long long* b, unsigned parity) {
+  for (unsigned it = 0; it < kSpinLimit; ++it)
+    if (mbar_try(b, parity)) return true;
+  return false;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes,
+                                         unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// K-major, no-swizzle shared-memory matrix descriptor: core matrices of 8 rows x
+// 16 bytes; 128 bytes between the two K-adjacent core matrices of a 16-wide K
+// slab, 256 bytes between row groups of 8.
+__device__ __forceinline__ unsigned long long kmajor_desc(const void* p) {
+  return static_cast<unsigned long long>((smem_u32(p) & 0x3FFFF) >> 4) | (8ull << 16) |
+         (16ull << 32) | (1ull << 46);
+}
+// byte offset of element (row r, k) in a K-major operand of `rows` rows: K slab
+// k / 16 of rows * 32 bytes, then the core-matrix layout inside the slab
+__device__ __forceinline__ int kmajor_off(int r, int k, int rows) {
+  return (k >> 4) * rows * 32 + (r >> 3) * 256 + ((k >> 3) & 1) * 128 + (r & 7) * 16 + (k & 7) * 2;
+}
+// instruction descriptor of kind::f16: float16 A and B (both K-major), float32 D
+__device__ __forceinline__ unsigned idesc_f16(int m, int n) {
+  return (1u << 4) | (static_cast<unsigned>(n >> 3) << 17) | (static_cast<unsigned>(m >> 4) << 24);
+}
+__device__ __forceinline__ void mma_f16(unsigned tmem_d, unsigned long long a, unsigned long long b,
+                                        unsigned idesc, unsigned accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(
+          tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(unsigned long long* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(unsigned addr, float* v) {
+  unsigned r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(addr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(r[q]);
+}
+
+__device__ __forceinline__ float silu(float v) { return v / (1.0f + expf(-v)); }
+
+// two floats rounded to float16, low half first
+__device__ __forceinline__ unsigned pack_half2(float lo, float hi) {
+  unsigned r;
+  asm("{ .reg .f16 a, b; cvt.rn.f16.f32 a, %1; cvt.rn.f16.f32 b, %2; mov.b32 %0, {a, b}; }"
+      : "=r"(r)
+      : "f"(lo), "f"(hi));
+  return r;
+}
+
+// Writes row r's values v[0..K) of a K-major operand as float16 hi and lo parts.
+template <int K>
+__device__ __forceinline__ void store_split_row(unsigned char* hi, unsigned char* lo, int r,
+                                                const float* v, int rows) {
+#pragma unroll
+  for (int k = 0; k < K; k += 2) {
+    const __half h0 = __float2half_rn(v[k]), h1 = __float2half_rn(v[k + 1]);
+    const __half l0 = __float2half_rn(v[k] - __half2float(h0));
+    const __half l1 = __float2half_rn(v[k + 1] - __half2float(h1));
+    const int off = kmajor_off(r, k, rows);
+    *reinterpret_cast<__half2*>(hi + off) = __halves2half2(h0, h1);
+    *reinterpret_cast<__half2*>(lo + off) = __halves2half2(l0, l1);
+  }
+}
+
+struct RadialArgs {
+  const float* vec;        // [E][4] edge vectors (x, y, z, unused)
+  long long num_edges;
+  const float* w0;         // [nb][H] float32 (layer 0, CUDA cores)
+  const unsigned char* wh; // hidden layers 1..L-1: per layer hi then lo, [H x H] K-major each
+  const unsigned char* wo; // output layer: per chunk hi then lo, [kChunk x H] K-major each
+  float w_scale_inv_h;     // 2^-s of the hidden weights' scale
+  float w_scale_inv_o;     // 2^-s of the output weights' scale
+  float pi_r, inv_r, norm; // pi / r_max, 1 / r_max and sqrt(2 / r_max)
+  int nb, layers;          // basis size, hidden layers L (>= 1)
+  int nout, chunks;        // P*C outputs, chunks of kChunk (the last padded with zero weights)
+  float r_max;
+  void* s;                 // [E][nout] float32 or float16
+  int out_f16;
+  unsigned* status;
+};
+
+// Shared memory of one CTA (bytes): w0 (nb x H float32), the hidden layers'
+// weights, the activations (hi, lo), two output-weight chunks (hi, lo each),
+// barriers and the tensor-memory slot.
+template <int H>
+struct Smem {
+  static constexpr int kAct = kTile * H * 2;     // one K-major [128 x H] float16 operand
+  static constexpr int kWhid = H * H * 2;        // one [H x H] float16 operand
+  static constexpr int kWout = kChunk * H * 2;   // one [128 x H] float16 operand
+};
+
+template <int H>
+__global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
+  extern __shared__ __align__(1024) unsigned char sm[];
+  using L = Smem<H>;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  float* w0s = reinterpret_cast<float*>(sm);                        // nb x H
+  unsigned char* whs = sm + ((a.nb * H * 4 + 1023) / 1024) * 1024;    // (layers-1) x (hi, lo)
+  unsigned char* act = whs + (a.layers - 1) * 2 * L::kWhid;           // hi, lo
+  unsigned char* wos = act + 2 * L::kAct;                             // 2 buffers x (hi, lo)
+  unsigned long long* bars = reinterpret_cast<unsigned long long*>(wos + 4 * L::kWout);
+  unsigned long long* bar_w = bars;        // [2] output-weight chunk landed
+  unsigned long long* bar_mma = bars + 2;  // [2] output MMAs of a chunk done
+  unsigned long long* bar_hid = bars + 4;  // hidden-layer MMAs done
+  unsigned long long* bar_wh = bars + 5;   // hidden weights landed
+  unsigned* tslot = reinterpret_cast<unsigned*>(bars + 6);
+
+  for (int q = tid; q < a.nb * H; q += 128) w0s[q] = a.w0[q];
+  if (tid == 0) {
+    for (int k = 0; k < 6; ++k) mbar_init(bars + k, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(tslot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_before();
+  __syncthreads();
+  tc_after();
+  const unsigned tmem = *tslot;
+  const unsigned t_hid = tmem;                 // columns [0, H): hidden-layer D
+  // output-layer D: two buffers of 128 columns at 256 and 384
+  const unsigned lane_off = static_cast<unsigned>(32 * warp) << 16;
+  bool ok = true;
+  // phase bits (bit b: buffer b) of the weight-chunk and output-MMA barriers
+  unsigned ph_w = 0, ph_mma = 0, ph_hid = 0;
+  // copies and MMAs thread 0 issued and has not yet seen complete (bit b: buffer b; drained on
+  // a timeout)
+  unsigned pend_w = 0, pend_mma = 0;
+  bool pend_hid = false, pend_wh = false;
+  if (a.layers > 1 && tid == 0) {
+    const unsigned bytes = static_cast<unsigned>((a.layers - 1) * 2 * L::kWhid);
+    mbar_expect(bar_wh, bytes);
+    bulk_g2s(whs, a.wh, bytes, bar_wh);
+    pend_wh = true;
+  }
+  if (a.layers > 1) {
+    ok = __syncthreads_and(mbar_wait(bar_wh, 0));
+    pend_wh = !ok;
+  }
+  const float pi_r = a.pi_r;
+  const float norm = a.norm;
+  const long long tiles = (a.num_edges + kTile - 1) / kTile;
+  for (long long tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+    const long long e = tile * kTile + tid;
+    const bool valid = e < a.num_edges;
+    // prefetch the first output-weight chunks of this tile
+    if (tid == 0) {
+      for (int c = 0; c < 2 && c < a.chunks; ++c) {
+        mbar_expect(bar_w + c, 2 * L::kWout);
+        bulk_g2s(wos + c * 2 * L::kWout, a.wo + static_cast<size_t>(c) * 2 * L::kWout,
+                 2 * L::kWout, bar_w + c);
+        pend_w |= 1u << c;
+      }
+    }
+    // layer 0 on the CUDA cores: basis x cutoff, then SiLU(h0 W0)
+    float h[H];
+    {
+      float d = 0.f;
+      if (valid) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(a.vec) + e);
+        d = sqrtf(fmaf(v.x, v.x, fmaf(v.y, v.y, v.z * v.z)));
+      }
+      const bool inside = valid && d < a.r_max;
+      const float t = d * a.inv_r;                        // d / r in [0, 1) inside
+      const float u = 0.5f * (1.0f + cospif(t));          // cos(pi d / r)
+      float b[kMaxBasis];
+#pragma unroll
+      for (int n = 0; n < kMaxBasis; ++n) {
+        b[n] = (!inside || n >= a.nb)
+                   ? 0.f
+                   : (d > 0.f ? norm * sinpif((n + 1) * t) / d : norm * (n + 1) * pi_r) * u;
+      }
+#pragma unroll
+      for (int j = 0; j < H; ++j) {
+        float z = 0.f;
+#pragma unroll
+        for (int n = 0; n < kMaxBasis; ++n)
+          if (n < a.nb) z = fmaf(b[n], w0s[n * H + j], z);
+        h[j] = silu(z);
+      }
+    }
+    // hidden layers 1 .. L-1 on the tensor cores
+    for (int l = 1; l < a.layers && ok; ++l) {
+      store_split_row<H>(act, act + L::kAct, tid, h, kTile);
+      fence_async_smem();
+      tc_before();
+      __syncthreads();
+      tc_after();
+      if (tid == 0) {
+        const unsigned char* whi = whs + (l - 1) * 2 * L::kWhid;
+        const unsigned char* wlo = whi + L::kWhid;
+        const unsigned id = idesc_f16(kTile, H);
+        unsigned acc = 0;
+        for (int ks = 0; ks < H / 16; ++ks) {
+          const int ao = ks * kTile * 32, bo = ks * H * 32;
+          mma_f16(t_hid, kmajor_desc(act + ao), kmajor_desc(whi + bo), id, acc);
+          acc = 1;
+          mma_f16(t_hid, kmajor_desc(act + ao), kmajor_desc(wlo + bo), id, 1);
+          mma_f16(t_hid, kmajor_desc(act + L::kAct + ao), kmajor_desc(whi + bo), id, 1);
+        }
+        mma_commit(bar_hid);
+        pend_hid = true;
+      }
+      ok = __syncthreads_and(mbar_wait(bar_hid, ph_hid));
+      tc_after();
+      if (!ok) break;
+      ph_hid ^= 1u;
+      pend_hid = false;
+#pragma unroll
+      for (int j0 = 0; j0 < H; j0 += 32) {
+        float v[32];
+        tmem_ld32(t_hid + lane_off + j0, v);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) h[j0 + q] = silu(v[q] * a.w_scale_inv_h);
+      }
+      tc_before();
+      __syncthreads();  // every thread has read D before the next layer's MMAs overwrite it
+      tc_after();
+    }
+    if (!ok) break;
+    // output layer: chunks of 128 columns
+    store_split_row<H>(act, act + L::kAct, tid, h, kTile);
+    fence_async_smem();
+    tc_before();
+    __syncthreads();
+    tc_after();
+    const unsigned id = idesc_f16(kTile, kChunk);
+    for (int c = 0; c <= a.chunks && ok; ++c) {
+      if (c < a.chunks) {
+        const int buf = c & 1;
+        ok = __syncthreads_and(mbar_wait(bar_w + buf, (ph_w >> buf) & 1u));
+        if (!ok) break;
+        ph_w ^= 1u << buf;
+        pend_w &= ~(1u << buf);
+        if (tid == 0) {
+          const unsigned char* whi = wos + buf * 2 * L::kWout;
+          const unsigned char* wlo = whi + L::kWout;
+          for (int ks = 0; ks < H / 16; ++ks) {
+            const int ao = ks * kTile * 32, bo = ks * kChunk * 32;
+            const unsigned td = tmem + 256u + 128u * buf;
+            mma_f16(td, kmajor_desc(act + ao), kmajor_desc(whi + bo), id, ks > 0);
+            mma_f16(td, kmajor_desc(act + ao), kmajor_desc(wlo + bo), id, 1);
+            mma_f16(td, kmajor_desc(act + L::kAct + ao), kmajor_desc(whi + bo), id, 1);
+          }
+          mma_commit(bar_mma + buf);
+          pend_mma |= 1u << buf;
+        }
+      }
+      if (c >= 1) {  // stores of chunk c-1, then its weight buffer takes chunk c+1
+        const int pb = (c - 1) & 1;
+        ok = __syncthreads_and(mbar_wait(bar_mma + pb, (ph_mma >> pb) & 1u));
+        tc_after();
+        if (!ok) break;
+        ph_mma ^= 1u << pb;
+        pend_mma &= ~(1u << pb);
+        if (tid == 0 && c + 1 < a.chunks) {
+          mbar_expect(bar_w + pb, 2 * L::kWout);
+          bulk_g2s(wos + pb * 2 * L::kWout, a.wo + static_cast<size_t>(c + 1) * 2 * L::kWout,
+                   2 * L::kWout, bar_w + pb);
+          pend_w |= 1u << pb;
+        }
+        const int col0 = (c - 1) * kChunk;
+#pragma unroll 1
+        for (int j0 = 0; j0 < kChunk; j0 += 32) {
+          float v[32];
+          tmem_ld32(tmem + 256u + 128u * pb + lane_off + j0, v);
+          if (valid) {
+            const int cols = min(32, a.nout - (col0 + j0));
+            if (cols > 0) {
+              if (a.out_f16) {
+                __half* dst = static_cast<__half*>(a.s) + e * a.nout + col0 + j0;
+                if (cols == 32 && ((a.nout & 7) == 0)) {
+#pragma unroll
+                  for (int q = 0; q < 32; q += 8) {
+                    const float f = a.w_scale_inv_o;
+                    *reinterpret_cast<uint4*>(dst + q) =
+                        make_uint4(pack_half2(v[q] * f, v[q + 1] * f), pack_half2(v[q + 2] * f, v[q + 3] * f),
+                                   pack_half2(v[q + 4] * f, v[q + 5] * f), pack_half2(v[q + 6] * f, v[q + 7] * f));
+                  }
+                } else {
+#pragma unroll
+                  for (int q = 0; q < 32; ++q)
+                    if (q < cols) dst[q] = __float2half_rn(v[q] * a.w_scale_inv_o);
+                }
+              } else {
+                float* dst = static_cast<float*>(a.s) + e * a.nout + col0 + j0;
+                if (cols == 32 && ((a.nout & 3) == 0)) {
+#pragma unroll
+                  for (int q = 0; q < 32; q += 4)
+                    *reinterpret_cast<float4*>(dst + q) =
+                        make_float4(v[q] * a.w_scale_inv_o, v[q + 1] * a.w_scale_inv_o,
+                                    v[q + 2] * a.w_scale_inv_o, v[q + 3] * a.w_scale_inv_o);
+                } else {
+#pragma unroll
+                  for (int q = 0; q < 32; ++q)
+                    if (q < cols) dst[q] = v[q] * a.w_scale_inv_o;
+                }
+              }
+            }
+          }
+        }
+        tc_before();
+        __syncthreads();  // chunk c-1's columns read by every thread before they are reused
+        tc_after();
+      }
+    }
+  }
+  if (!ok && tid == 0) {
+    atomicOr(a.status, 4u);
+    // drain (bounded): copies and MMAs issued but not seen complete
+    for (int b = 0; b < 2; ++b) {
+      if ((pend_w >> b) & 1u) mbar_wait(bar_w + b, (ph_w >> b) & 1u);
+      if ((pend_mma >> b) & 1u) mbar_wait(bar_mma + b, (ph_mma >> b) & 1u);
+    }
+    if (pend_hid) mbar_wait(bar_hid, ph_hid);
+    if (pend_wh) mbar_wait(bar_wh, 0);
+  }
+  tc_before();
+  __syncthreads();
+  tc_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+}
+
+// ---- host: packing of float32 weights into K-major float16 hi / lo operands
+
+// out[r][k] layout of kmajor_off for a [rows x K] operand from w(r, k) (row r = output).
+template <typename F>
+void pack_kmajor(std::vector<unsigned char>& buf, size_t base, int rows, int K, F w) {
+  for (int r = 0; r < rows; ++r)
+    for (int k = 0; k < K; ++k) {
+      const int off = (k >> 4) * rows * 32 + (r >> 3) * 256 + ((k >> 3) & 1) * 128 + (r & 7) * 16 +
+                      (k & 7) * 2;
+      const float v = w(r, k);
+      const __half h = __float2half_rn(v);
+      const __half l = __float2half_rn(v - __half2float(h));
+      std::memcpy(&buf[base + off], &h, 2);
+      std::memcpy(&buf[base + rows * K * 2 + off], &l, 2);
+    }
+}
+
+// power of two 2^s with max |w| 2^s <= 2^14 (so hi parts stay far from float16 overflow and
+// lo parts are normal float16 numbers for the larger weights)
+int weight_scale_exp(const float* w, size_t n) {
+  float m = 0.f;
+  for (size_t q = 0; q < n; ++q) m = std::max(m, std::fabs(w[q]));
+  if (!(m > 0.f)) return 0;
+  int e = 0;
+  std::frexp(m, &e);  // m = f 2^e, f in [0.5, 1)
+  return 14 - e;
+}
+
+}  // namespace
+
+int radial_prepare(RadialPlan& rp, int nb, double r_max, int hidden, int layers, const float* w0,
+                   const float* const* wh, const float* wo, int nout, std::string& err) {
+  if (hidden != 64 && hidden != 32 && hidden != 128) {
+    err = "radial hidden width must be 32, 64 or 128";
+    return E3CONV_ERR_UNSUPPORTED;
+  }
+  if (nb < 1 || nb > kMaxBasis || layers < 1 || layers > 4 || !(r_max > 0) || nout < 1) {
+    err = "radial MLP: 1 <= num_basis <= 16, 1 <= layers <= 4, r_max > 0";
+    return E3CONV_ERR_INVALID_ARG;
+  }
+  rp = RadialPlan{};
+  rp.nb = nb;
+  rp.hidden = hidden;
+  rp.layers = layers;
+  rp.r_max = r_max;
+  rp.nout = nout;
+  rp.chunks = (nout + kChunk - 1) / kChunk;
+  rp.w0.assign(w0, w0 + static_cast<size_t>(nb) * hidden);
+  // hidden weights: one scale for all hidden layers
+  int sh = 30;
+  for (int l = 1; l < layers; ++l)
+    sh = std::min(sh, weight_scale_exp(wh[l - 1], static_cast<size_t>(hidden) * hidden));
+  if (layers == 1) sh = 0;
+  rp.scale_exp_h = sh;
+  const float fh = std::ldexp(1.0f, sh);
+  rp.wh.assign(static_cast<size_t>(layers - 1) * 2 * hidden * hidden * 2, 0);
+  for (int l = 1; l < layers; ++l)
+    pack_kmajor(rp.wh, static_cast<size_t>(l - 1) * 2 * hidden * hidden * 2, hidden, hidden,
+                [&](int r, int k) { return wh[l - 1][static_cast<size_t>(k) * hidden + r] * fh; });
+  const int so = weight_scale_exp(wo, static_cast<size_t>(hidden) * nout);
+  rp.scale_exp_o = so;
+  const float fo = std::ldexp(1.0f, so);
+  const size_t chunk_bytes = static_cast<size_t>(kChunk) * hidden * 2;
+  rp.wo.assign(static_cast<size_t>(rp.chunks) * 2 * chunk_bytes, 0);
+  for (int c = 0; c < rp.chunks; ++c)
+    pack_kmajor(rp.wo, static_cast<size_t>(c) * 2 * chunk_bytes, kChunk, hidden, [&](int r, int k) {
+      const int col = c * kChunk + r;
+      return col < nout ? wo[static_cast<size_t>(k) * nout + col] * fo : 0.f;
+    });
+  return E3CONV_OK;
+}
+
+size_t radial_smem_bytes(const RadialPlan& rp) {
+  const size_t H = rp.hidden;
+  const size_t w0 = (rp.nb * H * 4 + 1023) / 1024 * 1024;
+  return w0 + (rp.layers - 1) * 2 * H * H * 2 + 2 * kTile * H * 2 + 4 * kChunk * H * 2 + 64;
+}
+
+int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, const void* dev_wo,
+                  const float* vec, long long num_edges, void* s, int out_f16, unsigned* status,
+                  int grid, cudaStream_t st, std::string& err) {
+  if (num_edges == 0) return E3CONV_OK;
+  RadialArgs a;
+  a.vec = vec;
+  a.num_edges = num_edges;
+  a.w0 = static_cast<const float*>(dev_w0);
+  a.wh = static_cast<const unsigned char*>(dev_wh);
+  a.wo = static_cast<const unsigned char*>(dev_wo);
+  a.w_scale_inv_h = std::ldexp(1.0f, -rp.scale_exp_h);
+  a.w_scale_inv_o = std::ldexp(1.0f, -rp.scale_exp_o);
+  a.pi_r = static_cast<float>(3.14159265358979323846 / rp.r_max);
+  a.inv_r = static_cast<float>(1.0 / rp.r_max);
+  a.norm = static_cast<float>(std::sqrt(2.0 / rp.r_max));
+  a.nb = rp.nb;
+  a.layers = rp.layers;
+  a.nout = rp.nout;
+  a.chunks = rp.chunks;
+  a.r_max = static_cast<float>(rp.r_max);
+  a.s = s;
+  a.out_f16 = out_f16;
+  a.status = status;
+  const size_t smem = radial_smem_bytes(rp);
+  const long long tiles = (num_edges + kTile - 1) / kTile;
+  const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, grid));
+  cudaError_t e = cudaSuccess;
+  switch (rp.hidden) {
+    case 32:
+      e = cudaFuncSetAttribute(k_radial<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e == cudaSuccess) k_radial<32><<<blocks, 128, smem, st>>>(a);
+      break;
+    case 64:
+      e = cudaFuncSetAttribute(k_radial<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e == cudaSuccess) k_radial<64><<<blocks, 128, smem, st>>>(a);
+      break;
+    default:
+      e = cudaFuncSetAttribute(k_radial<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e == cudaSuccess) k_radial<128><<<blocks, 128, smem, st>>>(a);
+      break;
+  }
+  if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) {
+    err = "radial kernel launch failed";
+    return E3CONV_ERR_CUDA;
+  }
+  return E3CONV_OK;
+}
+
+}  // namespace e3c

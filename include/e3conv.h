@@ -178,6 +178,13 @@ E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane,
  *   above, l <= the plan's lmax; a zero vector gives Y_0 = 1, the rest 0),
  *   in float32, instead of reading ny harmonics per edge. */
 #define E3CONV_OPT_EDGE_VECTORS 4
+/*   E3CONV_OPT_A_LAYOUT: -1 automatic (default), 0, 1 or 2: the shared-memory
+ *   layout of the contract-first A entries where a lane holds channel pairs:
+ *   0 float entries in the order they are formed (a lane duplicates each into
+ *   a pair), 1 the entries stored as (a, a) pairs in that order, 2 (a, a)
+ *   pairs in the order they are applied, read two per 16-byte load.
+ *   Automatic: 1 with one channel pair per lane, else 0.  Same arithmetic. */
+#define E3CONV_OPT_A_LAYOUT 5
 E3CONV_API int e3conv_set_option(e3conv_plan plan, int option, int value);
 
 /* The current value of an option (as set; -1 where automatic). */
@@ -276,6 +283,41 @@ E3CONV_API int e3conv_forward_rows(e3conv_plan plan, const void* node_features, 
                                    const int32_t* senders, const int32_t* receiver_row_ptr,
                                    int64_t row_begin, int64_t row_end, float* out,
                                    e3conv_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * Radial scalars: the edge scalars s_ab as an MLP of radial-basis encodings of
+ * the edge length (e3j "Convolution" docstring: the scalars are an MLP of RBF
+ * encodings; gate_points_2102 page, "Scope": bessel bases, cosine cutoff, and
+ * its number_of_basis / radial_layers / radial_neurons parameters):
+ *   h_0[n] = sqrt(2/r) sin((n+1) pi d / r) / d * (1 + cos(pi d / r)) / 2,
+ *            n < num_basis, d = |r_ab| < r (0 for d >= r; d = 0: the limit)
+ *   h_l    = SiLU(h_{l-1} W_{l-1}),  l = 1 .. layers   (SiLU(v) = v / (1 + e^-v))
+ *   s_ab   = h_layers W_layers, reshaped [P][C]          (no biases)
+ * The hidden layers and the output layer run on the tensor cores (tcgen05,
+ * float16 hi + lo splits of both operands: float32 accuracy); layer 0 on the
+ * CUDA cores.
+ */
+
+/* Sets the plan's radial MLP from HOST float32 weights (row-major, input
+ * index first, as in h W):
+ *   w0       [num_basis][hidden]
+ *   w_hidden [layers-1][hidden][hidden] (NULL when layers == 1)
+ *   w_out    [hidden][P*C], output column p*C + u = path p, channel u.
+ * 1 <= num_basis <= 16, hidden in {32, 64, 128}, 1 <= layers <= 4, r_max > 0.
+ * Packs the weights and copies them to device memory the plan owns (this
+ * call allocates; the radial calls below do not).  Replaces an earlier MLP. */
+E3CONV_API int e3conv_set_radial_mlp(e3conv_plan plan, int num_basis, double r_max, int hidden,
+                                     int layers, const float* w0, const float* w_hidden,
+                                     const float* w_out);
+
+/* edge_scalars[e] = s(r_e) for e < num_edges (device): edge_vectors float32
+ * [num_edges][4] (x, y, z, ignored), edge_scalars [num_edges][P][C] in the
+ * plan's input dtype.  Both 16-byte aligned.  One kernel launch on `stream`
+ * (a persistent grid of one CTA per SM); no allocation, no host
+ * synchronisation.  A timed-out pipeline wait sets the status word
+ * (e3conv_check reports E3CONV_ERR_CUDA). */
+E3CONV_API int e3conv_radial_scalars(e3conv_plan plan, const float* edge_vectors, int64_t num_edges,
+                                     void* edge_scalars, e3conv_stream stream);
 
 /* Partition of the receiver rows into `parts` contiguous CSR row ranges for
  * as many ranks (host only; row_ptr is HOST memory here, int32

@@ -101,8 +101,9 @@ def _emulate_phase1(c, src, Y, expect_entries):
     slots against the dense CG tables; returns the number of entries seen."""
     seen = 0
     for sfx, items in re.findall(r"// A layout(\S*) \(entry: path i k slot\):(.*)", src):
-        m = re.search(r"// A rounds" + re.escape(sfx) + r" \(lanes (\d+), pairs (\d)\):(.*)", src)
-        rw, pairs, terms = int(m.group(1)), int(m.group(2)), [int(v) for v in m.group(3).split()]
+        m = re.search(r"// A rounds" + re.escape(sfx) + r" \(lanes (\d+), mode (\d)\):(.*)", src)
+        rw, mode, terms = int(m.group(1)), int(m.group(2)), [int(v) for v in m.group(3).split()]
+        pairs = mode == 2
         entries = [tuple(int(v) for v in it.split(":")) for it in items.split()]
         tab = re.search(r"e3_atab" + re.escape(sfx) + r"\[\] = \{(.*?)\};", src, re.S).group(1)
         cells = [(int(a), int(b)) for a, b in re.findall(r"\{(-?\d+), (\d+)\}", tab)]
