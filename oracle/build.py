@@ -1,4 +1,5 @@
-"""Builds oracle/liboracle.so from forward.c with gcc and OpenMP (test infrastructure)."""
+"""Builds oracle/liboracle.so from forward.c and backward.c with gcc and OpenMP (test
+infrastructure)."""
 from __future__ import annotations
 
 import os
@@ -8,9 +9,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 
 
 def build(verbose: bool = False) -> str:
-    src = os.path.join(_HERE, "forward.c")
+    srcs = [os.path.join(_HERE, "forward.c"), os.path.join(_HERE, "backward.c")]
     out = os.path.join(_HERE, "liboracle.so")
-    cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp", src, "-o", out + ".tmp"]
+    cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp", *srcs, "-o", out + ".tmp"]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)

@@ -292,6 +292,40 @@ def radial_mlp(d, r_max: float, weights) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Irreps linear layer (cuEquivariance-JAX notes, "Flax NNX layers": channel
+# mixing within matching irreps, scale / sqrt(mul_in), unmatched outputs zero),
+# on the convolution's layout: per node, each irrep block is [2l+1][mul].
+
+
+def irreps_linear(irreps_in: str, irreps_out: str, scale: float, x, weights) -> np.ndarray:
+    """y [N][dim_out] (float64): for each output irrep matching an input irrep (same l and
+    parity), y_o[n, k, v] = scale / sqrt(mul_in) * sum_u x_o[n, k, u] W[u, v], with the next
+    weight block of `weights` (one per matched output irrep, in output order); others 0."""
+    ins, outs = parse_irreps(irreps_in), parse_irreps(irreps_out)
+    x = np.asarray(x, dtype=np.float64)
+    n = x.shape[0]
+    dim_out = sum(ir.dim * ir.mul for ir in outs)
+    y = np.zeros((n, dim_out))
+    w_iter = iter(weights)
+    off_out = 0
+    for ir in outs:
+        off_in = 0
+        match = None
+        for jr in ins:
+            if (jr.l, jr.p) == (ir.l, ir.p):
+                match = (jr, off_in)
+            off_in += jr.dim * jr.mul
+        if match is not None:
+            jr, oi = match
+            W = np.asarray(next(w_iter), dtype=np.float64)
+            xb = x[:, oi:oi + jr.dim * jr.mul].reshape(n, jr.dim, jr.mul)
+            yb = scale / sqrt(jr.mul) * np.einsum("nku,uv->nkv", xb, W)
+            y[:, off_out:off_out + ir.dim * ir.mul] = yb.reshape(n, -1)
+        off_out += ir.dim * ir.mul
+    return y
+
+
+# ---------------------------------------------------------------------------
 # Forward (explicit loops in forward.c)
 
 _lib = None
@@ -311,6 +345,10 @@ def _load():
             [f64p, f64p, f64p, i64p, i64p] + [i32p] * 6 + [f64p, i64p, ctypes.c_double, f64p,
                                                           ctypes.c_int]
         lib.oracle_forward.restype = ctypes.c_int
+        lib.oracle_backward.argtypes = [ctypes.c_int64, ctypes.c_int64] + [ctypes.c_int] * 5 + \
+            [f64p, f64p, f64p, i64p, i64p] + [i32p] * 6 + [f64p, i64p, ctypes.c_double, f64p,
+                                                          f64p, f64p, f64p]
+        lib.oracle_backward.restype = ctypes.c_int
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -351,3 +389,40 @@ def forward(irreps_node: str, irreps_sh: str, irreps_out: str, x, Y, s, senders,
     if rc != 0:
         raise ValueError("oracle_forward: index out of range" if rc == -1 else "oracle_forward failed")
     return out
+
+
+def backward(irreps_node: str, irreps_sh: str, irreps_out: str, x, Y, s, senders, receivers,
+             num_nodes: int, avg_num_neighbors: float, grad_out,
+             normalization: str = "SQRT_DIM_OUT"):
+    """(grad_x [N][nx][C], grad_Y [E][ny], grad_s [E][P][C]) in float64: the gradients of
+    sum(grad_out * forward(...)) with respect to x, Y and s (explicit loops in backward.c)."""
+    pl = plan(irreps_node, irreps_sh, irreps_out)
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    Y = np.ascontiguousarray(np.asarray(Y, dtype=np.float64))
+    s = np.ascontiguousarray(np.asarray(s, dtype=np.float64))
+    g = np.ascontiguousarray(np.asarray(grad_out, dtype=np.float64))
+    senders = np.ascontiguousarray(np.asarray(senders, dtype=np.int64))
+    receivers = np.ascontiguousarray(np.asarray(receivers, dtype=np.int64))
+    E = len(senders)
+    P = len(pl.paths)
+    assert x.shape == (num_nodes, pl.nx, pl.C) and Y.shape == (E, pl.ny)
+    assert s.shape == (E, P, pl.C) and g.shape == (num_nodes, pl.nout, pl.C)
+    cols = {k: np.array([getattr(p, k) for p in pl.paths] or [0], dtype=np.int32)
+            for k in ("l1", "x_off", "l2", "y_off", "l3", "out_off")}
+    cgs = [cg(p.l1, p.l2, p.l3, normalization).ravel() for p in pl.paths]
+    offs = np.zeros(max(1, P), dtype=np.int64)
+    if P:
+        offs[1:P] = np.cumsum([c.size for c in cgs])[:-1]
+    cgcat = np.concatenate(cgs) if cgs else np.zeros(1)
+    gx = np.zeros_like(x)
+    gY = np.zeros_like(Y) if E else np.zeros((1, pl.ny))
+    gs = np.zeros_like(s) if E else np.zeros((1, P, pl.C))
+    rc = _load().oracle_backward(num_nodes, E, pl.C, pl.nx, pl.ny, P, pl.nout, x,
+                                 Y if E else np.zeros((1, pl.ny)), s if E else np.zeros((1, P, pl.C)),
+                                 senders if E else np.zeros(1, np.int64),
+                                 receivers if E else np.zeros(1, np.int64),
+                                 cols["l1"], cols["x_off"], cols["l2"], cols["y_off"], cols["l3"],
+                                 cols["out_off"], cgcat, offs, 1.0 / avg_num_neighbors, g, gx, gY, gs)
+    if rc != 0:
+        raise ValueError("oracle_backward: index out of range")
+    return gx, gY[:E], gs[:E]
