@@ -71,6 +71,13 @@ _partition = _sig("e3conv_partition_rows", ctypes.c_int, _vp, _i64, ctypes.c_int
 _set_radial = _sig("e3conv_set_radial_mlp", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_double,
                    ctypes.c_int, ctypes.c_int, _vp, _vp, _vp)
 _radial_scalars = _sig("e3conv_radial_scalars", ctypes.c_int, _vp, _vp, _i64, _vp, _vp)
+_lin_create = _sig("e3conv_linear_create", ctypes.c_int, ctypes.POINTER(_vp), ctypes.c_char_p,
+                   ctypes.c_char_p, ctypes.c_double)
+_lin_destroy = _sig("e3conv_linear_destroy", None, _vp)
+_lin_query = _sig("e3conv_linear_query", ctypes.c_int, _vp, *([_c_int_p] * 5))
+_lin_set = _sig("e3conv_linear_set_weights", ctypes.c_int, _vp, _vp)
+_lin_forward = _sig("e3conv_linear_forward", ctypes.c_int, _vp, _vp, _i64, _vp, _vp)
+_lin_check = _sig("e3conv_linear_check", ctypes.c_int, _vp, _vp)
 _csr_ws = _sig("e3conv_csr_workspace_size", ctypes.c_int, _i64, _i64,
                ctypes.POINTER(ctypes.c_size_t))
 _build_csr = _sig("e3conv_build_csr", ctypes.c_int, _vp, _i64, _i64, _vp, _vp, _vp,
@@ -88,7 +95,9 @@ EXPORTED = ["e3conv_create", "e3conv_destroy", "e3conv_set_input_dtype",
             "e3conv_spherical_harmonics", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
             "e3conv_output_irrep", "e3conv_cg", "e3conv_kernel_info", "e3conv_kernel_source",
             "e3conv_forward", "e3conv_forward_rows", "e3conv_check", "e3conv_partition_rows",
-            "e3conv_set_radial_mlp", "e3conv_radial_scalars", "e3conv_csr_workspace_size", "e3conv_build_csr",
+            "e3conv_set_radial_mlp", "e3conv_radial_scalars", "e3conv_linear_create",
+            "e3conv_linear_destroy", "e3conv_linear_query", "e3conv_linear_set_weights",
+            "e3conv_linear_forward", "e3conv_linear_check", "e3conv_csr_workspace_size", "e3conv_build_csr",
             "e3conv_csr_check", "e3conv_build_csr_noalloc", "e3conv_csr_kernel_count", "e3conv_permute_rows", "e3conv_strerror", "e3conv_last_error",
             "e3conv_version"]
 
@@ -364,6 +373,54 @@ class Conv:
         if rc == ERR_BAD_INDEX:
             return False
         _ok(rc, "e3conv_check")
+        return True
+
+
+class IrrepsLinear:
+    """Channel mixing within matching irreps on the tensor cores (e3conv_linear_*), on the
+    convolution's feature layout."""
+
+    def __init__(self, irreps_in: str, irreps_out: str, scale: float = 1.0):
+        h = _vp()
+        _ok(_lin_create(ctypes.byref(h), irreps_in.encode(), irreps_out.encode(), float(scale)),
+            "e3conv_linear_create")
+        self._h = h
+        v = [ctypes.c_int() for _ in range(5)]
+        _ok(_lin_query(h, *[ctypes.byref(q) for q in v]), "e3conv_linear_query")
+        self.dim_in, self.dim_out, self.num_weight_blocks, self.mul_in, self.mul_out = \
+            (q.value for q in v)
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h and _lin_destroy is not None:
+            _lin_destroy(h)
+            self._h = None
+
+    def set_weights(self, weights):
+        """weights: num_weight_blocks arrays [mul_in][mul_out] (host), matched irreps in
+        output order."""
+        w = np.ascontiguousarray(np.stack([np.asarray(q, dtype=np.float32) for q in weights])) \
+            if len(weights) else np.zeros(1, np.float32)
+        if len(weights) != self.num_weight_blocks:
+            raise ValueError(f"{self.num_weight_blocks} weight blocks expected")
+        _ok(_lin_set(self._h, w.ctypes.data_as(_vp)), "e3conv_linear_set_weights")
+
+    def __call__(self, x, out=None, stream=None):
+        import torch
+        _require("x", x, dtype=torch.float32)
+        N = x.shape[0]
+        if x.numel() != N * self.dim_in:
+            raise ValueError(f"x must hold {self.dim_in} floats per node")
+        if out is None:
+            out = torch.empty((N, self.dim_out), dtype=torch.float32, device=x.device)
+        else:
+            _require("out", out, x.device, torch.float32, N * self.dim_out)
+        _ok(_lin_forward(self._h, _ptr(x), N, _ptr(out), _stream_handle(stream)),
+            "e3conv_linear_forward")
+        return out
+
+    def check(self, stream=None) -> bool:
+        _ok(_lin_check(self._h, _stream_handle(stream)), "e3conv_linear_check")
         return True
 
 

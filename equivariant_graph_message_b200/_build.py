@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libe3conv.so")
 CUDA_HOME = os.environ.get("CUDA_HOME", "/usr/local/cuda")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-SOURCES = ["api.cpp", "irreps.cpp", "cg.cpp", "sh.cpp", "codegen.cpp", "csr.cu", "radial.cu"]
+SOURCES = ["api.cpp", "irreps.cpp", "cg.cpp", "sh.cpp", "codegen.cpp", "csr.cu", "radial.cu", "linear.cu"]
 
 
 def _nvcc() -> str:
@@ -30,7 +30,8 @@ def _nvcc() -> str:
 
 def sources() -> list[str]:
     return [os.path.join(CSRC, s) for s in SOURCES] + \
-        [os.path.join(CSRC, "plan.h"), os.path.join(CSRC, "exports.map"),
+        [os.path.join(CSRC, "plan.h"), os.path.join(CSRC, "tc_common.cuh"),
+         os.path.join(CSRC, "exports.map"),
          os.path.join(os.path.dirname(PKG), "include", "e3conv.h")]
 
 

@@ -703,6 +703,117 @@ int e3conv_radial_scalars(e3conv_plan h, const float* edge_vectors, int64_t num_
   return rc == E3CONV_OK ? rc : fail(rc, err);
 }
 
+int e3conv_linear_create(e3conv_linear* out, const char* irreps_in, const char* irreps_out,
+                         double scale) {
+  if (!out) return fail(E3CONV_ERR_INVALID_ARG, "linear pointer is NULL");
+  *out = nullptr;
+  if (!std::isfinite(scale)) return fail(E3CONV_ERR_INVALID_ARG, "scale must be finite");
+  std::vector<Irrep> in, o;
+  std::string err;
+  if (!parse_irreps(irreps_in, in, err) || !parse_irreps(irreps_out, o, err))
+    return fail(E3CONV_ERR_IRREPS, err);
+  e3conv_linear h = new (std::nothrow) e3conv_linear_s;
+  if (!h) return fail(E3CONV_ERR_NOMEM, "host allocation failed");
+  const int rc = linear_prepare(h->p, in, o, scale, err);
+  if (rc != E3CONV_OK) {
+    delete h;
+    return fail(rc, err);
+  }
+  if (has_device()) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaMalloc(&h->p.status, sizeof(unsigned)) != cudaSuccess) {
+      cudaGetLastError();
+      delete h;
+      return fail(E3CONV_ERR_NOMEM, "cudaMalloc of the status word failed");
+    }
+    cudaMemset(h->p.status, 0, sizeof(unsigned));
+    h->p.device = dev;
+  }
+  *out = h;
+  return E3CONV_OK;
+}
+
+void e3conv_linear_destroy(e3conv_linear h) {
+  if (!h) return;
+  {
+    DeviceGuard g(h->p.device);
+    if (h->p.d_w) cudaFree(h->p.d_w);
+    if (h->p.status) cudaFree(h->p.status);
+  }
+  delete h;
+}
+
+int e3conv_linear_query(e3conv_linear h, int* dim_in, int* dim_out, int* num_weight_blocks,
+                        int* mul_in, int* mul_out) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "linear is NULL");
+  if (dim_in) *dim_in = h->p.dim_in;
+  if (dim_out) *dim_out = h->p.dim_out;
+  if (num_weight_blocks) *num_weight_blocks = h->p.num_weight_blocks;
+  if (mul_in) *mul_in = h->p.K;
+  if (mul_out) *mul_out = h->p.N;
+  return E3CONV_OK;
+}
+
+int e3conv_linear_set_weights(e3conv_linear h, const float* w) {
+  if (!h || (!w && h->p.num_weight_blocks > 0)) return fail(E3CONV_ERR_INVALID_ARG, "NULL argument");
+  LinearPlan& lp = h->p;
+  std::string err;
+  int rc = linear_pack(lp, w, err);
+  if (rc != E3CONV_OK) return fail(rc, err);
+  if (lp.device >= 0 && !lp.packed.empty()) {
+    DeviceGuard g(lp.device);
+    if (!lp.d_w && cudaMalloc(&lp.d_w, lp.packed.size()) != cudaSuccess) {
+      cudaGetLastError();
+      lp.d_w = nullptr;
+      return fail(E3CONV_ERR_NOMEM, "cudaMalloc of the packed weights failed");
+    }
+    if (cudaMemcpy(lp.d_w, lp.packed.data(), lp.packed.size(), cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(E3CONV_ERR_CUDA, "copying the packed weights failed");
+    }
+  }
+  lp.weights_set = true;
+  return E3CONV_OK;
+}
+
+int e3conv_linear_forward(e3conv_linear h, const float* x, int64_t num_nodes, float* y,
+                          e3conv_stream stream) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "linear is NULL");
+  LinearPlan& lp = h->p;
+  if (num_nodes < 0 || num_nodes >= (1ll << 31))
+    return fail(E3CONV_ERR_INVALID_ARG, "num_nodes out of range");
+  if (num_nodes == 0) return E3CONV_OK;
+  if (!lp.weights_set) return fail(E3CONV_ERR_INVALID_ARG, "weights not set (e3conv_linear_set_weights)");
+  if (!x || !y) return fail(E3CONV_ERR_INVALID_ARG, "NULL buffer");
+  if (!aligned16(x) || !aligned16(y)) return fail(E3CONV_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
+  if (lp.device < 0) return fail(E3CONV_ERR_NO_DEVICE, "no CUDA device");
+  int cur = -1, sms = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess || cur != lp.device)
+    return fail(E3CONV_ERR_INVALID_ARG, "current device differs from the linear layer's device");
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, lp.device) != cudaSuccess)
+    return fail(E3CONV_ERR_CUDA, "cannot query the SM count");
+  std::string err;
+  const int rc = linear_launch(lp, lp.d_w, x, num_nodes, y, lp.status, sms,
+                               reinterpret_cast<cudaStream_t>(stream), err);
+  return rc == E3CONV_OK ? rc : fail(rc, err);
+}
+
+int e3conv_linear_check(e3conv_linear h, e3conv_stream stream) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "linear is NULL");
+  if (h->p.device < 0) return fail(E3CONV_ERR_NO_DEVICE, "no device");
+  unsigned st = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&st, h->p.status, sizeof st, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return fail(E3CONV_ERR_CUDA, "reading the status word failed");
+  if (st) {
+    cudaMemsetAsync(h->p.status, 0, sizeof st, s);
+    cudaStreamSynchronize(s);
+    return fail(E3CONV_ERR_CUDA, "a pipeline wait of the linear layer timed out");
+  }
+  return E3CONV_OK;
+}
+
 int e3conv_partition_rows(const int32_t* row_ptr, int64_t num_nodes, int parts, int64_t* bounds) {
   if (!row_ptr || !bounds) return fail(E3CONV_ERR_INVALID_ARG, "row_ptr and bounds are required");
   if (parts < 1) return fail(E3CONV_ERR_INVALID_ARG, "parts must be at least 1");

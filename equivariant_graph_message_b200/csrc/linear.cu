@@ -1,0 +1,353 @@
+// Irreps linear layer on the tensor cores: channel mixing within matching
+// irreps (cuEquivariance-JAX notes, "Flax NNX layers": IrrepsLinear mixes the
+// channels of matching irreps with scale / sqrt(mul_in) normalisation;
+// unmatched outputs are zero):
+//   y[n, o, k, v] = scale / sqrt(mul_in(o)) * sum_u x[n, o, k, u] W_o[u, v]
+// for every output irrep o that also appears among the input irreps, and 0
+// for the others.  Features use the convolution's trailing-channel layout:
+// per node, each irrep block is [2l+1][mul] (components outer, channels
+// inner).
+//
+// Per matched irrep the rows (n, k) form a GEMM [N (2l+1) x mul_in] x
+// [mul_in x mul_out].  One CTA of 128 threads per contiguous range of
+// 128-row tiles: thread t loads row t of the tile (mul_in float32 values),
+// splits it into float16 hi + lo parts in shared memory (A, K-major), the
+// weights W_o^T (B, K-major, prepacked hi / lo, scaled by a power of two)
+// are bulk-copied in when the irrep changes, D = A_hi B_hi + A_hi B_lo +
+// A_lo B_hi accumulates in tensor memory (float32), and thread t stores its
+// row of D.  The next tile's rows are loaded while the MMAs run.  All waits
+// are bounded (timeout: status bit 4, drain, stop).
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <string>
+#include <vector>
+
+#include "plan.h"
+#include "tc_common.cuh"
+
+namespace e3c {
+
+namespace {
+
+using namespace tc;
+using namespace tc_host;
+
+constexpr int kTile = 128;
+
+struct LinArgs {
+  const float* x;
+  float* y;
+  const unsigned char* w;   // packed hi / lo operands of the matched irreps
+  long long nodes;
+  int dim_in, dim_out, n_out;  // row lengths; mul_out (MMA N)
+  int nblocks;                 // output irrep blocks
+  int tiles_total;
+  unsigned* status;
+  LinBlock blk[kLinMaxBlocks];
+};
+
+template <int K>
+__global__ void __launch_bounds__(128, 1) k_linear(LinArgs a) {
+  extern __shared__ __align__(1024) unsigned char sm[];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int N = a.n_out;
+  unsigned char* bw = sm;                                   // hi then lo, [N x K] each
+  unsigned char* act = sm + 2 * N * K * 2;                  // hi then lo, [128 x K] each
+  unsigned long long* bars = reinterpret_cast<unsigned long long*>(act + 2 * kTile * K * 2);
+  unsigned long long* bar_w = bars;
+  unsigned long long* bar_mma = bars + 1;
+  unsigned* tslot = reinterpret_cast<unsigned*>(bars + 2);
+  if (tid == 0) {
+    mbar_init(bar_w, 1);
+    mbar_init(bar_mma, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+                     smem_u32(tslot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_before();
+  __syncthreads();
+  tc_after();
+  const unsigned tmem = *tslot;
+  const unsigned lane_off = static_cast<unsigned>(32 * warp) << 16;
+  // contiguous tile range of this CTA
+  const long long per = (a.tiles_total + gridDim.x - 1) / gridDim.x;
+  const long long t0 = blockIdx.x * per;
+  const long long t1 = (t0 + per < a.tiles_total) ? t0 + per : static_cast<long long>(a.tiles_total);
+  bool ok = true;
+  unsigned ph_w = 0, ph_mma = 0;
+  bool pend_w = false, pend_mma = false;
+  int cur = -1;  // block whose weights are in shared memory
+  // where tile t's row of this thread lives
+  auto locate = [&](long long t, int& b, const float*& src, float*& dst) {
+    b = 0;
+    while (b + 1 < a.nblocks && t >= a.blk[b + 1].first_tile) ++b;
+    const LinBlock& B = a.blk[b];
+    const long long r = (t - B.first_tile) * kTile + tid;
+    src = nullptr;
+    dst = nullptr;
+    if (r < a.nodes * B.dim) {
+      const long long n = r / B.dim, k = r - n * B.dim;
+      dst = a.y + n * a.dim_out + B.out_off + k * N;
+      if (B.w_off >= 0) src = a.x + n * a.dim_in + B.in_off + k * K;
+    }
+  };
+  float R[K];
+  auto load = [&](const float* src) {
+#pragma unroll
+    for (int q = 0; q < K; q += 4) {
+      const float4 v = src ? __ldg(reinterpret_cast<const float4*>(src + q)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      R[q] = v.x;
+      R[q + 1] = v.y;
+      R[q + 2] = v.z;
+      R[q + 3] = v.w;
+    }
+  };
+  int b;
+  const float* src;
+  float* dst;
+  if (t0 < t1) {
+    locate(t0, b, src, dst);
+    load(src);
+  }
+  for (long long t = t0; t < t1 && ok; ++t) {
+    locate(t, b, src, dst);
+    const LinBlock& B = a.blk[b];
+    if (B.w_off < 0) {  // output irrep without a matching input irrep: zeros
+      if (dst)
+        for (int q = 0; q < N; q += 4) *reinterpret_cast<float4*>(dst + q) = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t + 1 < t1) {
+        int b2;
+        const float* s2;
+        float* d2;
+        locate(t + 1, b2, s2, d2);
+        load(s2);
+      }
+      continue;
+    }
+    if (b != cur) {  // this irrep's weights
+      __syncthreads();
+      if (tid == 0) {
+        const unsigned bytes = static_cast<unsigned>(2 * N * K * 2);
+        mbar_expect(bar_w, bytes);
+        bulk_g2s(bw, a.w + B.w_off, bytes, bar_w);
+        pend_w = true;
+      }
+      ok = __syncthreads_and(mbar_wait(bar_w, ph_w));
+      if (!ok) break;
+      ph_w ^= 1u;
+      pend_w = false;
+      cur = b;
+    }
+    store_split_row<K>(act, act + kTile * K * 2, tid, R, kTile);
+    fence_async_smem();
+    tc_before();
+    __syncthreads();
+    tc_after();
+    if (tid == 0) {
+      const unsigned id = idesc_f16(kTile, N);
+      const unsigned char* whi = bw;
+      const unsigned char* wlo = bw + N * K * 2;
+      for (int ks = 0; ks < K / 16; ++ks) {
+        const int ao = ks * kTile * 32, bo = ks * N * 32;
+        mma_f16(tmem, kmajor_desc(act + ao), kmajor_desc(whi + bo), id, ks > 0);
+        mma_f16(tmem, kmajor_desc(act + ao), kmajor_desc(wlo + bo), id, 1);
+        mma_f16(tmem, kmajor_desc(act + kTile * K * 2 + ao), kmajor_desc(whi + bo), id, 1);
+      }
+      mma_commit(bar_mma);
+      pend_mma = true;
+    }
+    if (t + 1 < t1) {  // the next tile's row, while the MMAs run
+      int b2;
+      const float* s2;
+      float* d2;
+      locate(t + 1, b2, s2, d2);
+      load(s2);
+    }
+    ok = __syncthreads_and(mbar_wait(bar_mma, ph_mma));
+    tc_after();
+    if (!ok) break;
+    ph_mma ^= 1u;
+    pend_mma = false;
+    for (int j0 = 0; j0 < N; j0 += 32) {
+      float v[32];
+      tmem_ld32(tmem + lane_off + j0, v);
+      if (dst) {
+        const int cols = min(32, N - j0);
+#pragma unroll
+        for (int q = 0; q < 32; q += 4)
+          if (q < cols)
+            *reinterpret_cast<float4*>(dst + j0 + q) =
+                make_float4(v[q] * B.scale, v[q + 1] * B.scale, v[q + 2] * B.scale, v[q + 3] * B.scale);
+      }
+    }
+    tc_before();
+    __syncthreads();  // every row read out of tensor memory before the next MMAs
+    tc_after();
+  }
+  if (!ok && tid == 0) {
+    atomicOr(a.status, 4u);
+    if (pend_w) mbar_wait(bar_w, ph_w);
+    if (pend_mma) mbar_wait(bar_mma, ph_mma);
+  }
+  tc_before();
+  __syncthreads();
+  tc_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+}
+
+}  // namespace
+
+int linear_prepare(LinearPlan& lp, const std::vector<Irrep>& in, const std::vector<Irrep>& out,
+                   double scale, std::string& err) {
+  lp = LinearPlan{};
+  if (in.empty() || out.empty()) {
+    err = "irreps_in and irreps_out must not be empty";
+    return E3CONV_ERR_IRREPS;
+  }
+  const int K = in[0].mul, N = out[0].mul;
+  for (const auto& ir : in)
+    if (ir.mul != K) {
+      err = "all input multiplicities must be equal";
+      return E3CONV_ERR_UNSUPPORTED;
+    }
+  for (const auto& ir : out)
+    if (ir.mul != N) {
+      err = "all output multiplicities must be equal";
+      return E3CONV_ERR_UNSUPPORTED;
+    }
+  if (K != 32 && K != 64 && K != 128) {
+    err = "input multiplicity must be 32, 64 or 128";
+    return E3CONV_ERR_UNSUPPORTED;
+  }
+  if (N < 16 || N > 256 || N % 16) {
+    err = "output multiplicity must be a multiple of 16 in [16, 256]";
+    return E3CONV_ERR_UNSUPPORTED;
+  }
+  if (static_cast<int>(out.size()) > kLinMaxBlocks) {
+    err = "too many output irreps";
+    return E3CONV_ERR_UNSUPPORTED;
+  }
+  for (size_t q = 0; q < in.size(); ++q)
+    for (size_t r = q + 1; r < in.size(); ++r)
+      if (in[q].l == in[r].l && in[q].p == in[r].p) {
+        err = "input irreps must be regrouped (each (l, parity) once)";
+        return E3CONV_ERR_IRREPS;
+      }
+  for (size_t q = 0; q < out.size(); ++q)
+    for (size_t r = q + 1; r < out.size(); ++r)
+      if (out[q].l == out[r].l && out[q].p == out[r].p) {
+        err = "output irreps must be regrouped (each (l, parity) once)";
+        return E3CONV_ERR_IRREPS;
+      }
+  lp.in = in;
+  lp.out = out;
+  lp.K = K;
+  lp.N = N;
+  lp.scale = scale;
+  int off = 0;
+  for (const auto& ir : in) off += ir.dim() * ir.mul;
+  lp.dim_in = off;
+  off = 0;
+  for (const auto& ir : out) {
+    LinBlock b{};
+    b.dim = ir.dim();
+    b.out_off = off;
+    b.in_off = -1;
+    b.w_off = -1;
+    int ioff = 0;
+    for (const auto& jr : in) {
+      if (jr.l == ir.l && jr.p == ir.p) {
+        b.in_off = ioff;
+        b.w_off = lp.num_weight_blocks++;  // packed offset fixed once weights are set
+      }
+      ioff += jr.dim() * jr.mul;
+    }
+    off += ir.dim() * ir.mul;
+    lp.blocks.push_back(b);
+  }
+  lp.dim_out = off;
+  return E3CONV_OK;
+}
+
+int linear_pack(LinearPlan& lp, const float* w, std::string& err) {
+  const int K = lp.K, N = lp.N;
+  const size_t per = static_cast<size_t>(K) * N;
+  const int s = weight_scale_exp(w, per * lp.num_weight_blocks);
+  const float f = std::ldexp(1.0f, s);
+  const size_t bytes = 2 * static_cast<size_t>(N) * K * 2;
+  lp.packed.assign(bytes * lp.num_weight_blocks, 0);
+  for (auto& b : lp.blocks) {
+    if (b.w_off < 0) continue;
+    const float* wb = w + per * static_cast<size_t>(b.w_off);
+    pack_kmajor(lp.packed, bytes * static_cast<size_t>(b.w_off), N, K,
+                [&](int r, int k) { return wb[static_cast<size_t>(k) * N + r] * f; });
+    b.scale = static_cast<float>(lp.scale / std::sqrt(static_cast<double>(K)) * std::ldexp(1.0, -s));
+  }
+  lp.scale_exp = s;
+  (void)err;
+  return E3CONV_OK;
+}
+
+size_t linear_smem_bytes(const LinearPlan& lp) {
+  return 2 * static_cast<size_t>(lp.N) * lp.K * 2 + 2 * static_cast<size_t>(kTile) * lp.K * 2 + 64;
+}
+
+int linear_launch(const LinearPlan& lp, const void* dev_w, const float* x, long long nodes, float* y,
+                  unsigned* status, int grid, cudaStream_t st, std::string& err) {
+  if (nodes == 0) return E3CONV_OK;
+  LinArgs a{};
+  a.x = x;
+  a.y = y;
+  a.w = static_cast<const unsigned char*>(dev_w);
+  a.nodes = nodes;
+  a.dim_in = lp.dim_in;
+  a.dim_out = lp.dim_out;
+  a.n_out = lp.N;
+  a.nblocks = static_cast<int>(lp.blocks.size());
+  a.status = status;
+  long long tiles = 0;
+  const size_t wbytes = 2 * static_cast<size_t>(lp.N) * lp.K * 2;
+  for (size_t q = 0; q < lp.blocks.size(); ++q) {
+    LinBlock b = lp.blocks[q];
+    b.first_tile = static_cast<int>(tiles);
+    if (b.w_off >= 0) b.w_off = static_cast<long long>(wbytes) * b.w_off;
+    a.blk[q] = b;
+    tiles += (nodes * b.dim + kTile - 1) / kTile;
+  }
+  if (tiles >= (1ll << 31)) {
+    err = "too many rows";
+    return E3CONV_ERR_UNSUPPORTED;
+  }
+  a.tiles_total = static_cast<int>(tiles);
+  const size_t smem = linear_smem_bytes(lp);
+  const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, grid));
+  cudaError_t e = cudaSuccess;
+  switch (lp.K) {
+    case 32:
+      e = cudaFuncSetAttribute(k_linear<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e == cudaSuccess) k_linear<32><<<blocks, 128, smem, st>>>(a);
+      break;
+    case 64:
+      e = cudaFuncSetAttribute(k_linear<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e == cudaSuccess) k_linear<64><<<blocks, 128, smem, st>>>(a);
+      break;
+    default:
+      e = cudaFuncSetAttribute(k_linear<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e == cudaSuccess) k_linear<128><<<blocks, 128, smem, st>>>(a);
+      break;
+  }
+  if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) {
+    err = "irreps linear kernel launch failed";
+    return E3CONV_ERR_CUDA;
+  }
+  return E3CONV_OK;
+}
+
+}  // namespace e3c

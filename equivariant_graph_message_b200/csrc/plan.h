@@ -114,6 +114,33 @@ struct RadialPlan {
   void* d_wo = nullptr;
 };
 
+// Irreps linear layer (e3conv_linear_*): per output irrep block, where its rows
+// come from and which packed weights mix them.
+constexpr int kLinMaxBlocks = 16;
+struct LinBlock {
+  int dim;          // 2l+1
+  int in_off;       // first input element of the matching input irrep (-1: none)
+  int out_off;      // first output element of the irrep
+  int first_tile;   // first 128-row tile of the irrep (set per launch)
+  long long w_off;  // matched weight block (prepare) / its byte offset (launch); -1: zeros
+  float scale;      // scale / sqrt(mul_in) / 2^s
+};
+
+struct LinearPlan {
+  std::vector<Irrep> in, out;
+  int K = 0, N = 0;                 // mul_in, mul_out
+  int dim_in = 0, dim_out = 0;      // floats per node row
+  double scale = 1.0;
+  int num_weight_blocks = 0;        // matched irreps, in output order
+  std::vector<LinBlock> blocks;     // one per output irrep
+  std::vector<unsigned char> packed;
+  int scale_exp = 0;
+  bool weights_set = false;
+  int device = -1;
+  void* d_w = nullptr;
+  unsigned* status = nullptr;
+};
+
 struct Plan {
   int C = 0, nx = 0, ny = 0, nout = 0, lmax = 0;
   std::vector<Irrep> node, filt;
@@ -156,6 +183,14 @@ int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, 
                   const float* vec, long long num_edges, void* s, int out_f16, unsigned* status,
                   int grid, cudaStream_t st, std::string& err);
 
+// linear.cu
+int linear_prepare(LinearPlan& lp, const std::vector<Irrep>& in, const std::vector<Irrep>& out,
+                   double scale, std::string& err);
+int linear_pack(LinearPlan& lp, const float* w, std::string& err);
+size_t linear_smem_bytes(const LinearPlan& lp);
+int linear_launch(const LinearPlan& lp, const void* dev_w, const float* x, long long nodes, float* y,
+                  unsigned* status, int grid, cudaStream_t st, std::string& err);
+
 // codegen.cpp
 std::vector<AEntry> build_a_entries(const Plan& plan);
 Shape choose_shape(const Plan& plan, int dtype);
@@ -165,4 +200,8 @@ std::string generate_forward_source(const Plan& plan, int dtype, const Shape& sh
 
 struct e3conv_plan_s {
   e3c::Plan p;
+};
+
+struct e3conv_linear_s {
+  e3c::LinearPlan p;
 };

@@ -1,0 +1,168 @@
+// Device and host helpers shared by the tensor-core GEMM kernels (radial MLP,
+// irreps linear): mbarrier waits with an iteration bound, bulk copies,
+// tcgen05 MMA issue / commit / tensor-memory loads, K-major no-swizzle
+// shared-memory operands of float16 hi + lo parts.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+namespace e3c {
+namespace tc {
+
+constexpr unsigned kSpinLimit = 1u << 22;
+
+__device__ __forceinline__ unsigned smem_u32(const void* p) {
+  return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(unsigned long long* b, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect(unsigned long long* b, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(unsigned long long* b, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait(unsigned long long* b, unsigned parity) {
+  for (unsigned it = 0; it < kSpinLimit; ++it)
+    if (mbar_try(b, parity)) return true;
+  return false;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes,
+                                         unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// K-major, no-swizzle shared-memory matrix descriptor: core matrices of 8 rows x
+// 16 bytes; 128 bytes between the two K-adjacent core matrices of a 16-wide K
+// slab, 256 bytes between row groups of 8.
+__device__ __forceinline__ unsigned long long kmajor_desc(const void* p) {
+  return static_cast<unsigned long long>((smem_u32(p) & 0x3FFFF) >> 4) | (8ull << 16) |
+         (16ull << 32) | (1ull << 46);
+}
+// byte offset of element (row r, k) in a K-major operand of `rows` rows: K slab
+// k / 16 of rows * 32 bytes, then the core-matrix layout inside the slab
+__device__ __forceinline__ int kmajor_off(int r, int k, int rows) {
+  return (k >> 4) * rows * 32 + (r >> 3) * 256 + ((k >> 3) & 1) * 128 + (r & 7) * 16 + (k & 7) * 2;
+}
+// instruction descriptor of kind::f16: float16 A and B (both K-major), float32 D
+__device__ __forceinline__ unsigned idesc_f16(int m, int n) {
+  return (1u << 4) | (static_cast<unsigned>(n >> 3) << 17) | (static_cast<unsigned>(m >> 4) << 24);
+}
+__device__ __forceinline__ void mma_f16(unsigned tmem_d, unsigned long long a, unsigned long long b,
+                                        unsigned idesc, unsigned accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(
+          tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(unsigned long long* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(unsigned addr, float* v) {
+  unsigned r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(addr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(r[q]);
+}
+
+__device__ __forceinline__ float silu(float v) { return v / (1.0f + expf(-v)); }
+
+// two floats rounded to float16, low half first
+__device__ __forceinline__ unsigned pack_half2(float lo, float hi) {
+  unsigned r;
+  asm("{ .reg .f16 a, b; cvt.rn.f16.f32 a, %1; cvt.rn.f16.f32 b, %2; mov.b32 %0, {a, b}; }"
+      : "=r"(r)
+      : "f"(lo), "f"(hi));
+  return r;
+}
+
+// Writes row r's values v[0..K) of a K-major operand as float16 hi and lo parts.
+template <int K>
+__device__ __forceinline__ void store_split_row(unsigned char* hi, unsigned char* lo, int r,
+                                                const float* v, int rows) {
+#pragma unroll
+  for (int k = 0; k < K; k += 2) {
+    const __half h0 = __float2half_rn(v[k]), h1 = __float2half_rn(v[k + 1]);
+    const __half l0 = __float2half_rn(v[k] - __half2float(h0));
+    const __half l1 = __float2half_rn(v[k + 1] - __half2float(h1));
+    const int off = kmajor_off(r, k, rows);
+    *reinterpret_cast<__half2*>(hi + off) = __halves2half2(h0, h1);
+    *reinterpret_cast<__half2*>(lo + off) = __halves2half2(l0, l1);
+  }
+}
+
+
+}  // namespace tc
+
+namespace tc_host {
+
+// ---- host: packing of float32 weights into K-major float16 hi / lo operands
+
+// out[r][k] layout of kmajor_off for a [rows x K] operand from w(r, k) (row r = output).
+template <typename F>
+inline void pack_kmajor(std::vector<unsigned char>& buf, size_t base, int rows, int K, F w) {
+  for (int r = 0; r < rows; ++r)
+    for (int k = 0; k < K; ++k) {
+      const int off = (k >> 4) * rows * 32 + (r >> 3) * 256 + ((k >> 3) & 1) * 128 + (r & 7) * 16 +
+                      (k & 7) * 2;
+      const float v = w(r, k);
+      const __half h = __float2half_rn(v);
+      const __half l = __float2half_rn(v - __half2float(h));
+      std::memcpy(&buf[base + off], &h, 2);
+      std::memcpy(&buf[base + rows * K * 2 + off], &l, 2);
+    }
+}
+
+// power of two 2^s with max |w| 2^s <= 2^14 (so hi parts stay far from float16 overflow and
+// lo parts are normal float16 numbers for the larger weights)
+inline int weight_scale_exp(const float* w, size_t n) {
+  float m = 0.f;
+  for (size_t q = 0; q < n; ++q) m = std::max(m, std::fabs(w[q]));
+  if (!(m > 0.f)) return 0;
+  int e = 0;
+  std::frexp(m, &e);  // m = f 2^e, f in [0.5, 1)
+  return 14 - e;
+}
+
+
+}  // namespace tc_host
+}  // namespace e3c

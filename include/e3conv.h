@@ -75,6 +75,7 @@ extern "C" {
 #endif
 
 typedef struct e3conv_plan_s* e3conv_plan;
+typedef struct e3conv_linear_s* e3conv_linear;
 typedef struct CUstream_st* e3conv_stream;
 
 /* error codes */
@@ -318,6 +319,46 @@ E3CONV_API int e3conv_set_radial_mlp(e3conv_plan plan, int num_basis, double r_m
  * (e3conv_check reports E3CONV_ERR_CUDA). */
 E3CONV_API int e3conv_radial_scalars(e3conv_plan plan, const float* edge_vectors, int64_t num_edges,
                                      void* edge_scalars, e3conv_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * Irreps linear layer (cuEquivariance-JAX notes, "Flax NNX layers":
+ * IrrepsLinear mixes the channels of matching irreps with
+ * scale / sqrt(mul_in) normalisation; unmatched outputs are zero), the layer
+ * that follows the convolution on its output:
+ *   y[n, o, k, v] = scale / sqrt(mul_in) * sum_u x[n, o, k, u] W_o[u, v]
+ * for each output irrep o = (l, p) also among the input irreps; 0 for the
+ * others.  Both feature arrays use the convolution's layout: per node, each
+ * irrep block is [2l+1][mul] (components outer, channels inner).  A GEMM per
+ * matched irrep on the tensor cores (tcgen05, float16 hi + lo splits of both
+ * operands: float32 accuracy).
+ */
+
+/* irreps_in / irreps_out: regrouped (each (l, parity) once), one multiplicity
+ * each: mul_in in {32, 64, 128}, mul_out a multiple of 16 in [16, 256], at
+ * most 16 output irreps.  scale finite.  Allocates a 4-byte device status word
+ * when a device is present. */
+E3CONV_API int e3conv_linear_create(e3conv_linear* linear, const char* irreps_in,
+                                    const char* irreps_out, double scale);
+E3CONV_API void e3conv_linear_destroy(e3conv_linear linear);
+
+/* Floats per node row of x and y, matched irreps (weight blocks), mul_in, mul_out. */
+E3CONV_API int e3conv_linear_query(e3conv_linear linear, int* dim_in, int* dim_out,
+                                   int* num_weight_blocks, int* mul_in, int* mul_out);
+
+/* HOST float32 weights [num_weight_blocks][mul_in][mul_out], one block per
+ * matched output irrep in output order.  Packs and copies them to device
+ * memory the layer owns (this call allocates). */
+E3CONV_API int e3conv_linear_set_weights(e3conv_linear linear, const float* w);
+
+/* y [num_nodes][dim_out] from x [num_nodes][dim_in] (device float32, 16-byte
+ * aligned).  One kernel launch on `stream`; no allocation, no host
+ * synchronisation. */
+E3CONV_API int e3conv_linear_forward(e3conv_linear linear, const float* x, int64_t num_nodes,
+                                     float* y, e3conv_stream stream);
+
+/* Synchronises `stream`, reads and clears the layer's status word:
+ * E3CONV_ERR_CUDA if a pipeline wait timed out. */
+E3CONV_API int e3conv_linear_check(e3conv_linear linear, e3conv_stream stream);
 
 /* Partition of the receiver rows into `parts` contiguous CSR row ranges for
  * as many ranks (host only; row_ptr is HOST memory here, int32

@@ -1,0 +1,60 @@
+"""GPU parity of the irreps linear layer on the tensor cores (e3conv_linear_*)
+against the oracle's float64 layer: the convolution's output irreps mixed into
+other multiplicities, unmatched output irreps, ragged row tiles, few nodes, and
+the convolution's full-size output of the large mixed-precision workload."""
+import numpy as np
+import pytest
+import torch
+
+import equivariant_graph_message_b200 as e3
+import oracle
+from parity import to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("ins,outs", [
+    ("128x0e+128x1o+128x2e+128x3o", "64x0e+64x1o+64x2e+64x3o"),
+    ("64x0e+64x1o+64x2e", "128x0e+128x1e+128x1o+128x2e+128x3o"),     # unmatched 1e, 3o
+    ("32x0e+32x1o", "256x1o+256x0e"),
+    ("128x0e+128x1o+128x2e+128x3o", "16x3o+16x0e"),
+])
+@pytest.mark.parametrize("nodes", [1, 5, 300, 2049])
+def test_linear_matches_the_oracle(cuda_device, ins, outs, nodes):
+    lin = e3.IrrepsLinear(ins, outs, 0.7)
+    rng = np.random.default_rng(nodes + len(ins))
+    ws = [rng.normal(size=(lin.mul_in, lin.mul_out)).astype(np.float32)
+          for _ in range(lin.num_weight_blocks)]
+    lin.set_weights(ws)
+    x = rng.normal(size=(nodes, lin.dim_in)).astype(np.float32)
+    y = torch.full((nodes, lin.dim_out), float("nan"), device="cuda")
+    lin(to_dev(x), out=y)
+    torch.cuda.synchronize()
+    assert lin.check()
+    ref = oracle.irreps_linear(ins, outs, 0.7, x, ws)
+    got = y.cpu().numpy()
+    scale = np.abs(ref).max(axis=0)
+    scale[scale == 0] = 1
+    assert (np.abs(got - ref) / scale).max() <= 1e-5
+    assert not np.isnan(got).any()
+
+
+def test_linear_on_the_convolution_output_full_size(cuda_device):
+    from parity import DeviceWorkload
+    w = DeviceWorkload("large_f16")
+    out = w.conv.forward(w.x, w.Y, w.s, w.senders, w.row_ptr)
+    conv_irreps = "+".join(f"128x{l}{'e' if p > 0 else 'o'}" for l, p, _ in w.conv.outputs)
+    lin = e3.IrrepsLinear(conv_irreps, conv_irreps, 1.0)
+    rng = np.random.default_rng(5)
+    ws = [rng.normal(size=(128, 128)).astype(np.float32) for _ in range(lin.num_weight_blocks)]
+    lin.set_weights(ws)
+    y = lin(out.view(w.N, -1))
+    torch.cuda.synchronize()
+    assert lin.check()
+    rows = np.unique(np.concatenate([[0, w.N - 1], rng.choice(w.N, 512, replace=False)]))
+    xr = out.view(w.N, -1)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    ref = oracle.irreps_linear(conv_irreps, conv_irreps, 1.0, xr, ws)
+    got = y[torch.from_numpy(rows).cuda()].cpu().numpy()
+    assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
+    del w, out, y
+    torch.cuda.empty_cache()

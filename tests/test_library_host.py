@@ -411,3 +411,18 @@ def test_path_split_tables_cover_every_entry_once(split):
     assert len(owned) == split
     assert set().union(*owned) == set(range(c.num_paths))
     assert sum(len(o) for o in owned) == c.num_paths          # each path in one warp
+
+
+def test_linear_layer_host_validation():
+    with pytest.raises(e3.E3ConvError):
+        e3.IrrepsLinear("48x0e", "64x0e")                 # mul_in not 32, 64 or 128
+    with pytest.raises(e3.E3ConvError):
+        e3.IrrepsLinear("64x0e", "20x0e")                 # mul_out not a multiple of 16
+    with pytest.raises(e3.E3ConvError):
+        e3.IrrepsLinear("64x0e+64x0e", "64x0e")           # not regrouped
+    with pytest.raises(e3.E3ConvError):
+        e3.IrrepsLinear("64x0e+32x1o", "64x0e")           # unequal input multiplicities
+    lin = e3.IrrepsLinear("64x0e+64x1o+64x2e", "32x2e+32x3o+32x0e")
+    assert (lin.dim_in, lin.dim_out, lin.num_weight_blocks) == (64 * 9, 32 * 13, 2)
+    with pytest.raises(ValueError):
+        lin.set_weights([np.zeros((64, 32))])            # two matched irreps need two blocks
