@@ -67,6 +67,11 @@ _forward = _sig("e3conv_forward", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i
 _forward_rows = _sig("e3conv_forward_rows", ctypes.c_int, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
                      _i64, _i64, _vp, _vp)
 _check = _sig("e3conv_check", ctypes.c_int, _vp, _vp)
+_backward = _sig("e3conv_backward", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                 _i64, _vp, _vp, _vp, _vp, _vp)
+_prepare_backward = _sig("e3conv_prepare_backward", ctypes.c_int, _vp)
+_backward_source = _sig("e3conv_backward_source", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_char_p,
+                        ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t))
 _partition = _sig("e3conv_partition_rows", ctypes.c_int, _vp, _i64, ctypes.c_int, _vp)
 _set_radial = _sig("e3conv_set_radial_mlp", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_double,
                    ctypes.c_int, ctypes.c_int, _vp, _vp, _vp)
@@ -95,6 +100,7 @@ EXPORTED = ["e3conv_create", "e3conv_destroy", "e3conv_set_input_dtype",
             "e3conv_spherical_harmonics", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
             "e3conv_output_irrep", "e3conv_cg", "e3conv_kernel_info", "e3conv_kernel_source",
             "e3conv_forward", "e3conv_forward_rows", "e3conv_check", "e3conv_partition_rows",
+            "e3conv_backward", "e3conv_prepare_backward", "e3conv_backward_source",
             "e3conv_set_radial_mlp", "e3conv_radial_scalars", "e3conv_linear_create",
             "e3conv_linear_destroy", "e3conv_linear_query", "e3conv_linear_set_weights",
             "e3conv_linear_forward", "e3conv_linear_check", "e3conv_csr_workspace_size", "e3conv_build_csr",
@@ -354,6 +360,44 @@ class Conv:
                             _ptr(out) if E else None, _stream_handle(stream)),
             "e3conv_radial_scalars")
         return out
+
+    def backward(self, x, Y, s, senders, row_ptr, grad_out, receivers=None, sender_row_ptr=None,
+                 sender_perm=None, need_x=True, need_edges=True, stream=None):
+        """(grad_x, grad_sh, grad_scalars) of sum(grad_out * forward(...)); grad_x needs the
+        edges' receivers and the sender CSR (e3conv_build_csr of `senders`)."""
+        import torch
+        N = x.shape[0]
+        E = senders.shape[0]
+        dev = x.device
+        self._check_inputs(x, Y, s, senders, row_ptr)
+        _require("grad_out", grad_out, dev, torch.float32, N * self.nout * self.C)
+        gx = gY = gs = None
+        if need_x:
+            for name, tt in (("receivers", receivers), ("sender_row_ptr", sender_row_ptr),
+                             ("sender_perm", sender_perm)):
+                if tt is None:
+                    raise ValueError(f"{name} is needed for grad_x")
+                _require(name, tt, dev, torch.int32)
+            gx = torch.empty((N, self.nx, self.C), dtype=torch.float32, device=dev)
+        if need_edges:
+            gY = torch.empty((E, self.ny), dtype=torch.float32, device=dev)
+            gs = torch.empty((E, self.num_paths, self.C), dtype=torch.float32, device=dev)
+        ne = E > 0
+        _ok(_backward(self._h, _ptr(x), _ptr(Y) if ne else None, _ptr(s) if ne else None,
+                      _ptr(senders) if ne else None, _ptr(receivers) if ne and need_x else None,
+                      _ptr(row_ptr), _ptr(sender_row_ptr) if need_x else None,
+                      _ptr(sender_perm) if ne and need_x else None, N, _ptr(grad_out),
+                      _ptr(gx), _ptr(gY) if ne and need_edges else None,
+                      _ptr(gs) if ne and need_edges else None, _stream_handle(stream)),
+            "e3conv_backward")
+        return gx, gY, gs
+
+    def backward_source(self, which: int) -> str:
+        n = ctypes.c_size_t()
+        _ok(_backward_source(self._h, which, None, 0, ctypes.byref(n)), "e3conv_backward_source")
+        buf = ctypes.create_string_buffer(n.value)
+        _ok(_backward_source(self._h, which, buf, n.value, ctypes.byref(n)), "e3conv_backward_source")
+        return buf.value.decode()
 
     def forward_raw(self, x_ptr, Y_ptr, s_ptr, senders_ptr, row_ptr_ptr, num_nodes, out_ptr,
                     stream_handle):

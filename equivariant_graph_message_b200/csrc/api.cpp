@@ -128,6 +128,77 @@ int compile_once(Plan& pl, int dtype) {
   return E3CONV_OK;
 }
 
+// NVRTC compile of `source` for sm_100a; fills cubin, log, registers and local bytes.
+int nvrtc_compile(const std::string& source, const char* name, std::vector<char>& cubin,
+                  std::string& log, int& regs, int& local_bytes) {
+  nvrtcProgram prog;
+  if (nvrtcCreateProgram(&prog, source.c_str(), name, 0, nullptr, nullptr) != NVRTC_SUCCESS)
+    return fail(E3CONV_ERR_COMPILE, "nvrtcCreateProgram failed");
+  const char* opts[] = {"--gpu-architecture=sm_100a", "--std=c++17", "-lineinfo",
+                        "--ptxas-options=-v"};
+  nvrtcResult rc = nvrtcCompileProgram(prog, 4, opts);
+  size_t log_size = 0;
+  nvrtcGetProgramLogSize(prog, &log_size);
+  log.assign(log_size, '\0');
+  if (log_size) nvrtcGetProgramLog(prog, &log[0]);
+  if (rc != NVRTC_SUCCESS) {
+    nvrtcDestroyProgram(&prog);
+    return fail(E3CONV_ERR_COMPILE, "NVRTC compile failed: " + log.substr(0, 2000));
+  }
+  size_t n = 0;
+  nvrtcGetCUBINSize(prog, &n);
+  cubin.resize(n);
+  nvrtcGetCUBIN(prog, cubin.data());
+  nvrtcDestroyProgram(&prog);
+  std::smatch m;
+  regs = -1;
+  if (std::regex_search(log, m, std::regex("Used ([0-9]+) registers"))) regs = std::stoi(m[1]);
+  int stack = 0, spill = 0;
+  if (std::regex_search(log, m, std::regex("([0-9]+) bytes stack frame"))) stack = std::stoi(m[1]);
+  if (std::regex_search(log, m, std::regex("([0-9]+) bytes spill stores"))) spill = std::stoi(m[1]);
+  local_bytes = std::max(stack, spill);
+  return E3CONV_OK;
+}
+
+// The backward kernels of the plan's current dtype: generated, compiled and (with a
+// device) loaded on first use.
+int prepare_backward(Plan& pl) {
+  BwdVariant& bv = pl.bwd[pl.dtype];
+  if (bv.compiled) return E3CONV_OK;
+  if (pl.req_vec) return fail(E3CONV_ERR_UNSUPPORTED, "backward with edge vectors as input");
+  BwdVariant v;
+  v.shape = choose_backward_shape(pl, pl.dtype);
+  if (!v.shape.ok)
+    return fail(E3CONV_ERR_UNSUPPORTED, "backward needs C <= 128 (float32) or <= 256 (float16)");
+  const char* names[2] = {"e3conv_bwd_edges", "e3conv_bwd_nodes"};
+  for (int k = 0; k < 2; ++k) {
+    v.source[k] = generate_backward_source(pl, pl.dtype, v.shape, k == 1);
+    const int rc = nvrtc_compile(v.source[k], k ? "e3conv_bwd_nodes.cu" : "e3conv_bwd_edges.cu",
+                                 v.cubin[k], v.log[k], v.regs[k], v.local_bytes[k]);
+    if (rc != E3CONV_OK) return rc;
+  }
+  if (pl.device >= 0) {
+    Driver& d = driver();
+    for (int k = 0; k < 2; ++k) {
+      if (d.ModuleLoadData(&v.module[k], v.cubin[k].data()) != CUDA_SUCCESS ||
+          d.ModuleGetFunction(&v.fn[k], v.module[k], names[k]) != CUDA_SUCCESS) {
+        for (int q = 0; q <= k; ++q)
+          if (v.module[q]) d.ModuleUnload(v.module[q]);
+        return fail(E3CONV_ERR_CUDA, "loading the backward kernels failed");
+      }
+    }
+  }
+  v.compiled = true;
+  bv = v;
+  return E3CONV_OK;
+}
+
+void release_backward(BwdVariant& v) {
+  for (int k = 0; k < 2; ++k)
+    if (v.module[k]) driver().ModuleUnload(v.module[k]);
+  v = BwdVariant{};
+}
+
 // Staged variant without a requested block size: a first compile gives the
 // register count R; the block size is then the one that keeps the most warps
 // resident per SM (228 KB of shared memory per SM with 1 KB reserved per
@@ -357,6 +428,7 @@ void e3conv_destroy(e3conv_plan h) {
   {
     DeviceGuard g(pl.device);
     for (auto& v : pl.var) release_variant(v);
+    for (auto& v : pl.bwd) release_backward(v);
     if (pl.status) cudaFree(pl.status);
     for (void* q : {pl.radial.d_w0, pl.radial.d_wh, pl.radial.d_wo})
       if (q) cudaFree(q);
@@ -430,6 +502,7 @@ int e3conv_set_option(e3conv_plan h, int option, int value) {
   const int other = pl.dtype == E3CONV_F32 ? E3CONV_F16 : E3CONV_F32;
   release_variant(pl.var[other]);
   release_variant(pl.var[pl.dtype]);
+  for (auto& v : pl.bwd) release_backward(v);
   return compile_variant(pl, pl.dtype);
 }
 
@@ -839,6 +912,76 @@ int e3conv_partition_rows(const int32_t* row_ptr, int64_t num_nodes, int parts, 
     bounds[r] = lo;
   }
   bounds[parts] = num_nodes;
+  return E3CONV_OK;
+}
+
+int e3conv_prepare_backward(e3conv_plan h) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  DeviceGuard g(h->p.device);
+  return prepare_backward(h->p);
+}
+
+int e3conv_backward(e3conv_plan h, const void* x, const void* Y, const void* s,
+                    const int32_t* senders, const int32_t* receivers, const int32_t* row_ptr,
+                    const int32_t* sender_row_ptr, const int32_t* sender_perm, int64_t num_nodes,
+                    const float* grad_out, float* grad_x, float* grad_sh, float* grad_scalars,
+                    e3conv_stream stream) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  Plan& pl = h->p;
+  if (num_nodes < 0 || num_nodes >= (1ll << 31))
+    return fail(E3CONV_ERR_INVALID_ARG, "num_nodes out of range");
+  if (num_nodes == 0) return E3CONV_OK;
+  if ((grad_sh == nullptr) != (grad_scalars == nullptr))
+    return fail(E3CONV_ERR_INVALID_ARG, "grad_sh and grad_scalars are computed together: give both or neither");
+  if (!row_ptr || !grad_out) return fail(E3CONV_ERR_INVALID_ARG, "receiver_row_ptr and grad_out are required");
+  if (grad_sh && !x) return fail(E3CONV_ERR_INVALID_ARG, "node_features is required for grad_sh / grad_scalars");
+  if (grad_x && (!receivers || !sender_row_ptr || !sender_perm))
+    return fail(E3CONV_ERR_INVALID_ARG, "grad_x needs receivers, sender_row_ptr and sender_perm");
+  if (!aligned16(x) || !aligned16(Y) || !aligned16(s) || !aligned16(grad_out) ||
+      !aligned16(grad_x) || !aligned16(grad_scalars))
+    return fail(E3CONV_ERR_INVALID_ARG, "feature and gradient buffers must be 16-byte aligned");
+  if (pl.device < 0) return fail(E3CONV_ERR_NO_DEVICE, "plan has no device module");
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess || cur != pl.device)
+    return fail(E3CONV_ERR_INVALID_ARG, "current device differs from the plan's device");
+  int rc = prepare_backward(pl);
+  if (rc != E3CONV_OK) return rc;
+  const BwdVariant& bv = pl.bwd[pl.dtype];
+  const BwdShape& b = bv.shape;
+  int n32 = static_cast<int>(num_nodes);
+  float inv_avg = static_cast<float>(1.0 / pl.avg);
+  const long long warps = (num_nodes + b.ipw - 1) / b.ipw;
+  const long long blocks = (warps * 32 + b.block - 1) / b.block;
+  if (blocks >= (1ll << 31)) return fail(E3CONV_ERR_UNSUPPORTED, "grid too large");
+  CUstream st = reinterpret_cast<CUstream>(stream);
+  if (grad_sh) {
+    void* args[] = {const_cast<void**>(&x), const_cast<void**>(&Y), const_cast<void**>(&s),
+                    const_cast<int32_t**>(&senders), const_cast<int32_t**>(&row_ptr), &n32,
+                    const_cast<float**>(&grad_out), &grad_sh, &grad_scalars, &inv_avg, &pl.status};
+    if (driver().LaunchKernel(bv.fn[0], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1, 0, st,
+                              args, nullptr) != CUDA_SUCCESS)
+      return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed (backward, edges)");
+  }
+  if (grad_x) {
+    void* args[] = {const_cast<void**>(&Y), const_cast<void**>(&s),
+                    const_cast<int32_t**>(&receivers), const_cast<int32_t**>(&row_ptr),
+                    const_cast<int32_t**>(&sender_row_ptr), const_cast<int32_t**>(&sender_perm),
+                    &n32, const_cast<float**>(&grad_out), &grad_x, &inv_avg, &pl.status};
+    if (driver().LaunchKernel(bv.fn[1], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1, 0, st,
+                              args, nullptr) != CUDA_SUCCESS)
+      return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed (backward, nodes)");
+  }
+  return E3CONV_OK;
+}
+
+int e3conv_backward_source(e3conv_plan h, int which, char* buf, size_t buf_len, size_t* needed) {
+  if (!h || which < 0 || which > 1) return fail(E3CONV_ERR_INVALID_ARG, "bad argument");
+  DeviceGuard g(h->p.device);
+  int rc = prepare_backward(h->p);
+  if (rc != E3CONV_OK) return rc;
+  const std::string& src = h->p.bwd[h->p.dtype].source[which];
+  if (needed) *needed = src.size() + 1;
+  if (buf && buf_len >= src.size() + 1) std::memcpy(buf, src.c_str(), src.size() + 1);
   return E3CONV_OK;
 }
 

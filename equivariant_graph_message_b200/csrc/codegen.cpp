@@ -1741,6 +1741,315 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Backward kernels (gradients of sum(g * out) for an upstream gradient g of the
+// forward's output).  The forward is linear in each of x, Y and s, so every
+// gradient is the forward's four-factor product with one factor removed:
+//   gs[e, p, u]       = inv_avg sum_{i,j,k} CG_p[i,j,k] x[a,i,u] Y[e,j] g[b,o_p+k,u]
+//   gY[e, j]          = inv_avg sum_p sum_u sum_{i,k} CG_p[i,j,k] s[e,p,u] x[a,i,u] g[b,o_p+k,u]
+//   gx[a, i, u]       = inv_avg sum_{e: senders[e] = a} sum_p sum_{j,k} CG_p[i,j,k] s[e,p,u] Y[e,j] g[b,o_p+k,u]
+// (a = sender, b = receiver of edge e).  Two kernels, every CG nonzero
+// unrolled as a constant:
+//  * edges (receiver order, like the forward): an item of TL lanes per
+//    receiver row holds the row's g in registers (V channels per lane), and
+//    for each edge writes gs and the channel-reduced gY (butterfly over the
+//    item's lanes; TL is a power of two, lanes past C contribute zeros);
+//  * nodes (sender order): an item per sender walks the sender's edges
+//    through the sender CSR (sender_row_ptr, sender_perm) and keeps gx in
+//    registers; one store per sender.
+
+BwdShape choose_backward_shape(const Plan& pl, int dtype) {
+  BwdShape b;
+  const int vmax = dtype == E3CONV_F16 ? 8 : 4;
+  int V = 1;
+  while (V < vmax && pl.C > 32 * V) V *= 2;
+  if (pl.C > 32 * V || pl.C % V != 0) {
+    // one item must cover every channel (the gY reduction stays inside a warp)
+    b.ok = false;
+    return b;
+  }
+  b.V = V;
+  int TL = 1;
+  while (TL * V < pl.C) TL *= 2;
+  b.TL = TL;
+  b.ipw = 32 / TL;
+  b.block = 128;
+  b.ok = true;
+  return b;
+}
+
+namespace {
+
+// Declares g loads: g{c}_{v} for the given output components at grow + c*C.
+void emit_g_load(Emitter& em, const Plan& pl, int V, const std::string& grow, int c0, int c1,
+                 const std::string& active) {
+  for (int c = c0; c < c1; ++c) {
+    std::string decl = "float";
+    for (int v = 0; v < V; ++v) decl += std::string(v ? "," : "") + " g" + S(c) + "_" + S(v) + " = 0.f";
+    em.line(decl + ";");
+    em.line("if (" + active + ") {");
+    em.ind++;
+    emit_vec_load(em, E3CONV_F32, V, "ldg", grow + " + " + S(c * pl.C), "g" + S(c));
+    em.ind--;
+    em.line("}");
+  }
+}
+
+std::string bwd_prelude(Emitter& em, const Plan& pl, int dtype, const BwdShape& b) {
+  const bool f16 = dtype == E3CONV_F16;
+  em.line(std::string("// generated by libe3conv: backward of the equivariant convolution (") +
+          "C=" + S(pl.C) + " nx=" + S(pl.nx) + " ny=" + S(pl.ny) + " nout=" + S(pl.nout) +
+          " paths=" + S(pl.paths.size()) + " dtype=" + (f16 ? "f16" : "f32") + " V=" + S(b.V) +
+          " TL=" + S(b.TL) + " ipw=" + S(b.ipw) + ")");
+  emit_prelude(em);
+  return f16 ? "unsigned short" : "float";
+}
+
+std::string bwd_edges_source(const Plan& pl, int dtype, const BwdShape& b) {
+  Emitter em;
+  const std::string T = bwd_prelude(em, pl, dtype, b);
+  const int V = b.V;
+  const long long s_row = static_cast<long long>(pl.paths.size()) * pl.C;
+  em.line("extern \"C\" __global__ void __launch_bounds__(" + S(b.block) + ") e3conv_bwd_edges(");
+  em.line("    const " + T + "* __restrict__ x, const " + T + "* __restrict__ Y, const " + T +
+          "* __restrict__ s,");
+  em.line("    const int* __restrict__ senders, const int* __restrict__ row_ptr, int num_nodes,");
+  em.line("    const float* __restrict__ g, float* __restrict__ gY, float* __restrict__ gs,");
+  em.line("    float inv_avg, unsigned int* __restrict__ status)");
+  em.line("{");
+  em.ind++;
+  em.line("const int lane = threadIdx.x & 31;");
+  em.line("const long long gwarp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;");
+  em.line("const int sub = lane / " + S(b.TL) + ";");
+  em.line("const int within = lane - sub * " + S(b.TL) + ";");
+  em.line("const unsigned int item_mask = " + std::string(b.TL == 32 ? "0xffffffffu" :
+          "((1u << " + S(b.TL) + ") - 1u) << (sub * " + S(b.TL) + ")") + ";");
+  em.line("const long long bb = gwarp * " + S(b.ipw) + " + sub;");
+  em.line("if (bb >= num_nodes) return;  // the whole item (lanes of one receiver) leaves");
+  em.line("const int u0 = within * " + S(V) + ";");
+  em.line("const bool active = u0 < " + S(pl.C) + ";");
+  em.line("const int e_base = __ldg(row_ptr), e_end = __ldg(row_ptr + num_nodes);");
+  em.line("int e0 = row_ptr[bb], e1 = row_ptr[bb + 1];");
+  em.line("if (e0 < e_base || e1 < e0 || e1 > e_end) { if (within == 0) atomicOr(status, 1u); e1 = e0; }");
+  em.line("if (e0 == e1) return;");
+  emit_g_load(em, pl, V, "g + bb * " + S(static_cast<long long>(pl.nout) * pl.C) + " + u0", 0,
+              pl.nout, "active");
+  em.line("#pragma unroll 1");
+  em.line("for (int e = e0; e < e1; ++e) {");
+  em.ind++;
+  em.line("const long long le = e - e_base;");
+  em.line("const int a = senders[le];");
+  em.line("const bool valid = (unsigned int)a < (unsigned int)num_nodes;");
+  em.line("if (!valid && within == 0) atomicOr(status, 2u);");
+  em.line("const " + T + "* yr = Y + le * " + S(pl.ny) + ";");
+  emit_y_load(em, pl, dtype, "ldg", "yr");
+  std::string dy = "float";
+  for (int j = 0; j < pl.ny; ++j) dy += std::string(j ? "," : "") + " dy" + S(j) + " = 0.f";
+  em.line(dy + ";");
+  em.line("const bool go = valid && active;");
+  em.line("const " + T + "* xr = x + (long long)(valid ? a : 0) * " + S(pl.nx * pl.C) + " + u0;");
+  em.line("const " + T + "* sr = s + le * " + S(s_row) + " + u0;");
+  em.line("float* gsr = gs + le * " + S(s_row) + " + u0;");
+  size_t p = 0;
+  while (p < pl.paths.size()) {
+    const int n1 = pl.paths[p].n1;
+    size_t q = p;
+    while (q < pl.paths.size() && pl.paths[q].n1 == n1) ++q;
+    const Path& first = pl.paths[p];
+    const int d1 = 2 * first.l1 + 1;
+    em.line("{  // node irrep " + S(n1) + " (l=" + S(first.l1) + ")");
+    em.ind++;
+    for (int i = 0; i < d1; ++i) {
+      std::string decl = "float";
+      for (int v = 0; v < V; ++v) decl += std::string(v ? "," : "") + " x" + S(i) + "_" + S(v) + " = 0.f";
+      em.line(decl + ";");
+      em.line("if (go) {");
+      em.ind++;
+      emit_vec_load(em, dtype, V, "ldg", "xr + " + S((first.x_off + i) * pl.C), "x" + S(i));
+      em.ind--;
+      em.line("}");
+    }
+    for (size_t r = p; r < q; ++r) {
+      const Path& P = pl.paths[r];
+      const int d3 = 2 * P.l3 + 1;
+      em.line("{  // path " + S(r) + ": " + S(P.l1) + " x " + S(P.l2) + " -> " + S(P.l3));
+      em.ind++;
+      {
+        std::string decl = "float";
+        for (int v = 0; v < V; ++v) decl += std::string(v ? "," : "") + " s_" + S(v) + " = 0.f";
+        em.line(decl + ";");
+        em.line("if (go) {");
+        em.ind++;
+        emit_vec_load(em, dtype, V, "ldg", "sr + " + S(static_cast<long long>(r) * pl.C), "s");
+        em.ind--;
+        em.line("}");
+      }
+      // t_k = sum (c Y_j) x_i   (for gs);  dY_j += c (s x_i) g_k   (summed over channels)
+      for (int k = 0; k < d3; ++k)
+        for (int v = 0; v < V; ++v) em.line("float t" + S(k) + "_" + S(v) + " = 0.f;");
+      for (int i = 0; i < d1; ++i)
+        for (int v = 0; v < V; ++v)
+          em.line("const float z" + S(i) + "_" + S(v) + " = s_" + S(v) + " * x" + S(i) + "_" + S(v) + ";");
+      for (const auto& n : P.nnz) {
+        const std::string c = flt(n.c);
+        const std::string yj = "y" + S(P.y_off + n.j);
+        for (int v = 0; v < V; ++v) {
+          const std::string xv = "x" + S(n.i) + "_" + S(v), zv = "z" + S(n.i) + "_" + S(v);
+          const std::string gv = "g" + S(P.out_off + n.k) + "_" + S(v);
+          em.line("t" + S(n.k) + "_" + S(v) + " = fmaf(" + c + " * " + yj + ", " + xv + ", t" +
+                  S(n.k) + "_" + S(v) + ");");
+          em.line("dy" + S(P.y_off + n.j) + " = fmaf(" + c + ", " + zv + " * " + gv + ", dy" +
+                  S(P.y_off + n.j) + ");");
+        }
+      }
+      // gs[e, p, u0..u0+V) = inv_avg sum_k g_k t_k
+      std::vector<std::string> dsv(V);
+      for (int v = 0; v < V; ++v) {
+        std::string acc = "0.f";
+        for (int k = 0; k < d3; ++k)
+          acc = "fmaf(g" + S(P.out_off + k) + "_" + S(v) + ", t" + S(k) + "_" + S(v) + ", " + acc + ")";
+        dsv[v] = "inv_avg * " + acc;
+      }
+      em.line("if (active) {");
+      em.ind++;
+      const std::string dst = "gsr + " + S(static_cast<long long>(r) * pl.C);
+      if (V % 4 == 0) {
+        for (int v = 0; v < V; v += 4)
+          em.line("*reinterpret_cast<float4*>(" + dst + " + " + S(v) + ") = make_float4(" + dsv[v] +
+                  ", " + dsv[v + 1] + ", " + dsv[v + 2] + ", " + dsv[v + 3] + ");");
+      } else if (V == 2) {
+        em.line("*reinterpret_cast<float2*>(" + dst + ") = make_float2(" + dsv[0] + ", " + dsv[1] + ");");
+      } else {
+        em.line("*(" + dst + ") = " + dsv[0] + ";");
+      }
+      em.ind--;
+      em.line("}");
+      em.ind--;
+      em.line("}");
+    }
+    em.ind--;
+    em.line("}");
+    p = q;
+  }
+  // channel reduction of dY over the item's lanes (butterfly inside the item's aligned group
+  // of TL lanes; items of one warp walk rows of different lengths, so the mask names only
+  // the item's own lanes), then one lane stores
+  for (int off = b.TL / 2; off >= 1; off /= 2)
+    for (int j = 0; j < pl.ny; ++j)
+      em.line("dy" + S(j) + " += __shfl_xor_sync(item_mask, dy" + S(j) + ", " + S(off) + ");");
+  em.line("if (within == 0) {");
+  em.ind++;
+  for (int j = 0; j < pl.ny; ++j)
+    em.line("gY[le * " + S(pl.ny) + " + " + S(j) + "] = inv_avg * dy" + S(j) + ";");
+  em.ind--;
+  em.line("}");
+  em.ind--;
+  em.line("}");
+  em.ind--;
+  em.line("}");
+  return em.o.str();
+}
+
+std::string bwd_nodes_source(const Plan& pl, int dtype, const BwdShape& b) {
+  Emitter em;
+  const std::string T = bwd_prelude(em, pl, dtype, b);
+  const int V = b.V;
+  const long long s_row = static_cast<long long>(pl.paths.size()) * pl.C;
+  em.line("extern \"C\" __global__ void __launch_bounds__(" + S(b.block) + ") e3conv_bwd_nodes(");
+  em.line("    const " + T + "* __restrict__ Y, const " + T + "* __restrict__ s,");
+  em.line("    const int* __restrict__ receivers, const int* __restrict__ row_ptr,");
+  em.line("    const int* __restrict__ sender_row_ptr, const int* __restrict__ sender_perm,");
+  em.line("    int num_nodes, const float* __restrict__ g, float* __restrict__ gx, float inv_avg,");
+  em.line("    unsigned int* __restrict__ status)");
+  em.line("{");
+  em.ind++;
+  em.line("const int lane = threadIdx.x & 31;");
+  em.line("const long long gwarp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;");
+  em.line("const int sub = lane / " + S(b.TL) + ";");
+  em.line("const int within = lane - sub * " + S(b.TL) + ";");
+  em.line("const long long a = gwarp * " + S(b.ipw) + " + sub;");
+  em.line("if (a >= num_nodes) return;");
+  em.line("const int u0 = within * " + S(V) + ";");
+  em.line("if (u0 >= " + S(pl.C) + ") return;");
+  em.line("const int e_base = __ldg(row_ptr), e_end = __ldg(row_ptr + num_nodes);");
+  em.line("const int ne = e_end - e_base;");
+  for (int i = 0; i < pl.nx; ++i) {
+    std::string l = "float";
+    for (int v = 0; v < V; ++v) l += std::string(v ? "," : "") + " h" + S(i) + "_" + S(v) + " = 0.f";
+    em.line(l + ";");
+  }
+  em.line("int t0 = sender_row_ptr[a], t1 = sender_row_ptr[a + 1];");
+  em.line("if (t0 < 0 || t1 < t0 || t1 > ne) { if (within == 0) atomicOr(status, 1u); t1 = t0; }");
+  em.line("#pragma unroll 1");
+  em.line("for (int t = t0; t < t1; ++t) {");
+  em.ind++;
+  em.line("const int le = sender_perm[t];");
+  em.line("if ((unsigned int)le >= (unsigned int)ne) { if (within == 0) atomicOr(status, 2u); continue; }");
+  em.line("const int bb = receivers[le];");
+  em.line("if ((unsigned int)bb >= (unsigned int)num_nodes) { if (within == 0) atomicOr(status, 2u); continue; }");
+  em.line("const " + T + "* yr = Y + (long long)le * " + S(pl.ny) + ";");
+  emit_y_load(em, pl, dtype, "ldg", "yr");
+  em.line("const " + T + "* sr = s + (long long)le * " + S(s_row) + " + u0;");
+  em.line("const float* gr = g + (long long)bb * " + S(static_cast<long long>(pl.nout) * pl.C) + " + u0;");
+  // paths grouped by output irrep: g of the irrep loaded once
+  for (size_t o = 0; o < pl.outputs.size(); ++o) {
+    const int d3 = 2 * pl.outputs[o].l + 1, off = pl.outputs[o].off;
+    em.line("{  // output irrep " + S(o));
+    em.ind++;
+    emit_g_load(em, pl, V, "gr", off, off + d3, "true");
+    for (size_t r = 0; r < pl.paths.size(); ++r) {
+      const Path& P = pl.paths[r];
+      if (P.o != static_cast<int>(o)) continue;
+      em.line("{  // path " + S(r) + ": " + S(P.l1) + " x " + S(P.l2) + " -> " + S(P.l3));
+      em.ind++;
+      {
+        std::string decl = "float";
+        for (int v = 0; v < V; ++v) decl += std::string(v ? "," : "") + " s_" + S(v);
+        em.line(decl + ";");
+        emit_vec_load(em, dtype, V, "ldg", "sr + " + S(static_cast<long long>(r) * pl.C), "s");
+      }
+      for (int k = 0; k < d3; ++k)
+        for (int v = 0; v < V; ++v)
+          em.line("const float w" + S(k) + "_" + S(v) + " = s_" + S(v) + " * g" + S(off + k) + "_" + S(v) + ";");
+      for (const auto& n : P.nnz)
+        for (int v = 0; v < V; ++v) {
+          const std::string h = "h" + S(P.x_off + n.i) + "_" + S(v);
+          em.line(h + " = fmaf(" + flt(n.c) + " * y" + S(P.y_off + n.j) + ", w" + S(n.k) + "_" +
+                  S(v) + ", " + h + ");");
+        }
+      em.ind--;
+      em.line("}");
+    }
+    em.ind--;
+    em.line("}");
+  }
+  em.ind--;
+  em.line("}");
+  em.line("float* xo = gx + a * " + S(static_cast<long long>(pl.nx) * pl.C) + " + u0;");
+  for (int i = 0; i < pl.nx; ++i) {
+    const std::string dst = "xo + " + S(i * pl.C);
+    auto h = [&](int v) { return "inv_avg * h" + S(i) + "_" + S(v); };
+    if (V % 4 == 0) {
+      for (int v = 0; v < V; v += 4)
+        em.line("*reinterpret_cast<float4*>(" + dst + " + " + S(v) + ") = make_float4(" + h(v) + ", " +
+                h(v + 1) + ", " + h(v + 2) + ", " + h(v + 3) + ");");
+    } else if (V == 2) {
+      em.line("*reinterpret_cast<float2*>(" + dst + ") = make_float2(" + h(0) + ", " + h(1) + ");");
+    } else {
+      em.line("*(" + dst + ") = " + h(0) + ";");
+    }
+  }
+  em.ind--;
+  em.line("}");
+  return em.o.str();
+}
+
+}  // namespace
+
+std::string generate_backward_source(const Plan& pl, int dtype, const BwdShape& b, bool nodes) {
+  return nodes ? bwd_nodes_source(pl, dtype, b) : bwd_edges_source(pl, dtype, b);
+}
+
 std::string generate_forward_source(const Plan& pl, int dtype, const Shape& sh) {
   if (sh.tc) return tc_source(pl, sh);
   return sh.stages > 0 ? staged_source(pl, dtype, sh) : direct_source(pl, dtype, sh);

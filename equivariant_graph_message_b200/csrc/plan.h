@@ -88,6 +88,24 @@ struct AEntry {
   std::vector<std::pair<int, double>> terms;  // (index into the edge's Y row, CG coefficient)
 };
 
+// Launch shape of the backward kernels: V channels per lane, TL lanes (a power
+// of two) per item, one item per node covering all C channels.
+struct BwdShape {
+  bool ok = false;
+  int V = 1, TL = 32, ipw = 1, block = 128;
+};
+
+struct BwdVariant {
+  bool compiled = false;
+  BwdShape shape;
+  std::string source[2];     // edges, nodes
+  std::vector<char> cubin[2];
+  std::string log[2];
+  CUmodule module[2] = {nullptr, nullptr};
+  CUfunction fn[2] = {nullptr, nullptr};
+  int regs[2] = {-1, -1}, local_bytes[2] = {-1, -1};
+};
+
 struct Variant {
   bool compiled = false;
   Shape shape;
@@ -162,6 +180,7 @@ struct Plan {
   CUcontext ctx = nullptr;
   unsigned int* status = nullptr;  // device status word
   Variant var[2];
+  BwdVariant bwd[2];               // backward kernels per input dtype (compiled on first use)
   RadialPlan radial;
 };
 
@@ -195,6 +214,8 @@ int linear_launch(const LinearPlan& lp, const void* dev_w, const float* x, long 
 std::vector<AEntry> build_a_entries(const Plan& plan);
 Shape choose_shape(const Plan& plan, int dtype);
 std::string generate_forward_source(const Plan& plan, int dtype, const Shape& shape);
+BwdShape choose_backward_shape(const Plan& plan, int dtype);
+std::string generate_backward_source(const Plan& plan, int dtype, const BwdShape& shape, bool nodes);
 
 }  // namespace e3c
 

@@ -374,6 +374,54 @@ E3CONV_API int e3conv_linear_check(e3conv_linear linear, e3conv_stream stream);
 E3CONV_API int e3conv_partition_rows(const int32_t* row_ptr, int64_t num_nodes, int parts,
                                      int64_t* bounds);
 
+/* ---------------------------------------------------------------------------
+ * Backward: gradients of sum(grad_out * out) for an upstream gradient grad_out
+ * of the forward's output.  The forward is linear in each of x, Y and s, so
+ * each gradient is the forward's product with one factor removed:
+ *   grad_scalars[e, p, u] = (1/N) sum_{i,j,k} CG_p[i,j,k] x[a,i,u] Y[e,j] grad_out[b, o_p+k, u]
+ *   grad_sh[e, j]         = (1/N) sum_{p,u,i,k} CG_p[i,j,k] s[e,p,u] x[a,i,u] grad_out[b, o_p+k, u]
+ *   grad_x[a, i, u]       = (1/N) sum_{e: senders[e] = a} sum_{p,j,k} CG_p[i,j,k] s[e,p,u] Y[e,j]
+ *                                                              grad_out[b, o_p+k, u]
+ * with a = senders[e], b = receivers[e] (p over the paths that involve the
+ * component).  grad_sh and grad_scalars come from one kernel in receiver order
+ * (each receiver's grad_out row read once, edges in CSR order, no atomics);
+ * grad_x from one kernel in sender order (e3j "graph_ordering" notes: the
+ * SENDER-ordered gather), which needs the edges sorted by sender: sender_row_ptr
+ * [num_nodes+1] and sender_perm [E] (sender_perm[t] = the t-th edge of the
+ * receiver-sorted arrays in sender order), which e3conv_build_csr makes from
+ * `senders`.  Every CG nonzero is unrolled as a constant; float32 accumulation.
+ *
+ *   node_features, edge_sh, edge_scalars, senders, receiver_row_ptr: as for
+ *                  e3conv_forward (harmonics as input: not with
+ *                  E3CONV_OPT_EDGE_VECTORS).
+ *   receivers:     device int32 [E], receiver of each (receiver-sorted) edge;
+ *                  needed for grad_x only.
+ *   grad_out:      device float32 [num_nodes][nout][C].
+ *   grad_x:        device float32 [num_nodes][nx][C], fully overwritten, or NULL.
+ *   grad_sh:       device float32 [E][ny], or NULL.
+ *   grad_scalars:  device float32 [E][P][C], or NULL (NULL exactly when
+ *                  grad_sh is NULL).
+ * C <= 128 (float32 inputs) or <= 256 (float16).  Out-of-range indices are
+ * skipped and set the status word (e3conv_check).  Up to two kernel launches
+ * on `stream`; no host synchronisation, no allocation.  The first call for a
+ * dtype generates and compiles the two kernels (host-side, blocking); call
+ * e3conv_prepare_backward to do that ahead of time. */
+E3CONV_API int e3conv_backward(e3conv_plan plan, const void* node_features, const void* edge_sh,
+                               const void* edge_scalars, const int32_t* senders,
+                               const int32_t* receivers, const int32_t* receiver_row_ptr,
+                               const int32_t* sender_row_ptr, const int32_t* sender_perm,
+                               int64_t num_nodes, const float* grad_out, float* grad_x,
+                               float* grad_sh, float* grad_scalars, e3conv_stream stream);
+
+/* Generates, compiles and loads the backward kernels of the plan's current
+ * dtype (host-side, blocking). */
+E3CONV_API int e3conv_prepare_backward(e3conv_plan plan);
+
+/* Generated CUDA source of a backward kernel (which = 0: edges, 1: nodes),
+ * as e3conv_kernel_source. */
+E3CONV_API int e3conv_backward_source(e3conv_plan plan, int which, char* buf, size_t buf_len,
+                                      size_t* needed);
+
 /* Synchronises `stream`, reads and clears the plan's status word.  Returns
  * E3CONV_OK, E3CONV_ERR_BAD_INDEX if a forward since the last check met an
  * out-of-range sender or row range, or E3CONV_ERR_CUDA if a pipeline wait

@@ -426,3 +426,26 @@ def test_linear_layer_host_validation():
     assert (lin.dim_in, lin.dim_out, lin.num_weight_blocks) == (64 * 9, 32 * 13, 2)
     with pytest.raises(ValueError):
         lin.set_weights([np.zeros((64, 32))])            # two matched irreps need two blocks
+
+
+@pytest.mark.parametrize("name", ORDER)
+def test_backward_kernels_generate_for_every_workload(name):
+    s = SPECS[name]
+    c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 10.0, dtype=s.dtype)
+    edges, nodes = c.backward_source(0), c.backward_source(1)
+    assert "e3conv_bwd_edges" in edges and "e3conv_bwd_nodes" in nodes
+    # every CG nonzero appears once per channel of a lane in each kernel
+    m = re.search(r"V=(\d+) TL=(\d+)", edges)
+    V = int(m.group(1))
+    nnz = sum(int((np.abs(c.cg(p)) > 1e-12).sum()) for p in range(c.num_paths))
+    assert edges.count("dy") >= nnz * V and nodes.count(" = fmaf(") >= nnz * V
+
+
+def test_backward_rejects_edge_vector_plans_and_wide_channels():
+    c = e3.Conv("8x0e+8x1o", "1x0e+1x1o", "8x0e+8x1o", 1.0)
+    c.set_edge_vectors(1)
+    with pytest.raises(e3.E3ConvError):
+        c.backward_source(0)
+    wide = e3.Conv("256x0e", "1x0e+1x1o", "256x0e+256x1o", 1.0)   # float32, C > 128
+    with pytest.raises(e3.E3ConvError):
+        wide.backward_source(0)
