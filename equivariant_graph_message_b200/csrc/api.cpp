@@ -480,9 +480,12 @@ int e3conv_set_option(e3conv_plan h, int option, int value) {
   Plan& pl = h->p;
   if (option != E3CONV_OPT_CONTRACT_FIRST && option != E3CONV_OPT_TENSOR_CORES &&
       option != E3CONV_OPT_PATH_SPLIT && option != E3CONV_OPT_EDGE_VECTORS &&
-      option != E3CONV_OPT_A_LAYOUT)
+      option != E3CONV_OPT_A_LAYOUT && option != E3CONV_OPT_COPY_GROUP)
     return fail(E3CONV_ERR_UNSUPPORTED, "unknown option");
-  if (option == E3CONV_OPT_A_LAYOUT) {
+  if (option == E3CONV_OPT_COPY_GROUP) {
+    if (value != -1 && (value < 1 || value > 4)) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1 or 1 .. 4");
+    pl.req_group = value;
+  } else if (option == E3CONV_OPT_A_LAYOUT) {
     if (value < -1 || value > 2) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1 .. 2");
     pl.req_alayout = value;
   } else if (option == E3CONV_OPT_EDGE_VECTORS) {
@@ -515,6 +518,7 @@ int e3conv_get_option(e3conv_plan h, int option, int* value) {
     case E3CONV_OPT_PATH_SPLIT: *value = pl.req_psplit; return E3CONV_OK;
     case E3CONV_OPT_EDGE_VECTORS: *value = pl.req_vec; return E3CONV_OK;
     case E3CONV_OPT_A_LAYOUT: *value = pl.req_alayout; return E3CONV_OK;
+    case E3CONV_OPT_COPY_GROUP: *value = pl.req_group; return E3CONV_OK;
     default: return fail(E3CONV_ERR_UNSUPPORTED, "unknown option");
   }
 }

@@ -182,10 +182,16 @@ Shape choose_shape(const Plan& pl, int dtype) {
     s.TL = 32;
     s.tiles = 1;
     s.ipw = 1;
+    // The ring: NS stages in regions of s rows, sender rows and Y rows (a group of G
+    // consecutive stages takes G consecutive edges' s rows and Y rows in one copy each).
+    s.group = pl.req_group > 0 ? pl.req_group : 1;
+    int S = pl.req_stages > 0 ? pl.req_stages : 2 * s.group;
+    S = (std::max(S, s.group) + s.group - 1) / s.group * s.group;
+    s.x_slot = align_up(s.x_bytes, 128);
     s.s_off = 0;
-    s.x_off = align_up(s.s_bytes, 128);
-    s.y_off = s.x_off + align_up(s.x_bytes, 128);
-    s.stage_bytes = s.y_off + align_up(s.y_bytes, 128);
+    s.x_off = align_up(S * s.s_bytes, 128);
+    s.y_off = s.x_off + S * s.x_slot;
+    s.stage_bytes = align_up(s.y_off + S * s.y_bytes, 128);  // the whole ring
     s.coop = pl.req_coop != 0 && (V == 1 || V % 2 == 0);
     s.psplit = s.coop ? psplit : 1;
     // A layout: float slots in round order (a lane broadcasts each entry to a pair), or
@@ -200,12 +206,11 @@ Shape choose_shape(const Plan& pl, int dtype) {
     if (s.coop)
       for (const auto& g : coop_groups(pl, s)) a_bytes += g.a_bytes;
     const int y_bytes = s.coop ? s.psplit * align_up(4 * pl.ny, 16) : 0;
-    const int S = pl.req_stages > 0 ? pl.req_stages : 2;
     s.stages = S;
-    s.a_off = S * s.stage_bytes;
+    s.a_off = s.stage_bytes;
     s.yf_off = s.a_off + a_bytes;
     s.bar_off = align_up(s.yf_off + y_bytes, 8);
-    s.hdr_off = s.bar_off + 8 * S;
+    s.hdr_off = s.bar_off + 8 * (S / s.group);
     s.warp_smem = align_up(s.hdr_off + 16 * S, 128);
     const int team_threads = 32 * team;
     int block = pl.req_block > 0 ? pl.req_block : (pl.auto_block > 0 ? pl.auto_block : 4 * team_threads);
@@ -863,8 +868,8 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh, con
     base += T.terms[r] * RW;
   }
   em.line(group_sync + ";");
-  em.line("const " + Ty + "* xs = reinterpret_cast<const " + Ty + "*>(stg + " + S(sh.x_off) + ") + u0;");
-  em.line("const " + Ty + "* ss = reinterpret_cast<const " + Ty + "*>(stg + " + S(sh.s_off) + ") + u0;");
+  em.line("const " + Ty + "* xs = reinterpret_cast<const " + Ty + "*>(stg_x) + u0;");
+  em.line("const " + Ty + "* ss = reinterpret_cast<const " + Ty + "*>(stg_s) + u0;");
   // entry index of (path, i, k)
   std::map<std::tuple<int, int, int>, int> idx;
   for (size_t n = 0; n < G.ent.size(); ++n)
@@ -1119,7 +1124,8 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("// C=" + S(pl.C) + " nx=" + S(pl.nx) + " ny=" + S(pl.ny) + " nout=" + S(pl.nout) +
           " paths=" + S(pl.paths.size()) + " dtype=" + (f16 ? "f16" : "f32") + " V=" + S(V) +
           " team=" + S(TW) + " teams/block=" + S(teams) + " stages=" + S(NS) +
-          " stage_bytes=" + S(sh.stage_bytes) + " contract_first=" + S(sh.coop ? 1 : 0) +
+          " ring_bytes=" + S(sh.stage_bytes) + " copy_group=" + S(sh.group) +
+          " contract_first=" + S(sh.coop ? 1 : 0) +
           " path_split=" + S(sh.coop ? sh.psplit : 1) + " a_layout=" + S(sh.amode));
   emit_prelude(em);
   std::vector<CoopGroup> groups;
@@ -1191,7 +1197,7 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("int* hdr = reinterpret_cast<int*>(tbase + " + S(sh.hdr_off) + ");  // per stage: sender, receiver, last");
   em.line("const bool issuer = tw == 0 && lane == 0;  // the lane that issues the team's copies");
   em.line("if (issuer) {");
-  em.line("  for (int k = 0; k < " + S(NS) + "; ++k) bar_init(bars + k);");
+  em.line("  for (int k = 0; k < " + S(NS / sh.group) + "; ++k) bar_init(bars + k);");
   em.line("  asm volatile(\"fence.mbarrier_init.release.cluster;\" ::: \"memory\");");
   em.line("}");
   em.line("team_sync();");
@@ -1213,7 +1219,13 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
     emit_acc_decl(em, pl, V);
   }
   // Every warp of the team walks the same rows (same decisions); only the
-  // issuer lane writes the stage header and issues the bulk copies.
+  // issuer lane writes the stage headers and issues the bulk copies.  The ring
+  // has NS stages in NG = NS / G groups; one produce() fills a group with up to
+  // G consecutive edges of one row: one bulk copy of their s rows, one of their
+  // Y rows (both contiguous in memory and in the ring), one per sender row, and
+  // one mbarrier per group.  Unused stages of a group are marked empty (-3).
+  const int G = sh.group, NG = NS / G;
+  const std::string s_at = "tbase + " + S(sh.s_off) + " + ";    // + stage * s_bytes
   em.line("auto produce = [&]() {");
   em.ind++;
   em.line("while (!pdone && pe >= pe1) {");
@@ -1230,51 +1242,72 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("  }");
   em.line("}");
   em.line("if (pdone) return;");
-  em.line("if (pwin < 0 || pe >= pwin + 32) {");
+  em.line("const int n = min(" + S(G) + ", pe1 - pe);  // edges in this group");
+  em.line("if (pwin < 0 || pe + n > pwin + 32) {");
   em.line("  pwin = pe;");
   em.line("  psw = (pe + lane < pe1) ? senders[pe + lane - e_base] : 0;");
   em.line("}");
-  em.line("const int a = __shfl_sync(0xffffffffu, psw, pe - pwin);");
-  em.line("const bool valid = (unsigned int)a < (unsigned int)num_nodes;");
-  em.line("const unsigned int st = ppos % " + S(NS) + ";");
+  em.line("const unsigned int g0 = (ppos % " + S(NG) + ") * " + S(G) + ";  // first stage of the group");
+  em.line("unsigned int xbytes = 0;");
+  for (int k = 0; k < G; ++k) {
+    em.line("const int a" + S(k) + " = __shfl_sync(0xffffffffu, psw, min(pe + " + S(k) + " - pwin, 31));");
+    em.line("const bool v" + S(k) + " = " + S(k) + " < n && (unsigned int)a" + S(k) +
+            " < (unsigned int)num_nodes;");
+    em.line("if (v" + S(k) + ") xbytes += " + S(sh.x_bytes) + "u;");
+  }
   em.line("if (issuer) {");
-  em.line("  unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
-  em.line("  hdr[4 * st] = valid ? a : -1;");
-  em.line("  hdr[4 * st + 1] = (int)(pb - row_begin);");
-  em.line("  // 1: last edge of the row, 2: last edge of a chunk, 4: an earlier chunk was flushed");
-  em.line("  hdr[4 * st + 2] = (pe + 1 == pe1 ? 1 : ((pe + 1 - pr0) % E3_ROW_CHUNK == 0 ? 2 : 0)) |");
-  em.line("                    (pe - pr0 >= E3_ROW_CHUNK ? 4 : 0);");
-  em.line("  fence_async_smem();");
-  em.line("  bar_expect(bars + st, " + S(sh.s_bytes + sh.y_bytes) + "u + (valid ? " +
-          S(sh.x_bytes) + "u : 0u));");
-  em.line("  bulk_g2s(stg + " + S(sh.s_off) + ", s + (long long)(pe - e_base) * " + S(s_row) + ", " +
-          S(sh.s_bytes) + "u, bars + st, pol_stream);");
-  em.line("  bulk_g2s(stg + " + S(sh.y_off) + ", Y + (long long)(pe - e_base) * " +
-          S(sh.vec ? 4 : pl.ny) + ", " + S(sh.y_bytes) + "u, bars + st, pol_stream);");
-  em.line("  if (valid) bulk_g2s(stg + " + S(sh.x_off) + ", x + (long long)a * " +
-          S(static_cast<long long>(pl.nx) * pl.C) + ", " + S(sh.x_bytes) +
-          "u, bars + st, pol_keep);");
+  em.ind++;
+  for (int k = 0; k < G; ++k) {
+    em.line("{");
+    em.line("  const unsigned int st = g0 + " + S(k) + ";");
+    em.line("  const int ek = pe + " + S(k) + ";");
+    em.line("  hdr[4 * st] = " + S(k) + " < n ? (v" + S(k) + " ? a" + S(k) + " : -1) : -3;");
+    em.line("  hdr[4 * st + 1] = (int)(pb - row_begin);");
+    em.line("  // 1: last edge of the row, 2: last edge of a chunk, 4: an earlier chunk was flushed");
+    em.line("  hdr[4 * st + 2] = (ek + 1 == pe1 ? 1 : ((ek + 1 - pr0) % E3_ROW_CHUNK == 0 ? 2 : 0)) |");
+    em.line("                    (ek - pr0 >= E3_ROW_CHUNK ? 4 : 0);");
+    em.line("}");
+  }
+  em.line("fence_async_smem();");
+  em.line("unsigned long long* bar = bars + ppos % " + S(NG) + ";");
+  em.line("bar_expect(bar, (unsigned int)n * " + S(sh.s_bytes + sh.y_bytes) + "u + xbytes);");
+  em.line("bulk_g2s(" + s_at + "g0 * " + S(sh.s_bytes) + ", s + (long long)(pe - e_base) * " +
+          S(s_row) + ", (unsigned int)n * " + S(sh.s_bytes) + "u, bar, pol_stream);");
+  em.line("bulk_g2s(tbase + " + S(sh.y_off) + " + g0 * " + S(sh.y_bytes) + ", Y + (long long)(pe - e_base) * " +
+          S(sh.vec ? 4 : pl.ny) + ", (unsigned int)n * " + S(sh.y_bytes) + "u, bar, pol_stream);");
+  for (int k = 0; k < G; ++k)
+    em.line("if (v" + S(k) + ") bulk_g2s(tbase + " + S(sh.x_off) + " + (g0 + " + S(k) + ") * " +
+            S(sh.x_slot) + ", x + (long long)a" + S(k) + " * " +
+            S(static_cast<long long>(pl.nx) * pl.C) + ", " + S(sh.x_bytes) + "u, bar, pol_keep);");
+  em.ind--;
   em.line("}");
-  em.line("++pe;");
+  em.line("pe += n;");
   em.line("++ppos;");
   em.ind--;
   em.line("};");
-  em.line("for (int k = 0; k < " + S(NS) + "; ++k) produce();");
+  em.line("for (int k = 0; k < " + S(NG) + "; ++k) produce();");
   em.line("team_sync();");
   em.line("#pragma unroll 1");
   em.line("while (cpos != ppos) {");
   em.ind++;
-  em.line("const unsigned int st = cpos % " + S(NS) + ";");
-  em.line("if (!team_all(bar_wait(bars + st, (cpos / " + S(NS) + ") & 1u))) {");
+  em.line("const unsigned int g0 = (cpos % " + S(NG) + ") * " + S(G) + ";");
+  em.line("if (!team_all(bar_wait(bars + cpos % " + S(NG) + ", (cpos / " + S(NG) + ") & 1u))) {");
   em.line("  // bounded wait ran out: flag it, let the issuer drain its copies (bounded), stop");
   em.line("  if (issuer) {");
   em.line("    atomicOr(status, 4u);");
-  em.line("    for (unsigned int q = cpos; q != ppos; ++q) bar_wait(bars + q % " + S(NS) + ", (q / " + S(NS) + ") & 1u);");
+  em.line("    for (unsigned int q = cpos; q != ppos; ++q) bar_wait(bars + q % " + S(NG) + ", (q / " + S(NG) + ") & 1u);");
   em.line("  }");
   em.line("  return;");
   em.line("}");
-  em.line("const unsigned char* stg = tbase + st * " + S(sh.stage_bytes) + ";");
+  em.line("#pragma unroll 1");
+  em.line("for (int k = 0; k < " + S(G) + "; ++k) {");
+  em.ind++;
+  em.line("const unsigned int st = g0 + k;");
   em.line("const int a = hdr[4 * st];");
+  em.line("if (a == -3) break;  // the group's unused stages");
+  em.line("const unsigned char* stg_s = tbase + " + S(sh.s_off) + " + st * " + S(sh.s_bytes) + ";");
+  em.line("const unsigned char* stg_x = tbase + " + S(sh.x_off) + " + st * " + S(sh.x_slot) + ";");
+  em.line("const unsigned char* stg_y = tbase + " + S(sh.y_off) + " + st * " + S(sh.y_bytes) + ";");
   em.line("const long long b = hdr[4 * st + 1];");
   em.line("const int flags = hdr[4 * st + 2];");
   em.line("if (a >= 0) {");
@@ -1286,7 +1319,7 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
       em.ind++;
       em.line("float* yfw = reinterpret_cast<float*>(tbase + " + S(sh.yf_off) + " + tw * " +
               S(yf_bytes) + ");");
-      emit_yf_fill(em, pl, dtype, sh, "stg + " + S(sh.y_off), "lane", 32, "yfw");
+      emit_yf_fill(em, pl, dtype, sh, "stg_y", "lane", 32, "yfw");
       em.ind--;
       em.line("}");
       em.line("__syncwarp();");
@@ -1302,7 +1335,7 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
       em.line("{");
       em.ind++;
       em.line("float* yfw = reinterpret_cast<float*>(tbase + " + S(sh.yf_off) + ");");
-      emit_yf_fill(em, pl, dtype, sh, "stg + " + S(sh.y_off), "tl", 32 * TW, "yfw");
+      emit_yf_fill(em, pl, dtype, sh, "stg_y", "tl", 32 * TW, "yfw");
       em.ind--;
       em.line("}");
       em.line("team_sync();");
@@ -1310,14 +1343,14 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
     }
   } else {
     if (sh.vec) {
-      em.line("const float4 v_ = *reinterpret_cast<const float4*>(stg + " + S(sh.y_off) + ");");
+      em.line("const float4 v_ = *reinterpret_cast<const float4*>(stg_y);");
       emit_sh_eval(em, pl, "v_.x", "v_.y", "v_.z");
     } else {
-      em.line("const " + T + "* ys = reinterpret_cast<const " + T + "*>(stg + " + S(sh.y_off) + ");");
+      em.line("const " + T + "* ys = reinterpret_cast<const " + T + "*>(stg_y);");
       emit_y_load(em, pl, dtype, "lds", "ys");
     }
-    em.line("const " + T + "* xs = reinterpret_cast<const " + T + "*>(stg + " + S(sh.x_off) + ") + u0;");
-    em.line("const " + T + "* ss = reinterpret_cast<const " + T + "*>(stg + " + S(sh.s_off) + ") + u0;");
+    em.line("const " + T + "* xs = reinterpret_cast<const " + T + "*>(stg_x) + u0;");
+    em.line("const " + T + "* ss = reinterpret_cast<const " + T + "*>(stg_s) + u0;");
     emit_edge_body(em, pl, dtype, V, "lds", "xs", "ss");
   }
   em.ind--;
@@ -1345,6 +1378,8 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   em.ind--;
   em.line("}");
   em.line("team_sync();  // stage and A area free for reuse");
+  em.ind--;
+  em.line("}");
   em.line("++cpos;");
   em.line("produce();");
   em.ind--;

@@ -46,7 +46,9 @@ struct Shape {
   int stages = 0;
   int s_bytes = 0, x_bytes = 0, y_bytes = 0;  // row sizes staged per edge
   int s_off = 0, x_off = 0, y_off = 0;        // offsets inside one stage
-  int stage_bytes = 0;                        // one stage, 128-byte aligned
+  int stage_bytes = 0;                        // tensor cores: one stage; staged: the whole ring
+  int group = 1;                              // staged: edges per ring group (one s / Y copy each)
+  int x_slot = 0;                             // staged: bytes between sender rows of the ring
   int team = 1;                               // warps that share one receiver row (32*V*team = C)
   int warp_smem = 0;                          // shared memory of one team (ring, A, barriers)
   int bar_off = 0, hdr_off = 0;               // offsets inside a team's region
@@ -171,6 +173,7 @@ struct Plan {
   int auto_block = 0;                              // block chosen after a first compile (0: none)
   int req_coop = -1;                               // -1: automatic, 0: off, 1: on
   int req_tc = -1;                                 // -1: automatic, 0: off, 1: on
+  int req_group = -1;                              // -1: automatic, else edges per ring group (1..4)
   int req_alayout = -1;                            // -1: automatic, else Shape::amode (channel pairs only)
   int req_vec = 0;                                 // 1: edges given as vectors, Y computed in the kernel
   int req_psplit = -1;                             // -1: automatic, 0/1: off, k: split a row's paths over k warps

@@ -186,6 +186,12 @@ E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane,
  *   pairs in the order they are applied, read two per 16-byte load.
  *   Automatic: 1 with one channel pair per lane, else 0.  Same arithmetic. */
 #define E3CONV_OPT_A_LAYOUT 5
+/*   E3CONV_OPT_COPY_GROUP: -1 automatic (default: 1) or 1..4: the staged
+ *   variant's ring takes up to this many consecutive edges of a row per group,
+ *   with one bulk copy of their edge scalars, one of their harmonics and one
+ *   mbarrier per group (sender rows stay one copy each).  The ring depth is
+ *   rounded up to a multiple of the group.  Same arithmetic. */
+#define E3CONV_OPT_COPY_GROUP 6
 E3CONV_API int e3conv_set_option(e3conv_plan plan, int option, int value);
 
 /* The current value of an option (as set; -1 where automatic). */

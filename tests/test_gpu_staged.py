@@ -195,3 +195,32 @@ def test_path_split_is_bitwise_the_unsplit_kernel(cuda_device, split, C, dt):
     assert np.array_equal(a, b)
     ref = oracle_out(irreps, x, Y, s, send, recv, n, 12.0)
     assert column_scaled_error(b, ref) <= 1e-5
+
+
+@pytest.mark.parametrize("group,stages", [(2, -1), (3, 6), (4, 4), (2, 8)])
+@pytest.mark.parametrize("C,dt", [(128, "f16"), (64, "f32"), (32, "f32")])
+def test_copy_groups_are_bitwise_the_single_edge_ring(cuda_device, group, stages, C, dt):
+    # a ring group takes up to `group` consecutive edges of a row with one copy of their
+    # scalars and one of their harmonics; rows shorter than a group, empty rows, a long row
+    # and row ends inside a group leave the arithmetic unchanged
+    irreps = IRREPS[C]
+    rng = np.random.default_rng(10 * group + C + stages)
+    n, e = 800, 12000
+    send, recv = _graph(rng, n, e, empty_frac=0.1)
+    recv[:300] = 5
+    recv[300:303] = 6                      # a row of 3 edges
+    o = np.lexsort((send, recv))
+    send, recv = send[o], recv[o]
+    pl, x, Y, s = _inputs(rng, irreps, n, e, dt)
+    base = e3.Conv(*irreps, 9.0, dtype=dt)
+    base.set_copy_group(1)
+    grp = e3.Conv(*irreps, 9.0, dtype=dt)
+    grp.set_copy_group(group)
+    if stages != -1:
+        grp.set_launch_config(0, 0, stages)
+    assert f"copy_group={group}" in grp.kernel_source()
+    a = run_gpu(base, x, Y, s, send, recv, n)
+    b = run_gpu(grp, x, Y, s, send, recv, n)
+    assert np.array_equal(a, b)
+    ref = oracle_out(irreps, x, Y, s, send, recv, n, 9.0)
+    assert column_scaled_error(b, ref) <= 1e-5
