@@ -68,6 +68,10 @@ def parse_args():
                     help="1: the tensor-core forward variant (float16 inputs, 128 channels)")
     ap.add_argument("--exchange", choices=["allgather", "halo"], default="allgather",
                     help="multi-GPU: how a rank receives its senders' node features")
+    ap.add_argument("--direct-pipeline", type=int, default=-1,
+                    help="small channel counts: 1 loads the next edge during this edge's products")
+    ap.add_argument("--copy-group", type=int, default=-1,
+                    help="edges per ring group of the staged variant (1..4)")
     ap.add_argument("--a-layout", type=int, default=-1,
                     help="shared-memory layout of the contract-first A entries (0, 1, 2)")
     ap.add_argument("--radial", action="store_true",
@@ -365,6 +369,10 @@ def run_ours(args):
         conv.set_path_split(args.path_split)
     if args.a_layout != -1:
         conv.set_a_layout(args.a_layout)
+    if args.copy_group != -1:
+        conv.set_copy_group(args.copy_group)
+    if args.direct_pipeline != -1:
+        conv.set_direct_pipeline(args.direct_pipeline)
     if args.radial:
         # the edge scalars come from the radial MLP on the tensor cores every step
         if spec.scalars != "mlp":

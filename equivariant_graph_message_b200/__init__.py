@@ -59,6 +59,7 @@ OPT_PATH_SPLIT = 3
 OPT_EDGE_VECTORS = 4
 OPT_A_LAYOUT = 5
 OPT_COPY_GROUP = 6
+OPT_DIRECT_PIPELINE = 7
 _get_option = _sig("e3conv_get_option", ctypes.c_int, _vp, ctypes.c_int, _c_int_p)
 _sh_host = _sig("e3conv_spherical_harmonics", ctypes.c_int, _vp, ctypes.POINTER(ctypes.c_double),
                 ctypes.POINTER(ctypes.c_double))
@@ -234,6 +235,9 @@ class Conv:
 
     def set_path_split(self, value: int = -1):
         _ok(_set_option(self._h, OPT_PATH_SPLIT, value), "e3conv_set_option")
+
+    def set_direct_pipeline(self, value: int = -1):
+        _ok(_set_option(self._h, OPT_DIRECT_PIPELINE, value), "e3conv_set_option")
 
     def set_copy_group(self, value: int = -1):
         _ok(_set_option(self._h, OPT_COPY_GROUP, value), "e3conv_set_option")

@@ -480,9 +480,13 @@ int e3conv_set_option(e3conv_plan h, int option, int value) {
   Plan& pl = h->p;
   if (option != E3CONV_OPT_CONTRACT_FIRST && option != E3CONV_OPT_TENSOR_CORES &&
       option != E3CONV_OPT_PATH_SPLIT && option != E3CONV_OPT_EDGE_VECTORS &&
-      option != E3CONV_OPT_A_LAYOUT && option != E3CONV_OPT_COPY_GROUP)
+      option != E3CONV_OPT_A_LAYOUT && option != E3CONV_OPT_COPY_GROUP &&
+      option != E3CONV_OPT_DIRECT_PIPELINE)
     return fail(E3CONV_ERR_UNSUPPORTED, "unknown option");
-  if (option == E3CONV_OPT_COPY_GROUP) {
+  if (option == E3CONV_OPT_DIRECT_PIPELINE) {
+    if (value < -1 || value > 1) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1, 0 or 1");
+    pl.req_dpipe = value;
+  } else if (option == E3CONV_OPT_COPY_GROUP) {
     if (value != -1 && (value < 1 || value > 4)) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1 or 1 .. 4");
     pl.req_group = value;
   } else if (option == E3CONV_OPT_A_LAYOUT) {
@@ -519,6 +523,7 @@ int e3conv_get_option(e3conv_plan h, int option, int* value) {
     case E3CONV_OPT_EDGE_VECTORS: *value = pl.req_vec; return E3CONV_OK;
     case E3CONV_OPT_A_LAYOUT: *value = pl.req_alayout; return E3CONV_OK;
     case E3CONV_OPT_COPY_GROUP: *value = pl.req_group; return E3CONV_OK;
+    case E3CONV_OPT_DIRECT_PIPELINE: *value = pl.req_dpipe; return E3CONV_OK;
     default: return fail(E3CONV_ERR_UNSUPPORTED, "unknown option");
   }
 }

@@ -258,6 +258,9 @@ Shape choose_shape(const Plan& pl, int dtype) {
     s.ipw = 32 / lanes;
   }
   s.block = pl.req_block > 0 ? pl.req_block : 128;
+  // software-pipelined row walk when two register sets of one edge's inputs stay small
+  const int per_edge = (pl.nx + static_cast<int>(pl.paths.size())) * V + pl.ny;
+  s.dpipe = pl.req_dpipe == 1 || (pl.req_dpipe == -1 && per_edge <= 64);
   return s;
 }
 
@@ -473,7 +476,12 @@ void emit_edge_body(Emitter& em, const Plan& pl, int dtype, int V, const std::st
       std::string decl = "float";
       for (int v = 0; v < V; ++v) decl += std::string(v ? "," : "") + " x" + S(i) + "_" + S(v);
       em.line(decl + ";");
-      emit_vec_load(em, dtype, V, pre, xr + " + " + S((first.x_off + i) * pl.C), "x" + S(i));
+      if (pre == "reg") {  // values already in registers cx<comp>_<v> (software pipeline)
+        for (int v = 0; v < V; ++v)
+          em.line("x" + S(i) + "_" + S(v) + " = cx" + S(first.x_off + i) + "_" + S(v) + ";");
+      } else {
+        emit_vec_load(em, dtype, V, pre, xr + " + " + S((first.x_off + i) * pl.C), "x" + S(i));
+      }
     }
     for (size_t r = p; r < q; ++r) {
       const Path& P = pl.paths[r];
@@ -485,7 +493,11 @@ void emit_edge_body(Emitter& em, const Plan& pl, int dtype, int V, const std::st
         std::string decl = "float";
         for (int v = 0; v < V; ++v) decl += std::string(v ? "," : "") + " s_" + S(v);
         em.line(decl + ";");
-        emit_vec_load(em, dtype, V, pre, sr + " + " + S(static_cast<long long>(r) * pl.C), "s");
+        if (pre == "reg") {
+          for (int v = 0; v < V; ++v) em.line("s_" + S(v) + " = cs" + S(r) + "_" + S(v) + ";");
+        } else {
+          emit_vec_load(em, dtype, V, pre, sr + " + " + S(static_cast<long long>(r) * pl.C), "s");
+        }
       }
       std::map<std::pair<float, int>, std::string> cy;
       auto cyname = [&](const Nnz& n) -> std::string {
@@ -621,6 +633,91 @@ void emit_edge_range(Emitter& em) {
 // Only rows longer than one chunk take the extra read-add-write.
 void emit_chunk_define(Emitter& em) { em.line("#define E3_ROW_CHUNK 128"); }
 
+// Loads edge `ee`'s sender row (all nx components), harmonics and scalars (all
+// paths) into registers <p>x<comp>_<v>, <p>y<j>, <p>s<path>_<v> and the flag <p>ok.
+void emit_direct_edge_load(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
+                           const std::string& T, const std::string& ee, const std::string& p) {
+  const int V = sh.V;
+  em.line("{");
+  em.ind++;
+  em.line("const long long le_ = " + ee + " - e_base;");
+  em.line("const int a_ = senders[le_];");
+  em.line(p + "ok = (unsigned int)a_ < (unsigned int)num_nodes;");
+  em.line("if (!" + p + "ok) atomicOr(status, 2u);");
+  if (sh.vec) {
+    em.line("const float4 v_ = __ldg(reinterpret_cast<const float4*>(Y) + le_);");
+    emit_sh_eval(em, pl, "v_.x", "v_.y", "v_.z");
+  } else {
+    em.line("const " + T + "* yr_ = Y + le_ * " + S(pl.ny) + ";");
+    emit_y_load(em, pl, dtype, "ldg", "yr_");
+  }
+  for (int j = 0; j < pl.ny; ++j) em.line(p + "y" + S(j) + " = y" + S(j) + ";");
+  em.line("const " + T + "* xr_ = x + (long long)(" + p + "ok ? a_ : 0) * " + S(pl.nx * pl.C) + " + u0;");
+  for (int i = 0; i < pl.nx; ++i) {
+    std::string decl = "float";
+    for (int v = 0; v < V; ++v) decl += std::string(v ? "," : "") + " t" + S(i) + "_" + S(v);
+    em.line(decl + ";");
+    emit_vec_load(em, dtype, V, "ldg", "xr_ + " + S(i * pl.C), "t" + S(i));
+    for (int v = 0; v < V; ++v) em.line(p + "x" + S(i) + "_" + S(v) + " = t" + S(i) + "_" + S(v) + ";");
+  }
+  em.line("const " + T + "* sr_ = s + le_ * " + S(static_cast<long long>(pl.paths.size()) * pl.C) + " + u0;");
+  for (size_t r = 0; r < pl.paths.size(); ++r) {
+    std::string decl = "float";
+    for (int v = 0; v < V; ++v) decl += std::string(v ? "," : "") + " q" + S(r) + "_" + S(v);
+    em.line(decl + ";");
+    emit_vec_load(em, dtype, V, "ldg", "sr_ + " + S(static_cast<long long>(r) * pl.C), "q" + S(r));
+    for (int v = 0; v < V; ++v) em.line(p + "s" + S(r) + "_" + S(v) + " = q" + S(r) + "_" + S(v) + ";");
+  }
+  em.ind--;
+  em.line("}");
+}
+
+// The direct variant's row walk, software-pipelined: edge e+1's loads are issued
+// before edge e's products, into a second register set.
+void emit_direct_pipelined(Emitter& em, const Plan& pl, int dtype, const Shape& sh,
+                           const std::string& T) {
+  const int V = sh.V;
+  for (const char* p : {"c", "n"}) {
+    const std::string P(p);
+    std::string d = "float";
+    bool first = true;
+    for (int i = 0; i < pl.nx; ++i)
+      for (int v = 0; v < V; ++v) { d += std::string(first ? " " : ", ") + P + "x" + S(i) + "_" + S(v); first = false; }
+    for (size_t r = 0; r < pl.paths.size(); ++r)
+      for (int v = 0; v < V; ++v) d += ", " + P + "s" + S(r) + "_" + S(v);
+    for (int j = 0; j < pl.ny; ++j) d += ", " + P + "y" + S(j);
+    em.line(d + ";");
+    em.line("bool " + P + "ok = false;");
+  }
+  em.line("if (e0 < e1)");
+  emit_direct_edge_load(em, pl, dtype, sh, T, "e0", "c");
+  em.line("#pragma unroll 1");
+  em.line("for (int e = e0; e < e1; ++e) {");
+  em.ind++;
+  em.line("if (e > e0 && (e - e0) % E3_ROW_CHUNK == 0) {  // chunk of a long row done");
+  em.ind++;
+  emit_flush(em, pl, V, "orow", "e - e0 > E3_ROW_CHUNK", true);
+  em.ind--;
+  em.line("}");
+  em.line("if (e + 1 < e1)");
+  emit_direct_edge_load(em, pl, dtype, sh, T, "e + 1", "n");
+  em.line("if (cok) {");
+  em.ind++;
+  for (int j = 0; j < pl.ny; ++j) em.line("const float y" + S(j) + " = cy" + S(j) + ";");
+  emit_edge_body(em, pl, dtype, V, "reg", "", "");
+  em.ind--;
+  em.line("}");
+  // the next edge becomes the current one
+  for (int i = 0; i < pl.nx; ++i)
+    for (int v = 0; v < V; ++v) em.line("cx" + S(i) + "_" + S(v) + " = nx" + S(i) + "_" + S(v) + ";");
+  for (size_t r = 0; r < pl.paths.size(); ++r)
+    for (int v = 0; v < V; ++v) em.line("cs" + S(r) + "_" + S(v) + " = ns" + S(r) + "_" + S(v) + ";");
+  for (int j = 0; j < pl.ny; ++j) em.line("cy" + S(j) + " = ny" + S(j) + ";");
+  em.line("cok = nok;");
+  em.ind--;
+  em.line("}");
+}
+
 std::string direct_source(const Plan& pl, int dtype, const Shape& sh) {
   Emitter em;
   const int V = sh.V;
@@ -629,7 +726,8 @@ std::string direct_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("// generated by libe3conv: fused equivariant convolution forward (direct loads)");
   em.line("// C=" + S(pl.C) + " nx=" + S(pl.nx) + " ny=" + S(pl.ny) + " nout=" + S(pl.nout) +
           " paths=" + S(pl.paths.size()) + " dtype=" + (f16 ? "f16" : "f32") + " V=" + S(V) +
-          " TL=" + S(sh.TL) + " tiles=" + S(sh.tiles) + " ipw=" + S(sh.ipw));
+          " TL=" + S(sh.TL) + " tiles=" + S(sh.tiles) + " ipw=" + S(sh.ipw) +
+          " pipelined=" + S(sh.dpipe ? 1 : 0));
   emit_prelude(em);
   emit_chunk_define(em);
   emit_signature(em, T, sh.block, 0, sh.vec);
@@ -652,6 +750,13 @@ std::string direct_source(const Plan& pl, int dtype, const Shape& sh) {
   em.line("int e1 = row_ptr[b + 1];");
   em.line("if (e0 < e_base || e1 < e0 || e1 > e_end) { atomicOr(status, 1u); e1 = e0; }");
   em.line("float* orow = out + (b - row_begin) * " + S(pl.nout * pl.C) + " + u0;");
+  if (sh.dpipe) {
+    emit_direct_pipelined(em, pl, dtype, sh, T);
+    emit_flush(em, pl, V, "orow", "e1 - e0 > E3_ROW_CHUNK", false);
+    em.ind--;
+    em.line("}");
+    return em.o.str();
+  }
   em.line("#pragma unroll 1");
   em.line("for (int e = e0; e < e1; ++e) {");
   em.ind++;

@@ -42,6 +42,7 @@ struct Shape {
   int tiles = 1;   // channel tiles per receiver
   int ipw = 1;     // items per warp
   int block = 128; // threads per block
+  bool dpipe = false;  // direct variant: the next edge's inputs loaded during this edge's products
   // Staged (persistent, shared-memory ring) variant; stages == 0: direct loads.
   int stages = 0;
   int s_bytes = 0, x_bytes = 0, y_bytes = 0;  // row sizes staged per edge
@@ -173,6 +174,7 @@ struct Plan {
   int auto_block = 0;                              // block chosen after a first compile (0: none)
   int req_coop = -1;                               // -1: automatic, 0: off, 1: on
   int req_tc = -1;                                 // -1: automatic, 0: off, 1: on
+  int req_dpipe = -1;                              // -1: automatic, 0/1: direct-variant pipelining
   int req_group = -1;                              // -1: automatic, else edges per ring group (1..4)
   int req_alayout = -1;                            // -1: automatic, else Shape::amode (channel pairs only)
   int req_vec = 0;                                 // 1: edges given as vectors, Y computed in the kernel

@@ -192,6 +192,12 @@ E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane,
  *   mbarrier per group (sender rows stay one copy each).  The ring depth is
  *   rounded up to a multiple of the group.  Same arithmetic. */
 #define E3CONV_OPT_COPY_GROUP 6
+/*   E3CONV_OPT_DIRECT_PIPELINE: -1 automatic (default), 0 or 1: the direct
+ *   variant (small channel counts) loads the next edge's sender row,
+ *   harmonics and scalars into a second set of registers while the current
+ *   edge's products run.  Automatic: on when one edge's inputs take at most 64
+ *   values per lane.  Same arithmetic. */
+#define E3CONV_OPT_DIRECT_PIPELINE 7
 E3CONV_API int e3conv_set_option(e3conv_plan plan, int option, int value);
 
 /* The current value of an option (as set; -1 where automatic). */
