@@ -47,7 +47,7 @@ using namespace tc_host;
 
 constexpr int kTile = 128;           // edges per tile (MMA M)
 constexpr int kMaxBasis = 16;        // radial bases (layer 0 is unrolled over them)
-constexpr int kChunk = 128;          // output columns per output-layer chunk (MMA N)
+constexpr int kChunk = 64;           // output columns per output-layer chunk (MMA N)
 
 struct RadialArgs {
   const float* vec;        // [E][4] edge vectors (x, y, z, unused)
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
                      smem_u32(tslot))
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
   tc_after();
   const unsigned tmem = *tslot;
   const unsigned t_hid = tmem;                 // columns [0, H): hidden-layer D
-  // output-layer D: two buffers of 128 columns at 256 and 384
+  // output-layer D: two buffers of kChunk columns at 128 and 128 + kChunk
   const unsigned lane_off = static_cast<unsigned>(32 * warp) << 16;
   bool ok = true;
   // phase bits (bit b: buffer b) of the weight-chunk and output-MMA barriers
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
           const unsigned char* wlo = whi + L::kWout;
           for (int ks = 0; ks < H / 16; ++ks) {
             const int ao = ks * kTile * 32, bo = ks * kChunk * 32;
-            const unsigned td = tmem + 256u + 128u * buf;
+            const unsigned td = tmem + 128u + static_cast<unsigned>(kChunk) * buf;
             mma_f16(td, kmajor_desc(act + ao), kmajor_desc(whi + bo), id, ks > 0);
             mma_f16(td, kmajor_desc(act + ao), kmajor_desc(wlo + bo), id, 1);
             mma_f16(td, kmajor_desc(act + L::kAct + ao), kmajor_desc(whi + bo), id, 1);
@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
 #pragma unroll 1
         for (int j0 = 0; j0 < kChunk; j0 += 32) {
           float v[32];
-          tmem_ld32(tmem + 256u + 128u * pb + lane_off + j0, v);
+          tmem_ld32(tmem + 128u + static_cast<unsigned>(kChunk) * pb + lane_off + j0, v);
           if (valid) {
             const int cols = min(32, a.nout - (col0 + j0));
             if (cols > 0) {
@@ -309,15 +309,15 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
   __syncthreads();
   tc_after();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
 }
 
 }  // namespace
 
 int radial_prepare(RadialPlan& rp, int nb, double r_max, int hidden, int layers, const float* w0,
                    const float* const* wh, const float* wo, int nout, std::string& err) {
-  if (hidden != 64 && hidden != 32 && hidden != 128) {
-    err = "radial hidden width must be 32, 64 or 128";
+  if (hidden != 64 && hidden != 32) {
+    err = "radial hidden width must be 32 or 64";
     return E3CONV_ERR_UNSUPPORTED;
   }
   if (nb < 1 || nb > kMaxBasis || layers < 1 || layers > 4 || !(r_max > 0) || nout < 1) {
@@ -387,22 +387,20 @@ int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, 
   a.status = status;
   const size_t smem = radial_smem_bytes(rp);
   const long long tiles = (num_edges + kTile - 1) / kTile;
-  const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, grid));
-  cudaError_t e = cudaSuccess;
-  switch (rp.hidden) {
-    case 32:
-      e = cudaFuncSetAttribute(k_radial<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e == cudaSuccess) k_radial<32><<<blocks, 128, smem, st>>>(a);
-      break;
-    case 64:
-      e = cudaFuncSetAttribute(k_radial<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e == cudaSuccess) k_radial<64><<<blocks, 128, smem, st>>>(a);
-      break;
-    default:
-      e = cudaFuncSetAttribute(k_radial<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e == cudaSuccess) k_radial<128><<<blocks, 128, smem, st>>>(a);
-      break;
-  }
+  auto launch = [&](auto kernel) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    int per_sm = 0;
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 128, smem);
+    if (e != cudaSuccess || per_sm < 1) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+    // tensor memory: 256 columns per CTA, so at most two CTAs per SM
+    per_sm = std::min(per_sm, 2);
+    const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, static_cast<long long>(grid) * per_sm));
+    kernel<<<blocks, 128, smem, st>>>(a);
+    return cudaSuccess;
+  };
+  cudaError_t e = rp.hidden == 32 ? launch(k_radial<32>) : launch(k_radial<64>);
   if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) {
     err = "radial kernel launch failed";
     return E3CONV_ERR_CUDA;

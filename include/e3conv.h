@@ -184,7 +184,7 @@ E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane,
  *   0 float entries in the order they are formed (a lane duplicates each into
  *   a pair), 1 the entries stored as (a, a) pairs in that order, 2 (a, a)
  *   pairs in the order they are applied, read two per 16-byte load.
- *   Automatic: 1 with one channel pair per lane, else 0.  Same arithmetic. */
+ *   Automatic: 0.  Same arithmetic. */
 #define E3CONV_OPT_A_LAYOUT 5
 /*   E3CONV_OPT_COPY_GROUP: -1 automatic (default: 1) or 1..4: the staged
  *   variant's ring takes up to this many consecutive edges of a row per group,
@@ -316,7 +316,8 @@ E3CONV_API int e3conv_forward_rows(e3conv_plan plan, const void* node_features, 
  *   w0       [num_basis][hidden]
  *   w_hidden [layers-1][hidden][hidden] (NULL when layers == 1)
  *   w_out    [hidden][P*C], output column p*C + u = path p, channel u.
- * 1 <= num_basis <= 16, hidden in {32, 64, 128}, 1 <= layers <= 4, r_max > 0.
+ * 1 <= num_basis <= 16, hidden in {32, 64}, 1 <= layers <= 4, r_max > 0 (shared
+ * memory: up to three hidden-to-hidden layers at width 64).
  * Packs the weights and copies them to device memory the plan owns (this
  * call allocates; the radial calls below do not).  Replaces an earlier MLP. */
 E3CONV_API int e3conv_set_radial_mlp(e3conv_plan plan, int num_basis, double r_max, int hidden,

