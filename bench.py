@@ -77,6 +77,9 @@ def parse_args():
     ap.add_argument("--radial", action="store_true",
                     help="edge scalars from the radial MLP on the tensor cores every step "
                          "(workloads with MLP scalars)")
+    ap.add_argument("--next-rows", action="store_true",
+                    help="after the timed region, time the backward and the irreps linear layer "
+                         "on the same workload (supplementary entries with their rooflines)")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the supplementary timing of the tensor-core variant")
     return ap.parse_args()
@@ -605,6 +608,9 @@ def run_ours(args):
     }
     if variants is not None:
         line["variants"] = variants
+    if args.next_rows and world == 1:
+        line["next_rows"] = time_next_rows(args, spec, g, conv, x, Y, s, senders, receivers,
+                                           row_ptr, out, stream, pk)
     if radial is not None:
         line["radial"] = radial
         line["config"]["step"] = ("e3conv_build_csr + e3conv_radial_scalars + e3conv_forward "
@@ -614,6 +620,81 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def _event_ms(fn, reps, stream):
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+
+def time_next_rows(args, spec, g, conv, x, Y, s, senders, receivers, row_ptr, out, stream, pk):
+    """Supplementary, after the timed region, on the same resident inputs: the backward
+    (gradients of x, Y and s for a seeded upstream gradient) and the irreps linear layer on
+    the forward's output (the output irreps mixed C -> C); CUDA events, inputs larger than L2."""
+    import numpy as np
+    import torch
+
+    import equivariant_graph_message_b200 as e3
+    N, E = g.num_nodes, g.num_edges
+    res = {}
+    reps = max(3, min(args.steps, 10))
+    if not conv.edge_vectors and conv.C <= (256 if spec.dtype == "f16" else 128):
+        gout = torch.randn(out.shape, generator=torch.Generator(device=out.device).manual_seed(7),
+                           device=out.device)
+        srp, sperm, _ = e3.build_csr(senders, N)
+        conv.backward(x, Y, s, senders, row_ptr, gout, receivers=receivers,
+                      sender_row_ptr=srp, sender_perm=sperm)      # compile and warm up
+        torch.cuda.synchronize()
+        ms = _event_ms(lambda: conv.backward(x, Y, s, senders, row_ptr, gout, receivers=receivers,
+                                             sender_row_ptr=srp, sender_perm=sperm), reps, stream)
+        assert conv.check(), "backward reported a bad index"
+        b = 2 if spec.dtype == "f16" else 4
+        nnz = sum(int((np.abs(conv.cg(p)) > 1e-12).sum()) for p in range(conv.num_paths))
+        mix = sum(2 * q.l3 + 1 for q in conv.paths)
+        # edges kernel reads Y, s, senders, x rows, grad_out rows; writes grad_Y and grad_s (f32);
+        # nodes kernel reads Y, s, receivers, perm, grad_out rows; writes grad_x
+        nbytes = (2 * E * (conv.ny + conv.num_paths * conv.C) * b + 12 * E
+                  + E * (conv.ny + conv.num_paths * conv.C) * 4
+                  + N * (conv.nx * conv.C * b + 2 * 4 * conv.nout * conv.C + 4 * conv.nx * conv.C))
+        flops = 2 * E * conv.C * (4 * nnz + mix)
+        res["backward"] = {
+            "kernels": "e3conv_bwd_edges + e3conv_bwd_nodes", "ms": ms, "edges_per_s": E / (ms / 1e3),
+            "algorithmic_bytes": nbytes, "hbm_gbs": nbytes / (ms / 1e3) / 1e9,
+            "hbm_frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+            "fp32_flops": flops, "fp32_tflops": flops / (ms / 1e3) / 1e12,
+            "fp32_frac": flops / (ms / 1e3) / 1e12 / pk["fp32_tflops"],
+            "note": "definition FLOPs: grad_s and grad_Y (3 per CG nonzero and channel), grad_x (1), "
+                    "the s-scaling (one per output component); float32 accumulation"}
+        del gout, srp, sperm
+    irreps = "+".join(f"{conv.C}x{l}{'e' if p > 0 else 'o'}" for l, p, _ in conv.outputs)
+    if conv.C in (32, 64, 128):
+        lin = e3.IrrepsLinear(irreps, irreps, 1.0)
+        rng = np.random.default_rng(3)
+        lin.set_weights([rng.normal(size=(conv.C, conv.C)).astype(np.float32)
+                         for _ in range(lin.num_weight_blocks)])
+        yl = torch.empty_like(out)
+        flat = out.view(N, -1)
+        lin(flat, out=yl.view(N, -1))
+        torch.cuda.synchronize()
+        ms = _event_ms(lambda: lin(flat, out=yl.view(N, -1)), reps, stream)
+        assert lin.check()
+        nbytes = 2 * out.numel() * 4
+        flops = 3 * 2 * N * conv.nout * conv.C * conv.C
+        res["irreps_linear"] = {
+            "kernel": "k_linear", "irreps": irreps, "ms": ms, "algorithmic_bytes": nbytes,
+            "hbm_gbs": nbytes / (ms / 1e3) / 1e9, "hbm_frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+            "tensor_flops": flops, "tensor_tflops": flops / (ms / 1e3) / 1e12,
+            "note": "x read and y written once (HBM bound); tensor FLOPs count the three "
+                    "float16 hi/lo MMAs per product"}
+        del lin, yl
+    return res
 
 
 def time_tensor_core_variant(args, spec, g, conv, x, Y, s, senders, row_ptr, out, stream):

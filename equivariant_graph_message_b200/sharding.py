@@ -98,6 +98,9 @@ def shard_graph(row_ptr: np.ndarray, senders: np.ndarray, rank: int, world: int,
         local = own * block + (snd - bounds[own])
         return RowShard(rank, world, exchange, bounds, b0, b1, e0, e1, local_rp,
                         local.astype(np.int32), world * block, block)
+    if requests is None:
+        raise ValueError("the halo exchange needs `requests` (e.g. torch_requests()) to tell the "
+                         "owners which rows each rank needs")
     needed = np.unique(snd)
     own = _owner(bounds, needed)
     recv_counts = np.bincount(own, minlength=world).astype(np.int64)

@@ -180,3 +180,24 @@ def test_two_rank_sharding_equals_the_whole_graph():
 def test_single_rank_reduction_is_identity():
     (a, b), e = bench.reduce_over_ranks([1.5, 2.5], 123, 1)
     assert (a, b, e) == (1.5, 2.5, 123.0)
+
+
+def test_single_process_shards_cover_the_graph():
+    # without any process group: every rank's all-gather shard, built alone, renumbers its
+    # senders into the padded table consistently, and the ranks' edges tile the edge list
+    send, recv, rp = _graph(4, 200, 3000, hub=7)
+    world = 3
+    bounds = e3.partition_rows(rp.astype(np.int32), world)
+    e_seen = 0
+    for r in range(world):
+        sh = sharding.shard_graph(rp, send, r, world, "allgather", bounds=bounds)
+        assert sh.edge_begin == e_seen
+        e_seen = sh.edge_end
+        owner = np.searchsorted(bounds, send[sh.edge_begin:sh.edge_end], side="right") - 1
+        back = bounds[owner] + (sh.senders.astype(np.int64) - owner * sh.block_rows)
+        assert np.array_equal(back, send[sh.edge_begin:sh.edge_end])
+        assert sh.table_rows == world * sh.block_rows
+        assert np.array_equal(sh.row_ptr, rp[sh.row_begin:sh.row_end + 1] - rp[sh.row_begin])
+    assert e_seen == len(send)
+    with pytest.raises(ValueError):
+        sharding.shard_graph(rp, send, 0, world, "halo", bounds=bounds)    # no request exchange
