@@ -246,17 +246,39 @@ def calibrated_rows(spec, graph, x_rows_fn, Y_fn, s_fn, target_s, seed=2024):
         n = int(min(graph.num_nodes, n * min(8.0, max(2.0, 0.3 * target_s / max(dt, 1e-9)))))
 
 
-def device_inputs_fns(x_d, Y_d, s_d):
+def oracle_input_fns(spec, graph, x_dev=None, s_dev=None):
+    """Host inputs of an oracle sample, as functions of the rows / edges it takes: x and
+    drawn s from the seeded generator (read back from its device form when given: the
+    numpy form draws ~6M values/s), Y and radial s from the oracle's own harmonics and
+    radial MLP of the edge vectors, rounded to the workload dtype as the GPU's inputs are."""
+    import numpy as np
     import torch
 
+    import oracle
+    from workloads import configs
+    dt = configs.np_dtype(spec)
+
     def xf(rows):
-        return x_d[torch.from_numpy(rows).to(x_d.device)].cpu().numpy()
+        if x_dev is None:
+            return configs.node_features_np(spec, graph.num_nodes, rows)
+        return x_dev[torch.from_numpy(rows).to(x_dev.device)].cpu().numpy()
 
     def yf(edges):
-        return Y_d[torch.from_numpy(edges).to(Y_d.device)].cpu().numpy()
+        v = graph.vec[edges]
+        return oracle.sh(spec.lmax, v / np.linalg.norm(v, axis=1, keepdims=True)).astype(dt)
 
-    def sf(edges):
-        return s_d[torch.from_numpy(edges).to(s_d.device)].cpu().numpy()
+    if spec.scalars == "normal":
+        def sf(edges):
+            if s_dev is None:
+                return configs.scalars_np(spec, graph, edges)
+            return s_dev[torch.from_numpy(edges).to(s_dev.device)].cpu().numpy()
+    else:
+        ws = configs.radial_weights(spec)
+
+        def sf(edges):
+            d = np.linalg.norm(graph.vec[edges], axis=1)
+            s = oracle.radial_mlp(d, spec.graph["r"], ws)
+            return s.reshape(len(edges), spec.num_paths, spec.C).astype(dt)
     return xf, yf, sf
 
 
@@ -290,16 +312,14 @@ def run_reference(args):
     except ImportError:
         on_gpu = False
     if on_gpu:
-        # the inputs are drawn with the counter generator's device form and the sample's rows
-        # copied to the host (the numpy form runs at ~6M values/s); the oracle runs on the host
+        # the drawn inputs come from the counter generator's device form (faster than the
+        # numpy form); the harmonics and radial scalars from the oracle; it runs on the host
         dev = torch.device("cuda", 0)
-        xf, yf, sf = device_inputs_fns(configs.node_features_torch(spec, g.num_nodes, dev),
-                                       torch.from_numpy(configs.edge_sh(spec, g)).to(dev),
-                                       configs.scalars_torch(spec, g, dev))
+        xf, yf, sf = oracle_input_fns(
+            spec, g, configs.node_features_torch(spec, g.num_nodes, dev),
+            configs.scalars_torch(spec, g, dev) if spec.scalars == "normal" else None)
     else:
-        xf = lambda rows: configs.node_features_np(spec, g.num_nodes, rows)
-        yf = lambda edges: configs.real_sh(g.vec[edges], spec.lmax).astype(configs.np_dtype(spec))
-        sf = lambda edges: configs.scalars_np(spec, g, edges)
+        xf, yf, sf = oracle_input_fns(spec, g)
     per_step = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
     rows = calibrated_rows(spec, g, xf, yf, sf, per_step)
     prep = prepare_sample(g, rows, xf, yf, sf)    # inputs generated once; steps time the oracle
@@ -328,15 +348,20 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def edge_input(configs, spec, g, e0, e1, vectors):
-    """The forward's per-edge geometry for edges e0..e1-1: the harmonics [E][ny] in the
-    workload dtype, or the edge vectors as float32 [E][4] (x, y, z, 0)."""
-    import numpy as np
-    if vectors:
-        v = np.zeros((e1 - e0, 4), np.float32)
-        v[:, :3] = g.vec[e0:e1]
-        return v
-    return configs.real_sh(g.vec[e0:e1], spec.lmax).astype(configs.np_dtype(spec))
+def edge_inputs(conv, configs, spec, g, e0, e1, vectors, dev):
+    """The forward's per-edge operands for edges e0..e1-1 on the device: the harmonics
+    [E][ny] in the workload dtype (e3conv_edge_harmonics of the edge vectors), or the edge
+    vectors float32 [E][4] themselves; and the edge scalars, drawn, or the radial MLP of
+    the edge vectors (e3conv_radial_scalars with the workload's seeded weights)."""
+    import torch
+    v4 = torch.from_numpy(configs.edge_vectors_np(g, e0, e1)).to(dev)
+    Y = v4 if vectors else conv.edge_harmonics(v4)
+    if spec.scalars == "normal":
+        s = configs.scalars_torch(spec, g, dev, edges=(e0, e1))
+    else:
+        s = conv.radial_scalars(v4)
+    torch.cuda.synchronize()
+    return v4, Y, s
 
 
 def run_ours(args):
@@ -376,12 +401,13 @@ def run_ours(args):
         conv.set_copy_group(args.copy_group)
     if args.direct_pipeline != -1:
         conv.set_direct_pipeline(args.direct_pipeline)
-    if args.radial:
-        # the edge scalars come from the radial MLP on the tensor cores every step
-        if spec.scalars != "mlp":
-            raise SystemExit("--radial needs a workload whose scalars are the radial MLP (mace)")
+    if spec.scalars == "radial":
         conv.set_radial_mlp(spec.graph["r"], [w.astype(np.float32)
                                                for w in configs.radial_weights(spec)])
+    if args.radial:
+        # the edge scalars come from the radial MLP on the tensor cores every step
+        if spec.scalars != "radial":
+            raise SystemExit("--radial needs a workload whose scalars are the radial MLP (mace)")
         args.edge_vectors = 1
     if args.edge_vectors:
         conv.set_edge_vectors(1)
@@ -391,8 +417,7 @@ def run_ours(args):
     if world == 1:
         rows, E_loc = N, E
         x = configs.node_features_torch(spec, N, dev)
-        Y = torch.from_numpy(edge_input(configs, spec, g, 0, E, args.edge_vectors)).to(dev)
-        s = configs.scalars_torch(spec, g, dev)
+        _, Y, s = edge_inputs(conv, configs, spec, g, 0, E, args.edge_vectors, dev)
         senders = torch.from_numpy(g.senders.astype(np.int32)).to(dev)
         receivers = torch.from_numpy(g.receivers.astype(np.int32)).to(dev)
         table = x
@@ -417,8 +442,7 @@ def run_ours(args):
                                    device=dev)
         del own
         table = torch.empty((shard.table_rows, conv.nx, conv.C), dtype=x.dtype, device=dev)
-        Y = torch.from_numpy(edge_input(configs, spec, g, e0, e1, args.edge_vectors)).to(dev)
-        s = configs.scalars_torch(spec, g, dev, edges=(e0, e1))
+        _, Y, s = edge_inputs(conv, configs, spec, g, e0, e1, args.edge_vectors, dev)
         senders = torch.from_numpy(shard.senders).to(dev)
         receivers = torch.from_numpy((g.receivers[e0:e1] - b0).astype(np.int32)).to(dev)
     row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=dev)
@@ -556,7 +580,7 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
-        xf, yf, sf = device_inputs_fns(x, Y, s)
+        xf, yf, sf = oracle_input_fns(spec, g, x, s if spec.scalars == "normal" else None)
         sample_rows = calibrated_rows(spec, g, xf, yf, sf, args.cpu_seconds)
         rate, ne, dt = oracle_sample_rate(spec, g, sample_rows, xf, yf, sf)
         cpu = {"value": rate, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",

@@ -63,6 +63,7 @@ OPT_DIRECT_PIPELINE = 7
 _get_option = _sig("e3conv_get_option", ctypes.c_int, _vp, ctypes.c_int, _c_int_p)
 _sh_host = _sig("e3conv_spherical_harmonics", ctypes.c_int, _vp, ctypes.POINTER(ctypes.c_double),
                 ctypes.POINTER(ctypes.c_double))
+_edge_sh = _sig("e3conv_edge_harmonics", ctypes.c_int, _vp, _vp, _i64, _vp, _vp)
 _kernel_source = _sig("e3conv_kernel_source", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_char_p,
                       ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t))
 _forward = _sig("e3conv_forward", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp)
@@ -99,7 +100,7 @@ _version = _sig("e3conv_version", ctypes.c_int)
 
 EXPORTED = ["e3conv_create", "e3conv_destroy", "e3conv_set_input_dtype",
             "e3conv_set_launch_config", "e3conv_set_option", "e3conv_get_option",
-            "e3conv_spherical_harmonics", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
+            "e3conv_spherical_harmonics", "e3conv_edge_harmonics", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
             "e3conv_output_irrep", "e3conv_cg", "e3conv_kernel_info", "e3conv_kernel_source",
             "e3conv_forward", "e3conv_forward_rows", "e3conv_check", "e3conv_partition_rows",
             "e3conv_backward", "e3conv_prepare_backward", "e3conv_backward_source",
@@ -262,6 +263,22 @@ class Conv:
         _ok(_sh_host(self._h, v.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
                      out.ctypes.data_as(ctypes.POINTER(ctypes.c_double))),
             "e3conv_spherical_harmonics")
+        return out
+
+    def edge_harmonics(self, edge_vectors, out=None, stream=None):
+        """Y [E][ny] (plan dtype) from edge vectors float32 [E][4] on the device."""
+        import torch
+        _require("edge_vectors", edge_vectors, dtype=torch.float32)
+        E = edge_vectors.shape[0]
+        if tuple(edge_vectors.shape) != (E, 4):
+            raise ValueError("edge_vectors must be [E][4]")
+        want = torch.float16 if self.dtype == "f16" else torch.float32
+        if out is None:
+            out = torch.empty((E, self.ny), dtype=want, device=edge_vectors.device)
+        else:
+            _require("out", out, edge_vectors.device, want, E * self.ny)
+        _ok(_edge_sh(self._h, _ptr(edge_vectors) if E else None, E, _ptr(out) if E else None,
+                     _stream_handle(stream)), "e3conv_edge_harmonics")
         return out
 
     def kernel_info(self, dtype: str | None = None) -> dict:

@@ -52,7 +52,8 @@ def build(verbose: bool = False, jobs: int = 8) -> str:
             obj = os.path.join(tmp, s + ".o")
             cmd = [nvcc, "-c", src, "-o", obj, "-O3", "-std=c++17", "-Xcompiler", "-fPIC",
                    "-Xcompiler", "-fvisibility=hidden", "-lineinfo", *ARCH,
-                   "-I", os.path.join(CUDA_HOME, "include")]
+                   "-I", os.path.join(CUDA_HOME, "include"),
+                   '-DE3CONV_NVRTC_PATH="%s"' % os.path.join(CUDA_HOME, "lib64", "libnvrtc.so.12")]
             if verbose:
                 print(" ".join(cmd))
             procs.append(subprocess.Popen(cmd))
@@ -62,8 +63,7 @@ def build(verbose: bool = False, jobs: int = 8) -> str:
                 raise RuntimeError("nvcc failed while building libe3conv.so")
         out_tmp = LIB + ".tmp"
         cmd = [nvcc, "-shared", "-o", out_tmp, *objs, *ARCH, "-cudart", "static",
-               "-L", os.path.join(CUDA_HOME, "lib64"), "-lnvrtc",
-               "-Xlinker", "-rpath," + os.path.join(CUDA_HOME, "lib64"),
+               "-ldl",
                "-Xlinker", "--version-script=" + os.path.join(CSRC, "exports.map")]
         if verbose:
             print(" ".join(cmd))

@@ -1,6 +1,7 @@
 // C ABI of libe3conv: plans, NVRTC compilation, launches.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <dlfcn.h>
 #include <nvrtc.h>
 
 #include <algorithm>
@@ -91,65 +92,74 @@ bool has_device() {
   return n > 0;
 }
 
-int compile_once(Plan& pl, int dtype) {
-  Variant& v = pl.var[dtype];
-  v = Variant{};
-  v.shape = choose_shape(pl, dtype);
-  v.source = generate_forward_source(pl, dtype, v.shape);
-  nvrtcProgram prog;
-  if (nvrtcCreateProgram(&prog, v.source.c_str(), "e3conv_fwd.cu", 0, nullptr, nullptr) !=
-      NVRTC_SUCCESS)
-    return fail(E3CONV_ERR_COMPILE, "nvrtcCreateProgram failed");
-  const char* opts[] = {"--gpu-architecture=sm_100a", "--std=c++17", "-lineinfo",
-                        "--ptxas-options=-v"};
-  nvrtcResult rc = nvrtcCompileProgram(prog, 4, opts);
-  size_t log_size = 0;
-  nvrtcGetProgramLogSize(prog, &log_size);
-  v.log.assign(log_size, '\0');
-  if (log_size) nvrtcGetProgramLog(prog, &v.log[0]);
-  if (rc != NVRTC_SUCCESS) {
-    nvrtcDestroyProgram(&prog);
-    return fail(E3CONV_ERR_COMPILE, "NVRTC compile failed: " + v.log.substr(0, 2000));
-  }
-  size_t n = 0;
-  nvrtcGetCUBINSize(prog, &n);
-  v.cubin.resize(n);
-  nvrtcGetCUBIN(prog, v.cubin.data());
-  nvrtcDestroyProgram(&prog);
-  std::smatch m;
-  if (std::regex_search(v.log, m, std::regex("Used ([0-9]+) registers"))) v.regs = std::stoi(m[1]);
-  // Local memory per thread: the stack frame (what the loaded function reports as
-  // CU_FUNC_ATTRIBUTE_LOCAL_SIZE_BYTES), or the spill stores if ptxas reports more.
-  int stack = 0, spill = 0;
-  if (std::regex_search(v.log, m, std::regex("([0-9]+) bytes stack frame"))) stack = std::stoi(m[1]);
-  if (std::regex_search(v.log, m, std::regex("([0-9]+) bytes spill stores"))) spill = std::stoi(m[1]);
-  v.local_bytes = std::max(stack, spill);
-  v.compiled = true;
-  return E3CONV_OK;
+// NVRTC, loaded from the toolkit the library was built with (E3CONV_NVRTC_PATH) rather
+// than through the dynamic linker: a process may already hold another libnvrtc.so.12
+// (PyTorch ships its own), and the generated kernels must not depend on which one was
+// loaded first.  Falls back to the default search for libnvrtc.so.12.
+struct Nvrtc {
+  nvrtcResult (*CreateProgram)(nvrtcProgram*, const char*, const char*, int, const char* const*,
+                               const char* const*) = nullptr;
+  nvrtcResult (*CompileProgram)(nvrtcProgram, int, const char* const*) = nullptr;
+  nvrtcResult (*GetProgramLogSize)(nvrtcProgram, size_t*) = nullptr;
+  nvrtcResult (*GetProgramLog)(nvrtcProgram, char*) = nullptr;
+  nvrtcResult (*GetCUBINSize)(nvrtcProgram, size_t*) = nullptr;
+  nvrtcResult (*GetCUBIN)(nvrtcProgram, char*) = nullptr;
+  nvrtcResult (*DestroyProgram)(nvrtcProgram*) = nullptr;
+  nvrtcResult (*Version)(int*, int*) = nullptr;
+  bool ok = false;
+};
+
+#ifndef E3CONV_NVRTC_PATH
+#define E3CONV_NVRTC_PATH "libnvrtc.so.12"
+#endif
+
+Nvrtc& nvrtc() {
+  static Nvrtc n;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* h = dlopen(E3CONV_NVRTC_PATH, RTLD_NOW | RTLD_LOCAL);
+    if (!h) h = dlopen("libnvrtc.so.12", RTLD_NOW | RTLD_LOCAL);
+    if (!h) return;
+    auto get = [h](const char* name, auto** fn) {
+      *reinterpret_cast<void**>(fn) = dlsym(h, name);
+      return *fn != nullptr;
+    };
+    n.ok = get("nvrtcCreateProgram", &n.CreateProgram) &&
+           get("nvrtcCompileProgram", &n.CompileProgram) &&
+           get("nvrtcGetProgramLogSize", &n.GetProgramLogSize) &&
+           get("nvrtcGetProgramLog", &n.GetProgramLog) &&
+           get("nvrtcGetCUBINSize", &n.GetCUBINSize) && get("nvrtcGetCUBIN", &n.GetCUBIN) &&
+           get("nvrtcDestroyProgram", &n.DestroyProgram) && get("nvrtcVersion", &n.Version);
+  });
+  return n;
 }
 
-// NVRTC compile of `source` for sm_100a; fills cubin, log, registers and local bytes.
+// NVRTC compile of `source` for sm_100a; fills cubin, log, registers and local bytes
+// (per thread: the stack frame, which is what the loaded function reports as
+// CU_FUNC_ATTRIBUTE_LOCAL_SIZE_BYTES, or the spill stores if ptxas reports more).
 int nvrtc_compile(const std::string& source, const char* name, std::vector<char>& cubin,
                   std::string& log, int& regs, int& local_bytes) {
+  Nvrtc& nv = nvrtc();
+  if (!nv.ok) return fail(E3CONV_ERR_COMPILE, "cannot load NVRTC (" E3CONV_NVRTC_PATH ")");
   nvrtcProgram prog;
-  if (nvrtcCreateProgram(&prog, source.c_str(), name, 0, nullptr, nullptr) != NVRTC_SUCCESS)
+  if (nv.CreateProgram(&prog, source.c_str(), name, 0, nullptr, nullptr) != NVRTC_SUCCESS)
     return fail(E3CONV_ERR_COMPILE, "nvrtcCreateProgram failed");
   const char* opts[] = {"--gpu-architecture=sm_100a", "--std=c++17", "-lineinfo",
                         "--ptxas-options=-v"};
-  nvrtcResult rc = nvrtcCompileProgram(prog, 4, opts);
+  nvrtcResult rc = nv.CompileProgram(prog, 4, opts);
   size_t log_size = 0;
-  nvrtcGetProgramLogSize(prog, &log_size);
+  nv.GetProgramLogSize(prog, &log_size);
   log.assign(log_size, '\0');
-  if (log_size) nvrtcGetProgramLog(prog, &log[0]);
+  if (log_size) nv.GetProgramLog(prog, &log[0]);
   if (rc != NVRTC_SUCCESS) {
-    nvrtcDestroyProgram(&prog);
+    nv.DestroyProgram(&prog);
     return fail(E3CONV_ERR_COMPILE, "NVRTC compile failed: " + log.substr(0, 2000));
   }
   size_t n = 0;
-  nvrtcGetCUBINSize(prog, &n);
+  nv.GetCUBINSize(prog, &n);
   cubin.resize(n);
-  nvrtcGetCUBIN(prog, cubin.data());
-  nvrtcDestroyProgram(&prog);
+  nv.GetCUBIN(prog, cubin.data());
+  nv.DestroyProgram(&prog);
   std::smatch m;
   regs = -1;
   if (std::regex_search(log, m, std::regex("Used ([0-9]+) registers"))) regs = std::stoi(m[1]);
@@ -157,6 +167,17 @@ int nvrtc_compile(const std::string& source, const char* name, std::vector<char>
   if (std::regex_search(log, m, std::regex("([0-9]+) bytes stack frame"))) stack = std::stoi(m[1]);
   if (std::regex_search(log, m, std::regex("([0-9]+) bytes spill stores"))) spill = std::stoi(m[1]);
   local_bytes = std::max(stack, spill);
+  return E3CONV_OK;
+}
+
+int compile_once(Plan& pl, int dtype) {
+  Variant& v = pl.var[dtype];
+  v = Variant{};
+  v.shape = choose_shape(pl, dtype);
+  v.source = generate_forward_source(pl, dtype, v.shape);
+  const int rc = nvrtc_compile(v.source, "e3conv_fwd.cu", v.cubin, v.log, v.regs, v.local_bytes);
+  if (rc != E3CONV_OK) return rc;
+  v.compiled = true;
   return E3CONV_OK;
 }
 
@@ -429,6 +450,8 @@ void e3conv_destroy(e3conv_plan h) {
     DeviceGuard g(pl.device);
     for (auto& v : pl.var) release_variant(v);
     for (auto& v : pl.bwd) release_backward(v);
+    for (auto& v : pl.shk)
+      if (v.module) driver().ModuleUnload(v.module);
     if (pl.status) cudaFree(pl.status);
     for (void* q : {pl.radial.d_w0, pl.radial.d_wh, pl.radial.d_wo})
       if (q) cudaFree(q);
@@ -545,6 +568,53 @@ int e3conv_spherical_harmonics(e3conv_plan h, const double* vec, double* out) {
       v += m.coef * std::pow(u[0], m.px) * std::pow(u[1], m.py) * std::pow(u[2], m.pz);
     out[j] = v;
   }
+  return E3CONV_OK;
+}
+
+int e3conv_edge_harmonics(e3conv_plan h, const float* edge_vectors, int64_t num_edges,
+                          void* edge_sh, e3conv_stream stream) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  Plan& pl = h->p;
+  if (num_edges < 0) return fail(E3CONV_ERR_INVALID_ARG, "num_edges < 0");
+  if (num_edges == 0) return E3CONV_OK;
+  if (!edge_vectors || !edge_sh) return fail(E3CONV_ERR_INVALID_ARG, "NULL buffer");
+  if (!aligned16(edge_vectors) || !aligned16(edge_sh))
+    return fail(E3CONV_ERR_INVALID_ARG, "edge_vectors and edge_sh must be 16-byte aligned");
+  // generated and compiled on the first call (also without a device, so a host can
+  // check the kernel builds); loaded once a device is there
+  ShVariant& v = pl.shk[pl.dtype];
+  if (v.cubin.empty()) {
+    ShVariant n;
+    n.source = generate_sh_source(pl, pl.dtype);
+    int rc = nvrtc_compile(n.source, "e3conv_edge_sh.cu", n.cubin, n.log, n.regs, n.local_bytes);
+    if (rc != E3CONV_OK) return rc;
+    v = n;
+  }
+  if (pl.device < 0) return fail(E3CONV_ERR_NO_DEVICE, "plan has no device");
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess || cur != pl.device)
+    return fail(E3CONV_ERR_INVALID_ARG, "current device differs from the plan's device");
+  if (!v.compiled) {
+    Driver& d = driver();
+    if (d.ModuleLoadData(&v.module, v.cubin.data()) != CUDA_SUCCESS)
+      return fail(E3CONV_ERR_CUDA, "cuModuleLoadData failed (harmonics)");
+    if (d.ModuleGetFunction(&v.fn, v.module, "e3conv_edge_sh") != CUDA_SUCCESS) {
+      d.ModuleUnload(v.module);
+      v.module = nullptr;
+      return fail(E3CONV_ERR_CUDA, "cuModuleGetFunction failed (harmonics)");
+    }
+    v.compiled = true;
+  }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, pl.device) != cudaSuccess)
+    return fail(E3CONV_ERR_CUDA, "cannot query the SM count");
+  const long long need = (num_edges + 255) / 256;
+  const long long blocks = std::min<long long>(need, static_cast<long long>(sms) * 8);
+  long long ne = num_edges;
+  void* args[] = {const_cast<float**>(&edge_vectors), &ne, &edge_sh};
+  if (driver().LaunchKernel(v.fn, static_cast<unsigned>(blocks), 1, 1, 256, 1, 1, 0,
+                            reinterpret_cast<CUstream>(stream), args, nullptr) != CUDA_SUCCESS)
+    return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed (harmonics)");
   return E3CONV_OK;
 }
 

@@ -2189,6 +2189,49 @@ std::string generate_backward_source(const Plan& pl, int dtype, const BwdShape& 
   return nodes ? bwd_nodes_source(pl, dtype, b) : bwd_edges_source(pl, dtype, b);
 }
 
+// Standalone harmonics: one thread per edge evaluates the plan's polynomials of
+// v / |v| (emit_sh_eval, as the forward does with edge vectors) and stores the row in
+// the input dtype; 16-byte stores where the row length allows.
+std::string generate_sh_source(const Plan& pl, int dtype) {
+  Emitter em;
+  const bool f16 = dtype == E3CONV_F16;
+  const std::string T = f16 ? "unsigned short" : "float";
+  em.line("// generated by libe3conv: real spherical harmonics of edge vectors");
+  em.line("// lmax=" + S(pl.lmax) + " ny=" + S(pl.ny) + " dtype=" + (f16 ? "f16" : "f32"));
+  em.line("__device__ __forceinline__ unsigned short f2h(float f) { unsigned short h; "
+          "asm(\"cvt.rn.f16.f32 %0, %1;\" : \"=h\"(h) : \"f\"(f)); return h; }");
+  em.line("__device__ __forceinline__ unsigned int pkh(float a, float b) { "
+          "return static_cast<unsigned int>(f2h(a)) | (static_cast<unsigned int>(f2h(b)) << 16); }");
+  em.line("extern \"C\" __global__ void __launch_bounds__(256) e3conv_edge_sh(const float4* "
+          "__restrict__ vec, long long num_edges, " + T + "* __restrict__ out) {");
+  em.ind++;
+  em.line("for (long long e = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; e < num_edges;"
+          " e += static_cast<long long>(gridDim.x) * 256) {");
+  em.ind++;
+  em.line("const float4 v_ = __ldg(vec + e);");
+  emit_sh_eval(em, pl, "v_.x", "v_.y", "v_.z");
+  em.line(T + "* o_ = out + e * " + S(pl.ny) + ";");
+  auto y = [](int j) { return "y" + S(j); };
+  if (!f16 && pl.ny % 4 == 0) {
+    for (int j = 0; j < pl.ny; j += 4)
+      em.line("reinterpret_cast<float4*>(o_)[" + S(j / 4) + "] = make_float4(" + y(j) + ", " +
+              y(j + 1) + ", " + y(j + 2) + ", " + y(j + 3) + ");");
+  } else if (f16 && pl.ny % 8 == 0) {
+    for (int j = 0; j < pl.ny; j += 8)
+      em.line("reinterpret_cast<uint4*>(o_)[" + S(j / 8) + "] = make_uint4(pkh(" + y(j) + ", " +
+              y(j + 1) + "), pkh(" + y(j + 2) + ", " + y(j + 3) + "), pkh(" + y(j + 4) + ", " +
+              y(j + 5) + "), pkh(" + y(j + 6) + ", " + y(j + 7) + "));");
+  } else {
+    for (int j = 0; j < pl.ny; ++j)
+      em.line("o_[" + S(j) + "] = " + (f16 ? "f2h(" + y(j) + ")" : y(j)) + ";");
+  }
+  em.ind--;
+  em.line("}");
+  em.ind--;
+  em.line("}");
+  return em.o.str();
+}
+
 std::string generate_forward_source(const Plan& pl, int dtype, const Shape& sh) {
   if (sh.tc) return tc_source(pl, sh);
   return sh.stages > 0 ? staged_source(pl, dtype, sh) : direct_source(pl, dtype, sh);

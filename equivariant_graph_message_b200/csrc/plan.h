@@ -109,6 +109,16 @@ struct BwdVariant {
   int regs[2] = {-1, -1}, local_bytes[2] = {-1, -1};
 };
 
+struct ShVariant {  // standalone harmonics kernel (compiled on first use)
+  bool compiled = false;
+  std::string source;
+  std::vector<char> cubin;
+  std::string log;
+  CUmodule module = nullptr;
+  CUfunction fn = nullptr;
+  int regs = -1, local_bytes = -1;
+};
+
 struct Variant {
   bool compiled = false;
   Shape shape;
@@ -186,6 +196,7 @@ struct Plan {
   unsigned int* status = nullptr;  // device status word
   Variant var[2];
   BwdVariant bwd[2];               // backward kernels per input dtype (compiled on first use)
+  ShVariant shk[2];                // standalone harmonics kernel per input dtype
   RadialPlan radial;
 };
 
@@ -221,6 +232,7 @@ Shape choose_shape(const Plan& plan, int dtype);
 std::string generate_forward_source(const Plan& plan, int dtype, const Shape& shape);
 BwdShape choose_backward_shape(const Plan& plan, int dtype);
 std::string generate_backward_source(const Plan& plan, int dtype, const BwdShape& shape, bool nodes);
+std::string generate_sh_source(const Plan& plan, int dtype);
 
 }  // namespace e3c
 

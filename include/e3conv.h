@@ -208,6 +208,16 @@ E3CONV_API int e3conv_get_option(e3conv_plan plan, int option, int* value);
  * out[ny]; a zero vector gives 1, 0, 0, ... */
 E3CONV_API int e3conv_spherical_harmonics(e3conv_plan plan, const double* vec, double* out);
 
+/* edge_sh[e] = Y(edge_vectors[e]) for e < num_edges (device): the polynomials
+ * of e3conv_spherical_harmonics, evaluated in float32 and stored in the plan's
+ * input dtype as the forward's edge_sh operand, [num_edges][ny].
+ * edge_vectors float32 [num_edges][4] (x, y, z, ignored).  Both buffers
+ * 16-byte aligned.  The first call compiles the kernel (NVRTC) and loads it;
+ * every call is one launch on `stream` with no allocation and no host
+ * synchronisation.  num_edges == 0 launches nothing (NULL buffers allowed). */
+E3CONV_API int e3conv_edge_harmonics(e3conv_plan plan, const float* edge_vectors, int64_t num_edges,
+                                     void* edge_sh, e3conv_stream stream);
+
 /* Sizes: C channels, nx node components, ny edge components, nout output
  * components, num_paths P.  Any pointer may be NULL. */
 E3CONV_API int e3conv_query(e3conv_plan plan, int* C, int* nx, int* ny, int* nout, int* num_paths);

@@ -13,10 +13,33 @@ import torch
 
 import equivariant_graph_message_b200 as e3
 import oracle
-from workloads import SPECS, edge_sh, make_graph, node_features_np, node_features_torch, \
+from workloads import SPECS, make_graph, node_features_np, node_features_torch, radial_weights, \
     scalars_np, scalars_torch
+from workloads.configs import np_dtype
 
 TOL = {"f32": 1e-5, "f16": 5e-3}
+
+
+def edge_sh(spec, graph, edges=None) -> np.ndarray:
+    """Y [E][ny] in the workload dtype: the oracle's harmonics of the edge vectors."""
+    v = graph.vec if edges is None else graph.vec[np.asarray(edges)]
+    u = v / np.linalg.norm(v, axis=1, keepdims=True)
+    return oracle.sh(spec.lmax, u).astype(np_dtype(spec))
+
+
+def edge_scalars(spec, graph, edges=None) -> np.ndarray:
+    """s [E][P][C] in the workload dtype: drawn, or the oracle's radial MLP of the edge
+    lengths with the workload's seeded weights."""
+    if spec.scalars == "normal":
+        return scalars_np(spec, graph, edges)
+    v = graph.vec if edges is None else graph.vec[np.asarray(edges)]
+    s = oracle.radial_mlp(np.linalg.norm(v, axis=1), spec.graph["r"], radial_weights(spec))
+    return s.reshape(len(v), spec.num_paths, spec.C).astype(np_dtype(spec))
+
+
+def workload_inputs(spec, graph):
+    """(x, Y, s) of a workload on the host, in its dtype."""
+    return node_features_np(spec, graph.num_nodes), edge_sh(spec, graph), edge_scalars(spec, graph)
 
 
 def column_scaled_error(gpu: np.ndarray, ref: np.ndarray) -> float:
@@ -96,7 +119,8 @@ class DeviceWorkload:
         tdt = torch.float16 if spec.dtype == "f16" else torch.float32
         self.x = node_features_torch(spec, g.num_nodes, device)
         self.Y = torch.from_numpy(edge_sh(spec, g)).to(device)
-        self.s = scalars_torch(spec, g, device)
+        self.s = scalars_torch(spec, g, device) if spec.scalars == "normal" else \
+            torch.from_numpy(edge_scalars(spec, g)).to(device)
         self.senders = torch.from_numpy(g.senders.astype(np.int32)).to(device)
         self.receivers = torch.from_numpy(g.receivers.astype(np.int32)).to(device)
         self.row_ptr = torch.from_numpy(row_ptr_of(g.receivers, g.num_nodes).astype(np.int32)).to(device)

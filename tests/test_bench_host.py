@@ -43,9 +43,7 @@ def test_peaks_are_positive_and_consistent():
 def test_cpu_baseline_sample_is_seeded_and_bounded():
     spec = configs.SPECS["tiny"]
     g = configs.make_graph(spec)
-    pl_x = lambda rows: configs.node_features_np(spec, g.num_nodes, rows)
-    yf = lambda edges: configs.real_sh(g.vec[edges], spec.lmax).astype(configs.np_dtype(spec))
-    sf = lambda edges: configs.scalars_np(spec, g, edges)
+    pl_x, yf, sf = bench.oracle_input_fns(spec, g)
     a = bench.calibrated_rows(spec, g, pl_x, yf, sf, 0.05)
     b = bench.calibrated_rows(spec, g, pl_x, yf, sf, 0.05)
     assert len(a) >= 1 and np.all(np.diff(a) > 0) and a[-1] < g.num_nodes

@@ -9,8 +9,8 @@ import torch
 
 import equivariant_graph_message_b200 as e3
 import oracle
-from parity import column_scaled_error, row_ptr_of, to_dev
-from workloads import SPECS, edge_sh, make_graph, node_features_np, scalars_np
+from parity import column_scaled_error, row_ptr_of, to_dev, workload_inputs
+from workloads import SPECS, make_graph
 
 pytestmark = pytest.mark.gpu
 
@@ -40,7 +40,7 @@ def _check(got, ref, tol):
 def test_backward_full_graphs(cuda_device, name):
     spec = SPECS[name]
     g = make_graph(spec)
-    x, Y, s = node_features_np(spec, g.num_nodes), edge_sh(spec, g), scalars_np(spec, g)
+    x, Y, s = workload_inputs(spec, g)
     irreps = (spec.irreps_node, spec.irreps_sh, spec.irreps_out)
     conv = e3.Conv(*irreps, g.avg_num_neighbors, dtype=spec.dtype)
     pl = oracle.plan(*irreps)
@@ -55,7 +55,7 @@ def test_backward_full_graphs(cuda_device, name):
 def test_backward_large_irreps(cuda_device, name):
     spec = SPECS[name]
     g = make_graph(spec, 1500)
-    x, Y, s = node_features_np(spec, g.num_nodes), edge_sh(spec, g), scalars_np(spec, g)
+    x, Y, s = workload_inputs(spec, g)
     irreps = (spec.irreps_node, spec.irreps_sh, spec.irreps_out)
     conv = e3.Conv(*irreps, g.avg_num_neighbors, dtype=spec.dtype)
     pl = oracle.plan(*irreps)

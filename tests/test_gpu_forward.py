@@ -6,8 +6,8 @@ import torch
 import equivariant_graph_message_b200 as e3
 import oracle
 from parity import TOL, DeviceWorkload, abs_bound, column_scaled_error, oracle_out, row_ptr_of, \
-    run_gpu, to_dev
-from workloads import SPECS, edge_sh, make_graph, node_features_np, scalars_np
+    run_gpu, to_dev, workload_inputs
+from workloads import SPECS, make_graph
 
 pytestmark = pytest.mark.gpu
 
@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 def _spec_inputs(name):
     spec = SPECS[name]
     g = make_graph(spec)
-    return spec, g, node_features_np(spec, g.num_nodes), edge_sh(spec, g), scalars_np(spec, g)
+    return (spec, g) + workload_inputs(spec, g)
 
 
 @pytest.mark.parametrize("name", ["tiny", "gate_points", "mace"])

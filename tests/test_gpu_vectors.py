@@ -10,8 +10,9 @@ import torch
 
 import equivariant_graph_message_b200 as e3
 import oracle
-from parity import TOL, DeviceWorkload, column_scaled_error, oracle_out, row_ptr_of, to_dev
-from workloads import SPECS, make_graph, node_features_np, scalars_np
+from parity import TOL, DeviceWorkload, column_scaled_error, edge_scalars, oracle_out, row_ptr_of, \
+    to_dev
+from workloads import SPECS, make_graph, node_features_np
 
 pytestmark = pytest.mark.gpu
 
@@ -46,7 +47,7 @@ def test_edge_vectors_full_graphs(cuda_device, name):
     spec = SPECS[name]
     g = make_graph(spec)
     x = node_features_np(spec, g.num_nodes)
-    s = scalars_np(spec, g)
+    s = edge_scalars(spec, g)
     v4 = _vec4(g.vec)
     irreps = (spec.irreps_node, spec.irreps_sh, spec.irreps_out)
     conv = e3.Conv(*irreps, g.avg_num_neighbors, dtype=spec.dtype)
@@ -126,3 +127,52 @@ def test_edge_vectors_full_size_sampled(cuda_device, name):
     assert column_scaled_error(gpu, ref) <= TOL[w.spec.dtype]
     del w, out, v4
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16"])
+@pytest.mark.parametrize("lmax", [0, 1, 2, 3, 6])
+def test_standalone_harmonics_match_the_oracle(cuda_device, lmax, dt):
+    # e3conv_edge_harmonics: the forward's edge_sh operand from edge vectors, against the
+    # oracle's float64 harmonics of the same float32 vectors (a zero vector, widely varying
+    # lengths, more edges than one grid pass covers); float32 evaluation within 1e-5 of the
+    # largest component, float16 storage within half an ulp of float16 more
+    irreps = ("8x0e", "+".join(f"1x{l}{'eo'[l % 2]}" for l in range(lmax + 1)), "8x0e")
+    conv = e3.Conv(*irreps, 1.0, dtype=dt)
+    rng = np.random.default_rng(10 * lmax + (dt == "f16"))
+    e = 148 * 8 * 256 + 1234
+    vec = rng.normal(size=(e, 3)) * rng.uniform(1e-3, 1e3, size=(e, 1))
+    vec[7] = 0.0
+    v4 = _vec4(vec)
+    got = conv.edge_harmonics(to_dev(v4)).float().cpu().numpy()
+    assert conv.check()
+    ref = _oracle_sh(lmax, v4)
+    scale = np.sqrt(2 * lmax + 1) * (2.0 if lmax else 1.0)
+    tol = 1e-5 * scale + (2.0 ** -11 * np.abs(ref) if dt == "f16" else 0.0)
+    assert np.all(np.abs(got - ref) <= tol)
+    assert got.shape == (e, (lmax + 1) ** 2)
+    assert conv.edge_harmonics(torch.zeros((0, 4), device="cuda")).shape == (0, (lmax + 1) ** 2)
+
+
+def test_standalone_harmonics_feed_the_forward(cuda_device):
+    # Y from the harmonics kernel fed to the forward, and the forward that evaluates the same
+    # polynomials from the vectors itself: both within the float32 bar of the oracle
+    spec = SPECS["mace"]
+    g = make_graph(spec)
+    x = node_features_np(spec, g.num_nodes)
+    s = edge_scalars(spec, g)
+    irreps = (spec.irreps_node, spec.irreps_sh, spec.irreps_out)
+    v4 = to_dev(_vec4(g.vec))
+    a = e3.Conv(*irreps, g.avg_num_neighbors, dtype="f32")
+    Y = a.edge_harmonics(v4)
+    rp = to_dev(row_ptr_of(g.receivers, g.num_nodes).astype(np.int32))
+    snd = to_dev(g.senders.astype(np.int32))
+    out_y = a.forward(to_dev(x), Y, to_dev(s), snd, rp)
+    b = e3.Conv(*irreps, g.avg_num_neighbors, dtype="f32")
+    b.set_edge_vectors(1)
+    out_v = b.forward(to_dev(x), v4, to_dev(s), snd, rp)
+    torch.cuda.synchronize()
+    assert a.check() and b.check()
+    ref = oracle_out(irreps, x, _oracle_sh(spec.lmax, _vec4(g.vec)), s, g.senders, g.receivers,
+                     g.num_nodes, g.avg_num_neighbors)
+    assert column_scaled_error(out_y.cpu().numpy(), ref) <= TOL["f32"]
+    assert column_scaled_error(out_v.cpu().numpy(), ref) <= TOL["f32"]

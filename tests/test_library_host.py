@@ -395,6 +395,20 @@ def test_edge_vector_kernels_compile_for_every_workload(name):
     assert "sqrtf(r2_)" in src and "const float* __restrict__ Y" in src
 
 
+@pytest.mark.parametrize("dtype", ["f32", "f16"])
+@pytest.mark.parametrize("lmax", [0, 1, 2, 3, 4])
+def test_standalone_harmonics_kernel_compiles(lmax, dtype):
+    # e3conv_edge_harmonics generates and compiles its kernel before it needs a device: on a
+    # host it gets as far as "no device" (a compile failure would be E3CONV_ERR_COMPILE)
+    sh = "+".join(f"1x{l}{'eo'[l % 2]}" for l in range(lmax + 1))
+    c = e3.Conv("4x0e", sh, "4x0e", 1.0, dtype=dtype)
+    rc = e3._edge_sh(c._h, ctypes.c_void_p(256), 5, ctypes.c_void_p(512), None)
+    assert rc == 7, e3._last_error()                                      # E3CONV_ERR_NO_DEVICE
+    assert e3._edge_sh(c._h, ctypes.c_void_p(256), 0, None, None) == 0    # empty: nothing to do
+    assert e3._edge_sh(c._h, ctypes.c_void_p(258), 5, ctypes.c_void_p(512), None) == \
+        1                                                                  # E3CONV_ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("split", [2, 3, 4])
 def test_path_split_tables_cover_every_entry_once(split):
     # the warps of a path-split team own disjoint output irreps; their tables together form

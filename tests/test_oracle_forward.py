@@ -3,7 +3,7 @@ import numpy as np
 import pytest
 
 import oracle
-from workloads import SPECS, edge_sh, make_graph, node_features_np, scalars_np
+from workloads import SPECS, make_graph, node_features_np, scalars_np
 from workloads import graphs as wgraphs
 
 RICH = ("2x0e+2x1o+2x2e+2x3o+2x1e", "1x0e+1x1o+1x2e+1x3o",
@@ -169,7 +169,8 @@ def test_tiny_workload_against_brute_force():
     spec = SPECS["tiny"]
     gr = make_graph(spec)
     x = node_features_np(spec, gr.num_nodes)
-    Y = edge_sh(spec, gr)
+    Y = oracle.sh(spec.lmax, gr.vec / np.linalg.norm(gr.vec, axis=1, keepdims=True))
+    Y = Y.astype(np.float32)
     s = scalars_np(spec, gr)
     irreps = (spec.irreps_node, spec.irreps_sh, spec.irreps_out)
     ref = _einsum_reference(irreps, x.astype(np.float64), Y.astype(np.float64),

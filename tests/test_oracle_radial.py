@@ -75,16 +75,3 @@ def test_mlp_against_explicit_loops():
             z = [sum(h[i] * w[i, j] for i in range(len(h))) for j in range(w.shape[1])]
             h = [zj / (1 + np.exp(-zj)) for zj in z] if layer < len(ws) - 1 else z
         np.testing.assert_allclose(got[q], h, rtol=1e-13, atol=1e-14)
-
-
-def test_workload_scalars_match_the_oracle_mlp():
-    from workloads import SPECS, configs, make_graph
-    spec = SPECS["mace"]
-    g = make_graph(spec)
-    edges = np.arange(0, g.num_edges, 997)
-    s = configs.scalars_np(spec, g, edges).astype(np.float64)
-    ws = configs.radial_weights(spec)
-    d = np.linalg.norm(g.vec[edges], axis=1)
-    ref = oracle.radial_mlp(d, spec.graph["r"], ws).reshape(len(edges), spec.num_paths, spec.C)
-    scale = np.abs(ref).max()
-    assert np.abs(s - ref).max() <= 2 ** -23 * scale * 4

@@ -6,7 +6,6 @@ import numpy as np
 import pytest
 
 import oracle
-from workloads import real_sh
 
 LMAX = 6
 
@@ -84,13 +83,3 @@ def test_l1_is_scaled_direction_in_yzx_order():
     v = _unit(np.random.default_rng(50), 20)
     np.testing.assert_allclose(oracle.sh_l(1, v), np.sqrt(3) * v[:, [1, 2, 0]], atol=1e-14)
     np.testing.assert_allclose(oracle.sh_l(0, v), 1.0)
-
-
-def test_workload_harmonics_match_oracle():
-    # two independent implementations (recurrence vs Rodrigues polynomial)
-    g = np.random.default_rng(60)
-    v = g.normal(size=(300, 3)) * g.uniform(0.1, 5, size=(300, 1))
-    u = v / np.linalg.norm(v, axis=1, keepdims=True)
-    np.testing.assert_allclose(real_sh(v, LMAX), oracle.sh(LMAX, u), atol=1e-11)
-    z = real_sh(np.zeros((2, 3)), 3)
-    assert np.all(z[:, 0] == 1) and np.all(z[:, 1:] == 0)

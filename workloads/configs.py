@@ -5,24 +5,30 @@ Inputs of workload w (all seeded, see rng.py for the generator):
 * graph: points and radius graph from graphs.py, edges sorted by (receiver,
   sender); edge e is the e-th edge of that order.
 * node features x[a, i, u] = normal(seed, TID_X, (a * nx + i) * C + u).
-* edge features Y[e] = real_sh(r_ab, lmax) (sh.py), l-major, m = -l..l.
-* edge scalars s[e, p, u] = normal(seed, TID_S, (e * P + p) * C + u), or for
-  the MACE-like layer the output of a radial MLP on Bessel bases (below).
+* edge vectors r_ab = p_b - p_a (float64 on the host; float32 [E][4] with a zero
+  fourth component for the device, `edge_vectors_np`).
+* edge scalars s[e, p, u] = normal(seed, TID_S, (e * P + p) * C + u), or, for
+  the MACE-like layer (scalars="radial"), the radial MLP of |r_ab| with the
+  seeded weights `radial_weights` (normal draws / sqrt(fan-in)).
 * avg_num_neighbors = E / N, the measured mean degree.
 
-Every tensor is rounded once from float64 to the workload dtype (float32 or
-float16); consumers that need float64 upcast the rounded values exactly.
-The layout is trailing channels: x [N][nx][C], Y [E][ny], s [E][P][C].
+The edge features Y (spherical harmonics of r_ab) and the radial scalars are
+functions the method itself computes, so this module does not: each side
+evaluates them with its own implementation (the oracle's, or the library's
+kernels) from the edge vectors and weights drawn here.
+
+Every drawn tensor is rounded once from float64 to the workload dtype
+(float32 or float16); consumers that need float64 upcast the rounded values
+exactly.  The layout is trailing channels: x [N][nx][C], Y [E][ny], s [E][P][C].
 """
 from __future__ import annotations
 
 from dataclasses import dataclass, field
-from math import pi, sqrt
+from math import sqrt
 
 import numpy as np
 
 from . import graphs, rng
-from .sh import real_sh
 
 TID_POS = 0
 TID_X = 1
@@ -43,7 +49,7 @@ class Spec:
     graph: dict = field(default_factory=dict)
     graph_seed: int = 0
     seed: int = 0
-    scalars: str = "normal"   # or 'mlp'
+    scalars: str = "normal"   # or 'radial' (the radial MLP of the edge lengths)
     description: str = ""
 
     @property
@@ -69,7 +75,7 @@ SPECS = {
         "mace", "128x0e+128x1o", 3, "128x0e+128x1o+128x2e+128x3o", C=128, nx=4, num_paths=10,
         dtype="f32",
         graph=dict(kind="cube", n=5000, box=44.36, r=5.0, periodic=True), graph_seed=3, seed=3,
-        scalars="mlp",
+        scalars="radial",
         description="5000 nodes, periodic box 44.36, r=5.0 (~30 neighbours); 128x(0e+1o), Y l<=3, "
                     "s = 2-layer SiLU MLP(64) on 8 Bessel bases x cosine cutoff, float32"),
     "large_f32": Spec(
@@ -140,9 +146,12 @@ def torch_dtype(spec: Spec):
     return torch.float16 if spec.dtype == "f16" else torch.float32
 
 
-def edge_sh(spec: Spec, graph: Graph) -> np.ndarray:
-    """[E][ny] in the spec dtype (host)."""
-    return real_sh(graph.vec, spec.lmax).astype(np_dtype(spec))
+def edge_vectors_np(graph: Graph, e0: int = 0, e1: int | None = None) -> np.ndarray:
+    """float32 [e1-e0][4]: (x, y, z, 0) of r_ab for edges e0..e1-1 (the device layout)."""
+    e1 = graph.num_edges if e1 is None else e1
+    v = np.zeros((e1 - e0, 4), np.float32)
+    v[:, :3] = graph.vec[e0:e1]
+    return v
 
 
 def node_features_np(spec: Spec, num_nodes: int, rows: np.ndarray | None = None) -> np.ndarray:
@@ -160,26 +169,15 @@ def node_features_torch(spec: Spec, num_nodes: int, device, first: int = 0):
                             start=first * per).view(num_nodes, spec.nx, spec.C)
 
 
-# --- radial scalars for the MACE-like layer ---------------------------------
+# --- edge scalars ------------------------------------------------------------
 
-def _bessel_cutoff(d: np.ndarray, r: float, nb: int = 8) -> np.ndarray:
-    """B_n(d) = sqrt(2/r) sin(n pi d / r) / d * (cos(pi d / r) + 1) / 2, n = 1..nb."""
-    n = np.arange(1, nb + 1)
-    b = sqrt(2.0 / r) * np.sin(n[None, :] * pi * d[:, None] / r) / d[:, None]
-    return b * (0.5 * (np.cos(pi * d / r) + 1.0))[:, None]
-
-
-RADIAL_BASIS = 8      # bessel bases of the MACE-like layer
+RADIAL_BASIS = 8      # bessel bases of the MACE-like layer's radial MLP
 RADIAL_HIDDEN = 64    # neurons of each of its two hidden layers
 
 
 def radial_weights(spec: Spec):
     """The seeded MLP weights [W_0 (8 x 64), W_1 (64 x 64), W_2 (64 x P*C)], float64."""
-    return _mlp_weights(spec, [RADIAL_BASIS, RADIAL_HIDDEN, RADIAL_HIDDEN,
-                               spec.num_paths * spec.C])
-
-
-def _mlp_weights(spec: Spec, sizes):
+    sizes = [RADIAL_BASIS, RADIAL_HIDDEN, RADIAL_HIDDEN, spec.num_paths * spec.C]
     ws = []
     for layer, (fi, fo) in enumerate(zip(sizes[:-1], sizes[1:])):
         w = rng.normal_np(spec.seed, TID_W + layer, np.arange(fi * fo, dtype=np.uint64))
@@ -187,36 +185,26 @@ def _mlp_weights(spec: Spec, sizes):
     return ws
 
 
-def _silu(v):
-    return v / (1.0 + np.exp(-v))
+def _drawn_scalars(spec: Spec):
+    if spec.scalars != "normal":
+        raise ValueError(f"{spec.name}: the edge scalars are the radial MLP of the edge lengths; "
+                         "evaluate it from edge_vectors_np and radial_weights")
 
 
 def scalars_np(spec: Spec, graph: Graph, edges: np.ndarray | None = None) -> np.ndarray:
     """Host s[edges] ([len(edges)][P][C]) in the spec dtype; edges default to all."""
+    _drawn_scalars(spec)
     P, C = spec.num_paths, spec.C
     edges = np.arange(graph.num_edges) if edges is None else np.asarray(edges)
-    if spec.scalars == "normal":
-        k = (edges[:, None, None] * P + np.arange(P)[None, :, None]) * C \
-            + np.arange(C)[None, None, :]
-        return rng.normal_np(spec.seed, TID_S, k.astype(np.uint64)).astype(np_dtype(spec))
-    r = spec.graph["r"]
-    w1, w2, w3 = radial_weights(spec)
-    out = np.empty((len(edges), P, C), dtype=np_dtype(spec))
-    for c0 in range(0, len(edges), 1 << 15):
-        e = edges[c0:c0 + (1 << 15)]
-        d = np.linalg.norm(graph.vec[e], axis=1)
-        h = _silu(_bessel_cutoff(d, r) @ w1)
-        h = _silu(h @ w2)
-        out[c0:c0 + len(e)] = (h @ w3).reshape(len(e), P, C).astype(np_dtype(spec))
-    return out
+    k = (edges[:, None, None] * P + np.arange(P)[None, :, None]) * C + np.arange(C)[None, None, :]
+    return rng.normal_np(spec.seed, TID_S, k.astype(np.uint64)).astype(np_dtype(spec))
 
 
 def scalars_torch(spec: Spec, graph: Graph, device, edges: tuple | None = None):
     """s[e0:e1] on the device for edges = (e0, e1) (all edges by default)."""
     import torch
+    _drawn_scalars(spec)
     e0, e1 = edges if edges is not None else (0, graph.num_edges)
     P, C = spec.num_paths, spec.C
-    if spec.scalars == "normal":
-        return rng.normal_torch(spec.seed, TID_S, (e1 - e0) * P * C, torch_dtype(spec), device,
-                                start=e0 * P * C).view(e1 - e0, P, C)
-    return torch.from_numpy(scalars_np(spec, graph, np.arange(e0, e1))).to(device)
+    return rng.normal_torch(spec.seed, TID_S, (e1 - e0) * P * C, torch_dtype(spec), device,
+                            start=e0 * P * C).view(e1 - e0, P, C)
