@@ -181,15 +181,17 @@ def kernel_hash(conv) -> str:
     return hashlib.sha1(conv.kernel_source().encode()).hexdigest()[:16]
 
 
-def traffic_for(workload, conv, E):
-    """DRAM bytes per forward launch from the committed ncu summary, if the kernel is unchanged."""
+def traffic_for(workload, conv, N, E, edge_vectors=False):
+    """DRAM bytes of one forward launch from a committed ncu capture of this same
+    configuration (workload, node count, unchanged kernel source), else None.  A capture of a
+    smaller graph is not scaled: the node table's L2 residency changes with the size."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
+    if workload is None or edge_vectors or not os.path.exists(p):
         return None, None
-    d = json.load(open(p)).get(workload)
-    if not d or d.get("kernel_sha1") != kernel_hash(conv):
+    d = json.load(open(p)).get(f"{workload}@{N}")
+    if not d or d.get("kernel_sha1") != kernel_hash(conv) or d.get("edges") != E:
         return None, None
-    return d["dram_bytes_per_edge"] * E, d.get("source")
+    return float(d["dram_read_bytes"] + d["dram_write_bytes"]), d.get("source")
 
 
 # ---------------------------------------------------------------------------
@@ -517,8 +519,8 @@ def run_ours(args):
     # balances edges + rows), against the slowest rank's forward time
     nbytes, flops, nnz, mix = algorithmic(conv, N, E, in_bytes)
     nbytes, flops = nbytes / world, flops / world
-    traffic, traffic_src = traffic_for(spec.name if args.nodes is None and world == 1 else None,
-                                       conv, E)
+    traffic, traffic_src = traffic_for(spec.name if world == 1 else None, conv, N, E,
+                                       bool(args.edge_vectors))
     sec = fwd_ms / 1000.0
     t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
     if info.get("tensor_cores"):

@@ -51,3 +51,21 @@ def test_cpu_baseline_sample_is_seeded_and_bounded():
     n = min(len(a), len(b))
     order = np.random.default_rng(2024).permutation(g.num_nodes)
     assert set(a[:n]) <= set(order[:max(len(a), len(b))])
+
+
+def test_traffic_is_reported_only_for_the_captured_configuration():
+    # the committed DRAM counters belong to one (workload, node count, kernel source); any
+    # other size or an edited kernel reports no traffic rather than a scaled guess
+    import json
+    d = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    for key, rec in d.items():
+        name, nodes = key.split("@")
+        spec = configs.SPECS[name]
+        c = e3.Conv(spec.irreps_node, spec.irreps_sh, spec.irreps_out, 40.0, dtype=spec.dtype)
+        t, src = bench.traffic_for(name, c, int(nodes), rec["edges"])
+        if rec["kernel_sha1"] == bench.kernel_hash(c):
+            assert t == rec["dram_read_bytes"] + rec["dram_write_bytes"] and src
+        else:
+            assert t is None
+        assert bench.traffic_for(name, c, int(nodes) * 10, rec["edges"] * 10) == (None, None)
+        assert bench.traffic_for(name, c, int(nodes), rec["edges"], edge_vectors=True) == (None, None)
