@@ -681,6 +681,12 @@ def time_next_rows(args, spec, g, conv, x, Y, s, senders, receivers, row_ptr, ou
         ms = _event_ms(lambda: conv.backward(x, Y, s, senders, row_ptr, gout, receivers=receivers,
                                              sender_row_ptr=srp, sender_perm=sperm), reps, stream)
         assert conv.check(), "backward reported a bad index"
+        # each kernel alone: grad_Y and grad_s (receiver order), grad_x (sender order)
+        ms_edges = _event_ms(lambda: conv.backward(x, Y, s, senders, row_ptr, gout, need_x=False),
+                             reps, stream)
+        ms_nodes = _event_ms(lambda: conv.backward(x, Y, s, senders, row_ptr, gout, receivers=receivers,
+                                                   sender_row_ptr=srp, sender_perm=sperm,
+                                                   need_edges=False), reps, stream)
         b = 2 if spec.dtype == "f16" else 4
         nnz = sum(int((np.abs(conv.cg(p)) > 1e-12).sum()) for p in range(conv.num_paths))
         mix = sum(2 * q.l3 + 1 for q in conv.paths)
@@ -691,7 +697,8 @@ def time_next_rows(args, spec, g, conv, x, Y, s, senders, receivers, row_ptr, ou
                   + N * (conv.nx * conv.C * b + 2 * 4 * conv.nout * conv.C + 4 * conv.nx * conv.C))
         flops = 2 * E * conv.C * (4 * nnz + mix)
         res["backward"] = {
-            "kernels": "e3conv_bwd_edges + e3conv_bwd_nodes", "ms": ms, "edges_per_s": E / (ms / 1e3),
+            "kernels": "e3conv_bwd_edges + e3conv_bwd_nodes", "ms": ms, "edges_ms": ms_edges,
+            "nodes_ms": ms_nodes, "edges_per_s": E / (ms / 1e3),
             "algorithmic_bytes": nbytes, "hbm_gbs": nbytes / (ms / 1e3) / 1e9,
             "hbm_frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
             "fp32_flops": flops, "fp32_tflops": flops / (ms / 1e3) / 1e12,

@@ -63,6 +63,8 @@ OPT_DIRECT_PIPELINE = 7
 _get_option = _sig("e3conv_get_option", ctypes.c_int, _vp, ctypes.c_int, _c_int_p)
 _sh_host = _sig("e3conv_spherical_harmonics", ctypes.c_int, _vp, ctypes.POINTER(ctypes.c_double),
                 ctypes.POINTER(ctypes.c_double))
+_kernel_log = _sig("e3conv_kernel_log", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_char_p,
+                   ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t))
 _edge_sh = _sig("e3conv_edge_harmonics", ctypes.c_int, _vp, _vp, _i64, _vp, _vp)
 _kernel_source = _sig("e3conv_kernel_source", ctypes.c_int, _vp, ctypes.c_int, ctypes.c_char_p,
                       ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t))
@@ -101,7 +103,7 @@ _version = _sig("e3conv_version", ctypes.c_int)
 EXPORTED = ["e3conv_create", "e3conv_destroy", "e3conv_set_input_dtype",
             "e3conv_set_launch_config", "e3conv_set_option", "e3conv_get_option",
             "e3conv_spherical_harmonics", "e3conv_edge_harmonics", "e3conv_query", "e3conv_path", "e3conv_num_outputs",
-            "e3conv_output_irrep", "e3conv_cg", "e3conv_kernel_info", "e3conv_kernel_source",
+            "e3conv_output_irrep", "e3conv_cg", "e3conv_kernel_info", "e3conv_kernel_source", "e3conv_kernel_log",
             "e3conv_forward", "e3conv_forward_rows", "e3conv_check", "e3conv_partition_rows",
             "e3conv_backward", "e3conv_prepare_backward", "e3conv_backward_source",
             "e3conv_set_radial_mlp", "e3conv_radial_scalars", "e3conv_linear_create",
@@ -288,6 +290,15 @@ class Conv:
         keys = ["channels_per_lane", "lanes_per_tile", "block_threads", "stages", "contract_first",
                 "tensor_cores", "registers", "local_bytes"]
         return dict(zip(keys, (x.value for x in v)))
+
+    def kernel_log(self, dtype: str | None = None) -> str:
+        """The launch-shape search's compile attempts and the kept compile's NVRTC log."""
+        d = {"f32": F32, "f16": F16}[dtype or self.dtype]
+        n = ctypes.c_size_t()
+        _ok(_kernel_log(self._h, d, None, 0, ctypes.byref(n)), "e3conv_kernel_log")
+        buf = ctypes.create_string_buffer(n.value)
+        _ok(_kernel_log(self._h, d, buf, n.value, ctypes.byref(n)), "e3conv_kernel_log")
+        return buf.value.decode()
 
     def kernel_source(self, dtype: str | None = None) -> str:
         d = {"f32": F32, "f16": F16}[dtype or self.dtype]

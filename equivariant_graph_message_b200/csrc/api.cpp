@@ -177,6 +177,29 @@ int compile_once(Plan& pl, int dtype) {
   v.source = generate_forward_source(pl, dtype, v.shape);
   const int rc = nvrtc_compile(v.source, "e3conv_fwd.cu", v.cubin, v.log, v.regs, v.local_bytes);
   if (rc != E3CONV_OK) return rc;
+  // With a device, registers and local memory come from the loaded function: the NVRTC
+  // log does not always carry ptxas' resource lines (a repeated compile of the same source
+  // was seen to return none), and the launch-shape search must not read a missing line as
+  // "no local memory".
+  if (pl.device >= 0) {
+    Driver& d = driver();
+    CUmodule m = nullptr;
+    CUfunction f = nullptr;
+    if (d.ModuleLoadData(&m, v.cubin.data()) == CUDA_SUCCESS) {
+      if (d.ModuleGetFunction(&f, m, "e3conv_fwd") == CUDA_SUCCESS) {
+        int regs = 0, local = 0;
+        if (d.FuncGetAttribute(&regs, CU_FUNC_ATTRIBUTE_NUM_REGS, f) == CUDA_SUCCESS) v.regs = regs;
+        if (d.FuncGetAttribute(&local, CU_FUNC_ATTRIBUTE_LOCAL_SIZE_BYTES, f) == CUDA_SUCCESS)
+          v.local_bytes = local;
+      }
+      d.ModuleUnload(m);
+    }
+  }
+  pl.trace[dtype] += "compile: block=" + std::to_string(v.shape.block) + " V=" +
+                     std::to_string(v.shape.V) + " team=" + std::to_string(v.shape.team) +
+                     " stages=" + std::to_string(v.shape.stages) + " tc=" +
+                     std::to_string(v.shape.tc ? 1 : 0) + " regs=" + std::to_string(v.regs) +
+                     " local=" + std::to_string(v.local_bytes) + "\n";
   v.compiled = true;
   return E3CONV_OK;
 }
@@ -236,6 +259,7 @@ int blocks_per_sm(const Shape& s, int regs, int block) {
 }
 
 int compile_variant(Plan& pl, int dtype) {
+  pl.trace[dtype].clear();
   pl.auto_block = 0;
   pl.tc_team_cap = 0;
   pl.tc_fallback = false;
@@ -294,6 +318,7 @@ int compile_variant(Plan& pl, int dtype) {
     d.FuncGetAttribute(&local, CU_FUNC_ATTRIBUTE_LOCAL_SIZE_BYTES, v.fn);
     v.regs = regs;
     v.local_bytes = local;
+    pl.trace[dtype] += "loaded: regs=" + std::to_string(regs) + " local=" + std::to_string(local) + "\n";
     if (v.shape.stages > 0) {
       const int smem = v.shape.tc ? v.shape.smem_request
                                   : v.shape.warp_smem * (v.shape.block / (32 * v.shape.team));
@@ -687,6 +712,18 @@ int e3conv_kernel_info(e3conv_plan h, int dtype, int* V, int* TL, int* block, in
   if (tensor_cores) *tensor_cores = v.shape.tc ? 1 : 0;
   if (regs) *regs = v.regs;
   if (local_bytes) *local_bytes = v.local_bytes;
+  return E3CONV_OK;
+}
+
+int e3conv_kernel_log(e3conv_plan h, int dtype, char* buf, size_t buf_len, size_t* needed) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "plan is NULL");
+  if (dtype != E3CONV_F32 && dtype != E3CONV_F16)
+    return fail(E3CONV_ERR_UNSUPPORTED, "unknown dtype");
+  const Variant& v = h->p.var[dtype];
+  if (!v.compiled) return fail(E3CONV_ERR_INVALID_ARG, "variant not compiled (set_input_dtype)");
+  const std::string text = h->p.trace[dtype] + v.log;
+  if (needed) *needed = text.size() + 1;
+  if (buf && buf_len >= text.size() + 1) std::memcpy(buf, text.c_str(), text.size() + 1);
   return E3CONV_OK;
 }
 

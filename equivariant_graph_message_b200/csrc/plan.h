@@ -197,6 +197,7 @@ struct Plan {
   Variant var[2];
   BwdVariant bwd[2];               // backward kernels per input dtype (compiled on first use)
   ShVariant shk[2];                // standalone harmonics kernel per input dtype
+  std::string trace[2];            // the forward's compile attempts (shape, registers, local bytes)
   RadialPlan radial;
 };
 

@@ -22,9 +22,12 @@
 // float32 rounding), which keeps the products at float32 accuracy; the
 // weights are scaled by a power of two before the split (undone exactly on
 // the way out) so that their lo parts stay normal float16 numbers.
-// The output layer runs in chunks of 128 columns, double-buffered in shared
-// memory (bulk copies of prepacked chunks) and in tensor memory (the MMAs of
-// chunk c overlap the stores of chunk c-1).  All waits are bounded: on
+// The output layer runs in chunks of 32 columns: their weights stream through
+// four shared-memory buffers (bulk copies of prepacked chunks, issued three
+// chunks ahead), their products alternate between two tensor-memory buffers
+// (the MMAs of chunk c overlap the stores of chunk c-1).  Stores go through a
+// per-warp shared-memory transpose so that each warp instruction writes one
+// edge row's 32 consecutive outputs (coalesced), not 32 rows' scattered ones.  All waits are bounded: on
 // timeout a CTA sets bit 4 of the status word, drains what it issued
 // (bounded) and stops.
 #include <cuda_runtime.h>
@@ -47,7 +50,10 @@ using namespace tc_host;
 
 constexpr int kTile = 128;           // edges per tile (MMA M)
 constexpr int kMaxBasis = 16;        // radial bases (layer 0 is unrolled over them)
-constexpr int kChunk = 64;           // output columns per output-layer chunk (MMA N)
+constexpr int kChunk = 32;           // output columns per output-layer chunk (MMA N)
+constexpr int kWBufs = 4;            // output-weight chunk buffers in shared memory
+constexpr int kStage = 36;           // floats per staged row (16-byte rows, conflict-free)
+constexpr int kOutCol = 64;          // tensor-memory column of the output buffers (>= hidden)
 
 struct RadialArgs {
   const float* vec;        // [E][4] edge vectors (x, y, z, unused)
@@ -73,7 +79,8 @@ template <int H>
 struct Smem {
   static constexpr int kAct = kTile * H * 2;     // one K-major [128 x H] float16 operand
   static constexpr int kWhid = H * H * 2;        // one [H x H] float16 operand
-  static constexpr int kWout = kChunk * H * 2;   // one [128 x H] float16 operand
+  static constexpr int kWout = kChunk * H * 2;   // one [kChunk x H] float16 operand
+  static constexpr int kStageBytes = 4 * 32 * kStage * 4;  // transpose rows of the 4 warps
 };
 
 template <int H>
@@ -85,20 +92,22 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
   unsigned char* whs = sm + ((a.nb * H * 4 + 1023) / 1024) * 1024;    // (layers-1) x (hi, lo)
   unsigned char* act = whs + (a.layers - 1) * 2 * L::kWhid;           // hi, lo
   unsigned char* wos = act + 2 * L::kAct;                             // 2 buffers x (hi, lo)
-  unsigned long long* bars = reinterpret_cast<unsigned long long*>(wos + 4 * L::kWout);
-  unsigned long long* bar_w = bars;        // [2] output-weight chunk landed
-  unsigned long long* bar_mma = bars + 2;  // [2] output MMAs of a chunk done
-  unsigned long long* bar_hid = bars + 4;  // hidden-layer MMAs done
-  unsigned long long* bar_wh = bars + 5;   // hidden weights landed
-  unsigned* tslot = reinterpret_cast<unsigned*>(bars + 6);
+  float* stage = reinterpret_cast<float*>(wos + kWBufs * 2 * L::kWout);
+  unsigned long long* bars = reinterpret_cast<unsigned long long*>(
+      reinterpret_cast<unsigned char*>(stage) + L::kStageBytes);
+  unsigned long long* bar_w = bars;                 // [kWBufs] output-weight chunk landed
+  unsigned long long* bar_mma = bars + kWBufs;      // [2] output MMAs of a chunk done
+  unsigned long long* bar_hid = bars + kWBufs + 2;  // hidden-layer MMAs done
+  unsigned long long* bar_wh = bars + kWBufs + 3;   // hidden weights landed
+  unsigned* tslot = reinterpret_cast<unsigned*>(bars + kWBufs + 4);
 
   for (int q = tid; q < a.nb * H; q += 128) w0s[q] = a.w0[q];
   if (tid == 0) {
-    for (int k = 0; k < 6; ++k) mbar_init(bars + k, 1);
+    for (int k = 0; k < kWBufs + 4; ++k) mbar_init(bars + k, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 128;" ::"r"(
                      smem_u32(tslot))
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -108,7 +117,7 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
   tc_after();
   const unsigned tmem = *tslot;
   const unsigned t_hid = tmem;                 // columns [0, H): hidden-layer D
-  // output-layer D: two buffers of kChunk columns at 128 and 128 + kChunk
+  // output-layer D: two buffers of kChunk columns at kOutCol and kOutCol + kChunk
   const unsigned lane_off = static_cast<unsigned>(32 * warp) << 16;
   bool ok = true;
   // phase bits (bit b: buffer b) of the weight-chunk and output-MMA barriers
@@ -133,9 +142,10 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
   for (long long tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
     const long long e = tile * kTile + tid;
     const bool valid = e < a.num_edges;
-    // prefetch the first output-weight chunks of this tile
+    // prefetch the first output-weight chunks of this tile (every buffer is free: the
+    // previous tile waited for all of its output MMAs)
     if (tid == 0) {
-      for (int c = 0; c < 2 && c < a.chunks; ++c) {
+      for (int c = 0; c < kWBufs && c < a.chunks; ++c) {
         mbar_expect(bar_w + c, 2 * L::kWout);
         bulk_g2s(wos + c * 2 * L::kWout, a.wo + static_cast<size_t>(c) * 2 * L::kWout,
                  2 * L::kWout, bar_w + c);
@@ -215,19 +225,22 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
     __syncthreads();
     tc_after();
     const unsigned id = idesc_f16(kTile, kChunk);
+    const int lane = tid & 31;
+    float* st = stage + warp * 32 * kStage;          // this warp's 32 staged rows
+    const long long row0 = tile * kTile + warp * 32;  // edge of staged row 0
     for (int c = 0; c <= a.chunks && ok; ++c) {
       if (c < a.chunks) {
-        const int buf = c & 1;
-        ok = __syncthreads_and(mbar_wait(bar_w + buf, (ph_w >> buf) & 1u));
+        const int wb = c % kWBufs, buf = c & 1;
+        ok = __syncthreads_and(mbar_wait(bar_w + wb, (ph_w >> wb) & 1u));
         if (!ok) break;
-        ph_w ^= 1u << buf;
-        pend_w &= ~(1u << buf);
+        ph_w ^= 1u << wb;
+        pend_w &= ~(1u << wb);
         if (tid == 0) {
-          const unsigned char* whi = wos + buf * 2 * L::kWout;
+          const unsigned char* whi = wos + wb * 2 * L::kWout;
           const unsigned char* wlo = whi + L::kWout;
+          const unsigned td = tmem + static_cast<unsigned>(kOutCol + kChunk * buf);
           for (int ks = 0; ks < H / 16; ++ks) {
             const int ao = ks * kTile * 32, bo = ks * kChunk * 32;
-            const unsigned td = tmem + 128u + static_cast<unsigned>(kChunk) * buf;
             mma_f16(td, kmajor_desc(act + ao), kmajor_desc(whi + bo), id, ks > 0);
             mma_f16(td, kmajor_desc(act + ao), kmajor_desc(wlo + bo), id, 1);
             mma_f16(td, kmajor_desc(act + L::kAct + ao), kmajor_desc(whi + bo), id, 1);
@@ -236,59 +249,44 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
           pend_mma |= 1u << buf;
         }
       }
-      if (c >= 1) {  // stores of chunk c-1, then its weight buffer takes chunk c+1
-        const int pb = (c - 1) & 1;
+      if (c >= 1) {  // chunk c-1: its weight buffer takes chunk c-1+kWBufs, then its stores
+        const int pb = (c - 1) & 1, pw = (c - 1) % kWBufs;
         ok = __syncthreads_and(mbar_wait(bar_mma + pb, (ph_mma >> pb) & 1u));
         tc_after();
         if (!ok) break;
         ph_mma ^= 1u << pb;
         pend_mma &= ~(1u << pb);
-        if (tid == 0 && c + 1 < a.chunks) {
-          mbar_expect(bar_w + pb, 2 * L::kWout);
-          bulk_g2s(wos + pb * 2 * L::kWout, a.wo + static_cast<size_t>(c + 1) * 2 * L::kWout,
-                   2 * L::kWout, bar_w + pb);
-          pend_w |= 1u << pb;
+        if (tid == 0 && c - 1 + kWBufs < a.chunks) {
+          mbar_expect(bar_w + pw, 2 * L::kWout);
+          bulk_g2s(wos + pw * 2 * L::kWout,
+                   a.wo + static_cast<size_t>(c - 1 + kWBufs) * 2 * L::kWout, 2 * L::kWout,
+                   bar_w + pw);
+          pend_w |= 1u << pw;
         }
-        const int col0 = (c - 1) * kChunk;
-#pragma unroll 1
-        for (int j0 = 0; j0 < kChunk; j0 += 32) {
-          float v[32];
-          tmem_ld32(tmem + 128u + static_cast<unsigned>(kChunk) * pb + lane_off + j0, v);
-          if (valid) {
-            const int cols = min(32, a.nout - (col0 + j0));
-            if (cols > 0) {
-              if (a.out_f16) {
-                __half* dst = static_cast<__half*>(a.s) + e * a.nout + col0 + j0;
-                if (cols == 32 && ((a.nout & 7) == 0)) {
+        float v[32];
+        tmem_ld32(tmem + static_cast<unsigned>(kOutCol + kChunk * pb) + lane_off, v);
+        const float f = a.w_scale_inv_o;
 #pragma unroll
-                  for (int q = 0; q < 32; q += 8) {
-                    const float f = a.w_scale_inv_o;
-                    *reinterpret_cast<uint4*>(dst + q) =
-                        make_uint4(pack_half2(v[q] * f, v[q + 1] * f), pack_half2(v[q + 2] * f, v[q + 3] * f),
-                                   pack_half2(v[q + 4] * f, v[q + 5] * f), pack_half2(v[q + 6] * f, v[q + 7] * f));
-                  }
-                } else {
-#pragma unroll
-                  for (int q = 0; q < 32; ++q)
-                    if (q < cols) dst[q] = __float2half_rn(v[q] * a.w_scale_inv_o);
-                }
-              } else {
-                float* dst = static_cast<float*>(a.s) + e * a.nout + col0 + j0;
-                if (cols == 32 && ((a.nout & 3) == 0)) {
-#pragma unroll
-                  for (int q = 0; q < 32; q += 4)
-                    *reinterpret_cast<float4*>(dst + q) =
-                        make_float4(v[q] * a.w_scale_inv_o, v[q + 1] * a.w_scale_inv_o,
-                                    v[q + 2] * a.w_scale_inv_o, v[q + 3] * a.w_scale_inv_o);
-                } else {
-#pragma unroll
-                  for (int q = 0; q < 32; ++q)
-                    if (q < cols) dst[q] = v[q] * a.w_scale_inv_o;
-                }
-              }
-            }
+        for (int q = 0; q < 32; q += 4)
+          *reinterpret_cast<float4*>(st + lane * kStage + q) =
+              make_float4(v[q] * f, v[q + 1] * f, v[q + 2] * f, v[q + 3] * f);
+        __syncwarp();
+        // lane l writes column (c-1) * kChunk + l of the warp's 32 rows: one row per instruction
+        const int col = (c - 1) * kChunk + lane;
+        if (col < a.nout) {
+          if (a.out_f16) {
+            __half* dst = static_cast<__half*>(a.s) + row0 * a.nout + col;
+#pragma unroll 8
+            for (int r = 0; r < 32; ++r)
+              if (row0 + r < a.num_edges) dst[static_cast<long long>(r) * a.nout] = __float2half_rn(st[r * kStage + lane]);
+          } else {
+            float* dst = static_cast<float*>(a.s) + row0 * a.nout + col;
+#pragma unroll 8
+            for (int r = 0; r < 32; ++r)
+              if (row0 + r < a.num_edges) dst[static_cast<long long>(r) * a.nout] = st[r * kStage + lane];
           }
         }
+        __syncwarp();  // staged rows read before the next chunk overwrites them
         tc_before();
         __syncthreads();  // chunk c-1's columns read by every thread before they are reused
         tc_after();
@@ -298,10 +296,10 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
   if (!ok && tid == 0) {
     atomicOr(a.status, 4u);
     // drain (bounded): copies and MMAs issued but not seen complete
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kWBufs; ++b)
       if ((pend_w >> b) & 1u) mbar_wait(bar_w + b, (ph_w >> b) & 1u);
+    for (int b = 0; b < 2; ++b)
       if ((pend_mma >> b) & 1u) mbar_wait(bar_mma + b, (ph_mma >> b) & 1u);
-    }
     if (pend_hid) mbar_wait(bar_hid, ph_hid);
     if (pend_wh) mbar_wait(bar_wh, 0);
   }
@@ -309,7 +307,7 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
   __syncthreads();
   tc_after();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 128;" ::"r"(tmem) : "memory");
 }
 
 }  // namespace
@@ -359,7 +357,8 @@ int radial_prepare(RadialPlan& rp, int nb, double r_max, int hidden, int layers,
 size_t radial_smem_bytes(const RadialPlan& rp) {
   const size_t H = rp.hidden;
   const size_t w0 = (rp.nb * H * 4 + 1023) / 1024 * 1024;
-  return w0 + (rp.layers - 1) * 2 * H * H * 2 + 2 * kTile * H * 2 + 4 * kChunk * H * 2 + 64;
+  return w0 + (rp.layers - 1) * 2 * H * H * 2 + 2 * kTile * H * 2 + kWBufs * 2 * kChunk * H * 2 +
+         4 * 32 * kStage * 4 + (kWBufs + 4) * 8 + 16;
 }
 
 int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, const void* dev_wo,
@@ -394,8 +393,8 @@ int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, 
     if (e == cudaSuccess)
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 128, smem);
     if (e != cudaSuccess || per_sm < 1) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
-    // tensor memory: 256 columns per CTA, so at most two CTAs per SM
-    per_sm = std::min(per_sm, 2);
+    // tensor memory: 128 columns per CTA, so at most four CTAs per SM
+    per_sm = std::min(per_sm, 4);
     const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, static_cast<long long>(grid) * per_sm));
     kernel<<<blocks, 128, smem, st>>>(a);
     return cudaSuccess;

@@ -252,6 +252,12 @@ E3CONV_API int e3conv_kernel_info(e3conv_plan plan, int dtype, int* channels_per
  * buf_len is large enough; *needed receives the required size in bytes. */
 E3CONV_API int e3conv_kernel_source(e3conv_plan plan, int dtype, char* buf, size_t buf_len, size_t* needed);
 
+/* The forward's compile record for `dtype`, as e3conv_kernel_source: one line
+ * per compile attempt of the launch-shape search (block, channels per lane,
+ * team, stages, registers, local bytes per thread; "loaded:" lines give what
+ * the loaded function reports), then the NVRTC log of the kept compile. */
+E3CONV_API int e3conv_kernel_log(e3conv_plan plan, int dtype, char* buf, size_t buf_len, size_t* needed);
+
 /* ---------------------------------------------------------------------------
  * Forward (the fused gather -> CG product -> scalar mix -> segmented sum ->
  * 1/N scale -> store of e3j's four plain steps; one kernel launch)
