@@ -231,6 +231,12 @@ int prepare_backward(Plan& pl) {
         return fail(E3CONV_ERR_CUDA, "loading the backward kernels failed");
       }
     }
+    if (v.shape.staged &&
+        d.FuncSetAttribute(v.fn[0], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES, v.shape.smem) !=
+            CUDA_SUCCESS) {
+      for (int q = 0; q < 2; ++q) d.ModuleUnload(v.module[q]);
+      return fail(E3CONV_ERR_CUDA, "cannot reserve the backward edges kernel's shared memory");
+    }
   }
   v.compiled = true;
   bv = v;
@@ -844,7 +850,7 @@ int e3conv_set_radial_mlp(e3conv_plan h, int num_basis, double r_max, int hidden
   if (pl.device >= 0) {
     DeviceGuard g(pl.device);
     struct Up { void** dst; const void* src; size_t n; };
-    const Up ups[3] = {{&rp.d_w0, rp.w0.data(), rp.w0.size() * sizeof(float)},
+    const Up ups[3] = {{&rp.d_w0, rp.w0.data(), rp.w0.size()},
                        {&rp.d_wh, rp.wh.data(), rp.wh.size()},
                        {&rp.d_wo, rp.wo.data(), rp.wo.size()}};
     for (const Up& u : ups) {
@@ -1074,8 +1080,9 @@ int e3conv_backward(e3conv_plan h, const void* x, const void* Y, const void* s,
     void* args[] = {const_cast<void**>(&x), const_cast<void**>(&Y), const_cast<void**>(&s),
                     const_cast<int32_t**>(&senders), const_cast<int32_t**>(&row_ptr), &n32,
                     const_cast<float**>(&grad_out), &grad_sh, &grad_scalars, &inv_avg, &pl.status};
-    if (driver().LaunchKernel(bv.fn[0], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1, 0, st,
-                              args, nullptr) != CUDA_SUCCESS)
+    if (driver().LaunchKernel(bv.fn[0], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1,
+                              b.staged ? static_cast<unsigned>(b.smem) : 0u, st, args,
+                              nullptr) != CUDA_SUCCESS)
       return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed (backward, edges)");
   }
   if (grad_x) {

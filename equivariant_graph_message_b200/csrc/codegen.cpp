@@ -338,6 +338,15 @@ void emit_prelude(Emitter& em) {
   }
 }
 
+// Packed float32x2 helpers: a register pair (lo, hi), broadcast, fma / mul / add.
+void emit_pair_ops(Emitter& em) {
+  em.line("__device__ __forceinline__ unsigned long long pk(float lo, float hi) { unsigned long long r; asm(\"mov.b64 %0, {%1, %2};\" : \"=l\"(r) : \"f\"(lo), \"f\"(hi)); return r; }");
+  em.line("__device__ __forceinline__ unsigned long long bc(float a) { return pk(a, a); }");
+  em.line("__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) { unsigned long long d; asm(\"fma.rn.f32x2 %0, %1, %2, %3;\" : \"=l\"(d) : \"l\"(a), \"l\"(b), \"l\"(c)); return d; }");
+  em.line("__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) { unsigned long long d; asm(\"mul.rn.f32x2 %0, %1, %2;\" : \"=l\"(d) : \"l\"(a), \"l\"(b)); return d; }");
+  em.line("__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) { unsigned long long d; asm(\"add.rn.f32x2 %0, %1, %2;\" : \"=l\"(d) : \"l\"(a), \"l\"(b)); return d; }");
+}
+
 // Declares and loads y0..y{ny-1} from `yr` (global or shared).
 void emit_y_load(Emitter& em, const Plan& pl, int dtype, const std::string& pre,
                  const std::string& yr) {
@@ -1237,11 +1246,7 @@ std::string staged_source(const Plan& pl, int dtype, const Shape& sh) {
   const Lanes L{V};
   const bool split = sh.coop && sh.psplit > 1;  // a row's paths split over the team's warps
   const int yf_bytes = align_up(4 * pl.ny, 16);
-  em.line("__device__ __forceinline__ unsigned long long pk(float lo, float hi) { unsigned long long r; asm(\"mov.b64 %0, {%1, %2};\" : \"=l\"(r) : \"f\"(lo), \"f\"(hi)); return r; }");
-  em.line("__device__ __forceinline__ unsigned long long bc(float a) { return pk(a, a); }");
-  em.line("__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) { unsigned long long d; asm(\"fma.rn.f32x2 %0, %1, %2, %3;\" : \"=l\"(d) : \"l\"(a), \"l\"(b), \"l\"(c)); return d; }");
-  em.line("__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) { unsigned long long d; asm(\"mul.rn.f32x2 %0, %1, %2;\" : \"=l\"(d) : \"l\"(a), \"l\"(b)); return d; }");
-  em.line("__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) { unsigned long long d; asm(\"add.rn.f32x2 %0, %1, %2;\" : \"=l\"(d) : \"l\"(a), \"l\"(b)); return d; }");
+  emit_pair_ops(em);
   emit_chunk_define(em);
   int nacc = pl.nout;
   if (sh.coop) {
@@ -1914,6 +1919,15 @@ BwdShape choose_backward_shape(const Plan& pl, int dtype) {
   b.ipw = 32 / TL;
   b.block = 128;
   b.ok = true;
+  // staged edges kernel: one receiver per warp, channel pairs per lane, 16-byte rows
+  const int elem = dtype == E3CONV_F16 ? 2 : 4;
+  b.s_bytes = static_cast<int>(pl.paths.size()) * pl.C * elem;
+  b.x_bytes = pl.nx * pl.C * elem;
+  b.y_bytes = (pl.ny * elem + 15) / 16 * 16;
+  b.stage_bytes = b.s_bytes + b.x_bytes + b.y_bytes;
+  b.smem = (b.block / 32) * 2 * b.stage_bytes;
+  b.staged = TL == 32 && V % 2 == 0 && b.s_bytes % 16 == 0 && b.x_bytes % 16 == 0 &&
+             (pl.ny * elem) % 4 == 0 && b.smem <= 112 * 1024;
   return b;
 }
 
@@ -2089,6 +2103,259 @@ std::string bwd_edges_source(const Plan& pl, int dtype, const BwdShape& b) {
   return em.o.str();
 }
 
+// Edges kernel, staged: a warp per receiver row (32 lanes x V channels = C), its g row in
+// registers as channel pairs; a two-stage per-warp ring in shared memory receives each edge's
+// s row, sender row x and Y row by 16-byte cp.async copies (the Y row by 4-byte copies),
+// issued one edge ahead.  Per edge and path, with A_ik = sum_j c_ijk Y_j formed per lane:
+//   t_k = sum_i A_ik x_i                       (channel pairs, fma.rn.f32x2)
+//   gs[e, p, c] = (1/N) sum_k g_k t_k
+//   W_ik = sum_{lane's channels} (s x_i) g_k,   dY_j += sum_{(i,k)} c_ijk W_ik
+// then dY is summed over the warp's lanes and lane 0 stores it.
+std::string bwd_edges_staged_source(const Plan& pl, int dtype, const BwdShape& b) {
+  Emitter em;
+  const std::string T = bwd_prelude(em, pl, dtype, b);
+  emit_pair_ops(em);
+  em.line("__device__ __forceinline__ void upk(unsigned long long w, float& lo, float& hi) { asm(\"mov.b64 {%0, %1}, %2;\" : \"=f\"(lo), \"=f\"(hi) : \"l\"(w)); }");
+  em.line("__device__ __forceinline__ void cp16(void* dst, const void* src) { asm volatile(\"cp.async.cg.shared.global [%0], [%1], 16;\" :: \"r\"(static_cast<unsigned int>(__cvta_generic_to_shared(dst))), \"l\"(src) : \"memory\"); }");
+  em.line("__device__ __forceinline__ void cp4(void* dst, const void* src) { asm volatile(\"cp.async.ca.shared.global [%0], [%1], 4;\" :: \"r\"(static_cast<unsigned int>(__cvta_generic_to_shared(dst))), \"l\"(src) : \"memory\"); }");
+  em.line("__device__ __forceinline__ void cp_commit() { asm volatile(\"cp.async.commit_group;\" ::: \"memory\"); }");
+  em.line("__device__ __forceinline__ void cp_wait1() { asm volatile(\"cp.async.wait_group 1;\" ::: \"memory\"); }");
+  em.line("__device__ __forceinline__ void cp_wait0() { asm volatile(\"cp.async.wait_group 0;\" ::: \"memory\"); }");
+  const bool f16 = dtype == E3CONV_F16;
+  const int V = b.V, NG = V / 2, elem = f16 ? 2 : 4;
+  const long long s_row = static_cast<long long>(pl.paths.size()) * pl.C;
+  const int SB = b.stage_bytes;
+  em.line("extern \"C\" __global__ void __launch_bounds__(" + S(b.block) + ") e3conv_bwd_edges(");
+  em.line("    const " + T + "* __restrict__ x, const " + T + "* __restrict__ Y, const " + T +
+          "* __restrict__ s,");
+  em.line("    const int* __restrict__ senders, const int* __restrict__ row_ptr, int num_nodes,");
+  em.line("    const float* __restrict__ g, float* __restrict__ gY, float* __restrict__ gs,");
+  em.line("    float inv_avg, unsigned int* __restrict__ status)");
+  em.line("{");
+  em.ind++;
+  em.line("extern __shared__ __align__(16) unsigned char smem_[];");
+  em.line("const int lane = threadIdx.x & 31;");
+  em.line("const long long bb = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;");
+  em.line("if (bb >= num_nodes) return;  // the whole warp (one receiver) leaves");
+  em.line("unsigned char* ring = smem_ + (threadIdx.x >> 5) * " + S(2 * SB) + ";");
+  em.line("const int u0 = lane * " + S(V) + ";");
+  em.line("const int e_base = __ldg(row_ptr), e_end = __ldg(row_ptr + num_nodes);");
+  em.line("int e0 = row_ptr[bb], e1 = row_ptr[bb + 1];");
+  em.line("if (e0 < e_base || e1 < e0 || e1 > e_end) { if (lane == 0) atomicOr(status, 1u); e1 = e0; }");
+  em.line("if (e0 == e1) return;");
+  // g row as pairs
+  for (int k = 0; k < pl.nout; ++k) {
+    const std::string src = "g + bb * " + S(static_cast<long long>(pl.nout) * pl.C) + " + " +
+                            S(static_cast<long long>(k) * pl.C) + " + u0";
+    if (NG == 2) {
+      em.line("unsigned long long g" + S(k) + "_0, g" + S(k) + "_1; { const float4 t_ = ldg_f4(" + src +
+              "); g" + S(k) + "_0 = pk(t_.x, t_.y); g" + S(k) + "_1 = pk(t_.z, t_.w); }");
+    } else {
+      for (int q = 0; q < NG; ++q)
+        em.line("unsigned long long g" + S(k) + "_" + S(q) + "; { const float2 t_ = ldg_f2(" + src +
+                " + " + S(2 * q) + "); g" + S(k) + "_" + S(q) + " = pk(t_.x, t_.y); }");
+    }
+  }
+  // copy issue of edge e into stage st (every lane; the s and x rows in 16-byte pieces)
+  em.line("auto issue = [&](int e, int st) {");
+  em.ind++;
+  em.line("const long long le = e - e_base;");
+  em.line("const int a = senders[le];");
+  em.line("const bool valid = (unsigned int)a < (unsigned int)num_nodes;");
+  em.line("if (!valid && lane == 0) atomicOr(status, 2u);");
+  em.line("unsigned char* dst = ring + st * " + S(SB) + ";");
+  em.line("const unsigned char* ssrc = reinterpret_cast<const unsigned char*>(s + le * " + S(s_row) + ");");
+  em.line("#pragma unroll");
+  em.line("for (int q = lane; q < " + S(b.s_bytes / 16) + "; q += 32) cp16(dst + 16 * q, ssrc + 16 * q);");
+  em.line("if (valid) {");
+  em.line("  const unsigned char* xsrc = reinterpret_cast<const unsigned char*>(x + (long long)a * " +
+          S(static_cast<long long>(pl.nx) * pl.C) + ");");
+  em.line("  #pragma unroll");
+  em.line("  for (int q = lane; q < " + S(b.x_bytes / 16) + "; q += 32) cp16(dst + " + S(b.s_bytes) +
+          " + 16 * q, xsrc + 16 * q);");
+  em.line("} else {");
+  em.line("  #pragma unroll");
+  em.line("  for (int q = lane; q < " + S(b.x_bytes / 16) + "; q += 32) *reinterpret_cast<uint4*>(dst + " +
+          S(b.s_bytes) + " + 16 * q) = make_uint4(0u, 0u, 0u, 0u);");
+  em.line("}");
+  em.line("const unsigned char* ysrc = reinterpret_cast<const unsigned char*>(Y + le * " + S(pl.ny) + ");");
+  em.line("for (int q = lane; q < " + S(pl.ny * elem / 4) + "; q += 32) cp4(dst + " +
+          S(b.s_bytes + b.x_bytes) + " + 4 * q, ysrc + 4 * q);");
+  em.line("cp_commit();");
+  em.ind--;
+  em.line("};");
+  em.line("const unsigned long long inv2 = bc(inv_avg);");
+  em.line("issue(e0, 0);");
+  em.line("#pragma unroll 1");
+  em.line("for (int e = e0; e < e1; ++e) {");
+  em.ind++;
+  em.line("const int st = (e - e0) & 1;");
+  em.line("if (e + 1 < e1) issue(e + 1, st ^ 1); else cp_commit();");
+  em.line("cp_wait1();");
+  em.line("__syncwarp();");
+  em.line("const long long le = e - e_base;");
+  em.line("const unsigned char* cur = ring + st * " + S(SB) + ";");
+  em.line("const " + T + "* ys = reinterpret_cast<const " + T + "*>(cur + " + S(b.s_bytes + b.x_bytes) + ");");
+  emit_y_load(em, pl, dtype, "lds", "ys");
+  em.line("const " + T + "* xs = reinterpret_cast<const " + T + "*>(cur + " + S(b.s_bytes) + ") + u0;");
+  em.line("const " + T + "* ss = reinterpret_cast<const " + T + "*>(cur) + u0;");
+  em.line("float* gsr = gs + le * " + S(s_row) + " + u0;");
+  {
+    std::string dy = "float";
+    for (int j = 0; j < pl.ny; ++j) dy += std::string(j ? "," : "") + " dy" + S(j) + " = 0.f";
+    em.line(dy + ";");
+  }
+  // loads V channels of a shared row into NG pairs name_0 .. name_{NG-1}
+  auto load_pairs = [&](const std::string& ptr, const std::string& name) {
+    if (f16) {
+      if (NG == 2) {
+        em.line("unsigned long long " + name + "_0, " + name + "_1; { const uint2 t_ = lds_u2(" + ptr +
+                "); " + name + "_0 = pk(lo_h2f(t_.x), hi_h2f(t_.x)); " + name +
+                "_1 = pk(lo_h2f(t_.y), hi_h2f(t_.y)); }");
+      } else {
+        for (int q = 0; q < NG; ++q)
+          em.line("unsigned long long " + name + "_" + S(q) + "; { const unsigned int t_ = lds_u1(" + ptr +
+                  " + " + S(2 * q) + "); " + name + "_" + S(q) + " = pk(lo_h2f(t_), hi_h2f(t_)); }");
+      }
+    } else {
+      if (NG == 2) {
+        em.line("unsigned long long " + name + "_0, " + name + "_1; { const float4 t_ = lds_f4(" + ptr +
+                "); " + name + "_0 = pk(t_.x, t_.y); " + name + "_1 = pk(t_.z, t_.w); }");
+      } else {
+        for (int q = 0; q < NG; ++q)
+          em.line("unsigned long long " + name + "_" + S(q) + "; { const float2 t_ = lds_f2(" + ptr +
+                  " + " + S(2 * q) + "); " + name + "_" + S(q) + " = pk(t_.x, t_.y); }");
+      }
+    }
+  };
+  size_t p = 0;
+  while (p < pl.paths.size()) {
+    const int n1 = pl.paths[p].n1;
+    size_t q = p;
+    while (q < pl.paths.size() && pl.paths[q].n1 == n1) ++q;
+    const Path& first = pl.paths[p];
+    const int d1 = 2 * first.l1 + 1;
+    em.line("{  // node irrep " + S(n1) + " (l=" + S(first.l1) + ")");
+    em.ind++;
+    for (size_t r = p; r < q; ++r) {
+      const Path& P = pl.paths[r];
+      const int d3 = 2 * P.l3 + 1;
+      em.line("{  // path " + S(r) + ": " + S(P.l1) + " x " + S(P.l2) + " -> " + S(P.l3));
+      em.ind++;
+      load_pairs("ss + " + S(static_cast<long long>(r) * pl.C), "s");
+      // distinct (i, k) of the path with their (j, c) terms
+      std::map<std::pair<int, int>, std::vector<std::pair<int, double>>> ik;
+      for (const auto& n : P.nnz) ik[{n.i, n.k}].push_back({n.j, n.c});
+      std::vector<bool> zi(d1, false), tk(d3, false);
+      for (const auto& kv : ik) {
+        zi[kv.first.first] = true;
+        tk[kv.first.second] = true;
+      }
+      {
+        std::string decl;
+        for (int k = 0; k < d3; ++k)
+          if (tk[k])
+            for (int g = 0; g < NG; ++g)
+              decl += (decl.empty() ? "" : ", ") + std::string("t") + S(k) + "_" + S(g) + " = 0ull";
+        if (!decl.empty()) em.line("unsigned long long " + decl + ";");
+      }
+      // (i, k) in i-major order: z_i = s x_i is formed just before its first use, so one z_i
+      // is live at a time
+      std::vector<bool> started(d3, false);
+      int zopen = -1;
+      for (const auto& kv : ik) {
+        const int i = kv.first.first, k = kv.first.second;
+        if (i != zopen) {
+          if (zopen >= 0) {
+            em.ind--;
+            em.line("}");
+          }
+          em.line("{  // x" + S(i) + " (from the ring) and z" + S(i) + " = s x" + S(i));
+          em.ind++;
+          load_pairs("xs + " + S((first.x_off + i) * pl.C), "x" + S(i));
+          for (int g = 0; g < NG; ++g)
+            em.line("const unsigned long long z" + S(i) + "_" + S(g) + " = mul2(s_" + S(g) + ", x" + S(i) +
+                    "_" + S(g) + ");");
+          zopen = i;
+        }
+        std::string expr;
+        for (const auto& jc : kv.second) {
+          const std::string yj = "y" + S(P.y_off + jc.first);
+          expr = expr.empty() ? flt(jc.second) + " * " + yj
+                              : "fmaf(" + flt(jc.second) + ", " + yj + ", " + expr + ")";
+        }
+        em.line("{  // (i, k) = (" + S(i) + ", " + S(k) + ")");
+        em.ind++;
+        em.line("const unsigned long long A_ = bc(" + expr + ");");
+        for (int g = 0; g < NG; ++g) {
+          const std::string tv = "t" + S(k) + "_" + S(g), xv = "x" + S(i) + "_" + S(g);
+          em.line(tv + " = " + (started[k] ? "fma2(A_, " + xv + ", " + tv + ")" : "mul2(A_, " + xv + ")") + ";");
+        }
+        started[k] = true;
+        std::string w = "mul2(z" + S(i) + "_0, g" + S(P.out_off + k) + "_0)";
+        for (int g = 1; g < NG; ++g)
+          w = "fma2(z" + S(i) + "_" + S(g) + ", g" + S(P.out_off + k) + "_" + S(g) + ", " + w + ")";
+        em.line("float wl_, wh_; upk(" + w + ", wl_, wh_);");
+        em.line("const float W_ = wl_ + wh_;");
+        for (const auto& jc : kv.second) {
+          const std::string dj = "dy" + S(P.y_off + jc.first);
+          em.line(dj + " = fmaf(" + flt(jc.second) + ", W_, " + dj + ");");
+        }
+        em.ind--;
+        em.line("}");
+      }
+      if (zopen >= 0) {
+        em.ind--;
+        em.line("}");
+      }
+      // gs[e, p, u0 ..] = inv_avg sum_k g_k t_k
+      em.line("{");
+      em.ind++;
+      for (int g = 0; g < NG; ++g) {
+        std::string a_;
+        for (int k = 0; k < d3; ++k) {
+          if (!tk[k]) continue;
+          const std::string gk = "g" + S(P.out_off + k) + "_" + S(g), tv = "t" + S(k) + "_" + S(g);
+          a_ = a_.empty() ? "mul2(" + gk + ", " + tv + ")" : "fma2(" + gk + ", " + tv + ", " + a_ + ")";
+        }
+        em.line("const unsigned long long o" + S(g) + "_ = " + (a_.empty() ? "0ull" : "mul2(inv2, " + a_ + ")") + ";");
+      }
+      const std::string dst = "gsr + " + S(static_cast<long long>(r) * pl.C);
+      if (NG == 2) {
+        em.line("float a0_, a1_, a2_, a3_; upk(o0_, a0_, a1_); upk(o1_, a2_, a3_);");
+        em.line("*reinterpret_cast<float4*>(" + dst + ") = make_float4(a0_, a1_, a2_, a3_);");
+      } else {
+        for (int g = 0; g < NG; ++g)
+          em.line("{ float a_, b_; upk(o" + S(g) + "_, a_, b_); *reinterpret_cast<float2*>(" + dst + " + " +
+                  S(2 * g) + ") = make_float2(a_, b_); }");
+      }
+      em.ind--;
+      em.line("}");
+      em.ind--;
+      em.line("}");
+    }
+    em.ind--;
+    em.line("}");
+    p = q;
+  }
+  for (int off = 16; off >= 1; off /= 2)
+    for (int j = 0; j < pl.ny; ++j)
+      em.line("dy" + S(j) + " += __shfl_xor_sync(0xffffffffu, dy" + S(j) + ", " + S(off) + ");");
+  em.line("if (lane == 0) {");
+  em.ind++;
+  for (int j = 0; j < pl.ny; ++j)
+    em.line("gY[le * " + S(pl.ny) + " + " + S(j) + "] = inv_avg * dy" + S(j) + ";");
+  em.ind--;
+  em.line("}");
+  em.line("__syncwarp();  // every lane has read this stage before the next edge's copies reuse it");
+  em.ind--;
+  em.line("}");
+  em.line("cp_wait0();");
+  em.ind--;
+  em.line("}");
+  return em.o.str();
+}
+
 std::string bwd_nodes_source(const Plan& pl, int dtype, const BwdShape& b) {
   Emitter em;
   const std::string T = bwd_prelude(em, pl, dtype, b);
@@ -2186,7 +2453,8 @@ std::string bwd_nodes_source(const Plan& pl, int dtype, const BwdShape& b) {
 }  // namespace
 
 std::string generate_backward_source(const Plan& pl, int dtype, const BwdShape& b, bool nodes) {
-  return nodes ? bwd_nodes_source(pl, dtype, b) : bwd_edges_source(pl, dtype, b);
+  if (nodes) return bwd_nodes_source(pl, dtype, b);
+  return b.staged ? bwd_edges_staged_source(pl, dtype, b) : bwd_edges_source(pl, dtype, b);
 }
 
 // Standalone harmonics: one thread per edge evaluates the plan's polynomials of

@@ -96,6 +96,12 @@ struct AEntry {
 struct BwdShape {
   bool ok = false;
   int V = 1, TL = 32, ipw = 1, block = 128;
+  // edges kernel with a per-warp shared-memory ring: the next edge's scalars, sender row
+  // and harmonics are copied (cp.async) while this edge's products run; packed float32x2
+  // arithmetic over channel pairs
+  bool staged = false;
+  int s_bytes = 0, x_bytes = 0, y_bytes = 0, stage_bytes = 0;  // one stage: s, x, Y rows
+  int smem = 0;                                                // dynamic shared memory per block
 };
 
 struct BwdVariant {
@@ -137,9 +143,8 @@ struct RadialPlan {
   bool set = false;
   int nb = 0, hidden = 0, layers = 0, nout = 0, chunks = 0;
   double r_max = 0.0;
-  int scale_exp_h = 0, scale_exp_o = 0;   // weights scaled by 2^s before the float16 split
-  std::vector<float> w0;                  // [nb][hidden] float32
-  std::vector<unsigned char> wh, wo;      // packed hi / lo float16 operands
+  int scale_exp_0 = 0, scale_exp_h = 0, scale_exp_o = 0;  // weights scaled by 2^s before the split
+  std::vector<unsigned char> w0, wh, wo;  // packed hi / lo float16 operands
   void* d_w0 = nullptr;
   void* d_wh = nullptr;
   void* d_wo = nullptr;

@@ -8,7 +8,7 @@
 //   h_0[n] = sqrt(2/r) sin((n+1) pi d / r) / d * (1 + cos(pi d / r)) / 2   (d < r; 0 beyond;
 //            evaluated as sinpi / cospi of (n+1) d / r and d / r
 //            d = 0 takes the limit (n+1) pi / r)
-//   h_1    = SiLU(h_0 W_0)                      (num_basis -> hidden, CUDA cores)
+//   h_1    = SiLU(h_0 W_0)                      (num_basis -> hidden, tensor cores, K padded to 16)
 //   h_l+1  = SiLU(h_l W_l),  l = 1 .. L-1       (hidden -> hidden, tensor cores)
 //   s      = h_L W_L                            (hidden -> P*C, tensor cores)
 // with SiLU(v) = v / (1 + exp(-v)), no biases.
@@ -22,14 +22,17 @@
 // float32 rounding), which keeps the products at float32 accuracy; the
 // weights are scaled by a power of two before the split (undone exactly on
 // the way out) so that their lo parts stay normal float16 numbers.
-// The output layer runs in chunks of 32 columns: their weights stream through
-// four shared-memory buffers (bulk copies of prepacked chunks, issued three
-// chunks ahead), their products alternate between two tensor-memory buffers
-// (the MMAs of chunk c overlap the stores of chunk c-1).  Stores go through a
-// per-warp shared-memory transpose so that each warp instruction writes one
-// edge row's 32 consecutive outputs (coalesced), not 32 rows' scattered ones.  All waits are bounded: on
-// timeout a CTA sets bit 4 of the status word, drains what it issued
-// (bounded) and stops.
+// The output layer runs in chunks of 128 columns (one N = 128 MMA per K step
+// and split term): their weights are double-buffered in shared memory (bulk
+// copies of prepacked chunks), their products alternate between two
+// tensor-memory buffers, so the MMAs of chunk c overlap the stores of chunk
+// c-1.  Stores: each thread writes its edge's row segment of the chunk into a
+// shared-memory staging tile and hands it to the bulk-copy engine as one
+// contiguous store (cp.async.bulk shared -> global), so the threads neither
+// issue per-element stores nor wait for them; rows whose length or address
+// is not a multiple of 16 bytes are stored element by element instead.  All
+// waits are bounded: on timeout a CTA sets bit 4 of the status word, drains
+// what it issued (bounded) and stops.
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 
@@ -49,18 +52,20 @@ using namespace tc;
 using namespace tc_host;
 
 constexpr int kTile = 128;           // edges per tile (MMA M)
-constexpr int kMaxBasis = 16;        // radial bases (layer 0 is unrolled over them)
-constexpr int kChunk = 32;           // output columns per output-layer chunk (MMA N)
-constexpr int kWBufs = 4;            // output-weight chunk buffers in shared memory
-constexpr int kStage = 36;           // floats per staged row (16-byte rows, conflict-free)
-constexpr int kOutCol = 64;          // tensor-memory column of the output buffers (>= hidden)
+constexpr int kMaxBasis = 16;        // radial bases = the K of layer 0's MMA (zero-padded)
+constexpr int kChunk = 128;          // output columns per output-layer chunk (MMA N)
+constexpr int kWBufs = 2;            // output-weight chunk buffers in shared memory
+constexpr int kStage = kChunk + 4;   // floats per staged row (16-byte rows, conflict-free)
+constexpr int kOutCol = 128;         // tensor-memory column of the output buffers (>= hidden)
+constexpr int kTmemCols = 512;       // hidden D [0, H) and two output buffers of kChunk
 
 struct RadialArgs {
   const float* vec;        // [E][4] edge vectors (x, y, z, unused)
   long long num_edges;
-  const float* w0;         // [nb][H] float32 (layer 0, CUDA cores)
+  const unsigned char* w0; // layer 0: hi then lo, [H x kMaxBasis] K-major each
   const unsigned char* wh; // hidden layers 1..L-1: per layer hi then lo, [H x H] K-major each
   const unsigned char* wo; // output layer: per chunk hi then lo, [kChunk x H] K-major each
+  float w_scale_inv_0;     // 2^-s of layer 0's weight scale
   float w_scale_inv_h;     // 2^-s of the hidden weights' scale
   float w_scale_inv_o;     // 2^-s of the output weights' scale
   float pi_r, inv_r, norm; // pi / r_max, 1 / r_max and sqrt(2 / r_max)
@@ -72,15 +77,17 @@ struct RadialArgs {
   unsigned* status;
 };
 
-// Shared memory of one CTA (bytes): w0 (nb x H float32), the hidden layers'
-// weights, the activations (hi, lo), two output-weight chunks (hi, lo each),
-// barriers and the tensor-memory slot.
+// Shared memory of one CTA (bytes): layer 0's and the hidden layers' weights,
+// the basis values and the activations (hi, lo each), two output-weight chunks
+// (hi, lo each), the staged output rows, barriers and the tensor-memory slot.
 template <int H>
 struct Smem {
+  static constexpr int kW0 = H * kMaxBasis * 2;          // one [H x 16] float16 operand
+  static constexpr int kBas = kTile * kMaxBasis * 2;     // one [128 x 16] float16 operand
   static constexpr int kAct = kTile * H * 2;     // one K-major [128 x H] float16 operand
   static constexpr int kWhid = H * H * 2;        // one [H x H] float16 operand
   static constexpr int kWout = kChunk * H * 2;   // one [kChunk x H] float16 operand
-  static constexpr int kStageBytes = 4 * 32 * kStage * 4;  // transpose rows of the 4 warps
+  static constexpr int kStageBytes = kTile * kStage * 4;   // one staged row per edge
 };
 
 template <int H>
@@ -88,9 +95,10 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
   extern __shared__ __align__(1024) unsigned char sm[];
   using L = Smem<H>;
   const int tid = threadIdx.x, warp = tid >> 5;
-  float* w0s = reinterpret_cast<float*>(sm);                        // nb x H
-  unsigned char* whs = sm + ((a.nb * H * 4 + 1023) / 1024) * 1024;    // (layers-1) x (hi, lo)
-  unsigned char* act = whs + (a.layers - 1) * 2 * L::kWhid;           // hi, lo
+  unsigned char* w0s = sm;                                            // layer 0 (hi, lo)
+  unsigned char* whs = w0s + 2 * L::kW0;                              // (layers-1) x (hi, lo)
+  unsigned char* bas = whs + (a.layers - 1) * 2 * L::kWhid;           // basis values (hi, lo)
+  unsigned char* act = bas + 2 * L::kBas;                             // hi, lo
   unsigned char* wos = act + 2 * L::kAct;                             // 2 buffers x (hi, lo)
   float* stage = reinterpret_cast<float*>(wos + kWBufs * 2 * L::kWout);
   unsigned long long* bars = reinterpret_cast<unsigned long long*>(
@@ -101,14 +109,13 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
   unsigned long long* bar_wh = bars + kWBufs + 3;   // hidden weights landed
   unsigned* tslot = reinterpret_cast<unsigned*>(bars + kWBufs + 4);
 
-  for (int q = tid; q < a.nb * H; q += 128) w0s[q] = a.w0[q];
   if (tid == 0) {
     for (int k = 0; k < kWBufs + 4; ++k) mbar_init(bars + k, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 128;" ::"r"(
-                     smem_u32(tslot))
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tslot)), "n"(kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -126,16 +133,15 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
   // a timeout)
   unsigned pend_w = 0, pend_mma = 0;
   bool pend_hid = false, pend_wh = false;
-  if (a.layers > 1 && tid == 0) {
-    const unsigned bytes = static_cast<unsigned>((a.layers - 1) * 2 * L::kWhid);
-    mbar_expect(bar_wh, bytes);
-    bulk_g2s(whs, a.wh, bytes, bar_wh);
+  if (tid == 0) {  // layer 0's and the hidden layers' weights, once per CTA
+    const unsigned hb = static_cast<unsigned>((a.layers - 1) * 2 * L::kWhid);
+    mbar_expect(bar_wh, 2 * L::kW0 + hb);
+    bulk_g2s(w0s, a.w0, 2 * L::kW0, bar_wh);
+    if (hb) bulk_g2s(whs, a.wh, hb, bar_wh);
     pend_wh = true;
   }
-  if (a.layers > 1) {
-    ok = __syncthreads_and(mbar_wait(bar_wh, 0));
-    pend_wh = !ok;
-  }
+  ok = __syncthreads_and(mbar_wait(bar_wh, 0));
+  pend_wh = !ok;
   const float pi_r = a.pi_r;
   const float norm = a.norm;
   const long long tiles = (a.num_edges + kTile - 1) / kTile;
@@ -152,7 +158,7 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
         pend_w |= 1u << c;
       }
     }
-    // layer 0 on the CUDA cores: basis x cutoff, then SiLU(h0 W0)
+    // layer 0: basis x cutoff on the CUDA cores, SiLU(h0 W0) with h0 W0 on the tensor cores
     float h[H];
     {
       float d = 0.f;
@@ -170,14 +176,34 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
                    ? 0.f
                    : (d > 0.f ? norm * sinpif((n + 1) * t) / d : norm * (n + 1) * pi_r) * u;
       }
-#pragma unroll
-      for (int j = 0; j < H; ++j) {
-        float z = 0.f;
-#pragma unroll
-        for (int n = 0; n < kMaxBasis; ++n)
-          if (n < a.nb) z = fmaf(b[n], w0s[n * H + j], z);
-        h[j] = silu(z);
+      store_split_row<kMaxBasis>(bas, bas + L::kBas, tid, b, kTile);
+      fence_async_smem();
+      tc_before();
+      __syncthreads();
+      tc_after();
+      if (tid == 0) {
+        const unsigned id0 = idesc_f16(kTile, H);
+        mma_f16(t_hid, kmajor_desc(bas), kmajor_desc(w0s), id0, 0);
+        mma_f16(t_hid, kmajor_desc(bas), kmajor_desc(w0s + L::kW0), id0, 1);
+        mma_f16(t_hid, kmajor_desc(bas + L::kBas), kmajor_desc(w0s), id0, 1);
+        mma_commit(bar_hid);
+        pend_hid = true;
       }
+      ok = __syncthreads_and(mbar_wait(bar_hid, ph_hid));
+      tc_after();
+      if (!ok) break;
+      ph_hid ^= 1u;
+      pend_hid = false;
+#pragma unroll
+      for (int j0 = 0; j0 < H; j0 += 32) {
+        float v[32];
+        tmem_ld32(t_hid + lane_off + j0, v);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) h[j0 + q] = silu(v[q] * a.w_scale_inv_0);
+      }
+      tc_before();
+      __syncthreads();  // every thread has read D before the next layer's MMAs overwrite it
+      tc_after();
     }
     // hidden layers 1 .. L-1 on the tensor cores
     for (int l = 1; l < a.layers && ok; ++l) {
@@ -225,9 +251,12 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
     __syncthreads();
     tc_after();
     const unsigned id = idesc_f16(kTile, kChunk);
-    const int lane = tid & 31;
-    float* st = stage + warp * 32 * kStage;          // this warp's 32 staged rows
-    const long long row0 = tile * kTile + warp * 32;  // edge of staged row 0
+    // descriptors: the activations' hi / lo operands and the weight buffers; K step ks adds
+    // its byte offset / 16 to the start-address field
+    const unsigned long long d_ahi = kmajor_desc(act), d_alo = kmajor_desc(act + L::kAct);
+    const int elem = a.out_f16 ? 2 : 4;
+    const bool bulk = (static_cast<long long>(a.nout) * elem) % 16 == 0;
+    float* srow = stage + tid * kStage;              // this thread's staged row
     for (int c = 0; c <= a.chunks && ok; ++c) {
       if (c < a.chunks) {
         const int wb = c % kWBufs, buf = c & 1;
@@ -236,20 +265,22 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
         ph_w ^= 1u << wb;
         pend_w &= ~(1u << wb);
         if (tid == 0) {
-          const unsigned char* whi = wos + wb * 2 * L::kWout;
-          const unsigned char* wlo = whi + L::kWout;
+          const unsigned long long d_whi = kmajor_desc(wos + wb * 2 * L::kWout);
+          const unsigned long long d_wlo = kmajor_desc(wos + wb * 2 * L::kWout + L::kWout);
           const unsigned td = tmem + static_cast<unsigned>(kOutCol + kChunk * buf);
+#pragma unroll
           for (int ks = 0; ks < H / 16; ++ks) {
-            const int ao = ks * kTile * 32, bo = ks * kChunk * 32;
-            mma_f16(td, kmajor_desc(act + ao), kmajor_desc(whi + bo), id, ks > 0);
-            mma_f16(td, kmajor_desc(act + ao), kmajor_desc(wlo + bo), id, 1);
-            mma_f16(td, kmajor_desc(act + L::kAct + ao), kmajor_desc(whi + bo), id, 1);
+            const unsigned long long ao = static_cast<unsigned long long>(ks * kTile * 32) >> 4;
+            const unsigned long long bo = static_cast<unsigned long long>(ks * kChunk * 32) >> 4;
+            mma_f16(td, d_ahi + ao, d_whi + bo, id, ks > 0);
+            mma_f16(td, d_ahi + ao, d_wlo + bo, id, 1);
+            mma_f16(td, d_alo + ao, d_whi + bo, id, 1);
           }
           mma_commit(bar_mma + buf);
           pend_mma |= 1u << buf;
         }
       }
-      if (c >= 1) {  // chunk c-1: its weight buffer takes chunk c-1+kWBufs, then its stores
+      if (c >= 1) {  // chunk c-1: its weight buffer takes chunk c+1, then its stores
         const int pb = (c - 1) & 1, pw = (c - 1) % kWBufs;
         ok = __syncthreads_and(mbar_wait(bar_mma + pb, (ph_mma >> pb) & 1u));
         tc_after();
@@ -263,36 +294,49 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
                    bar_w + pw);
           pend_w |= 1u << pw;
         }
-        float v[32];
-        tmem_ld32(tmem + static_cast<unsigned>(kOutCol + kChunk * pb) + lane_off, v);
+        const int col0 = (c - 1) * kChunk;
+        const int cols = min(kChunk, a.nout - col0);
         const float f = a.w_scale_inv_o;
-#pragma unroll
-        for (int q = 0; q < 32; q += 4)
-          *reinterpret_cast<float4*>(st + lane * kStage + q) =
-              make_float4(v[q] * f, v[q + 1] * f, v[q + 2] * f, v[q + 3] * f);
-        __syncwarp();
-        // lane l writes column (c-1) * kChunk + l of the warp's 32 rows: one row per instruction
-        const int col = (c - 1) * kChunk + lane;
-        if (col < a.nout) {
+        // the previous chunk's bulk store has finished reading this thread's staged row
+        bulk_wait_read();
+#pragma unroll 1
+        for (int j0 = 0; j0 < kChunk; j0 += 32) {
+          float v[32];
+          tmem_ld32(tmem + static_cast<unsigned>(kOutCol + kChunk * pb + j0) + lane_off, v);
           if (a.out_f16) {
-            __half* dst = static_cast<__half*>(a.s) + row0 * a.nout + col;
-#pragma unroll 8
-            for (int r = 0; r < 32; ++r)
-              if (row0 + r < a.num_edges) dst[static_cast<long long>(r) * a.nout] = __float2half_rn(st[r * kStage + lane]);
+            unsigned* hrow = reinterpret_cast<unsigned*>(srow) + j0 / 2;
+#pragma unroll
+            for (int q = 0; q < 32; q += 8)
+              *reinterpret_cast<uint4*>(hrow + q / 2) =
+                  make_uint4(pack_half2(v[q] * f, v[q + 1] * f), pack_half2(v[q + 2] * f, v[q + 3] * f),
+                             pack_half2(v[q + 4] * f, v[q + 5] * f), pack_half2(v[q + 6] * f, v[q + 7] * f));
           } else {
-            float* dst = static_cast<float*>(a.s) + row0 * a.nout + col;
-#pragma unroll 8
-            for (int r = 0; r < 32; ++r)
-              if (row0 + r < a.num_edges) dst[static_cast<long long>(r) * a.nout] = st[r * kStage + lane];
+#pragma unroll
+            for (int q = 0; q < 32; q += 4)
+              *reinterpret_cast<float4*>(srow + j0 + q) =
+                  make_float4(v[q] * f, v[q + 1] * f, v[q + 2] * f, v[q + 3] * f);
           }
         }
-        __syncwarp();  // staged rows read before the next chunk overwrites them
+        if (valid) {
+          unsigned char* dst = static_cast<unsigned char*>(a.s) +
+                               (e * a.nout + col0) * static_cast<long long>(elem);
+          if (bulk) {
+            fence_async_smem();
+            bulk_s2g(dst, srow, static_cast<unsigned>(cols * elem));
+          } else if (a.out_f16) {
+            const unsigned short* hs = reinterpret_cast<const unsigned short*>(srow);
+            for (int q = 0; q < cols; ++q) reinterpret_cast<unsigned short*>(dst)[q] = hs[q];
+          } else {
+            for (int q = 0; q < cols; ++q) reinterpret_cast<float*>(dst)[q] = srow[q];
+          }
+        }
         tc_before();
         __syncthreads();  // chunk c-1's columns read by every thread before they are reused
         tc_after();
       }
     }
   }
+  bulk_wait_all();  // every row store of this thread has landed
   if (!ok && tid == 0) {
     atomicOr(a.status, 4u);
     // drain (bounded): copies and MMAs issued but not seen complete
@@ -307,7 +351,8 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
   __syncthreads();
   tc_after();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 128;" ::"r"(tmem) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kTmemCols)
+                 : "memory");
 }
 
 }  // namespace
@@ -329,7 +374,14 @@ int radial_prepare(RadialPlan& rp, int nb, double r_max, int hidden, int layers,
   rp.r_max = r_max;
   rp.nout = nout;
   rp.chunks = (nout + kChunk - 1) / kChunk;
-  rp.w0.assign(w0, w0 + static_cast<size_t>(nb) * hidden);
+  // layer 0: W_0^T as the MMA's B operand, [hidden x 16] K-major, bases beyond nb zero
+  const int s0 = weight_scale_exp(w0, static_cast<size_t>(nb) * hidden);
+  rp.scale_exp_0 = s0;
+  const float f0 = std::ldexp(1.0f, s0);
+  rp.w0.assign(static_cast<size_t>(2) * hidden * kMaxBasis * 2, 0);
+  pack_kmajor(rp.w0, 0, hidden, kMaxBasis, [&](int r, int k) {
+    return k < nb ? w0[static_cast<size_t>(k) * hidden + r] * f0 : 0.f;
+  });
   // hidden weights: one scale for all hidden layers
   int sh = 30;
   for (int l = 1; l < layers; ++l)
@@ -356,9 +408,9 @@ int radial_prepare(RadialPlan& rp, int nb, double r_max, int hidden, int layers,
 
 size_t radial_smem_bytes(const RadialPlan& rp) {
   const size_t H = rp.hidden;
-  const size_t w0 = (rp.nb * H * 4 + 1023) / 1024 * 1024;
-  return w0 + (rp.layers - 1) * 2 * H * H * 2 + 2 * kTile * H * 2 + kWBufs * 2 * kChunk * H * 2 +
-         4 * 32 * kStage * 4 + (kWBufs + 4) * 8 + 16;
+  return 2 * H * kMaxBasis * 2 + (rp.layers - 1) * 2 * H * H * 2 + 2 * kTile * kMaxBasis * 2 +
+         2 * kTile * H * 2 + kWBufs * 2 * kChunk * H * 2 +
+         static_cast<size_t>(kTile) * kStage * 4 + (kWBufs + 4) * 8 + 16;
 }
 
 int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, const void* dev_wo,
@@ -368,7 +420,8 @@ int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, 
   RadialArgs a;
   a.vec = vec;
   a.num_edges = num_edges;
-  a.w0 = static_cast<const float*>(dev_w0);
+  a.w0 = static_cast<const unsigned char*>(dev_w0);
+  a.w_scale_inv_0 = std::ldexp(1.0f, -rp.scale_exp_0);
   a.wh = static_cast<const unsigned char*>(dev_wh);
   a.wo = static_cast<const unsigned char*>(dev_wo);
   a.w_scale_inv_h = std::ldexp(1.0f, -rp.scale_exp_h);
@@ -393,8 +446,8 @@ int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, 
     if (e == cudaSuccess)
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 128, smem);
     if (e != cudaSuccess || per_sm < 1) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
-    // tensor memory: 128 columns per CTA, so at most four CTAs per SM
-    per_sm = std::min(per_sm, 4);
+    // tensor memory: all 512 columns per CTA, so one CTA per SM
+    per_sm = 1;
     const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, static_cast<long long>(grid) * per_sm));
     kernel<<<blocks, 128, smem, st>>>(a);
     return cudaSuccess;

@@ -49,6 +49,22 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// bulk store shared -> global of one thread's contiguous segment (both addresses and the
+// size multiples of 16 bytes), in this thread's bulk async-group
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, unsigned bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// this thread's bulk stores have finished reading their shared-memory source
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// this thread's bulk stores are complete
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -104,7 +120,8 @@ __device__ __forceinline__ void tmem_ld32(unsigned addr, float* v) {
   for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(r[q]);
 }
 
-__device__ __forceinline__ float silu(float v) { return v / (1.0f + expf(-v)); }
+// SiLU(v) = v / (1 + e^-v): expf, then the correctly rounded reciprocal instead of a division
+__device__ __forceinline__ float silu(float v) { return v * __frcp_rn(1.0f + expf(-v)); }
 
 // two floats rounded to float16, low half first
 __device__ __forceinline__ unsigned pack_half2(float lo, float hi) {

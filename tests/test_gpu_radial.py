@@ -112,3 +112,26 @@ def test_radial_rejects_widths_beyond_shared_memory():
     rng = np.random.default_rng(0)
     with pytest.raises(e3.E3ConvError):
         conv.set_radial_mlp(2.0, _weights(rng, 8, 128, 2, conv.num_paths * conv.C))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16"])
+def test_radial_scalars_rows_not_multiple_of_16_bytes(cuda_device, dtype):
+    # P*C = 5 * 3 = 15 scalars per edge: rows of 60 (float32) or 30 (float16) bytes take the
+    # element-by-element store path instead of the bulk row copies
+    irreps = ("3x0e+3x1o", SH3, "3x0e+3x1o")
+    conv = e3.Conv(*irreps, 10.0, dtype=dtype)
+    nout = conv.num_paths * conv.C
+    assert (nout * (2 if dtype == "f16" else 4)) % 16 != 0
+    rng = np.random.default_rng(21)
+    ws = _weights(rng, 8, 64, 2, nout)
+    conv.set_radial_mlp(3.0, ws)
+    E = 300
+    v4 = _vec4(rng.normal(size=(E, 3)))
+    s = conv.radial_scalars(to_dev(v4))
+    torch.cuda.synchronize()
+    assert conv.check()
+    got = s.float().cpu().numpy().reshape(E, nout)
+    ref = _reference(v4, 3.0, ws)
+    scale = np.abs(ref).max(axis=0)
+    err = (np.abs(got - ref) / np.where(scale > 0, scale, 1)).max()
+    assert err <= (2e-3 if dtype == "f16" else 1e-5), err
