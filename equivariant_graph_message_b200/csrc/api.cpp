@@ -231,9 +231,12 @@ int prepare_backward(Plan& pl) {
         return fail(E3CONV_ERR_CUDA, "loading the backward kernels failed");
       }
     }
-    if (v.shape.staged &&
-        d.FuncSetAttribute(v.fn[0], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES, v.shape.smem) !=
-            CUDA_SUCCESS) {
+    if ((v.shape.staged &&
+         d.FuncSetAttribute(v.fn[0], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES, v.shape.smem) !=
+             CUDA_SUCCESS) ||
+        (v.shape.nstaged &&
+         d.FuncSetAttribute(v.fn[1], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES, v.shape.nsmem) !=
+             CUDA_SUCCESS)) {
       for (int q = 0; q < 2; ++q) d.ModuleUnload(v.module[q]);
       return fail(E3CONV_ERR_CUDA, "cannot reserve the backward edges kernel's shared memory");
     }
@@ -1090,8 +1093,9 @@ int e3conv_backward(e3conv_plan h, const void* x, const void* Y, const void* s,
                     const_cast<int32_t**>(&receivers), const_cast<int32_t**>(&row_ptr),
                     const_cast<int32_t**>(&sender_row_ptr), const_cast<int32_t**>(&sender_perm),
                     &n32, const_cast<float**>(&grad_out), &grad_x, &inv_avg, &pl.status};
-    if (driver().LaunchKernel(bv.fn[1], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1, 0, st,
-                              args, nullptr) != CUDA_SUCCESS)
+    if (driver().LaunchKernel(bv.fn[1], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1,
+                              b.nstaged ? static_cast<unsigned>(b.nsmem) : 0u, st, args,
+                              nullptr) != CUDA_SUCCESS)
       return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed (backward, nodes)");
   }
   return E3CONV_OK;

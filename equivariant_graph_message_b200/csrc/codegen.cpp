@@ -1928,6 +1928,11 @@ BwdShape choose_backward_shape(const Plan& pl, int dtype) {
   b.smem = (b.block / 32) * 2 * b.stage_bytes;
   b.staged = TL == 32 && V % 2 == 0 && b.s_bytes % 16 == 0 && b.x_bytes % 16 == 0 &&
              (pl.ny * elem) % 4 == 0 && b.smem <= 112 * 1024;
+  b.g_bytes = pl.nout * pl.C * 4;
+  b.nstage_bytes = b.s_bytes + b.g_bytes + b.y_bytes;
+  b.nsmem = (b.block / 32) * 2 * b.nstage_bytes;
+  b.nstaged = TL == 32 && V % 2 == 0 && b.s_bytes % 16 == 0 && b.g_bytes % 16 == 0 &&
+              (pl.ny * elem) % 4 == 0 && b.nsmem <= 220 * 1024;
   return b;
 }
 
@@ -2356,6 +2361,192 @@ std::string bwd_edges_staged_source(const Plan& pl, int dtype, const BwdShape& b
   return em.o.str();
 }
 
+// Nodes kernel, staged: a warp per sender (32 lanes x V channels = C) walks the sender's
+// edges in sender order; a two-stage per-warp ring receives each edge's s row, its
+// receiver's gradient row g (float32) and its Y row by cp.async, one edge ahead.  Per edge
+// and path, with A_ik = sum_j c_ijk Y_j formed per lane and u_k = s g_k (channel pairs):
+//   h_i += sum_k A_ik u_k,   grad_x[a] = (1/N) h.
+std::string bwd_nodes_staged_source(const Plan& pl, int dtype, const BwdShape& b) {
+  Emitter em;
+  const std::string T = bwd_prelude(em, pl, dtype, b);
+  emit_pair_ops(em);
+  em.line("__device__ __forceinline__ void upk(unsigned long long w, float& lo, float& hi) { asm(\"mov.b64 {%0, %1}, %2;\" : \"=f\"(lo), \"=f\"(hi) : \"l\"(w)); }");
+  em.line("__device__ __forceinline__ void cp16(void* dst, const void* src) { asm volatile(\"cp.async.cg.shared.global [%0], [%1], 16;\" :: \"r\"(static_cast<unsigned int>(__cvta_generic_to_shared(dst))), \"l\"(src) : \"memory\"); }");
+  em.line("__device__ __forceinline__ void cp4(void* dst, const void* src) { asm volatile(\"cp.async.ca.shared.global [%0], [%1], 4;\" :: \"r\"(static_cast<unsigned int>(__cvta_generic_to_shared(dst))), \"l\"(src) : \"memory\"); }");
+  em.line("__device__ __forceinline__ void cp_commit() { asm volatile(\"cp.async.commit_group;\" ::: \"memory\"); }");
+  em.line("__device__ __forceinline__ void cp_wait1() { asm volatile(\"cp.async.wait_group 1;\" ::: \"memory\"); }");
+  em.line("__device__ __forceinline__ void cp_wait0() { asm volatile(\"cp.async.wait_group 0;\" ::: \"memory\"); }");
+  const bool f16 = dtype == E3CONV_F16;
+  const int V = b.V, NG = V / 2, elem = f16 ? 2 : 4;
+  const long long s_row = static_cast<long long>(pl.paths.size()) * pl.C;
+  const long long g_row = static_cast<long long>(pl.nout) * pl.C;
+  const int SB = b.nstage_bytes;
+  const int g_off = b.s_bytes, y_off = b.s_bytes + b.g_bytes;
+  em.line("extern \"C\" __global__ void __launch_bounds__(" + S(b.block) + ") e3conv_bwd_nodes(");
+  em.line("    const " + T + "* __restrict__ Y, const " + T + "* __restrict__ s,");
+  em.line("    const int* __restrict__ receivers, const int* __restrict__ row_ptr,");
+  em.line("    const int* __restrict__ sender_row_ptr, const int* __restrict__ sender_perm,");
+  em.line("    int num_nodes, const float* __restrict__ g, float* __restrict__ gx, float inv_avg,");
+  em.line("    unsigned int* __restrict__ status)");
+  em.line("{");
+  em.ind++;
+  em.line("extern __shared__ __align__(16) unsigned char smem_[];");
+  em.line("const int lane = threadIdx.x & 31;");
+  em.line("const long long a = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;");
+  em.line("if (a >= num_nodes) return;  // the whole warp (one sender) leaves");
+  em.line("unsigned char* ring = smem_ + (threadIdx.x >> 5) * " + S(2 * SB) + ";");
+  em.line("const int u0 = lane * " + S(V) + ";");
+  em.line("const int e_base = __ldg(row_ptr), e_end = __ldg(row_ptr + num_nodes);");
+  em.line("const int ne = e_end - e_base;");
+  for (int i = 0; i < pl.nx; ++i) {
+    std::string l = "unsigned long long";
+    for (int g = 0; g < NG; ++g) l += std::string(g ? "," : "") + " h" + S(i) + "_" + S(g) + " = 0ull";
+    em.line(l + ";");
+  }
+  em.line("int t0 = sender_row_ptr[a], t1 = sender_row_ptr[a + 1];");
+  em.line("if (t0 < 0 || t1 < t0 || t1 > ne) { if (lane == 0) atomicOr(status, 1u); t1 = t0; }");
+  em.line("auto issue = [&](int t, int st) {");
+  em.ind++;
+  em.line("int le = sender_perm[t];");
+  em.line("bool valid = (unsigned int)le < (unsigned int)ne;");
+  em.line("const int bb = valid ? receivers[le] : 0;");
+  em.line("valid = valid && (unsigned int)bb < (unsigned int)num_nodes;");
+  em.line("if (!valid && lane == 0) atomicOr(status, 2u);");
+  em.line("unsigned char* dst = ring + st * " + S(SB) + ";");
+  em.line("if (valid) {");
+  em.ind++;
+  em.line("const unsigned char* ssrc = reinterpret_cast<const unsigned char*>(s + (long long)le * " + S(s_row) + ");");
+  em.line("const unsigned char* gsrc = reinterpret_cast<const unsigned char*>(g + (long long)bb * " + S(g_row) + ");");
+  em.line("const unsigned char* ysrc = reinterpret_cast<const unsigned char*>(Y + (long long)le * " + S(pl.ny) + ");");
+  em.line("#pragma unroll");
+  em.line("for (int q = lane; q < " + S(b.s_bytes / 16) + "; q += 32) cp16(dst + 16 * q, ssrc + 16 * q);");
+  em.line("#pragma unroll");
+  em.line("for (int q = lane; q < " + S(b.g_bytes / 16) + "; q += 32) cp16(dst + " + S(g_off) + " + 16 * q, gsrc + 16 * q);");
+  em.line("for (int q = lane; q < " + S(pl.ny * elem / 4) + "; q += 32) cp4(dst + " + S(y_off) + " + 4 * q, ysrc + 4 * q);");
+  em.ind--;
+  em.line("} else {  // a bad index contributes nothing: a zero row of scalars and harmonics");
+  em.ind++;
+  em.line("#pragma unroll");
+  em.line("for (int q = lane; q < " + S(b.s_bytes / 16) + "; q += 32) *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(0u, 0u, 0u, 0u);");
+  em.line("#pragma unroll");
+  em.line("for (int q = lane; q < " + S(b.g_bytes / 16) + "; q += 32) *reinterpret_cast<uint4*>(dst + " + S(g_off) + " + 16 * q) = make_uint4(0u, 0u, 0u, 0u);");
+  em.line("for (int q = lane; q < " + S(b.y_bytes / 4) + "; q += 32) *reinterpret_cast<unsigned int*>(dst + " + S(y_off) + " + 4 * q) = 0u;");
+  em.ind--;
+  em.line("}");
+  em.line("cp_commit();");
+  em.ind--;
+  em.line("};");
+  em.line("if (t0 < t1) issue(t0, 0);");
+  em.line("#pragma unroll 1");
+  em.line("for (int t = t0; t < t1; ++t) {");
+  em.ind++;
+  em.line("const int st = (t - t0) & 1;");
+  em.line("if (t + 1 < t1) issue(t + 1, st ^ 1); else cp_commit();");
+  em.line("cp_wait1();");
+  em.line("__syncwarp();");
+  em.line("const unsigned char* cur = ring + st * " + S(SB) + ";");
+  em.line("const " + T + "* ys = reinterpret_cast<const " + T + "*>(cur + " + S(y_off) + ");");
+  emit_y_load(em, pl, dtype, "lds", "ys");
+  em.line("const " + T + "* ss = reinterpret_cast<const " + T + "*>(cur) + u0;");
+  em.line("const float* gs_ = reinterpret_cast<const float*>(cur + " + S(g_off) + ") + u0;");
+  auto load_s = [&](const std::string& ptr) {
+    if (f16) {
+      if (NG == 2)
+        em.line("unsigned long long s_0, s_1; { const uint2 t_ = lds_u2(" + ptr + "); s_0 = pk(lo_h2f(t_.x), hi_h2f(t_.x)); s_1 = pk(lo_h2f(t_.y), hi_h2f(t_.y)); }");
+      else
+        for (int q = 0; q < NG; ++q)
+          em.line("unsigned long long s_" + S(q) + "; { const unsigned int t_ = lds_u1(" + ptr + " + " + S(2 * q) + "); s_" + S(q) + " = pk(lo_h2f(t_), hi_h2f(t_)); }");
+    } else {
+      if (NG == 2)
+        em.line("unsigned long long s_0, s_1; { const float4 t_ = lds_f4(" + ptr + "); s_0 = pk(t_.x, t_.y); s_1 = pk(t_.z, t_.w); }");
+      else
+        for (int q = 0; q < NG; ++q)
+          em.line("unsigned long long s_" + S(q) + "; { const float2 t_ = lds_f2(" + ptr + " + " + S(2 * q) + "); s_" + S(q) + " = pk(t_.x, t_.y); }");
+    }
+  };
+  for (size_t o = 0; o < pl.outputs.size(); ++o) {
+    const int d3 = 2 * pl.outputs[o].l + 1, off = pl.outputs[o].off;
+    bool any = false;
+    for (const auto& P : pl.paths) any = any || P.o == static_cast<int>(o);
+    if (!any) continue;
+    em.line("{  // output irrep " + S(o));
+    em.ind++;
+    for (int k = 0; k < d3; ++k) {
+      if (NG == 2)
+        em.line("unsigned long long g" + S(k) + "_0, g" + S(k) + "_1; { const float4 t_ = lds_f4(gs_ + " +
+                S((off + k) * pl.C) + "); g" + S(k) + "_0 = pk(t_.x, t_.y); g" + S(k) + "_1 = pk(t_.z, t_.w); }");
+      else
+        for (int q = 0; q < NG; ++q)
+          em.line("unsigned long long g" + S(k) + "_" + S(q) + "; { const float2 t_ = lds_f2(gs_ + " +
+                  S((off + k) * pl.C + 2 * q) + "); g" + S(k) + "_" + S(q) + " = pk(t_.x, t_.y); }");
+    }
+    for (size_t r = 0; r < pl.paths.size(); ++r) {
+      const Path& P = pl.paths[r];
+      if (P.o != static_cast<int>(o)) continue;
+      em.line("{  // path " + S(r) + ": " + S(P.l1) + " x " + S(P.l2) + " -> " + S(P.l3));
+      em.ind++;
+      load_s("ss + " + S(static_cast<long long>(r) * pl.C));
+      std::map<std::pair<int, int>, std::vector<std::pair<int, double>>> ki;  // k-major
+      for (const auto& n : P.nnz) ki[{n.k, n.i}].push_back({n.j, n.c});
+      int uopen = -1;
+      for (const auto& kv : ki) {
+        const int k = kv.first.first, i = kv.first.second;
+        if (k != uopen) {
+          if (uopen >= 0) {
+            em.ind--;
+            em.line("}");
+          }
+          em.line("{  // u" + S(k) + " = s g" + S(k));
+          em.ind++;
+          for (int g = 0; g < NG; ++g)
+            em.line("const unsigned long long u" + S(k) + "_" + S(g) + " = mul2(s_" + S(g) + ", g" + S(k) + "_" + S(g) + ");");
+          uopen = k;
+        }
+        std::string expr;
+        for (const auto& jc : kv.second) {
+          const std::string yj = "y" + S(P.y_off + jc.first);
+          expr = expr.empty() ? flt(jc.second) + " * " + yj
+                              : "fmaf(" + flt(jc.second) + ", " + yj + ", " + expr + ")";
+        }
+        em.line("{ const unsigned long long A_ = bc(" + expr + ");");
+        for (int g = 0; g < NG; ++g) {
+          const std::string hv = "h" + S(P.x_off + i) + "_" + S(g);
+          em.line("  " + hv + " = fma2(A_, u" + S(k) + "_" + S(g) + ", " + hv + ");");
+        }
+        em.line("}");
+      }
+      if (uopen >= 0) {
+        em.ind--;
+        em.line("}");
+      }
+      em.ind--;
+      em.line("}");
+    }
+    em.ind--;
+    em.line("}");
+  }
+  em.line("__syncwarp();  // every lane has read this stage before the next edge's copies reuse it");
+  em.ind--;
+  em.line("}");
+  em.line("cp_wait0();");
+  em.line("const unsigned long long inv2 = bc(inv_avg);");
+  em.line("float* xo = gx + a * " + S(static_cast<long long>(pl.nx) * pl.C) + " + u0;");
+  for (int i = 0; i < pl.nx; ++i) {
+    const std::string dst = "xo + " + S(i * pl.C);
+    if (NG == 2) {
+      em.line("{ float a0_, a1_, a2_, a3_; upk(mul2(inv2, h" + S(i) + "_0), a0_, a1_); upk(mul2(inv2, h" + S(i) +
+              "_1), a2_, a3_); *reinterpret_cast<float4*>(" + dst + ") = make_float4(a0_, a1_, a2_, a3_); }");
+    } else {
+      for (int g = 0; g < NG; ++g)
+        em.line("{ float a_, b_; upk(mul2(inv2, h" + S(i) + "_" + S(g) + "), a_, b_); *reinterpret_cast<float2*>(" +
+                dst + " + " + S(2 * g) + ") = make_float2(a_, b_); }");
+    }
+  }
+  em.ind--;
+  em.line("}");
+  return em.o.str();
+}
+
 std::string bwd_nodes_source(const Plan& pl, int dtype, const BwdShape& b) {
   Emitter em;
   const std::string T = bwd_prelude(em, pl, dtype, b);
@@ -2453,7 +2644,7 @@ std::string bwd_nodes_source(const Plan& pl, int dtype, const BwdShape& b) {
 }  // namespace
 
 std::string generate_backward_source(const Plan& pl, int dtype, const BwdShape& b, bool nodes) {
-  if (nodes) return bwd_nodes_source(pl, dtype, b);
+  if (nodes) return b.nstaged ? bwd_nodes_staged_source(pl, dtype, b) : bwd_nodes_source(pl, dtype, b);
   return b.staged ? bwd_edges_staged_source(pl, dtype, b) : bwd_edges_source(pl, dtype, b);
 }
 

@@ -102,6 +102,9 @@ struct BwdShape {
   bool staged = false;
   int s_bytes = 0, x_bytes = 0, y_bytes = 0, stage_bytes = 0;  // one stage: s, x, Y rows
   int smem = 0;                                                // dynamic shared memory per block
+  // nodes kernel (grad_x, sender order) with the same kind of ring: s, g (float32) and Y rows
+  bool nstaged = false;
+  int g_bytes = 0, nstage_bytes = 0, nsmem = 0;
 };
 
 struct BwdVariant {

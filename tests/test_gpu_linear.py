@@ -18,6 +18,7 @@ pytestmark = pytest.mark.gpu
     ("64x0e+64x1o+64x2e", "128x0e+128x1e+128x1o+128x2e+128x3o"),     # unmatched 1e, 3o
     ("32x0e+32x1o", "256x1o+256x0e"),
     ("128x0e+128x1o+128x2e+128x3o", "16x3o+16x0e"),
+    ("128x0e+128x1o", "256x0e+256x1o"),                               # one staging buffer
 ])
 @pytest.mark.parametrize("nodes", [1, 5, 300, 2049])
 def test_linear_matches_the_oracle(cuda_device, ins, outs, nodes):
