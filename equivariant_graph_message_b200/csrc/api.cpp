@@ -895,9 +895,31 @@ int e3conv_radial_scalars(e3conv_plan h, const float* edge_vectors, int64_t num_
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, pl.device) != cudaSuccess)
     return fail(E3CONV_ERR_CUDA, "cannot query the SM count");
   std::string err;
+  // the output as a 2-D tensor [num_edges][P*C] for the kernel's TMA stores: boxes of 128 edge
+  // rows x 128 bytes, 128-byte swizzle; rows whose byte length is not a multiple of 16 cannot
+  // be described (the kernel then stores element by element)
+  const int elem = pl.dtype == E3CONV_F16 ? 2 : 4;
+  const int nout = static_cast<int>(pl.paths.size()) * pl.C;
+  CUtensorMap smap;
+  std::memset(&smap, 0, sizeof smap);
+  bool tma = (static_cast<long long>(nout) * elem) % 16 == 0 && num_edges < (1ll << 31) - 256 &&
+             driver().ok;
+  if (tma) {
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(nout), static_cast<cuuint64_t>(num_edges)};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(nout) * elem};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem), 128};
+    const cuuint32_t estr[2] = {1, 1};
+    tma = driver().TensorMapEncodeTiled(&smap, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                                        2, edge_scalars, gdim, gstride, box, estr,
+                                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                        CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
   const int rc = radial_launch(pl.radial, pl.radial.d_w0, pl.radial.d_wh, pl.radial.d_wo,
                                edge_vectors, num_edges, edge_scalars, pl.dtype == E3CONV_F16 ? 1 : 0,
-                               pl.status, sms, reinterpret_cast<cudaStream_t>(stream), err);
+                               pl.status, sms, reinterpret_cast<cudaStream_t>(stream), err,
+                               tma ? &smap : nullptr);
   return rc == E3CONV_OK ? rc : fail(rc, err);
 }
 

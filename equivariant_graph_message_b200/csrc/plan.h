@@ -225,7 +225,7 @@ int radial_prepare(RadialPlan& rp, int nb, double r_max, int hidden, int layers,
 size_t radial_smem_bytes(const RadialPlan& rp);
 int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, const void* dev_wo,
                   const float* vec, long long num_edges, void* s, int out_f16, unsigned* status,
-                  int grid, cudaStream_t st, std::string& err);
+                  int grid, cudaStream_t st, std::string& err, const CUtensorMap* smap);
 
 // linear.cu
 int linear_prepare(LinearPlan& lp, const std::vector<Irrep>& in, const std::vector<Irrep>& out,

@@ -26,13 +26,15 @@
 // and split term): their weights are double-buffered in shared memory (bulk
 // copies of prepacked chunks), their products alternate between two
 // tensor-memory buffers, so the MMAs of chunk c overlap the stores of chunk
-// c-1.  Stores: each thread writes its edge's row segment of the chunk into a
-// shared-memory staging tile and hands it to the bulk-copy engine as one
-// contiguous store (cp.async.bulk shared -> global), so the threads neither
-// issue per-element stores nor wait for them; rows whose length or address
-// is not a multiple of 16 bytes are stored element by element instead.  All
+// c-1.  Stores: the threads write the chunk's [128 edges x 128 columns] tile
+// into shared memory in the TMA's 128-byte swizzle (thread t, row t: its
+// 16-byte pieces land in distinct banks), and one thread stores it with 2-D
+// TMA tensor stores of 128 rows x 128 bytes (rows past the last edge and
+// columns past P*C are clipped by the TMA); rows whose byte length is not a
+// multiple of 16 are stored element by element instead.  All
 // waits are bounded: on timeout a CTA sets bit 4 of the status word, drains
 // what it issued (bounded) and stops.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 
@@ -55,7 +57,7 @@ constexpr int kTile = 128;           // edges per tile (MMA M)
 constexpr int kMaxBasis = 16;        // radial bases = the K of layer 0's MMA (zero-padded)
 constexpr int kChunk = 128;          // output columns per output-layer chunk (MMA N)
 constexpr int kWBufs = 2;            // output-weight chunk buffers in shared memory
-constexpr int kStage = kChunk + 4;   // floats per staged row (16-byte rows, conflict-free)
+constexpr int kStageBytes = kTile * kChunk * 4;  // one chunk's output tile (float32)
 constexpr int kOutCol = 128;         // tensor-memory column of the output buffers (>= hidden)
 constexpr int kTmemCols = 512;       // hidden D [0, H) and two output buffers of kChunk
 
@@ -74,6 +76,7 @@ struct RadialArgs {
   float r_max;
   void* s;                 // [E][nout] float32 or float16
   int out_f16;
+  int tma;                 // 1: TMA tensor stores through the map; 0: element stores
   unsigned* status;
 };
 
@@ -87,11 +90,11 @@ struct Smem {
   static constexpr int kAct = kTile * H * 2;     // one K-major [128 x H] float16 operand
   static constexpr int kWhid = H * H * 2;        // one [H x H] float16 operand
   static constexpr int kWout = kChunk * H * 2;   // one [kChunk x H] float16 operand
-  static constexpr int kStageBytes = kTile * kStage * 4;   // one staged row per edge
+
 };
 
 template <int H>
-__global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
+__global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a, const __grid_constant__ CUtensorMap smap) {
   extern __shared__ __align__(1024) unsigned char sm[];
   using L = Smem<H>;
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -100,9 +103,8 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
   unsigned char* bas = whs + (a.layers - 1) * 2 * L::kWhid;           // basis values (hi, lo)
   unsigned char* act = bas + 2 * L::kBas;                             // hi, lo
   unsigned char* wos = act + 2 * L::kAct;                             // 2 buffers x (hi, lo)
-  float* stage = reinterpret_cast<float*>(wos + kWBufs * 2 * L::kWout);
-  unsigned long long* bars = reinterpret_cast<unsigned long long*>(
-      reinterpret_cast<unsigned char*>(stage) + L::kStageBytes);
+  unsigned char* stage = wos + kWBufs * 2 * L::kWout;  // 1024-byte aligned (128-byte swizzle)
+  unsigned long long* bars = reinterpret_cast<unsigned long long*>(stage + kStageBytes);
   unsigned long long* bar_w = bars;                 // [kWBufs] output-weight chunk landed
   unsigned long long* bar_mma = bars + kWBufs;      // [2] output MMAs of a chunk done
   unsigned long long* bar_hid = bars + kWBufs + 2;  // hidden-layer MMAs done
@@ -254,9 +256,6 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
     // descriptors: the activations' hi / lo operands and the weight buffers; K step ks adds
     // its byte offset / 16 to the start-address field
     const unsigned long long d_ahi = kmajor_desc(act), d_alo = kmajor_desc(act + L::kAct);
-    const int elem = a.out_f16 ? 2 : 4;
-    const bool bulk = (static_cast<long long>(a.nout) * elem) % 16 == 0;
-    float* srow = stage + tid * kStage;              // this thread's staged row
     for (int c = 0; c <= a.chunks && ok; ++c) {
       if (c < a.chunks) {
         const int wb = c % kWBufs, buf = c & 1;
@@ -282,6 +281,9 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
       }
       if (c >= 1) {  // chunk c-1: its weight buffer takes chunk c+1, then its stores
         const int pb = (c - 1) & 1, pw = (c - 1) % kWBufs;
+        // the previous chunk's TMA stores have read the staging tile (thread 0 issued them);
+        // the barrier below publishes that to every thread
+        if (tid == 0) bulk_wait_read();
         ok = __syncthreads_and(mbar_wait(bar_mma + pb, (ph_mma >> pb) & 1u));
         tc_after();
         if (!ok) break;
@@ -297,37 +299,59 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a) {
         const int col0 = (c - 1) * kChunk;
         const int cols = min(kChunk, a.nout - col0);
         const float f = a.w_scale_inv_o;
-        // the previous chunk's bulk store has finished reading this thread's staged row
-        bulk_wait_read();
+        if (a.tma) {
+          // staging tile: per 128-byte column box (32 floats or 64 halves), row r at r * 128,
+          // its 16-byte piece q at (q ^ (r & 7)) * 16
 #pragma unroll 1
-        for (int j0 = 0; j0 < kChunk; j0 += 32) {
-          float v[32];
-          tmem_ld32(tmem + static_cast<unsigned>(kOutCol + kChunk * pb + j0) + lane_off, v);
-          if (a.out_f16) {
-            unsigned* hrow = reinterpret_cast<unsigned*>(srow) + j0 / 2;
+          for (int j0 = 0; j0 < kChunk; j0 += 32) {
+            float v[32];
+            tmem_ld32(tmem + static_cast<unsigned>(kOutCol + kChunk * pb + j0) + lane_off, v);
+            if (a.out_f16) {
+              unsigned char* box = stage + (j0 / 64) * (kTile * 128) + tid * 128;
 #pragma unroll
-            for (int q = 0; q < 32; q += 8)
-              *reinterpret_cast<uint4*>(hrow + q / 2) =
-                  make_uint4(pack_half2(v[q] * f, v[q + 1] * f), pack_half2(v[q + 2] * f, v[q + 3] * f),
-                             pack_half2(v[q + 4] * f, v[q + 5] * f), pack_half2(v[q + 6] * f, v[q + 7] * f));
-          } else {
+              for (int q = 0; q < 4; ++q) {
+                const int piece = (j0 % 64) / 8 + q;
+                *reinterpret_cast<uint4*>(box + ((piece ^ (tid & 7)) * 16)) =
+                    make_uint4(pack_half2(v[8 * q] * f, v[8 * q + 1] * f),
+                               pack_half2(v[8 * q + 2] * f, v[8 * q + 3] * f),
+                               pack_half2(v[8 * q + 4] * f, v[8 * q + 5] * f),
+                               pack_half2(v[8 * q + 6] * f, v[8 * q + 7] * f));
+              }
+            } else {
+              unsigned char* box = stage + (j0 / 32) * (kTile * 128) + tid * 128;
 #pragma unroll
-            for (int q = 0; q < 32; q += 4)
-              *reinterpret_cast<float4*>(srow + j0 + q) =
-                  make_float4(v[q] * f, v[q + 1] * f, v[q + 2] * f, v[q + 3] * f);
+              for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<float4*>(box + ((q ^ (tid & 7)) * 16)) =
+                    make_float4(v[4 * q] * f, v[4 * q + 1] * f, v[4 * q + 2] * f, v[4 * q + 3] * f);
+            }
           }
-        }
-        if (valid) {
-          unsigned char* dst = static_cast<unsigned char*>(a.s) +
-                               (e * a.nout + col0) * static_cast<long long>(elem);
-          if (bulk) {
-            fence_async_smem();
-            bulk_s2g(dst, srow, static_cast<unsigned>(cols * elem));
-          } else if (a.out_f16) {
-            const unsigned short* hs = reinterpret_cast<const unsigned short*>(srow);
-            for (int q = 0; q < cols; ++q) reinterpret_cast<unsigned short*>(dst)[q] = hs[q];
-          } else {
-            for (int q = 0; q < cols; ++q) reinterpret_cast<float*>(dst)[q] = srow[q];
+          fence_async_smem();
+          __syncthreads();  // the whole tile is staged
+          if (tid == 0) {
+            const int boxes = a.out_f16 ? kChunk / 64 : kChunk / 32;
+            const int bcols = a.out_f16 ? 64 : 32;
+            for (int q = 0; q < boxes; ++q)
+              if (col0 + q * bcols < a.nout)
+                tma_store_2d(&smap, stage + q * (kTile * 128), col0 + q * bcols,
+                             static_cast<int>(tile * kTile));
+            bulk_commit();
+          }
+        } else {
+#pragma unroll 1
+          for (int j0 = 0; j0 < kChunk; j0 += 32) {
+            float v[32];
+            tmem_ld32(tmem + static_cast<unsigned>(kOutCol + kChunk * pb + j0) + lane_off, v);
+            if (valid) {
+              const long long base = e * a.nout + col0 + j0;
+#pragma unroll
+              for (int q = 0; q < 32; ++q) {
+                if (j0 + q >= cols) continue;
+                if (a.out_f16)
+                  static_cast<__half*>(a.s)[base + q] = __float2half_rn(v[q] * f);
+                else
+                  static_cast<float*>(a.s)[base + q] = v[q] * f;
+              }
+            }
           }
         }
         tc_before();
@@ -409,15 +433,18 @@ int radial_prepare(RadialPlan& rp, int nb, double r_max, int hidden, int layers,
 size_t radial_smem_bytes(const RadialPlan& rp) {
   const size_t H = rp.hidden;
   return 2 * H * kMaxBasis * 2 + (rp.layers - 1) * 2 * H * H * 2 + 2 * kTile * kMaxBasis * 2 +
-         2 * kTile * H * 2 + kWBufs * 2 * kChunk * H * 2 +
-         static_cast<size_t>(kTile) * kStage * 4 + (kWBufs + 4) * 8 + 16;
+         2 * kTile * H * 2 + kWBufs * 2 * kChunk * H * 2 + kStageBytes + (kWBufs + 4) * 8 + 16;
 }
 
 int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, const void* dev_wo,
                   const float* vec, long long num_edges, void* s, int out_f16, unsigned* status,
-                  int grid, cudaStream_t st, std::string& err) {
+                  int grid, cudaStream_t st, std::string& err, const CUtensorMap* smap) {
   if (num_edges == 0) return E3CONV_OK;
   RadialArgs a;
+  CUtensorMap map;
+  std::memset(&map, 0, sizeof map);
+  a.tma = smap != nullptr;
+  if (smap) map = *smap;
   a.vec = vec;
   a.num_edges = num_edges;
   a.w0 = static_cast<const unsigned char*>(dev_w0);
@@ -449,7 +476,7 @@ int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, 
     // tensor memory: all 512 columns per CTA, so one CTA per SM
     per_sm = 1;
     const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, static_cast<long long>(grid) * per_sm));
-    kernel<<<blocks, 128, smem, st>>>(a);
+    kernel<<<blocks, 128, smem, st>>>(a, map);
     return cudaSuccess;
   };
   cudaError_t e = rp.hidden == 32 ? launch(k_radial<32>) : launch(k_radial<64>);

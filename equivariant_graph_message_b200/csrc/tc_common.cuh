@@ -57,6 +57,17 @@ __device__ __forceinline__ void bulk_s2g(void* dst, const void* src, unsigned by
                : "memory");
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
+// 2-D TMA tensor store of one box from shared memory at coordinates (x inner, y), in this
+// thread's bulk async-group (commit with bulk_commit)
+__device__ __forceinline__ void tma_store_2d(const void* map, const void* src, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+      "r"(smem_u32(src)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
 // this thread's bulk stores have finished reading their shared-memory source
 __device__ __forceinline__ void bulk_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
