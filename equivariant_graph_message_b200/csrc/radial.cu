@@ -13,8 +13,9 @@
 //   s      = h_L W_L                            (hidden -> P*C, tensor cores)
 // with SiLU(v) = v / (1 + exp(-v)), no biases.
 //
-// Tensor-core layers: one CTA of 128 threads per tile of 128 edges (thread t
-// <-> edge row t <-> tensor-memory lane t).  A = the tile's activations
+// Tensor-core layers: one CTA of 256 threads per tile of 128 edges: threads t
+// and t + 128 share edge row t (tensor-memory lane t) and each reads, applies
+// SiLU to, and stores half of the row's columns.  A = the tile's activations
 // [128 edges x hidden], B = the weights [N outputs x hidden] (both K-major,
 // float16, core matrices of 8 rows x 16 bytes, no swizzle), D = A B^T in
 // tensor memory (float32).  Both operands are split into float16 hi + lo
@@ -94,10 +95,12 @@ struct Smem {
 };
 
 template <int H>
-__global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a, const __grid_constant__ CUtensorMap smap) {
+__global__ void __launch_bounds__(256, 1) k_radial(RadialArgs a, const __grid_constant__ CUtensorMap smap) {
   extern __shared__ __align__(1024) unsigned char sm[];
   using L = Smem<H>;
+  constexpr int HH = H / 2;                       // hidden columns of one thread
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int row = tid & (kTile - 1), half = tid >> 7;  // edge row, which half of its columns
   unsigned char* w0s = sm;                                            // layer 0 (hi, lo)
   unsigned char* whs = w0s + 2 * L::kW0;                              // (layers-1) x (hi, lo)
   unsigned char* bas = whs + (a.layers - 1) * 2 * L::kWhid;           // basis values (hi, lo)
@@ -127,7 +130,8 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a, const __grid_co
   const unsigned tmem = *tslot;
   const unsigned t_hid = tmem;                 // columns [0, H): hidden-layer D
   // output-layer D: two buffers of kChunk columns at kOutCol and kOutCol + kChunk
-  const unsigned lane_off = static_cast<unsigned>(32 * warp) << 16;
+  // warps w and w + 4 both read tensor-memory lanes 32 (w % 4) .. + 31
+  const unsigned lane_off = static_cast<unsigned>(32 * (warp & 3)) << 16;
   bool ok = true;
   // phase bits (bit b: buffer b) of the weight-chunk and output-MMA barriers
   unsigned ph_w = 0, ph_mma = 0, ph_hid = 0;
@@ -148,7 +152,7 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a, const __grid_co
   const float norm = a.norm;
   const long long tiles = (a.num_edges + kTile - 1) / kTile;
   for (long long tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-    const long long e = tile * kTile + tid;
+    const long long e = tile * kTile + row;
     const bool valid = e < a.num_edges;
     // prefetch the first output-weight chunks of this tile (every buffer is free: the
     // previous tile waited for all of its output MMAs)
@@ -161,8 +165,8 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a, const __grid_co
       }
     }
     // layer 0: basis x cutoff on the CUDA cores, SiLU(h0 W0) with h0 W0 on the tensor cores
-    float h[H];
-    {
+    float h[HH];  // this thread's half of the row's hidden values: columns half * HH ..
+    if (half == 0) {
       float d = 0.f;
       if (valid) {
         const float4 v = __ldg(reinterpret_cast<const float4*>(a.vec) + e);
@@ -178,8 +182,10 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a, const __grid_co
                    ? 0.f
                    : (d > 0.f ? norm * sinpif((n + 1) * t) / d : norm * (n + 1) * pi_r) * u;
       }
-      store_split_row<kMaxBasis>(bas, bas + L::kBas, tid, b, kTile);
+      store_split_row<kMaxBasis>(bas, bas + L::kBas, row, b, kTile);
       fence_async_smem();
+    }
+    {
       tc_before();
       __syncthreads();
       tc_after();
@@ -196,12 +202,11 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a, const __grid_co
       if (!ok) break;
       ph_hid ^= 1u;
       pend_hid = false;
-#pragma unroll
-      for (int j0 = 0; j0 < H; j0 += 32) {
+      {
         float v[32];
-        tmem_ld32(t_hid + lane_off + j0, v);
+        tmem_ld32(t_hid + lane_off + half * HH, v);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) h[j0 + q] = silu(v[q] * a.w_scale_inv_0);
+        for (int q = 0; q < HH; ++q) h[q] = silu(v[q] * a.w_scale_inv_0);
       }
       tc_before();
       __syncthreads();  // every thread has read D before the next layer's MMAs overwrite it
@@ -209,22 +214,23 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a, const __grid_co
     }
     // hidden layers 1 .. L-1 on the tensor cores
     for (int l = 1; l < a.layers && ok; ++l) {
-      store_split_row<H>(act, act + L::kAct, tid, h, kTile);
+      store_split_part<HH>(act, act + L::kAct, row, h, kTile, half * HH);
       fence_async_smem();
       tc_before();
       __syncthreads();
       tc_after();
       if (tid == 0) {
         const unsigned char* whi = whs + (l - 1) * 2 * L::kWhid;
-        const unsigned char* wlo = whi + L::kWhid;
         const unsigned id = idesc_f16(kTile, H);
-        unsigned acc = 0;
+        const unsigned long long d_ahi = kmajor_desc(act), d_alo = kmajor_desc(act + L::kAct);
+        const unsigned long long d_whi = kmajor_desc(whi), d_wlo = kmajor_desc(whi + L::kWhid);
+#pragma unroll
         for (int ks = 0; ks < H / 16; ++ks) {
-          const int ao = ks * kTile * 32, bo = ks * H * 32;
-          mma_f16(t_hid, kmajor_desc(act + ao), kmajor_desc(whi + bo), id, acc);
-          acc = 1;
-          mma_f16(t_hid, kmajor_desc(act + ao), kmajor_desc(wlo + bo), id, 1);
-          mma_f16(t_hid, kmajor_desc(act + L::kAct + ao), kmajor_desc(whi + bo), id, 1);
+          const unsigned long long ao = static_cast<unsigned long long>(ks * kTile * 32) >> 4;
+          const unsigned long long bo = static_cast<unsigned long long>(ks * H * 32) >> 4;
+          mma_f16(t_hid, d_ahi + ao, d_whi + bo, id, ks > 0);
+          mma_f16(t_hid, d_ahi + ao, d_wlo + bo, id, 1);
+          mma_f16(t_hid, d_alo + ao, d_whi + bo, id, 1);
         }
         mma_commit(bar_hid);
         pend_hid = true;
@@ -234,12 +240,11 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a, const __grid_co
       if (!ok) break;
       ph_hid ^= 1u;
       pend_hid = false;
-#pragma unroll
-      for (int j0 = 0; j0 < H; j0 += 32) {
+      {
         float v[32];
-        tmem_ld32(t_hid + lane_off + j0, v);
+        tmem_ld32(t_hid + lane_off + half * HH, v);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) h[j0 + q] = silu(v[q] * a.w_scale_inv_h);
+        for (int q = 0; q < HH; ++q) h[q] = silu(v[q] * a.w_scale_inv_h);
       }
       tc_before();
       __syncthreads();  // every thread has read D before the next layer's MMAs overwrite it
@@ -247,7 +252,7 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a, const __grid_co
     }
     if (!ok) break;
     // output layer: chunks of 128 columns
-    store_split_row<H>(act, act + L::kAct, tid, h, kTile);
+    store_split_part<HH>(act, act + L::kAct, row, h, kTile, half * HH);
     fence_async_smem();
     tc_before();
     __syncthreads();
@@ -303,25 +308,25 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a, const __grid_co
           // staging tile: per 128-byte column box (32 floats or 64 halves), row r at r * 128,
           // its 16-byte piece q at (q ^ (r & 7)) * 16
 #pragma unroll 1
-          for (int j0 = 0; j0 < kChunk; j0 += 32) {
+          for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
             float v[32];
             tmem_ld32(tmem + static_cast<unsigned>(kOutCol + kChunk * pb + j0) + lane_off, v);
             if (a.out_f16) {
-              unsigned char* box = stage + (j0 / 64) * (kTile * 128) + tid * 128;
+              unsigned char* box = stage + (j0 / 64) * (kTile * 128) + row * 128;
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const int piece = (j0 % 64) / 8 + q;
-                *reinterpret_cast<uint4*>(box + ((piece ^ (tid & 7)) * 16)) =
+                *reinterpret_cast<uint4*>(box + ((piece ^ (row & 7)) * 16)) =
                     make_uint4(pack_half2(v[8 * q] * f, v[8 * q + 1] * f),
                                pack_half2(v[8 * q + 2] * f, v[8 * q + 3] * f),
                                pack_half2(v[8 * q + 4] * f, v[8 * q + 5] * f),
                                pack_half2(v[8 * q + 6] * f, v[8 * q + 7] * f));
               }
             } else {
-              unsigned char* box = stage + (j0 / 32) * (kTile * 128) + tid * 128;
+              unsigned char* box = stage + (j0 / 32) * (kTile * 128) + row * 128;
 #pragma unroll
               for (int q = 0; q < 8; ++q)
-                *reinterpret_cast<float4*>(box + ((q ^ (tid & 7)) * 16)) =
+                *reinterpret_cast<float4*>(box + ((q ^ (row & 7)) * 16)) =
                     make_float4(v[4 * q] * f, v[4 * q + 1] * f, v[4 * q + 2] * f, v[4 * q + 3] * f);
             }
           }
@@ -338,7 +343,7 @@ __global__ void __launch_bounds__(128, 1) k_radial(RadialArgs a, const __grid_co
           }
         } else {
 #pragma unroll 1
-          for (int j0 = 0; j0 < kChunk; j0 += 32) {
+          for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
             float v[32];
             tmem_ld32(tmem + static_cast<unsigned>(kOutCol + kChunk * pb + j0) + lane_off, v);
             if (valid) {
@@ -471,12 +476,12 @@ int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, 
                                          static_cast<int>(smem));
     int per_sm = 0;
     if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 128, smem);
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, smem);
     if (e != cudaSuccess || per_sm < 1) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
     // tensor memory: all 512 columns per CTA, so one CTA per SM
     per_sm = 1;
     const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, static_cast<long long>(grid) * per_sm));
-    kernel<<<blocks, 128, smem, st>>>(a, map);
+    kernel<<<blocks, 256, smem, st>>>(a, map);
     return cudaSuccess;
   };
   cudaError_t e = rp.hidden == 32 ? launch(k_radial<32>) : launch(k_radial<64>);

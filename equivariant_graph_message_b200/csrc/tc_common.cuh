@@ -159,6 +159,22 @@ __device__ __forceinline__ void store_split_row(unsigned char* hi, unsigned char
 }
 
 
+// Writes values v[0..N) of row r at K columns k0 .. k0 + N - 1 (k0 a multiple of 16) of a
+// K-major operand as float16 hi and lo parts.
+template <int N>
+__device__ __forceinline__ void store_split_part(unsigned char* hi, unsigned char* lo, int r,
+                                                 const float* v, int rows, int k0) {
+#pragma unroll
+  for (int k = 0; k < N; k += 2) {
+    const __half h0 = __float2half_rn(v[k]), h1 = __float2half_rn(v[k + 1]);
+    const __half l0 = __float2half_rn(v[k] - __half2float(h0));
+    const __half l1 = __float2half_rn(v[k + 1] - __half2float(h1));
+    const int off = kmajor_off(r, k0 + k, rows);
+    *reinterpret_cast<__half2*>(hi + off) = __halves2half2(h0, h1);
+    *reinterpret_cast<__half2*>(lo + off) = __halves2half2(l0, l1);
+  }
+}
+
 }  // namespace tc
 
 namespace tc_host {
