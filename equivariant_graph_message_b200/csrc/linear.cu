@@ -44,6 +44,7 @@ struct LinArgs {
   int dim_in, dim_out, n_out;  // row lengths; mul_out (MMA N)
   int nblocks;                 // output irrep blocks
   int tiles_total;
+  unsigned tmem_cols;          // tensor-memory columns of a CTA: the power of two >= mul_out
   unsigned* status;
   LinBlock blk[kLinMaxBlocks];
 };
@@ -65,8 +66,8 @@ __global__ void __launch_bounds__(128, 1) k_linear(LinArgs a) {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
-                     smem_u32(tslot))
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tslot)), "r"(a.tmem_cols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -199,7 +200,8 @@ __global__ void __launch_bounds__(128, 1) k_linear(LinArgs a) {
   __syncthreads();
   tc_after();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(a.tmem_cols)
+                 : "memory");
 }
 
 }  // namespace
@@ -327,22 +329,25 @@ int linear_launch(const LinearPlan& lp, const void* dev_w, const float* x, long 
   }
   a.tiles_total = static_cast<int>(tiles);
   const size_t smem = linear_smem_bytes(lp);
-  const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, grid));
-  cudaError_t e = cudaSuccess;
-  switch (lp.K) {
-    case 32:
-      e = cudaFuncSetAttribute(k_linear<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e == cudaSuccess) k_linear<32><<<blocks, 128, smem, st>>>(a);
-      break;
-    case 64:
-      e = cudaFuncSetAttribute(k_linear<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e == cudaSuccess) k_linear<64><<<blocks, 128, smem, st>>>(a);
-      break;
-    default:
-      e = cudaFuncSetAttribute(k_linear<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e == cudaSuccess) k_linear<128><<<blocks, 128, smem, st>>>(a);
-      break;
-  }
+  a.tmem_cols = 32;
+  while (a.tmem_cols < static_cast<unsigned>(lp.N)) a.tmem_cols *= 2;
+  // CTAs per SM: shared memory (occupancy calculator, carveout at its maximum) and tensor
+  // memory (512 columns per SM)
+  auto launch = [&](auto kernel) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    int per_sm = 0;
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 128, smem);
+    if (e != cudaSuccess) return e;
+    per_sm = std::max(1, std::min(per_sm, static_cast<int>(512 / a.tmem_cols)));
+    const unsigned blocks =
+        static_cast<unsigned>(std::min<long long>(tiles, static_cast<long long>(grid) * per_sm));
+    kernel<<<blocks, 128, smem, st>>>(a);
+    return cudaSuccess;
+  };
+  cudaError_t e = lp.K == 32 ? launch(k_linear<32>) : lp.K == 64 ? launch(k_linear<64>) : launch(k_linear<128>);
   if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) {
     err = "irreps linear kernel launch failed";
     return E3CONV_ERR_CUDA;
