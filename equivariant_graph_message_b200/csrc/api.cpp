@@ -214,16 +214,20 @@ int prepare_backward(Plan& pl) {
   v.shape = choose_backward_shape(pl, pl.dtype);
   if (!v.shape.ok)
     return fail(E3CONV_ERR_UNSUPPORTED, "backward needs C <= 128 (float32) or <= 256 (float16)");
-  const char* names[2] = {"e3conv_bwd_edges", "e3conv_bwd_nodes"};
-  for (int k = 0; k < 2; ++k) {
-    v.source[k] = generate_backward_source(pl, pl.dtype, v.shape, k == 1);
-    const int rc = nvrtc_compile(v.source[k], k ? "e3conv_bwd_nodes.cu" : "e3conv_bwd_edges.cu",
-                                 v.cubin[k], v.log[k], v.regs[k], v.local_bytes[k]);
+  // modules: 0 edges (part 0), 1 nodes, 2 edges part 1 when the edges kernel is split
+  const int nmod = v.shape.eparts > 1 ? 3 : 2;
+  const char* names[3] = {"e3conv_bwd_edges", "e3conv_bwd_nodes", "e3conv_bwd_edges"};
+  const char* files[3] = {"e3conv_bwd_edges.cu", "e3conv_bwd_nodes.cu", "e3conv_bwd_edges_1.cu"};
+  for (int k = 0; k < nmod; ++k) {
+    v.source[k] = k == 2 ? generate_backward_edges_part(pl, pl.dtype, v.shape, 1)
+                         : generate_backward_source(pl, pl.dtype, v.shape, k == 1);
+    const int rc = nvrtc_compile(v.source[k], files[k], v.cubin[k], v.log[k], v.regs[k],
+                                 v.local_bytes[k]);
     if (rc != E3CONV_OK) return rc;
   }
   if (pl.device >= 0) {
     Driver& d = driver();
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < nmod; ++k) {
       if (d.ModuleLoadData(&v.module[k], v.cubin[k].data()) != CUDA_SUCCESS ||
           d.ModuleGetFunction(&v.fn[k], v.module[k], names[k]) != CUDA_SUCCESS) {
         for (int q = 0; q <= k; ++q)
@@ -231,14 +235,17 @@ int prepare_backward(Plan& pl) {
         return fail(E3CONV_ERR_CUDA, "loading the backward kernels failed");
       }
     }
-    if ((v.shape.staged &&
-         d.FuncSetAttribute(v.fn[0], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES, v.shape.smem) !=
-             CUDA_SUCCESS) ||
-        (v.shape.nstaged &&
-         d.FuncSetAttribute(v.fn[1], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES, v.shape.nsmem) !=
-             CUDA_SUCCESS)) {
-      for (int q = 0; q < 2; ++q) d.ModuleUnload(v.module[q]);
-      return fail(E3CONV_ERR_CUDA, "cannot reserve the backward edges kernel's shared memory");
+    bool ok = true;
+    if (v.shape.staged)
+      for (int p = 0; p < v.shape.eparts; ++p)
+        ok = ok && d.FuncSetAttribute(v.fn[p == 0 ? 0 : 2], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES,
+                                      v.shape.esmem[p]) == CUDA_SUCCESS;
+    if (v.shape.nstaged)
+      ok = ok && d.FuncSetAttribute(v.fn[1], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES,
+                                    v.shape.nsmem) == CUDA_SUCCESS;
+    if (!ok) {
+      for (int q = 0; q < nmod; ++q) d.ModuleUnload(v.module[q]);
+      return fail(E3CONV_ERR_CUDA, "cannot reserve the backward kernels' shared memory");
     }
   }
   v.compiled = true;
@@ -247,7 +254,7 @@ int prepare_backward(Plan& pl) {
 }
 
 void release_backward(BwdVariant& v) {
-  for (int k = 0; k < 2; ++k)
+  for (int k = 0; k < 3; ++k)
     if (v.module[k]) driver().ModuleUnload(v.module[k]);
   v = BwdVariant{};
 }
@@ -1105,10 +1112,11 @@ int e3conv_backward(e3conv_plan h, const void* x, const void* Y, const void* s,
     void* args[] = {const_cast<void**>(&x), const_cast<void**>(&Y), const_cast<void**>(&s),
                     const_cast<int32_t**>(&senders), const_cast<int32_t**>(&row_ptr), &n32,
                     const_cast<float**>(&grad_out), &grad_sh, &grad_scalars, &inv_avg, &pl.status};
-    if (driver().LaunchKernel(bv.fn[0], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1,
-                              b.staged ? static_cast<unsigned>(b.smem) : 0u, st, args,
-                              nullptr) != CUDA_SUCCESS)
-      return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed (backward, edges)");
+    for (int p = 0; p < b.eparts; ++p)
+      if (driver().LaunchKernel(bv.fn[p == 0 ? 0 : 2], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1,
+                                b.staged ? static_cast<unsigned>(b.esmem[p]) : 0u, st, args,
+                                nullptr) != CUDA_SUCCESS)
+        return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed (backward, edges)");
   }
   if (grad_x) {
     void* args[] = {const_cast<void**>(&Y), const_cast<void**>(&s),
@@ -1124,10 +1132,12 @@ int e3conv_backward(e3conv_plan h, const void* x, const void* Y, const void* s,
 }
 
 int e3conv_backward_source(e3conv_plan h, int which, char* buf, size_t buf_len, size_t* needed) {
-  if (!h || which < 0 || which > 1) return fail(E3CONV_ERR_INVALID_ARG, "bad argument");
+  if (!h || which < 0 || which > 2) return fail(E3CONV_ERR_INVALID_ARG, "bad argument");
   DeviceGuard g(h->p.device);
   int rc = prepare_backward(h->p);
   if (rc != E3CONV_OK) return rc;
+  if (which == 2 && h->p.bwd[h->p.dtype].shape.eparts < 2)
+    return fail(E3CONV_ERR_INVALID_ARG, "the edges kernel of this plan is not split");
   const std::string& src = h->p.bwd[h->p.dtype].source[which];
   if (needed) *needed = src.size() + 1;
   if (buf && buf_len >= src.size() + 1) std::memcpy(buf, src.c_str(), src.size() + 1);

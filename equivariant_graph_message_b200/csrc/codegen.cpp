@@ -32,7 +32,9 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <functional>
 #include <map>
+#include <set>
 #include <sstream>
 
 #include "plan.h"
@@ -1928,6 +1930,40 @@ BwdShape choose_backward_shape(const Plan& pl, int dtype) {
   b.smem = (b.block / 32) * 2 * b.stage_bytes;
   b.staged = TL == 32 && V % 2 == 0 && b.s_bytes % 16 == 0 && b.x_bytes % 16 == 0 &&
              (pl.ny * elem) % 4 == 0 && b.smem <= 112 * 1024;
+  // a grad_out row of more than 64 registers per lane: the edges kernel runs as two launches,
+  // each over half of the output irreps (balanced by their (i, k) terms), so each holds half
+  // of the row and stages only its paths' scalars
+  b.eparts = 1;
+  b.out_part.assign(pl.outputs.size(), 0);
+  b.esmem[0] = b.esmem[1] = b.smem;
+  if (b.staged && pl.nout * V > 64 && pl.outputs.size() > 1 && (pl.C * elem) % 16 == 0) {
+    std::vector<std::pair<long long, int>> work;  // (terms, output irrep)
+    for (size_t o = 0; o < pl.outputs.size(); ++o) {
+      long long w = 0;
+      for (const auto& P : pl.paths)
+        if (P.o == static_cast<int>(o)) {
+          std::set<std::pair<int, int>> ik;
+          for (const auto& n : P.nnz) ik.insert({n.i, n.k});
+          w += static_cast<long long>(ik.size());
+        }
+      work.push_back({w, static_cast<int>(o)});
+    }
+    std::sort(work.begin(), work.end(), std::greater<std::pair<long long, int>>());
+    long long load[2] = {0, 0};
+    for (const auto& wo : work) {
+      const int t = load[0] <= load[1] ? 0 : 1;
+      b.out_part[wo.second] = t;
+      load[t] += wo.first;
+    }
+    if (load[0] > 0 && load[1] > 0) {
+      b.eparts = 2;
+      for (int t = 0; t < 2; ++t) {
+        int np = 0;
+        for (const auto& P : pl.paths) np += b.out_part[P.o] == t;
+        b.esmem[t] = (b.block / 32) * 2 * (np * pl.C * elem + b.x_bytes + b.y_bytes);
+      }
+    }
+  }
   b.g_bytes = pl.nout * pl.C * 4;
   b.nstage_bytes = b.s_bytes + b.g_bytes + b.y_bytes;
   b.nsmem = (b.block / 32) * 2 * b.nstage_bytes;
@@ -2116,8 +2152,19 @@ std::string bwd_edges_source(const Plan& pl, int dtype, const BwdShape& b) {
 //   gs[e, p, c] = (1/N) sum_k g_k t_k
 //   W_ik = sum_{lane's channels} (s x_i) g_k,   dY_j += sum_{(i,k)} c_ijk W_ik
 // then dY is summed over the warp's lanes and lane 0 stores it.
-std::string bwd_edges_staged_source(const Plan& pl, int dtype, const BwdShape& b) {
+std::string bwd_edges_staged_source(const Plan& pl, int dtype, const BwdShape& b, int part) {
   Emitter em;
+  // this launch's output irreps and paths: the part's outputs, or all of them
+  std::vector<bool> own_out(pl.outputs.size(), true), own_path(pl.paths.size(), true);
+  if (b.eparts > 1)
+    for (size_t o = 0; o < pl.outputs.size(); ++o) own_out[o] = b.out_part[o] == part;
+  std::vector<int> slot(pl.paths.size(), -1);  // the path's s segment in the ring
+  int nslots = 0;
+  for (size_t r = 0; r < pl.paths.size(); ++r) {
+    own_path[r] = own_out[pl.paths[r].o];
+    if (own_path[r]) slot[r] = nslots++;
+  }
+  const bool accumulate = b.eparts > 1 && part > 0;  // adds to the grad_Y an earlier part stored
   const std::string T = bwd_prelude(em, pl, dtype, b);
   emit_pair_ops(em);
   em.line("__device__ __forceinline__ void upk(unsigned long long w, float& lo, float& hi) { asm(\"mov.b64 {%0, %1}, %2;\" : \"=f\"(lo), \"=f\"(hi) : \"l\"(w)); }");
@@ -2129,8 +2176,14 @@ std::string bwd_edges_staged_source(const Plan& pl, int dtype, const BwdShape& b
   const bool f16 = dtype == E3CONV_F16;
   const int V = b.V, NG = V / 2, elem = f16 ? 2 : 4;
   const long long s_row = static_cast<long long>(pl.paths.size()) * pl.C;
-  const int SB = b.stage_bytes;
-  em.line("extern \"C\" __global__ void __launch_bounds__(" + S(b.block) + ") e3conv_bwd_edges(");
+  const int s_bytes = nslots * pl.C * elem;             // the part's scalars in the ring
+  const int SB = s_bytes + b.x_bytes + b.y_bytes;
+  em.line("// part " + S(part) + " of " + S(b.eparts) + ": " + S(nslots) + " of " + S(pl.paths.size()) +
+          " paths" + (accumulate ? ", grad_Y added to the earlier part's" : ""));
+  // a split launch holds less: as many blocks per SM as shared memory allows (at most three)
+  const int minb = b.eparts > 1 ? std::max(1, std::min(3, (220 * 1024) / std::max(1, b.esmem[part]))) : 1;
+  em.line("extern \"C\" __global__ void __launch_bounds__(" + S(b.block) +
+          (minb > 1 ? ", " + S(minb) : std::string()) + ") e3conv_bwd_edges(");
   em.line("    const " + T + "* __restrict__ x, const " + T + "* __restrict__ Y, const " + T +
           "* __restrict__ s,");
   em.line("    const int* __restrict__ senders, const int* __restrict__ row_ptr, int num_nodes,");
@@ -2148,8 +2201,13 @@ std::string bwd_edges_staged_source(const Plan& pl, int dtype, const BwdShape& b
   em.line("int e0 = row_ptr[bb], e1 = row_ptr[bb + 1];");
   em.line("if (e0 < e_base || e1 < e0 || e1 > e_end) { if (lane == 0) atomicOr(status, 1u); e1 = e0; }");
   em.line("if (e0 == e1) return;");
-  // g row as pairs
+  // g row as pairs (the part's output components)
+  std::vector<bool> own_k(pl.nout, false);
+  for (size_t o = 0; o < pl.outputs.size(); ++o)
+    if (own_out[o])
+      for (int k = 0; k < 2 * pl.outputs[o].l + 1; ++k) own_k[pl.outputs[o].off + k] = true;
   for (int k = 0; k < pl.nout; ++k) {
+    if (!own_k[k]) continue;
     const std::string src = "g + bb * " + S(static_cast<long long>(pl.nout) * pl.C) + " + " +
                             S(static_cast<long long>(k) * pl.C) + " + u0";
     if (NG == 2) {
@@ -2170,22 +2228,31 @@ std::string bwd_edges_staged_source(const Plan& pl, int dtype, const BwdShape& b
   em.line("if (!valid && lane == 0) atomicOr(status, 2u);");
   em.line("unsigned char* dst = ring + st * " + S(SB) + ";");
   em.line("const unsigned char* ssrc = reinterpret_cast<const unsigned char*>(s + le * " + S(s_row) + ");");
-  em.line("#pragma unroll");
-  em.line("for (int q = lane; q < " + S(b.s_bytes / 16) + "; q += 32) cp16(dst + 16 * q, ssrc + 16 * q);");
+  if (nslots == static_cast<int>(pl.paths.size())) {
+    em.line("#pragma unroll");
+    em.line("for (int q = lane; q < " + S(s_bytes / 16) + "; q += 32) cp16(dst + 16 * q, ssrc + 16 * q);");
+  } else {
+    // the part's paths: one contiguous C-channel segment each
+    const int seg = pl.C * elem / 16;
+    for (size_t r = 0; r < pl.paths.size(); ++r)
+      if (own_path[r])
+        em.line("for (int q = lane; q < " + S(seg) + "; q += 32) cp16(dst + " + S(slot[r] * pl.C * elem) +
+                " + 16 * q, ssrc + " + S(static_cast<long long>(r) * pl.C * elem) + " + 16 * q);");
+  }
   em.line("if (valid) {");
   em.line("  const unsigned char* xsrc = reinterpret_cast<const unsigned char*>(x + (long long)a * " +
           S(static_cast<long long>(pl.nx) * pl.C) + ");");
   em.line("  #pragma unroll");
-  em.line("  for (int q = lane; q < " + S(b.x_bytes / 16) + "; q += 32) cp16(dst + " + S(b.s_bytes) +
+  em.line("  for (int q = lane; q < " + S(b.x_bytes / 16) + "; q += 32) cp16(dst + " + S(s_bytes) +
           " + 16 * q, xsrc + 16 * q);");
   em.line("} else {");
   em.line("  #pragma unroll");
   em.line("  for (int q = lane; q < " + S(b.x_bytes / 16) + "; q += 32) *reinterpret_cast<uint4*>(dst + " +
-          S(b.s_bytes) + " + 16 * q) = make_uint4(0u, 0u, 0u, 0u);");
+          S(s_bytes) + " + 16 * q) = make_uint4(0u, 0u, 0u, 0u);");
   em.line("}");
   em.line("const unsigned char* ysrc = reinterpret_cast<const unsigned char*>(Y + le * " + S(pl.ny) + ");");
   em.line("for (int q = lane; q < " + S(pl.ny * elem / 4) + "; q += 32) cp4(dst + " +
-          S(b.s_bytes + b.x_bytes) + " + 4 * q, ysrc + 4 * q);");
+          S(s_bytes + b.x_bytes) + " + 4 * q, ysrc + 4 * q);");
   em.line("cp_commit();");
   em.ind--;
   em.line("};");
@@ -2200,9 +2267,9 @@ std::string bwd_edges_staged_source(const Plan& pl, int dtype, const BwdShape& b
   em.line("__syncwarp();");
   em.line("const long long le = e - e_base;");
   em.line("const unsigned char* cur = ring + st * " + S(SB) + ";");
-  em.line("const " + T + "* ys = reinterpret_cast<const " + T + "*>(cur + " + S(b.s_bytes + b.x_bytes) + ");");
+  em.line("const " + T + "* ys = reinterpret_cast<const " + T + "*>(cur + " + S(s_bytes + b.x_bytes) + ");");
   emit_y_load(em, pl, dtype, "lds", "ys");
-  em.line("const " + T + "* xs = reinterpret_cast<const " + T + "*>(cur + " + S(b.s_bytes) + ") + u0;");
+  em.line("const " + T + "* xs = reinterpret_cast<const " + T + "*>(cur + " + S(s_bytes) + ") + u0;");
   em.line("const " + T + "* ss = reinterpret_cast<const " + T + "*>(cur) + u0;");
   em.line("float* gsr = gs + le * " + S(s_row) + " + u0;");
   {
@@ -2243,11 +2310,12 @@ std::string bwd_edges_staged_source(const Plan& pl, int dtype, const BwdShape& b
     em.line("{  // node irrep " + S(n1) + " (l=" + S(first.l1) + ")");
     em.ind++;
     for (size_t r = p; r < q; ++r) {
+      if (!own_path[r]) continue;
       const Path& P = pl.paths[r];
       const int d3 = 2 * P.l3 + 1;
       em.line("{  // path " + S(r) + ": " + S(P.l1) + " x " + S(P.l2) + " -> " + S(P.l3));
       em.ind++;
-      load_pairs("ss + " + S(static_cast<long long>(r) * pl.C), "s");
+      load_pairs("ss + " + S(static_cast<long long>(slot[r]) * pl.C), "s");
       // distinct (i, k) of the path with their (j, c) terms
       std::map<std::pair<int, int>, std::vector<std::pair<int, double>>> ik;
       for (const auto& n : P.nnz) ik[{n.i, n.k}].push_back({n.j, n.c});
@@ -2349,7 +2417,9 @@ std::string bwd_edges_staged_source(const Plan& pl, int dtype, const BwdShape& b
   em.line("if (lane == 0) {");
   em.ind++;
   for (int j = 0; j < pl.ny; ++j)
-    em.line("gY[le * " + S(pl.ny) + " + " + S(j) + "] = inv_avg * dy" + S(j) + ";");
+    em.line("gY[le * " + S(pl.ny) + " + " + S(j) + "] = " +
+            (accumulate ? "gY[le * " + S(pl.ny) + " + " + S(j) + "] + " : std::string()) + "inv_avg * dy" +
+            S(j) + ";");
   em.ind--;
   em.line("}");
   em.line("__syncwarp();  // every lane has read this stage before the next edge's copies reuse it");
@@ -2645,7 +2715,11 @@ std::string bwd_nodes_source(const Plan& pl, int dtype, const BwdShape& b) {
 
 std::string generate_backward_source(const Plan& pl, int dtype, const BwdShape& b, bool nodes) {
   if (nodes) return b.nstaged ? bwd_nodes_staged_source(pl, dtype, b) : bwd_nodes_source(pl, dtype, b);
-  return b.staged ? bwd_edges_staged_source(pl, dtype, b) : bwd_edges_source(pl, dtype, b);
+  return b.staged ? bwd_edges_staged_source(pl, dtype, b, 0) : bwd_edges_source(pl, dtype, b);
+}
+
+std::string generate_backward_edges_part(const Plan& pl, int dtype, const BwdShape& b, int part) {
+  return bwd_edges_staged_source(pl, dtype, b, part);
 }
 
 // Standalone harmonics: one thread per edge evaluates the plan's polynomials of

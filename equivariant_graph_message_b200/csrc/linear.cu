@@ -336,12 +336,22 @@ int linear_launch(const LinearPlan& lp, const void* dev_w, const float* x, long 
   auto launch = [&](auto kernel) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    int per_sm = 0;
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 128, smem);
+    cudaFuncAttributes fa;
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, kernel);
     if (e != cudaSuccess) return e;
-    per_sm = std::max(1, std::min(per_sm, static_cast<int>(512 / a.tmem_cols)));
+    // by hand: 228 KB of shared memory per SM (1 KB reserved per block), 64K registers
+    // (allocated per warp in units of 256), 512 tensor-memory columns
+    const int regs_warp = (fa.numRegs * 32 + 255) / 256 * 256;
+    const int by_smem = static_cast<int>((228 * 1024) / (smem + 1024));
+    const int by_regs = 65536 / (regs_warp * 4);
+    int per_sm = std::min({by_smem, by_regs, static_cast<int>(512 / a.tmem_cols), 8});
+    per_sm = std::max(per_sm, 1);
+    // several CTAs need the shared-memory carveout that holds them (the rest stays L1)
+    if (per_sm > 1) {
+      const int pct = static_cast<int>((per_sm * (smem + 1024) * 100 + 228 * 1024 - 1) / (228 * 1024));
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, std::min(pct, 100));
+      if (e != cudaSuccess) return e;
+    }
     const unsigned blocks =
         static_cast<unsigned>(std::min<long long>(tiles, static_cast<long long>(grid) * per_sm));
     kernel<<<blocks, 128, smem, st>>>(a);

@@ -105,17 +105,22 @@ struct BwdShape {
   // nodes kernel (grad_x, sender order) with the same kind of ring: s, g (float32) and Y rows
   bool nstaged = false;
   int g_bytes = 0, nstage_bytes = 0, nsmem = 0;
+  // edges kernel split over output irreps: eparts launches, out_part[o] = the launch of
+  // output irrep o, esmem[p] = its dynamic shared memory per block
+  int eparts = 1;
+  std::vector<int> out_part;
+  int esmem[2] = {0, 0};
 };
 
 struct BwdVariant {
   bool compiled = false;
   BwdShape shape;
-  std::string source[2];     // edges, nodes
-  std::vector<char> cubin[2];
-  std::string log[2];
-  CUmodule module[2] = {nullptr, nullptr};
-  CUfunction fn[2] = {nullptr, nullptr};
-  int regs[2] = {-1, -1}, local_bytes[2] = {-1, -1};
+  std::string source[3];     // edges (part 0), nodes, edges part 1 (when the edges kernel is split)
+  std::vector<char> cubin[3];
+  std::string log[3];
+  CUmodule module[3] = {nullptr, nullptr, nullptr};
+  CUfunction fn[3] = {nullptr, nullptr, nullptr};
+  int regs[3] = {-1, -1, -1}, local_bytes[3] = {-1, -1, -1};
 };
 
 struct ShVariant {  // standalone harmonics kernel (compiled on first use)
@@ -242,6 +247,7 @@ std::string generate_forward_source(const Plan& plan, int dtype, const Shape& sh
 BwdShape choose_backward_shape(const Plan& plan, int dtype);
 std::string generate_backward_source(const Plan& plan, int dtype, const BwdShape& shape, bool nodes);
 std::string generate_sh_source(const Plan& plan, int dtype);
+std::string generate_backward_edges_part(const Plan& plan, int dtype, const BwdShape& shape, int part);
 
 }  // namespace e3c
 
