@@ -214,13 +214,17 @@ int prepare_backward(Plan& pl) {
   v.shape = choose_backward_shape(pl, pl.dtype);
   if (!v.shape.ok)
     return fail(E3CONV_ERR_UNSUPPORTED, "backward needs C <= 128 (float32) or <= 256 (float16)");
-  // modules: 0 edges (part 0), 1 nodes, 2 edges part 1 when the edges kernel is split
-  const int nmod = v.shape.eparts > 1 ? 3 : 2;
-  const char* names[3] = {"e3conv_bwd_edges", "e3conv_bwd_nodes", "e3conv_bwd_edges"};
-  const char* files[3] = {"e3conv_bwd_edges.cu", "e3conv_bwd_nodes.cu", "e3conv_bwd_edges_1.cu"};
+  // modules: 0 edges (part 0), 1 nodes (part 0), 2 edges part 1 and 3 nodes part 1 where the
+  // kernels are split over the output irreps (the nodes kernel only when it is staged)
+  const bool esplit = v.shape.eparts > 1, nsplit = esplit && v.shape.nstaged;
+  const int nmod = nsplit ? 4 : esplit ? 3 : 2;
+  const char* names[4] = {"e3conv_bwd_edges", "e3conv_bwd_nodes", "e3conv_bwd_edges", "e3conv_bwd_nodes"};
+  const char* files[4] = {"e3conv_bwd_edges.cu", "e3conv_bwd_nodes.cu", "e3conv_bwd_edges_1.cu",
+                          "e3conv_bwd_nodes_1.cu"};
   for (int k = 0; k < nmod; ++k) {
-    v.source[k] = k == 2 ? generate_backward_edges_part(pl, pl.dtype, v.shape, 1)
-                         : generate_backward_source(pl, pl.dtype, v.shape, k == 1);
+    v.source[k] = k == 2   ? generate_backward_edges_part(pl, pl.dtype, v.shape, 1)
+                  : k == 3 ? generate_backward_nodes_part(pl, pl.dtype, v.shape, 1)
+                           : generate_backward_source(pl, pl.dtype, v.shape, k == 1);
     const int rc = nvrtc_compile(v.source[k], files[k], v.cubin[k], v.log[k], v.regs[k],
                                  v.local_bytes[k]);
     if (rc != E3CONV_OK) return rc;
@@ -241,8 +245,9 @@ int prepare_backward(Plan& pl) {
         ok = ok && d.FuncSetAttribute(v.fn[p == 0 ? 0 : 2], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES,
                                       v.shape.esmem[p]) == CUDA_SUCCESS;
     if (v.shape.nstaged)
-      ok = ok && d.FuncSetAttribute(v.fn[1], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES,
-                                    v.shape.nsmem) == CUDA_SUCCESS;
+      for (int p = 0; p < (nsplit ? 2 : 1); ++p)
+        ok = ok && d.FuncSetAttribute(v.fn[p == 0 ? 1 : 3], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES,
+                                      nsplit ? v.shape.nsmem_p[p] : v.shape.nsmem) == CUDA_SUCCESS;
     if (!ok) {
       for (int q = 0; q < nmod; ++q) d.ModuleUnload(v.module[q]);
       return fail(E3CONV_ERR_CUDA, "cannot reserve the backward kernels' shared memory");
@@ -254,7 +259,7 @@ int prepare_backward(Plan& pl) {
 }
 
 void release_backward(BwdVariant& v) {
-  for (int k = 0; k < 3; ++k)
+  for (int k = 0; k < 4; ++k)
     if (v.module[k]) driver().ModuleUnload(v.module[k]);
   v = BwdVariant{};
 }
@@ -1123,21 +1128,23 @@ int e3conv_backward(e3conv_plan h, const void* x, const void* Y, const void* s,
                     const_cast<int32_t**>(&receivers), const_cast<int32_t**>(&row_ptr),
                     const_cast<int32_t**>(&sender_row_ptr), const_cast<int32_t**>(&sender_perm),
                     &n32, const_cast<float**>(&grad_out), &grad_x, &inv_avg, &pl.status};
-    if (driver().LaunchKernel(bv.fn[1], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1,
-                              b.nstaged ? static_cast<unsigned>(b.nsmem) : 0u, st, args,
-                              nullptr) != CUDA_SUCCESS)
-      return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed (backward, nodes)");
+    const bool nsplit = b.eparts > 1 && b.nstaged;
+    for (int p = 0; p < (nsplit ? 2 : 1); ++p)
+      if (driver().LaunchKernel(bv.fn[p == 0 ? 1 : 3], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1,
+                                b.nstaged ? static_cast<unsigned>(nsplit ? b.nsmem_p[p] : b.nsmem) : 0u,
+                                st, args, nullptr) != CUDA_SUCCESS)
+        return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed (backward, nodes)");
   }
   return E3CONV_OK;
 }
 
 int e3conv_backward_source(e3conv_plan h, int which, char* buf, size_t buf_len, size_t* needed) {
-  if (!h || which < 0 || which > 2) return fail(E3CONV_ERR_INVALID_ARG, "bad argument");
+  if (!h || which < 0 || which > 3) return fail(E3CONV_ERR_INVALID_ARG, "bad argument");
   DeviceGuard g(h->p.device);
   int rc = prepare_backward(h->p);
   if (rc != E3CONV_OK) return rc;
-  if (which == 2 && h->p.bwd[h->p.dtype].shape.eparts < 2)
-    return fail(E3CONV_ERR_INVALID_ARG, "the edges kernel of this plan is not split");
+  if (which >= 2 && h->p.bwd[h->p.dtype].source[which].empty())
+    return fail(E3CONV_ERR_INVALID_ARG, "this plan's backward kernels are not split");
   const std::string& src = h->p.bwd[h->p.dtype].source[which];
   if (needed) *needed = src.size() + 1;
   if (buf && buf_len >= src.size() + 1) std::memcpy(buf, src.c_str(), src.size() + 1);

@@ -1930,12 +1930,19 @@ BwdShape choose_backward_shape(const Plan& pl, int dtype) {
   b.smem = (b.block / 32) * 2 * b.stage_bytes;
   b.staged = TL == 32 && V % 2 == 0 && b.s_bytes % 16 == 0 && b.x_bytes % 16 == 0 &&
              (pl.ny * elem) % 4 == 0 && b.smem <= 112 * 1024;
-  // a grad_out row of more than 64 registers per lane: the edges kernel runs as two launches,
-  // each over half of the output irreps (balanced by their (i, k) terms), so each holds half
-  // of the row and stages only its paths' scalars
+  b.g_bytes = pl.nout * pl.C * 4;
+  b.nstage_bytes = b.s_bytes + b.g_bytes + b.y_bytes;
+  b.nsmem = (b.block / 32) * 2 * b.nstage_bytes;
+  b.nstaged = TL == 32 && V % 2 == 0 && b.s_bytes % 16 == 0 && b.g_bytes % 16 == 0 &&
+              (pl.ny * elem) % 4 == 0 && b.nsmem <= 220 * 1024;
+  // a grad_out row of more than 64 registers per lane: the edges kernel (and the staged nodes
+  // kernel) run as two launches, each over half of the output irreps (balanced by their (i, k)
+  // terms), so each holds half of the row and stages only its paths' scalars (and, for grad_x,
+  // only its outputs' gradient rows)
   b.eparts = 1;
   b.out_part.assign(pl.outputs.size(), 0);
   b.esmem[0] = b.esmem[1] = b.smem;
+  b.nsmem_p[0] = b.nsmem_p[1] = b.nsmem;
   if (b.staged && pl.nout * V > 64 && pl.outputs.size() > 1 && (pl.C * elem) % 16 == 0) {
     std::vector<std::pair<long long, int>> work;  // (terms, output irrep)
     for (size_t o = 0; o < pl.outputs.size(); ++o) {
@@ -1958,17 +1965,15 @@ BwdShape choose_backward_shape(const Plan& pl, int dtype) {
     if (load[0] > 0 && load[1] > 0) {
       b.eparts = 2;
       for (int t = 0; t < 2; ++t) {
-        int np = 0;
+        int np = 0, nc = 0;
         for (const auto& P : pl.paths) np += b.out_part[P.o] == t;
+        for (size_t o = 0; o < pl.outputs.size(); ++o)
+          if (b.out_part[o] == t) nc += 2 * pl.outputs[o].l + 1;
         b.esmem[t] = (b.block / 32) * 2 * (np * pl.C * elem + b.x_bytes + b.y_bytes);
+        b.nsmem_p[t] = (b.block / 32) * 2 * (np * pl.C * elem + nc * pl.C * 4 + b.y_bytes);
       }
     }
   }
-  b.g_bytes = pl.nout * pl.C * 4;
-  b.nstage_bytes = b.s_bytes + b.g_bytes + b.y_bytes;
-  b.nsmem = (b.block / 32) * 2 * b.nstage_bytes;
-  b.nstaged = TL == 32 && V % 2 == 0 && b.s_bytes % 16 == 0 && b.g_bytes % 16 == 0 &&
-              (pl.ny * elem) % 4 == 0 && b.nsmem <= 220 * 1024;
   return b;
 }
 
@@ -2436,8 +2441,22 @@ std::string bwd_edges_staged_source(const Plan& pl, int dtype, const BwdShape& b
 // receiver's gradient row g (float32) and its Y row by cp.async, one edge ahead.  Per edge
 // and path, with A_ik = sum_j c_ijk Y_j formed per lane and u_k = s g_k (channel pairs):
 //   h_i += sum_k A_ik u_k,   grad_x[a] = (1/N) h.
-std::string bwd_nodes_staged_source(const Plan& pl, int dtype, const BwdShape& b) {
+std::string bwd_nodes_staged_source(const Plan& pl, int dtype, const BwdShape& b, int part) {
   Emitter em;
+  // this launch's output irreps (their gradient rows and paths), as in the edges kernel
+  std::vector<bool> own_out(pl.outputs.size(), true);
+  if (b.eparts > 1)
+    for (size_t o = 0; o < pl.outputs.size(); ++o) own_out[o] = b.out_part[o] == part;
+  std::vector<int> slot(pl.paths.size(), -1), gpos(pl.outputs.size(), -1);
+  int nslots = 0, ncomp = 0;
+  for (size_t r = 0; r < pl.paths.size(); ++r)
+    if (own_out[pl.paths[r].o]) slot[r] = nslots++;
+  for (size_t o = 0; o < pl.outputs.size(); ++o)
+    if (own_out[o]) {
+      gpos[o] = ncomp;
+      ncomp += 2 * pl.outputs[o].l + 1;
+    }
+  const bool accumulate = b.eparts > 1 && part > 0;
   const std::string T = bwd_prelude(em, pl, dtype, b);
   emit_pair_ops(em);
   em.line("__device__ __forceinline__ void upk(unsigned long long w, float& lo, float& hi) { asm(\"mov.b64 {%0, %1}, %2;\" : \"=f\"(lo), \"=f\"(hi) : \"l\"(w)); }");
@@ -2450,9 +2469,14 @@ std::string bwd_nodes_staged_source(const Plan& pl, int dtype, const BwdShape& b
   const int V = b.V, NG = V / 2, elem = f16 ? 2 : 4;
   const long long s_row = static_cast<long long>(pl.paths.size()) * pl.C;
   const long long g_row = static_cast<long long>(pl.nout) * pl.C;
-  const int SB = b.nstage_bytes;
-  const int g_off = b.s_bytes, y_off = b.s_bytes + b.g_bytes;
-  em.line("extern \"C\" __global__ void __launch_bounds__(" + S(b.block) + ") e3conv_bwd_nodes(");
+  const int s_bytes = nslots * pl.C * elem, g_bytes = ncomp * pl.C * 4;
+  const int SB = s_bytes + g_bytes + b.y_bytes;
+  const int g_off = s_bytes, y_off = s_bytes + g_bytes;
+  em.line("// part " + S(part) + " of " + S(b.eparts) + ": " + S(nslots) + " of " + S(pl.paths.size()) +
+          " paths" + (accumulate ? ", grad_x added to the earlier part's" : ""));
+  const int minb = std::max(1, std::min(3, (220 * 1024) / std::max(1, (b.block / 32) * 2 * SB)));
+  em.line("extern \"C\" __global__ void __launch_bounds__(" + S(b.block) +
+          (minb > 1 ? ", " + S(minb) : std::string()) + ") e3conv_bwd_nodes(");
   em.line("    const " + T + "* __restrict__ Y, const " + T + "* __restrict__ s,");
   em.line("    const int* __restrict__ receivers, const int* __restrict__ row_ptr,");
   em.line("    const int* __restrict__ sender_row_ptr, const int* __restrict__ sender_perm,");
@@ -2488,18 +2512,24 @@ std::string bwd_nodes_staged_source(const Plan& pl, int dtype, const BwdShape& b
   em.line("const unsigned char* ssrc = reinterpret_cast<const unsigned char*>(s + (long long)le * " + S(s_row) + ");");
   em.line("const unsigned char* gsrc = reinterpret_cast<const unsigned char*>(g + (long long)bb * " + S(g_row) + ");");
   em.line("const unsigned char* ysrc = reinterpret_cast<const unsigned char*>(Y + (long long)le * " + S(pl.ny) + ");");
-  em.line("#pragma unroll");
-  em.line("for (int q = lane; q < " + S(b.s_bytes / 16) + "; q += 32) cp16(dst + 16 * q, ssrc + 16 * q);");
-  em.line("#pragma unroll");
-  em.line("for (int q = lane; q < " + S(b.g_bytes / 16) + "; q += 32) cp16(dst + " + S(g_off) + " + 16 * q, gsrc + 16 * q);");
+  for (size_t r = 0; r < pl.paths.size(); ++r)      // the part's paths' scalars
+    if (slot[r] >= 0)
+      em.line("for (int q = lane; q < " + S(pl.C * elem / 16) + "; q += 32) cp16(dst + " +
+              S(slot[r] * pl.C * elem) + " + 16 * q, ssrc + " + S(static_cast<long long>(r) * pl.C * elem) +
+              " + 16 * q);");
+  for (size_t o = 0; o < pl.outputs.size(); ++o)     // the part's gradient components
+    if (gpos[o] >= 0)
+      em.line("for (int q = lane; q < " + S((2 * pl.outputs[o].l + 1) * pl.C * 4 / 16) + "; q += 32) cp16(dst + " +
+              S(g_off + gpos[o] * pl.C * 4) + " + 16 * q, gsrc + " +
+              S(static_cast<long long>(pl.outputs[o].off) * pl.C * 4) + " + 16 * q);");
   em.line("for (int q = lane; q < " + S(pl.ny * elem / 4) + "; q += 32) cp4(dst + " + S(y_off) + " + 4 * q, ysrc + 4 * q);");
   em.ind--;
   em.line("} else {  // a bad index contributes nothing: a zero row of scalars and harmonics");
   em.ind++;
   em.line("#pragma unroll");
-  em.line("for (int q = lane; q < " + S(b.s_bytes / 16) + "; q += 32) *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(0u, 0u, 0u, 0u);");
+  em.line("for (int q = lane; q < " + S(s_bytes / 16) + "; q += 32) *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(0u, 0u, 0u, 0u);");
   em.line("#pragma unroll");
-  em.line("for (int q = lane; q < " + S(b.g_bytes / 16) + "; q += 32) *reinterpret_cast<uint4*>(dst + " + S(g_off) + " + 16 * q) = make_uint4(0u, 0u, 0u, 0u);");
+  em.line("for (int q = lane; q < " + S(g_bytes / 16) + "; q += 32) *reinterpret_cast<uint4*>(dst + " + S(g_off) + " + 16 * q) = make_uint4(0u, 0u, 0u, 0u);");
   em.line("for (int q = lane; q < " + S(b.y_bytes / 4) + "; q += 32) *reinterpret_cast<unsigned int*>(dst + " + S(y_off) + " + 4 * q) = 0u;");
   em.ind--;
   em.line("}");
@@ -2535,7 +2565,8 @@ std::string bwd_nodes_staged_source(const Plan& pl, int dtype, const BwdShape& b
     }
   };
   for (size_t o = 0; o < pl.outputs.size(); ++o) {
-    const int d3 = 2 * pl.outputs[o].l + 1, off = pl.outputs[o].off;
+    if (!own_out[o]) continue;
+    const int d3 = 2 * pl.outputs[o].l + 1, off = gpos[o];  // off: the component in the ring
     bool any = false;
     for (const auto& P : pl.paths) any = any || P.o == static_cast<int>(o);
     if (!any) continue;
@@ -2555,7 +2586,7 @@ std::string bwd_nodes_staged_source(const Plan& pl, int dtype, const BwdShape& b
       if (P.o != static_cast<int>(o)) continue;
       em.line("{  // path " + S(r) + ": " + S(P.l1) + " x " + S(P.l2) + " -> " + S(P.l3));
       em.ind++;
-      load_s("ss + " + S(static_cast<long long>(r) * pl.C));
+      load_s("ss + " + S(static_cast<long long>(slot[r]) * pl.C));
       std::map<std::pair<int, int>, std::vector<std::pair<int, double>>> ki;  // k-major
       for (const auto& n : P.nnz) ki[{n.k, n.i}].push_back({n.j, n.c});
       int uopen = -1;
@@ -2605,11 +2636,17 @@ std::string bwd_nodes_staged_source(const Plan& pl, int dtype, const BwdShape& b
     const std::string dst = "xo + " + S(i * pl.C);
     if (NG == 2) {
       em.line("{ float a0_, a1_, a2_, a3_; upk(mul2(inv2, h" + S(i) + "_0), a0_, a1_); upk(mul2(inv2, h" + S(i) +
-              "_1), a2_, a3_); *reinterpret_cast<float4*>(" + dst + ") = make_float4(a0_, a1_, a2_, a3_); }");
+              "_1), a2_, a3_);");
+      if (accumulate)
+        em.line("  const float4 p_ = *reinterpret_cast<const float4*>(" + dst + "); a0_ += p_.x; a1_ += p_.y; a2_ += p_.z; a3_ += p_.w;");
+      em.line("  *reinterpret_cast<float4*>(" + dst + ") = make_float4(a0_, a1_, a2_, a3_); }");
     } else {
-      for (int g = 0; g < NG; ++g)
-        em.line("{ float a_, b_; upk(mul2(inv2, h" + S(i) + "_" + S(g) + "), a_, b_); *reinterpret_cast<float2*>(" +
-                dst + " + " + S(2 * g) + ") = make_float2(a_, b_); }");
+      for (int g = 0; g < NG; ++g) {
+        em.line("{ float a_, b_; upk(mul2(inv2, h" + S(i) + "_" + S(g) + "), a_, b_);");
+        if (accumulate)
+          em.line("  const float2 p_ = *reinterpret_cast<const float2*>(" + dst + " + " + S(2 * g) + "); a_ += p_.x; b_ += p_.y;");
+        em.line("  *reinterpret_cast<float2*>(" + dst + " + " + S(2 * g) + ") = make_float2(a_, b_); }");
+      }
     }
   }
   em.ind--;
@@ -2714,12 +2751,16 @@ std::string bwd_nodes_source(const Plan& pl, int dtype, const BwdShape& b) {
 }  // namespace
 
 std::string generate_backward_source(const Plan& pl, int dtype, const BwdShape& b, bool nodes) {
-  if (nodes) return b.nstaged ? bwd_nodes_staged_source(pl, dtype, b) : bwd_nodes_source(pl, dtype, b);
+  if (nodes) return b.nstaged ? bwd_nodes_staged_source(pl, dtype, b, 0) : bwd_nodes_source(pl, dtype, b);
   return b.staged ? bwd_edges_staged_source(pl, dtype, b, 0) : bwd_edges_source(pl, dtype, b);
 }
 
 std::string generate_backward_edges_part(const Plan& pl, int dtype, const BwdShape& b, int part) {
   return bwd_edges_staged_source(pl, dtype, b, part);
+}
+
+std::string generate_backward_nodes_part(const Plan& pl, int dtype, const BwdShape& b, int part) {
+  return bwd_nodes_staged_source(pl, dtype, b, part);
 }
 
 // Standalone harmonics: one thread per edge evaluates the plan's polynomials of

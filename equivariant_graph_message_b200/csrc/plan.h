@@ -110,17 +110,20 @@ struct BwdShape {
   int eparts = 1;
   std::vector<int> out_part;
   int esmem[2] = {0, 0};
+  int nsmem_p[2] = {0, 0};  // the staged nodes kernel's launches, likewise
 };
 
 struct BwdVariant {
   bool compiled = false;
   BwdShape shape;
-  std::string source[3];     // edges (part 0), nodes, edges part 1 (when the edges kernel is split)
-  std::vector<char> cubin[3];
-  std::string log[3];
-  CUmodule module[3] = {nullptr, nullptr, nullptr};
-  CUfunction fn[3] = {nullptr, nullptr, nullptr};
-  int regs[3] = {-1, -1, -1}, local_bytes[3] = {-1, -1, -1};
+  // 0 edges, 1 nodes, and where the kernels are split over the output irreps: 2 edges part 1,
+  // 3 nodes part 1
+  std::string source[4];
+  std::vector<char> cubin[4];
+  std::string log[4];
+  CUmodule module[4] = {nullptr, nullptr, nullptr, nullptr};
+  CUfunction fn[4] = {nullptr, nullptr, nullptr, nullptr};
+  int regs[4] = {-1, -1, -1, -1}, local_bytes[4] = {-1, -1, -1, -1};
 };
 
 struct ShVariant {  // standalone harmonics kernel (compiled on first use)
@@ -248,6 +251,7 @@ BwdShape choose_backward_shape(const Plan& plan, int dtype);
 std::string generate_backward_source(const Plan& plan, int dtype, const BwdShape& shape, bool nodes);
 std::string generate_sh_source(const Plan& plan, int dtype);
 std::string generate_backward_edges_part(const Plan& plan, int dtype, const BwdShape& shape, int part);
+std::string generate_backward_nodes_part(const Plan& plan, int dtype, const BwdShape& shape, int part);
 
 }  // namespace e3c
 

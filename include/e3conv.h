@@ -446,9 +446,10 @@ E3CONV_API int e3conv_backward(e3conv_plan plan, const void* node_features, cons
  * dtype (host-side, blocking). */
 E3CONV_API int e3conv_prepare_backward(e3conv_plan plan);
 
-/* Generated CUDA source of a backward kernel (which = 0: edges, 1: nodes,
- * 2: the second edges launch where the edges kernel is split over the output
- * irreps; E3CONV_ERR_INVALID_ARG where it is not), as e3conv_kernel_source. */
+/* Generated CUDA source of a backward kernel (which = 0: edges, 1: nodes;
+ * where the kernels are split over the output irreps, 2: the second edges
+ * launch and 3: the second nodes launch; E3CONV_ERR_INVALID_ARG where they are
+ * not), as e3conv_kernel_source. */
 E3CONV_API int e3conv_backward_source(e3conv_plan plan, int which, char* buf, size_t buf_len,
                                       size_t* needed);
 

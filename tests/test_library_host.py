@@ -447,10 +447,12 @@ def test_backward_kernels_generate_for_every_workload(name):
     s = SPECS[name]
     c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 10.0, dtype=s.dtype)
     edges, nodes = c.backward_source(0), c.backward_source(1)
-    if "// part 0 of 2" in edges:      # the edges kernel split over the output irreps: both launches
+    if "// part 0 of 2" in edges:      # kernels split over the output irreps: both launches each
         second = c.backward_source(2)
         assert "// part 1 of 2" in second and "gY[le * " in second
         edges += second
+        if "cp.async" in nodes:
+            nodes += c.backward_source(3)
     else:
         with pytest.raises(e3.E3ConvError):
             c.backward_source(2)
