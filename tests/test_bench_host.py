@@ -1,5 +1,5 @@
 """Host-side checks of bench.py's accounting: the roofline's algorithmic bytes and FLOPs per
-edge against the survey's independently enumerated per-config sizes, the peaks it divides by,
+edge against independently enumerated per-config sizes, the peaks it divides by,
 and the CPU-baseline sample sizing."""
 import os
 import sys
