@@ -559,7 +559,7 @@ int e3conv_set_option(e3conv_plan h, int option, int value) {
     if (value != -1 && (value < 1 || value > 4)) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1 or 1 .. 4");
     pl.req_group = value;
   } else if (option == E3CONV_OPT_A_LAYOUT) {
-    if (value < -1 || value > 2) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1 .. 2");
+    if (value < -1 || value > 3) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1 .. 3");
     pl.req_alayout = value;
   } else if (option == E3CONV_OPT_EDGE_VECTORS) {
     if (value != 0 && value != 1) return fail(E3CONV_ERR_INVALID_ARG, "value must be 0 or 1");

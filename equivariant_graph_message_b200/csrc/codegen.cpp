@@ -201,7 +201,7 @@ Shape choose_shape(const Plan& pl, int dtype) {
     // broadcast pairs in apply order read two per 16-byte load
     s.amode = 0;  // measured fastest for every workload (large_f32 4.05 vs 4.83 ms with pairs)
     if (s.coop && V % 2 == 0 && pl.req_alayout >= 0) s.amode = pl.req_alayout;
-    s.dup_a = s.amode >= 1;
+    s.dup_a = s.amode == 1 || s.amode == 2;
     s.na = s.coop ? static_cast<int>(build_a_entries(pl).size()) : 0;
     int a_bytes = 0;
     if (s.coop)
@@ -895,12 +895,14 @@ CoopTables coop_tables(const CoopGroup& G) {
     return ent[a].terms.size() > ent[b].terms.size();
   });
   T.slot.assign(ent.size(), -1);
-  if (G.amode == 2) {
+  if (G.amode == 2 || G.amode == 3) {
+    // apply order, each path's run padded to the load width (2 pairs or 4 floats per 16 bytes)
+    const int w = G.amode == 2 ? 2 : 4;
     int pos = 0;
     for (int p : G.paths) {
       for (size_t n = 0; n < ent.size(); ++n)
         if (ent[n].path == p) T.slot[n] = pos++;
-      pos += pos & 1;
+      pos = (pos + w - 1) / w * w;
     }
   } else {
     for (size_t q = 0; q < order.size(); ++q) T.slot[order[q]] = static_cast<int>(q);
@@ -929,7 +931,7 @@ CoopTables coop_tables(const CoopGroup& G) {
           j = ent[order[q]].terms[t].first;
           cv = ent[order[q]].terms[t].second;
         }
-        if (G.amode == 2 && t == 0 && q < order.size()) j |= T.slot[order[q]] << 8;
+        if (G.amode >= 2 && t == 0 && q < order.size()) j |= T.slot[order[q]] << 8;
         const float cf = static_cast<float>(cv);
         unsigned int bits;
         std::memcpy(&bits, &cf, sizeof bits);
@@ -955,7 +957,7 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh, con
   const Lanes L{sh.V};
   const int RW = G.RW;
   const std::string& ln = G.lane;
-  if (G.amode >= 1)
+  if (G.amode == 1 || G.amode == 2)
     em.line("unsigned long long* Aw = reinterpret_cast<unsigned long long*>(tbase + " + S(G.a_off) + ");");
   else
     em.line("float* Aw = reinterpret_cast<float*>(tbase + " + S(G.a_off) + ");");
@@ -968,12 +970,12 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh, con
     for (int t = 0; t < T.terms[r]; ++t)
       em.line("const int2 k" + S(t) + " = __ldg(&e3_atab" + G.sfx + "[" + S(base + t * RW) + " + " +
               ln + "]);");
-    const std::string j0 = G.amode == 2 ? "(k0.y & 255)" : "k0.y";
+    const std::string j0 = G.amode >= 2 ? "(k0.y & 255)" : "k0.y";
     std::string v = "__int_as_float(k0.x) * yf[" + j0 + "]";
     for (int t = 1; t < T.terms[r]; ++t)
       v = "fmaf(__int_as_float(k" + S(t) + ".x), yf[k" + S(t) + ".y], " + v + ")";
-    const std::string dst = G.amode == 2 ? "Aw[k0.y >> 8]" : "Aw[" + S(r * RW) + " + " + ln + "]";
-    if (G.amode >= 1) v = "bc(" + v + ")";
+    const std::string dst = G.amode >= 2 ? "Aw[k0.y >> 8]" : "Aw[" + S(r * RW) + " + " + ln + "]";
+    if (G.amode == 1 || G.amode == 2) v = "bc(" + v + ")";
     if ((r + 1) * RW <= na)
       em.line(dst + " = " + v + ";");
     else
@@ -1032,6 +1034,21 @@ void emit_coop_edge(Emitter& em, const Plan& pl, int dtype, const Shape& sh, con
                     "); " + aval(bys[m]) + " = t_.x; " + aval(bys[m + 1]) + " = t_.y; }");
           else
             em.line("const unsigned long long " + aval(bys[m]) + " = Aw[" + S(s0) + "];");
+        }
+      } else if (G.amode == 3) {
+        // float entries in slot order, four per 16-byte load, broadcast to pairs
+        std::vector<const AEntry*> bys(pe);
+        std::sort(bys.begin(), bys.end(), [&](const AEntry* a, const AEntry* b) {
+          return T.slot[idx[{a->path, a->i, a->k}]] < T.slot[idx[{b->path, b->i, b->k}]];
+        });
+        const char* comp[4] = {"x", "y", "z", "w"};
+        for (size_t m = 0; m < bys.size(); m += 4) {
+          const int s0 = T.slot[idx[{bys[m]->path, bys[m]->i, bys[m]->k}]];
+          std::string decl = "const float4 a4_" + S(s0) + " = *reinterpret_cast<const float4*>(Aw + " + S(s0) + ");";
+          em.line(decl);
+          for (size_t u = 0; u < 4 && m + u < bys.size(); ++u)
+            em.line("const " + L.type() + " " + aval(bys[m + u]) + " = " +
+                    L.bc("a4_" + S(s0) + "." + comp[u]) + ";");
         }
       } else {
         for (const AEntry* e : pe) {
@@ -1191,16 +1208,17 @@ std::vector<CoopGroupInfo> coop_groups(const Plan& pl, const Shape& sh) {
   }
   for (auto& g : gs) {
     int slots = 0;
-    if (g.amode == 2) {
+    if (g.amode == 2 || g.amode == 3) {
+      const int w = g.amode == 2 ? 2 : 4;
       for (int p : g.paths) {
         int n = 0;
         for (const auto& e : g.ent) n += e.path == p;
-        slots += n + (n & 1);
+        slots += (n + w - 1) / w * w;
       }
     } else {
       slots = static_cast<int>(g.ent.size());
     }
-    g.a_bytes = align_up((g.amode >= 1 ? 8 : 4) * slots, 16);
+    g.a_bytes = align_up((g.amode == 1 || g.amode == 2 ? 8 : 4) * slots, 16);
     g.nacc = 0;
     for (int a : g.acc) g.nacc = std::max(g.nacc, a + 1);
   }

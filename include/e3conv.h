@@ -179,11 +179,12 @@ E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane,
  *   above, l <= the plan's lmax; a zero vector gives Y_0 = 1, the rest 0),
  *   in float32, instead of reading ny harmonics per edge. */
 #define E3CONV_OPT_EDGE_VECTORS 4
-/*   E3CONV_OPT_A_LAYOUT: -1 automatic (default), 0, 1 or 2: the shared-memory
+/*   E3CONV_OPT_A_LAYOUT: -1 automatic (default), 0 .. 3: the shared-memory
  *   layout of the contract-first A entries where a lane holds channel pairs:
  *   0 float entries in the order they are formed (a lane duplicates each into
  *   a pair), 1 the entries stored as (a, a) pairs in that order, 2 (a, a)
- *   pairs in the order they are applied, read two per 16-byte load.
+ *   pairs in the order they are applied, read two per 16-byte load, 3 float
+ *   entries in the order they are applied, read four per 16-byte load.
  *   Automatic: 0.  Same arithmetic. */
 #define E3CONV_OPT_A_LAYOUT 5
 /*   E3CONV_OPT_COPY_GROUP: -1 automatic (default: 1) or 1..4: the staged

@@ -224,3 +224,28 @@ def test_copy_groups_are_bitwise_the_single_edge_ring(cuda_device, group, stages
     assert np.array_equal(a, b)
     ref = oracle_out(irreps, x, Y, s, send, recv, n, 9.0)
     assert column_scaled_error(b, ref) <= 1e-5
+
+
+@pytest.mark.parametrize("layout", [1, 2, 3])
+@pytest.mark.parametrize("C,dt", [(128, "f16"), (64, "f32")])
+def test_a_layouts_are_bitwise_the_default(cuda_device, layout, C, dt):
+    # the A entries' shared-memory layout changes where each entry is stored and how it is
+    # loaded, not the products or their order: every layout gives the default's bits
+    irreps = IRREPS[C]
+    rng = np.random.default_rng(20 * layout + C)
+    n, e = 700, 10000
+    send, recv = _graph(rng, n, e, empty_frac=0.1)
+    recv[:260] = 11                        # a row of more than two 128-edge chunks
+    o = np.lexsort((send, recv))
+    send, recv = send[o], recv[o]
+    pl, x, Y, s = _inputs(rng, irreps, n, e, dt)
+    base = e3.Conv(*irreps, 11.0, dtype=dt)
+    base.set_a_layout(0)
+    lay = e3.Conv(*irreps, 11.0, dtype=dt)
+    lay.set_a_layout(layout)
+    assert f"a_layout={layout}" in lay.kernel_source()
+    a = run_gpu(base, x, Y, s, send, recv, n)
+    b = run_gpu(lay, x, Y, s, send, recv, n)
+    assert np.array_equal(a, b)
+    ref = oracle_out(irreps, x, Y, s, send, recv, n, 11.0)
+    assert column_scaled_error(b, ref) <= (5e-3 if dt == "f16" else 1e-5)

@@ -103,7 +103,7 @@ def _emulate_phase1(c, src, Y, expect_entries):
     for sfx, items in re.findall(r"// A layout(\S*) \(entry: path i k slot\):(.*)", src):
         m = re.search(r"// A rounds" + re.escape(sfx) + r" \(lanes (\d+), mode (\d)\):(.*)", src)
         rw, mode, terms = int(m.group(1)), int(m.group(2)), [int(v) for v in m.group(3).split()]
-        pairs = mode == 2
+        encoded = mode >= 2          # apply-order layouts: the slot travels in the first index
         entries = [tuple(int(v) for v in it.split(":")) for it in items.split()]
         tab = re.search(r"e3_atab" + re.escape(sfx) + r"\[\] = \{(.*?)\};", src, re.S).group(1)
         cells = [(int(a), int(b)) for a, b in re.findall(r"\{(-?\d+), (\d+)\}", tab)]
@@ -117,7 +117,7 @@ def _emulate_phase1(c, src, Y, expect_entries):
                 v, slot = 0.0, q
                 for term in range(nterms):
                     cb, j = cells[base + term * rw + lane]
-                    if pairs and term == 0:
+                    if encoded and term == 0:
                         slot, j = j >> 8, j & 255
                     v += np.frombuffer(np.int32(cb).tobytes(), np.float32)[0] * Y[j]
                 slots[slot] = v
@@ -132,6 +132,26 @@ def _emulate_phase1(c, src, Y, expect_entries):
         seen += len(entries)
     assert seen == expect_entries
     return seen
+
+
+@pytest.mark.parametrize("layout", [0, 1, 2, 3])
+@pytest.mark.parametrize("name", ["large_f16", "large_f32", "mace"])
+def test_a_layouts_form_every_entry_and_load_within_the_area(name, layout):
+    # every A layout: the generated phase-1 tables form each entry in its own slot; the
+    # apply-order float layout (3) reads 16-byte groups that start on a multiple of four slots
+    s = SPECS[name]
+    c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 40.0, dtype=s.dtype)
+    c.set_a_layout(layout)
+    src = c.kernel_source()
+    assert f"a_layout={layout}" in src and c.kernel_info()["local_bytes"] == 0
+    na = sum(int((np.abs(c.cg(p)) > 1e-12).any(axis=1).sum()) for p in range(c.num_paths))
+    _emulate_phase1(c, src, np.random.default_rng(layout).normal(size=c.ny), expect_entries=na)
+    if layout == 3:
+        starts = [int(v) for v in re.findall(r"const float4 a4_\d+ = \*reinterpret_cast<const float4\*>\(Aw \+ (\d+)\)", src)]
+        assert starts and all(v % 4 == 0 for v in starts)
+        slots = [int(it.split(":")[3]) for it in
+                 re.search(r"// A layout \(entry: path i k slot\):(.*)", src).group(1).split()]
+        assert max(starts) + 4 <= (max(slots) + 4) // 4 * 4
 
 
 def test_generated_kernel_unrolls_every_coefficient():
