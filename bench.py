@@ -77,9 +77,12 @@ def parse_args():
     ap.add_argument("--radial", action="store_true",
                     help="edge scalars from the radial MLP on the tensor cores every step "
                          "(workloads with MLP scalars)")
-    ap.add_argument("--next-rows", action="store_true",
+    ap.add_argument("--next-rows", dest="next_rows", action="store_true", default=True,
                     help="after the timed region, time the backward and the irreps linear layer "
-                         "on the same workload (supplementary entries with their rooflines)")
+                         "on the same workload (supplementary entries with their rooflines; on "
+                         "by default)")
+    ap.add_argument("--no-next-rows", dest="next_rows", action="store_false",
+                    help="skip the supplementary next-row timings")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the supplementary timing of the tensor-core variant")
     return ap.parse_args()
