@@ -83,6 +83,9 @@ def parse_args():
                          "by default)")
     ap.add_argument("--no-next-rows", dest="next_rows", action="store_false",
                     help="skip the supplementary next-row timings")
+    ap.add_argument("--no-graphs", action="store_true",
+                    help="launch the step's kernels one by one instead of replaying CUDA graphs "
+                         "of the CSR build and of the forward")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the supplementary timing of the tensor-core variant")
     return ap.parse_args()
@@ -466,22 +469,42 @@ def run_ours(args):
         else:
             sharding.exchange_rows(shard, x, table)
 
+    def csr_part(h):
+        e3._ok(e3._build_csr(precv, E_loc, rows, prp, pperm, pws, ws_bytes, h), "e3conv_build_csr")
+
+    def radial_part(h):
+        e3._ok(e3._radial_scalars(conv._h, pY, E_loc, ps, h), "e3conv_radial_scalars")
+
+    def forward_part(h):
+        if shard is None:
+            conv.forward_raw(ptab, pY, ps, psend, prp, N, pout, h)
+        else:
+            conv.forward_rows_raw(ptab, shard.table_rows, pY, ps, psend, prp, 0, rows, pout, h)
+
+    graphs = None
+
     def step(fwd_events=None, radial_events=None):
-        e3._ok(e3._build_csr(precv, E_loc, rows, prp, pperm, pws, ws_bytes, sh), "e3conv_build_csr")
+        if graphs:
+            graphs["csr"].replay()
+        else:
+            csr_part(sh)
         if shard is not None:
             exchange()
         if args.radial:
             if radial_events:
                 radial_events[0].record(stream)
-            e3._ok(e3._radial_scalars(conv._h, pY, E_loc, ps, sh), "e3conv_radial_scalars")
+            if graphs:
+                graphs["radial"].replay()
+            else:
+                radial_part(sh)
             if radial_events:
                 radial_events[1].record(stream)
         if fwd_events:
             fwd_events[0].record(stream)
-        if shard is None:
-            conv.forward_raw(ptab, pY, ps, psend, prp, N, pout, sh)
+        if graphs:
+            graphs["forward"].replay()
         else:
-            conv.forward_rows_raw(ptab, shard.table_rows, pY, ps, psend, prp, 0, rows, pout, sh)
+            forward_part(sh)
         if fwd_events:
             fwd_events[1].record(stream)
 
@@ -489,6 +512,22 @@ def run_ours(args):
         step()
     torch.cuda.synchronize()
     assert e3.csr_check(ws) and conv.check(), "bad index met during warm-up"
+    if not args.no_graphs and world == 1:
+        # one CUDA graph per part of the step (the library's calls launch on the capture
+        # stream and neither allocate nor synchronise): a replay per part and step
+        graphs = {}
+        parts = [("csr", csr_part), ("forward", forward_part)]
+        if args.radial:
+            parts.insert(1, ("radial", radial_part))
+        for name, fn in parts:
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                fn(e3._stream_handle(torch.cuda.current_stream()))
+            graphs[name] = gr
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        assert e3.csr_check(ws) and conv.check(), "bad index met during the graph warm-up"
     info = conv.kernel_info()
 
     clocks = Clocks(local)
@@ -627,6 +666,8 @@ def run_ours(args):
                                    f"receiver rows sharded over {world} ranks "
                                    f"(e3conv_partition_rows), {args.exchange} exchange"),
                    "l2": f"inputs larger than L2 ({nbytes / 1e9:.1f} GB read per forward per GPU)",
+                   "launch": ("CUDA graph replays (one graph per part of the step)" if graphs
+                              else "eager launches"),
                    "forward_edges_per_s": total_edges / (fwd_ms / 1000.0),
                    "kernel": info},
         "roofline": roof,
