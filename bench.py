@@ -83,6 +83,8 @@ def parse_args():
                          "by default)")
     ap.add_argument("--no-next-rows", dest="next_rows", action="store_false",
                     help="skip the supplementary next-row timings")
+    ap.add_argument("--backward-parts", type=int, default=-1,
+                    help="launches of each backward kernel in the next-row timing (-1 automatic)")
     ap.add_argument("--no-graphs", action="store_true",
                     help="launch the step's kernels one by one instead of replaying CUDA graphs "
                          "of the CSR build and of the forward")
@@ -715,6 +717,8 @@ def time_next_rows(args, spec, g, conv, x, Y, s, senders, receivers, row_ptr, ou
     N, E = g.num_nodes, g.num_edges
     res = {}
     reps = max(3, min(args.steps, 10))
+    if args.backward_parts != -1:
+        conv.set_backward_parts(args.backward_parts)
     if not conv.edge_vectors and conv.C <= (256 if spec.dtype == "f16" else 128):
         gout = torch.randn(out.shape, generator=torch.Generator(device=out.device).manual_seed(7),
                            device=out.device)

@@ -60,6 +60,7 @@ OPT_EDGE_VECTORS = 4
 OPT_A_LAYOUT = 5
 OPT_COPY_GROUP = 6
 OPT_DIRECT_PIPELINE = 7
+OPT_BACKWARD_PARTS = 8
 _get_option = _sig("e3conv_get_option", ctypes.c_int, _vp, ctypes.c_int, _c_int_p)
 _sh_host = _sig("e3conv_spherical_harmonics", ctypes.c_int, _vp, ctypes.POINTER(ctypes.c_double),
                 ctypes.POINTER(ctypes.c_double))
@@ -241,6 +242,10 @@ class Conv:
 
     def set_direct_pipeline(self, value: int = -1):
         _ok(_set_option(self._h, OPT_DIRECT_PIPELINE, value), "e3conv_set_option")
+
+    def set_backward_parts(self, value: int = -1):
+        """Launches of each staged backward kernel (-1 automatic, 1 .. 4)."""
+        _ok(_set_option(self._h, OPT_BACKWARD_PARTS, value), "e3conv_set_option")
 
     def set_copy_group(self, value: int = -1):
         _ok(_set_option(self._h, OPT_COPY_GROUP, value), "e3conv_set_option")

@@ -214,42 +214,48 @@ int prepare_backward(Plan& pl) {
   v.shape = choose_backward_shape(pl, pl.dtype);
   if (!v.shape.ok)
     return fail(E3CONV_ERR_UNSUPPORTED, "backward needs C <= 128 (float32) or <= 256 (float16)");
-  // modules: 0 edges (part 0), 1 nodes (part 0), 2 edges part 1 and 3 nodes part 1 where the
-  // kernels are split over the output irreps (the nodes kernel only when it is staged)
-  const bool esplit = v.shape.eparts > 1, nsplit = esplit && v.shape.nstaged;
-  const int nmod = nsplit ? 4 : esplit ? 3 : 2;
-  const char* names[4] = {"e3conv_bwd_edges", "e3conv_bwd_nodes", "e3conv_bwd_edges", "e3conv_bwd_nodes"};
-  const char* files[4] = {"e3conv_bwd_edges.cu", "e3conv_bwd_nodes.cu", "e3conv_bwd_edges_1.cu",
-                          "e3conv_bwd_nodes_1.cu"};
-  for (int k = 0; k < nmod; ++k) {
-    v.source[k] = k == 2   ? generate_backward_edges_part(pl, pl.dtype, v.shape, 1)
-                  : k == 3 ? generate_backward_nodes_part(pl, pl.dtype, v.shape, 1)
-                           : generate_backward_source(pl, pl.dtype, v.shape, k == 1);
-    const int rc = nvrtc_compile(v.source[k], files[k], v.cubin[k], v.log[k], v.regs[k],
-                                 v.local_bytes[k]);
+  // modules 2 p + k: part p of the edges (k = 0) and nodes (k = 1) kernels; the nodes kernel
+  // is split only when it is staged
+  const int np_e = v.shape.eparts, np_n = v.shape.nstaged ? v.shape.eparts : 1;
+  std::vector<int> mods;
+  for (int p = 0; p < np_e; ++p) mods.push_back(2 * p);
+  for (int p = 0; p < np_n; ++p) mods.push_back(2 * p + 1);
+  for (int m : mods) {
+    const int p = m / 2;
+    const bool nodes = m % 2 == 1;
+    v.source[m] = p == 0 ? generate_backward_source(pl, pl.dtype, v.shape, nodes)
+                  : nodes ? generate_backward_nodes_part(pl, pl.dtype, v.shape, p)
+                          : generate_backward_edges_part(pl, pl.dtype, v.shape, p);
+    const std::string file = std::string(nodes ? "e3conv_bwd_nodes_" : "e3conv_bwd_edges_") +
+                             std::to_string(p) + ".cu";
+    const int rc = nvrtc_compile(v.source[m], file.c_str(), v.cubin[m], v.log[m], v.regs[m],
+                                 v.local_bytes[m]);
     if (rc != E3CONV_OK) return rc;
   }
   if (pl.device >= 0) {
     Driver& d = driver();
-    for (int k = 0; k < nmod; ++k) {
-      if (d.ModuleLoadData(&v.module[k], v.cubin[k].data()) != CUDA_SUCCESS ||
-          d.ModuleGetFunction(&v.fn[k], v.module[k], names[k]) != CUDA_SUCCESS) {
-        for (int q = 0; q <= k; ++q)
-          if (v.module[q]) d.ModuleUnload(v.module[q]);
+    for (size_t q = 0; q < mods.size(); ++q) {
+      const int m = mods[q];
+      if (d.ModuleLoadData(&v.module[m], v.cubin[m].data()) != CUDA_SUCCESS ||
+          d.ModuleGetFunction(&v.fn[m], v.module[m], m % 2 ? "e3conv_bwd_nodes" : "e3conv_bwd_edges") !=
+              CUDA_SUCCESS) {
+        for (size_t r = 0; r <= q; ++r)
+          if (v.module[mods[r]]) d.ModuleUnload(v.module[mods[r]]);
         return fail(E3CONV_ERR_CUDA, "loading the backward kernels failed");
       }
     }
     bool ok = true;
-    if (v.shape.staged)
-      for (int p = 0; p < v.shape.eparts; ++p)
-        ok = ok && d.FuncSetAttribute(v.fn[p == 0 ? 0 : 2], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES,
+    for (int m : mods) {
+      const int p = m / 2;
+      if (m % 2 == 0 && v.shape.staged)
+        ok = ok && d.FuncSetAttribute(v.fn[m], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES,
                                       v.shape.esmem[p]) == CUDA_SUCCESS;
-    if (v.shape.nstaged)
-      for (int p = 0; p < (nsplit ? 2 : 1); ++p)
-        ok = ok && d.FuncSetAttribute(v.fn[p == 0 ? 1 : 3], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES,
-                                      nsplit ? v.shape.nsmem_p[p] : v.shape.nsmem) == CUDA_SUCCESS;
+      if (m % 2 == 1 && v.shape.nstaged)
+        ok = ok && d.FuncSetAttribute(v.fn[m], CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES,
+                                      np_n > 1 ? v.shape.nsmem_p[p] : v.shape.nsmem) == CUDA_SUCCESS;
+    }
     if (!ok) {
-      for (int q = 0; q < nmod; ++q) d.ModuleUnload(v.module[q]);
+      for (int m : mods) d.ModuleUnload(v.module[m]);
       return fail(E3CONV_ERR_CUDA, "cannot reserve the backward kernels' shared memory");
     }
   }
@@ -259,7 +265,7 @@ int prepare_backward(Plan& pl) {
 }
 
 void release_backward(BwdVariant& v) {
-  for (int k = 0; k < 4; ++k)
+  for (int k = 0; k < 8; ++k)
     if (v.module[k]) driver().ModuleUnload(v.module[k]);
   v = BwdVariant{};
 }
@@ -550,8 +556,15 @@ int e3conv_set_option(e3conv_plan h, int option, int value) {
   if (option != E3CONV_OPT_CONTRACT_FIRST && option != E3CONV_OPT_TENSOR_CORES &&
       option != E3CONV_OPT_PATH_SPLIT && option != E3CONV_OPT_EDGE_VECTORS &&
       option != E3CONV_OPT_A_LAYOUT && option != E3CONV_OPT_COPY_GROUP &&
-      option != E3CONV_OPT_DIRECT_PIPELINE)
+      option != E3CONV_OPT_DIRECT_PIPELINE && option != E3CONV_OPT_BACKWARD_PARTS)
     return fail(E3CONV_ERR_UNSUPPORTED, "unknown option");
+  if (option == E3CONV_OPT_BACKWARD_PARTS) {  // backward kernels only: the forward stays
+    if (value != -1 && (value < 1 || value > 4)) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1 or 1 .. 4");
+    pl.req_bparts = value;
+    DeviceGuard g(pl.device);
+    for (auto& v : pl.bwd) release_backward(v);
+    return E3CONV_OK;
+  }
   if (option == E3CONV_OPT_DIRECT_PIPELINE) {
     if (value < -1 || value > 1) return fail(E3CONV_ERR_INVALID_ARG, "value must be -1, 0 or 1");
     pl.req_dpipe = value;
@@ -592,6 +605,7 @@ int e3conv_get_option(e3conv_plan h, int option, int* value) {
     case E3CONV_OPT_EDGE_VECTORS: *value = pl.req_vec; return E3CONV_OK;
     case E3CONV_OPT_A_LAYOUT: *value = pl.req_alayout; return E3CONV_OK;
     case E3CONV_OPT_COPY_GROUP: *value = pl.req_group; return E3CONV_OK;
+    case E3CONV_OPT_BACKWARD_PARTS: *value = pl.req_bparts; return E3CONV_OK;
     case E3CONV_OPT_DIRECT_PIPELINE: *value = pl.req_dpipe; return E3CONV_OK;
     default: return fail(E3CONV_ERR_UNSUPPORTED, "unknown option");
   }
@@ -1118,7 +1132,7 @@ int e3conv_backward(e3conv_plan h, const void* x, const void* Y, const void* s,
                     const_cast<int32_t**>(&senders), const_cast<int32_t**>(&row_ptr), &n32,
                     const_cast<float**>(&grad_out), &grad_sh, &grad_scalars, &inv_avg, &pl.status};
     for (int p = 0; p < b.eparts; ++p)
-      if (driver().LaunchKernel(bv.fn[p == 0 ? 0 : 2], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1,
+      if (driver().LaunchKernel(bv.fn[2 * p], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1,
                                 b.staged ? static_cast<unsigned>(b.esmem[p]) : 0u, st, args,
                                 nullptr) != CUDA_SUCCESS)
         return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed (backward, edges)");
@@ -1128,10 +1142,10 @@ int e3conv_backward(e3conv_plan h, const void* x, const void* Y, const void* s,
                     const_cast<int32_t**>(&receivers), const_cast<int32_t**>(&row_ptr),
                     const_cast<int32_t**>(&sender_row_ptr), const_cast<int32_t**>(&sender_perm),
                     &n32, const_cast<float**>(&grad_out), &grad_x, &inv_avg, &pl.status};
-    const bool nsplit = b.eparts > 1 && b.nstaged;
-    for (int p = 0; p < (nsplit ? 2 : 1); ++p)
-      if (driver().LaunchKernel(bv.fn[p == 0 ? 1 : 3], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1,
-                                b.nstaged ? static_cast<unsigned>(nsplit ? b.nsmem_p[p] : b.nsmem) : 0u,
+    const int nparts = b.nstaged ? b.eparts : 1;
+    for (int p = 0; p < nparts; ++p)
+      if (driver().LaunchKernel(bv.fn[2 * p + 1], static_cast<unsigned>(blocks), 1, 1, b.block, 1, 1,
+                                b.nstaged ? static_cast<unsigned>(nparts > 1 ? b.nsmem_p[p] : b.nsmem) : 0u,
                                 st, args, nullptr) != CUDA_SUCCESS)
         return fail(E3CONV_ERR_CUDA, "cuLaunchKernel failed (backward, nodes)");
   }
@@ -1139,7 +1153,7 @@ int e3conv_backward(e3conv_plan h, const void* x, const void* Y, const void* s,
 }
 
 int e3conv_backward_source(e3conv_plan h, int which, char* buf, size_t buf_len, size_t* needed) {
-  if (!h || which < 0 || which > 3) return fail(E3CONV_ERR_INVALID_ARG, "bad argument");
+  if (!h || which < 0 || which > 7) return fail(E3CONV_ERR_INVALID_ARG, "bad argument");
   DeviceGuard g(h->p.device);
   int rc = prepare_backward(h->p);
   if (rc != E3CONV_OK) return rc;

@@ -1959,9 +1959,14 @@ BwdShape choose_backward_shape(const Plan& pl, int dtype) {
   // only its outputs' gradient rows)
   b.eparts = 1;
   b.out_part.assign(pl.outputs.size(), 0);
-  b.esmem[0] = b.esmem[1] = b.smem;
-  b.nsmem_p[0] = b.nsmem_p[1] = b.nsmem;
-  if (b.staged && pl.nout * V > 64 && pl.outputs.size() > 1 && (pl.C * elem) % 16 == 0) {
+  for (int t = 0; t < 4; ++t) {
+    b.esmem[t] = b.smem;
+    b.nsmem_p[t] = b.nsmem;
+  }
+  // parts: as requested (E3CONV_OPT_BACKWARD_PARTS), else one per 64 registers of the row
+  int want = pl.req_bparts > 0 ? pl.req_bparts : (pl.nout * V + 63) / 64;
+  want = std::min<int>({want, 4, static_cast<int>(pl.outputs.size())});
+  if (b.staged && want > 1 && (pl.C * elem) % 16 == 0) {
     std::vector<std::pair<long long, int>> work;  // (terms, output irrep)
     for (size_t o = 0; o < pl.outputs.size(); ++o) {
       long long w = 0;
@@ -1974,15 +1979,15 @@ BwdShape choose_backward_shape(const Plan& pl, int dtype) {
       work.push_back({w, static_cast<int>(o)});
     }
     std::sort(work.begin(), work.end(), std::greater<std::pair<long long, int>>());
-    long long load[2] = {0, 0};
+    std::vector<long long> load(want, 0);
     for (const auto& wo : work) {
-      const int t = load[0] <= load[1] ? 0 : 1;
+      const int t = static_cast<int>(std::min_element(load.begin(), load.end()) - load.begin());
       b.out_part[wo.second] = t;
       load[t] += wo.first;
     }
-    if (load[0] > 0 && load[1] > 0) {
-      b.eparts = 2;
-      for (int t = 0; t < 2; ++t) {
+    if (*std::min_element(load.begin(), load.end()) > 0) {
+      b.eparts = want;
+      for (int t = 0; t < want; ++t) {
         int np = 0, nc = 0;
         for (const auto& P : pl.paths) np += b.out_part[P.o] == t;
         for (size_t o = 0; o < pl.outputs.size(); ++o)

@@ -109,21 +109,21 @@ struct BwdShape {
   // output irrep o, esmem[p] = its dynamic shared memory per block
   int eparts = 1;
   std::vector<int> out_part;
-  int esmem[2] = {0, 0};
-  int nsmem_p[2] = {0, 0};  // the staged nodes kernel's launches, likewise
+  int esmem[4] = {0, 0, 0, 0};
+  int nsmem_p[4] = {0, 0, 0, 0};  // the staged nodes kernel's launches, likewise
 };
 
 struct BwdVariant {
   bool compiled = false;
   BwdShape shape;
-  // 0 edges, 1 nodes, and where the kernels are split over the output irreps: 2 edges part 1,
-  // 3 nodes part 1
-  std::string source[4];
-  std::vector<char> cubin[4];
-  std::string log[4];
-  CUmodule module[4] = {nullptr, nullptr, nullptr, nullptr};
-  CUfunction fn[4] = {nullptr, nullptr, nullptr, nullptr};
-  int regs[4] = {-1, -1, -1, -1}, local_bytes[4] = {-1, -1, -1, -1};
+  // module 2 p + k: part p (of the split over the output irreps; part 0 when not split) of the
+  // edges (k = 0) or nodes (k = 1) kernel
+  std::string source[8];
+  std::vector<char> cubin[8];
+  std::string log[8];
+  CUmodule module[8] = {};
+  CUfunction fn[8] = {};
+  int regs[8] = {-1, -1, -1, -1, -1, -1, -1, -1}, local_bytes[8] = {-1, -1, -1, -1, -1, -1, -1, -1};
 };
 
 struct ShVariant {  // standalone harmonics kernel (compiled on first use)
@@ -205,6 +205,7 @@ struct Plan {
   int req_alayout = -1;                            // -1: automatic, else Shape::amode (channel pairs only)
   int req_vec = 0;                                 // 1: edges given as vectors, Y computed in the kernel
   int req_psplit = -1;                             // -1: automatic, 0/1: off, k: split a row's paths over k warps
+  int req_bparts = -1;                             // -1: automatic, else launches of each backward kernel (1..4)
   int tc_team_cap = 0;                             // > 0: at most this many tensor-core teams per block
   bool tc_fallback = false;                        // tensor cores requested but the kernel spills: float32 variant
   int device = -1;                 // -1: host-only plan

@@ -93,3 +93,25 @@ def test_backward_isolated_nodes_and_bad_indices(cuda_device):
                   sender_row_ptr=srp, sender_perm=sperm)
     assert not conv.check()
     assert conv.check()
+
+
+@pytest.mark.parametrize("parts", [1, 2, 3, 4])
+@pytest.mark.parametrize("name", ["large_f16", "mace"])
+def test_backward_split_over_output_irreps(cuda_device, name, parts):
+    # one to four launches of each backward kernel, each over a share of the output irreps;
+    # the later launches add to grad_Y and grad_x: every split meets the oracle
+    spec = SPECS[name]
+    g = make_graph(spec, 1200)
+    x, Y, s = workload_inputs(spec, g)
+    irreps = (spec.irreps_node, spec.irreps_sh, spec.irreps_out)
+    conv = e3.Conv(*irreps, g.avg_num_neighbors, dtype=spec.dtype)
+    conv.set_backward_parts(parts)
+    want = min(parts, len(conv.outputs))
+    assert f"// part 0 of {want}" in conv.backward_source(0)
+    pl = oracle.plan(*irreps)
+    gout = np.random.default_rng(parts).normal(size=(g.num_nodes, pl.nout, pl.C))
+    got = _run(conv, x, Y, s, g.senders, g.receivers, g.num_nodes, gout)
+    xs, Ys, ss = (np.asarray(a, np.float64) for a in (x, Y, s))
+    ref = oracle.backward(*irreps, xs, Ys, ss, g.senders, g.receivers, g.num_nodes,
+                          g.avg_num_neighbors, gout.astype(np.float32))
+    _check(got, ref, 1e-5)
