@@ -1963,8 +1963,10 @@ BwdShape choose_backward_shape(const Plan& pl, int dtype) {
     b.esmem[t] = b.smem;
     b.nsmem_p[t] = b.nsmem;
   }
-  // parts: as requested (E3CONV_OPT_BACKWARD_PARTS), else one per 64 registers of the row
-  int want = pl.req_bparts > 0 ? pl.req_bparts : (pl.nout * V + 63) / 64;
+  // parts: as requested (E3CONV_OPT_BACKWARD_PARTS), else one while a lane's row takes at most
+  // 64 registers and one per 44 beyond (measured on large_f16: 2 / 3 / 4 launches 69.8 / 63.5 /
+  // 66.9 ms; one launch is fastest for mace and large_f32)
+  int want = pl.req_bparts > 0 ? pl.req_bparts : pl.nout * V <= 64 ? 1 : (pl.nout * V + 43) / 44;
   want = std::min<int>({want, 4, static_cast<int>(pl.outputs.size())});
   if (b.staged && want > 1 && (pl.C * elem) % 16 == 0) {
     std::vector<std::pair<long long, int>> work;  // (terms, output irrep)

@@ -203,8 +203,9 @@ E3CONV_API int e3conv_set_launch_config(e3conv_plan plan, int channels_per_lane,
  *   backward kernels run as this many launches each, every launch over a
  *   share of the output irreps (balanced by their terms) that holds only its
  *   outputs' gradient rows and stages only its paths' scalars; the later
- *   launches add to the earlier ones' grad_Y and grad_x.  Automatic: one per
- *   64 registers of a lane's gradient row.  Affects e3conv_backward only. */
+ *   launches add to the earlier ones' grad_Y and grad_x.  Automatic: one
+ *   while a lane's gradient row takes at most 64 registers, else one per 44
+ *   of them.  Affects e3conv_backward only. */
 #define E3CONV_OPT_BACKWARD_PARTS 8
 E3CONV_API int e3conv_set_option(e3conv_plan plan, int option, int value);
 

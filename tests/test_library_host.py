@@ -467,15 +467,15 @@ def test_backward_kernels_generate_for_every_workload(name):
     s = SPECS[name]
     c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 10.0, dtype=s.dtype)
     edges, nodes = c.backward_source(0), c.backward_source(1)
-    if "// part 0 of 2" in edges:      # kernels split over the output irreps: both launches each
-        second = c.backward_source(2)
-        assert "// part 1 of 2" in second and "gY[le * " in second
-        edges += second
+    parts = int(re.search(r"// part 0 of (\d+)", edges).group(1)) if "// part 0 of" in edges else 1
+    for p in range(1, parts):          # kernels split over the output irreps: every launch
+        later = c.backward_source(2 * p)
+        assert f"// part {p} of {parts}" in later and "gY[le * " in later
+        edges += later
         if "cp.async" in nodes:
-            nodes += c.backward_source(3)
-    else:
-        with pytest.raises(e3.E3ConvError):
-            c.backward_source(2)
+            nodes += c.backward_source(2 * p + 1)
+    with pytest.raises(e3.E3ConvError):
+        c.backward_source(2 * parts)
     assert "e3conv_bwd_edges" in edges and "e3conv_bwd_nodes" in nodes
     # every CG nonzero appears once per channel of a lane in each kernel
     m = re.search(r"V=(\d+) TL=(\d+)", edges)
