@@ -506,3 +506,15 @@ def test_backward_rejects_edge_vector_plans_and_wide_channels():
     wide = e3.Conv("256x0e", "1x0e+1x1o", "256x0e+256x1o", 1.0)   # float32, C > 128
     with pytest.raises(e3.E3ConvError):
         wide.backward_source(0)
+
+
+def test_kernel_log_records_the_launch_shape_search():
+    # e3conv_kernel_log: one line per compile of the search, then the kept compile's log
+    s = SPECS["large_f16"]
+    c = e3.Conv(s.irreps_node, s.irreps_sh, s.irreps_out, 40.0, dtype=s.dtype)
+    log = c.kernel_log()
+    lines = [ln for ln in log.splitlines() if ln.startswith("compile: ")]
+    assert lines and all(re.search(r"block=\d+ V=\d+ team=\d+ stages=\d+ tc=\d regs=-?\d+ local=\d+", ln)
+                         for ln in lines)
+    info = c.kernel_info()
+    assert f"block={info['block_threads']}" in lines[-1]
