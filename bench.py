@@ -765,11 +765,15 @@ def time_next_rows(args, spec, g, conv, x, Y, s, senders, receivers, row_ptr, ou
         lin(flat, out=yl.view(N, -1))
         torch.cuda.synchronize()
         ms = _event_ms(lambda: lin(flat, out=yl.view(N, -1)), reps, stream)
+        kernel = "k_linear_tma" if lin.uses_tma else "k_linear"
+        lin.set_tma(False)                 # the row-per-thread kernel, for comparison
+        ms_rows = _event_ms(lambda: lin(flat, out=yl.view(N, -1)), reps, stream)
         assert lin.check()
         nbytes = 2 * out.numel() * 4
         flops = 3 * 2 * N * conv.nout * conv.C * conv.C
         res["irreps_linear"] = {
-            "kernel": "k_linear", "irreps": irreps, "ms": ms, "algorithmic_bytes": nbytes,
+            "kernel": kernel, "irreps": irreps, "ms": ms, "row_per_thread_kernel_ms": ms_rows,
+            "algorithmic_bytes": nbytes,
             "hbm_gbs": nbytes / (ms / 1e3) / 1e9, "hbm_frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
             "tensor_flops": flops, "tensor_tflops": flops / (ms / 1e3) / 1e12,
             "note": "x read and y written once (HBM bound); tensor FLOPs count the three "

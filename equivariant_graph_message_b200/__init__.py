@@ -89,6 +89,8 @@ _lin_query = _sig("e3conv_linear_query", ctypes.c_int, _vp, *([_c_int_p] * 5))
 _lin_set = _sig("e3conv_linear_set_weights", ctypes.c_int, _vp, _vp)
 _lin_forward = _sig("e3conv_linear_forward", ctypes.c_int, _vp, _vp, _i64, _vp, _vp)
 _lin_check = _sig("e3conv_linear_check", ctypes.c_int, _vp, _vp)
+_lin_uses_tma = _sig("e3conv_linear_uses_tma", ctypes.c_int, _vp, _c_int_p)
+_lin_set_tma = _sig("e3conv_linear_set_tma", ctypes.c_int, _vp, ctypes.c_int)
 _csr_ws = _sig("e3conv_csr_workspace_size", ctypes.c_int, _i64, _i64,
                ctypes.POINTER(ctypes.c_size_t))
 _build_csr = _sig("e3conv_build_csr", ctypes.c_int, _vp, _i64, _i64, _vp, _vp, _vp,
@@ -109,7 +111,8 @@ EXPORTED = ["e3conv_create", "e3conv_destroy", "e3conv_set_input_dtype",
             "e3conv_backward", "e3conv_prepare_backward", "e3conv_backward_source",
             "e3conv_set_radial_mlp", "e3conv_radial_scalars", "e3conv_linear_create",
             "e3conv_linear_destroy", "e3conv_linear_query", "e3conv_linear_set_weights",
-            "e3conv_linear_forward", "e3conv_linear_check", "e3conv_csr_workspace_size", "e3conv_build_csr",
+            "e3conv_linear_forward", "e3conv_linear_check", "e3conv_linear_uses_tma",
+            "e3conv_linear_set_tma", "e3conv_csr_workspace_size", "e3conv_build_csr",
             "e3conv_csr_check", "e3conv_build_csr_noalloc", "e3conv_csr_kernel_count", "e3conv_permute_rows", "e3conv_strerror", "e3conv_last_error",
             "e3conv_version"]
 
@@ -480,6 +483,18 @@ class IrrepsLinear:
         if h and _lin_destroy is not None:
             _lin_destroy(h)
             self._h = None
+
+    @property
+    def uses_tma(self) -> bool:
+        """True when the forward runs the tensor-map kernel (else the row-per-thread one)."""
+        t = ctypes.c_int()
+        _ok(_lin_uses_tma(self._h, ctypes.byref(t)), "e3conv_linear_uses_tma")
+        return bool(t.value)
+
+    def set_tma(self, enable: bool):
+        """False: always the row-per-thread kernel; True (default): the tensor-map kernel
+        where the shape allows it."""
+        _ok(_lin_set_tma(self._h, int(bool(enable))), "e3conv_linear_set_tma")
 
     def set_weights(self, weights):
         """weights: num_weight_blocks arrays [mul_in][mul_out] (host), matched irreps in

@@ -1000,6 +1000,19 @@ int e3conv_linear_query(e3conv_linear h, int* dim_in, int* dim_out, int* num_wei
   return E3CONV_OK;
 }
 
+int e3conv_linear_uses_tma(e3conv_linear h, int* uses_tma) {
+  if (!h || !uses_tma) return fail(E3CONV_ERR_INVALID_ARG, "NULL argument");
+  *uses_tma = linear_uses_tma(h->p) ? 1 : 0;
+  return E3CONV_OK;
+}
+
+int e3conv_linear_set_tma(e3conv_linear h, int enable) {
+  if (!h) return fail(E3CONV_ERR_INVALID_ARG, "linear is NULL");
+  if (enable != 0 && enable != 1) return fail(E3CONV_ERR_INVALID_ARG, "enable must be 0 or 1");
+  h->p.allow_tma = enable == 1;
+  return E3CONV_OK;
+}
+
 int e3conv_linear_set_weights(e3conv_linear h, const float* w) {
   if (!h || (!w && h->p.num_weight_blocks > 0)) return fail(E3CONV_ERR_INVALID_ARG, "NULL argument");
   LinearPlan& lp = h->p;
@@ -1040,7 +1053,8 @@ int e3conv_linear_forward(e3conv_linear h, const float* x, int64_t num_nodes, fl
     return fail(E3CONV_ERR_CUDA, "cannot query the SM count");
   std::string err;
   const int rc = linear_launch(lp, lp.d_w, x, num_nodes, y, lp.status, sms,
-                               reinterpret_cast<cudaStream_t>(stream), err);
+                               reinterpret_cast<cudaStream_t>(stream),
+                               driver().ok ? driver().TensorMapEncodeTiled : nullptr, err);
   return rc == E3CONV_OK ? rc : fail(rc, err);
 }
 

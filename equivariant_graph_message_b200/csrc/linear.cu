@@ -20,7 +20,9 @@
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <cmath>
+#include <cstring>
 #include <string>
 #include <vector>
 
@@ -204,6 +206,274 @@ __global__ void __launch_bounds__(128, 1) k_linear(LinArgs a) {
                  : "memory");
 }
 
+
+// ---- tensor-map variant: node-aligned tiles moved by TMA, warp roles, pipelined
+//
+// A tile of irrep block b holds nn = floor(128 / (2l+1)) whole nodes: rows (n, k) in order,
+// nn (2l+1) <= 128 of the MMA's 128 rows.  Its input rows are one 3-D box per 32 channels
+// ({32 channels, 2l+1, nn} of the [nodes][2l+1][mul_in] view, 128-byte swizzle), its output
+// one 3-D box per 32 output channels, stored from a swizzled staging tile.  Nodes past the
+// end are zero-filled on load and clipped on store.  Warps 0-3 (thread t <-> row t <->
+// tensor-memory lane t) split the landed rows into the float16 hi / lo operand, then read
+// out the previous tile's accumulator (double-buffered in tensor memory) into the staging
+// tile; warp 4 issues the loads into a ring of raw stages; warp 5 fetches the weights when
+// the irrep changes and issues the MMAs.
+
+constexpr int kChunkBytes = kTile * 128;  // 128 rows x 32 float32: one box of a stage
+constexpr int kTmaMaxBlocks = 8;
+
+struct LinTmaBlock {
+  int dim, nn, first_tile, out_off;
+  long long w_off;  // byte offset of the packed weights; -1: zeros
+  float scale;
+};
+
+struct LinTmaArgs {
+  CUtensorMap in_map[kTmaMaxBlocks];   // {mul_in, 2l+1, nodes} of x at the matched input irrep
+  CUtensorMap out_map[kTmaMaxBlocks];  // {mul_out, 2l+1, nodes} of y at the output irrep
+  LinTmaBlock blk[kTmaMaxBlocks];
+  float* y;
+  const unsigned char* w;
+  long long nodes;
+  int dim_out, n_out, nblocks, tiles_total, stages;
+  unsigned tmem_half;  // tensor-memory columns of one accumulator buffer (power of two >= mul_out)
+  unsigned* status;
+};
+
+struct LinTmaLayout {
+  size_t raw, stg, act, bw, bars, total;  // offsets from the 1024-byte aligned base; total size
+};
+
+__host__ __device__ inline LinTmaLayout lin_tma_layout(int K, int N, int stages) {
+  LinTmaLayout L;
+  L.raw = 0;
+  L.stg = L.raw + static_cast<size_t>(stages) * (K / 32) * kChunkBytes;
+  L.act = L.stg + 2 * static_cast<size_t>(kChunkBytes);
+  L.bw = L.act + 2 * static_cast<size_t>(kTile) * K * 2;
+  L.bars = L.bw + 2 * static_cast<size_t>(N) * K * 2;
+  L.total = L.bars + 8 * (2 * 4 + 8) + 1024;  // barriers, and room to align the base
+  return L;
+}
+
+template <int K>
+__global__ void __launch_bounds__(192, 1) k_linear_tma(const __grid_constant__ LinTmaArgs a) {
+  extern __shared__ __align__(1024) unsigned char sm_raw[];
+  unsigned char* sm = sm_raw + ((1024 - (smem_u32(sm_raw) & 1023)) & 1023);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int N = a.n_out, RS = a.stages;
+  const LinTmaLayout L = lin_tma_layout(K, N, RS);
+  unsigned char* raw = sm + L.raw;
+  unsigned char* stg = sm + L.stg;
+  unsigned char* act = sm + L.act;
+  unsigned char* bw = sm + L.bw;
+  unsigned long long* bars = reinterpret_cast<unsigned long long*>(sm + L.bars);
+  unsigned long long* raw_full = bars;       // [4]
+  unsigned long long* raw_empty = bars + 4;  // [4]
+  unsigned long long* act_full = bars + 8;
+  unsigned long long* act_empty = bars + 9;
+  unsigned long long* mma_done = bars + 10;  // [2]
+  unsigned long long* tm_empty = bars + 12;  // [2]
+  unsigned long long* bar_w = bars + 14;
+  unsigned* tslot = reinterpret_cast<unsigned*>(bars + 15);
+  if (tid == 0) {
+    for (int s = 0; s < RS; ++s) {
+      mbar_init(raw_full + s, 1);
+      mbar_init(raw_empty + s, 4);
+    }
+    mbar_init(act_full, 4);
+    mbar_init(act_empty, 1);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(mma_done + q, 1);
+      mbar_init(tm_empty + q, 4);
+    }
+    mbar_init(bar_w, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tslot)), "r"(2 * a.tmem_half)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_before();
+  __syncthreads();
+  tc_after();
+  const unsigned tmem = *tslot;
+  const long long per = (a.tiles_total + gridDim.x - 1) / gridDim.x;
+  const long long t0 = blockIdx.x * per;
+  const long long t1 = (t0 + per < a.tiles_total) ? t0 + per : static_cast<long long>(a.tiles_total);
+  auto block_of = [&](long long t) {
+    int b = 0;
+    while (b + 1 < a.nblocks && t >= a.blk[b + 1].first_tile) ++b;
+    return b;
+  };
+  bool ok = true;
+
+  if (warp == 4) {  // ---- loads
+    int mj = 0;
+    if (lane == 0) {
+      for (long long t = t0; t < t1 && ok; ++t) {
+        const int b = block_of(t);
+        const LinTmaBlock& B = a.blk[b];
+        if (B.w_off < 0) continue;
+        const int s = mj % RS;
+        if (mj >= RS) ok = mbar_wait(raw_empty + s, ((mj / RS) - 1) & 1);
+        if (!ok) break;
+        const int node0 = static_cast<int>((t - B.first_tile) * B.nn);
+        mbar_expect(raw_full + s, static_cast<unsigned>((K / 32) * 128 * B.dim * B.nn));
+        for (int c = 0; c < K / 32; ++c)
+          tma_load_3d(raw + (static_cast<size_t>(s) * (K / 32) + c) * kChunkBytes, &a.in_map[b], raw_full + s,
+                      32 * c, 0, node0);
+        ++mj;
+      }
+      // no load outlives the block: wait for the last ones to land (already seen by the rows)
+      for (int q = (mj > RS ? mj - RS : 0); q < mj; ++q) mbar_wait(raw_full + q % RS, (q / RS) & 1);
+      if (!ok) atomicOr(a.status, 4u);
+    }
+  } else if (warp == 5) {  // ---- weights and MMAs
+    int mj = 0;
+    if (lane == 0) {
+      int cur = -1;
+      unsigned ph_w = 0;
+      const unsigned id = idesc_f16(kTile, N);
+      for (long long t = t0; t < t1 && ok; ++t) {
+        const int b = block_of(t);
+        const LinTmaBlock& B = a.blk[b];
+        if (B.w_off < 0) continue;
+        if (b != cur) {  // every MMA on the previous weights has completed before they are replaced
+          if (mj > 0) ok = mbar_wait(mma_done + ((mj - 1) & 1), ((mj - 1) >> 1) & 1);
+          if (!ok) break;
+          const unsigned bytes = static_cast<unsigned>(2 * N * K * 2);
+          mbar_expect(bar_w, bytes);
+          bulk_g2s(bw, a.w + B.w_off, bytes, bar_w);
+          ok = mbar_wait(bar_w, ph_w);
+          if (!ok) break;
+          ph_w ^= 1u;
+          cur = b;
+        }
+        ok = mbar_wait(act_full, mj & 1);
+        if (ok && mj >= 2) ok = mbar_wait(tm_empty + (mj & 1), ((mj - 2) >> 1) & 1);
+        if (!ok) break;
+        tc_after();
+        const unsigned d = tmem + (mj & 1) * a.tmem_half;
+        const unsigned char* whi = bw;
+        const unsigned char* wlo = bw + N * K * 2;
+        const unsigned char* ahi = act;
+        const unsigned char* alo = act + kTile * K * 2;
+        for (int ks = 0; ks < K / 16; ++ks) {
+          const int ao = ks * kTile * 32, bo = ks * N * 32;
+          mma_f16(d, kmajor_desc(ahi + ao), kmajor_desc(whi + bo), id, ks > 0);
+          mma_f16(d, kmajor_desc(ahi + ao), kmajor_desc(wlo + bo), id, 1);
+          mma_f16(d, kmajor_desc(alo + ao), kmajor_desc(whi + bo), id, 1);
+        }
+        mma_commit(mma_done + (mj & 1));
+        mma_commit(act_empty);
+        ++mj;
+      }
+      if (mj > 0) {  // nothing in flight at exit: both commits of the last tile have arrived
+        mbar_wait(mma_done + ((mj - 1) & 1), ((mj - 1) >> 1) & 1);
+        mbar_wait(act_empty, (mj - 1) & 1);
+      }
+      if (!ok) atomicOr(a.status, 4u);
+    }
+  } else {  // ---- warps 0-3: operand rows, then the previous tile's output
+    const unsigned lane_off = static_cast<unsigned>(32 * warp) << 16;
+    // the 128 row threads agree on every wait's outcome, so they leave the loop together
+    auto team_and = [](bool p) {
+      unsigned r;
+      asm volatile(
+          "{ .reg .pred q, o; setp.ne.u32 q, %1, 0; bar.red.and.pred o, 1, 128, q; selp.u32 %0, 1, 0, o; }"
+          : "=r"(r)
+          : "r"(static_cast<unsigned>(p))
+          : "memory");
+      return r != 0;
+    };
+    int mj = 0, chunk = 0;
+    float R[K];
+    // the output of MMA tile q (block b, first node node0) through the staging tiles
+    auto drain = [&](int q, int b, int node0) {
+      const LinTmaBlock& B = a.blk[b];
+      ok = team_and(ok && mbar_wait(mma_done + (q & 1), (q >> 1) & 1));
+      tc_after();
+      for (int j0 = 0; j0 < N && ok; j0 += 32) {
+        float v[32];
+        tmem_ld32(tmem + (q & 1) * a.tmem_half + lane_off + j0, v);
+        if (j0 + 32 >= N) {  // the accumulator is read: free it for the tile after next
+          tc_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tm_empty + (q & 1));
+        }
+        unsigned char* st = stg + (chunk & 1) * kChunkBytes;
+        if (tid == 0) bulk_wait_read_but1();  // the store issued from this staging tile has read it
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<float4*>(st + tid * 128 + ((i ^ (tid & 7)) << 4)) =
+              make_float4(v[4 * i] * B.scale, v[4 * i + 1] * B.scale, v[4 * i + 2] * B.scale,
+                          v[4 * i + 3] * B.scale);
+        fence_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (tid == 0) {
+          tma_store_3d(&a.out_map[b], st, j0, 0, node0);
+          bulk_commit();
+        }
+        ++chunk;
+      }
+    };
+    int pb = -1, pnode = 0;  // the MMA tile whose output is pending
+    for (long long t = t0; t < t1 && ok; ++t) {
+      const int b = block_of(t);
+      const LinTmaBlock& B = a.blk[b];
+      const int node0 = static_cast<int>((t - B.first_tile) * B.nn);
+      if (B.w_off < 0) {  // output irrep without a matching input irrep: zeros
+        const int n = node0 + tid / B.dim;
+        if (tid < B.dim * B.nn && n < a.nodes) {
+          float* dst = a.y + static_cast<long long>(n) * a.dim_out + B.out_off + (tid % B.dim) * N;
+          for (int q = 0; q < N; q += 4) *reinterpret_cast<float4*>(dst + q) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        continue;
+      }
+      const int s = mj % RS;
+      ok = team_and(mbar_wait(raw_full + s, (mj / RS) & 1));
+      if (!ok) break;
+      const bool live = tid < B.dim * B.nn;
+#pragma unroll
+      for (int c = 0; c < K / 32; ++c) {
+        const unsigned char* src = raw + (static_cast<size_t>(s) * (K / 32) + c) * kChunkBytes + tid * 128;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 v = live ? *reinterpret_cast<const float4*>(src + ((i ^ (tid & 7)) << 4))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+          R[32 * c + 4 * i] = v.x;
+          R[32 * c + 4 * i + 1] = v.y;
+          R[32 * c + 4 * i + 2] = v.z;
+          R[32 * c + 4 * i + 3] = v.w;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(raw_empty + s);  // the stage may be refilled
+      ok = team_and(mj == 0 || mbar_wait(act_empty, (mj - 1) & 1));  // the previous MMAs read the operand
+      if (!ok) break;
+      store_split_row<K>(act, act + kTile * K * 2, tid, R, kTile);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(act_full);
+      if (pb >= 0) drain(mj - 1, pb, pnode);  // overlaps this tile's MMAs
+      pb = b;
+      pnode = node0;
+      ++mj;
+    }
+    if (ok && pb >= 0) drain(mj - 1, pb, pnode);
+    if (tid == 0) bulk_wait_all();
+    if (!ok && tid == 0) atomicOr(a.status, 4u);
+  }
+  tc_before();
+  __syncthreads();
+  tc_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * a.tmem_half)
+                 : "memory");
+}
 }  // namespace
 
 int linear_prepare(LinearPlan& lp, const std::vector<Irrep>& in, const std::vector<Irrep>& out,
@@ -301,9 +571,104 @@ size_t linear_smem_bytes(const LinearPlan& lp) {
   return 2 * static_cast<size_t>(lp.N) * lp.K * 2 + 2 * static_cast<size_t>(kTile) * lp.K * 2 + 64;
 }
 
+// raw stages of the tensor-map kernel that fit in shared memory next to the rest (0: none)
+static int linear_tma_stages(const LinearPlan& lp) {
+  int s = 0;
+  while (s < 4 && lin_tma_layout(lp.K, lp.N, s + 1).total <= 227 * 1024) ++s;
+  return s;
+}
+
+bool linear_uses_tma(const LinearPlan& lp) {
+  if (!lp.allow_tma || lp.N % 32 != 0 || static_cast<int>(lp.blocks.size()) > kTmaMaxBlocks) return false;
+  for (const LinBlock& b : lp.blocks)
+    if (b.dim > kTile) return false;
+  return linear_tma_stages(lp) >= 1;
+}
+
+static int linear_launch_tma(const LinearPlan& lp, const void* dev_w, const float* x, long long nodes,
+                             float* y, unsigned* status, int grid, cudaStream_t st,
+                             TensorMapEncodeFn encode, std::string& err) {
+  LinTmaArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.y = y;
+  a.w = static_cast<const unsigned char*>(dev_w);
+  a.nodes = nodes;
+  a.dim_out = lp.dim_out;
+  a.n_out = lp.N;
+  a.nblocks = static_cast<int>(lp.blocks.size());
+  a.status = status;
+  a.stages = linear_tma_stages(lp);
+  a.tmem_half = 32;
+  while (a.tmem_half < static_cast<unsigned>(lp.N)) a.tmem_half *= 2;
+  const size_t wbytes = 2 * static_cast<size_t>(lp.N) * lp.K * 2;
+  long long tiles = 0, mma_tiles = 0;
+  for (size_t q = 0; q < lp.blocks.size(); ++q) {
+    const LinBlock& b = lp.blocks[q];
+    LinTmaBlock& B = a.blk[q];
+    B.dim = b.dim;
+    B.nn = kTile / b.dim;
+    B.first_tile = static_cast<int>(tiles);
+    B.out_off = b.out_off;
+    B.w_off = b.w_off >= 0 ? static_cast<long long>(wbytes) * b.w_off : -1;
+    B.scale = b.scale;
+    const long long nt = (nodes + B.nn - 1) / B.nn;
+    tiles += nt;
+    if (b.w_off >= 0) mma_tiles += nt;
+    if (tiles >= (1ll << 31)) {
+      err = "too many rows";
+      return E3CONV_ERR_UNSUPPORTED;
+    }
+    // y viewed as [nodes][2l+1][mul_out] at the irrep; x as [nodes][2l+1][mul_in] at the match
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const cuuint64_t ostr[2] = {static_cast<cuuint64_t>(lp.N) * 4, static_cast<cuuint64_t>(lp.dim_out) * 4};
+    const cuuint64_t odim[3] = {static_cast<cuuint64_t>(lp.N), static_cast<cuuint64_t>(b.dim),
+                                static_cast<cuuint64_t>(nodes)};
+    const cuuint32_t obox[3] = {32, static_cast<cuuint32_t>(b.dim), static_cast<cuuint32_t>(B.nn)};
+    if (encode(&a.out_map[q], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, y + b.out_off, odim, ostr, obox, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+      err = "cuTensorMapEncodeTiled failed for the linear output";
+      return E3CONV_ERR_CUDA;
+    }
+    if (b.w_off >= 0) {
+      const cuuint64_t istr[2] = {static_cast<cuuint64_t>(lp.K) * 4, static_cast<cuuint64_t>(lp.dim_in) * 4};
+      const cuuint64_t idim[3] = {static_cast<cuuint64_t>(lp.K), static_cast<cuuint64_t>(b.dim),
+                                  static_cast<cuuint64_t>(nodes)};
+      if (encode(&a.in_map[q], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(x) + b.in_off, idim,
+                 istr, obox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+        err = "cuTensorMapEncodeTiled failed for the linear input";
+        return E3CONV_ERR_CUDA;
+      }
+    }
+  }
+  a.tiles_total = static_cast<int>(tiles);
+  const size_t smem = lin_tma_layout(lp.K, lp.N, a.stages).total;
+  // one CTA per SM (shared memory); as many as there are tiles, at most one per SM
+  const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, grid));
+  auto launch = [&](auto kernel) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kernel<<<blocks, 192, smem, st>>>(a);
+    return cudaGetLastError();
+  };
+  (void)mma_tiles;
+  cudaError_t e = lp.K == 32 ? launch(k_linear_tma<32>) : lp.K == 64 ? launch(k_linear_tma<64>)
+                                                                      : launch(k_linear_tma<128>);
+  if (e != cudaSuccess) {
+    err = "irreps linear kernel launch failed";
+    return E3CONV_ERR_CUDA;
+  }
+  return E3CONV_OK;
+}
+
 int linear_launch(const LinearPlan& lp, const void* dev_w, const float* x, long long nodes, float* y,
-                  unsigned* status, int grid, cudaStream_t st, std::string& err) {
+                  unsigned* status, int grid, cudaStream_t st, TensorMapEncodeFn encode,
+                  std::string& err) {
   if (nodes == 0) return E3CONV_OK;
+  if (encode && linear_uses_tma(lp))
+    return linear_launch_tma(lp, dev_w, x, nodes, y, status, grid, st, encode, err);
   LinArgs a{};
   a.x = x;
   a.y = y;

@@ -183,6 +183,7 @@ struct LinearPlan {
   std::vector<unsigned char> packed;
   int scale_exp = 0;
   bool weights_set = false;
+  bool allow_tma = true;            // the tensor-map kernel where the shape allows it
   int device = -1;
   void* d_w = nullptr;
   unsigned* status = nullptr;
@@ -241,8 +242,16 @@ int linear_prepare(LinearPlan& lp, const std::vector<Irrep>& in, const std::vect
                    double scale, std::string& err);
 int linear_pack(LinearPlan& lp, const float* w, std::string& err);
 size_t linear_smem_bytes(const LinearPlan& lp);
+// cuTensorMapEncodeTiled, resolved by the caller through the runtime (nullptr: no tensor maps)
+using TensorMapEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                       const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                       const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                       CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 int linear_launch(const LinearPlan& lp, const void* dev_w, const float* x, long long nodes, float* y,
-                  unsigned* status, int grid, cudaStream_t st, std::string& err);
+                  unsigned* status, int grid, cudaStream_t st, TensorMapEncodeFn encode,
+                  std::string& err);
+// whether linear_launch runs the tensor-map kernel for this layer (given an encoder)
+bool linear_uses_tma(const LinearPlan& lp);
 
 // codegen.cpp
 std::vector<AEntry> build_a_entries(const Plan& plan);

@@ -65,6 +65,30 @@ __device__ __forceinline__ void tma_store_2d(const void* map, const void* src, i
       "r"(smem_u32(src)), "r"(x), "r"(y)
       : "memory");
 }
+// 3-D TMA tensor load of one box into shared memory at coordinates (x inner, y, z); completes
+// `bytes` of transaction on the mbarrier
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* map, unsigned long long* bar, int x,
+                                            int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+// 3-D TMA tensor store of one box from shared memory, in this thread's bulk async-group
+__device__ __forceinline__ void tma_store_3d(const void* map, const void* src, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+      "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+// all but the most recent of this thread's bulk groups have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_but1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(unsigned long long* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -143,35 +167,52 @@ __device__ __forceinline__ unsigned pack_half2(float lo, float hi) {
   return r;
 }
 
-// Writes row r's values v[0..K) of a K-major operand as float16 hi and lo parts.
+// hi and lo float16 parts of v[0..8), packed as two 16-byte vectors
+__device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
+  unsigned h[4], l[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __half h0 = __float2half_rn(v[2 * q]), h1 = __float2half_rn(v[2 * q + 1]);
+    const __half l0 = __float2half_rn(v[2 * q] - __half2float(h0));
+    const __half l1 = __float2half_rn(v[2 * q + 1] - __half2float(h1));
+    const __half2 hh = __halves2half2(h0, h1), ll = __halves2half2(l0, l1);
+    h[q] = *reinterpret_cast<const unsigned*>(&hh);
+    l[q] = *reinterpret_cast<const unsigned*>(&ll);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Writes row r's values v[0..K) of a K-major operand as float16 hi and lo parts: eight
+// K-consecutive values are one 16-byte row of a core matrix, so a warp's 32 rows store
+// 4 x 128 contiguous bytes per instruction.
 template <int K>
 __device__ __forceinline__ void store_split_row(unsigned char* hi, unsigned char* lo, int r,
                                                 const float* v, int rows) {
+  static_assert(K % 8 == 0, "K must be a multiple of 8");
 #pragma unroll
-  for (int k = 0; k < K; k += 2) {
-    const __half h0 = __float2half_rn(v[k]), h1 = __float2half_rn(v[k + 1]);
-    const __half l0 = __float2half_rn(v[k] - __half2float(h0));
-    const __half l1 = __float2half_rn(v[k + 1] - __half2float(h1));
+  for (int k = 0; k < K; k += 8) {
+    uint4 h, l;
+    split8(v + k, h, l);
     const int off = kmajor_off(r, k, rows);
-    *reinterpret_cast<__half2*>(hi + off) = __halves2half2(h0, h1);
-    *reinterpret_cast<__half2*>(lo + off) = __halves2half2(l0, l1);
+    *reinterpret_cast<uint4*>(hi + off) = h;
+    *reinterpret_cast<uint4*>(lo + off) = l;
   }
 }
-
 
 // Writes values v[0..N) of row r at K columns k0 .. k0 + N - 1 (k0 a multiple of 16) of a
 // K-major operand as float16 hi and lo parts.
 template <int N>
 __device__ __forceinline__ void store_split_part(unsigned char* hi, unsigned char* lo, int r,
                                                  const float* v, int rows, int k0) {
+  static_assert(N % 8 == 0, "N must be a multiple of 8");
 #pragma unroll
-  for (int k = 0; k < N; k += 2) {
-    const __half h0 = __float2half_rn(v[k]), h1 = __float2half_rn(v[k + 1]);
-    const __half l0 = __float2half_rn(v[k] - __half2float(h0));
-    const __half l1 = __float2half_rn(v[k + 1] - __half2float(h1));
+  for (int k = 0; k < N; k += 8) {
+    uint4 h, l;
+    split8(v + k, h, l);
     const int off = kmajor_off(r, k0 + k, rows);
-    *reinterpret_cast<__half2*>(hi + off) = __halves2half2(h0, h1);
-    *reinterpret_cast<__half2*>(lo + off) = __halves2half2(l0, l1);
+    *reinterpret_cast<uint4*>(hi + off) = h;
+    *reinterpret_cast<uint4*>(lo + off) = l;
   }
 }
 

@@ -1,7 +1,8 @@
 """GPU parity of the irreps linear layer on the tensor cores (e3conv_linear_*)
-against the oracle's float64 layer: the convolution's output irreps mixed into
-other multiplicities, unmatched output irreps, ragged row tiles, few nodes, and
-the convolution's full-size output of the large mixed-precision workload."""
+against the oracle's float64 layer, for both kernels (tensor-map tiles and
+row-per-thread): the convolution's output irreps mixed into other
+multiplicities, unmatched output irreps, ragged row tiles, few nodes, and the
+convolution's full-size output of the large mixed-precision workload."""
 import numpy as np
 import pytest
 import torch
@@ -13,16 +14,24 @@ from parity import to_dev
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("ins,outs", [
-    ("128x0e+128x1o+128x2e+128x3o", "64x0e+64x1o+64x2e+64x3o"),
-    ("64x0e+64x1o+64x2e", "128x0e+128x1e+128x1o+128x2e+128x3o"),     # unmatched 1e, 3o
-    ("32x0e+32x1o", "256x1o+256x0e"),
-    ("128x0e+128x1o+128x2e+128x3o", "16x3o+16x0e"),
-    ("128x0e+128x1o", "256x0e+256x1o"),                               # one staging buffer
-])
+# (irreps_in, irreps_out, whether the tensor-map kernel takes the shape)
+SHAPES = [
+    ("128x0e+128x1o+128x2e+128x3o", "64x0e+64x1o+64x2e+64x3o", True),
+    ("64x0e+64x1o+64x2e", "128x0e+128x1e+128x1o+128x2e+128x3o", True),     # unmatched 1e, 3o
+    ("32x0e+32x1o", "256x1o+256x0e", True),
+    ("128x0e+128x1o+128x2e+128x3o", "16x3o+16x0e", False),                  # mul_out 16
+    ("128x0e+128x1o", "256x0e+256x1o", False),                              # no room for a stage
+    ("64x0e+64x1o+64x2e+64x3o+64x4e+64x5o+64x6e", "96x6e+96x0e+96x4e+96x5o", True),  # 13 rows a node
+]
+
+
+@pytest.mark.parametrize("tma", [True, False])
+@pytest.mark.parametrize("ins,outs,fits", SHAPES)
 @pytest.mark.parametrize("nodes", [1, 5, 300, 2049])
-def test_linear_matches_the_oracle(cuda_device, ins, outs, nodes):
+def test_linear_matches_the_oracle(cuda_device, ins, outs, fits, nodes, tma):
     lin = e3.IrrepsLinear(ins, outs, 0.7)
+    lin.set_tma(tma)
+    assert lin.uses_tma == (tma and fits)
     rng = np.random.default_rng(nodes + len(ins))
     ws = [rng.normal(size=(lin.mul_in, lin.mul_out)).astype(np.float32)
           for _ in range(lin.num_weight_blocks)]
@@ -54,13 +63,19 @@ def test_linear_on_the_convolution_output_full_size(cuda_device):
     rng = np.random.default_rng(5)
     ws = [rng.normal(size=(128, 128)).astype(np.float32) for _ in range(lin.num_weight_blocks)]
     lin.set_weights(ws)
+    assert lin.uses_tma
     y = lin(out.view(w.N, -1))
+    lin.set_tma(False)
+    y_rows = lin(out.view(w.N, -1))       # the row-per-thread kernel on the same input
     torch.cuda.synchronize()
     assert lin.check()
+    # both kernels form the same three float16 products per term and accumulate them in
+    # float32 on the tensor cores in the same order: the same results
+    assert torch.equal(y, y_rows)
     rows = np.unique(np.concatenate([[0, w.N - 1], rng.choice(w.N, 512, replace=False)]))
     xr = out.view(w.N, -1)[torch.from_numpy(rows).cuda()].cpu().numpy()
     ref = oracle.irreps_linear(conv_irreps, conv_irreps, 1.0, xr, ws)
     got = y[torch.from_numpy(rows).cuda()].cpu().numpy()
     assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
-    del w, out, y
+    del w, out, y, y_rows
     torch.cuda.empty_cache()
