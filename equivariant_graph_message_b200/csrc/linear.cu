@@ -211,16 +211,22 @@ __global__ void __launch_bounds__(128, 1) k_linear(LinArgs a) {
 //
 // A tile of irrep block b holds nn = floor(128 / (2l+1)) whole nodes: rows (n, k) in order,
 // nn (2l+1) <= 128 of the MMA's 128 rows.  Its input rows are one 3-D box per 32 channels
-// ({32 channels, 2l+1, nn} of the [nodes][2l+1][mul_in] view, 128-byte swizzle), its output
-// one 3-D box per 32 output channels, stored from a swizzled staging tile.  Nodes past the
-// end are zero-filled on load and clipped on store.  Warps 0-3 (thread t <-> row t <->
-// tensor-memory lane t) split the landed rows into the float16 hi / lo operand, then read
-// out the previous tile's accumulator (double-buffered in tensor memory) into the staging
-// tile; warp 4 issues the loads into a ring of raw stages; warp 5 fetches the weights when
-// the irrep changes and issues the MMAs.
+// ({32 channels, 2l+1, nn} of the [nodes][2l+1][mul_in] view, 128-byte swizzle) into a stage
+// of a ring; its output one 3-D box per 32 output channels, stored from a swizzled staging
+// tile.  Nodes past the end are zero-filled on load and clipped on store.  Roles:
+//   warp 12       issues the loads of a stage once the MMAs have released it;
+//   warps 4-11    (256 threads: row r, half h of its channels) read the landed float32 rows,
+//                 then overwrite the same stage with their float16 hi / lo operand (the
+//                 128 x mul_in float32 tile and its two float16 parts take the same bytes);
+//   warp 13       fetches the irrep's weights when it changes, issues the MMAs of a stage into
+//                 one of two tensor-memory accumulators and releases the stage;
+//   warps 0-3     (thread t <-> row t <-> tensor-memory lane t) read an accumulator out into
+//                 the staging tiles and store them; they also write the zero tiles.
 
 constexpr int kChunkBytes = kTile * 128;  // 128 rows x 32 float32: one box of a stage
 constexpr int kTmaMaxBlocks = 8;
+constexpr int kTmaMaxStages = 6;
+constexpr int kTmaThreads = 448;
 
 struct LinTmaBlock {
   int dim, nn, first_tile, out_off;
@@ -241,47 +247,43 @@ struct LinTmaArgs {
 };
 
 struct LinTmaLayout {
-  size_t raw, stg, act, bw, bars, total;  // offsets from the 1024-byte aligned base; total size
+  size_t stage, stg, bw, bars, total;  // offsets from the 1024-byte aligned base; total size
 };
 
 __host__ __device__ inline LinTmaLayout lin_tma_layout(int K, int N, int stages) {
   LinTmaLayout L;
-  L.raw = 0;
-  L.stg = L.raw + static_cast<size_t>(stages) * (K / 32) * kChunkBytes;
-  L.act = L.stg + 2 * static_cast<size_t>(kChunkBytes);
-  L.bw = L.act + 2 * static_cast<size_t>(kTile) * K * 2;
+  L.stage = static_cast<size_t>(K / 32) * kChunkBytes;  // = 128 x K x (2 + 2) operand bytes
+  L.stg = static_cast<size_t>(stages) * L.stage;
+  L.bw = L.stg + 2 * static_cast<size_t>(kChunkBytes);
   L.bars = L.bw + 2 * static_cast<size_t>(N) * K * 2;
-  L.total = L.bars + 8 * (2 * 4 + 8) + 1024;  // barriers, and room to align the base
+  L.total = L.bars + 8 * 32 + 1024;  // barriers, and room to align the base
   return L;
 }
 
 template <int K>
-__global__ void __launch_bounds__(192, 1) k_linear_tma(const __grid_constant__ LinTmaArgs a) {
+__global__ void __launch_bounds__(kTmaThreads, 1) k_linear_tma(const __grid_constant__ LinTmaArgs a) {
   extern __shared__ __align__(1024) unsigned char sm_raw[];
   unsigned char* sm = sm_raw + ((1024 - (smem_u32(sm_raw) & 1023)) & 1023);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int N = a.n_out, RS = a.stages;
   const LinTmaLayout L = lin_tma_layout(K, N, RS);
-  unsigned char* raw = sm + L.raw;
   unsigned char* stg = sm + L.stg;
-  unsigned char* act = sm + L.act;
   unsigned char* bw = sm + L.bw;
   unsigned long long* bars = reinterpret_cast<unsigned long long*>(sm + L.bars);
-  unsigned long long* raw_full = bars;       // [4]
-  unsigned long long* raw_empty = bars + 4;  // [4]
-  unsigned long long* act_full = bars + 8;
-  unsigned long long* act_empty = bars + 9;
-  unsigned long long* mma_done = bars + 10;  // [2]
-  unsigned long long* tm_empty = bars + 12;  // [2]
-  unsigned long long* bar_w = bars + 14;
-  unsigned* tslot = reinterpret_cast<unsigned*>(bars + 15);
+  unsigned long long* st_full = bars;                       // [RS] loads landed
+  unsigned long long* st_empty = bars + kTmaMaxStages;      // [RS] MMAs done with the stage
+  unsigned long long* op_full = bars + 2 * kTmaMaxStages;   // [RS] operand written
+  unsigned long long* mma_done = bars + 3 * kTmaMaxStages;  // [2]
+  unsigned long long* tm_empty = mma_done + 2;              // [2]
+  unsigned long long* bar_w = mma_done + 4;
+  unsigned* tslot = reinterpret_cast<unsigned*>(mma_done + 5);
+  auto stage = [&](int s) { return sm + static_cast<size_t>(s) * L.stage; };
   if (tid == 0) {
     for (int s = 0; s < RS; ++s) {
-      mbar_init(raw_full + s, 1);
-      mbar_init(raw_empty + s, 4);
+      mbar_init(st_full + s, 1);
+      mbar_init(st_empty + s, 1);
+      mbar_init(op_full + s, 8);
     }
-    mbar_init(act_full, 4);
-    mbar_init(act_empty, 1);
     for (int q = 0; q < 2; ++q) {
       mbar_init(mma_done + q, 1);
       mbar_init(tm_empty + q, 4);
@@ -307,33 +309,41 @@ __global__ void __launch_bounds__(192, 1) k_linear_tma(const __grid_constant__ L
     while (b + 1 < a.nblocks && t >= a.blk[b + 1].first_tile) ++b;
     return b;
   };
+  // a named barrier of `count` threads that also ANDs a predicate over them
+  auto team_and = [](int id, int count, bool p) {
+    unsigned r;
+    asm volatile(
+        "{ .reg .pred q, o; setp.ne.u32 q, %1, 0; bar.red.and.pred o, %2, %3, q; selp.u32 %0, 1, 0, o; }"
+        : "=r"(r)
+        : "r"(static_cast<unsigned>(p)), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+  };
   bool ok = true;
 
-  if (warp == 4) {  // ---- loads
-    int mj = 0;
+  if (warp == 12) {  // ---- loads
     if (lane == 0) {
+      int j = 0;
       for (long long t = t0; t < t1 && ok; ++t) {
         const int b = block_of(t);
         const LinTmaBlock& B = a.blk[b];
         if (B.w_off < 0) continue;
-        const int s = mj % RS;
-        if (mj >= RS) ok = mbar_wait(raw_empty + s, ((mj / RS) - 1) & 1);
+        const int s = j % RS;
+        if (j >= RS) ok = mbar_wait(st_empty + s, ((j / RS) - 1) & 1);
         if (!ok) break;
         const int node0 = static_cast<int>((t - B.first_tile) * B.nn);
-        mbar_expect(raw_full + s, static_cast<unsigned>((K / 32) * 128 * B.dim * B.nn));
+        mbar_expect(st_full + s, static_cast<unsigned>((K / 32) * 128 * B.dim * B.nn));
         for (int c = 0; c < K / 32; ++c)
-          tma_load_3d(raw + (static_cast<size_t>(s) * (K / 32) + c) * kChunkBytes, &a.in_map[b], raw_full + s,
-                      32 * c, 0, node0);
-        ++mj;
+          tma_load_3d(stage(s) + c * kChunkBytes, &a.in_map[b], st_full + s, 32 * c, 0, node0);
+        ++j;
       }
-      // no load outlives the block: wait for the last ones to land (already seen by the rows)
-      for (int q = (mj > RS ? mj - RS : 0); q < mj; ++q) mbar_wait(raw_full + q % RS, (q / RS) & 1);
+      // no load outlives the block: wait for the last ones to land
+      for (int q = (j > RS ? j - RS : 0); q < j; ++q) mbar_wait(st_full + q % RS, (q / RS) & 1);
       if (!ok) atomicOr(a.status, 4u);
     }
-  } else if (warp == 5) {  // ---- weights and MMAs
-    int mj = 0;
+  } else if (warp == 13) {  // ---- weights and MMAs
     if (lane == 0) {
-      int cur = -1;
+      int j = 0, cur = -1;
       unsigned ph_w = 0;
       const unsigned id = idesc_f16(kTile, N);
       for (long long t = t0; t < t1 && ok; ++t) {
@@ -341,7 +351,7 @@ __global__ void __launch_bounds__(192, 1) k_linear_tma(const __grid_constant__ L
         const LinTmaBlock& B = a.blk[b];
         if (B.w_off < 0) continue;
         if (b != cur) {  // every MMA on the previous weights has completed before they are replaced
-          if (mj > 0) ok = mbar_wait(mma_done + ((mj - 1) & 1), ((mj - 1) >> 1) & 1);
+          if (j > 0) ok = mbar_wait(mma_done + ((j - 1) & 1), ((j - 1) >> 1) & 1);
           if (!ok) break;
           const unsigned bytes = static_cast<unsigned>(2 * N * K * 2);
           mbar_expect(bar_w, bytes);
@@ -351,76 +361,69 @@ __global__ void __launch_bounds__(192, 1) k_linear_tma(const __grid_constant__ L
           ph_w ^= 1u;
           cur = b;
         }
-        ok = mbar_wait(act_full, mj & 1);
-        if (ok && mj >= 2) ok = mbar_wait(tm_empty + (mj & 1), ((mj - 2) >> 1) & 1);
+        const int s = j % RS;
+        ok = mbar_wait(op_full + s, (j / RS) & 1);
+        if (ok && j >= 2) ok = mbar_wait(tm_empty + (j & 1), ((j - 2) >> 1) & 1);
         if (!ok) break;
         tc_after();
-        const unsigned d = tmem + (mj & 1) * a.tmem_half;
+        const unsigned d = tmem + (j & 1) * a.tmem_half;
         const unsigned char* whi = bw;
         const unsigned char* wlo = bw + N * K * 2;
-        const unsigned char* ahi = act;
-        const unsigned char* alo = act + kTile * K * 2;
+        const unsigned char* ahi = stage(s);
+        const unsigned char* alo = ahi + kTile * K * 2;
         for (int ks = 0; ks < K / 16; ++ks) {
           const int ao = ks * kTile * 32, bo = ks * N * 32;
           mma_f16(d, kmajor_desc(ahi + ao), kmajor_desc(whi + bo), id, ks > 0);
           mma_f16(d, kmajor_desc(ahi + ao), kmajor_desc(wlo + bo), id, 1);
           mma_f16(d, kmajor_desc(alo + ao), kmajor_desc(whi + bo), id, 1);
         }
-        mma_commit(mma_done + (mj & 1));
-        mma_commit(act_empty);
-        ++mj;
+        mma_commit(mma_done + (j & 1));
+        mma_commit(st_empty + s);
+        ++j;
       }
-      if (mj > 0) {  // nothing in flight at exit: both commits of the last tile have arrived
-        mbar_wait(mma_done + ((mj - 1) & 1), ((mj - 1) >> 1) & 1);
-        mbar_wait(act_empty, (mj - 1) & 1);
-      }
+      // nothing in flight at exit: every commit of the last tiles has arrived
+      if (j > 0) mbar_wait(mma_done + ((j - 1) & 1), ((j - 1) >> 1) & 1);
+      for (int q = (j > RS ? j - RS : 0); q < j; ++q) mbar_wait(st_empty + q % RS, (q / RS) & 1);
       if (!ok) atomicOr(a.status, 4u);
     }
-  } else {  // ---- warps 0-3: operand rows, then the previous tile's output
-    const unsigned lane_off = static_cast<unsigned>(32 * warp) << 16;
-    // the 128 row threads agree on every wait's outcome, so they leave the loop together
-    auto team_and = [](bool p) {
-      unsigned r;
-      asm volatile(
-          "{ .reg .pred q, o; setp.ne.u32 q, %1, 0; bar.red.and.pred o, 1, 128, q; selp.u32 %0, 1, 0, o; }"
-          : "=r"(r)
-          : "r"(static_cast<unsigned>(p))
-          : "memory");
-      return r != 0;
-    };
-    int mj = 0, chunk = 0;
-    float R[K];
-    // the output of MMA tile q (block b, first node node0) through the staging tiles
-    auto drain = [&](int q, int b, int node0) {
+  } else if (warp >= 4) {  // ---- warps 4-11: float32 rows -> float16 hi / lo operand, in place
+    constexpr int KH = K / 2;  // channels of one thread
+    const int st = tid - 128, r = st & (kTile - 1), h = st >> 7;
+    int j = 0;
+    float R[KH];
+    for (long long t = t0; t < t1 && ok; ++t) {
+      const int b = block_of(t);
       const LinTmaBlock& B = a.blk[b];
-      ok = team_and(ok && mbar_wait(mma_done + (q & 1), (q >> 1) & 1));
-      tc_after();
-      for (int j0 = 0; j0 < N && ok; j0 += 32) {
-        float v[32];
-        tmem_ld32(tmem + (q & 1) * a.tmem_half + lane_off + j0, v);
-        if (j0 + 32 >= N) {  // the accumulator is read: free it for the tile after next
-          tc_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tm_empty + (q & 1));
-        }
-        unsigned char* st = stg + (chunk & 1) * kChunkBytes;
-        if (tid == 0) bulk_wait_read_but1();  // the store issued from this staging tile has read it
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (B.w_off < 0) continue;
+      const int s = j % RS;
+      ok = team_and(2, 256, mbar_wait(st_full + s, (j / RS) & 1));
+      if (!ok) break;
+      unsigned char* base = stage(s);
+      const bool live = r < B.dim * B.nn;
+      // channels [h KH, (h + 1) KH) of row r: 16-byte pieces (h KH + 4 i) / 4 of the row's
+      // 32-channel boxes, each at piece ^ (r & 7) within its 128-byte row
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          *reinterpret_cast<float4*>(st + tid * 128 + ((i ^ (tid & 7)) << 4)) =
-              make_float4(v[4 * i] * B.scale, v[4 * i + 1] * B.scale, v[4 * i + 2] * B.scale,
-                          v[4 * i + 3] * B.scale);
-        fence_async_smem();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (tid == 0) {
-          tma_store_3d(&a.out_map[b], st, j0, 0, node0);
-          bulk_commit();
-        }
-        ++chunk;
+      for (int i = 0; i < KH / 4; ++i) {
+        const int q = h * (KH / 4) + i;  // piece of the row
+        const float4 v = live ? *reinterpret_cast<const float4*>(base + (q >> 3) * kChunkBytes + r * 128 +
+                                                                 (((q & 7) ^ (r & 7)) << 4))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        R[4 * i] = v.x;
+        R[4 * i + 1] = v.y;
+        R[4 * i + 2] = v.z;
+        R[4 * i + 3] = v.w;
       }
-    };
-    int pb = -1, pnode = 0;  // the MMA tile whose output is pending
+      asm volatile("bar.sync 2, 256;" ::: "memory");  // the stage is read: overwrite it
+      store_split_part<KH>(base, base + kTile * K * 2, r, R, kTile, h * KH);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(op_full + s);
+      ++j;
+    }
+    if (!ok && st == 0) atomicOr(a.status, 4u);
+  } else {  // ---- warps 0-3: accumulators out, zero tiles
+    const unsigned lane_off = static_cast<unsigned>(32 * warp) << 16;
+    int j = 0, chunk = 0;
     for (long long t = t0; t < t1 && ok; ++t) {
       const int b = block_of(t);
       const LinTmaBlock& B = a.blk[b];
@@ -433,37 +436,35 @@ __global__ void __launch_bounds__(192, 1) k_linear_tma(const __grid_constant__ L
         }
         continue;
       }
-      const int s = mj % RS;
-      ok = team_and(mbar_wait(raw_full + s, (mj / RS) & 1));
+      ok = team_and(1, 128, mbar_wait(mma_done + (j & 1), (j >> 1) & 1));
       if (!ok) break;
-      const bool live = tid < B.dim * B.nn;
-#pragma unroll
-      for (int c = 0; c < K / 32; ++c) {
-        const unsigned char* src = raw + (static_cast<size_t>(s) * (K / 32) + c) * kChunkBytes + tid * 128;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 v = live ? *reinterpret_cast<const float4*>(src + ((i ^ (tid & 7)) << 4))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-          R[32 * c + 4 * i] = v.x;
-          R[32 * c + 4 * i + 1] = v.y;
-          R[32 * c + 4 * i + 2] = v.z;
-          R[32 * c + 4 * i + 3] = v.w;
+      tc_after();
+      for (int j0 = 0; j0 < N; j0 += 32) {
+        float v[32];
+        tmem_ld32(tmem + (j & 1) * a.tmem_half + lane_off + j0, v);
+        if (j0 + 32 >= N) {  // the accumulator is read: free it for the tile after next
+          tc_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tm_empty + (j & 1));
         }
+        unsigned char* sg = stg + (chunk & 1) * kChunkBytes;
+        if (tid == 0) bulk_wait_read_but1();  // the store issued from this staging tile has read it
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<float4*>(sg + tid * 128 + ((i ^ (tid & 7)) << 4)) =
+              make_float4(v[4 * i] * B.scale, v[4 * i + 1] * B.scale, v[4 * i + 2] * B.scale,
+                          v[4 * i + 3] * B.scale);
+        fence_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (tid == 0) {
+          tma_store_3d(&a.out_map[b], sg, j0, 0, node0);
+          bulk_commit();
+        }
+        ++chunk;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(raw_empty + s);  // the stage may be refilled
-      ok = team_and(mj == 0 || mbar_wait(act_empty, (mj - 1) & 1));  // the previous MMAs read the operand
-      if (!ok) break;
-      store_split_row<K>(act, act + kTile * K * 2, tid, R, kTile);
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(act_full);
-      if (pb >= 0) drain(mj - 1, pb, pnode);  // overlaps this tile's MMAs
-      pb = b;
-      pnode = node0;
-      ++mj;
+      ++j;
     }
-    if (ok && pb >= 0) drain(mj - 1, pb, pnode);
     if (tid == 0) bulk_wait_all();
     if (!ok && tid == 0) atomicOr(a.status, 4u);
   }
@@ -474,6 +475,7 @@ __global__ void __launch_bounds__(192, 1) k_linear_tma(const __grid_constant__ L
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * a.tmem_half)
                  : "memory");
 }
+
 }  // namespace
 
 int linear_prepare(LinearPlan& lp, const std::vector<Irrep>& in, const std::vector<Irrep>& out,
@@ -571,10 +573,10 @@ size_t linear_smem_bytes(const LinearPlan& lp) {
   return 2 * static_cast<size_t>(lp.N) * lp.K * 2 + 2 * static_cast<size_t>(kTile) * lp.K * 2 + 64;
 }
 
-// raw stages of the tensor-map kernel that fit in shared memory next to the rest (0: none)
+// stages of the tensor-map kernel that fit in shared memory next to the rest
 static int linear_tma_stages(const LinearPlan& lp) {
   int s = 0;
-  while (s < 4 && lin_tma_layout(lp.K, lp.N, s + 1).total <= 227 * 1024) ++s;
+  while (s < kTmaMaxStages && lin_tma_layout(lp.K, lp.N, s + 1).total <= 227 * 1024) ++s;
   return s;
 }
 
@@ -582,7 +584,7 @@ bool linear_uses_tma(const LinearPlan& lp) {
   if (!lp.allow_tma || lp.N % 32 != 0 || static_cast<int>(lp.blocks.size()) > kTmaMaxBlocks) return false;
   for (const LinBlock& b : lp.blocks)
     if (b.dim > kTile) return false;
-  return linear_tma_stages(lp) >= 1;
+  return linear_tma_stages(lp) >= 2;  // one stage would serialise load, split and MMAs
 }
 
 static int linear_launch_tma(const LinearPlan& lp, const void* dev_w, const float* x, long long nodes,
@@ -650,7 +652,7 @@ static int linear_launch_tma(const LinearPlan& lp, const void* dev_w, const floa
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kernel<<<blocks, 192, smem, st>>>(a);
+    kernel<<<blocks, kTmaThreads, smem, st>>>(a);
     return cudaGetLastError();
   };
   (void)mma_tiles;

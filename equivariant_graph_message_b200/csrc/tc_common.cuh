@@ -167,17 +167,15 @@ __device__ __forceinline__ unsigned pack_half2(float lo, float hi) {
   return r;
 }
 
-// hi and lo float16 parts of v[0..8), packed as two 16-byte vectors
+// hi and lo float16 parts of v[0..8), packed as two 16-byte vectors (pairs converted by one
+// cvt.rn.f16x2.f32 each, round to nearest like __float2half_rn)
 __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
   unsigned h[4], l[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const __half h0 = __float2half_rn(v[2 * q]), h1 = __float2half_rn(v[2 * q + 1]);
-    const __half l0 = __float2half_rn(v[2 * q] - __half2float(h0));
-    const __half l1 = __float2half_rn(v[2 * q + 1] - __half2float(h1));
-    const __half2 hh = __halves2half2(h0, h1), ll = __halves2half2(l0, l1);
-    h[q] = *reinterpret_cast<const unsigned*>(&hh);
-    l[q] = *reinterpret_cast<const unsigned*>(&ll);
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h[q]) : "f"(v[2 * q + 1]), "f"(v[2 * q]));
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[q]));
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(l[q]) : "f"(v[2 * q + 1] - f.y), "f"(v[2 * q] - f.x));
   }
   hi = make_uint4(h[0], h[1], h[2], h[3]);
   lo = make_uint4(l[0], l[1], l[2], l[3]);

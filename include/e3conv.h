@@ -385,10 +385,10 @@ E3CONV_API int e3conv_linear_query(e3conv_linear linear, int* dim_in, int* dim_o
 
 /* *uses_tma = 1 when e3conv_linear_forward runs the tensor-map kernel for
  * this layer (mul_out a multiple of 32, at most 8 output irreps, 2l+1 <= 128,
- * and its shared-memory stages fit: every shape but mul_in = 128 with
- * mul_out > 128): whole-node tiles moved by 3-D TMA boxes in and out, warp
- * roles pipelined over a ring of input stages and two tensor-memory
- * accumulators.  0: the row-per-thread kernel (thread t loads and stores row
+ * and two input stages fit in shared memory: every shape but mul_in = 128
+ * with mul_out > 128): whole-node tiles moved by 3-D TMA boxes in and out,
+ * warp roles pipelined over a ring of input stages (each split in place into
+ * the float16 operand) and two tensor-memory accumulators.  0: the row-per-thread kernel (thread t loads and stores row
  * t of a 128-row tile).  Both give the same results up to float32 rounding. */
 E3CONV_API int e3conv_linear_uses_tma(e3conv_linear linear, int* uses_tma);
 /* enable = 0: always the row-per-thread kernel; 1 (the default): the

@@ -20,7 +20,7 @@ SHAPES = [
     ("64x0e+64x1o+64x2e", "128x0e+128x1e+128x1o+128x2e+128x3o", True),     # unmatched 1e, 3o
     ("32x0e+32x1o", "256x1o+256x0e", True),
     ("128x0e+128x1o+128x2e+128x3o", "16x3o+16x0e", False),                  # mul_out 16
-    ("128x0e+128x1o", "256x0e+256x1o", False),                              # no room for a stage
+    ("128x0e+128x1o", "256x0e+256x1o", False),                              # room for one stage
     ("64x0e+64x1o+64x2e+64x3o+64x4e+64x5o+64x6e", "96x6e+96x0e+96x4e+96x5o", True),  # 13 rows a node
 ]
 

@@ -463,20 +463,20 @@ def test_linear_layer_host_validation():
 
 
 @pytest.mark.parametrize("ins,outs,fits", [
-    ("128x0e+128x1o+128x2e+128x3o", "128x0e+128x1o+128x2e+128x3o", True),   # one raw stage
+    ("128x0e+128x1o+128x2e+128x3o", "128x0e+128x1o+128x2e+128x3o", True),   # two stages
     ("64x0e+64x1o", "64x0e+64x1o", True),
     ("32x0e", "256x0e", True),
     ("64x0e", "64x0e+64x1o+64x1e", True),                     # unmatched outputs: zero tiles
     ("128x0e", "16x0e", False),                               # mul_out not a multiple of 32
     ("128x0e", "48x0e", False),
-    ("128x0e+128x1o", "256x0e+256x1o", False),                # weights + operand leave no stage
+    ("128x0e+128x1o", "256x0e+256x1o", False),                # weights leave one stage
     ("64x0e", "+".join(f"64x{l}{'eo'[l % 2]}" for l in range(9)), False),  # 9 output irreps
 ])
 def test_linear_kernel_choice(ins, outs, fits):
     # the tensor-map kernel takes a shape when mul_out is a multiple of 32 (32-column output
     # boxes), there are at most 8 output irreps (two tensor maps each as kernel parameters)
-    # and a raw input stage fits in shared memory next to the weights, the operand and the
-    # staging tiles; set_tma(False) always selects the row-per-thread kernel
+    # and two input stages fit in shared memory next to the weights and the staging tiles;
+    # set_tma(False) always selects the row-per-thread kernel
     lin = e3.IrrepsLinear(ins, outs)
     assert lin.uses_tma == fits
     lin.set_tma(False)
