@@ -13,28 +13,31 @@
 //   s      = h_L W_L                            (hidden -> P*C, tensor cores)
 // with SiLU(v) = v / (1 + exp(-v)), no biases.
 //
-// Tensor-core layers: one CTA of 256 threads per tile of 128 edges: threads t
-// and t + 128 share edge row t (tensor-memory lane t) and each reads, applies
-// SiLU to, and stores half of the row's columns.  A = the tile's activations
-// [128 edges x hidden], B = the weights [N outputs x hidden] (both K-major,
-// float16, core matrices of 8 rows x 16 bytes, no swizzle), D = A B^T in
-// tensor memory (float32).  Both operands are split into float16 hi + lo
-// parts, D = A_hi B_hi + A_hi B_lo + A_lo B_hi (the lo x lo term is below
-// float32 rounding), which keeps the products at float32 accuracy; the
-// weights are scaled by a power of two before the split (undone exactly on
-// the way out) so that their lo parts stay normal float16 numbers.
-// The output layer runs in chunks of 128 columns (one N = 128 MMA per K step
-// and split term): their weights are double-buffered in shared memory (bulk
-// copies of prepacked chunks), their products alternate between two
-// tensor-memory buffers, so the MMAs of chunk c overlap the stores of chunk
-// c-1.  Stores: the threads write the chunk's [128 edges x 128 columns] tile
-// into shared memory in the TMA's 128-byte swizzle (thread t, row t: its
-// 16-byte pieces land in distinct banks), and one thread stores it with 2-D
-// TMA tensor stores of 128 rows x 128 bytes (rows past the last edge and
-// columns past P*C are clipped by the TMA); rows whose byte length is not a
-// multiple of 16 are stored element by element instead.  All
-// waits are bounded: on timeout a CTA sets bit 4 of the status word, drains
-// what it issued (bounded) and stops.
+// Tensor-core layers: A = a tile's activations [128 edges x K], B = the
+// weights [N outputs x K] (both K-major, float16, core matrices of 8 rows x 16
+// bytes, no swizzle), D = A B^T in tensor memory (float32).  Both operands are
+// split into float16 hi + lo parts, D = A_hi B_hi + A_hi B_lo + A_lo B_hi (the
+// lo x lo term is below float32 rounding), which keeps the products at float32
+// accuracy; the weights are scaled by a power of two before the split (undone
+// exactly on the way out) so that their lo parts stay normal float16 numbers.
+//
+// One persistent CTA per SM over tiles of 128 edges, in warp roles that hand
+// work over through mbarriers:
+//   warps 4-11  (two threads per edge row, each half of the row's columns)
+//               compute the bases, read the hidden accumulator, apply SiLU and
+//               write the next activation operand;
+//   warp 12     issues every MMA (layer 0, hidden layers, output chunks) and
+//               the bulk copies of the output-weight chunks (double-buffered);
+//   warps 0-3   (thread t <-> edge row t <-> tensor-memory lane t) read each
+//               output chunk of 128 columns out of one of three tensor-memory
+//               accumulators into a ring of swizzled [128 rows x 128 bytes]
+//               staging boxes, each stored by a 2-D TMA tensor store as soon as
+//               it is written (rows past the last edge and columns past P*C are
+//               clipped by the TMA; rows whose byte length is not a multiple of
+//               16 are stored element by element instead).
+// So the output stores of one tile stream while the next tile's bases and
+// hidden layers run.  All waits are bounded: on timeout a CTA sets bit 4 of
+// the status word, drains what it issued (bounded) and stops.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
@@ -94,13 +97,16 @@ struct Smem {
 
 };
 
+constexpr int kOutBufs = 3;             // output-layer accumulators in tensor memory
+constexpr int kRadThreads = 416;        // 4 drain warps, 8 compute warps, 1 MMA warp
+constexpr int kRadBars = 18;            // mbarriers (and the tensor-memory slot after them)
+
 template <int H>
-__global__ void __launch_bounds__(256, 1) k_radial(RadialArgs a, const __grid_constant__ CUtensorMap smap) {
+__global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const __grid_constant__ CUtensorMap smap) {
   extern __shared__ __align__(1024) unsigned char sm[];
   using L = Smem<H>;
-  constexpr int HH = H / 2;                       // hidden columns of one thread
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int row = tid & (kTile - 1), half = tid >> 7;  // edge row, which half of its columns
+  constexpr int HH = H / 2;  // hidden columns of one compute thread
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   unsigned char* w0s = sm;                                            // layer 0 (hi, lo)
   unsigned char* whs = w0s + 2 * L::kW0;                              // (layers-1) x (hi, lo)
   unsigned char* bas = whs + (a.layers - 1) * 2 * L::kWhid;           // basis values (hi, lo)
@@ -108,14 +114,28 @@ __global__ void __launch_bounds__(256, 1) k_radial(RadialArgs a, const __grid_co
   unsigned char* wos = act + 2 * L::kAct;                             // 2 buffers x (hi, lo)
   unsigned char* stage = wos + kWBufs * 2 * L::kWout;  // 1024-byte aligned (128-byte swizzle)
   unsigned long long* bars = reinterpret_cast<unsigned long long*>(stage + kStageBytes);
-  unsigned long long* bar_w = bars;                 // [kWBufs] output-weight chunk landed
-  unsigned long long* bar_mma = bars + kWBufs;      // [2] output MMAs of a chunk done
-  unsigned long long* bar_hid = bars + kWBufs + 2;  // hidden-layer MMAs done
-  unsigned long long* bar_wh = bars + kWBufs + 3;   // hidden weights landed
-  unsigned* tslot = reinterpret_cast<unsigned*>(bars + kWBufs + 4);
-
+  unsigned long long* bar_wh = bars;         // layer 0's and the hidden layers' weights landed
+  unsigned long long* bar_w = bars + 1;      // [2] output-weight chunk landed
+  unsigned long long* w_free = bars + 3;     // [2] MMAs done with an output-weight chunk
+  unsigned long long* bas_full = bars + 5;   // basis operand written (8 compute warps)
+  unsigned long long* act_full = bars + 6;   // activation operand written (8 compute warps)
+  unsigned long long* hid_read = bars + 7;   // hidden accumulator read (8 compute warps)
+  unsigned long long* hid_done = bars + 8;   // hidden-layer MMAs done
+  unsigned long long* act_free = bars + 9;   // a tile's output MMAs done (operand reusable)
+  unsigned long long* mma_done = bars + 10;  // [3] output chunk in an accumulator
+  unsigned long long* tm_empty = bars + 13;  // [3] accumulator read (4 drain warps)
+  unsigned* tslot = reinterpret_cast<unsigned*>(bars + 16);
   if (tid == 0) {
-    for (int k = 0; k < kWBufs + 4; ++k) mbar_init(bars + k, 1);
+    for (int k = 0; k < 5; ++k) mbar_init(bars + k, 1);
+    mbar_init(bas_full, 8);
+    mbar_init(act_full, 8);
+    mbar_init(hid_read, 8);
+    mbar_init(hid_done, 1);
+    mbar_init(act_free, 1);
+    for (int b = 0; b < kOutBufs; ++b) {
+      mbar_init(mma_done + b, 1);
+      mbar_init(tm_empty + b, 4);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -128,253 +148,274 @@ __global__ void __launch_bounds__(256, 1) k_radial(RadialArgs a, const __grid_co
   __syncthreads();
   tc_after();
   const unsigned tmem = *tslot;
-  const unsigned t_hid = tmem;                 // columns [0, H): hidden-layer D
-  // output-layer D: two buffers of kChunk columns at kOutCol and kOutCol + kChunk
-  // warps w and w + 4 both read tensor-memory lanes 32 (w % 4) .. + 31
-  const unsigned lane_off = static_cast<unsigned>(32 * (warp & 3)) << 16;
-  bool ok = true;
-  // phase bits (bit b: buffer b) of the weight-chunk and output-MMA barriers
-  unsigned ph_w = 0, ph_mma = 0, ph_hid = 0;
-  // copies and MMAs thread 0 issued and has not yet seen complete (bit b: buffer b; drained on
-  // a timeout)
-  unsigned pend_w = 0, pend_mma = 0;
-  bool pend_hid = false, pend_wh = false;
-  if (tid == 0) {  // layer 0's and the hidden layers' weights, once per CTA
-    const unsigned hb = static_cast<unsigned>((a.layers - 1) * 2 * L::kWhid);
-    mbar_expect(bar_wh, 2 * L::kW0 + hb);
-    bulk_g2s(w0s, a.w0, 2 * L::kW0, bar_wh);
-    if (hb) bulk_g2s(whs, a.wh, hb, bar_wh);
-    pend_wh = true;
-  }
-  ok = __syncthreads_and(mbar_wait(bar_wh, 0));
-  pend_wh = !ok;
-  const float pi_r = a.pi_r;
-  const float norm = a.norm;
+  const unsigned t_hid = tmem;  // columns [0, H): hidden-layer accumulator
+  auto t_out = [&](int b) { return tmem + static_cast<unsigned>(kOutCol + kChunk * b); };
   const long long tiles = (a.num_edges + kTile - 1) / kTile;
-  for (long long tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-    const long long e = tile * kTile + row;
-    const bool valid = e < a.num_edges;
-    // prefetch the first output-weight chunks of this tile (every buffer is free: the
-    // previous tile waited for all of its output MMAs)
-    if (tid == 0) {
-      for (int c = 0; c < kWBufs && c < a.chunks; ++c) {
-        mbar_expect(bar_w + c, 2 * L::kWout);
-        bulk_g2s(wos + c * 2 * L::kWout, a.wo + static_cast<size_t>(c) * 2 * L::kWout,
-                 2 * L::kWout, bar_w + c);
-        pend_w |= 1u << c;
+  const long long my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const long long total = my_tiles * a.chunks;  // this CTA's output chunks, tile by tile
+  // a named barrier of `count` threads that also ANDs a predicate over them
+  auto team_and = [](int id, int count, bool p) {
+    unsigned r;
+    asm volatile(
+        "{ .reg .pred q, o; setp.ne.u32 q, %1, 0; bar.red.and.pred o, %2, %3, q; selp.u32 %0, 1, 0, o; }"
+        : "=r"(r)
+        : "r"(static_cast<unsigned>(p)), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+  };
+  bool ok = true;
+
+  if (warp == 12) {  // ---- weights and MMAs
+    if (lane == 0) {
+      // layer 0's and the hidden layers' weights once; the first output-weight chunk
+      const unsigned hb = static_cast<unsigned>((a.layers - 1) * 2 * L::kWhid);
+      mbar_expect(bar_wh, 2 * L::kW0 + hb);
+      bulk_g2s(w0s, a.w0, 2 * L::kW0, bar_wh);
+      if (hb) bulk_g2s(whs, a.wh, hb, bar_wh);
+      if (total > 0) {
+        mbar_expect(bar_w, 2 * L::kWout);
+        bulk_g2s(wos, a.wo, 2 * L::kWout, bar_w);
       }
-    }
-    // layer 0: basis x cutoff on the CUDA cores, SiLU(h0 W0) with h0 W0 on the tensor cores
-    float h[HH];  // this thread's half of the row's hidden values: columns half * HH ..
-    if (half == 0) {
-      float d = 0.f;
-      if (valid) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(a.vec) + e);
-        d = sqrtf(fmaf(v.x, v.x, fmaf(v.y, v.y, v.z * v.z)));
-      }
-      const bool inside = valid && d < a.r_max;
-      const float t = d * a.inv_r;                        // d / r in [0, 1) inside
-      const float u = 0.5f * (1.0f + cospif(t));          // cos(pi d / r)
-      float b[kMaxBasis];
-#pragma unroll
-      for (int n = 0; n < kMaxBasis; ++n) {
-        b[n] = (!inside || n >= a.nb)
-                   ? 0.f
-                   : (d > 0.f ? norm * sinpif((n + 1) * t) / d : norm * (n + 1) * pi_r) * u;
-      }
-      store_split_row<kMaxBasis>(bas, bas + L::kBas, row, b, kTile);
-      fence_async_smem();
-    }
-    {
-      tc_before();
-      __syncthreads();
-      tc_after();
-      if (tid == 0) {
-        const unsigned id0 = idesc_f16(kTile, H);
+      ok = mbar_wait(bar_wh, 0);
+      long long g = 0;       // output chunks issued
+      int nhid = 0, nact = 0;  // hidden MMA groups issued, activation operands consumed
+      const unsigned id0 = idesc_f16(kTile, H), idh = idesc_f16(kTile, H), ido = idesc_f16(kTile, kChunk);
+      for (long long k = 0; k < my_tiles && ok; ++k) {
+        // layer 0: basis operand x W0 into the hidden accumulator
+        ok = mbar_wait(bas_full, k & 1);
+        if (ok && nhid > 0) ok = mbar_wait(hid_read, (nhid - 1) & 1);
+        if (!ok) break;
+        tc_after();
         mma_f16(t_hid, kmajor_desc(bas), kmajor_desc(w0s), id0, 0);
         mma_f16(t_hid, kmajor_desc(bas), kmajor_desc(w0s + L::kW0), id0, 1);
         mma_f16(t_hid, kmajor_desc(bas + L::kBas), kmajor_desc(w0s), id0, 1);
-        mma_commit(bar_hid);
-        pend_hid = true;
-      }
-      ok = __syncthreads_and(mbar_wait(bar_hid, ph_hid));
-      tc_after();
-      if (!ok) break;
-      ph_hid ^= 1u;
-      pend_hid = false;
-      {
-        float v[32];
-        tmem_ld32(t_hid + lane_off + half * HH, v);
+        mma_commit(hid_done);
+        ++nhid;
+        for (int l = 1; l < a.layers && ok; ++l) {  // hidden layers
+          ok = mbar_wait(act_full, nact & 1) && mbar_wait(hid_read, (nhid - 1) & 1);
+          if (!ok) break;
+          ++nact;
+          tc_after();
+          const unsigned char* whi = whs + (l - 1) * 2 * L::kWhid;
+          const unsigned long long d_ahi = kmajor_desc(act), d_alo = kmajor_desc(act + L::kAct);
+          const unsigned long long d_whi = kmajor_desc(whi), d_wlo = kmajor_desc(whi + L::kWhid);
 #pragma unroll
-        for (int q = 0; q < HH; ++q) h[q] = silu(v[q] * a.w_scale_inv_0);
-      }
-      tc_before();
-      __syncthreads();  // every thread has read D before the next layer's MMAs overwrite it
-      tc_after();
-    }
-    // hidden layers 1 .. L-1 on the tensor cores
-    for (int l = 1; l < a.layers && ok; ++l) {
-      store_split_part<HH>(act, act + L::kAct, row, h, kTile, half * HH);
-      fence_async_smem();
-      tc_before();
-      __syncthreads();
-      tc_after();
-      if (tid == 0) {
-        const unsigned char* whi = whs + (l - 1) * 2 * L::kWhid;
-        const unsigned id = idesc_f16(kTile, H);
-        const unsigned long long d_ahi = kmajor_desc(act), d_alo = kmajor_desc(act + L::kAct);
-        const unsigned long long d_whi = kmajor_desc(whi), d_wlo = kmajor_desc(whi + L::kWhid);
-#pragma unroll
-        for (int ks = 0; ks < H / 16; ++ks) {
-          const unsigned long long ao = static_cast<unsigned long long>(ks * kTile * 32) >> 4;
-          const unsigned long long bo = static_cast<unsigned long long>(ks * H * 32) >> 4;
-          mma_f16(t_hid, d_ahi + ao, d_whi + bo, id, ks > 0);
-          mma_f16(t_hid, d_ahi + ao, d_wlo + bo, id, 1);
-          mma_f16(t_hid, d_alo + ao, d_whi + bo, id, 1);
+          for (int ks = 0; ks < H / 16; ++ks) {
+            const unsigned long long ao = static_cast<unsigned long long>(ks * kTile * 32) >> 4;
+            const unsigned long long bo = static_cast<unsigned long long>(ks * H * 32) >> 4;
+            mma_f16(t_hid, d_ahi + ao, d_whi + bo, idh, ks > 0);
+            mma_f16(t_hid, d_ahi + ao, d_wlo + bo, idh, 1);
+            mma_f16(t_hid, d_alo + ao, d_whi + bo, idh, 1);
+          }
+          mma_commit(hid_done);
+          ++nhid;
         }
-        mma_commit(bar_hid);
-        pend_hid = true;
-      }
-      ok = __syncthreads_and(mbar_wait(bar_hid, ph_hid));
-      tc_after();
-      if (!ok) break;
-      ph_hid ^= 1u;
-      pend_hid = false;
-      {
-        float v[32];
-        tmem_ld32(t_hid + lane_off + half * HH, v);
-#pragma unroll
-        for (int q = 0; q < HH; ++q) h[q] = silu(v[q] * a.w_scale_inv_h);
-      }
-      tc_before();
-      __syncthreads();  // every thread has read D before the next layer's MMAs overwrite it
-      tc_after();
-    }
-    if (!ok) break;
-    // output layer: chunks of 128 columns
-    store_split_part<HH>(act, act + L::kAct, row, h, kTile, half * HH);
-    fence_async_smem();
-    tc_before();
-    __syncthreads();
-    tc_after();
-    const unsigned id = idesc_f16(kTile, kChunk);
-    // descriptors: the activations' hi / lo operands and the weight buffers; K step ks adds
-    // its byte offset / 16 to the start-address field
-    const unsigned long long d_ahi = kmajor_desc(act), d_alo = kmajor_desc(act + L::kAct);
-    for (int c = 0; c <= a.chunks && ok; ++c) {
-      if (c < a.chunks) {
-        const int wb = c % kWBufs, buf = c & 1;
-        ok = __syncthreads_and(mbar_wait(bar_w + wb, (ph_w >> wb) & 1u));
         if (!ok) break;
-        ph_w ^= 1u << wb;
-        pend_w &= ~(1u << wb);
-        if (tid == 0) {
+        // output layer: chunks of 128 columns
+        ok = mbar_wait(act_full, nact & 1);
+        if (!ok) break;
+        ++nact;
+        tc_after();
+        const unsigned long long d_ahi = kmajor_desc(act), d_alo = kmajor_desc(act + L::kAct);
+        for (int c = 0; c < a.chunks && ok; ++c, ++g) {
+          // the next chunk's weights into the other buffer, once the MMAs of the chunk before
+          // this one have read it
+          if (g + 1 < total) {
+            const int nb = static_cast<int>((g + 1) & 1);
+            if (g >= 1) ok = mbar_wait(w_free + nb, ((g - 1) >> 1) & 1);
+            if (!ok) break;
+            const long long cn = (g + 1) % a.chunks;
+            mbar_expect(bar_w + nb, 2 * L::kWout);
+            bulk_g2s(wos + nb * 2 * L::kWout, a.wo + static_cast<size_t>(cn) * 2 * L::kWout, 2 * L::kWout,
+                     bar_w + nb);
+          }
+          const int wb = static_cast<int>(g & 1), b = static_cast<int>(g % kOutBufs);
+          ok = mbar_wait(bar_w + wb, (g >> 1) & 1);
+          if (ok && g >= kOutBufs) ok = mbar_wait(tm_empty + b, ((g / kOutBufs) - 1) & 1);
+          if (!ok) break;
+          tc_after();
           const unsigned long long d_whi = kmajor_desc(wos + wb * 2 * L::kWout);
           const unsigned long long d_wlo = kmajor_desc(wos + wb * 2 * L::kWout + L::kWout);
-          const unsigned td = tmem + static_cast<unsigned>(kOutCol + kChunk * buf);
 #pragma unroll
           for (int ks = 0; ks < H / 16; ++ks) {
             const unsigned long long ao = static_cast<unsigned long long>(ks * kTile * 32) >> 4;
             const unsigned long long bo = static_cast<unsigned long long>(ks * kChunk * 32) >> 4;
-            mma_f16(td, d_ahi + ao, d_whi + bo, id, ks > 0);
-            mma_f16(td, d_ahi + ao, d_wlo + bo, id, 1);
-            mma_f16(td, d_alo + ao, d_whi + bo, id, 1);
+            mma_f16(t_out(b), d_ahi + ao, d_whi + bo, ido, ks > 0);
+            mma_f16(t_out(b), d_ahi + ao, d_wlo + bo, ido, 1);
+            mma_f16(t_out(b), d_alo + ao, d_whi + bo, ido, 1);
           }
-          mma_commit(bar_mma + buf);
-          pend_mma |= 1u << buf;
+          mma_commit(mma_done + b);
+          mma_commit(w_free + wb);
         }
-      }
-      if (c >= 1) {  // chunk c-1: its weight buffer takes chunk c+1, then its stores
-        const int pb = (c - 1) & 1, pw = (c - 1) % kWBufs;
-        // the previous chunk's TMA stores have read the staging tile (thread 0 issued them);
-        // the barrier below publishes that to every thread
-        if (tid == 0) bulk_wait_read();
-        ok = __syncthreads_and(mbar_wait(bar_mma + pb, (ph_mma >> pb) & 1u));
-        tc_after();
         if (!ok) break;
-        ph_mma ^= 1u << pb;
-        pend_mma &= ~(1u << pb);
-        if (tid == 0 && c - 1 + kWBufs < a.chunks) {
-          mbar_expect(bar_w + pw, 2 * L::kWout);
-          bulk_g2s(wos + pw * 2 * L::kWout,
-                   a.wo + static_cast<size_t>(c - 1 + kWBufs) * 2 * L::kWout, 2 * L::kWout,
-                   bar_w + pw);
-          pend_w |= 1u << pw;
+        mma_commit(act_free);
+      }
+      // nothing in flight at exit: the last commits have arrived (bounded waits)
+      if (nhid > 0) mbar_wait(hid_done, (nhid - 1) & 1);
+      for (long long q = (g > 2 ? g - 2 : 0); q < g; ++q) mbar_wait(w_free + (q & 1), (q >> 1) & 1);
+      if (g > 0) mbar_wait(mma_done + (g - 1) % kOutBufs, ((g - 1) / kOutBufs) & 1);
+      if (ok && my_tiles > 0) mbar_wait(act_free, (my_tiles - 1) & 1);
+      if (!ok) {  // copies issued but never waited for
+        mbar_wait(bar_wh, 0);
+        if (g + 1 < total && g < total) mbar_wait(bar_w + ((g + 1) & 1), ((g + 1) >> 1) & 1);
+        if (g < total) mbar_wait(bar_w + (g & 1), (g >> 1) & 1);
+        atomicOr(a.status, 4u);
+      }
+    }
+  } else if (warp >= 4) {  // ---- warps 4-11: bases, SiLU, activation operands
+    const int st = tid - 128, row = st & (kTile - 1), half = st >> 7;
+    // warps w and w + 4 read tensor-memory lanes 32 (w % 4) .. + 31: this thread's row
+    const unsigned lane_off = static_cast<unsigned>(32 * (warp & 3)) << 16;
+    const float pi_r = a.pi_r, norm = a.norm;
+    int nhid = 0, nact = 0;  // hidden accumulators read, activation operands written
+    float h[HH];
+    auto read_hidden = [&](float scale_inv) {  // SiLU(D) of this thread's half of the row
+      ok = team_and(2, 256, mbar_wait(hid_done, nhid & 1));
+      if (!ok) return;
+      tc_after();
+      float v[32];
+      tmem_ld32(t_hid + lane_off + half * HH, v);
+      tc_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(hid_read);
+      ++nhid;
+#pragma unroll
+      for (int q = 0; q < HH; ++q) h[q] = silu(v[q] * scale_inv);
+    };
+    auto write_act = [&](long long k) {  // h -> activation operand (after the last tile's use)
+      if (nact % a.layers == 0 && k > 0) {
+        ok = team_and(2, 256, mbar_wait(act_free, (k - 1) & 1));
+        if (!ok) return;
+      }
+      store_split_part<HH>(act, act + L::kAct, row, h, kTile, half * HH);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(act_full);
+      ++nact;
+    };
+    for (long long k = 0; k < my_tiles && ok; ++k) {
+      const long long tile = blockIdx.x + k * gridDim.x;
+      const long long e = tile * kTile + row;
+      // layer 0's input: bessel basis x cosine cutoff on the CUDA cores (the previous tile's
+      // layer-0 MMAs have read the basis operand: this thread waited for them)
+      if (half == 0) {
+        float d = 0.f;
+        const bool valid = e < a.num_edges;
+        if (valid) {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(a.vec) + e);
+          d = sqrtf(fmaf(v.x, v.x, fmaf(v.y, v.y, v.z * v.z)));
         }
-        const int col0 = (c - 1) * kChunk;
-        const int cols = min(kChunk, a.nout - col0);
-        const float f = a.w_scale_inv_o;
-        if (a.tma) {
-          // staging tile: per 128-byte column box (32 floats or 64 halves), row r at r * 128,
-          // its 16-byte piece q at (q ^ (r & 7)) * 16
-#pragma unroll 1
-          for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
-            float v[32];
-            tmem_ld32(tmem + static_cast<unsigned>(kOutCol + kChunk * pb + j0) + lane_off, v);
-            if (a.out_f16) {
-              unsigned char* box = stage + (j0 / 64) * (kTile * 128) + row * 128;
+        const bool inside = valid && d < a.r_max;
+        const float t = d * a.inv_r;                // d / r in [0, 1) inside
+        const float u = 0.5f * (1.0f + cospif(t));  // cos(pi d / r)
+        float b[kMaxBasis];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int piece = (j0 % 64) / 8 + q;
-                *reinterpret_cast<uint4*>(box + ((piece ^ (row & 7)) * 16)) =
-                    make_uint4(pack_half2(v[8 * q] * f, v[8 * q + 1] * f),
-                               pack_half2(v[8 * q + 2] * f, v[8 * q + 3] * f),
-                               pack_half2(v[8 * q + 4] * f, v[8 * q + 5] * f),
-                               pack_half2(v[8 * q + 6] * f, v[8 * q + 7] * f));
-              }
-            } else {
-              unsigned char* box = stage + (j0 / 32) * (kTile * 128) + row * 128;
+        for (int n = 0; n < kMaxBasis; ++n) {
+          b[n] = (!inside || n >= a.nb) ? 0.f
+                                        : (d > 0.f ? norm * sinpif((n + 1) * t) / d : norm * (n + 1) * pi_r) * u;
+        }
+        store_split_row<kMaxBasis>(bas, bas + L::kBas, row, b, kTile);
+        fence_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bas_full);
+      read_hidden(a.w_scale_inv_0);
+      for (int l = 1; l < a.layers && ok; ++l) {
+        write_act(k);
+        if (!ok) break;
+        read_hidden(a.w_scale_inv_h);
+      }
+      if (!ok) break;
+      write_act(k);  // the output layer's input
+    }
+    if (!ok && st == 0) atomicOr(a.status, 4u);
+  } else {  // ---- warps 0-3: output chunks out of tensor memory (thread t <-> row t <-> lane t)
+    const unsigned lane_off = static_cast<unsigned>(32 * warp) << 16;
+    const int row = tid;
+    const float f = a.w_scale_inv_o;
+    const int boxes = a.out_f16 ? kChunk / 64 : kChunk / 32;  // 128-byte column boxes per chunk
+    const int bcols = a.out_f16 ? 64 : 32;
+    for (long long g = 0; g < total && ok; ++g) {
+      const long long tile = blockIdx.x + (g / a.chunks) * gridDim.x;
+      const int c = static_cast<int>(g % a.chunks), b = static_cast<int>(g % kOutBufs);
+      const long long e = tile * kTile + row;
+      const int col0 = c * kChunk;
+      ok = team_and(1, 128, mbar_wait(mma_done + b, (g / kOutBufs) & 1));
+      if (!ok) break;
+      tc_after();
+      if (a.tma) {
+        // staging: a ring of `boxes` slots of [128 rows x 128 bytes], row r at r * 128, its
+        // 16-byte piece q at (q ^ (r & 7)) * 16; box q of this chunk reuses slot q of the
+        // previous one (thread 0 waits until that store has read it) and is stored as soon as
+        // it is written, so the stores stream while the next boxes are staged
+        for (int q = 0; q < boxes; ++q) {
+          unsigned char* slot = stage + q * (kTile * 128);
+          if (tid == 0) {
+            if (boxes == 4)
+              bulk_wait_read_but<3>();
+            else
+              bulk_wait_read_but<1>();
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");  // slot q is free
+          unsigned char* dst = slot + row * 128;
+          if (a.out_f16) {
 #pragma unroll
-              for (int q = 0; q < 8; ++q)
-                *reinterpret_cast<float4*>(box + ((q ^ (row & 7)) * 16)) =
-                    make_float4(v[4 * q] * f, v[4 * q + 1] * f, v[4 * q + 2] * f, v[4 * q + 3] * f);
+            for (int hh = 0; hh < 2; ++hh) {
+              float v[32];
+              tmem_ld32(t_out(b) + lane_off + q * 64 + hh * 32, v);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<uint4*>(dst + (((hh * 4 + i) ^ (row & 7)) * 16)) =
+                    make_uint4(pack_half2(v[8 * i] * f, v[8 * i + 1] * f),
+                               pack_half2(v[8 * i + 2] * f, v[8 * i + 3] * f),
+                               pack_half2(v[8 * i + 4] * f, v[8 * i + 5] * f),
+                               pack_half2(v[8 * i + 6] * f, v[8 * i + 7] * f));
             }
+          } else {
+            float v[32];
+            tmem_ld32(t_out(b) + lane_off + q * 32, v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              *reinterpret_cast<float4*>(dst + ((i ^ (row & 7)) * 16)) =
+                  make_float4(v[4 * i] * f, v[4 * i + 1] * f, v[4 * i + 2] * f, v[4 * i + 3] * f);
+          }
+          if (q == boxes - 1) {  // the accumulator is read: free it for the chunk after next
+            tc_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tm_empty + b);
           }
           fence_async_smem();
-          __syncthreads();  // the whole tile is staged
+          asm volatile("bar.sync 1, 128;" ::: "memory");  // box q is staged
           if (tid == 0) {
-            const int boxes = a.out_f16 ? kChunk / 64 : kChunk / 32;
-            const int bcols = a.out_f16 ? 64 : 32;
-            for (int q = 0; q < boxes; ++q)
-              if (col0 + q * bcols < a.nout)
-                tma_store_2d(&smap, stage + q * (kTile * 128), col0 + q * bcols,
-                             static_cast<int>(tile * kTile));
-            bulk_commit();
+            if (col0 + q * bcols < a.nout)
+              tma_store_2d(&smap, slot, col0 + q * bcols, static_cast<int>(tile * kTile));
+            bulk_commit();  // one group per box (empty past the last column)
           }
-        } else {
-#pragma unroll 1
-          for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
-            float v[32];
-            tmem_ld32(tmem + static_cast<unsigned>(kOutCol + kChunk * pb + j0) + lane_off, v);
-            if (valid) {
-              const long long base = e * a.nout + col0 + j0;
+        }
+      } else {  // rows whose byte length is not a multiple of 16: element stores
+        const int cols = min(kChunk, a.nout - col0);
+        for (int j0 = 0; j0 < kChunk; j0 += 32) {
+          float v[32];
+          tmem_ld32(t_out(b) + lane_off + j0, v);
+          if (e < a.num_edges) {
+            const long long base = e * a.nout + col0 + j0;
 #pragma unroll
-              for (int q = 0; q < 32; ++q) {
-                if (j0 + q >= cols) continue;
-                if (a.out_f16)
-                  static_cast<__half*>(a.s)[base + q] = __float2half_rn(v[q] * f);
-                else
-                  static_cast<float*>(a.s)[base + q] = v[q] * f;
-              }
+            for (int q = 0; q < 32; ++q) {
+              if (j0 + q >= cols) continue;
+              if (a.out_f16)
+                static_cast<__half*>(a.s)[base + q] = __float2half_rn(v[q] * f);
+              else
+                static_cast<float*>(a.s)[base + q] = v[q] * f;
             }
           }
         }
         tc_before();
-        __syncthreads();  // chunk c-1's columns read by every thread before they are reused
-        tc_after();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tm_empty + b);
       }
     }
-  }
-  bulk_wait_all();  // every row store of this thread has landed
-  if (!ok && tid == 0) {
-    atomicOr(a.status, 4u);
-    // drain (bounded): copies and MMAs issued but not seen complete
-    for (int b = 0; b < kWBufs; ++b)
-      if ((pend_w >> b) & 1u) mbar_wait(bar_w + b, (ph_w >> b) & 1u);
-    for (int b = 0; b < 2; ++b)
-      if ((pend_mma >> b) & 1u) mbar_wait(bar_mma + b, (ph_mma >> b) & 1u);
-    if (pend_hid) mbar_wait(bar_hid, ph_hid);
-    if (pend_wh) mbar_wait(bar_wh, 0);
+    if (tid == 0) bulk_wait_all();  // every store has landed
+    if (!ok && tid == 0) atomicOr(a.status, 4u);
   }
   tc_before();
   __syncthreads();
@@ -438,7 +479,7 @@ int radial_prepare(RadialPlan& rp, int nb, double r_max, int hidden, int layers,
 size_t radial_smem_bytes(const RadialPlan& rp) {
   const size_t H = rp.hidden;
   return 2 * H * kMaxBasis * 2 + (rp.layers - 1) * 2 * H * H * 2 + 2 * kTile * kMaxBasis * 2 +
-         2 * kTile * H * 2 + kWBufs * 2 * kChunk * H * 2 + kStageBytes + (kWBufs + 4) * 8 + 16;
+         2 * kTile * H * 2 + kWBufs * 2 * kChunk * H * 2 + kStageBytes + kRadBars * 8;
 }
 
 int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, const void* dev_wo,
@@ -476,12 +517,12 @@ int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, 
                                          static_cast<int>(smem));
     int per_sm = 0;
     if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, smem);
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kRadThreads, smem);
     if (e != cudaSuccess || per_sm < 1) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
     // tensor memory: all 512 columns per CTA, so one CTA per SM
     per_sm = 1;
     const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, static_cast<long long>(grid) * per_sm));
-    kernel<<<blocks, 256, smem, st>>>(a, map);
+    kernel<<<blocks, kRadThreads, smem, st>>>(a, map);
     return cudaSuccess;
   };
   cudaError_t e = rp.hidden == 32 ? launch(k_radial<32>) : launch(k_radial<64>);
