@@ -13,31 +13,38 @@
 //   s      = h_L W_L                            (hidden -> P*C, tensor cores)
 // with SiLU(v) = v / (1 + exp(-v)), no biases.
 //
-// Tensor-core layers: A = a tile's activations [128 edges x K], B = the
-// weights [N outputs x K] (both K-major, float16, core matrices of 8 rows x 16
-// bytes, no swizzle), D = A B^T in tensor memory (float32).  Both operands are
-// split into float16 hi + lo parts, D = A_hi B_hi + A_hi B_lo + A_lo B_hi (the
-// lo x lo term is below float32 rounding), which keeps the products at float32
-// accuracy; the weights are scaled by a power of two before the split (undone
-// exactly on the way out) so that their lo parts stay normal float16 numbers.
+// Tensor-core layers: D = A B^T in tensor memory (float32) with both operands
+// K-major float16 in shared memory (core matrices of 8 rows x 16 bytes, no
+// swizzle).  Both operands are split into float16 hi + lo parts,
+// D = A_hi B_hi + A_hi B_lo + A_lo B_hi (the lo x lo term is below float32
+// rounding), which keeps the products at float32 accuracy; the weights are
+// scaled by a power of two before the split (undone exactly on the way out)
+// so that their lo parts stay normal float16 numbers.  Every layer puts the
+// tile's 128 edges on the MMA's M side: A = activations [128 x K], B = weights
+// [N x K]; the output layer runs in chunks of N = 128 columns.
 //
 // One persistent CTA per SM over tiles of 128 edges, in warp roles that hand
 // work over through mbarriers:
-//   warps 4-11  (two threads per edge row, each half of the row's columns)
-//               compute the bases, read the hidden accumulator, apply SiLU and
-//               write the next activation operand;
-//   warp 12     issues every MMA (layer 0, hidden layers, output chunks) and
-//               the bulk copies of the output-weight chunks (double-buffered);
+//   warps 4-11  (two threads per edge row, each half of the row's hidden
+//               columns) compute the bases, read the hidden accumulator, apply
+//               SiLU and write the activation operands (two buffers where
+//               shared memory allows: the next tile's hidden layers run while
+//               the output layer still reads this tile's);
+//   warp 12     issues layer 0's and the hidden layers' MMAs;
+//   warp 13     issues the output layer's MMAs, chunk by chunk, into three
+//               tensor-memory accumulators, and the bulk copies of the
+//               output-weight chunks into a ring of 2-4 buffers;
 //   warps 0-3   (thread t <-> edge row t <-> tensor-memory lane t) read each
-//               output chunk of 128 columns out of one of three tensor-memory
-//               accumulators into a ring of swizzled [128 rows x 128 bytes]
-//               staging boxes, each stored by a 2-D TMA tensor store as soon as
-//               it is written (rows past the last edge and columns past P*C are
-//               clipped by the TMA; rows whose byte length is not a multiple of
-//               16 are stored element by element instead).
-// So the output stores of one tile stream while the next tile's bases and
-// hidden layers run.  All waits are bounded: on timeout a CTA sets bit 4 of
-// the status word, drains what it issued (bounded) and stops.
+//               output chunk out of its accumulator into a ring of swizzled
+//               [128 rows x 128 bytes] staging boxes, each stored by a 2-D TMA
+//               tensor store as soon as it is written (rows past the last edge
+//               and columns past P*C are clipped by the TMA; rows whose byte
+//               length is not a multiple of 16 are stored element by element).
+// The stores stream at the SM's store rate while the next tile's bases and
+// hidden layers run; what is left between chunks is the output MMAs' wait for
+// a free accumulator.
+// All waits are bounded: on timeout a CTA sets bit 4 of the status word,
+// drains what it issued (bounded) and stops.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
@@ -60,10 +67,13 @@ using namespace tc_host;
 constexpr int kTile = 128;           // edges per tile (MMA M)
 constexpr int kMaxBasis = 16;        // radial bases = the K of layer 0's MMA (zero-padded)
 constexpr int kChunk = 128;          // output columns per output-layer chunk (MMA N)
-constexpr int kWBufs = 2;            // output-weight chunk buffers in shared memory
-constexpr int kStageBytes = kTile * kChunk * 4;  // one chunk's output tile (float32)
-constexpr int kOutCol = 128;         // tensor-memory column of the output buffers (>= hidden)
-constexpr int kTmemCols = 512;       // hidden D [0, H) and two output buffers of kChunk
+constexpr int kStageBytes = kTile * kChunk * 4;  // staging ring: four boxes of 128 rows x 128 bytes
+constexpr int kMaxWBufs = 4;         // output-weight chunk buffers in shared memory (at most)
+constexpr int kOutBufs = 3;          // output-layer accumulators in tensor memory
+constexpr int kOutCol = 128;         // tensor-memory column of the output accumulators (>= hidden)
+constexpr int kTmemCols = 512;       // hidden D [0, H) and three output accumulators of 128
+constexpr int kRadThreads = 448;     // 4 drain warps, 8 compute warps, 2 MMA warps
+constexpr int kRadBars = 24;         // mbarriers (and the tensor-memory slot after them)
 
 struct RadialArgs {
   const float* vec;        // [E][4] edge vectors (x, y, z, unused)
@@ -77,6 +87,7 @@ struct RadialArgs {
   float pi_r, inv_r, norm; // pi / r_max, 1 / r_max and sqrt(2 / r_max)
   int nb, layers;          // basis size, hidden layers L (>= 1)
   int nout, chunks;        // P*C outputs, chunks of kChunk (the last padded with zero weights)
+  int wbufs, abufs;        // output-weight chunk buffers, activation buffers
   float r_max;
   void* s;                 // [E][nout] float32 or float16
   int out_f16;
@@ -84,9 +95,10 @@ struct RadialArgs {
   unsigned* status;
 };
 
-// Shared memory of one CTA (bytes): layer 0's and the hidden layers' weights,
-// the basis values and the activations (hi, lo each), two output-weight chunks
-// (hi, lo each), the staged output rows, barriers and the tensor-memory slot.
+// Shared memory of one CTA (bytes): the staging ring, layer 0's and the hidden layers' weights,
+// the basis values and the activations (hi, lo each; one or two activation
+// buffers), the output-weight chunk ring (hi, lo each), barriers and the
+// tensor-memory slot.
 template <int H>
 struct Smem {
   static constexpr int kW0 = H * kMaxBasis * 2;          // one [H x 16] float16 operand
@@ -94,12 +106,13 @@ struct Smem {
   static constexpr int kAct = kTile * H * 2;     // one K-major [128 x H] float16 operand
   static constexpr int kWhid = H * H * 2;        // one [H x H] float16 operand
   static constexpr int kWout = kChunk * H * 2;   // one [kChunk x H] float16 operand
-
 };
 
-constexpr int kOutBufs = 3;             // output-layer accumulators in tensor memory
-constexpr int kRadThreads = 416;        // 4 drain warps, 8 compute warps, 1 MMA warp
-constexpr int kRadBars = 18;            // mbarriers (and the tensor-memory slot after them)
+inline size_t radial_smem_for(int H, int layers, int abufs, int wbufs) {
+  const size_t h = static_cast<size_t>(H);
+  return kStageBytes + 2 * h * kMaxBasis * 2 + (layers - 1) * 2 * h * h * 2 + 2 * kTile * kMaxBasis * 2 +
+         abufs * 2 * kTile * h * 2 + wbufs * 2 * kChunk * h * 2 + kRadBars * 8;
+}
 
 template <int H>
 __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const __grid_constant__ CUtensorMap smap) {
@@ -107,34 +120,44 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
   using L = Smem<H>;
   constexpr int HH = H / 2;  // hidden columns of one compute thread
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  unsigned char* w0s = sm;                                            // layer 0 (hi, lo)
+  const int A = a.abufs, W = a.wbufs;
+  unsigned char* stage = sm;                                          // 1024-byte aligned (swizzle)
+  unsigned char* w0s = stage + kStageBytes;                           // layer 0 (hi, lo)
   unsigned char* whs = w0s + 2 * L::kW0;                              // (layers-1) x (hi, lo)
   unsigned char* bas = whs + (a.layers - 1) * 2 * L::kWhid;           // basis values (hi, lo)
-  unsigned char* act = bas + 2 * L::kBas;                             // hi, lo
-  unsigned char* wos = act + 2 * L::kAct;                             // 2 buffers x (hi, lo)
-  unsigned char* stage = wos + kWBufs * 2 * L::kWout;  // 1024-byte aligned (128-byte swizzle)
-  unsigned long long* bars = reinterpret_cast<unsigned long long*>(stage + kStageBytes);
+  unsigned char* acts = bas + 2 * L::kBas;                            // A x (hi, lo)
+  unsigned char* wos = acts + A * 2 * L::kAct;                        // W x (hi, lo)
+  unsigned long long* bars = reinterpret_cast<unsigned long long*>(wos + W * 2 * L::kWout);
   unsigned long long* bar_wh = bars;         // layer 0's and the hidden layers' weights landed
-  unsigned long long* bar_w = bars + 1;      // [2] output-weight chunk landed
-  unsigned long long* w_free = bars + 3;     // [2] MMAs done with an output-weight chunk
-  unsigned long long* bas_full = bars + 5;   // basis operand written (8 compute warps)
-  unsigned long long* act_full = bars + 6;   // activation operand written (8 compute warps)
-  unsigned long long* hid_read = bars + 7;   // hidden accumulator read (8 compute warps)
-  unsigned long long* hid_done = bars + 8;   // hidden-layer MMAs done
-  unsigned long long* act_free = bars + 9;   // a tile's output MMAs done (operand reusable)
-  unsigned long long* mma_done = bars + 10;  // [3] output chunk in an accumulator
-  unsigned long long* tm_empty = bars + 13;  // [3] accumulator read (4 drain warps)
-  unsigned* tslot = reinterpret_cast<unsigned*>(bars + 16);
+  unsigned long long* bas_full = bars + 1;   // basis operand written (8 compute warps)
+  unsigned long long* act_full = bars + 2;   // a hidden layer's input written (8 compute warps)
+  unsigned long long* hid_read = bars + 3;   // hidden accumulator read (8 compute warps)
+  unsigned long long* hid_done = bars + 4;   // layer-0 / hidden-layer MMAs done
+  unsigned long long* out_full = bars + 5;   // [2] the output layer's input written (8 warps)
+  unsigned long long* act_free = bars + 7;   // [2] a tile's output MMAs done with its buffer
+  unsigned long long* mma_done = bars + 9;   // [3] output chunk in an accumulator
+  unsigned long long* tm_empty = bars + 12;  // [3] accumulator read (4 drain warps)
+  unsigned long long* bar_w = bars + 15;     // [4] output-weight chunk landed
+  unsigned long long* w_free = bars + 19;    // [4] MMAs done with an output-weight chunk
+  unsigned* tslot = reinterpret_cast<unsigned*>(bars + 23);
+  auto act = [&](long long k) { return acts + static_cast<int>(k % A) * 2 * L::kAct; };
   if (tid == 0) {
-    for (int k = 0; k < 5; ++k) mbar_init(bars + k, 1);
+    mbar_init(bar_wh, 1);
     mbar_init(bas_full, 8);
     mbar_init(act_full, 8);
     mbar_init(hid_read, 8);
     mbar_init(hid_done, 1);
-    mbar_init(act_free, 1);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(out_full + q, 8);
+      mbar_init(act_free + q, 1);
+    }
     for (int b = 0; b < kOutBufs; ++b) {
       mbar_init(mma_done + b, 1);
       mbar_init(tm_empty + b, 4);
+    }
+    for (int q = 0; q < kMaxWBufs; ++q) {
+      mbar_init(bar_w + q, 1);
+      mbar_init(w_free + q, 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -165,39 +188,32 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
   };
   bool ok = true;
 
-  if (warp == 12) {  // ---- weights and MMAs
+  if (warp == 12) {  // ---- layer 0's and the hidden layers' MMAs
     if (lane == 0) {
-      // layer 0's and the hidden layers' weights once; the first output-weight chunk
       const unsigned hb = static_cast<unsigned>((a.layers - 1) * 2 * L::kWhid);
       mbar_expect(bar_wh, 2 * L::kW0 + hb);
       bulk_g2s(w0s, a.w0, 2 * L::kW0, bar_wh);
       if (hb) bulk_g2s(whs, a.wh, hb, bar_wh);
-      if (total > 0) {
-        mbar_expect(bar_w, 2 * L::kWout);
-        bulk_g2s(wos, a.wo, 2 * L::kWout, bar_w);
-      }
       ok = mbar_wait(bar_wh, 0);
-      long long g = 0;       // output chunks issued
-      int nhid = 0, nact = 0;  // hidden MMA groups issued, activation operands consumed
-      const unsigned id0 = idesc_f16(kTile, H), idh = idesc_f16(kTile, H), ido = idesc_f16(kTile, kChunk);
+      int nhid = 0, nact = 0;  // MMA groups issued, hidden-layer inputs consumed
+      const unsigned idh = idesc_f16(kTile, H);
       for (long long k = 0; k < my_tiles && ok; ++k) {
-        // layer 0: basis operand x W0 into the hidden accumulator
         ok = mbar_wait(bas_full, k & 1);
         if (ok && nhid > 0) ok = mbar_wait(hid_read, (nhid - 1) & 1);
         if (!ok) break;
         tc_after();
-        mma_f16(t_hid, kmajor_desc(bas), kmajor_desc(w0s), id0, 0);
-        mma_f16(t_hid, kmajor_desc(bas), kmajor_desc(w0s + L::kW0), id0, 1);
-        mma_f16(t_hid, kmajor_desc(bas + L::kBas), kmajor_desc(w0s), id0, 1);
+        mma_f16(t_hid, kmajor_desc(bas), kmajor_desc(w0s), idh, 0);
+        mma_f16(t_hid, kmajor_desc(bas), kmajor_desc(w0s + L::kW0), idh, 1);
+        mma_f16(t_hid, kmajor_desc(bas + L::kBas), kmajor_desc(w0s), idh, 1);
         mma_commit(hid_done);
         ++nhid;
-        for (int l = 1; l < a.layers && ok; ++l) {  // hidden layers
+        for (int l = 1; l < a.layers && ok; ++l) {
           ok = mbar_wait(act_full, nact & 1) && mbar_wait(hid_read, (nhid - 1) & 1);
           if (!ok) break;
           ++nact;
           tc_after();
           const unsigned char* whi = whs + (l - 1) * 2 * L::kWhid;
-          const unsigned long long d_ahi = kmajor_desc(act), d_alo = kmajor_desc(act + L::kAct);
+          const unsigned long long d_ahi = kmajor_desc(act(k)), d_alo = kmajor_desc(act(k) + L::kAct);
           const unsigned long long d_whi = kmajor_desc(whi), d_wlo = kmajor_desc(whi + L::kWhid);
 #pragma unroll
           for (int ks = 0; ks < H / 16; ++ks) {
@@ -210,27 +226,47 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
           mma_commit(hid_done);
           ++nhid;
         }
+      }
+      if (nhid > 0) mbar_wait(hid_done, (nhid - 1) & 1);  // nothing in flight at exit
+      if (!ok) {
+        mbar_wait(bar_wh, 0);
+        atomicOr(a.status, 4u);
+      }
+    }
+  } else if (warp == 13) {  // ---- the output layer's MMAs and weight chunks
+    if (lane == 0) {
+      long long g = 0, gl = 0;  // chunks issued, chunk weights requested
+      auto load = [&](long long q) {
+        const int wb = static_cast<int>(q % W);
+        mbar_expect(bar_w + wb, 2 * L::kWout);
+        bulk_g2s(wos + wb * 2 * L::kWout, a.wo + static_cast<size_t>(q % a.chunks) * 2 * L::kWout,
+                 2 * L::kWout, bar_w + wb);
+      };
+      const unsigned ido = idesc_f16(kTile, kChunk);
+      for (long long k = 0; k < my_tiles && ok; ++k) {
+        ok = mbar_wait(out_full + (k % A), (k / A) & 1);
         if (!ok) break;
-        // output layer: chunks of 128 columns
-        ok = mbar_wait(act_full, nact & 1);
-        if (!ok) break;
-        ++nact;
         tc_after();
-        const unsigned long long d_ahi = kmajor_desc(act), d_alo = kmajor_desc(act + L::kAct);
+        const unsigned long long d_hhi = kmajor_desc(act(k)), d_hlo = kmajor_desc(act(k) + L::kAct);
         for (int c = 0; c < a.chunks && ok; ++c, ++g) {
-          // the next chunk's weights into the other buffer, once the MMAs of the chunk before
-          // this one have read it
-          if (g + 1 < total) {
-            const int nb = static_cast<int>((g + 1) & 1);
-            if (g >= 1) ok = mbar_wait(w_free + nb, ((g - 1) >> 1) & 1);
-            if (!ok) break;
-            const long long cn = (g + 1) % a.chunks;
-            mbar_expect(bar_w + nb, 2 * L::kWout);
-            bulk_g2s(wos + nb * 2 * L::kWout, a.wo + static_cast<size_t>(cn) * 2 * L::kWout, 2 * L::kWout,
-                     bar_w + nb);
+          // weight chunks requested as far ahead as the ring has buffers whose MMAs are done
+          // (chunk g's own request waits for its buffer, the later ones only look)
+          while (gl < total && gl < g + W) {
+            if (gl >= W) {
+              const int wb = static_cast<int>(gl % W);
+              const unsigned par = static_cast<unsigned>(((gl / W) - 1) & 1);
+              if (gl > g) {
+                if (!mbar_try(w_free + wb, par)) break;
+              } else if (!(ok = mbar_wait(w_free + wb, par))) {
+                break;
+              }
+            }
+            load(gl);
+            ++gl;
           }
-          const int wb = static_cast<int>(g & 1), b = static_cast<int>(g % kOutBufs);
-          ok = mbar_wait(bar_w + wb, (g >> 1) & 1);
+          if (!ok) break;
+          const int wb = static_cast<int>(g % W), b = static_cast<int>(g % kOutBufs);
+          ok = mbar_wait(bar_w + wb, (g / W) & 1);
           if (ok && g >= kOutBufs) ok = mbar_wait(tm_empty + b, ((g / kOutBufs) - 1) & 1);
           if (!ok) break;
           tc_after();
@@ -238,36 +274,31 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
           const unsigned long long d_wlo = kmajor_desc(wos + wb * 2 * L::kWout + L::kWout);
 #pragma unroll
           for (int ks = 0; ks < H / 16; ++ks) {
-            const unsigned long long ao = static_cast<unsigned long long>(ks * kTile * 32) >> 4;
-            const unsigned long long bo = static_cast<unsigned long long>(ks * kChunk * 32) >> 4;
-            mma_f16(t_out(b), d_ahi + ao, d_whi + bo, ido, ks > 0);
-            mma_f16(t_out(b), d_ahi + ao, d_wlo + bo, ido, 1);
-            mma_f16(t_out(b), d_alo + ao, d_whi + bo, ido, 1);
+            const unsigned long long ho = static_cast<unsigned long long>(ks * kTile * 32) >> 4;
+            const unsigned long long wo = static_cast<unsigned long long>(ks * kChunk * 32) >> 4;
+            mma_f16(t_out(b), d_hhi + ho, d_whi + wo, ido, ks > 0);
+            mma_f16(t_out(b), d_hhi + ho, d_wlo + wo, ido, 1);
+            mma_f16(t_out(b), d_hlo + ho, d_whi + wo, ido, 1);
           }
           mma_commit(mma_done + b);
           mma_commit(w_free + wb);
         }
         if (!ok) break;
-        mma_commit(act_free);
+        mma_commit(act_free + (k % A));
       }
-      // nothing in flight at exit: the last commits have arrived (bounded waits)
-      if (nhid > 0) mbar_wait(hid_done, (nhid - 1) & 1);
-      for (long long q = (g > 2 ? g - 2 : 0); q < g; ++q) mbar_wait(w_free + (q & 1), (q >> 1) & 1);
+      // nothing in flight at exit: the last commits have arrived, every requested chunk landed
+      for (long long q = (g > W ? g - W : 0); q < g; ++q) mbar_wait(w_free + q % W, (q / W) & 1);
       if (g > 0) mbar_wait(mma_done + (g - 1) % kOutBufs, ((g - 1) / kOutBufs) & 1);
-      if (ok && my_tiles > 0) mbar_wait(act_free, (my_tiles - 1) & 1);
-      if (!ok) {  // copies issued but never waited for
-        mbar_wait(bar_wh, 0);
-        if (g + 1 < total && g < total) mbar_wait(bar_w + ((g + 1) & 1), ((g + 1) >> 1) & 1);
-        if (g < total) mbar_wait(bar_w + (g & 1), (g >> 1) & 1);
-        atomicOr(a.status, 4u);
-      }
+      for (long long q = g; q < gl; ++q) mbar_wait(bar_w + q % W, (q / W) & 1);
+      if (ok && my_tiles > 0) mbar_wait(act_free + (my_tiles - 1) % A, ((my_tiles - 1) / A) & 1);
+      if (!ok) atomicOr(a.status, 4u);
     }
   } else if (warp >= 4) {  // ---- warps 4-11: bases, SiLU, activation operands
     const int st = tid - 128, row = st & (kTile - 1), half = st >> 7;
     // warps w and w + 4 read tensor-memory lanes 32 (w % 4) .. + 31: this thread's row
     const unsigned lane_off = static_cast<unsigned>(32 * (warp & 3)) << 16;
     const float pi_r = a.pi_r, norm = a.norm;
-    int nhid = 0, nact = 0;  // hidden accumulators read, activation operands written
+    int nhid = 0;  // hidden accumulators read
     float h[HH];
     auto read_hidden = [&](float scale_inv) {  // SiLU(D) of this thread's half of the row
       ok = team_and(2, 256, mbar_wait(hid_done, nhid & 1));
@@ -281,17 +312,6 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
       ++nhid;
 #pragma unroll
       for (int q = 0; q < HH; ++q) h[q] = silu(v[q] * scale_inv);
-    };
-    auto write_act = [&](long long k) {  // h -> activation operand (after the last tile's use)
-      if (nact % a.layers == 0 && k > 0) {
-        ok = team_and(2, 256, mbar_wait(act_free, (k - 1) & 1));
-        if (!ok) return;
-      }
-      store_split_part<HH>(act, act + L::kAct, row, h, kTile, half * HH);
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(act_full);
-      ++nact;
     };
     for (long long k = 0; k < my_tiles && ok; ++k) {
       const long long tile = blockIdx.x + k * gridDim.x;
@@ -320,13 +340,23 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
       __syncwarp();
       if (lane == 0) mbar_arrive(bas_full);
       read_hidden(a.w_scale_inv_0);
+      if (!ok) break;
+      // this tile's activation buffer: free once the output MMAs of tile k - A are done
+      if (k >= A) ok = team_and(2, 256, mbar_wait(act_free + (k % A), ((k / A) - 1) & 1));
+      if (!ok) break;
+      unsigned char* ab = act(k);
       for (int l = 1; l < a.layers && ok; ++l) {
-        write_act(k);
-        if (!ok) break;
+        store_split_part<HH>(ab, ab + L::kAct, row, h, kTile, half * HH);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(act_full);
         read_hidden(a.w_scale_inv_h);
       }
       if (!ok) break;
-      write_act(k);  // the output layer's input
+      store_split_part<HH>(ab, ab + L::kAct, row, h, kTile, half * HH);  // the output layer's input
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(out_full + (k % A));
     }
     if (!ok && st == 0) atomicOr(a.status, 4u);
   } else {  // ---- warps 0-3: output chunks out of tensor memory (thread t <-> row t <-> lane t)
@@ -476,10 +506,20 @@ int radial_prepare(RadialPlan& rp, int nb, double r_max, int hidden, int layers,
   return E3CONV_OK;
 }
 
+// activation and output-weight buffers: two and as many chunk buffers (2-4) as fit, else one
+// activation buffer and two chunk buffers
+static void radial_buffers(const RadialPlan& rp, int& abufs, int& wbufs) {
+  constexpr size_t kMax = 227 * 1024;
+  abufs = 2;
+  for (wbufs = kMaxWBufs; wbufs > 2; --wbufs)
+    if (radial_smem_for(rp.hidden, rp.layers, abufs, wbufs) <= kMax) return;
+  if (radial_smem_for(rp.hidden, rp.layers, abufs, wbufs) > kMax) abufs = 1;
+}
+
 size_t radial_smem_bytes(const RadialPlan& rp) {
-  const size_t H = rp.hidden;
-  return 2 * H * kMaxBasis * 2 + (rp.layers - 1) * 2 * H * H * 2 + 2 * kTile * kMaxBasis * 2 +
-         2 * kTile * H * 2 + kWBufs * 2 * kChunk * H * 2 + kStageBytes + kRadBars * 8;
+  int abufs = 0, wbufs = 0;
+  radial_buffers(rp, abufs, wbufs);
+  return radial_smem_for(rp.hidden, rp.layers, abufs, wbufs);
 }
 
 int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, const void* dev_wo,
@@ -510,7 +550,8 @@ int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, 
   a.s = s;
   a.out_f16 = out_f16;
   a.status = status;
-  const size_t smem = radial_smem_bytes(rp);
+  radial_buffers(rp, a.abufs, a.wbufs);
+  const size_t smem = radial_smem_for(rp.hidden, rp.layers, a.abufs, a.wbufs);
   const long long tiles = (num_edges + kTile - 1) / kTile;
   auto launch = [&](auto kernel) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
