@@ -1010,6 +1010,7 @@ int e3conv_linear_set_tma(e3conv_linear h, int enable) {
   if (!h) return fail(E3CONV_ERR_INVALID_ARG, "linear is NULL");
   if (enable != 0 && enable != 1) return fail(E3CONV_ERR_INVALID_ARG, "enable must be 0 or 1");
   h->p.allow_tma = enable == 1;
+  h->p.tma_args.clear();
   return E3CONV_OK;
 }
 
@@ -1019,6 +1020,7 @@ int e3conv_linear_set_weights(e3conv_linear h, const float* w) {
   std::string err;
   int rc = linear_pack(lp, w, err);
   if (rc != E3CONV_OK) return fail(rc, err);
+  lp.tma_args.clear();  // the block scales of the kernel arguments follow the weights
   if (lp.device >= 0 && !lp.packed.empty()) {
     DeviceGuard g(lp.device);
     if (!lp.d_w && cudaMalloc(&lp.d_w, lp.packed.size()) != cudaSuccess) {

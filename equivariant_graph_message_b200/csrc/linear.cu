@@ -587,10 +587,53 @@ bool linear_uses_tma(const LinearPlan& lp) {
   return linear_tma_stages(lp) >= 2;  // one stage would serialise load, split and MMAs
 }
 
+static int encode_linear_args(const LinearPlan& lp, const void* dev_w, const float* x, long long nodes,
+                              float* y, unsigned* status, TensorMapEncodeFn encode, LinTmaArgs& a,
+                              std::string& err);
+
 static int linear_launch_tma(const LinearPlan& lp, const void* dev_w, const float* x, long long nodes,
                              float* y, unsigned* status, int grid, cudaStream_t st,
                              TensorMapEncodeFn encode, std::string& err) {
   LinTmaArgs a;
+  const bool cached = lp.tma_args.size() == sizeof a && lp.tma_x == x && lp.tma_y == y &&
+                      lp.tma_w == dev_w && lp.tma_nodes == nodes;
+  if (cached) {
+    std::memcpy(&a, lp.tma_args.data(), sizeof a);
+  } else {
+    const int rc = encode_linear_args(lp, dev_w, x, nodes, y, status, encode, a, err);
+    if (rc != E3CONV_OK) return rc;
+    lp.tma_args.assign(reinterpret_cast<const unsigned char*>(&a),
+                       reinterpret_cast<const unsigned char*>(&a) + sizeof a);
+    lp.tma_x = x;
+    lp.tma_y = y;
+    lp.tma_w = dev_w;
+    lp.tma_nodes = nodes;
+  }
+  const long long tiles = a.tiles_total;
+  const size_t smem = lin_tma_layout(lp.K, lp.N, a.stages).total;
+  // one CTA per SM (shared memory); as many as there are tiles, at most one per SM
+  const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, grid));
+  auto launch = [&](auto kernel) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kernel<<<blocks, kTmaThreads, smem, st>>>(a);
+    return cudaGetLastError();
+  };
+  cudaError_t e = lp.K == 32 ? launch(k_linear_tma<32>) : lp.K == 64 ? launch(k_linear_tma<64>)
+                                                                      : launch(k_linear_tma<128>);
+  if (e != cudaSuccess) {
+    err = "irreps linear kernel launch failed";
+    return E3CONV_ERR_CUDA;
+  }
+  return E3CONV_OK;
+}
+
+// the tensor-map kernel's arguments: per irrep block its tile geometry and the tensor maps of
+// its input rows and output rows
+static int encode_linear_args(const LinearPlan& lp, const void* dev_w, const float* x, long long nodes,
+                              float* y, unsigned* status, TensorMapEncodeFn encode, LinTmaArgs& a,
+                              std::string& err) {
   std::memset(&a, 0, sizeof a);
   a.y = y;
   a.w = static_cast<const unsigned char*>(dev_w);
@@ -645,23 +688,7 @@ static int linear_launch_tma(const LinearPlan& lp, const void* dev_w, const floa
     }
   }
   a.tiles_total = static_cast<int>(tiles);
-  const size_t smem = lin_tma_layout(lp.K, lp.N, a.stages).total;
-  // one CTA per SM (shared memory); as many as there are tiles, at most one per SM
-  const unsigned blocks = static_cast<unsigned>(std::min<long long>(tiles, grid));
-  auto launch = [&](auto kernel) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    kernel<<<blocks, kTmaThreads, smem, st>>>(a);
-    return cudaGetLastError();
-  };
   (void)mma_tiles;
-  cudaError_t e = lp.K == 32 ? launch(k_linear_tma<32>) : lp.K == 64 ? launch(k_linear_tma<64>)
-                                                                      : launch(k_linear_tma<128>);
-  if (e != cudaSuccess) {
-    err = "irreps linear kernel launch failed";
-    return E3CONV_ERR_CUDA;
-  }
   return E3CONV_OK;
 }
 

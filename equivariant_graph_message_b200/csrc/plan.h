@@ -187,6 +187,13 @@ struct LinearPlan {
   int device = -1;
   void* d_w = nullptr;
   unsigned* status = nullptr;
+  // arguments of the last tensor-map launch, reused while x, y and the node count repeat (a
+  // layer is used from one host thread at a time)
+  mutable std::vector<unsigned char> tma_args;
+  mutable const void* tma_x = nullptr;
+  mutable const void* tma_y = nullptr;
+  mutable const void* tma_w = nullptr;
+  mutable long long tma_nodes = -1;
 };
 
 struct Plan {

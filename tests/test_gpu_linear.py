@@ -79,3 +79,43 @@ def test_linear_on_the_convolution_output_full_size(cuda_device):
     assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
     del w, out, y, y_rows
     torch.cuda.empty_cache()
+
+
+def test_linear_repeated_and_changed_buffers(cuda_device):
+    # the tensor-map kernel keeps the arguments of its last launch: repeated calls on the same
+    # buffers (new contents), then other buffers and node counts, and new weights, all match
+    ins = outs = "64x0e+64x1o+64x2e"
+    lin = e3.IrrepsLinear(ins, outs, 1.0)
+    assert lin.uses_tma
+    rng = np.random.default_rng(11)
+
+    def weights():
+        ws = [rng.normal(size=(64, 64)).astype(np.float32) for _ in range(lin.num_weight_blocks)]
+        lin.set_weights(ws)
+        return ws
+
+    def check(x, y, ws):
+        torch.cuda.synchronize()
+        assert lin.check()
+        xs = x.cpu().numpy()
+        ref = oracle.irreps_linear(ins, outs, 1.0, xs, ws)
+        mag = oracle.irreps_linear(ins, outs, 1.0, np.abs(xs), [np.abs(w) for w in ws])
+        assert np.all(np.abs(y.cpu().numpy() - ref) <= 1e-5 * mag + 1e-30)
+
+    ws = weights()
+    x1 = torch.from_numpy(rng.normal(size=(777, lin.dim_in)).astype(np.float32)).cuda()
+    y1 = torch.empty((777, lin.dim_out), device="cuda")
+    lin(x1, out=y1)
+    check(x1, y1, ws)
+    x1.copy_(torch.from_numpy(rng.normal(size=(777, lin.dim_in)).astype(np.float32)))
+    lin(x1, out=y1)                                   # same buffers, new contents
+    check(x1, y1, ws)
+    lin(x1[:300], out=y1[:300])                       # same pointers, fewer nodes
+    check(x1[:300], y1[:300], ws)
+    x2 = torch.from_numpy(rng.normal(size=(1500, lin.dim_in)).astype(np.float32)).cuda()
+    y2 = torch.empty((1500, lin.dim_out), device="cuda")
+    lin(x2, out=y2)                                   # other buffers
+    check(x2, y2, ws)
+    ws = weights()                                    # new weights on the same buffers
+    lin(x2, out=y2)
+    check(x2, y2, ws)
