@@ -78,17 +78,18 @@ __global__ void __launch_bounds__(kHistThreads) k_histogram(const int* __restric
   }
 }
 
-// Exclusive scan of one 4096-element tile per block; writes the tile total.
-// `in` and `out` may alias: every thread reads its items before the first
-// barrier and writes them after it.
+// Exclusive scan of one tile of kScanThreads x ITEMS elements per block (thread t: the ITEMS
+// consecutive elements from t x ITEMS); writes the tile total.  `in` and `out` may alias: every
+// thread reads its items before the first barrier and writes them after it.
+template <int ITEMS>
 __global__ void __launch_bounds__(kScanThreads) k_scan_tile(const int* in, int* out, long long n,
                                                            int* __restrict__ totals) {
   __shared__ int warp_sums[kScanThreads / 32];
-  const long long base = (long long)blockIdx.x * kScanTile + (long long)threadIdx.x * kScanItems;
-  int v[kScanItems];
+  const long long base = (long long)blockIdx.x * kScanThreads * ITEMS + (long long)threadIdx.x * ITEMS;
+  int v[ITEMS];
   int sum = 0;
 #pragma unroll
-  for (int q = 0; q < kScanItems; ++q) {
+  for (int q = 0; q < ITEMS; ++q) {
     v[q] = (base + q < n) ? in[base + q] : 0;
     sum += v[q];
   }
@@ -115,10 +116,54 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_tile(const int* in, int* 
   __syncthreads();
   int run = warp_sums[warp] + incl - sum;
 #pragma unroll
-  for (int q = 0; q < kScanItems; ++q) {
+  for (int q = 0; q < ITEMS; ++q) {
     if (base + q < n) out[base + q] = run;
     run += v[q];
   }
+}
+
+// One block scans up to kScanThreads x kScanItemsOne elements in a single launch: coalesced
+// loads into shared memory, each thread scans its consecutive run there, a block scan of the
+// run totals, coalesced stores.  `in` and `out` may alias (every load precedes the first
+// barrier, every store follows the last).
+constexpr int kScanItemsOne = 32;
+__global__ void __launch_bounds__(kScanThreads) k_scan_one(const int* in, int* out, int n) {
+  extern __shared__ int sv[];  // n values
+  __shared__ int warp_sums[kScanThreads / 32];
+  for (int i = threadIdx.x; i < n; i += kScanThreads) sv[i] = in[i];
+  __syncthreads();
+  const int per = (n + kScanThreads - 1) / kScanThreads;
+  const int b0 = threadIdx.x * per, b1 = min(n, b0 + per);
+  int sum = 0;
+  for (int i = b0; i < b1; ++i) sum += sv[i];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = sum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    int t = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += t;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+    int wi = w;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      int t = __shfl_up_sync(0xffffffffu, wi, d);
+      if (lane >= d) wi += t;
+    }
+    warp_sums[lane] = wi - w;
+  }
+  __syncthreads();
+  int run = warp_sums[warp] + incl - sum;
+  for (int i = b0; i < b1; ++i) {
+    const int v = sv[i];
+    sv[i] = run;
+    run += v;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += kScanThreads) out[i] = sv[i];
 }
 
 __global__ void __launch_bounds__(kScanThreads) k_scan_add(int* __restrict__ out, long long n,
@@ -134,15 +179,22 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_add(int* __restrict__ out
 // With `count` set, only counts the kernels it would launch.
 void exclusive_scan(const int* in, int* out, int64_t n, int* scratch, cudaStream_t st, int* count) {
   if (n <= 0) return;
-  const int64_t blocks = ceil_div(n, kScanTile);
-  if (blocks == 1) {
-    if (count) ++*count;
-    else k_scan_tile<<<1, kScanThreads, 0, st>>>(in, out, n, nullptr);
+  if (n <= static_cast<int64_t>(kScanThreads) * kScanItemsOne) {  // one launch
+    if (count) {
+      ++*count;
+    } else if (n <= kScanTile) {
+      k_scan_tile<kScanItems><<<1, kScanThreads, 0, st>>>(in, out, n, nullptr);
+    } else {
+      const int smem = static_cast<int>(n * sizeof(int));
+      cudaFuncSetAttribute(k_scan_one, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      k_scan_one<<<1, kScanThreads, smem, st>>>(in, out, static_cast<int>(n));
+    }
     return;
   }
+  const int64_t blocks = ceil_div(n, kScanTile);
   int* totals = scratch;
   if (count) ++*count;
-  else k_scan_tile<<<static_cast<unsigned>(blocks), kScanThreads, 0, st>>>(in, out, n, totals);
+  else k_scan_tile<kScanItems><<<static_cast<unsigned>(blocks), kScanThreads, 0, st>>>(in, out, n, totals);
   exclusive_scan(totals, totals, blocks, scratch + blocks, st, count);
   if (count) ++*count;
   else k_scan_add<<<static_cast<unsigned>(blocks), kScanThreads, 0, st>>>(out, n, totals);
@@ -293,8 +345,9 @@ int csr_build(const int* recv, int64_t E, int64_t N, int* row_ptr, int* perm, vo
   int* vals_b = reinterpret_cast<int*>(w + L.vals_b);
   const int e32 = static_cast<int>(E), n32 = static_cast<int>(N);
 
-  if (!count && (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess ||
-      cudaMemsetAsync(counts, 0, sizeof(int) * static_cast<size_t>(N + 1), st) != cudaSuccess)) {
+  // the status word and the counts are adjacent in the workspace: one memset clears both
+  if (!count && cudaMemsetAsync(status, 0, L.counts - L.status + sizeof(int) * static_cast<size_t>(N + 1),
+                                st) != cudaSuccess) {
     err = "cudaMemsetAsync failed";
     return E3CONV_ERR_CUDA;
   }
