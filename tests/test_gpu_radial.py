@@ -65,6 +65,35 @@ def test_radial_scalars_match_the_oracle(cuda_device, hidden, layers, nb, dtype)
     assert np.all(got[4] == 0) and np.all(got[5] == 0)
 
 
+@pytest.mark.parametrize("hidden,layers,nb", [(64, 2, 8), (32, 1, 5), (32, 3, 16), (64, 4, 8)])
+@pytest.mark.parametrize("dtype", ["f32", "f16"])
+def test_radial_scalars_many_tiles_per_cta(cuda_device, hidden, layers, nb, dtype):
+    # every CTA runs three or four tiles of four output chunks (the last ragged), so the
+    # kernel reuses its activation buffers, its output-weight ring and its three output
+    # accumulators across chunks and tiles; widths and depths cover one and two activation
+    # buffers and rings of two to four weight chunks
+    irreps = ("64x0e+64x1o", SH3, "64x0e+64x1o+64x2e")       # P*C = 7 * 64 = 448: 4 chunks
+    conv = e3.Conv(*irreps, 10.0, dtype=dtype)
+    P, C = conv.num_paths, conv.C
+    rng = np.random.default_rng(7 * hidden + layers)
+    r_max = 2.5
+    ws = _weights(rng, nb, hidden, layers, P * C)
+    conv.set_radial_mlp(r_max, ws)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    E = sms * 128 * 3 + 77                                    # 3 tiles per CTA, some 4
+    vec = rng.normal(size=(E, 3))
+    vec *= rng.uniform(0.05, 1.2 * r_max, size=(E, 1)) / np.linalg.norm(vec, axis=1, keepdims=True)
+    v4 = _vec4(vec)
+    s = conv.radial_scalars(to_dev(v4))
+    torch.cuda.synchronize()
+    assert conv.check()
+    got = s.float().cpu().numpy().reshape(E, P * C)
+    ref = _reference(v4, r_max, ws)
+    scale = np.abs(ref).max(axis=0)
+    err = (np.abs(got - ref) / np.where(scale > 0, scale, 1)).max()
+    assert err <= (2e-3 if dtype == "f16" else 1e-5 * max(1, layers - 1)), err
+
+
 def test_radial_scalars_few_edges_and_none(cuda_device):
     conv = e3.Conv("128x0e+128x1o", SH3, "128x0e+128x1o", 3.0)
     rng = np.random.default_rng(3)
