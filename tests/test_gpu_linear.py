@@ -119,3 +119,30 @@ def test_linear_repeated_and_changed_buffers(cuda_device):
     ws = weights()                                    # new weights on the same buffers
     lin(x2, out=y2)
     check(x2, y2, ws)
+
+
+@pytest.mark.parametrize("ins,outs", [
+    ("64x0e+64x1o+64x2e", "64x0e+64x1o+64x2e"),                 # five 32 KB stages
+    ("32x0e+32x1o", "256x1o+256x0e"),                           # six 16 KB stages, N = 256
+    ("64x0e+64x1o+64x2e+64x3o", "96x3o+96x1e+96x0e"),           # unmatched 1e among them
+])
+def test_linear_many_tiles_per_cta(cuda_device, ins, outs):
+    # 20,000 nodes: every CTA runs many tiles of several irreps, so the tensor-map kernel
+    # wraps its ring of input stages, reuses both accumulators and changes weights mid-range
+    lin = e3.IrrepsLinear(ins, outs, 0.9)
+    assert lin.uses_tma
+    rng = np.random.default_rng(21)
+    ws = [rng.normal(size=(lin.mul_in, lin.mul_out)).astype(np.float32)
+          for _ in range(lin.num_weight_blocks)]
+    lin.set_weights(ws)
+    n = 20000
+    x = rng.normal(size=(n, lin.dim_in)).astype(np.float32)
+    y = torch.full((n, lin.dim_out), float("nan"), device="cuda")
+    lin(to_dev(x), out=y)
+    torch.cuda.synchronize()
+    assert lin.check()
+    got = y.cpu().numpy()
+    ref = oracle.irreps_linear(ins, outs, 0.9, x, ws)
+    mag = oracle.irreps_linear(ins, outs, 0.9, np.abs(x), [np.abs(w) for w in ws])
+    assert np.all(np.abs(got - ref) <= 1e-5 * mag + 1e-30)
+    assert not np.isnan(got).any()
