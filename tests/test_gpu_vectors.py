@@ -176,3 +176,24 @@ def test_standalone_harmonics_feed_the_forward(cuda_device):
                      g.num_nodes, g.avg_num_neighbors)
     assert column_scaled_error(out_y.cpu().numpy(), ref) <= TOL["f32"]
     assert column_scaled_error(out_v.cpu().numpy(), ref) <= TOL["f32"]
+
+
+def test_harmonics_worked_example_of_the_pages(cuda_device):
+    # the pages' worked example (tests/golden/sh_worked_example.json): e3conv_edge_harmonics of
+    # its two vectors against the closed forms of the unit-direction harmonics up to l = 2
+    import json
+    import pathlib
+    fx = json.loads((pathlib.Path(__file__).parent / "golden" / "sh_worked_example.json").read_text())
+    v = np.asarray(fx["vectors"], dtype=np.float32)
+    conv = e3.Conv("8x0e", "1x0e+1x1o+1x2e", "8x0e", 1.0, dtype="f32")
+    got = conv.edge_harmonics(to_dev(_vec4(v))).cpu().numpy().astype(np.float64)
+    assert conv.check()
+    u = v.astype(np.float64)
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    x, y, z = u[:, 0], u[:, 1], u[:, 2]
+    ref = np.concatenate([np.ones((2, 1)), np.sqrt(3) * np.stack([y, z, x], 1),
+                          np.sqrt(15) * np.stack([x * y, y * z, (3 * z * z - 1) / (2 * np.sqrt(3)),
+                                                  x * z, (x * x - y * y) / 2], 1)], 1)
+    assert got.shape == (2, 9)
+    # float32 evaluation: 1e-5 of the largest component (sqrt(5) * 2 for l = 2)
+    assert np.abs(got - ref).max() <= 1e-5 * np.sqrt(5) * 2

@@ -83,3 +83,26 @@ def test_l1_is_scaled_direction_in_yzx_order():
     v = _unit(np.random.default_rng(50), 20)
     np.testing.assert_allclose(oracle.sh_l(1, v), np.sqrt(3) * v[:, [1, 2, 0]], atol=1e-14)
     np.testing.assert_allclose(oracle.sh_l(0, v), 1.0)
+
+
+def test_worked_example_of_the_pages():
+    # the pages' worked example (tests/golden/sh_worked_example.json, with its citation): two
+    # vectors, harmonics up to l = 2 as one (2l+1)-component block per l; the values are pinned
+    # by closed forms of the unit-direction harmonics, not by stored oracle output
+    import json
+    import pathlib
+    fx = json.loads((pathlib.Path(__file__).parent / "golden" / "sh_worked_example.json").read_text())
+    v = np.asarray(fx["vectors"], dtype=np.float64)
+    u = v / np.linalg.norm(v, axis=1, keepdims=True)
+    Y = oracle.sh(fx["lmax"], u)
+    blocks = {l: Y[:, l * l:(l + 1) ** 2].reshape(len(v), 1, 2 * l + 1) for l in range(fx["lmax"] + 1)}
+    assert {str(l): list(b.shape) for l, b in blocks.items()} == fx["shapes"]
+    x, y, z = u[:, 0], u[:, 1], u[:, 2]
+    np.testing.assert_allclose(blocks[0][:, 0, 0], 1.0, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(blocks[1][:, 0], np.sqrt(3) * np.stack([y, z, x], 1), rtol=0, atol=1e-14)
+    # l = 2, m = -2..2 (component normalisation, no Condon-Shortley phase, z polar axis)
+    Y2 = np.sqrt(15) * np.stack([x * y, y * z, (3 * z * z - 1) / (2 * np.sqrt(3)), x * z,
+                                 (x * x - y * y) / 2], 1)
+    np.testing.assert_allclose(blocks[2][:, 0], Y2, rtol=0, atol=1e-13)
+    for l, b in blocks.items():   # sum over m of Y_lm^2 = 2l+1 for unit directions
+        np.testing.assert_allclose((b[:, 0] ** 2).sum(1), 2 * l + 1, rtol=1e-13)
