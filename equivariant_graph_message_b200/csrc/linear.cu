@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) k_linear_tma(const __grid_cons
           if (lane == 0) mbar_arrive(tm_empty + (j & 1));
         }
         unsigned char* sg = stg + (chunk & 1) * kChunkBytes;
-        if (tid == 0) bulk_wait_read_but1();  // the store issued from this staging tile has read it
+        if (tid == 0) bulk_wait_read_but<1>();  // the store issued from this staging tile has read it
         asm volatile("bar.sync 1, 128;" ::: "memory");
 #pragma unroll
         for (int i = 0; i < 8; ++i)

@@ -49,14 +49,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
-// bulk store shared -> global of one thread's contiguous segment (both addresses and the
-// size multiples of 16 bytes), in this thread's bulk async-group
-__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, unsigned bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
-               "r"(smem_u32(src)), "r"(bytes)
-               : "memory");
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
 // 2-D TMA tensor store of one box from shared memory at coordinates (x inner, y), in this
 // thread's bulk async-group (commit with bulk_commit)
 __device__ __forceinline__ void tma_store_2d(const void* map, const void* src, int x, int y) {
@@ -82,19 +74,11 @@ __device__ __forceinline__ void tma_store_3d(const void* map, const void* src, i
       "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
-// all but the most recent of this thread's bulk groups have finished reading shared memory
-__device__ __forceinline__ void bulk_wait_read_but1() {
-  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
 __device__ __forceinline__ void mbar_arrive(unsigned long long* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
 }
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// this thread's bulk stores have finished reading their shared-memory source
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 // this thread's bulk stores are complete
 __device__ __forceinline__ void bulk_wait_all() {
@@ -155,19 +139,6 @@ __device__ __forceinline__ void tmem_ld32(unsigned addr, float* v) {
   for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(r[q]);
 }
 
-__device__ __forceinline__ void tmem_ld16(unsigned addr, float* v) {
-  unsigned r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-      "%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(addr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(r[q]);
-}
 // all but the `n` most recent of this thread's bulk groups have finished reading shared memory
 template <int n>
 __device__ __forceinline__ void bulk_wait_read_but() {
