@@ -537,7 +537,7 @@ def run_ours(args):
     global _flush
     in_bytes = 2 if spec.dtype == "f16" else 4
     step_bytes = algorithmic(conv, N, E, in_bytes)[0] / world
-    _flush = L2Flush(stream) if step_bytes < 2 * L2_BYTES else None
+    _flush = L2Flush(stream) if needs_l2_flush(step_bytes) else None
     clocks = Clocks(local)
     clocks.start()
     steps_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -735,6 +735,11 @@ class L2Flush:
 
 
 _flush = None   # set for workloads whose inputs fit in L2
+
+
+def needs_l2_flush(step_bytes: float) -> bool:
+    """Inputs smaller than twice the L2 would be partly read from it by the next step."""
+    return step_bytes < 2 * L2_BYTES
 
 
 def _event_ms(fn, reps, stream):

@@ -69,3 +69,17 @@ def test_traffic_is_reported_only_for_the_captured_configuration():
             assert t is None
         assert bench.traffic_for(name, c, int(nodes) * 10, rec["edges"] * 10) == (None, None)
         assert bench.traffic_for(name, c, int(nodes), rec["edges"], edge_vectors=True) == (None, None)
+
+
+@pytest.mark.parametrize("name,flushed", [("tiny", True), ("gate_points", True), ("mace", False),
+                                          ("large_f32", False), ("large_f16", False)])
+def test_l2_flush_for_the_workloads_that_fit_in_l2(name, flushed):
+    # a step's inputs smaller than twice the L2 are flushed before every timed step; the
+    # workloads' full sizes decide which
+    from workloads import make_graph
+    spec = configs.SPECS[name]
+    conv = e3.Conv(spec.irreps_node, spec.irreps_sh, spec.irreps_out, 10.0, dtype=spec.dtype)
+    g = make_graph(spec)
+    b = 2 if spec.dtype == "f16" else 4
+    step_bytes = bench.algorithmic(conv, g.num_nodes, g.num_edges, b)[0]
+    assert bench.needs_l2_flush(step_bytes) == flushed
