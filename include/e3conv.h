@@ -331,9 +331,9 @@ E3CONV_API int e3conv_forward_rows(e3conv_plan plan, const void* node_features, 
  *            n < num_basis, d = |r_ab| < r (0 for d >= r; d = 0: the limit)
  *   h_l    = SiLU(h_{l-1} W_{l-1}),  l = 1 .. layers   (SiLU(v) = v / (1 + e^-v))
  *   s_ab   = h_layers W_layers, reshaped [P][C]          (no biases)
- * The hidden layers and the output layer run on the tensor cores (tcgen05,
- * float16 hi + lo splits of both operands: float32 accuracy); layer 0 on the
- * CUDA cores.
+ * Every layer's product runs on the tensor cores (tcgen05, float16 hi + lo
+ * splits of both operands: float32 accuracy; layer 0 with the bases zero-padded
+ * to K = 16); the bases, the cutoff and SiLU on the CUDA cores.
  */
 
 /* Sets the plan's radial MLP from HOST float32 weights (row-major, input
