@@ -401,8 +401,10 @@ E3CONV_API int e3conv_linear_set_tma(e3conv_linear linear, int enable);
 E3CONV_API int e3conv_linear_set_weights(e3conv_linear linear, const float* w);
 
 /* y [num_nodes][dim_out] from x [num_nodes][dim_in] (device float32, 16-byte
- * aligned).  One kernel launch on `stream`; no allocation, no host
- * synchronisation. */
+ * aligned).  One kernel launch on `stream`; no device allocation, no host
+ * synchronisation.  The tensor-map kernel's arguments (its tensor maps of x and
+ * y) are kept in the layer's host memory and reused while x, y, num_nodes and
+ * the weights repeat; a layer is to be called from one host thread at a time. */
 E3CONV_API int e3conv_linear_forward(e3conv_linear linear, const float* x, int64_t num_nodes,
                                      float* y, e3conv_stream stream);
 
