@@ -54,7 +54,7 @@
  *
  * Streams: every device call is stream-ordered on the given stream (NULL is
  * the legacy default stream), does not synchronise the host and does not
- * allocate memory.  e3conv_stream has the same type as cudaStream_t.
+ * allocate device memory.  e3conv_stream has the same type as cudaStream_t.
  */
 #ifndef E3CONV_H
 #define E3CONV_H
