@@ -26,6 +26,9 @@ CASES = {
     "hub": (np.where(np.random.default_rng(3).random(70000) < 0.6, 7,
                      np.random.default_rng(4).integers(0, 257, 70000)), 257),
     "many_nodes": (np.random.default_rng(5).integers(0, 70000, 300000), 70001),
+    # row counts scanned in one launch up to 32,768 entries (N + 1 = 32,768), in levels above
+    "scan_one_launch_max": (np.random.default_rng(7).integers(0, 32767, 40000), 32767),
+    "scan_levels_min": (np.random.default_rng(8).integers(0, 32768, 40000), 32768),
     "large": (np.random.default_rng(6).integers(0, 100000, 4_000_000), 100000),
 }
 
