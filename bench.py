@@ -829,6 +829,32 @@ def time_next_rows(args, spec, g, conv, x, Y, s, senders, receivers, row_ptr, ou
             "note": "x read and y written once (HBM bound); tensor FLOPs count the three "
                     "float16 hi/lo MMAs per product"}
         del lin, yl
+    if not args.radial and g.vec is not None and conv.C >= 32:
+        # the radial MLP at this workload's size and dtype: seeded weights (8 bases, 64 x 2
+        # hidden, P*C outputs), the scalars written over this workload's s (last use of it)
+        rng = np.random.default_rng(11)
+        sizes = [8, 64, 64, conv.num_paths * conv.C]
+        ws = [(rng.normal(size=(a_, b_)) / np.sqrt(a_)).astype(np.float32)
+              for a_, b_ in zip(sizes[:-1], sizes[1:])]
+        v = np.zeros((E, 4), np.float32)
+        v[:, :3] = g.vec
+        r_max = float(np.linalg.norm(g.vec, axis=1).max()) * 1.01
+        conv.set_radial_mlp(r_max, ws)
+        v4 = torch.from_numpy(v).to(out.device)
+        conv.radial_scalars(v4, out=s)
+        torch.cuda.synchronize()
+        ms = _event_ms(lambda: conv.radial_scalars(v4, out=s), reps, stream)
+        assert conv.check()
+        nbytes = s.numel() * s.element_size()
+        flops = 3 * 2 * E * 64 * (64 + conv.num_paths * conv.C)
+        res["radial_mlp"] = {
+            "kernel": "k_radial", "outputs": conv.num_paths * conv.C, "dtype": spec.dtype, "ms": ms,
+            "scalars_bytes_written": nbytes, "write_gbs": nbytes / (ms / 1e3) / 1e9,
+            "hbm_frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+            "tensor_flops": flops, "tensor_tflops": flops / (ms / 1e3) / 1e12,
+            "note": "edge scalars from the edge vectors (bessel x cutoff, SiLU MLP) at this "
+                    "workload's size, seeded weights; supplementary"}
+        del v4
     return res
 
 
