@@ -378,7 +378,8 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
         // 16-byte piece q at (q ^ (r & 7)) * 16; box q of this chunk reuses slot q of the
         // previous one (thread 0 waits until that store has read it) and is stored as soon as
         // it is written, so the stores stream while the next boxes are staged
-        for (int q = 0; q < boxes; ++q) {
+        // staging and storing box q of this chunk in slot q (a ring across chunks)
+        auto stage_box = [&](int q, auto&& write) {
           unsigned char* slot = stage + q * (kTile * 128);
           if (tid == 0) {
             if (boxes == 4)
@@ -387,28 +388,7 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
               bulk_wait_read_but<1>();
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");  // slot q is free
-          unsigned char* dst = slot + row * 128;
-          if (a.out_f16) {
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              float v[32];
-              tmem_ld32(t_out(b) + lane_off + q * 64 + hh * 32, v);
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<uint4*>(dst + (((hh * 4 + i) ^ (row & 7)) * 16)) =
-                    make_uint4(pack_half2(v[8 * i] * f, v[8 * i + 1] * f),
-                               pack_half2(v[8 * i + 2] * f, v[8 * i + 3] * f),
-                               pack_half2(v[8 * i + 4] * f, v[8 * i + 5] * f),
-                               pack_half2(v[8 * i + 6] * f, v[8 * i + 7] * f));
-            }
-          } else {
-            float v[32];
-            tmem_ld32(t_out(b) + lane_off + q * 32, v);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              *reinterpret_cast<float4*>(dst + ((i ^ (row & 7)) * 16)) =
-                  make_float4(v[4 * i] * f, v[4 * i + 1] * f, v[4 * i + 2] * f, v[4 * i + 3] * f);
-          }
+          write(slot + row * 128);
           if (q == boxes - 1) {  // the accumulator is read: free it for the chunk after next
             tc_before();
             __syncwarp();
@@ -421,6 +401,60 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
               tma_store_2d(&smap, slot, col0 + q * bcols, static_cast<int>(tile * kTile));
             bulk_commit();  // one group per box (empty past the last column)
           }
+        };
+        if (a.out_f16) {
+          // float16, two boxes of 64 columns: four loads of 32 columns, each issued one ahead
+          unsigned r0[32], r1[32];
+          auto writeh = [&](unsigned char* dst, int hh, const unsigned* r) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              *reinterpret_cast<uint4*>(dst + (((hh * 4 + i) ^ (row & 7)) * 16)) = make_uint4(
+                  pack_half2(__uint_as_float(r[8 * i]) * f, __uint_as_float(r[8 * i + 1]) * f),
+                  pack_half2(__uint_as_float(r[8 * i + 2]) * f, __uint_as_float(r[8 * i + 3]) * f),
+                  pack_half2(__uint_as_float(r[8 * i + 4]) * f, __uint_as_float(r[8 * i + 5]) * f),
+                  pack_half2(__uint_as_float(r[8 * i + 6]) * f, __uint_as_float(r[8 * i + 7]) * f));
+          };
+          tmem_ld32_async(t_out(b) + lane_off, r0);
+          tmem_wait32(r0);
+          tmem_ld32_async(t_out(b) + lane_off + 32, r1);
+          stage_box(0, [&](unsigned char* dst) {
+            writeh(dst, 0, r0);
+            tmem_wait32(r1);
+            tmem_ld32_async(t_out(b) + lane_off + 64, r0);
+            writeh(dst, 1, r1);
+          });
+          tmem_wait32(r0);
+          tmem_ld32_async(t_out(b) + lane_off + 96, r1);
+          stage_box(1, [&](unsigned char* dst) {
+            writeh(dst, 0, r0);
+            tmem_wait32(r1);
+            writeh(dst, 1, r1);
+          });
+        } else {
+          // float32, four boxes: each box's tensor-memory load is issued one box ahead, so its
+          // latency overlaps the staging and the barriers of the box before it
+          unsigned r0[32], r1[32];
+          auto write32 = [&](unsigned* r) {
+            return [&, r](unsigned char* dst) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                *reinterpret_cast<float4*>(dst + ((i ^ (row & 7)) * 16)) =
+                    make_float4(__uint_as_float(r[4 * i]) * f, __uint_as_float(r[4 * i + 1]) * f,
+                                __uint_as_float(r[4 * i + 2]) * f, __uint_as_float(r[4 * i + 3]) * f);
+            };
+          };
+          tmem_ld32_async(t_out(b) + lane_off, r0);
+          tmem_wait32(r0);
+          tmem_ld32_async(t_out(b) + lane_off + 32, r1);
+          stage_box(0, write32(r0));
+          tmem_wait32(r1);
+          tmem_ld32_async(t_out(b) + lane_off + 64, r0);
+          stage_box(1, write32(r1));
+          tmem_wait32(r0);
+          tmem_ld32_async(t_out(b) + lane_off + 96, r1);
+          stage_box(2, write32(r0));
+          tmem_wait32(r1);
+          stage_box(3, write32(r1));
         }
       } else {  // rows whose byte length is not a multiple of 16: element stores
         const int cols = min(kChunk, a.nout - col0);
