@@ -1627,9 +1627,11 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
   }
   std::vector<AEntry> ent = build_a_entries(pl);
   BTable tab = tc_tables(pl, ent, colbase, 128);
+  // T is read in pieces of at most 16 columns, each load issued one piece ahead of the FMAs that
+  // use the piece before it (two pieces of registers live, as one 32-column piece would be)
   std::vector<std::pair<int, int>> chunks;  // (start column, width), start a multiple of width
   for (int pos = 0; pos < ncols_raw;) {
-    int w = 32;
+    int w = 16;
     while (w > 1 && (pos % w != 0 || pos + w > ncols_raw)) w /= 2;
     chunks.push_back({pos, w});
     pos += w;
@@ -1859,18 +1861,28 @@ std::string tc_source(const Plan& pl, const Shape& sh) {
     em.line("const float s" + S(p) + " = h2f(sv[" + S(static_cast<long long>(p) * pl.C) + "]);");
   em.line("ok = bar_wait(tdone, v & 1u);");
   em.line("tc_after();");
+  // the wait names the registers of the piece it completes, so that no use moves above it
+  auto wait_piece = [&](size_t k) {
+    std::string ops;
+    for (int r = 0; r < chunks[k].second; ++r)
+      ops += std::string(r ? ", " : "") + "\"+r\"(r" + S(k) + "_[" + S(r) + "])";
+    em.line("asm volatile(\"tcgen05.wait::ld.sync.aligned;\" : " + ops + " :: \"memory\");");
+  };
+  auto load_piece = [&](size_t k) {
+    em.line("unsigned int r" + S(k) + "_[" + S(chunks[k].second) + "];");
+    em.line("TMEM_LD" + S(chunks[k].second) + "(tcol + " + S(chunks[k].first) + "u, r" + S(k) + "_);");
+  };
+  load_piece(0);
+  wait_piece(0);
   for (size_t k = 0; k < chunks.size(); ++k) {
-    em.line("{");
-    em.line("  unsigned int r[" + S(chunks[k].second) + "];");
-    em.line("  TMEM_LD" + S(chunks[k].second) + "(tcol + " + S(chunks[k].first) + "u, r);");
-    em.line("  asm volatile(\"tcgen05.wait::ld.sync.aligned;\" ::: \"memory\");");
+    if (k + 1 < chunks.size()) load_piece(k + 1);
     for (int col = chunks[k].first; col < chunks[k].first + chunks[k].second; ++col) {
       size_t p = 0;
       while (!(col >= colbase[p] && col < colbase[p] + 2 * pl.paths[p].l3 + 1)) ++p;
       const std::string acc = "a" + S(pl.paths[p].out_off + col - colbase[p]);
-      em.line("  " + acc + " = fmaf(s" + S(p) + ", __uint_as_float(r[" + S(col - chunks[k].first) + "]), " + acc + ");");
+      em.line(acc + " = fmaf(s" + S(p) + ", __uint_as_float(r" + S(k) + "_[" + S(col - chunks[k].first) + "]), " + acc + ");");
     }
-    em.line("}");
+    if (k + 1 < chunks.size()) wait_piece(k + 1);
   }
   em.line("++v;");
   em.ind--;
