@@ -32,8 +32,9 @@
 //               the output layer still reads this tile's);
 //   warp 12     issues layer 0's and the hidden layers' MMAs;
 //   warp 13     issues the output layer's MMAs, chunk by chunk, into three
-//               tensor-memory accumulators, and the bulk copies of the
-//               output-weight chunks into a ring of 2-4 buffers;
+//               tensor-memory accumulators;
+//   warp 14     requests the output-weight chunks into a ring of 2-4 buffers,
+//               each as soon as its buffer is free;
 //   warps 0-3   (thread t <-> edge row t <-> tensor-memory lane t) read each
 //               output chunk out of its accumulator into a ring of swizzled
 //               [128 rows x 128 bytes] staging boxes, each stored by a 2-D TMA
@@ -72,7 +73,7 @@ constexpr int kMaxWBufs = 4;         // output-weight chunk buffers in shared me
 constexpr int kOutBufs = 3;          // output-layer accumulators in tensor memory
 constexpr int kOutCol = 128;         // tensor-memory column of the output accumulators (>= hidden)
 constexpr int kTmemCols = 512;       // hidden D [0, H) and three output accumulators of 128
-constexpr int kRadThreads = 448;     // 4 drain warps, 8 compute warps, 2 MMA warps
+constexpr int kRadThreads = 480;     // 4 drain warps, 8 compute warps, 2 MMA warps, 1 loader
 constexpr int kRadBars = 24;         // mbarriers (and the tensor-memory slot after them)
 
 struct RadialArgs {
@@ -88,6 +89,7 @@ struct RadialArgs {
   int nb, layers;          // basis size, hidden layers L (>= 1)
   int nout, chunks;        // P*C outputs, chunks of kChunk (the last padded with zero weights)
   int wbufs, abufs;        // output-weight chunk buffers, activation buffers
+  int stage_bytes;         // staging ring of the drain (its boxes for the output dtype)
   float r_max;
   void* s;                 // [E][nout] float32 or float16
   int out_f16;
@@ -108,9 +110,9 @@ struct Smem {
   static constexpr int kWout = kChunk * H * 2;   // one [kChunk x H] float16 operand
 };
 
-inline size_t radial_smem_for(int H, int layers, int abufs, int wbufs) {
+inline size_t radial_smem_for(int H, int layers, int abufs, int wbufs, int stage_bytes) {
   const size_t h = static_cast<size_t>(H);
-  return kStageBytes + 2 * h * kMaxBasis * 2 + (layers - 1) * 2 * h * h * 2 + 2 * kTile * kMaxBasis * 2 +
+  return stage_bytes + 2 * h * kMaxBasis * 2 + (layers - 1) * 2 * h * h * 2 + 2 * kTile * kMaxBasis * 2 +
          abufs * 2 * kTile * h * 2 + wbufs * 2 * kChunk * h * 2 + kRadBars * 8;
 }
 
@@ -122,7 +124,7 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int A = a.abufs, W = a.wbufs;
   unsigned char* stage = sm;                                          // 1024-byte aligned (swizzle)
-  unsigned char* w0s = stage + kStageBytes;                           // layer 0 (hi, lo)
+  unsigned char* w0s = stage + a.stage_bytes;                         // layer 0 (hi, lo)
   unsigned char* whs = w0s + 2 * L::kW0;                              // (layers-1) x (hi, lo)
   unsigned char* bas = whs + (a.layers - 1) * 2 * L::kWhid;           // basis values (hi, lo)
   unsigned char* acts = bas + 2 * L::kBas;                            // A x (hi, lo)
@@ -235,13 +237,7 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
     }
   } else if (warp == 13) {  // ---- the output layer's MMAs and weight chunks
     if (lane == 0) {
-      long long g = 0, gl = 0;  // chunks issued, chunk weights requested
-      auto load = [&](long long q) {
-        const int wb = static_cast<int>(q % W);
-        mbar_expect(bar_w + wb, 2 * L::kWout);
-        bulk_g2s(wos + wb * 2 * L::kWout, a.wo + static_cast<size_t>(q % a.chunks) * 2 * L::kWout,
-                 2 * L::kWout, bar_w + wb);
-      };
+      long long g = 0;  // chunks issued (their weights come from the loader warp)
       const unsigned ido = idesc_f16(kTile, kChunk);
       for (long long k = 0; k < my_tiles && ok; ++k) {
         ok = mbar_wait(out_full + (k % A), (k / A) & 1);
@@ -249,22 +245,6 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
         tc_after();
         const unsigned long long d_hhi = kmajor_desc(act(k)), d_hlo = kmajor_desc(act(k) + L::kAct);
         for (int c = 0; c < a.chunks && ok; ++c, ++g) {
-          // weight chunks requested as far ahead as the ring has buffers whose MMAs are done
-          // (chunk g's own request waits for its buffer, the later ones only look)
-          while (gl < total && gl < g + W) {
-            if (gl >= W) {
-              const int wb = static_cast<int>(gl % W);
-              const unsigned par = static_cast<unsigned>(((gl / W) - 1) & 1);
-              if (gl > g) {
-                if (!mbar_try(w_free + wb, par)) break;
-              } else if (!(ok = mbar_wait(w_free + wb, par))) {
-                break;
-              }
-            }
-            load(gl);
-            ++gl;
-          }
-          if (!ok) break;
           const int wb = static_cast<int>(g % W), b = static_cast<int>(g % kOutBufs);
           ok = mbar_wait(bar_w + wb, (g / W) & 1);
           if (ok && g >= kOutBufs) ok = mbar_wait(tm_empty + b, ((g / kOutBufs) - 1) & 1);
@@ -286,11 +266,27 @@ __global__ void __launch_bounds__(kRadThreads, 1) k_radial(RadialArgs a, const _
         if (!ok) break;
         mma_commit(act_free + (k % A));
       }
-      // nothing in flight at exit: the last commits have arrived, every requested chunk landed
+      // nothing in flight at exit: the last commits have arrived
       for (long long q = (g > W ? g - W : 0); q < g; ++q) mbar_wait(w_free + q % W, (q / W) & 1);
       if (g > 0) mbar_wait(mma_done + (g - 1) % kOutBufs, ((g - 1) / kOutBufs) & 1);
-      for (long long q = g; q < gl; ++q) mbar_wait(bar_w + q % W, (q / W) & 1);
       if (ok && my_tiles > 0) mbar_wait(act_free + (my_tiles - 1) % A, ((my_tiles - 1) / A) & 1);
+      if (!ok) atomicOr(a.status, 4u);
+    }
+  } else if (warp == 14) {  // ---- output-weight chunks into the ring
+    // lane 0 requests chunk q's weights as soon as the MMAs of chunk q - W have released its
+    // buffer, independently of the MMA warp's own waits
+    if (lane == 0) {
+      long long q = 0;
+      for (; q < total && ok; ++q) {
+        const int wb = static_cast<int>(q % W);
+        if (q >= W) ok = mbar_wait(w_free + wb, static_cast<unsigned>(((q / W) - 1) & 1));
+        if (!ok) break;
+        mbar_expect(bar_w + wb, 2 * L::kWout);
+        bulk_g2s(wos + wb * 2 * L::kWout, a.wo + static_cast<size_t>(q % a.chunks) * 2 * L::kWout,
+                 2 * L::kWout, bar_w + wb);
+      }
+      // no copy outlives the block: the last requested chunks have landed (bounded)
+      for (long long p = (q > W ? q - W : 0); p < q; ++p) mbar_wait(bar_w + p % W, (p / W) & 1);
       if (!ok) atomicOr(a.status, 4u);
     }
   } else if (warp >= 4) {  // ---- warps 4-11: bases, SiLU, activation operands
@@ -542,18 +538,21 @@ int radial_prepare(RadialPlan& rp, int nb, double r_max, int hidden, int layers,
 
 // activation and output-weight buffers: two and as many chunk buffers (2-4) as fit, else one
 // activation buffer and two chunk buffers
-static void radial_buffers(const RadialPlan& rp, int& abufs, int& wbufs) {
+// staging for the output dtype (float16 scalars need half of it), then two activation buffers
+// and as many chunk buffers (2-4) as fit, else one activation buffer and two chunk buffers
+static void radial_buffers(const RadialPlan& rp, int out_f16, int& abufs, int& wbufs, int& stage) {
   constexpr size_t kMax = 227 * 1024;
+  stage = out_f16 ? kStageBytes / 2 : kStageBytes;
   abufs = 2;
   for (wbufs = kMaxWBufs; wbufs > 2; --wbufs)
-    if (radial_smem_for(rp.hidden, rp.layers, abufs, wbufs) <= kMax) return;
-  if (radial_smem_for(rp.hidden, rp.layers, abufs, wbufs) > kMax) abufs = 1;
+    if (radial_smem_for(rp.hidden, rp.layers, abufs, wbufs, stage) <= kMax) return;
+  if (radial_smem_for(rp.hidden, rp.layers, abufs, wbufs, stage) > kMax) abufs = 1;
 }
 
-size_t radial_smem_bytes(const RadialPlan& rp) {
-  int abufs = 0, wbufs = 0;
-  radial_buffers(rp, abufs, wbufs);
-  return radial_smem_for(rp.hidden, rp.layers, abufs, wbufs);
+size_t radial_smem_bytes(const RadialPlan& rp) {  // the float32 scalars' (the larger) need
+  int abufs = 0, wbufs = 0, stage = 0;
+  radial_buffers(rp, 0, abufs, wbufs, stage);
+  return radial_smem_for(rp.hidden, rp.layers, abufs, wbufs, stage);
 }
 
 int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, const void* dev_wo,
@@ -584,8 +583,8 @@ int radial_launch(const RadialPlan& rp, const void* dev_w0, const void* dev_wh, 
   a.s = s;
   a.out_f16 = out_f16;
   a.status = status;
-  radial_buffers(rp, a.abufs, a.wbufs);
-  const size_t smem = radial_smem_for(rp.hidden, rp.layers, a.abufs, a.wbufs);
+  radial_buffers(rp, out_f16, a.abufs, a.wbufs, a.stage_bytes);
+  const size_t smem = radial_smem_for(rp.hidden, rp.layers, a.abufs, a.wbufs, a.stage_bytes);
   const long long tiles = (num_edges + kTile - 1) / kTile;
   auto launch = [&](auto kernel) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
